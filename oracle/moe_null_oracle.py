@@ -1,0 +1,287 @@
+"""CPU oracle: forward pass of a token-choice MoE layer with zero-compute null experts.
+
+TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's
+CPU-baseline leg may import this module. The CUDA library never calls it, and it
+shares no code with the CUDA library: it is a plain, slow, float64 NumPy
+restatement of what the pages define, so that a reader can check it against
+them line by line.
+
+Sources (cited by page title and section):
+
+[KR]  "Improving MoE Compute Efficiency by Composing Weight and Data Sparsity"
+      (Kilian et al.), paper-review page, section 三 技术架构 (architecture):
+      核心公式 / Token-Choice MoE (layer equation), Null Expert 机制 (null expert,
+      M copies of the null logit before top-K, renormalisation over the selected
+      real experts), 阈值解释 (threshold reading), 负载均衡损失 (L_bal),
+      Z-Loss (L_z), 关键特性 / 解决方案空间保持 (K^4_0.5 reproduces K^2_1.0),
+      实现 (argsort moves null indices >= N to the end, truncate, grouped matmul).
+[SS]  same paper, sciencestack page: Figure 3 caption (rho = real / all
+      selected experts), Figure 4/5 captions (compute intensity = fraction of
+      top-K slots filled by real experts).
+[T44] "【Transformer 与注意力机制】44｜MoE：稀疏激活的万亿模型路径", section 三
+      (router softmax(W_g x), top-k then renormalise over the k), section 4.2
+      (aux loss alpha*E*sum f_i P_i), section 4.3 (router z-loss).
+[MPP] MoE++ explainer page, section "Gating 机制与残差门控": topk over all
+      logits, softmax over the k, zero the zero-compute experts' weights,
+      divide by the remaining sum.
+
+Readings where the pages are silent (each is listed in the design notes):
+* pool = N real slots followed by M null copies (indices N..N+M-1); with M = 0
+  there is no null slot at all;
+* top-K order is (logit descending, pool index ascending); a real logit equal
+  to the null logit therefore precedes every copy, and copies fill in index
+  order;
+* gates are a softmax over the selected real logits; a token with no real
+  expert gets only the shared expert;
+* the shared expert is ungated; every expert is SwiGLU W_d(silu(W_g z) * W_u z);
+* f_i = count_i / T, so sum_i f_i = K; P_i = mean_t p_{t,i} over the pool;
+* rows within an expert's segment are in ascending token order (stable argsort).
+
+Parity status: every function below is pinned by the CPU tests in
+tests/test_oracle_pins.py (brute force, closed forms, textbook reductions,
+library routines); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "router_logits", "expanded_pool", "pool_logsumexp", "pool_probs", "topk_pool",
+    "threshold_real_count", "renormalised_gates", "dispatch", "swiglu",
+    "layer_output", "aux_stats", "aux_partial_sums", "aux_finalize", "route",
+    "bf16_round_f64",
+]
+
+
+def router_logits(x, w_router, bias=None, tok_null_bias=None):
+    """Router logits s[t, j], j = 0..N (N real experts, then the null logit).
+
+    [KR] 三/Null Expert 机制: the router is widened to N+1 logits, the last one
+    belonging to the null expert. [T44] 三: the router is a linear map of the
+    token's hidden state. ``bias`` [N+1] is added to every logit; the optional
+    per-token ``tok_null_bias`` [T] is added to the null logit only.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_router, dtype=np.float64)
+    s = x @ w.T
+    if bias is not None:
+        s = s + np.asarray(bias, dtype=np.float64)[None, :]
+    if tok_null_bias is not None:
+        s[:, -1] += np.asarray(tok_null_bias, dtype=np.float64)
+    return s
+
+
+def expanded_pool(s, M):
+    """The expanded logit vector [s_0..s_{N-1}, s_N repeated M times].
+
+    [KR] 三/Null Expert 机制: the null logit is copied M times before top-K.
+    Returns v [T, N+M].
+    """
+    s = np.asarray(s, dtype=np.float64)
+    N = s.shape[1] - 1
+    real = s[:, :N]
+    if M == 0:
+        return real.copy()
+    null = np.repeat(s[:, N:N + 1], M, axis=1)
+    return np.concatenate([real, null], axis=1)
+
+
+def pool_logsumexp(v):
+    """lse_t = log sum_i exp(v_{t,i}) over the whole pool ([KR] 三/Z-Loss)."""
+    v = np.asarray(v, dtype=np.float64)
+    m = v.max(axis=1)
+    return m + np.log(np.exp(v - m[:, None]).sum(axis=1))
+
+
+def pool_probs(v, lse):
+    """p_{t,i} = exp(v_{t,i} - lse_t): the routing softmax over the pool."""
+    return np.exp(np.asarray(v, dtype=np.float64) - np.asarray(lse)[:, None])
+
+
+def topk_pool(v, K):
+    """Top-K pool indices per token, in rank order (value desc, index asc).
+
+    A stable sort of the pool: primary key the value (descending), secondary
+    key the pool index (ascending). Returns int64 [T, K].
+    """
+    v = np.asarray(v, dtype=np.float64)
+    T, P = v.shape
+    if K > P:
+        raise ValueError("K exceeds the pool size N+M")
+    index = np.broadcast_to(np.arange(P), v.shape)
+    order = np.lexsort((index, -v), axis=-1)
+    return order[:, :K].astype(np.int64)
+
+
+def threshold_real_count(s, M, K):
+    """Number of real experts a token selects, from the threshold reading.
+
+    [KR] 三/阈值解释: a token keeps exactly the real experts whose logit beats
+    the null logit, the remaining slots going to null copies. With a = #{i < N :
+    s_i >= s_null} (ties go to the real expert, whose index is lower), the
+    token takes min(K, a) reals first, then up to M null copies, then, only if
+    the copies run out, further reals: r = min(K,a) + max(0, K - min(K,a) - M).
+    """
+    s = np.asarray(s, dtype=np.float64)
+    N = s.shape[1] - 1
+    a = (s[:, :N] >= s[:, N:N + 1]).sum(axis=1)
+    first = np.minimum(K, a)
+    return first + np.maximum(0, K - first - M)
+
+
+def renormalised_gates(s, idx, N):
+    """Gate of each selected slot: softmax over the token's selected real logits.
+
+    [KR] 三/Null Expert 机制: routing weights are renormalised over the selected
+    real experts only, so null routing does not change the output's magnitude.
+    Null slots get weight 0; a token with no real expert gets all zeros.
+    Returns float64 [T, K].
+    """
+    s = np.asarray(s, dtype=np.float64)
+    idx = np.asarray(idx)
+    T, K = idx.shape
+    g = np.zeros((T, K), dtype=np.float64)
+    for t in range(T):
+        sel = [k for k in range(K) if idx[t, k] < N]
+        if not sel:
+            continue
+        vals = np.array([s[t, idx[t, k]] for k in sel])
+        e = np.exp(vals - vals.max())
+        g[t, sel] = e / e.sum()
+    return g
+
+
+def dispatch(idx, N):
+    """Expert-contiguous list of the real (token, expert) slots.
+
+    [KR] 三/实现: an argsort moves null indices (>= N) to the end and the
+    sorted list is truncated before the grouped matmul. The sort here is a
+    stable one on (expert, token), so rows inside an expert's segment are in
+    ascending token order. Returns counts [N], offsets [N+1], perm_tok [R]
+    (token of each row) and slot_row [T, K] (row of each slot, -1 for nulls).
+    """
+    idx = np.asarray(idx)
+    T, K = idx.shape
+    tok = np.repeat(np.arange(T), K)
+    kk = np.tile(np.arange(K), T)
+    e = idx.reshape(-1)
+    real = e < N
+    tok_r, k_r, e_r = tok[real], kk[real], e[real]
+    order = np.lexsort((tok_r, e_r))
+    counts = np.bincount(e_r, minlength=N).astype(np.int64)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    perm_tok = tok_r[order].astype(np.int64)
+    slot_row = np.full((T, K), -1, dtype=np.int64)
+    slot_row[tok_r[order], k_r[order]] = np.arange(order.size)
+    return counts, offsets, perm_tok, slot_row
+
+
+def bf16_round_f64(a):
+    """Round to the nearest bf16 value (ties to even), returned as float64."""
+    f = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def swiglu(z, w_gate, w_up, w_down, round_h=False):
+    """One SwiGLU expert E(z) = (silu(z W_g^T) * (z W_u^T)) W_d^T in float64.
+
+    silu(a) = a * sigmoid(a). w_gate, w_up: [F, d]; w_down: [d, F].
+    ``round_h`` rounds the hidden activation to bf16 (the CUDA path stores it
+    in bf16 between its two matmuls).
+    """
+    z = np.asarray(z, dtype=np.float64)
+    a = z @ np.asarray(w_gate, dtype=np.float64).T
+    b = z @ np.asarray(w_up, dtype=np.float64).T
+    h = a / (1.0 + np.exp(-a)) * b
+    if round_h:
+        h = bf16_round_f64(h)
+    return h @ np.asarray(w_down, dtype=np.float64).T
+
+
+def layer_output(x, idx, gates, N, experts, shared, tokens=None, round_h=False):
+    """y_t = E_shared(x_t) + sum over the selected real experts of g_i E_i(x_t).
+
+    [KR] 三/核心公式 (Token-Choice MoE): y = E_shared(x) + sum_{i in top-K}
+    g_i(x) E_i(x); null experts output zero ([KR] 三/Null Expert 机制), so only
+    real slots contribute. ``experts`` = (w_gate [N,F,d], w_up [N,F,d],
+    w_down [N,d,F]); ``shared`` = (ws_gate, ws_up, ws_down). ``tokens`` limits
+    the computation to a subset of token indices (rows of the result follow
+    that order).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    idx = np.asarray(idx)
+    gates = np.asarray(gates, dtype=np.float64)
+    if tokens is None:
+        tokens = np.arange(x.shape[0])
+    tokens = np.asarray(tokens)
+    xt = x[tokens]
+    y = swiglu(xt, *shared, round_h=round_h)
+    wg, wu, wd = experts
+    sub_idx = idx[tokens]
+    sub_g = gates[tokens]
+    for e in range(N):
+        rows, ks = np.nonzero(sub_idx == e)
+        if rows.size == 0:
+            continue
+        ye = swiglu(xt[rows], wg[e], wu[e], wd[e], round_h=round_h)
+        y[rows] += sub_g[rows, ks][:, None] * ye
+    return y
+
+
+def aux_stats(idx, p, lse, N, M):
+    """Load-balance and Z-loss statistics over the expanded pool.
+
+    [KR] 三/负载均衡损失: L_bal = N * sum_{i=1}^{N+M} f_i P_i, f_i the fraction
+    of tokens routed to slot i (count_i / T), P_i the mean routing probability.
+    [KR] 三/Z-Loss: L_z = (1/T) sum_t (log sum_{i=1}^{N+M} exp s_i)^2.
+    Returns counts_ext [N+M], f, P, L_bal, L_z.
+    """
+    idx = np.asarray(idx)
+    T = idx.shape[0]
+    counts_ext = np.bincount(idx.reshape(-1), minlength=N + M)[:N + M].astype(np.int64)
+    f = counts_ext / float(T)
+    P = np.asarray(p, dtype=np.float64).mean(axis=0)
+    L_bal = N * float(np.sum(f * P))
+    L_z = float(np.mean(np.asarray(lse, dtype=np.float64) ** 2))
+    return counts_ext, f, P, L_bal, L_z
+
+
+def aux_partial_sums(idx, p, lse, N, M):
+    """Additive statistics of a token shard, for data-parallel reduction.
+
+    Returns (counts_ext [N+M] int64, sum_t p [N+M] float64, sum_t lse^2, T).
+    Summing these over shards and calling :func:`aux_finalize` equals
+    :func:`aux_stats` on the concatenated tokens, because f_i and P_i are means
+    over all tokens ([KR] 三/负载均衡损失).
+    """
+    idx = np.asarray(idx)
+    counts_ext = np.bincount(idx.reshape(-1), minlength=N + M)[:N + M].astype(np.int64)
+    psum = np.asarray(p, dtype=np.float64).sum(axis=0)
+    lsq = float(np.sum(np.asarray(lse, dtype=np.float64) ** 2))
+    return counts_ext, psum, lsq, int(idx.shape[0])
+
+
+def aux_finalize(counts_ext, psum, lsq, T, N):
+    """L_bal and L_z from summed statistics (see :func:`aux_partial_sums`)."""
+    f = np.asarray(counts_ext, dtype=np.float64) / float(T)
+    P = np.asarray(psum, dtype=np.float64) / float(T)
+    return f, P, N * float(np.sum(f * P)), float(lsq) / float(T)
+
+
+def route(s, M, K):
+    """All routing outputs from logits s [T, N+1] (float64 or the GPU's fp32).
+
+    Returns a dict with the pool v, lse, p, top-K indices, per-token real count
+    ("compute intensity" numerator, [SS] Figure 4/5 captions) and gates.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    N = s.shape[1] - 1
+    v = expanded_pool(s, M)
+    lse = pool_logsumexp(v)
+    p = pool_probs(v, lse)
+    idx = topk_pool(v, K)
+    n_real = (idx < N).sum(axis=1)
+    gates = renormalised_gates(s, idx, N)
+    return dict(v=v, lse=lse, p=p, idx=idx, n_real=n_real, gates=gates)
