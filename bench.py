@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the null-expert MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config qwen3_0p6b]
+
+A step is one full forward of the layer (route -> dispatch + aux -> grouped
+gate/up SwiGLU GEMM -> grouped down GEMM -> combine) over one batch of T
+synthetic tokens that is already resident in HBM. L2 is flushed (a 256 MiB
+write) between timed steps; each step is timed with CUDA events on the
+launching stream. Prints one JSON line (rank 0).
+
+Metric: real (token, expert) slots per second for the layer forward, i.e. R /
+t_step summed over ranks (null slots are not counted). Multi-GPU runs are data
+parallel (each rank its own T tokens, weak scaling) with one NCCL all-reduce
+of the additive aux statistics per step, the layer's only exchange.
+
+--impl reference times the CPU oracle (the float64 NumPy restatement used by
+the tests) on a bounded token sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "real-slot tokens/s per MoE layer fwd; grouped-GEMM TFLOP/s vs BF16 peak"
+UNIT = "real-slot tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline object)
+
+def oracle_sample_run(inp, S):
+    """Full oracle forward on the first S tokens; returns (seconds, real slots)."""
+    import numpy as np
+    import oracle as O
+    from token_choice_routing_b200 import inputs as I
+    cfg = inp.cfg
+    f = lambda b: I.bf16_to_f32(b).astype(np.float64)
+    t0 = time.perf_counter()
+    x = f(inp.x[:S])
+    tnb = None if inp.tok_null_bias is None else inp.tok_null_bias[:S]
+    s = O.router_logits(x, inp.w_router, inp.bias, tnb)
+    r = O.route(s, cfg.M, cfg.K)
+    O.dispatch(r["idx"], cfg.N)
+    O.layer_output(x, r["idx"], r["gates"], cfg.N, (f(inp.w_gate), f(inp.w_up), f(inp.w_down)),
+                   (f(inp.ws_gate), f(inp.ws_up), f(inp.ws_down)))
+    O.aux_stats(r["idx"], r["p"], r["lse"], cfg.N, cfg.M)
+    dt = time.perf_counter() - t0
+    return dt, int(r["n_real"].sum())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def calibrate_sample(inp, target_s):
+    S0 = min(inp.cfg.T, 512)
+    dt, _ = oracle_sample_run(inp, S0)
+    S = int(S0 * target_s / max(dt, 1e-3))
+    return max(64, min(inp.cfg.T, S))
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from token_choice_routing_b200 import inputs as I
+    cfg = I.CONFIGS[args.config]
+    inp = I.make_inputs(cfg)
+    S = calibrate_sample(inp, args.ref_step_seconds)
+    for _ in range(args.warmup):
+        oracle_sample_run(inp, S)
+    tot_t, tot_r = 0.0, 0
+    for _ in range(args.steps):
+        dt, R = oracle_sample_run(inp, S)
+        tot_t += dt
+        tot_r += R
+    value = tot_r / tot_t
+    cores = blas_threads()
+    sample = f"first {S} of {cfg.T} tokens per step (full oracle forward: route, dispatch, experts, aux)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,1/fan_in) weights)",
+        "config": workload_config(cfg, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, args):
+    return {"workload": f"{cfg.name}: MoE layer fwd T={cfg.T} d={cfg.d} N={cfg.N} F={cfg.F} "
+                        f"F_shared={cfg.F_shared} K={cfg.K} M={cfg.M} rho={cfg.rho:.3g}",
+            "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "K": cfg.K, "F": cfg.F, "F_shared": cfg.F_shared,
+            "global_batch_tokens": cfg.T * args.gpus, "parallelism": f"dp{args.gpus}",
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+# ----------------------------------------------------------------------------------------
+# GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="qwen3_0p6b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
+    ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from token_choice_routing_b200 import binding as B
+    from token_choice_routing_b200 import inputs as I
+    from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    assert world == args.gpus or world == 1, "launch with torchrun for --gpus > 1"
+
+    cfg = I.CONFIGS[args.config]
+    inp = I.make_inputs(cfg)
+    layer = MoENullLayer.from_inputs(inp, dev)
+    x = bf16_tensor(inp.x, dev)
+    tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
+    T = cfg.T
+    out = layer.alloc(T, logits=False)
+    dm = layer.dims(T)
+    nsum = B.aux_sums_count(dm)
+    sums = torch.zeros(nsum, dtype=torch.float64, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        if world == 1:
+            layer.forward(x, tnb, out)
+            return
+        # data parallel: local route/dispatch, global aux statistics, local experts
+        B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, out["topk_idx"], out["topk_gate"],
+                out["n_real"], out["workspace"])
+        B.aux_sums(dm, out["workspace"], sums)
+        dist.all_reduce(sums)
+        B.aux_finalize(dm, sums, out["counts_ext"], out["P"], out["losses"])
+        B.dispatch(dm, x, out["topk_idx"], out["workspace"], out["counts"], out["offsets"], out["perm_tok"],
+                   out["slot_row"], out["xs"])
+        B.expert_ffn(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.w_down, layer.shared_gate_up,
+                     layer.shared_down, out["h"], out["h_shared"], out["ys"], out["shared_out"], out["workspace"])
+        B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"])
+
+    kernels_per_step = 5 if world == 1 else 7  # route, dispatch, gate_up, down, combine (+ aux sums/finalize)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = B.get_device_status(out["workspace"])
+    if st != B.OK:
+        raise SystemExit(f"device status after warm-up: {B.status_string(st)}")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record()
+            step()
+            e1.record()
+        torch.cuda.synchronize()
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    R = int(out["offsets"][-1].item())
+    value = world * R * args.steps / (total_ms * 1e-3)
+    st = B.get_device_status(out["workspace"])
+    if st != B.OK:
+        raise SystemExit(f"device status after timing: {B.status_string(st)}")
+
+    # ---- per-kernel breakdown (separately timed steps, same launches, CUDA events between them)
+    names = ["route", "dispatch", "gate_up", "down", "combine"]
+    acc = {n: 0.0 for n in names}
+    nb = max(3, min(args.steps, 10))
+    for _ in range(nb):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        ev[0].record()
+        B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, out["topk_idx"], out["topk_gate"],
+                out["n_real"], out["workspace"])
+        ev[1].record()
+        B.dispatch(dm, x, out["topk_idx"], out["workspace"], out["counts"], out["offsets"], out["perm_tok"],
+                   out["slot_row"], out["xs"])  # the aux reduction rides in this launch, as in moe_forward
+        ev[2].record()
+        B.expert_gate_up(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, out["h"],
+                         out["h_shared"], out["workspace"])
+        ev[3].record()
+        B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down, out["ys"],
+                      out["shared_out"], out["workspace"])
+        ev[4].record()
+        B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"])
+        ev[5].record()
+        torch.cuda.synchronize()
+        for i, n in enumerate(names):
+            acc[n] += ev[i].elapsed_time(ev[i + 1])
+    kms = {n: acc[n] / nb for n in names}
+
+    peaks, peak_kind = load_peaks()
+    d, F, Fs, N, K = cfg.d, cfg.F, cfg.F_shared, cfg.N, cfg.K
+    flops_gu = 4.0 * d * F * R + 4.0 * d * Fs * T
+    flops_dn = 2.0 * d * F * R + 2.0 * d * Fs * T
+    bytes_route = 2.0 * d * T + (8.0 * K + 4.0) * T
+    bytes_dispatch = 4.0 * d * R + 4.0 * K * T
+    bytes_combine = 2.0 * d * R + 4.0 * d * T
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fp32_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+    breakdown = {
+        "route": {"ms": kms["route"], "bound": "alu", "TFLOP/s": 2.0 * (N + 1) * d * T / (kms["route"] * 1e9),
+                  "GB/s": bytes_route / (kms["route"] * 1e6)},
+        "dispatch": {"ms": kms["dispatch"], "bound": "hbm", "GB/s": bytes_dispatch / (kms["dispatch"] * 1e6)},
+        "gate_up": {"ms": kms["gate_up"], "bound": "tensor", "TFLOP/s": flops_gu / (kms["gate_up"] * 1e9)},
+        "down": {"ms": kms["down"], "bound": "tensor", "TFLOP/s": flops_dn / (kms["down"] * 1e9)},
+        "combine": {"ms": kms["combine"], "bound": "hbm", "GB/s": bytes_combine / (kms["combine"] * 1e6)},
+    }
+    breakdown["route"]["frac_fp32_alu"] = breakdown["route"]["TFLOP/s"] / fp32_peak
+    breakdown["dispatch"]["frac"] = breakdown["dispatch"]["GB/s"] / hbm_peak
+    breakdown["combine"]["frac"] = breakdown["combine"]["GB/s"] / hbm_peak
+    breakdown["gate_up"]["frac"] = breakdown["gate_up"]["TFLOP/s"] / bf16_peak
+    breakdown["down"]["frac"] = breakdown["down"]["TFLOP/s"] / bf16_peak
+    ffn_ms = kms["gate_up"] + kms["down"]
+    routed_tflops = 6.0 * d * F * R / (ffn_ms * 1e9)
+
+    achieved = breakdown["gate_up"]["TFLOP/s"]
+    roofline = {"kernel": "grouped gate/up SwiGLU GEMM (tcgen05)", "bound": "tensor", "achieved": achieved,
+                "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
+                "peak_kind": f"{peak_kind} bf16 burst", "traffic": None,
+                "flops_per_launch": flops_gu, "ms_per_launch": kms["gate_up"]}
+
+    # ---- end to end through the C ABI with host buffers
+    x_pin = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    loss_pin = torch.empty(2, dtype=torch.float32).pin_memory()
+    cext_pin = torch.empty(N + cfg.M, dtype=torch.int32).pin_memory()
+    xin = torch.empty_like(x)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        xin.copy_(x_pin, non_blocking=True)
+        layer.forward(xin, tnb, out)
+        loss_pin.copy_(out["losses"], non_blocking=True)
+        cext_pin.copy_(out["counts_ext"], non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e = {"value": world * R * args.steps / (e2e_total * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(8 + 4 * (N + cfg.M)),
+           "ms_per_step": e2e_total / args.steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        S = calibrate_sample(inp, args.cpu_seconds)
+        dt, Rs = oracle_sample_run(inp, S)
+        cpu = {"value": Rs / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {S} of {T} tokens, one full oracle forward ({dt:.1f} s)"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 tokens, N(0,1/fan_in) bf16 weights, fp32 router)",
+            "config": workload_config(cfg, args),
+            "real_slots_per_step": R, "tokens_per_s": world * T * args.steps / (total_ms * 1e-3),
+            "routed_ffn_tflops_real_rows": routed_tflops,
+            "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": kernels_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,233 @@
+/*
+ * moe_null.h -- C ABI of the B200 (sm_100a) forward hot path of a token-choice
+ * MoE layer with zero-compute null experts.
+ *
+ * The layer (Kilian et al., "Improving MoE Compute Efficiency by Composing
+ * Weight and Data Sparsity", paper-review page, section 三 技术架构):
+ *
+ *   y = E_shared(x) + sum_{i in top-K, i real} g_i(x) * E_i(x)
+ *
+ * The router emits N real logits plus one null logit (Null Expert 机制); the
+ * null logit is replicated M times before top-K, so the pool has N+M slots
+ * (indices N..N+M-1 are the null copies, which compute nothing). Gates are
+ * renormalised over the selected real experts only. The layer also emits the
+ * load-balance statistics L_bal = N * sum_{i<N+M} f_i P_i (负载均衡损失) and the
+ * Z-loss L_z = mean_t (log sum_{i<N+M} e^{s_i})^2 (Z-Loss).
+ *
+ * Conventions shared by every entry point:
+ *  - All pointers except `dims`, `w` and `out` (host structs) are DEVICE
+ *    pointers on the current CUDA device. bf16 tensors are passed as uint16_t
+ *    bit patterns. All tensors are dense row-major.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
+ *    only enqueues work on it and returns; none synchronises the host except
+ *    moe_get_device_status.
+ *  - The caller allocates and owns every buffer, the workspace included. The
+ *    library allocates no device memory and keeps no per-call state; it does
+ *    cache, per device and process, the SM count and kernel attributes.
+ *  - Return value: MOE_OK (0) or a negative moe_status_t. Argument errors are
+ *    detected on the host before anything is enqueued. A failure detected on
+ *    the device (a bounded wait that ran out, a guard) is recorded in a status
+ *    word inside the workspace; read it with moe_get_device_status.
+ *  - T = 0 is a no-op that returns MOE_OK.
+ *  - Non-finite inputs give undefined routing.
+ *  - Limits: 1 <= N <= 64, 0 <= M, 1 <= K <= 16, K <= N + M, d a multiple of
+ *    128 (128..8192), F and F_shared multiples of 64 (64..16384), T*K < 2^31.
+ *    Outside them: MOE_ERR_UNSUPPORTED (or MOE_ERR_INVALID_ARG for values that
+ *    are never valid, e.g. K < 1, M < 0, T < 0).
+ *
+ * Workspace: moe_workspace_bytes(dims) bytes, 256-byte aligned. moe_route
+ * writes it (it clears what must start at zero itself); moe_dispatch,
+ * moe_aux* and moe_expert_ffn read it. One workspace serves one layer call at
+ * a time: two calls in flight on different streams must use two workspaces.
+ */
+#ifndef MOE_NULL_H
+#define MOE_NULL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_NULL_ABI_VERSION 1
+
+typedef void* moe_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,   /* null pointer, negative size, K < 1, ... */
+  MOE_ERR_UNSUPPORTED = -2,   /* valid but outside this build's limits */
+  MOE_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed */
+  MOE_ERR_TIMEOUT = -4,       /* a device-side bounded wait ran out */
+  MOE_ERR_DEVICE_BOUNDS = -5  /* a device-side guard saw an out-of-range index */
+} moe_status_t;
+
+/* Layer sizes. T tokens, model width d, N real experts, M null copies, top-K,
+ * routed expert ffn width F, shared expert ffn width F_shared. flags: 0. */
+typedef struct moe_dims {
+  int32_t T, d, N, M, K, F, F_shared;
+  uint32_t flags;
+} moe_dims_t;
+
+/* Weights of one layer (device pointers). */
+typedef struct moe_weights {
+  const float* w_router;        /* [N+1, d] fp32; row N is the null logit       */
+  const float* router_bias;     /* [N+1] fp32 or NULL (added to every logit)    */
+  const uint16_t* gate_up;      /* [N, 2F, d] bf16, from moe_pack_gate_up       */
+  const uint16_t* w_down;       /* [N, d, F] bf16                               */
+  const uint16_t* shared_gate_up; /* [2F_shared, d] bf16, from moe_pack_gate_up */
+  const uint16_t* shared_down;  /* [d, F_shared] bf16                           */
+} moe_weights_t;
+
+/* Outputs and intermediates of moe_forward (device pointers). R_cap = T*K. */
+typedef struct moe_outputs {
+  float* logits;        /* [T, N+1] fp32, or NULL to skip                        */
+  int32_t* topk_idx;    /* [T, K] pool indices in rank order                     */
+  float* topk_gate;     /* [T, K] fp32, 0 for null slots                         */
+  int32_t* n_real;      /* [T] real experts per token                            */
+  int32_t* counts;      /* [N] rows per expert                                   */
+  int32_t* offsets;     /* [N+1] exclusive scan of counts; offsets[N] = R        */
+  int32_t* perm_tok;    /* [R_cap] token of each expert-contiguous row (first R) */
+  int32_t* slot_row;    /* [T, K] row of each slot in xs/h/ys, -1 for nulls      */
+  uint16_t* xs;         /* [R_cap, d] bf16 gathered rows                         */
+  uint16_t* h;          /* [R_cap, F] bf16 routed SwiGLU activations             */
+  uint16_t* h_shared;   /* [T, F_shared] bf16 shared SwiGLU activations          */
+  uint16_t* ys;         /* [R_cap, d] bf16 routed expert outputs                 */
+  uint16_t* shared_out; /* [T, d] bf16 shared expert output                      */
+  uint16_t* y;          /* [T, d] bf16 layer output                              */
+  int32_t* counts_ext;  /* [N+M] tokens per pool slot                            */
+  float* P;             /* [N+M] mean routing probability per pool slot          */
+  float* losses;        /* [2] = {L_bal, L_z}                                    */
+} moe_outputs_t;
+
+/* ABI version (MOE_NULL_ABI_VERSION) of the loaded library. */
+MOE_API int moe_abi_version(void);
+
+/* Static text for a moe_status_t value. Never NULL. */
+MOE_API const char* moe_status_string(int status);
+
+/* Host-side check of `dims` against the limits above. */
+MOE_API int moe_check_dims(const moe_dims_t* dims);
+
+/* Workspace size in bytes for `dims` (0 if dims are invalid). */
+MOE_API size_t moe_workspace_bytes(const moe_dims_t* dims);
+
+/* Element count (bf16) of the packed gate/up weights: routed N*2F*d and shared
+ * 2*F_shared*d. Packing interleaves gate and up rows in panels of 64 rows
+ * (64 gate rows of a panel, then the matching 64 up rows), so that one
+ * tensor-core tile holds matching gate and up columns for the SwiGLU epilogue.
+ * Either output pointer of moe_pack_gate_up may be NULL to skip that part. */
+MOE_API size_t moe_packed_gate_up_elems(const moe_dims_t* dims, int shared);
+
+/* One-time weight packing (device copy kernel). w_gate/w_up [N, F, d] ->
+ * gate_up [N, 2F, d]; ws_gate/ws_up [F_shared, d] -> shared_gate_up
+ * [2F_shared, d]. */
+MOE_API int moe_pack_gate_up(const moe_dims_t* dims, const uint16_t* w_gate, const uint16_t* w_up,
+                     const uint16_t* ws_gate, const uint16_t* ws_up, uint16_t* gate_up,
+                     uint16_t* shared_gate_up, moe_stream_t stream);
+
+/* Routing (section 三: Null Expert 机制, 阈值解释, 负载均衡损失, Z-Loss).
+ *  s[t, j] = sum_c fp32(x[t,c]) * w_router[j,c] + bias[j] (+ tok_null_bias[t]
+ *  for j = N), computed in fp32 on CUDA cores. Over the pool [s_0..s_{N-1},
+ *  s_N x M]: lse_t, p_{t,i}; top-K in (value desc, index asc) order -- a real
+ *  logit equal to the null logit precedes every copy, copies fill N, N+1, ...;
+ *  gates = softmax over the selected real logits (0 for nulls, all 0 if none).
+ *  With M = 0 the null logit takes no part in anything.
+ *  x [T, d] bf16; tok_null_bias [T] or NULL; logits_out [T, N+1] or NULL;
+ *  topk_idx [T, K]; topk_gate [T, K]; n_real [T]. Also fills the workspace
+ *  with per-block statistics and the dispatch scan (counts, offsets). */
+MOE_API int moe_route(const moe_dims_t* dims, const uint16_t* x, const float* w_router,
+              const float* router_bias, const float* tok_null_bias, float* logits_out,
+              int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* workspace,
+              moe_stream_t stream);
+
+/* Dispatch (section 三 / 实现: nulls sorted to the end and truncated). After
+ * moe_route with the same workspace. counts [N], offsets [N+1]; the real slots
+ * are laid out expert by expert, tokens ascending inside an expert: perm_tok
+ * [T*K] (first offsets[N] entries valid), slot_row [T, K] (-1 for nulls), and
+ * xs [T*K, d] bf16 with xs[slot_row[t,k]] = x[t]. Null slots cause no memory
+ * traffic. Also reduces the aux statistics into the workspace (see moe_aux). */
+MOE_API int moe_dispatch(const moe_dims_t* dims, const uint16_t* x, const int32_t* topk_idx,
+                 void* workspace, int32_t* counts, int32_t* offsets, int32_t* perm_tok,
+                 int32_t* slot_row, uint16_t* xs, moe_stream_t stream);
+
+/* Expert FFNs (section 三 / 核心公式; 实现: grouped matmul over the truncated
+ * list). Two persistent tcgen05/TMEM/TMA grouped GEMMs with per-expert row
+ * counts read from `offsets` on the device:
+ *   h[r]  = bf16(silu(xs[r] Wg_e^T) * (xs[r] Wu_e^T)),  ys[r] = bf16(h[r] Wd_e^T)
+ * for rows r in [offsets[e], offsets[e+1]); the shared expert is one more group
+ * over all T rows of x: h_shared, shared_out. bf16 in, fp32 accumulation.
+ * h [T*K, F], h_shared [T, F_shared], ys [T*K, d], shared_out [T, d]. */
+MOE_API int moe_expert_ffn(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x,
+                   const int32_t* offsets, const uint16_t* gate_up, const uint16_t* w_down,
+                   const uint16_t* shared_gate_up, const uint16_t* shared_down, uint16_t* h,
+                   uint16_t* h_shared, uint16_t* ys, uint16_t* shared_out, void* workspace,
+                   moe_stream_t stream);
+
+/* The two halves of moe_expert_ffn, for callers that time or schedule them
+ * separately. moe_expert_gate_up writes h and h_shared (the SwiGLU grouped
+ * GEMM); moe_expert_down reads them and writes ys and shared_out. */
+MOE_API int moe_expert_gate_up(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x,
+                       const int32_t* offsets, const uint16_t* gate_up,
+                       const uint16_t* shared_gate_up, uint16_t* h, uint16_t* h_shared,
+                       void* workspace, moe_stream_t stream);
+MOE_API int moe_expert_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* h,
+                    const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* shared_down,
+                    uint16_t* ys, uint16_t* shared_out, void* workspace, moe_stream_t stream);
+
+/* Combine (section 三 / 核心公式): y[t] = bf16(shared_out[t] + sum over real
+ * slots k, in rank order, of topk_gate[t,k] * ys[slot_row[t,k]]), fp32
+ * accumulation, one rounding. y [T, d]. */
+MOE_API int moe_combine(const moe_dims_t* dims, const uint16_t* ys, const uint16_t* shared_out,
+                const float* topk_gate, const int32_t* slot_row, uint16_t* y,
+                moe_stream_t stream);
+
+/* Number of doubles in the additive aux statistics of a token shard:
+ * [counts_real (N) | null histogram (K+1) | sum_t p (N+1) | sum_t lse^2 | T]. */
+MOE_API size_t moe_aux_sums_count(const moe_dims_t* dims);
+
+/* Additive aux statistics of this call's tokens (layout above), for a
+ * data-parallel all-reduce across ranks. After moe_route. sums: device. */
+MOE_API int moe_aux_sums(const moe_dims_t* dims, const void* workspace, double* sums,
+                 moe_stream_t stream);
+
+/* L_bal / L_z from (possibly all-reduced) sums (section 三 / 负载均衡损失,
+ * Z-Loss): counts_ext [N+M] (copy j counts the tokens with more than j null
+ * slots), P [N+M] (copies share the null probability), losses [2] =
+ * {L_bal = N * sum_i f_i P_i with f_i = counts_ext_i / T_total, L_z}. */
+MOE_API int moe_aux_finalize(const moe_dims_t* dims, const double* sums, int32_t* counts_ext,
+                     float* P, float* losses, moe_stream_t stream);
+
+/* moe_aux_sums + moe_aux_finalize on this call's tokens alone. */
+MOE_API int moe_aux(const moe_dims_t* dims, const void* workspace, int32_t* counts_ext, float* P,
+            float* losses, moe_stream_t stream);
+
+/* The whole forward: route, dispatch (+aux), expert FFNs, combine. */
+MOE_API int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* x,
+                const float* tok_null_bias, const moe_outputs_t* out, void* workspace,
+                moe_stream_t stream);
+
+/* Synchronises `stream`, then returns MOE_OK or the first device-side error
+ * recorded in the workspace status word (MOE_ERR_TIMEOUT, ...). */
+MOE_API int moe_get_device_status(const void* workspace, moe_stream_t stream);
+
+/* Clears the workspace status word (enqueued on `stream`). */
+MOE_API int moe_clear_device_status(void* workspace, moe_stream_t stream);
+
+/* Test aid for the failure path: one CTA waits, with the same bounded wait
+ * the GEMM uses, on a shared-memory barrier that nothing arrives at, gives up
+ * after `limit_ns` nanoseconds (1e3..1e10), records MOE_ERR_TIMEOUT in the
+ * workspace status word and returns. The context stays usable. */
+MOE_API int moe_selftest_bounded_wait(void* workspace, uint64_t limit_ns, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_NULL_H */

@@ -1,0 +1,126 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
+and compare with the CPU oracle on the same seeded inputs."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+from token_choice_routing_b200 import inputs as I
+
+# Tolerances for floating-point outputs of the layer.
+Y_REL_FRO = 1e-2        # ||y - y_ref||_F / ||y_ref||_F
+Y_MAX_REL = 5e-2        # max|y - y_ref| / max|y_ref|
+LOSS_REL = 1e-5         # L_bal, L_z
+GATE_REL = 1e-6         # gates from identical fp32 logits
+P_REL = 1e-5
+
+
+def f64(bits):
+    return I.bf16_to_f32(bits).astype(np.float64)
+
+
+def t2bits(t: torch.Tensor) -> np.ndarray:
+    """torch bf16 tensor -> host uint16 bits."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().float().numpy().astype(np.float64)
+
+
+def make_layer(inp, device="cuda"):
+    from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
+    layer = MoENullLayer.from_inputs(inp, device)
+    x = bf16_tensor(inp.x, device)
+    tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(device)
+    return layer, x, tnb
+
+
+def run_forward(inp, device="cuda"):
+    from token_choice_routing_b200 import binding as B
+    layer, x, tnb = make_layer(inp, device)
+    out = layer.forward(x, tnb)
+    torch.cuda.synchronize()
+    st = B.get_device_status(out["workspace"])
+    assert st == B.OK, B.status_string(st)
+    return layer, x, tnb, out
+
+
+def logit_bound(inp):
+    """Rigorous bound on |fp32 router logit - exact| for a length-d fp32 dot
+    product evaluated by sequential FMAs plus bias additions:
+    (d + 3) * 2^-24 * (sum_c |x_c w_jc| + |bias_j| + |offset|) per element."""
+    x = np.abs(f64(inp.x))
+    w = np.abs(inp.w_router.astype(np.float64))
+    mag = x @ w.T + np.abs(inp.bias.astype(np.float64))[None, :]
+    if inp.tok_null_bias is not None:
+        mag[:, -1] += np.abs(inp.tok_null_bias.astype(np.float64))
+    return (inp.cfg.d + 3) * 2.0 ** -24 * mag + 1e-30
+
+
+def oracle_logits(inp):
+    return O.router_logits(f64(inp.x), inp.w_router, inp.bias, inp.tok_null_bias)
+
+
+def check_routing(inp, out, full_gates=True):
+    """Logits within the fp32 bound; top-K, n_real, gates from the GPU logits."""
+    cfg = inp.cfg
+    N, M, K = cfg.N, cfg.M, cfg.K
+    s_gpu = out["logits"].cpu().numpy().astype(np.float64)
+    s_ref = oracle_logits(inp)
+    err = np.abs(s_gpu - s_ref)
+    assert np.all(err <= logit_bound(inp)), float((err / logit_bound(inp)).max())
+    r = O.route(s_gpu, M, K)
+    idx = out["topk_idx"].cpu().numpy()
+    assert np.array_equal(idx, r["idx"]), np.argwhere(idx != r["idx"])[:5]
+    assert np.array_equal(out["n_real"].cpu().numpy(), r["n_real"])
+    g = out["topk_gate"].cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(g, r["gates"], rtol=GATE_REL, atol=1e-7)
+    return r
+
+
+def check_dispatch(inp, out, r):
+    N = inp.cfg.N
+    counts, offsets, perm, slot_row = O.dispatch(r["idx"], N)
+    assert np.array_equal(out["counts"].cpu().numpy(), counts)
+    assert np.array_equal(out["offsets"].cpu().numpy(), offsets)
+    R = int(offsets[-1])
+    assert np.array_equal(out["perm_tok"][:R].cpu().numpy(), perm)
+    assert np.array_equal(out["slot_row"].cpu().numpy(), slot_row)
+    xs = t2bits(out["xs"][:R])
+    assert np.array_equal(xs, inp.x[perm])
+    return counts, offsets, perm, slot_row
+
+
+def check_aux(inp, out, r):
+    cfg = inp.cfg
+    counts_ext, f, P, L_bal, L_z = O.aux_stats(r["idx"], r["p"], r["lse"], cfg.N, cfg.M)
+    assert np.array_equal(out["counts_ext"].cpu().numpy(), counts_ext)
+    np.testing.assert_allclose(out["P"].cpu().numpy(), P, rtol=P_REL, atol=1e-9)
+    lb, lz = out["losses"].cpu().numpy().astype(np.float64)
+    assert abs(lb - L_bal) <= LOSS_REL * abs(L_bal), (lb, L_bal)
+    assert abs(lz - L_z) <= LOSS_REL * abs(L_z), (lz, L_z)
+
+
+def expert_weights(inp):
+    return ((f64(inp.w_gate), f64(inp.w_up), f64(inp.w_down)),
+            (f64(inp.ws_gate), f64(inp.ws_up), f64(inp.ws_down)))
+
+
+def check_y(y_gpu, y_ref):
+    num = np.linalg.norm(y_gpu - y_ref)
+    den = np.linalg.norm(y_ref)
+    assert num <= Y_REL_FRO * den, (num / den)
+    assert np.abs(y_gpu - y_ref).max() <= Y_MAX_REL * np.abs(y_ref).max()
+
+
+def check_layer_output(inp, out, r, tokens=None):
+    ex, sh = expert_weights(inp)
+    x = f64(inp.x)
+    y_ref = O.layer_output(x, r["idx"], r["gates"], inp.cfg.N, ex, sh, tokens=tokens)
+    y_gpu = bf16_f64(out["y"][:inp.cfg.T])
+    if tokens is not None:
+        y_gpu = y_gpu[tokens]
+    check_y(y_gpu, y_ref)
+    return y_ref

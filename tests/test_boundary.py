@@ -1,0 +1,102 @@
+"""The C-ABI library: it loads, exports every entry point the header declares,
+and rejects bad arguments on the host (no GPU needed for any call here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_null.h")
+LIB = os.path.join(ROOT, "token_choice_routing_b200", "libmoe_null.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from token_choice_routing_b200 import build
+        build.build()
+    from token_choice_routing_b200 import binding
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux", "moe_forward",
+                 "moe_workspace_bytes", "moe_get_device_status", "moe_aux_sums", "moe_aux_finalize"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    so = C.CDLL(LIB)
+    for name in declared_functions():
+        assert hasattr(so, name), name
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.LIB.moe_abi_version() == 1
+    for code in (0, -1, -2, -3, -4, -5, 7):
+        assert isinstance(lib.status_string(code), str) and lib.status_string(code)
+
+
+def good():
+    from token_choice_routing_b200 import binding as B
+    return B.dims(256, 128, 8, 8, 4, 64, 64)
+
+
+def test_check_dims(lib):
+    B = lib
+    assert B.check_dims(good()) == B.OK
+    bad_arg = [dict(T=-1), dict(K=0), dict(M=-1), dict(N=0), dict(K=17 + 0, N=8, M=8), dict(d=0), dict(F=0)]
+    for kw in bad_arg:
+        v = dict(T=256, d=128, N=8, M=8, K=4, F=64, F_shared=64)
+        v.update(kw)
+        assert B.check_dims(B.dims(**v)) == B.ERR_INVALID_ARG, kw
+    unsupported = [dict(N=65, M=0, K=4), dict(K=17, N=64, M=64), dict(d=192), dict(d=16384), dict(F=96),
+                   dict(F_shared=32), dict(T=1 << 29, K=8)]
+    for kw in unsupported:
+        v = dict(T=256, d=128, N=8, M=8, K=4, F=64, F_shared=64)
+        v.update(kw)
+        assert B.check_dims(B.dims(**v)) == B.ERR_UNSUPPORTED, kw
+    dm = good()
+    dm.flags = 1
+    assert B.check_dims(dm) == B.ERR_INVALID_ARG
+
+
+def test_workspace_and_sizes(lib):
+    B = lib
+    assert B.workspace_bytes(good()) > 0
+    assert B.workspace_bytes(B.dims(-1, 128, 8, 8, 4, 64, 64)) == 0
+    small = B.workspace_bytes(B.dims(1000, 1024, 64, 64, 4, 768, 768))
+    big = B.workspace_bytes(B.dims(100000, 1024, 64, 64, 4, 768, 768))
+    assert big > small and big % 256 == 0
+    assert B.aux_sums_count(good()) == 8 + 5 + 9 + 2
+    assert B.packed_gate_up_elems(good(), False) == 8 * 2 * 64 * 128
+    assert B.packed_gate_up_elems(good(), True) == 2 * 64 * 128
+
+
+def test_host_side_rejections_touch_no_device(lib):
+    B = lib
+    L = B.LIB
+    dm = good()
+    nul = None
+    # null pointers with valid dims -> INVALID_ARG before any CUDA call
+    assert L.moe_route(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_dispatch(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_combine(C.byref(dm), nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_aux(C.byref(dm), nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_forward(C.byref(dm), nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_get_device_status(nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(nul, 1000, nul) == B.ERR_INVALID_ARG
+    # invalid dims are rejected first
+    bad = B.dims(256, 100, 8, 8, 4, 64, 64)
+    assert L.moe_route(C.byref(bad), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_UNSUPPORTED
+    assert L.moe_check_dims(None) == B.ERR_INVALID_ARG
+    # T = 0 is a no-op
+    zero = B.dims(0, 128, 8, 8, 4, 64, 64)
+    assert L.moe_route(C.byref(zero), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.OK

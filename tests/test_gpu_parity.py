@@ -1,0 +1,205 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Routing outputs (top-K indices, counts, offsets, permutation, slot rows, the
+gathered rows) must be bit-exact with the oracle run on the GPU's fp32 logits;
+logits within a rigorous fp32 dot-product bound of the oracle's fp64 logits;
+gates to 1e-6; y to rel. Frobenius 1e-2 and max|dy| <= 5e-2 max|y|; L_bal and
+L_z to 1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from token_choice_routing_b200 import inputs as I
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": I.CONFIGS["tiny"],
+    # several route tiles with a ragged tail, N not a multiple of 8, M < K
+    "ragged_a": I.small_config("ragged_a", T=200, d=256, N=5, F=128, F_shared=192, K=3, M=1, config_id=901),
+    "ragged_b": I.small_config("ragged_b", T=333, d=384, N=13, F=192, F_shared=64, K=5, M=9, config_id=902),
+    "m0": I.small_config("m0", T=130, d=256, N=16, F=128, F_shared=128, K=2, M=0, config_id=903),
+    "k1": I.small_config("k1", T=257, d=128, N=32, F=64, F_shared=64, K=1, M=32, config_id=904),
+    "n64_k16": I.small_config("n64_k16", T=190, d=512, N=64, F=256, F_shared=256, K=16, M=48, config_id=905),
+    "t1": I.small_config("t1", T=1, d=128, N=8, F=64, F_shared=64, K=4, M=8, config_id=906),
+    "skew_small": I.small_config("skew_small", T=512, d=256, N=64, F=128, F_shared=128, K=8, M=64,
+                                 config_id=907, skew=True, seqs=2),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layer_full_parity(name):
+    cfg = SMALL[name]
+    inp = I.make_inputs(cfg)
+    if cfg.name.startswith("ragged") or cfg.name in ("k1", "n64_k16", "t1"):
+        inp.bias[cfg.N] = np.float32(0.3)
+    layer, x, tnb, out = H.run_forward(inp)
+    r = H.check_routing(inp, out)
+    H.check_dispatch(inp, out, r)
+    H.check_aux(inp, out, r)
+    # each GEMM against the oracle's definition on the GPU's own inputs
+    counts, offsets, perm, slot_row = O.dispatch(r["idx"], cfg.N)
+    R = int(offsets[-1])
+    ex, sh = H.expert_weights(inp)
+    xs = H.f64(inp.x)[perm]
+    h_gpu = H.bf16_f64(out["h"][:R])
+    for e in range(cfg.N):
+        a, b = offsets[e], offsets[e + 1]
+        if a == b:
+            continue
+        g = xs[a:b] @ ex[0][e].T
+        u = xs[a:b] @ ex[1][e].T
+        h_ref = g / (1 + np.exp(-g)) * u
+        H.check_y(h_gpu[a:b], h_ref)
+        ys_ref = h_gpu[a:b] @ ex[2][e].T
+        H.check_y(H.bf16_f64(out["ys"][a:b]), ys_ref)
+    xf = H.f64(inp.x)
+    g = xf @ sh[0].T
+    u = xf @ sh[1].T
+    H.check_y(H.bf16_f64(out["h_shared"][:cfg.T]), g / (1 + np.exp(-g)) * u)
+    H.check_y(H.bf16_f64(out["shared_out"][:cfg.T]), H.bf16_f64(out["h_shared"][:cfg.T]) @ sh[2].T)
+    H.check_layer_output(inp, out, r)
+
+
+@pytest.mark.parametrize("name", ["qwen3_0p6b", "qwen3_1p7b"])
+def test_full_size_layer_parity_sampled(name):
+    cfg = I.CONFIGS[name]
+    inp = I.make_inputs(cfg)
+    layer, x, tnb, out = H.run_forward(inp)
+    r = H.check_routing(inp, out)
+    H.check_dispatch(inp, out, r)
+    H.check_aux(inp, out, r)
+    rng = np.random.default_rng(0)
+    tokens = np.sort(rng.choice(cfg.T, size=384, replace=False))
+    tokens = np.concatenate([tokens, [0, cfg.T - 1]])
+    H.check_layer_output(inp, out, r, tokens=tokens)
+    # mean real count near rho*K (the calibrated null bias)
+    assert abs(out["n_real"].float().mean().item() - cfg.rho * cfg.K) < 0.02
+
+
+@pytest.mark.parametrize("name", ["sweep_k2_m0", "sweep_k3_m32", "sweep_k4_m64", "sweep_k8_m192", "skew"])
+def test_large_configs_routing_and_sampled_output(name):
+    cfg = I.CONFIGS[name]
+    inp = I.make_inputs(cfg)
+    layer, x, tnb, out = H.run_forward(inp)
+    r = H.check_routing(inp, out)
+    H.check_dispatch(inp, out, r)
+    H.check_aux(inp, out, r)
+    rng = np.random.default_rng(1)
+    tokens = np.sort(rng.choice(cfg.T, size=192, replace=False))
+    H.check_layer_output(inp, out, r, tokens=tokens)
+
+
+def test_all_null_tokens_get_only_the_shared_expert():
+    cfg = I.small_config("allnull", T=100, d=256, N=8, F=64, F_shared=128, K=4, M=8, config_id=910)
+    inp = I.make_inputs(cfg, null_bias=1000.0)
+    layer, x, tnb, out = H.run_forward(inp)
+    assert int(out["n_real"].sum()) == 0
+    assert int(out["offsets"][-1]) == 0
+    assert torch.equal(out["y"][:cfg.T], out["shared_out"][:cfg.T])
+    assert torch.all(out["topk_gate"] == 0)
+    r = H.check_routing(inp, out)
+    H.check_aux(inp, out, r)
+    H.check_layer_output(inp, out, r)
+
+
+def test_exact_ties_break_by_index():
+    # duplicated router rows make exactly equal fp32 logits; the null row is a
+    # copy of real row 2, so real 2 ties the null logit and must precede every copy
+    cfg = I.small_config("ties", T=150, d=256, N=8, F=64, F_shared=64, K=6, M=4, config_id=911)
+    inp = I.make_inputs(cfg)
+    w = inp.w_router
+    w[3] = w[1]
+    w[5] = w[1]
+    w[cfg.N] = w[2]
+    inp.bias[:] = 0
+    layer, x, tnb, out = H.run_forward(inp)
+    lg = out["logits"].cpu().numpy()
+    assert np.array_equal(lg[:, 3], lg[:, 1]) and np.array_equal(lg[:, cfg.N], lg[:, 2])
+    r = H.check_routing(inp, out)
+    H.check_dispatch(inp, out, r)
+    idx = out["topk_idx"].cpu().numpy()
+    for t in range(cfg.T):
+        row = idx[t].tolist()
+        if 2 in row and cfg.N in row:
+            assert row.index(2) < row.index(cfg.N)
+    H.check_layer_output(inp, out, r)
+
+
+def _subset(inp, cfg, rows):
+    import dataclasses
+    return dataclasses.replace(inp, cfg=cfg, x=np.ascontiguousarray(inp.x[rows]),
+                               tok_null_bias=None if inp.tok_null_bias is None else inp.tok_null_bias[rows])
+
+
+def test_k4_half_reproduces_k2_dense_bitwise():
+    """Solution-space preservation (review page, section 三 / 解决方案空间保持):
+    with each token's null logit strictly between its 2nd and 3rd real logit,
+    K=4/M=64 selects the same two reals as K=2/M=0 and gives the same y."""
+    T, d, N, F = 1000, 512, 64, 256
+    draw = I.small_config("k4k2_draw", T=1400, d=d, N=N, F=F, F_shared=F, K=4, M=64, config_id=912)
+    inp = I.make_inputs(draw)
+    inp.bias[:] = 0
+    s = O.router_logits(H.f64(inp.x), inp.w_router, inp.bias)
+    srt = -np.sort(-s[:, :N], axis=1)
+    gap = srt[:, 1] - srt[:, 2]
+    rows = np.nonzero(gap > 1e-2)[0][:T]  # a margin the fp32 logits cannot cross
+    assert rows.size == T
+    cfg4 = I.small_config("k4k2", T=T, d=d, N=N, F=F, F_shared=F, K=4, M=64, config_id=912)
+    cfg2 = I.small_config("k4k2_dense", T=T, d=d, N=N, F=F, F_shared=F, K=2, M=0, config_id=912)
+    inp4 = _subset(inp, cfg4, rows)
+    inp4.tok_null_bias = (0.5 * (srt[rows, 1] + srt[rows, 2]) - s[rows, N]).astype(np.float32)
+    inp2 = _subset(inp, cfg2, rows)
+    layer4, _, _, out4 = H.run_forward(inp4)
+    layer2, _, _, out2 = H.run_forward(inp2)
+    assert np.all(out4["n_real"].cpu().numpy() == 2)
+    H.check_routing(inp4, out4)
+    H.check_routing(inp2, out2)
+    assert torch.equal(out4["topk_idx"][:, :2], out2["topk_idx"])
+    assert torch.all(out4["topk_idx"][:, 2:] >= N)
+    assert torch.equal(out4["topk_gate"][:, :2], out2["topk_gate"])
+    assert torch.equal(out4["counts"], out2["counts"])
+    assert torch.equal(out4["offsets"], out2["offsets"])
+    R = int(out2["offsets"][-1])
+    assert torch.equal(out4["perm_tok"][:R], out2["perm_tok"][:R])
+    assert torch.equal(out4["y"], out2["y"])
+
+
+def test_zero_tokens_is_a_noop():
+    from token_choice_routing_b200 import binding as B
+    cfg = I.CONFIGS["tiny"]
+    inp = I.make_inputs(cfg)
+    layer, x, tnb, _ = H.make_layer(inp)
+    out = layer.alloc(0)
+    layer.forward(x[:0], None, out)
+    torch.cuda.synchronize()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    from token_choice_routing_b200 import binding as B
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    B.selftest_bounded_wait(ws, 2_000_000)  # 2 ms on a barrier nothing arrives at
+    assert B.get_device_status(ws) == B.ERR_TIMEOUT
+    B.clear_device_status(ws)
+    assert B.get_device_status(ws) == B.OK
+    # the context is still usable: a full small forward afterwards
+    inp = I.make_inputs(I.CONFIGS["tiny"])
+    layer, x, tnb, out = H.run_forward(inp)
+    r = H.check_routing(inp, out)
+    H.check_layer_output(inp, out, r)
+
+
+def test_repeated_calls_same_workspace_deterministic():
+    inp = I.make_inputs(I.CONFIGS["tiny"])
+    layer, x, tnb = H.make_layer(inp)
+    out = layer.alloc(inp.cfg.T)
+    layer.forward(x, tnb, out)
+    y1 = out["y"].clone()
+    l1 = out["losses"].clone()
+    for _ in range(3):
+        layer.forward(x, tnb, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out["y"], y1) and torch.equal(out["losses"], l1)

@@ -1,0 +1,202 @@
+"""ctypes binding of libmoe_null.so (include/moe_null.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. Tensors are torch CUDA tensors; their data pointers and the current
+CUDA stream are passed through the C ABI. There is no CPU fallback: if the
+library is missing this module raises on import.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_null.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_BOUNDS = 0, -1, -2, -3, -4, -5
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({status_string(code)})")
+        self.code = code
+
+
+class Dims(C.Structure):
+    _fields_ = [("T", C.c_int32), ("d", C.c_int32), ("N", C.c_int32), ("M", C.c_int32),
+                ("K", C.c_int32), ("F", C.c_int32), ("F_shared", C.c_int32), ("flags", C.c_uint32)]
+
+
+class Weights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("w_router", "router_bias", "gate_up", "w_down",
+                                           "shared_gate_up", "shared_down")]
+
+
+OUTPUT_FIELDS = ("logits", "topk_idx", "topk_gate", "n_real", "counts", "offsets", "perm_tok",
+                 "slot_row", "xs", "h", "h_shared", "ys", "shared_out", "y", "counts_ext", "P",
+                 "losses")
+
+
+class Outputs(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in OUTPUT_FIELDS]
+
+
+def _load() -> C.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
+                          "(run python -m token_choice_routing_b200.build)")
+    lib = C.CDLL(LIB_PATH)
+    vp, i32, sz = C.c_void_p, C.c_int, C.c_size_t
+    pd = C.POINTER(Dims)
+    sig = {
+        "moe_abi_version": (i32, []),
+        "moe_status_string": (C.c_char_p, [i32]),
+        "moe_check_dims": (i32, [pd]),
+        "moe_workspace_bytes": (sz, [pd]),
+        "moe_packed_gate_up_elems": (sz, [pd, i32]),
+        "moe_pack_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_route": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_dispatch": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_ffn": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_combine": (i32, [pd, vp, vp, vp, vp, vp, vp]),
+        "moe_aux_sums_count": (sz, [pd]),
+        "moe_aux_sums": (i32, [pd, vp, vp, vp]),
+        "moe_aux_finalize": (i32, [pd, vp, vp, vp, vp, vp]),
+        "moe_aux": (i32, [pd, vp, vp, vp, vp, vp]),
+        "moe_forward": (i32, [pd, C.POINTER(Weights), vp, vp, C.POINTER(Outputs), vp, vp]),
+        "moe_get_device_status": (i32, [vp, vp]),
+        "moe_clear_device_status": (i32, [vp, vp]),
+        "moe_selftest_bounded_wait": (i32, [vp, C.c_uint64, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    if lib.moe_abi_version() != 1:
+        raise ImportError("libmoe_null ABI version mismatch")
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(code: int) -> str:
+    return LIB.moe_status_string(int(code)).decode()
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, code: int):
+    if code != OK:
+        raise MoEError(fn, code)
+
+
+def dims(T, d, N, M, K, F, F_shared) -> Dims:
+    return Dims(int(T), int(d), int(N), int(M), int(K), int(F), int(F_shared), 0)
+
+
+def check_dims(dm: Dims) -> int:
+    return LIB.moe_check_dims(C.byref(dm))
+
+
+def workspace_bytes(dm: Dims) -> int:
+    return int(LIB.moe_workspace_bytes(C.byref(dm)))
+
+
+def aux_sums_count(dm: Dims) -> int:
+    return int(LIB.moe_aux_sums_count(C.byref(dm)))
+
+
+def packed_gate_up_elems(dm: Dims, shared: bool) -> int:
+    return int(LIB.moe_packed_gate_up_elems(C.byref(dm), 1 if shared else 0))
+
+
+def pack_gate_up(dm, w_gate, w_up, ws_gate, ws_up, gate_up, shared_gate_up, stream=None):
+    _check("moe_pack_gate_up", LIB.moe_pack_gate_up(C.byref(dm), _p(w_gate), _p(w_up), _p(ws_gate),
+                                                     _p(ws_up), _p(gate_up), _p(shared_gate_up),
+                                                     _stream(stream)))
+
+
+def route(dm, x, w_router, bias, tok_null_bias, logits, topk_idx, topk_gate, n_real, ws, stream=None):
+    _check("moe_route", LIB.moe_route(C.byref(dm), _p(x), _p(w_router), _p(bias), _p(tok_null_bias),
+                                      _p(logits), _p(topk_idx), _p(topk_gate), _p(n_real), _p(ws),
+                                      _stream(stream)))
+
+
+def dispatch(dm, x, topk_idx, ws, counts, offsets, perm_tok, slot_row, xs, stream=None):
+    _check("moe_dispatch", LIB.moe_dispatch(C.byref(dm), _p(x), _p(topk_idx), _p(ws), _p(counts),
+                                            _p(offsets), _p(perm_tok), _p(slot_row), _p(xs),
+                                            _stream(stream)))
+
+
+def expert_ffn(dm, xs, x, offsets, gate_up, w_down, shared_gate_up, shared_down, h, h_shared, ys,
+               shared_out, ws, stream=None):
+    _check("moe_expert_ffn", LIB.moe_expert_ffn(C.byref(dm), _p(xs), _p(x), _p(offsets), _p(gate_up),
+                                                _p(w_down), _p(shared_gate_up), _p(shared_down), _p(h),
+                                                _p(h_shared), _p(ys), _p(shared_out), _p(ws),
+                                                _stream(stream)))
+
+
+def expert_gate_up(dm, xs, x, offsets, gate_up, shared_gate_up, h, h_shared, ws, stream=None):
+    _check("moe_expert_gate_up", LIB.moe_expert_gate_up(C.byref(dm), _p(xs), _p(x), _p(offsets), _p(gate_up),
+                                                        _p(shared_gate_up), _p(h), _p(h_shared), _p(ws),
+                                                        _stream(stream)))
+
+
+def expert_down(dm, offsets, h, h_shared, w_down, shared_down, ys, shared_out, ws, stream=None):
+    _check("moe_expert_down", LIB.moe_expert_down(C.byref(dm), _p(offsets), _p(h), _p(h_shared), _p(w_down),
+                                                  _p(shared_down), _p(ys), _p(shared_out), _p(ws),
+                                                  _stream(stream)))
+
+
+def combine(dm, ys, shared_out, topk_gate, slot_row, y, stream=None):
+    _check("moe_combine", LIB.moe_combine(C.byref(dm), _p(ys), _p(shared_out), _p(topk_gate),
+                                          _p(slot_row), _p(y), _stream(stream)))
+
+
+def aux(dm, ws, counts_ext, P, losses, stream=None):
+    _check("moe_aux", LIB.moe_aux(C.byref(dm), _p(ws), _p(counts_ext), _p(P), _p(losses), _stream(stream)))
+
+
+def aux_sums(dm, ws, sums, stream=None):
+    _check("moe_aux_sums", LIB.moe_aux_sums(C.byref(dm), _p(ws), _p(sums), _stream(stream)))
+
+
+def aux_finalize(dm, sums, counts_ext, P, losses, stream=None):
+    _check("moe_aux_finalize", LIB.moe_aux_finalize(C.byref(dm), _p(sums), _p(counts_ext), _p(P),
+                                                    _p(losses), _stream(stream)))
+
+
+def forward(dm, weights: Weights, x, tok_null_bias, outputs: Outputs, ws, stream=None):
+    _check("moe_forward", LIB.moe_forward(C.byref(dm), C.byref(weights), _p(x), _p(tok_null_bias),
+                                          C.byref(outputs), _p(ws), _stream(stream)))
+
+
+def get_device_status(ws, stream=None) -> int:
+    return LIB.moe_get_device_status(_p(ws), _stream(stream))
+
+
+def clear_device_status(ws, stream=None):
+    _check("moe_clear_device_status", LIB.moe_clear_device_status(_p(ws), _stream(stream)))
+
+
+def selftest_bounded_wait(ws, limit_ns: int, stream=None):
+    _check("moe_selftest_bounded_wait", LIB.moe_selftest_bounded_wait(_p(ws), int(limit_ns), _stream(stream)))

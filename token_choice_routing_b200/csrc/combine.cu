@@ -1,0 +1,75 @@
+// moe_combine: y[t] = E_shared(x_t) + sum over the token's real slots of
+// g_{t,k} * E_e(x_t) (Kilian et al., "Improving MoE Compute Efficiency by
+// Composing Weight and Data Sparsity", review page, section 三 / 核心公式).
+// Null experts output zero, so null slots (slot_row = -1) are skipped.
+// Written as a gather (each token reads its own rows of ys) so it is
+// deterministic: fp32 accumulation in rank order, one bf16 rounding.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
+               const float* __restrict__ gate, const int32_t* __restrict__ slot_row,
+               uint16_t* __restrict__ y, int T, int d, int K, long long rcap, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = kCombineThreads / 32;
+  const int nch = d >> 3;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    int row = -1;
+    float g = 0.f;
+    if (lane < K) {
+      row = __ldg(slot_row + (size_t)t * K + lane);
+      g = __ldg(gate + (size_t)t * K + lane);
+      if (row >= rcap) {
+        if (status) atomicOr(status, kStatusBounds);
+        row = -1;
+      }
+    }
+    for (int c0 = 0; c0 < nch; c0 += 32) {
+      const int c = c0 + lane;
+      const bool ok = c < nch;
+      float acc[8];
+      {
+        const uint4 v = ok ? __ldg(reinterpret_cast<const uint4*>(sh + (size_t)t * d) + c)
+                           : make_uint4(0u, 0u, 0u, 0u);
+        acc[0] = bf16lo(v.x); acc[1] = bf16hi(v.x); acc[2] = bf16lo(v.y); acc[3] = bf16hi(v.y);
+        acc[4] = bf16lo(v.z); acc[5] = bf16hi(v.z); acc[6] = bf16lo(v.w); acc[7] = bf16hi(v.w);
+      }
+      for (int k = 0; k < K; ++k) {
+        const int r = __shfl_sync(0xffffffffu, row, k);
+        const float gk = __shfl_sync(0xffffffffu, g, k);
+        if (r >= 0 && ok) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(ys + (size_t)r * d) + c);
+          acc[0] = fmaf(gk, bf16lo(v.x), acc[0]); acc[1] = fmaf(gk, bf16hi(v.x), acc[1]);
+          acc[2] = fmaf(gk, bf16lo(v.y), acc[2]); acc[3] = fmaf(gk, bf16hi(v.y), acc[3]);
+          acc[4] = fmaf(gk, bf16lo(v.z), acc[4]); acc[5] = fmaf(gk, bf16hi(v.z), acc[5]);
+          acc[6] = fmaf(gk, bf16lo(v.w), acc[6]); acc[7] = fmaf(gk, bf16hi(v.w), acc[7]);
+        }
+      }
+      if (ok) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        reinterpret_cast<uint4*>(y + (size_t)t * d)[c] = o;
+      }
+    }
+  }
+}
+
+int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
+                   const float* topk_gate, const int32_t* slot_row, uint16_t* y, cudaStream_t st) {
+  const int wpb = kCombineThreads / 32;
+  int grid = (d.T + wpb - 1) / wpb;
+  const int cap = sm_count() * 8;
+  if (grid > cap) grid = cap;
+  combine_kernel<<<grid, kCombineThreads, 0, st>>>(ys, shared_out, topk_gate, slot_row, y, d.T, d.d,
+                                                   d.K, (long long)d.T * d.K, nullptr);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace moe

@@ -1,0 +1,284 @@
+// moe_dispatch: the expert-contiguous permutation of the real (token, expert)
+// slots, with the row gather of x into xs; and the aux-loss reductions.
+//
+// Kilian et al., "Improving MoE Compute Efficiency by Composing Weight and Data
+// Sparsity" (review page, section 三 / 实现): null indices (>= N) are moved to
+// the end of the sorted (token, expert) list and cut off before the grouped
+// matmul. Here no sort is run: the route kernel already produced, per block of
+// 64 tokens, each slot's rank among the block's tokens that chose the same
+// expert, and the per-(expert, block) base row. A slot's row is base + rank,
+// which is the stable (expert, token) order. Null slots are skipped before any
+// load, so they cost no memory traffic.
+//
+// Aux (same page, 负载均衡损失 and Z-Loss): L_bal = N * sum_{i<N+M} f_i P_i with
+// f_i = count_i / T and P_i = mean_t p_{t,i}; L_z = mean_t lse_t^2. Per-block
+// fp32 partials from the route kernel are summed here in fp64 in block order.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+struct AuxPtrs {
+  const int32_t* counts;  // [N] real counts (route scan)
+  const float* ppart;     // [nblk][N+1]
+  const float* lsq;       // [nblk]
+  const int32_t* hist;    // [nblk][K+1]
+  int nblk, N, M, K, T;
+};
+
+// sums layout: [counts_real N | hist K+1 | psum N+1 | lsq | T]
+__device__ void aux_sums_block(const AuxPtrs& p, double* sums) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int N = p.N, K = p.K, nblk = p.nblk;
+  double* s_cnt = sums;
+  double* s_hist = sums + N;
+  double* s_psum = s_hist + (K + 1);
+  double* s_lsq = s_psum + (N + 1);
+  for (int e = tid; e < N; e += blockDim.x) s_cnt[e] = (double)p.counts[e];
+  // null histogram: one warp per bucket, lanes stride over blocks
+  for (int c = warp; c <= K; c += nwarps) {
+    long long acc = 0;
+    for (int b = lane; b < nblk; b += 32) acc += p.hist[(size_t)b * (K + 1) + c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) s_hist[c] = (double)acc;
+  }
+  // probability sums: column i, phases over blocks; then phases combined in order
+  __shared__ double s_ph[8][kMaxN + 1];
+  const int ncol = N + 1;
+  const int nph = min(8, (int)blockDim.x / ncol);
+  {
+    const int col = tid % ncol, ph = tid / ncol;
+    if (ph < nph) {
+      double acc = 0.0;
+      for (int b = ph; b < nblk; b += nph) acc += (double)p.ppart[(size_t)b * ncol + col];
+      s_ph[ph][col] = acc;
+    }
+  }
+  // lse^2: last warp, lane-strided then a fixed shuffle tree
+  if (warp == nwarps - 1) {
+    double acc = 0.0;
+    for (int b = lane; b < nblk; b += 32) acc += (double)p.lsq[b];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      *s_lsq = acc;
+      s_lsq[1] = (double)p.T;
+    }
+  }
+  __syncthreads();
+  for (int col = tid; col < ncol; col += blockDim.x) {
+    double acc = 0.0;
+    for (int ph = 0; ph < nph; ++ph) acc += s_ph[ph][col];
+    s_psum[col] = acc;
+  }
+  __syncthreads();
+}
+
+__device__ void aux_finalize_block(const double* sums, int N, int M, int K, int32_t* counts_ext,
+                                   float* P, float* losses) {
+  const int tid = threadIdx.x;
+  const double* s_cnt = sums;
+  const double* s_hist = sums + N;
+  const double* s_psum = s_hist + (K + 1);
+  const double Tt = s_psum[N + 1 + 1];
+  const double inv = Tt > 0.0 ? 1.0 / Tt : 0.0;
+  for (int i = tid; i < N + M; i += blockDim.x) {
+    if (i < N) {
+      if (counts_ext) counts_ext[i] = (int32_t)s_cnt[i];
+      if (P) P[i] = (float)(s_psum[i] * inv);
+    } else {
+      const int j = i - N;  // copy j is taken by tokens with more than j null slots
+      double c = 0.0;
+      for (int q = j + 1; q <= K; ++q) c += s_hist[q];
+      if (counts_ext) counts_ext[i] = (int32_t)c;
+      if (P) P[i] = (float)(s_psum[N] * inv);
+    }
+  }
+  if (tid == 0 && losses) {
+    double acc = 0.0;
+    for (int i = 0; i < N; ++i) acc += s_cnt[i] * s_psum[i];
+    double nulls = 0.0;
+    for (int q = 1; q <= K; ++q) nulls += (double)q * s_hist[q];
+    acc += nulls * s_psum[N];
+    losses[0] = (float)((double)N * acc * inv * inv);
+    losses[1] = (float)(s_psum[N + 1] * inv);
+  }
+}
+
+__global__ void __launch_bounds__(256) aux_kernel(AuxPtrs p, double* sums_out, const double* sums_in,
+                                                  int32_t* counts_ext, float* P, float* losses) {
+  __shared__ double s_sums[kMaxN + kMaxK + 1 + kMaxN + 1 + 2];
+  const int n = p.N + (p.K + 1) + (p.N + 1) + 2;
+  if (sums_in == nullptr) {
+    aux_sums_block(p, s_sums);
+    if (sums_out)
+      for (int i = threadIdx.x; i < n; i += blockDim.x) sums_out[i] = s_sums[i];
+  } else {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_sums[i] = sums_in[i];
+    __syncthreads();
+  }
+  if (counts_ext || P || losses) aux_finalize_block(s_sums, p.N, p.M, p.K, counts_ext, P, losses);
+}
+
+struct DispatchArgs {
+  const uint16_t* x;
+  const int32_t* topk_idx;
+  const int32_t* lrank;
+  const int32_t* bases;  // [N][nblk]
+  const int32_t* ws_counts;
+  const int32_t* ws_offsets;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm_tok;
+  int32_t* slot_row;
+  uint16_t* xs;
+  uint32_t* status;
+  // fused aux (block 0) outputs, or all null
+  AuxPtrs aux;
+  double* sums;
+  int32_t* counts_ext;
+  float* P;
+  float* losses;
+  int fuse_aux;
+  int T, d, N, M, K, nblk;
+};
+
+constexpr int kDispatchThreads = 256;
+
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs a) {
+  int blk = blockIdx.x;
+  if (a.fuse_aux) {
+    if (blk == 0) {  // scheduled first, so the reduction overlaps the gather
+      __shared__ double s_sums[kMaxN + kMaxK + 1 + kMaxN + 1 + 2];
+      aux_sums_block(a.aux, s_sums);
+      if (a.sums)
+        for (int i = threadIdx.x; i < a.N + a.K + 1 + a.N + 1 + 2; i += blockDim.x) a.sums[i] = s_sums[i];
+      aux_finalize_block(s_sums, a.N, a.M, a.K, a.counts_ext, a.P, a.losses);
+      return;
+    }
+    --blk;
+  }
+  const int nblocks = gridDim.x - (a.fuse_aux ? 1 : 0);
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (blk == 0) {
+    for (int i = tid; i <= a.N; i += blockDim.x) {
+      a.offsets[i] = a.ws_offsets[i];
+      if (i < a.N) a.counts[i] = a.ws_counts[i];
+    }
+  }
+  const int K = a.K, N = a.N, d = a.d;
+  const long long rcap = (long long)a.T * K;
+  const int nch = d >> 3;  // 16-byte chunks per row
+  const int wpb = kDispatchThreads / 32;
+  for (int t = blk * wpb + (tid >> 5); t < a.T; t += nblocks * wpb) {
+    int dest = -1;
+    if (lane < K) {
+      const int id = __ldg(a.topk_idx + (size_t)t * K + lane);
+      if (id >= 0 && id < N) {
+        dest = __ldg(a.bases + (size_t)id * a.nblk + t / kRouteTokens) + __ldg(a.lrank + (size_t)t * K + lane);
+        if (dest < 0 || dest >= rcap) {
+          atomicOr(a.status, kStatusBounds);
+          dest = -1;
+        } else {
+          a.perm_tok[dest] = t;
+        }
+      } else if (id < 0 || id >= N + a.M) {
+        atomicOr(a.status, kStatusBounds);
+      }
+      a.slot_row[(size_t)t * K + lane] = dest;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * d);
+    for (int c0 = 0; c0 < nch; c0 += 32) {  // warp-uniform trip count (shuffles below)
+      const int c = c0 + lane;
+      const bool ok = c < nch;
+      const uint4 v = ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+      for (int k = 0; k < K; ++k) {
+        const int dk = __shfl_sync(0xffffffffu, dest, k);
+        if (dk >= 0 && ok) reinterpret_cast<uint4*>(a.xs + (size_t)dk * d)[c] = v;
+      }
+    }
+  }
+}
+
+static AuxPtrs aux_ptrs(const moe_dims_t& d, const void* ws) {
+  const WsLayout L = ws_layout(d);
+  AuxPtrs p{};
+  p.counts = ws_ptr<int32_t>(ws, L.counts);
+  p.ppart = ws_ptr<float>(ws, L.ppart);
+  p.lsq = ws_ptr<float>(ws, L.lsq);
+  p.hist = ws_ptr<int32_t>(ws, L.hist);
+  p.nblk = L.nblk;
+  p.N = d.N;
+  p.M = d.M;
+  p.K = d.K;
+  p.T = d.T;
+  return p;
+}
+
+int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_idx, void* ws,
+                    int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* slot_row,
+                    uint16_t* xs, int32_t* counts_ext, float* P, float* losses, cudaStream_t st) {
+  const WsLayout L = ws_layout(d);
+  DispatchArgs a{};
+  a.x = x;
+  a.topk_idx = topk_idx;
+  a.lrank = ws_ptr<int32_t>(ws, L.lrank);
+  a.bases = ws_ptr<int32_t>(ws, L.bases);
+  a.ws_counts = ws_ptr<int32_t>(ws, L.counts);
+  a.ws_offsets = ws_ptr<int32_t>(ws, L.offsets);
+  a.counts = counts;
+  a.offsets = offsets;
+  a.perm_tok = perm_tok;
+  a.slot_row = slot_row;
+  a.xs = xs;
+  a.status = ws_ptr<uint32_t>(ws, L.hdr);
+  a.aux = aux_ptrs(d, ws);
+  a.sums = ws_ptr<double>(ws, L.sums);
+  a.counts_ext = counts_ext;
+  a.P = P;
+  a.losses = losses;
+  a.fuse_aux = 1;
+  a.T = d.T;
+  a.d = d.d;
+  a.N = d.N;
+  a.M = d.M;
+  a.K = d.K;
+  a.nblk = L.nblk;
+  const int wpb = kDispatchThreads / 32;
+  int grid = (d.T + wpb - 1) / wpb;
+  const int cap = sm_count() * 8;
+  if (grid > cap) grid = cap;
+  dispatch_kernel<<<grid + 1, kDispatchThreads, 0, st>>>(a);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const double* sums_in,
+               int32_t* counts_ext, float* P, float* losses, cudaStream_t st) {
+  aux_kernel<<<1, 256, 0, st>>>(aux_ptrs(d, ws), sums_out, sums_in, counts_ext, P, losses);
+  return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------------------
+// Test aid: a bounded wait on a barrier that nothing arrives at.
+__global__ void selftest_wait_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    (void)mbar_wait_bounded(smem_u32(&bar), 0, limit_ns, &abort_flag, status);
+  }
+  __syncthreads();
+}
+
+int launch_selftest_wait(void* ws, unsigned long long limit_ns, cudaStream_t st) {
+  selftest_wait_kernel<<<1, 32, 0, st>>>(reinterpret_cast<uint32_t*>(ws), limit_ns);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace moe

@@ -1,0 +1,496 @@
+// moe_expert_ffn: the routed experts and the shared expert as two persistent
+// grouped GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Kilian et al., "Improving MoE Compute Efficiency by Composing Weight and Data
+// Sparsity" (review page, section 三 / 实现): after null slots are cut from the
+// expert-sorted list, the same grouped matmul runs on the real rows only; the
+// layer is y = E_shared(x) + sum g_i E_i(x) (核心公式). Each expert is SwiGLU:
+//   GEMM 1: h  = bf16(silu(A W_g^T) * (A W_u^T))   (gate and up in one tile)
+//   GEMM 2: ys = bf16(h W_d^T)
+// Group e < N covers rows [offsets[e], offsets[e+1]) of xs/h/ys, read on the
+// device (no host synchronisation on the data-dependent row counts); group N
+// is the shared expert over all T rows of x.
+//
+// Kernel: one CTA per SM, 6 warps. Warp 0 issues TMA loads (128B-swizzled
+// K-major tiles of 128 x 64 for A and BN x 64 for B) into a 4-stage mbarrier
+// ring; warp 1 owns TMEM (2 x BN fp32 columns, double-buffered accumulators)
+// and issues tcgen05.mma (M=128, N=BN, K=16) from a single thread, releasing
+// smem stages with tcgen05.commit; warps 2-5 drain TMEM with tcgen05.ld, apply
+// the epilogue, stage bf16 rows in shared memory and store them with
+// coalesced, row-masked 16-byte stores (a tile may run past its expert's last
+// row; those rows are computed but never stored). Tiles are handed out
+// round-robin (all tiles of a GEMM have the same cost). Every wait is bounded.
+#include "moe_internal.cuh"
+
+#include <cudaTypedefs.h>
+#include <mutex>
+
+namespace moe {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr int kStgRow = 64 * 2 + 16;  // staging row: 64 bf16 + 16 B pad
+
+struct GemmArgs {
+  const int32_t* offsets;  // [N+1]
+  int N, T;
+  int kb_r, kb_s;          // 64-wide k-blocks per tile: routed, shared
+  int nt_r, nt_s;          // n-tiles per group: routed, shared
+  int brows_r;             // B rows per routed expert
+  long long rows_cap;      // rows of the routed A/out buffers
+  uint16_t* out_r;
+  int ld_r;
+  uint16_t* out_s;
+  int ld_s;
+  uint32_t* status;
+  unsigned long long limit_ns;
+  int has_shared;
+};
+
+template <int BN>
+struct GemmSmem {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr size_t off_a = 0;
+  static constexpr size_t off_b = off_a + (size_t)kStages * A_BYTES;
+  static constexpr size_t off_stg = off_b + (size_t)kStages * B_BYTES;
+  static constexpr size_t off_bar = off_stg + (size_t)kBM * kStgRow;
+  static constexpr int n_bar = 2 * kStages + 5;  // full, empty, tfull[2], tempty[2], drain
+  static constexpr size_t off_misc = off_bar + 8 * n_bar;
+  static constexpr size_t off_tab = off_misc + 16;
+  static constexpr size_t end = off_tab + sizeof(int) * 3 * (kMaxN + 2);
+  static constexpr size_t bytes = end + 1024;  // slack for 1024-byte alignment
+};
+
+struct TileInfo {
+  int g, arow, mvalid, brow, nkb, col0;
+};
+
+template <int BN, bool SWIGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
+                    const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s,
+                    const GemmArgs a) {
+  using SM = GemmSmem<BN>;
+  constexpr int OUTC = SWIGLU ? BN / 2 : BN;  // output columns per tile
+  constexpr int NCHUNK = OUTC / 64;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN);
+  constexpr uint32_t TX_BYTES = SM::A_BYTES + SM::B_BYTES;
+
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base + SM::off_a;
+  unsigned char* sB = base + SM::off_b;
+  unsigned char* stg = base + SM::off_stg;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + SM::off_bar);
+  volatile int* misc = reinterpret_cast<volatile int*>(base + SM::off_misc);  // [0] tmem, [1] abort
+  int* s_tstart = reinterpret_cast<int*>(base + SM::off_tab);  // [N+2]
+  int* s_row0 = s_tstart + (kMaxN + 2);                       // [N+1]
+  int* s_m = s_row0 + (kMaxN + 2);                            // [N+1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + kStages + s); };
+  auto tfull_bar = [&](int s) { return smem_u32(bars + 2 * kStages + s); };
+  auto tempty_bar = [&](int s) { return smem_u32(bars + 2 * kStages + 2 + s); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * kStages + 4);
+  volatile int* abort_flag = misc + 1;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA_r);
+    prefetch_tmap(&tmB_r);
+    if (a.has_shared) {
+      prefetch_tmap(&tmA_s);
+      prefetch_tmap(&tmB_s);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(tfull_bar(s), 1);
+      mbar_init(tempty_bar(s), 128);
+    }
+    mbar_init(drain_bar, 1);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<int*>(misc)), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 2 && lane == 0) {
+    // Per-group tile table from the device-resident offsets.
+    int acc = 0;
+    int prev = 0;
+    bool bad = false;
+    for (int g = 0; g <= N; ++g) {
+      int m, row0, nt;
+      if (g < N) {
+        const int o0 = a.offsets[g], o1 = a.offsets[g + 1];
+        if (o0 != prev || o1 < o0 || (long long)o1 > a.rows_cap) bad = true;
+        prev = o1;
+        m = bad ? 0 : o1 - o0;
+        row0 = o0;
+        nt = a.nt_r;
+      } else {
+        m = a.has_shared ? a.T : 0;
+        row0 = 0;
+        nt = a.nt_s;
+      }
+      s_tstart[g] = acc;
+      s_row0[g] = row0;
+      s_m[g] = m;
+      acc += ((m + kBM - 1) / kBM) * nt;
+    }
+    s_tstart[N + 1] = acc;
+    if (bad) atomicOr(a.status, kStatusBounds);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = (uint32_t)misc[0];
+  const int total = s_tstart[N + 1];
+
+  auto decode = [&](int tile) {
+    TileInfo ti;
+    int lo = 0, hi = N;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    ti.g = lo;
+    const int nt = (lo < N) ? a.nt_r : a.nt_s;
+    const int local = tile - s_tstart[lo];
+    const int mt = local / nt;
+    const int ntile = local - mt * nt;
+    ti.arow = s_row0[lo] + mt * kBM;
+    ti.mvalid = min(kBM, s_m[lo] - mt * kBM);
+    ti.brow = (lo < N ? lo * a.brows_r : 0) + ntile * BN;
+    ti.nkb = (lo < N) ? a.kb_r : a.kb_s;
+    ti.col0 = ntile * OUTC;
+    return ti;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo ti = decode(tile);
+        const void* ta = (ti.g < N) ? (const void*)&tmA_r : (const void*)&tmA_s;
+        const void* tb = (ti.g < N) ? (const void*)&tmB_r : (const void*)&tmB_s;
+        bool ok = true;
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, a.limit_ns, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), TX_BYTES);
+          tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), ta, full_bar(stage), kb * kBK, ti.arow);
+          tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), tb, full_bar(stage), kb * kBK, ti.brow);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // let every issued copy land before the CTA can exit
+        for (int s = 0; s < kStages; ++s)
+          if (armed & (1u << s))
+            (void)mbar_wait_bounded(full_bar(s), (armed_par >> s) & 1u, a.limit_ns, nullptr, a.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------ MMA issuer (single thread)
+      int stage = 0;
+      uint32_t phase = 0;
+      int li = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++li) {
+        const TileInfo ti = decode(tile);
+        const int acc = li & 1;
+        const uint32_t ap = (uint32_t)(li >> 1) & 1u;
+        if (!mbar_wait_bounded(tempty_bar(acc), ap ^ 1u, a.limit_ns, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, a.limit_ns, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * SM::A_BYTES));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * SM::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // +32 bytes along K inside the 128-byte swizzle atom = +2 in the address field
+            tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
+                       (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+      }
+      // all MMAs issued by this thread have completed once the drain barrier fires
+      tc_commit(drain_bar);
+      (void)mbar_wait_bounded(drain_bar, 0, a.limit_ns, nullptr, a.status);
+    }
+  } else {
+    // ------------------------------ epilogue warpgroup (warps 2..5)
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;      // tile row held by this thread
+    const int etid = (warp - 2) * 32 + lane;
+    int li = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++li) {
+      const TileInfo ti = decode(tile);
+      const int acc = li & 1;
+      const uint32_t ap = (uint32_t)(li >> 1) & 1u;
+      if (!mbar_wait_bounded(tfull_bar(acc), ap, a.limit_ns, abort_flag, a.status)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      uint16_t* out = (ti.g < N) ? a.out_r : a.out_s;
+      const int ld = (ti.g < N) ? a.ld_r : a.ld_s;
+#pragma unroll 1
+      for (int c = 0; c < NCHUNK; ++c) {
+#pragma unroll
+        for (int g16 = 0; g16 < 4; ++g16) {
+          uint32_t packed[8];
+          if constexpr (SWIGLU) {
+            uint32_t gr[16], ur[16];
+            tmem_ld16(tb + (uint32_t)(c * 128 + g16 * 16), gr);
+            tmem_ld16(tb + (uint32_t)(c * 128 + 64 + g16 * 16), ur);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float g0 = __uint_as_float(gr[2 * j]), g1 = __uint_as_float(gr[2 * j + 1]);
+              const float u0 = __uint_as_float(ur[2 * j]), u1 = __uint_as_float(ur[2 * j + 1]);
+              const float h0 = __fdividef(g0, 1.f + __expf(-g0)) * u0;
+              const float h1 = __fdividef(g1, 1.f + __expf(-g1)) * u1;
+              packed[j] = pack_bf16x2(h0, h1);
+            }
+          } else {
+            uint32_t r[16];
+            tmem_ld16(tb + (uint32_t)(c * 64 + g16 * 16), r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              packed[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+          }
+          uint4* dst = reinterpret_cast<uint4*>(stg + row * kStgRow + g16 * 32);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        }
+        if (c == NCHUNK - 1) {
+          tc_fence_before();
+          mbar_arrive(tempty_bar(acc));  // TMEM buffer free for the next-but-one tile
+        }
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int idx = it * 128 + etid;
+          const int r = idx >> 3, ch = idx & 7;
+          if (r < ti.mvalid) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * kStgRow + ch * 16);
+            *reinterpret_cast<uint4*>(out + (size_t)(ti.arow + r) * ld + ti.col0 + c * 64 + ch * 8) = v;
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Gate/up packing: 64-row panels, gate panel then the matching up panel.
+__global__ void pack_gate_up_kernel(const uint16_t* __restrict__ wg, const uint16_t* __restrict__ wu,
+                                    uint16_t* __restrict__ out, int groups, int F, int d) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)groups * 2 * F;
+  const int nch = d >> 3;
+  for (long long pr = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pr < rows;
+       pr += (long long)gridDim.x * (blockDim.x >> 5)) {
+    const long long e = pr / (2 * F);
+    const int r = (int)(pr - e * 2 * F);
+    const int pair = r >> 7, within = r & 127;
+    const uint16_t* src = (within < 64 ? wg : wu) + ((size_t)e * F + pair * 64 + (within & 63)) * d;
+    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)pr * d);
+    for (int c = lane; c < nch; c += 32) dst[c] = __ldg(reinterpret_cast<const uint4*>(src) + c);
+  }
+}
+
+int launch_pack_gate_up(const moe_dims_t& d, const uint16_t* w_gate, const uint16_t* w_up,
+                        const uint16_t* ws_gate, const uint16_t* ws_up, uint16_t* gate_up,
+                        uint16_t* sgate_up, cudaStream_t st) {
+  const int grid = sm_count() * 8;
+  if (gate_up) {
+    pack_gate_up_kernel<<<grid, 256, 0, st>>>(w_gate, w_up, gate_up, d.N, d.F, d.d);
+    int r = cuda_status(cudaGetLastError());
+    if (r != MOE_OK) return r;
+  }
+  if (sgate_up) {
+    pack_gate_up_kernel<<<grid, 256, 0, st>>>(ws_gate, ws_up, sgate_up, 1, d.F_shared, d.d);
+    int r = cuda_status(cudaGetLastError());
+    if (r != MOE_OK) return r;
+  }
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side: tensor maps and launches.
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous), box = box_rows x 64 cols, 128B swizzle.
+static bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWIGLU>
+static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUtensorMap& as_,
+                       const CUtensorMap& bs, const GemmArgs& a, long long max_tiles, cudaStream_t st) {
+  using SM = GemmSmem<BN>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, SWIGLU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::bytes);
+    if (e != cudaSuccess) return cuda_status(e);
+    attr_set[dev] = true;
+  }
+  long long grid = sm_count();
+  if (max_tiles < grid) grid = max_tiles;
+  if (grid < 1) grid = 1;
+  grouped_gemm_kernel<BN, SWIGLU><<<(int)grid, kGemmThreads, SM::bytes, st>>>(ar, br, as_, bs, a);
+  return cuda_status(cudaGetLastError());
+}
+
+struct FfnPlan {
+  int BN1, BN2;
+  long long max1, max2;
+  GemmArgs g1, g2;
+};
+
+static FfnPlan plan_ffn(const moe_dims_t& d, const int32_t* offsets, void* ws) {
+  const WsLayout L = ws_layout(d);
+  FfnPlan p{};
+  const long long rcap = (long long)d.T * d.K;
+  p.BN1 = (d.F % 128 == 0 && d.F_shared % 128 == 0) ? 256 : 128;
+  p.BN2 = (d.d % 256 == 0) ? 256 : 128;
+  const long long mtiles_r = rcap / kBM + d.N;  // sum_e ceil(m_e/128) <= R/128 + N
+  const long long mtiles_s = (d.T + kBM - 1) / kBM;
+  GemmArgs& g1 = p.g1;
+  g1.offsets = offsets;
+  g1.N = d.N;
+  g1.T = d.T;
+  g1.kb_r = d.d / kBK;
+  g1.kb_s = d.d / kBK;
+  g1.nt_r = 2 * d.F / p.BN1;
+  g1.nt_s = 2 * d.F_shared / p.BN1;
+  g1.brows_r = 2 * d.F;
+  g1.rows_cap = rcap;
+  g1.ld_r = d.F;
+  g1.ld_s = d.F_shared;
+  g1.status = ws_ptr<uint32_t>(ws, L.hdr);
+  g1.limit_ns = kWaitLimitNs;
+  g1.has_shared = 1;
+  p.max1 = mtiles_r * g1.nt_r + mtiles_s * g1.nt_s;
+  GemmArgs& g2 = p.g2;
+  g2 = g1;
+  g2.kb_r = d.F / kBK;
+  g2.kb_s = d.F_shared / kBK;
+  g2.nt_r = d.d / p.BN2;
+  g2.nt_s = d.d / p.BN2;
+  g2.brows_r = d.d;
+  g2.ld_r = d.d;
+  g2.ld_s = d.d;
+  p.max2 = mtiles_r * g2.nt_r + mtiles_s * g2.nt_s;
+  return p;
+}
+
+int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                   const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
+                   void* ws, cudaStream_t st) {
+  FfnPlan p = plan_ffn(d, offsets, ws);
+  const long long rcap = (long long)d.T * d.K;
+  CUtensorMap ar, br, as_, bs;
+  if (!(make_tmap(&ar, xs, rcap, d.d, kBM) && make_tmap(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, p.BN1) &&
+        make_tmap(&as_, x, d.T, d.d, kBM) && make_tmap(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, p.BN1)))
+    return MOE_ERR_CUDA;
+  p.g1.out_r = h;
+  p.g1.out_s = h_shared;
+  return (p.BN1 == 256) ? launch_gemm<256, true>(ar, br, as_, bs, p.g1, p.max1, st)
+                        : launch_gemm<128, true>(ar, br, as_, bs, p.g1, p.max1, st);
+}
+
+int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
+                const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys, uint16_t* shared_out, void* ws,
+                cudaStream_t st) {
+  FfnPlan p = plan_ffn(d, offsets, ws);
+  const long long rcap = (long long)d.T * d.K;
+  CUtensorMap ar, br, as_, bs;
+  if (!(make_tmap(&ar, h, rcap, d.F, kBM) && make_tmap(&br, w_down, (uint64_t)d.N * d.d, d.F, p.BN2) &&
+        make_tmap(&as_, h_shared, d.T, d.F_shared, kBM) && make_tmap(&bs, sdown, d.d, d.F_shared, p.BN2)))
+    return MOE_ERR_CUDA;
+  p.g2.out_r = ys;
+  p.g2.out_s = shared_out;
+  return (p.BN2 == 256) ? launch_gemm<256, false>(ar, br, as_, bs, p.g2, p.max2, st)
+                        : launch_gemm<128, false>(ar, br, as_, bs, p.g2, p.max2, st);
+}
+
+int launch_expert_ffn(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                      const uint16_t* gate_up, const uint16_t* w_down, const uint16_t* sgate_up,
+                      const uint16_t* sdown, uint16_t* h, uint16_t* h_shared, uint16_t* ys,
+                      uint16_t* shared_out, void* ws, cudaStream_t st) {
+  const int r = launch_gate_up(d, xs, x, offsets, gate_up, sgate_up, h, h_shared, ws, st);
+  if (r != MOE_OK) return r;
+  return launch_down(d, offsets, h, h_shared, w_down, sdown, ys, shared_out, ws, st);
+}
+
+}  // namespace moe

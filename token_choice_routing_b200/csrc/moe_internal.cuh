@@ -1,0 +1,272 @@
+// Internal declarations shared by the CUDA translation units of libmoe_null.
+// Device helpers are thin inline-PTX wrappers for sm_100a: mbarriers, TMA
+// tensor loads, tcgen05 (TMEM allocation, MMA, commit, loads) and fences.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/moe_null.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------------------------
+// Tiling constants of the route kernel (fp32 CUDA-core router GEMM + routing).
+constexpr int kRouteTokens = 64;    // tokens per route CTA
+constexpr int kRouteBK = 32;        // d-slice per pipeline stage
+constexpr int kRouteThreads = 128;  // 16 token groups x 8 logit groups
+constexpr int kMaxN = 64;
+constexpr int kMaxK = 16;
+
+// Status bits recorded on the device (the host maps them to moe_status_t).
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBounds = 2u;
+
+// Default limit of every device-side wait, in ns of %globaltimer.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// Workspace layout, computed identically on the host for every entry point.
+struct WsLayout {
+  int nblk;          // route CTAs = ceil(T / kRouteTokens)
+  size_t hdr;        // uint32 status, uint32 done-counter (256 B)
+  size_t counts_blk; // int32 [N][nblk]
+  size_t bases;      // int32 [N][nblk]
+  size_t ppart;      // float [nblk][N+1]
+  size_t lsq;        // float [nblk]
+  size_t hist;       // int32 [nblk][K+1]
+  size_t lrank;      // int32 [T][K]
+  size_t counts;     // int32 [N]
+  size_t offsets;    // int32 [N+1]
+  size_t sums;       // double [aux sums count]
+  size_t total;
+};
+
+constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline size_t aux_sums_count(const moe_dims_t& d) {
+  return (size_t)d.N + (size_t)(d.K + 1) + (size_t)(d.N + 1) + 2;
+}
+
+inline WsLayout ws_layout(const moe_dims_t& d) {
+  WsLayout L{};
+  L.nblk = (d.T + kRouteTokens - 1) / kRouteTokens;
+  size_t o = 0;
+  L.hdr = o; o += 256;
+  L.counts_blk = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N * L.nblk, 256);
+  L.bases = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N * L.nblk, 256);
+  L.ppart = o; o = align_up(o + sizeof(float) * (size_t)(d.N + 1) * L.nblk, 256);
+  L.lsq = o; o = align_up(o + sizeof(float) * (size_t)L.nblk, 256);
+  L.hist = o; o = align_up(o + sizeof(int32_t) * (size_t)(d.K + 1) * L.nblk, 256);
+  L.lrank = o; o = align_up(o + sizeof(int32_t) * (size_t)d.T * d.K, 256);
+  L.counts = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N, 256);
+  L.offsets = o; o = align_up(o + sizeof(int32_t) * (size_t)(d.N + 1), 256);
+  L.sums = o; o = align_up(o + sizeof(double) * aux_sums_count(d), 256);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+inline T* ws_ptr(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+template <typename T>
+inline const T* ws_ptr(const void* ws, size_t off) {
+  return reinterpret_cast<const T*>(static_cast<const char*>(ws) + off);
+}
+
+// Host helpers implemented in api.cu.
+int check_dims(const moe_dims_t* d);
+int sm_count();
+int cuda_status(cudaError_t e);
+
+// Launchers (each returns a moe_status_t after enqueuing).
+int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router,
+                 const float* bias, const float* tok_null_bias, float* logits_out,
+                 int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* ws,
+                 cudaStream_t st);
+int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_idx, void* ws,
+                    int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* slot_row,
+                    uint16_t* xs, int32_t* counts_ext, float* P, float* losses,
+                    cudaStream_t st);
+int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const double* sums_in,
+               int32_t* counts_ext, float* P, float* losses, cudaStream_t st);
+int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
+                   const float* topk_gate, const int32_t* slot_row, uint16_t* y,
+                   cudaStream_t st);
+int launch_expert_ffn(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x,
+                      const int32_t* offsets, const uint16_t* gate_up, const uint16_t* w_down,
+                      const uint16_t* sgate_up, const uint16_t* sdown, uint16_t* h,
+                      uint16_t* h_shared, uint16_t* ys, uint16_t* shared_out, void* ws,
+                      cudaStream_t st);
+int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                   const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
+                   void* ws, cudaStream_t st);
+int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
+                const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys, uint16_t* shared_out, void* ws,
+                cudaStream_t st);
+int launch_pack_gate_up(const moe_dims_t& d, const uint16_t* w_gate, const uint16_t* w_up,
+                        const uint16_t* ws_gate, const uint16_t* ws_up, uint16_t* gate_up,
+                        uint16_t* sgate_up, cudaStream_t st);
+int launch_selftest_wait(void* ws, unsigned long long limit_ns, cudaStream_t st);
+
+// ------------------------------------------------------------------------------------
+// Device helpers.
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with parity `parity` of an mbarrier. Returns
+// false (and records a timeout in *status) if `limit_ns` passed, or if
+// *abort (CTA shared flag, may be null) became non-zero meanwhile.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns,
+                                                  volatile int* abort, uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++spins & 63u) == 0u) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (status) atomicOr(status, kStatusTimeout);
+        if (abort) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// TMEM allocation: warp-wide. The allocated base address is written to smem.
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 inputs, fp32 accumulate).
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on an mbarrier when all prior tcgen05 async ops of this thread finish.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// 32 lanes x 32 bit, 16 consecutive columns: thread i gets TMEM lane (base+i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05) for a K-major tile whose rows are
+// 128 bytes (64 bf16) stored with the 128-byte swizzle, 8-row groups 1024 B
+// apart: start address, LBO = 16 B (unused for this layout), SBO = 1024 B,
+// descriptor version 1, layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)64 << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: D fp32, A bf16, B bf16, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace moe

@@ -1,0 +1,428 @@
+// moe_route: router GEMM (fp32, CUDA cores) fused with the expanded-pool
+// softmax statistics, top-K over the pool, renormalised gates and the
+// per-block statistics that dispatch and the aux losses need.
+//
+// Method (Kilian et al., "Improving MoE Compute Efficiency by Composing Weight
+// and Data Sparsity", review page, section 三 技术架构):
+//  * Null Expert 机制: N real logits plus one null logit; the null logit is
+//    replicated M times before top-K, so the pool is [s_0..s_{N-1}, s_N x M].
+//    The pool is never materialised here: a copy is a (value, multiplicity).
+//  * 阈值解释: the token keeps the real experts whose logit beats the null
+//    logit; so top-K over the pool is K rounds of "best remaining real vs the
+//    null logit", the real winning ties (lower index), copies taken in index
+//    order N, N+1, ... while any remain.
+//  * renormalisation over the selected reals: gates = softmax over their
+//    logits; null slots weigh 0.
+//  * Z-Loss / 负载均衡损失: lse_t over the N+M pool and p_{t,i} are reduced per
+//    block here (fp32 over 64 tokens) and across blocks in fp64 later.
+//
+// Layout: one CTA = 64 tokens x all N+1 logits, 128 threads in 16 token groups
+// x 8 logit groups; a thread owns 4 tokens (stride 16) x N/8 reals (stride 8)
+// and one eighth of the d-range of the null logit. x (bf16) is widened to fp32
+// once when staged in shared memory; W_r slices arrive by cp.async.
+#include "moe_internal.cuh"
+
+#include <cstdio>
+
+namespace moe {
+
+struct RouteArgs {
+  const uint16_t* x;
+  const float* w;     // [N+1, d]
+  const float* bias;  // [N+1] or null
+  const float* tnb;   // [T] or null
+  float* logits;      // [T, N+1] or null
+  int32_t* topk_idx;
+  float* topk_gate;
+  int32_t* n_real;
+  // workspace
+  uint32_t* hdr;  // [0] status, [1] done counter
+  int32_t* counts_blk;
+  int32_t* bases;
+  float* ppart;
+  float* lsq;
+  int32_t* hist;
+  int32_t* lrank;
+  int32_t* counts;
+  int32_t* offsets;
+  int T, d, N, M, K, nblk;
+};
+
+constexpr int kXS = kRouteBK + 4;  // padded fp32 row stride of staged tiles
+
+template <int NPAD>
+struct RouteSmem {
+  static constexpr int LS = NPAD + 1;  // odd stride: conflict-free per-token rows
+  static constexpr size_t main_bytes =
+      sizeof(float) * (2 * kRouteTokens * kXS + 2 * (NPAD + 1) * kXS);
+  static constexpr size_t off_s = 0;
+  static constexpr size_t off_p = off_s + sizeof(float) * kRouteTokens * LS;
+  static constexpr size_t off_npart = off_p + sizeof(float) * kRouteTokens * LS;
+  static constexpr size_t off_lse2 = off_npart + sizeof(float) * 8 * kRouteTokens;
+  static constexpr size_t off_nul = off_lse2 + sizeof(float) * kRouteTokens;
+  static constexpr size_t off_mask = align_up(off_nul + sizeof(int) * kRouteTokens, 16);
+  static constexpr size_t off_tk = off_mask + sizeof(unsigned long long) * kRouteTokens;
+  static constexpr size_t off_rtab = off_tk + sizeof(int) * kRouteTokens * kMaxK;
+  static constexpr size_t epi_bytes = off_rtab + (size_t)kRouteTokens * NPAD;
+  static constexpr size_t bytes = main_bytes > epi_bytes ? main_bytes : epi_bytes;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int RPT>
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
+  constexpr int NPAD = 8 * RPT;
+  using SM = RouteSmem<NPAD>;
+  constexpr int LS = SM::LS;
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* xst = reinterpret_cast<float*>(smem);              // [2][64][kXS]
+  float* wst = xst + 2 * kRouteTokens * kXS;                // [2][NPAD+1][kXS]
+  __shared__ int s_last;
+  __shared__ int s_tot[kMaxN];
+  __shared__ int s_off[kMaxN + 1];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tg = (warp & 1) * 8 + (lane & 7);   // token group 0..15
+  const int lg = (warp >> 1) * 4 + (lane >> 3); // logit group 0..7
+  const int b = blockIdx.x;
+  const int T = a.T, d = a.d, N = a.N, M = a.M, K = a.K;
+  const int tok0 = b * kRouteTokens;
+  const int nvalid = min(kRouteTokens, T - tok0);
+  const int nkt = d / kRouteBK;
+
+  float acc[4][RPT];
+  float accn[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    accn[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) acc[i][j] = 0.f;
+  }
+
+  uint4 xr[2];
+  auto load_x = [&](int kt) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int c = tid + kRouteThreads * q;
+      const int row = c >> 2, col8 = (c & 3) * 8;
+      const int tok = tok0 + row;
+      if (tok < T) {
+        xr[q] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok * d + (size_t)kt * kRouteBK + col8));
+      } else {
+        xr[q] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  };
+  auto store_x = [&](int buf) {
+    float* xb = xst + buf * kRouteTokens * kXS;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int c = tid + kRouteThreads * q;
+      const int row = c >> 2, col8 = (c & 3) * 8;
+      float4* dst = reinterpret_cast<float4*>(xb + row * kXS + col8);
+      dst[0] = make_float4(bf16lo(xr[q].x), bf16hi(xr[q].x), bf16lo(xr[q].y), bf16hi(xr[q].y));
+      dst[1] = make_float4(bf16lo(xr[q].z), bf16hi(xr[q].z), bf16lo(xr[q].w), bf16hi(xr[q].w));
+    }
+  };
+  auto load_w = [&](int kt, int buf) {
+    float* wb = wst + buf * (NPAD + 1) * kXS;
+    for (int c = tid; c < (NPAD + 1) * 8; c += kRouteThreads) {
+      const int r = c >> 3, col4 = (c & 7) * 4;
+      const int src_row = (r < N) ? r : (r == NPAD ? N : -1);
+      const float* src = a.w + (size_t)(src_row < 0 ? 0 : src_row) * d + (size_t)kt * kRouteBK + col4;
+      cp_async16(smem_u32(wb + r * kXS + col4), src, src_row < 0 ? 0 : 16);
+    }
+    cp_async_commit();
+  };
+
+  load_x(0);
+  load_w(0, 0);
+  for (int kt = 0; kt < nkt; ++kt) {
+    const int buf = kt & 1;
+    store_x(buf);
+    cp_async_wait_all();
+    __syncthreads();
+    if (kt + 1 < nkt) {
+      load_x(kt + 1);
+      load_w(kt + 1, buf ^ 1);
+    }
+    const float* xb = xst + buf * kRouteTokens * kXS;
+    const float* wb = wst + buf * (NPAD + 1) * kXS;
+#pragma unroll
+    for (int kk = 0; kk < kRouteBK / 4; ++kk) {
+      float4 xv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(xb + (tg + 16 * i) * kXS + kk * 4);
+#pragma unroll
+      for (int jj = 0; jj < RPT; ++jj) {
+        const float4 wv = *reinterpret_cast<const float4*>(wb + (lg + 8 * jj) * kXS + kk * 4);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float s = acc[i][jj];
+          s = fmaf(xv[i].x, wv.x, s);
+          s = fmaf(xv[i].y, wv.y, s);
+          s = fmaf(xv[i].z, wv.z, s);
+          s = fmaf(xv[i].w, wv.w, s);
+          acc[i][jj] = s;
+        }
+      }
+    }
+    {  // the null logit: this logit group's 4-wide slice of the d-tile
+      const float4 wn = *reinterpret_cast<const float4*>(wb + NPAD * kXS + lg * 4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 xv = *reinterpret_cast<const float4*>(xb + (tg + 16 * i) * kXS + lg * 4);
+        float s = accn[i];
+        s = fmaf(xv.x, wn.x, s);
+        s = fmaf(xv.y, wn.y, s);
+        s = fmaf(xv.z, wn.z, s);
+        s = fmaf(xv.w, wn.w, s);
+        accn[i] = s;
+      }
+    }
+  }
+  __syncthreads();  // main-loop buffers are reused below
+
+  float* s_l = reinterpret_cast<float*>(smem + SM::off_s);
+  float* p_s = reinterpret_cast<float*>(smem + SM::off_p);
+  float* npart = reinterpret_cast<float*>(smem + SM::off_npart);
+  float* lse2 = reinterpret_cast<float*>(smem + SM::off_lse2);
+  int* nul = reinterpret_cast<int*>(smem + SM::off_nul);
+  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem + SM::off_mask);
+  int* tk = reinterpret_cast<int*>(smem + SM::off_tk);
+  unsigned char* rtab = smem + SM::off_rtab;
+
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = tg + 16 * i;
+#pragma unroll
+    for (int jj = 0; jj < RPT; ++jj) {
+      const int j = lg + 8 * jj;
+      if (j < N) s_l[t * LS + j] = acc[i][jj] + (a.bias ? __ldg(a.bias + j) : 0.f);
+    }
+    npart[lg * kRouteTokens + t] = accn[i];
+  }
+  __syncthreads();
+
+  if (tid < nvalid) {
+    const int t = tid;
+    const int tok = tok0 + t;
+    float* st = s_l + t * LS;
+    float sn = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sn += npart[q * kRouteTokens + t];
+    if (a.bias) sn += __ldg(a.bias + N);
+    if (a.tnb) sn += __ldg(a.tnb + tok);
+    st[NPAD] = sn;
+
+    // softmax statistics over the pool (M copies of the null logit)
+    float m = -INFINITY;
+    for (int i = 0; i < N; ++i) m = fmaxf(m, st[i]);
+    if (M > 0) m = fmaxf(m, sn);
+    float Z = 0.f;
+    for (int i = 0; i < N; ++i) Z += expf(st[i] - m);
+    if (M > 0) Z += (float)M * expf(sn - m);
+    const float lse = m + logf(Z);
+    float* pt = p_s + t * LS;
+    for (int i = 0; i < N; ++i) pt[i] = expf(st[i] - lse);
+    pt[NPAD] = (M > 0) ? expf(sn - lse) : 0.f;
+    lse2[t] = lse * lse;
+
+    // top-K over the pool, in rank order
+    unsigned long long sel = 0ull;
+    int used = 0, r = 0;
+    for (int k = 0; k < K; ++k) {
+      float bv = -INFINITY;
+      int bi = -1;
+      for (int i = 0; i < N; ++i) {
+        if (!((sel >> i) & 1ull)) {
+          const float v = st[i];
+          if (bi < 0 || v > bv) { bv = v; bi = i; }
+        }
+      }
+      const bool take_null = (used < M) && (bi < 0 || bv < sn);
+      int id;
+      if (take_null) {
+        id = N + used;
+        ++used;
+      } else {
+        id = bi;
+        sel |= 1ull << bi;
+        ++r;
+      }
+      tk[t * kMaxK + k] = id;
+    }
+    // gates: softmax over the selected real logits (rank order => first real is the max)
+    float smax = 0.f, gsum = 0.f;
+    bool first = true;
+    for (int k = 0; k < K; ++k) {
+      const int id = tk[t * kMaxK + k];
+      if (id < N) {
+        if (first) { smax = st[id]; first = false; }
+        gsum += expf(st[id] - smax);
+      }
+    }
+    for (int k = 0; k < K; ++k) {
+      const int id = tk[t * kMaxK + k];
+      const float g = (id < N) ? expf(st[id] - smax) / gsum : 0.f;
+      a.topk_idx[(size_t)tok * K + k] = id;
+      a.topk_gate[(size_t)tok * K + k] = g;
+    }
+    a.n_real[tok] = r;
+    nul[t] = K - r;
+    mask[t] = sel;
+    if (a.logits) {
+      float* lo = a.logits + (size_t)tok * (N + 1);
+      for (int i = 0; i < N; ++i) lo[i] = st[i];
+      lo[N] = sn;
+    }
+  }
+  __syncthreads();
+
+  // Per-block ranks and counts (ascending token order inside an expert), P sums.
+  if (tid < N) {
+    const int e = tid;
+    int cnt = 0;
+    for (int t = 0; t < nvalid; ++t) {
+      if ((mask[t] >> e) & 1ull) rtab[t * NPAD + e] = (unsigned char)(cnt++);
+    }
+    a.counts_blk[(size_t)e * a.nblk + b] = cnt;
+  }
+  if (tid <= N) {
+    const int col = (tid < N) ? tid : NPAD;
+    float s = 0.f;
+    for (int t = 0; t < nvalid; ++t) s += p_s[t * LS + col];
+    a.ppart[(size_t)b * (N + 1) + tid] = s;
+  }
+  __syncthreads();
+  if (tid <= K) {
+    int cnt = 0;
+    for (int t = 0; t < nvalid; ++t) cnt += (nul[t] == tid);
+    a.hist[(size_t)b * (K + 1) + tid] = cnt;
+  }
+  if (tid == 32) {
+    float s = 0.f;
+    for (int t = 0; t < nvalid; ++t) s += lse2[t];
+    a.lsq[b] = s;
+  }
+  if (tid < nvalid) {
+    const int tok = tok0 + tid;
+    for (int k = 0; k < K; ++k) {
+      const int id = tk[tid * kMaxK + k];
+      a.lrank[(size_t)tok * K + k] = (id < N) ? (int)rtab[tid * NPAD + id] : -1;
+    }
+  }
+
+  // The last block to finish turns the per-block counts into offsets and
+  // per-block bases (exclusive scans; integer, so exact and order-free).
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned prev = atomicAdd(&a.hdr[1], 1u);
+    s_last = (prev == (unsigned)(a.nblk - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int nblk = a.nblk;
+  for (int e = warp; e < N; e += kRouteThreads / 32) {
+    int s = 0;
+    for (int bb = lane; bb < nblk; bb += 32) s += __ldcg(a.counts_blk + (size_t)e * nblk + bb);
+    s = warp_sum_i(s);
+    if (lane == 0) s_tot[e] = s;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < N; ++e) {
+      s_off[e] = run;
+      run += s_tot[e];
+    }
+    s_off[N] = run;
+  }
+  __syncthreads();
+  if (tid <= N) a.offsets[tid] = s_off[tid];
+  if (tid < N) a.counts[tid] = s_tot[tid];
+  for (int e = warp; e < N; e += kRouteThreads / 32) {
+    int run = s_off[e];
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+      const int bb = b0 + lane;
+      const int v = (bb < nblk) ? __ldcg(a.counts_blk + (size_t)e * nblk + bb) : 0;
+      int inc = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+      }
+      if (bb < nblk) a.bases[(size_t)e * nblk + bb] = run + inc - v;
+      run += __shfl_sync(0xffffffffu, inc, 31);
+    }
+  }
+  if (tid == 0) a.hdr[1] = 0u;
+}
+
+template <int RPT>
+static int launch_route_t(const RouteArgs& a, cudaStream_t st) {
+  using SM = RouteSmem<8 * RPT>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SM::bytes);
+    if (e != cudaSuccess) return cuda_status(e);
+    attr_set[dev] = true;
+  }
+  route_kernel<RPT><<<a.nblk, kRouteThreads, SM::bytes, st>>>(a);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, const float* bias,
+                 const float* tok_null_bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
+                 int32_t* n_real, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(d);
+  RouteArgs a{};
+  a.x = x;
+  a.w = w_router;
+  a.bias = bias;
+  a.tnb = tok_null_bias;
+  a.logits = logits_out;
+  a.topk_idx = topk_idx;
+  a.topk_gate = topk_gate;
+  a.n_real = n_real;
+  a.hdr = ws_ptr<uint32_t>(ws, L.hdr);
+  a.counts_blk = ws_ptr<int32_t>(ws, L.counts_blk);
+  a.bases = ws_ptr<int32_t>(ws, L.bases);
+  a.ppart = ws_ptr<float>(ws, L.ppart);
+  a.lsq = ws_ptr<float>(ws, L.lsq);
+  a.hist = ws_ptr<int32_t>(ws, L.hist);
+  a.lrank = ws_ptr<int32_t>(ws, L.lrank);
+  a.counts = ws_ptr<int32_t>(ws, L.counts);
+  a.offsets = ws_ptr<int32_t>(ws, L.offsets);
+  a.T = d.T;
+  a.d = d.d;
+  a.N = d.N;
+  a.M = d.M;
+  a.K = d.K;
+  a.nblk = L.nblk;
+  // status and the done counter start at zero for every layer call
+  cudaError_t e = cudaMemsetAsync(a.hdr, 0, 2 * sizeof(uint32_t), st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (d.N <= 8) return launch_route_t<1>(a, st);
+  if (d.N <= 16) return launch_route_t<2>(a, st);
+  if (d.N <= 32) return launch_route_t<4>(a, st);
+  return launch_route_t<8>(a, st);
+}
+
+}  // namespace moe

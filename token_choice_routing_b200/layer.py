@@ -1,0 +1,95 @@
+"""A null-expert MoE layer object over the C ABI.
+
+Holds the device weights (gate/up packed once by the library), allocates the
+caller-owned buffers and workspace with torch, and runs the forward through
+``moe_forward``. PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+def bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
+    """uint16 bf16 bit array (host) -> torch.bfloat16 tensor on ``device``."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device)
+
+
+class MoENullLayer:
+    def __init__(self, d: int, N: int, M: int, K: int, F: int, F_shared: int, *,
+                 w_router: torch.Tensor, router_bias: Optional[torch.Tensor],
+                 w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                 ws_gate: torch.Tensor, ws_up: torch.Tensor, ws_down: torch.Tensor):
+        self.d, self.N, self.M, self.K, self.F, self.F_shared = d, N, M, K, F, F_shared
+        dev = w_router.device
+        self.device = dev
+        self.w_router = w_router.contiguous()
+        self.router_bias = None if router_bias is None else router_bias.contiguous()
+        self.w_down = w_down.contiguous()
+        self.shared_down = ws_down.contiguous()
+        dm = self.dims(1)
+        code = B.check_dims(dm)
+        if code != B.OK:
+            raise B.MoEError("moe_check_dims", code)
+        self.gate_up = torch.empty(B.packed_gate_up_elems(dm, False), dtype=torch.bfloat16, device=dev)
+        self.shared_gate_up = torch.empty(B.packed_gate_up_elems(dm, True), dtype=torch.bfloat16, device=dev)
+        B.pack_gate_up(dm, w_gate.contiguous(), w_up.contiguous(), ws_gate.contiguous(), ws_up.contiguous(),
+                       self.gate_up, self.shared_gate_up)
+        self._weights = B.Weights(self.w_router.data_ptr(),
+                                  None if self.router_bias is None else self.router_bias.data_ptr(),
+                                  self.gate_up.data_ptr(), self.w_down.data_ptr(),
+                                  self.shared_gate_up.data_ptr(), self.shared_down.data_ptr())
+
+    @classmethod
+    def from_inputs(cls, inp, device="cuda") -> "MoENullLayer":
+        c = inp.cfg
+        f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        return cls(c.d, c.N, c.M, c.K, c.F, c.F_shared,
+                   w_router=f32(inp.w_router), router_bias=f32(inp.bias),
+                   w_gate=bf16_tensor(inp.w_gate, device), w_up=bf16_tensor(inp.w_up, device),
+                   w_down=bf16_tensor(inp.w_down, device), ws_gate=bf16_tensor(inp.ws_gate, device),
+                   ws_up=bf16_tensor(inp.ws_up, device), ws_down=bf16_tensor(inp.ws_down, device))
+
+    def dims(self, T: int) -> B.Dims:
+        return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared)
+
+    def alloc(self, T: int, logits: bool = True) -> Dict[str, torch.Tensor]:
+        """Caller-owned buffers for a T-token call (R_cap = T*K rows)."""
+        dev, d, N, M, K, F, Fs = self.device, self.d, self.N, self.M, self.K, self.F, self.F_shared
+        R = T * K
+        i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+        out = dict(
+            logits=torch.empty((T, N + 1), dtype=f32, device=dev) if logits else None,
+            topk_idx=torch.empty((T, K), dtype=i32, device=dev),
+            topk_gate=torch.empty((T, K), dtype=f32, device=dev),
+            n_real=torch.empty((T,), dtype=i32, device=dev),
+            counts=torch.empty((N,), dtype=i32, device=dev),
+            offsets=torch.empty((N + 1,), dtype=i32, device=dev),
+            perm_tok=torch.empty((max(R, 1),), dtype=i32, device=dev),
+            slot_row=torch.empty((T, K), dtype=i32, device=dev),
+            xs=torch.empty((max(R, 1), d), dtype=bf, device=dev),
+            h=torch.empty((max(R, 1), F), dtype=bf, device=dev),
+            h_shared=torch.empty((max(T, 1), Fs), dtype=bf, device=dev),
+            ys=torch.empty((max(R, 1), d), dtype=bf, device=dev),
+            shared_out=torch.empty((max(T, 1), d), dtype=bf, device=dev),
+            y=torch.empty((max(T, 1), d), dtype=bf, device=dev),
+            counts_ext=torch.empty((N + M,), dtype=i32, device=dev),
+            P=torch.empty((N + M,), dtype=f32, device=dev),
+            losses=torch.empty((2,), dtype=f32, device=dev),
+        )
+        out["workspace"] = torch.empty((max(B.workspace_bytes(self.dims(T)), 256),), dtype=torch.uint8, device=dev)
+        return out
+
+    def forward(self, x: torch.Tensor, tok_null_bias: Optional[torch.Tensor] = None,
+                out: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
+        T = x.shape[0]
+        if out is None:
+            out = self.alloc(T)
+        o = B.Outputs(*[None if out.get(n) is None else out[n].data_ptr() for n in B.OUTPUT_FIELDS])
+        B.forward(self.dims(T), self._weights, x, tok_null_bias, o, out["workspace"], stream)
+        return out
