@@ -50,58 +50,62 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """Samples the GPU's SM clock and clock-event (throttle) reasons through NVML
+    from a background thread while the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device_index: int, period_s: float = 0.002):
+        self.idx = torch_device_index
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.idx).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+            self.nv = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self._ok = True
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except Exception:
-            self.proc = None
+            time.sleep(0.05)
+        except Exception as e:  # NVML missing: the line says so
+            self.err = repr(e)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self._stop.set()
+        if self._ok:
+            self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
 # ----------------------------------------------------------------------------------------
@@ -190,7 +194,7 @@ def workload_config(cfg, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="qwen3_0p6b")
@@ -207,6 +211,7 @@ def main():
 
     from token_choice_routing_b200 import binding as B
     from token_choice_routing_b200 import inputs as I
+    from token_choice_routing_b200.dist import dp_forward
     from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
 
     rank = int(os.environ.get("RANK", "0"))
@@ -233,20 +238,11 @@ def main():
     def step():
         if world == 1:
             layer.forward(x, tnb, out)
-            return
-        # data parallel: local route/dispatch, global aux statistics, local experts
-        B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, out["topk_idx"], out["topk_gate"],
-                out["n_real"], out["workspace"])
-        B.aux_sums(dm, out["workspace"], sums)
-        dist.all_reduce(sums)
-        B.aux_finalize(dm, sums, out["counts_ext"], out["P"], out["losses"])
-        B.dispatch(dm, x, out["topk_idx"], out["workspace"], out["counts"], out["offsets"], out["perm_tok"],
-                   out["slot_row"], out["xs"])
-        B.expert_ffn(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.w_down, layer.shared_gate_up,
-                     layer.shared_down, out["h"], out["h_shared"], out["ys"], out["shared_out"], out["workspace"])
-        B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"])
+        else:
+            dp_forward(layer, x, tnb, out, sums)
 
-    kernels_per_step = 5 if world == 1 else 7  # route, dispatch, gate_up, down, combine (+ aux sums/finalize)
+    # route, scan, dispatch(+aux), gate_up, down, combine (+ aux sums and finalize when data parallel)
+    kernels_per_step = 6 if world == 1 else 8
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -280,7 +276,7 @@ def main():
         raise SystemExit(f"device status after timing: {B.status_string(st)}")
 
     # ---- per-kernel breakdown (separately timed steps, same launches, CUDA events between them)
-    names = ["route", "dispatch", "gate_up", "down", "combine"]
+    names = ["route", "dispatch", "gate_up", "down", "combine"]  # "route" = route + scan launches
     acc = {n: 0.0 for n in names}
     nb = max(3, min(args.steps, 10))
     for _ in range(nb):

@@ -1,0 +1,112 @@
+"""Data-parallel aux statistics on CPU ranks (gloo, world size 2).
+
+Each rank takes half of the tokens, builds its additive statistics in the
+library's float64 layout (from the oracle, on CPU), and all-reduces them with
+the package's host logic. The reduced vector must equal the single-process
+statistics (integers exactly, float64 sums to 1e-13), and L_bal / L_z formed
+from it must equal the oracle's on all tokens.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle as O
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def packed_sums(idx, p, lse, N, M, K):
+    from token_choice_routing_b200.dist import aux_sums_slices
+    sl = aux_sums_slices(N, K)
+    v = np.zeros(sl["T"].stop)
+    counts_ext, psum, lsq, T = O.aux_partial_sums(idx, p, lse, N, M)
+    v[sl["counts_real"]] = counts_ext[:N]
+    nulls = (np.asarray(idx) >= N).sum(axis=1)
+    v[sl["null_hist"]] = np.bincount(nulls, minlength=K + 1)[:K + 1]
+    v[sl["psum"]] = np.concatenate([psum[:N], [psum[N] if M else 0.0]])
+    v[sl["lse2"]] = lsq
+    v[sl["T"]] = T
+    return v
+
+
+def finalize(v, N, M, K):
+    from token_choice_routing_b200.dist import aux_sums_slices
+    sl = aux_sums_slices(N, K)
+    hist = v[sl["null_hist"]]
+    counts_ext = np.concatenate([v[sl["counts_real"]], [hist[j + 1:].sum() for j in range(M)]])
+    psum = v[sl["psum"]]
+    psum_ext = np.concatenate([psum[:N], np.full(M, psum[N])])
+    T = v[sl["T"]][0]
+    return O.aux_finalize(counts_ext, psum_ext, v[sl["lse2"]][0], T, N)
+
+
+def _case():
+    rng = np.random.default_rng(77)
+    T, N, M, K = 400, 8, 24, 6
+    s = rng.standard_normal((T, N + 1))
+    s[:, N] += 0.8
+    return s, N, M, K
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from token_choice_routing_b200.dist import allreduce_aux_sums
+        s, N, M, K = _case()
+        shard = np.array_split(np.arange(s.shape[0]), world)[rank]
+        r = O.route(s[shard], M, K)
+        v = torch.from_numpy(packed_sums(r["idx"], r["p"], r["lse"], N, M, K))
+        allreduce_aux_sums(v)
+        q.put((rank, v.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_aux_allreduce_matches_single_process():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    s, N, M, K = _case()
+    r = O.route(s, M, K)
+    whole = packed_sums(r["idx"], r["p"], r["lse"], N, M, K)
+    from token_choice_routing_b200.dist import aux_sums_slices
+    sl = aux_sums_slices(N, K)
+    for rank in (0, 1):
+        v = res[rank]
+        for key in ("counts_real", "null_hist", "T"):
+            assert np.array_equal(v[sl[key]], whole[sl[key]]), key
+        np.testing.assert_allclose(v, whole, rtol=1e-13, atol=1e-12)
+        f, P, L_bal, L_z = finalize(v, N, M, K)
+        _, f0, P0, L_bal0, L_z0 = O.aux_stats(r["idx"], r["p"], r["lse"], N, M)
+        assert L_bal == pytest.approx(L_bal0, rel=1e-13)
+        assert L_z == pytest.approx(L_z0, rel=1e-13)
+        np.testing.assert_allclose(P, P0, rtol=1e-13)
+    # both ranks agree bit for bit
+    assert np.array_equal(res[0], res[1])
+
+
+def test_sums_layout_matches_library_count():
+    from token_choice_routing_b200.dist import aux_sums_slices
+    from token_choice_routing_b200 import binding as B
+    for N, M, K in ((8, 4, 4), (64, 8, 8), (5, 16, 16)):
+        assert aux_sums_slices(N, K)["T"].stop == B.aux_sums_count(B.dims(10, 128, N, M, K, 64, 64))

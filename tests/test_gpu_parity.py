@@ -107,25 +107,37 @@ def test_all_null_tokens_get_only_the_shared_expert():
 
 
 def test_exact_ties_break_by_index():
-    # duplicated router rows make exactly equal fp32 logits; the null row is a
-    # copy of real row 2, so real 2 ties the null logit and must precede every copy
+    # Integer-valued x and multiples of 1/8 in W_r make every router logit an
+    # exact fp32 value whatever the summation order, so equal rows give equal
+    # logits: many real-real ties, and the null row is a copy of real row 2, so
+    # real 2 ties the null logit and must precede every copy.
     cfg = I.small_config("ties", T=150, d=256, N=8, F=64, F_shared=64, K=6, M=4, config_id=911)
     inp = I.make_inputs(cfg)
-    w = inp.w_router
+    rng = np.random.default_rng(911)
+    inp.x = I.bf16_round(rng.integers(-3, 4, size=(cfg.T, cfg.d)).astype(np.float32))
+    w = (rng.integers(-4, 5, size=(cfg.N + 1, cfg.d)) / 8.0).astype(np.float32)
     w[3] = w[1]
     w[5] = w[1]
     w[cfg.N] = w[2]
+    inp.w_router = w
     inp.bias[:] = 0
     layer, x, tnb, out = H.run_forward(inp)
     lg = out["logits"].cpu().numpy()
+    assert np.array_equal(lg, H.oracle_logits(inp).astype(np.float32))
     assert np.array_equal(lg[:, 3], lg[:, 1]) and np.array_equal(lg[:, cfg.N], lg[:, 2])
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
+    H.check_aux(inp, out, r)
     idx = out["topk_idx"].cpu().numpy()
+    n_tie = 0
     for t in range(cfg.T):
         row = idx[t].tolist()
         if 2 in row and cfg.N in row:
             assert row.index(2) < row.index(cfg.N)
+            n_tie += 1
+        if 1 in row and 3 in row:
+            assert row.index(1) < row.index(3)
+    assert n_tie > 0
     H.check_layer_output(inp, out, r)
 
 
@@ -172,7 +184,7 @@ def test_zero_tokens_is_a_noop():
     from token_choice_routing_b200 import binding as B
     cfg = I.CONFIGS["tiny"]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, _ = H.make_layer(inp)
+    layer, x, tnb = H.make_layer(inp)
     out = layer.alloc(0)
     layer.forward(x[:0], None, out)
     torch.cuda.synchronize()

@@ -24,13 +24,16 @@ constexpr int kMaxK = 16;
 constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusBounds = 2u;
 
+// Byte offset of the per-expert row totals inside the workspace header.
+constexpr size_t kHdrTotOffset = 16;
+
 // Default limit of every device-side wait, in ns of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // Workspace layout, computed identically on the host for every entry point.
 struct WsLayout {
   int nblk;          // route CTAs = ceil(T / kRouteTokens)
-  size_t hdr;        // uint32 status, uint32 done-counter (256 B)
+  size_t hdr;        // uint32 status at 0; int32 per-expert totals at kHdrTotOffset (512 B)
   size_t counts_blk; // int32 [N][nblk]
   size_t bases;      // int32 [N][nblk]
   size_t ppart;      // float [nblk][N+1]
@@ -53,7 +56,7 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   WsLayout L{};
   L.nblk = (d.T + kRouteTokens - 1) / kRouteTokens;
   size_t o = 0;
-  L.hdr = o; o += 256;
+  L.hdr = o; o += 512;
   L.counts_blk = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N * L.nblk, 256);
   L.bases = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N * L.nblk, 256);
   L.ppart = o; o = align_up(o + sizeof(float) * (size_t)(d.N + 1) * L.nblk, 256);

@@ -36,7 +36,8 @@ struct RouteArgs {
   float* topk_gate;
   int32_t* n_real;
   // workspace
-  uint32_t* hdr;  // [0] status, [1] done counter
+  uint32_t* hdr;  // [0] status
+  int32_t* tot;   // [N] rows per expert (integer atomics)
   int32_t* counts_blk;
   int32_t* bases;
   float* ppart;
@@ -74,12 +75,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int sr
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-__device__ __forceinline__ int warp_sum_i(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 template <int RPT>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   constexpr int NPAD = 8 * RPT;
@@ -88,9 +83,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   float* xst = reinterpret_cast<float*>(smem);              // [2][64][kXS]
   float* wst = xst + 2 * kRouteTokens * kXS;                // [2][NPAD+1][kXS]
-  __shared__ int s_last;
-  __shared__ int s_tot[kMaxN];
-  __shared__ int s_off[kMaxN + 1];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tg = (warp & 1) * 8 + (lane & 7);   // token group 0..15
@@ -234,9 +226,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
     for (int i = 0; i < N; ++i) Z += expf(st[i] - m);
     if (M > 0) Z += (float)M * expf(sn - m);
     const float lse = m + logf(Z);
+    // p_i = e^{s_i - lse} evaluated as e^{s_i - m} / Z: no cancellation when |m| is large
     float* pt = p_s + t * LS;
-    for (int i = 0; i < N; ++i) pt[i] = expf(st[i] - lse);
-    pt[NPAD] = (M > 0) ? expf(sn - lse) : 0.f;
+    for (int i = 0; i < N; ++i) pt[i] = expf(st[i] - m) / Z;
+    pt[NPAD] = (M > 0) ? expf(sn - m) / Z : 0.f;
     lse2[t] = lse * lse;
 
     // top-K over the pool, in rank order
@@ -298,6 +291,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
       if ((mask[t] >> e) & 1ull) rtab[t * NPAD + e] = (unsigned char)(cnt++);
     }
     a.counts_blk[(size_t)e * a.nblk + b] = cnt;
+    if (cnt) atomicAdd(a.tot + e, cnt);
   }
   if (tid <= N) {
     const int col = (tid < N) ? tid : NPAD;
@@ -324,52 +318,62 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
     }
   }
 
-  // The last block to finish turns the per-block counts into offsets and
-  // per-block bases (exclusive scans; integer, so exact and order-free).
-  __threadfence();
-  __syncthreads();
+}
+
+// Per-expert scan over route blocks: bases[e][b] = offsets[e] + sum_{b' < b}
+// counts_blk[e][b'] (ascending token order inside an expert's segment), with
+// offsets[e] = sum_{e' < e} tot[e'] from the route blocks' integer atomics.
+// Integer sums, so the result does not depend on any execution order.
+constexpr int kScanThreads = 256;
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t* __restrict__ counts_blk,
+                                                            const int32_t* __restrict__ tot,
+                                                            int32_t* __restrict__ bases,
+                                                            int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets, int N, int nblk) {
+  __shared__ int s_warp[kScanThreads / 32];
+  __shared__ int s_off;
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
-    const unsigned prev = atomicAdd(&a.hdr[1], 1u);
-    s_last = (prev == (unsigned)(a.nblk - 1));
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const int nblk = a.nblk;
-  for (int e = warp; e < N; e += kRouteThreads / 32) {
-    int s = 0;
-    for (int bb = lane; bb < nblk; bb += 32) s += __ldcg(a.counts_blk + (size_t)e * nblk + bb);
-    s = warp_sum_i(s);
-    if (lane == 0) s_tot[e] = s;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int e = 0; e < N; ++e) {
-      s_off[e] = run;
-      run += s_tot[e];
-    }
-    s_off[N] = run;
-  }
-  __syncthreads();
-  if (tid <= N) a.offsets[tid] = s_off[tid];
-  if (tid < N) a.counts[tid] = s_tot[tid];
-  for (int e = warp; e < N; e += kRouteThreads / 32) {
-    int run = s_off[e];
-    for (int b0 = 0; b0 < nblk; b0 += 32) {
-      const int bb = b0 + lane;
-      const int v = (bb < nblk) ? __ldcg(a.counts_blk + (size_t)e * nblk + bb) : 0;
-      int inc = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += u;
+    int o = 0;
+    for (int q = 0; q < e; ++q) o += tot[q];
+    s_off = o;
+    if (e == 0) {
+      int run = 0;
+      for (int q = 0; q < N; ++q) {
+        offsets[q] = run;
+        counts[q] = tot[q];
+        run += tot[q];
       }
-      if (bb < nblk) a.bases[(size_t)e * nblk + bb] = run + inc - v;
-      run += __shfl_sync(0xffffffffu, inc, 31);
+      offsets[N] = run;
     }
   }
-  if (tid == 0) a.hdr[1] = 0u;
+  const int per = (nblk + kScanThreads - 1) / kScanThreads;
+  const int b0 = tid * per;
+  const int32_t* c = counts_blk + (size_t)e * nblk;
+  int loc = 0;
+  for (int q = 0; q < per; ++q) {
+    const int b = b0 + q;
+    if (b < nblk) loc += c[b];
+  }
+  int inc = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  int wpre = 0;
+  for (int w = 0; w < warp; ++w) wpre += s_warp[w];
+  int run = s_off + wpre + inc - loc;
+  for (int q = 0; q < per; ++q) {
+    const int b = b0 + q;
+    if (b < nblk) {
+      bases[(size_t)e * nblk + b] = run;
+      run += c[b];
+    }
+  }
 }
 
 template <int RPT>
@@ -402,6 +406,7 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.topk_gate = topk_gate;
   a.n_real = n_real;
   a.hdr = ws_ptr<uint32_t>(ws, L.hdr);
+  a.tot = ws_ptr<int32_t>(ws, L.hdr + kHdrTotOffset);
   a.counts_blk = ws_ptr<int32_t>(ws, L.counts_blk);
   a.bases = ws_ptr<int32_t>(ws, L.bases);
   a.ppart = ws_ptr<float>(ws, L.ppart);
@@ -416,13 +421,17 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.M = d.M;
   a.K = d.K;
   a.nblk = L.nblk;
-  // status and the done counter start at zero for every layer call
-  cudaError_t e = cudaMemsetAsync(a.hdr, 0, 2 * sizeof(uint32_t), st);
+  // the status word and the per-expert totals start at zero for every layer call
+  cudaError_t e = cudaMemsetAsync(a.hdr, 0, kHdrTotOffset + sizeof(int32_t) * d.N, st);
   if (e != cudaSuccess) return cuda_status(e);
-  if (d.N <= 8) return launch_route_t<1>(a, st);
-  if (d.N <= 16) return launch_route_t<2>(a, st);
-  if (d.N <= 32) return launch_route_t<4>(a, st);
-  return launch_route_t<8>(a, st);
+  int r;
+  if (d.N <= 8) r = launch_route_t<1>(a, st);
+  else if (d.N <= 16) r = launch_route_t<2>(a, st);
+  else if (d.N <= 32) r = launch_route_t<4>(a, st);
+  else r = launch_route_t<8>(a, st);
+  if (r != MOE_OK) return r;
+  scan_kernel<<<d.N, kScanThreads, 0, st>>>(a.counts_blk, a.tot, a.bases, a.counts, a.offsets, d.N, L.nblk);
+  return cuda_status(cudaGetLastError());
 }
 
 }  // namespace moe

@@ -1,0 +1,61 @@
+"""Data-parallel execution of the null-expert MoE layer.
+
+Every rank holds the full router and expert weights and runs the layer on its
+own tokens; y needs no exchange. The load-balance loss is a product of global
+means (f_i and P_i are averages over all tokens: Kilian et al., "Improving MoE
+Compute Efficiency by Composing Weight and Data Sparsity", review page,
+section 三 / 负载均衡损失), so ranks all-reduce the additive statistics, not the
+per-rank losses: one SUM all-reduce of a float64 vector laid out as
+
+    [counts_real (N) | null-slot histogram (K+1) | sum_t p (N+1) | sum_t lse^2 | T]
+
+(moe_aux_sums writes it, moe_aux_finalize reads it). Counts are integers held
+exactly in float64, so the reduced statistics equal a single-rank run's up to
+the order of the float64 sums.
+"""
+from __future__ import annotations
+
+from typing import Dict
+
+import torch
+import torch.distributed as dist
+
+
+def aux_sums_slices(N: int, K: int) -> Dict[str, slice]:
+    o = 0
+    out = {}
+    for name, n in (("counts_real", N), ("null_hist", K + 1), ("psum", N + 1), ("lse2", 1), ("T", 1)):
+        out[name] = slice(o, o + n)
+        o += n
+    return out
+
+
+def allreduce_aux_sums(sums: torch.Tensor, group=None) -> torch.Tensor:
+    """In-place SUM all-reduce of one rank's aux statistics vector."""
+    if sums.dtype != torch.float64:
+        raise TypeError("aux statistics are float64")
+    dist.all_reduce(sums, op=dist.ReduceOp.SUM, group=group)
+    return sums
+
+
+def dp_forward(layer, x, tok_null_bias, out, sums, group=None):
+    """One data-parallel layer step on this rank's tokens (stream-ordered).
+
+    route -> local aux sums -> all-reduce -> global L_bal/L_z -> dispatch ->
+    expert GEMMs -> combine. ``out`` comes from ``layer.alloc``; ``sums`` is a
+    float64 CUDA tensor of ``aux_sums_count`` elements.
+    """
+    from . import binding as B
+    dm = layer.dims(x.shape[0])
+    ws = out["workspace"]
+    B.route(dm, x, layer.w_router, layer.router_bias, tok_null_bias, out.get("logits"), out["topk_idx"],
+            out["topk_gate"], out["n_real"], ws)
+    B.aux_sums(dm, ws, sums)
+    allreduce_aux_sums(sums, group)
+    B.aux_finalize(dm, sums, out["counts_ext"], out["P"], out["losses"])
+    B.dispatch(dm, x, out["topk_idx"], ws, out["counts"], out["offsets"], out["perm_tok"], out["slot_row"],
+               out["xs"])
+    B.expert_ffn(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.w_down, layer.shared_gate_up,
+                 layer.shared_down, out["h"], out["h_shared"], out["ys"], out["shared_out"], ws)
+    B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"])
+    return out
