@@ -148,6 +148,26 @@ MOE_API int moe_route(const moe_dims_t* dims, const uint16_t* x, const float* w_
               int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* workspace,
               moe_stream_t stream);
 
+/* moe_route without a workspace argument, for callers that cannot allocate
+ * device memory: plugin-style interfaces that receive only their input and
+ * output buffers, and hot paths that must not call cudaMalloc because it can
+ * synchronise the device. The paper has no counterpart of this entry point; it
+ * is a deployment convenience. Same inputs, outputs and results as moe_route.
+ * Its internal scratch is a fixed MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES array in
+ * the library's own device memory, held by every GPU that loads the library
+ * until the process exits. Shapes whose moe_workspace_bytes exceeds that size
+ * are rejected with MOE_ERR_UNSUPPORTED before anything is enqueued. The first
+ * call on each device looks up the array's device address once; make that
+ * first call before any stream capture. All calls on a device share the array
+ * (each call clears what must start at zero): calls whose GPU work overlaps,
+ * e.g. on two unordered streams, race and give wrong results. It allocates
+ * nothing and does not fill a workspace for moe_dispatch. */
+#define MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES ((size_t)8 << 20)
+MOE_API int moe_route_noalloc(const moe_dims_t* dims, const uint16_t* x, const float* w_router,
+                              const float* router_bias, const float* tok_null_bias, float* logits_out,
+                              int32_t* topk_idx, float* topk_gate, int32_t* n_real,
+                              moe_stream_t stream);
+
 /* Dispatch (section 三 / 实现: nulls sorted to the end and truncated). After
  * moe_route with the same workspace. counts [N], offsets [N+1]; the real slots
  * are laid out expert by expert, tokens ascending inside an expert: perm_tok
