@@ -38,15 +38,29 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
         acc[0] = bf16lo(v.x); acc[1] = bf16hi(v.x); acc[2] = bf16lo(v.y); acc[3] = bf16hi(v.y);
         acc[4] = bf16lo(v.z); acc[5] = bf16hi(v.z); acc[6] = bf16lo(v.w); acc[7] = bf16hi(v.w);
       }
-      for (int k = 0; k < K; ++k) {
-        const int r = __shfl_sync(0xffffffffu, row, k);
-        const float gk = __shfl_sync(0xffffffffu, g, k);
-        if (r >= 0 && ok) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(ys + (size_t)r * d) + c);
-          acc[0] = fmaf(gk, bf16lo(v.x), acc[0]); acc[1] = fmaf(gk, bf16hi(v.x), acc[1]);
-          acc[2] = fmaf(gk, bf16lo(v.y), acc[2]); acc[3] = fmaf(gk, bf16hi(v.y), acc[3]);
-          acc[4] = fmaf(gk, bf16lo(v.z), acc[4]); acc[5] = fmaf(gk, bf16hi(v.z), acc[5]);
-          acc[6] = fmaf(gk, bf16lo(v.w), acc[6]); acc[7] = fmaf(gk, bf16hi(v.w), acc[7]);
+      // slots in rank order, four at a time: issue the real rows' loads before using any
+      for (int k0 = 0; k0 < K; k0 += 4) {
+        uint4 v[4];
+        float gq[4];
+        int rq[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = k0 + u;
+          rq[u] = __shfl_sync(0xffffffffu, row, k & 31);
+          gq[u] = __shfl_sync(0xffffffffu, g, k & 31);
+          if (k >= K) rq[u] = -1;
+          v[u] = (rq[u] >= 0 && ok) ? __ldg(reinterpret_cast<const uint4*>(ys + (size_t)rq[u] * d) + c)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (rq[u] >= 0) {
+            const float gk = gq[u];
+            acc[0] = fmaf(gk, bf16lo(v[u].x), acc[0]); acc[1] = fmaf(gk, bf16hi(v[u].x), acc[1]);
+            acc[2] = fmaf(gk, bf16lo(v[u].y), acc[2]); acc[3] = fmaf(gk, bf16hi(v[u].y), acc[3]);
+            acc[4] = fmaf(gk, bf16lo(v[u].z), acc[4]); acc[5] = fmaf(gk, bf16hi(v[u].z), acc[5]);
+            acc[6] = fmaf(gk, bf16lo(v[u].w), acc[6]); acc[7] = fmaf(gk, bf16hi(v[u].w), acc[7]);
+          }
         }
       }
       if (ok) {

@@ -5,73 +5,44 @@
 // Sparsity" (review page, section 三 / 实现): null indices (>= N) are moved to
 // the end of the sorted (token, expert) list and cut off before the grouped
 // matmul. Here no sort is run: the route kernel already produced, per block of
-// 64 tokens, each slot's rank among the block's tokens that chose the same
+// 32 tokens, each slot's rank among the block's tokens that chose the same
 // expert, and the per-(expert, block) base row. A slot's row is base + rank,
 // which is the stable (expert, token) order. Null slots are skipped before any
 // load, so they cost no memory traffic.
 //
 // Aux (same page, 负载均衡损失 and Z-Loss): L_bal = N * sum_{i<N+M} f_i P_i with
 // f_i = count_i / T and P_i = mean_t p_{t,i}; L_z = mean_t lse_t^2. Per-block
-// fp32 partials from the route kernel are summed here in fp64 in block order.
+// fp32 partials from the route kernel are summed in fp64, first over fixed
+// slices of blocks (in the scan launch), then over the slices here.
 #include "moe_internal.cuh"
 
 namespace moe {
 
 struct AuxPtrs {
   const int32_t* counts;  // [N] real counts (route scan)
-  const float* ppart;     // [nblk][N+1]
-  const float* lsq;       // [nblk]
-  const int32_t* hist;    // [nblk][K+1]
-  int nblk, N, M, K, T;
+  const double* auxp;     // [nparts][(N+1) + (K+1) + 1] fp64 partials (scan launch)
+  int nparts, N, M, K, T;
 };
 
-// sums layout: [counts_real N | hist K+1 | psum N+1 | lsq | T]
+// sums layout: [counts_real N | hist K+1 | psum N+1 | lsq | T]; the
+// first-level partials are combined in their fixed order (deterministic).
 __device__ void aux_sums_block(const AuxPtrs& p, double* sums) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
-  const int N = p.N, K = p.K, nblk = p.nblk;
+  const int tid = threadIdx.x;
+  const int N = p.N, K = p.K;
   double* s_cnt = sums;
   double* s_hist = sums + N;
   double* s_psum = s_hist + (K + 1);
   double* s_lsq = s_psum + (N + 1);
+  const int c1 = N + 1, c2 = c1 + K + 1, cols = c2 + 1;
   for (int e = tid; e < N; e += blockDim.x) s_cnt[e] = (double)p.counts[e];
-  // null histogram: one warp per bucket, lanes stride over blocks
-  for (int c = warp; c <= K; c += nwarps) {
-    long long acc = 0;
-    for (int b = lane; b < nblk; b += 32) acc += p.hist[(size_t)b * (K + 1) + c];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) s_hist[c] = (double)acc;
-  }
-  // probability sums: column i, phases over blocks; then phases combined in order
-  __shared__ double s_ph[8][kMaxN + 1];
-  const int ncol = N + 1;
-  const int nph = min(8, (int)blockDim.x / ncol);
-  {
-    const int col = tid % ncol, ph = tid / ncol;
-    if (ph < nph) {
-      double acc = 0.0;
-      for (int b = ph; b < nblk; b += nph) acc += (double)p.ppart[(size_t)b * ncol + col];
-      s_ph[ph][col] = acc;
-    }
-  }
-  // lse^2: last warp, lane-strided then a fixed shuffle tree
-  if (warp == nwarps - 1) {
+  for (int c = tid; c < cols; c += blockDim.x) {
     double acc = 0.0;
-    for (int b = lane; b < nblk; b += 32) acc += (double)p.lsq[b];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      *s_lsq = acc;
-      s_lsq[1] = (double)p.T;
-    }
+    for (int g = 0; g < p.nparts; ++g) acc += p.auxp[(size_t)g * cols + c];
+    if (c < c1) s_psum[c] = acc;
+    else if (c < c2) s_hist[c - c1] = acc;
+    else s_lsq[0] = acc;
   }
-  __syncthreads();
-  for (int col = tid; col < ncol; col += blockDim.x) {
-    double acc = 0.0;
-    for (int ph = 0; ph < nph; ++ph) acc += s_ph[ph][col];
-    s_psum[col] = acc;
-  }
+  if (tid == 0) s_lsq[1] = (double)p.T;
   __syncthreads();
 }
 
@@ -205,10 +176,8 @@ static AuxPtrs aux_ptrs(const moe_dims_t& d, const void* ws) {
   const WsLayout L = ws_layout(d);
   AuxPtrs p{};
   p.counts = ws_ptr<int32_t>(ws, L.counts);
-  p.ppart = ws_ptr<float>(ws, L.ppart);
-  p.lsq = ws_ptr<float>(ws, L.lsq);
-  p.hist = ws_ptr<int32_t>(ws, L.hist);
-  p.nblk = L.nblk;
+  p.auxp = ws_ptr<double>(ws, L.auxp);
+  p.nparts = L.nparts;
   p.N = d.N;
   p.M = d.M;
   p.K = d.K;

@@ -14,9 +14,9 @@ namespace moe {
 
 // ------------------------------------------------------------------------------------
 // Tiling constants of the route kernel (fp32 CUDA-core router GEMM + routing).
-constexpr int kRouteTokens = 64;    // tokens per route CTA
+constexpr int kRouteTokens = 32;    // tokens per route CTA
 constexpr int kRouteBK = 32;        // d-slice per pipeline stage
-constexpr int kRouteThreads = 128;  // 16 token groups x 8 logit groups
+constexpr int kRouteThreads = 128;  // 8 token groups x 16 logit groups
 constexpr int kMaxN = 64;
 constexpr int kMaxK = 16;
 
@@ -43,10 +43,17 @@ struct WsLayout {
   size_t counts;     // int32 [N]
   size_t offsets;    // int32 [N+1]
   size_t sums;       // double [aux sums count]
+  int nparts;        // first-level aux partials = min(kAuxParts, nblk)
+  size_t auxp;       // double [nparts][aux_part_cols]
   size_t total;
 };
 
 constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// First-level aux partials: each of up to kAuxParts CTAs reduces a fixed,
+// contiguous slice of route blocks in fp64: [sum p (N+1) | null hist (K+1) | sum lse^2].
+constexpr int kAuxParts = 64;
+inline int aux_part_cols(const moe_dims_t& d) { return (d.N + 1) + (d.K + 1) + 1; }
 
 inline size_t aux_sums_count(const moe_dims_t& d) {
   return (size_t)d.N + (size_t)(d.K + 1) + (size_t)(d.N + 1) + 2;
@@ -66,6 +73,8 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   L.counts = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N, 256);
   L.offsets = o; o = align_up(o + sizeof(int32_t) * (size_t)(d.N + 1), 256);
   L.sums = o; o = align_up(o + sizeof(double) * aux_sums_count(d), 256);
+  L.nparts = L.nblk < kAuxParts ? L.nblk : kAuxParts;
+  L.auxp = o; o = align_up(o + sizeof(double) * (size_t)L.nparts * aux_part_cols(d), 256);
   L.total = o;
   return L;
 }
