@@ -5,7 +5,7 @@
 // Sparsity" (review page, section 三 / 实现): null indices (>= N) are moved to
 // the end of the sorted (token, expert) list and cut off before the grouped
 // matmul. Here no sort is run: the route kernel already produced, per block of
-// 32 tokens, each slot's rank among the block's tokens that chose the same
+// 64 tokens, each slot's rank among the block's tokens that chose the same
 // expert, and the per-(expert, block) base row. A slot's row is base + rank,
 // which is the stable (expert, token) order. Null slots are skipped before any
 // load, so they cost no memory traffic.
@@ -24,10 +24,11 @@ struct AuxPtrs {
   int nparts, N, M, K, T;
 };
 
-// sums layout: [counts_real N | hist K+1 | psum N+1 | lsq | T]; the
-// first-level partials are combined in their fixed order (deterministic).
+// sums layout: [counts_real N | hist K+1 | psum N+1 | lsq | T]. The first-level
+// partials (at most kAuxParts = 64 of them) are combined one column per warp:
+// lane l adds partials l and l+32, then a fixed shuffle tree (deterministic).
 __device__ void aux_sums_block(const AuxPtrs& p, double* sums) {
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   const int N = p.N, K = p.K;
   double* s_cnt = sums;
   double* s_hist = sums + N;
@@ -35,12 +36,17 @@ __device__ void aux_sums_block(const AuxPtrs& p, double* sums) {
   double* s_lsq = s_psum + (N + 1);
   const int c1 = N + 1, c2 = c1 + K + 1, cols = c2 + 1;
   for (int e = tid; e < N; e += blockDim.x) s_cnt[e] = (double)p.counts[e];
-  for (int c = tid; c < cols; c += blockDim.x) {
+  for (int c = warp; c < cols; c += nwarps) {
     double acc = 0.0;
-    for (int g = 0; g < p.nparts; ++g) acc += p.auxp[(size_t)g * cols + c];
-    if (c < c1) s_psum[c] = acc;
-    else if (c < c2) s_hist[c - c1] = acc;
-    else s_lsq[0] = acc;
+    if (lane < p.nparts) acc = p.auxp[(size_t)lane * cols + c];
+    if (lane + 32 < p.nparts) acc += p.auxp[(size_t)(lane + 32) * cols + c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      if (c < c1) s_psum[c] = acc;
+      else if (c < c2) s_hist[c - c1] = acc;
+      else s_lsq[0] = acc;
+    }
   }
   if (tid == 0) s_lsq[1] = (double)p.T;
   __syncthreads();

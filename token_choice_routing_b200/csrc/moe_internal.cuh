@@ -14,9 +14,9 @@ namespace moe {
 
 // ------------------------------------------------------------------------------------
 // Tiling constants of the route kernel (fp32 CUDA-core router GEMM + routing).
-constexpr int kRouteTokens = 32;    // tokens per route CTA
+constexpr int kRouteTokens = 64;    // tokens per route CTA
 constexpr int kRouteBK = 32;        // d-slice per pipeline stage
-constexpr int kRouteThreads = 128;  // 8 token groups x 16 logit groups
+constexpr int kRouteThreads = 256;  // 8 token groups x logit groups x d-slices
 constexpr int kMaxN = 64;
 constexpr int kMaxK = 16;
 

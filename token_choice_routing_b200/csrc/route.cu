@@ -14,9 +14,9 @@
 //  * renormalisation over the selected reals: gates = softmax over their
 //    logits; null slots weigh 0.
 //  * Z-Loss / 负载均衡损失: lse_t over the N+M pool and p_{t,i} are reduced per
-//    block here (fp32 over 32 tokens) and across blocks in fp64 later.
+//    block here (fp32 over 64 tokens) and across blocks in fp64 later.
 //
-// Layout: one CTA = 32 tokens x all N+1 logits (see route_kernel). x (bf16) is
+// Layout: one CTA = 64 tokens x all N+1 logits (see route_kernel). x (bf16) is
 // widened to fp32 once when staged in shared memory; W_r slices arrive by
 // cp.async, double-buffered.
 #include "moe_internal.cuh"
@@ -50,22 +50,51 @@ struct RouteArgs {
 
 constexpr int kXS = kRouteBK + 4;  // padded fp32 row stride of staged tiles
 
-template <int NPAD>
-struct RouteSmem {
-  static constexpr int LS = NPAD + 1;  // odd stride: conflict-free per-token rows
+// Thread tile of the router product: 8 tokens x 8 reals. Shared memory, not
+// the FMA pipe, bounds an fp32 CUDA-core GEMM: an a x b register tile loads
+// (a + b) / (a b) floats per FMA, and 8 x 8 keeps that at 1/4, the balance
+// point of an SM. Staged tiles are stored k-major (x^T and W^T) so a thread
+// fetches its 8 tokens and 8 reals at one d-column with four 16-byte loads.
+// To keep enough warps, the d-columns of each staged tile are split over S
+// thread slices whose partial sums are added once at the end.
+constexpr int kTileT = 8;  // tokens per thread
+constexpr int kTileR = 8;  // reals per thread
+constexpr int kXT = kRouteTokens + 4;  // row stride of the staged x^T tile
+
+template <int LG>
+struct RouteGeo {
+  static constexpr int NPAD = kTileR * LG;            // padded real count
+  static constexpr int TG = kRouteTokens / kTileT;    // token groups (8)
+  static constexpr int S = kRouteThreads / (TG * LG); // d-slices per staged tile
+  static constexpr int KS = kRouteBK / S;             // d-columns per slice per tile (= LG)
+  static_assert(S * KS == kRouteBK, "slices must tile the staged d-range");
+  static constexpr int WT = NPAD + 4;                 // row stride of the staged W^T tile (null at NPAD)
+  static constexpr int WCH = (NPAD + 1) * (kRouteBK / 8);  // 8-float chunks of a W tile
+  static constexpr int WPT = (WCH + kRouteThreads - 1) / kRouteThreads;  // chunks per thread
+  static constexpr int LS = NPAD + 1;                 // odd row stride
+  // per-thread cp.async landing slot: 16 B of x (8 bf16) then WPT 8-float W chunks
+  static constexpr int LAND = WPT * 8 + 4;
   static constexpr size_t main_bytes =
-      sizeof(float) * (2 * kRouteTokens * kXS + 2 * (NPAD + 1) * kXS);
-  static constexpr size_t off_s = 0;
-  static constexpr size_t off_p = off_s + sizeof(float) * kRouteTokens * LS;
-  static constexpr size_t off_npart = off_p + sizeof(float) * kRouteTokens * LS;
-  static constexpr size_t off_lse2 = off_npart + sizeof(float) * 16 * kRouteTokens;
+      sizeof(float) * (2 * kRouteBK * (kXT + WT) + 2 * (size_t)kRouteThreads * LAND);
+  // slice partial sums [S][64][NPAD+1] alias the main-loop buffers
+  static constexpr size_t red_bytes = sizeof(float) * S * kRouteTokens * (NPAD + 1);
+  static constexpr size_t regionB = align_up(main_bytes > red_bytes ? main_bytes : red_bytes, 16);
+  // region C (after B): null partials and the logits
+  static constexpr int NNP = kRouteThreads / kRouteTokens;  // null partial sums per token (4)
+  static constexpr size_t off_npart = regionB;
+  static constexpr size_t off_s = off_npart + sizeof(float) * NNP * kRouteTokens;
+  static constexpr size_t endC = off_s + sizeof(float) * kRouteTokens * LS;
+  // per-token scratch reuses region B once the partial sums are folded
+  static constexpr size_t off_p = 0;
+  static constexpr size_t off_lse2 = off_p + sizeof(float) * kRouteTokens * LS;
   static constexpr size_t off_nul = off_lse2 + sizeof(float) * kRouteTokens;
   static constexpr size_t off_mask = align_up(off_nul + sizeof(int) * kRouteTokens, 16);
   static constexpr size_t off_tk = off_mask + sizeof(unsigned long long) * kRouteTokens;
   static constexpr size_t off_tkv = off_tk + sizeof(int) * kRouteTokens * kMaxK;
-  static constexpr size_t off_rtab = off_tkv + sizeof(float) * kRouteTokens * kMaxK;
-  static constexpr size_t epi_bytes = off_rtab + (size_t)kRouteTokens * NPAD;
-  static constexpr size_t bytes = main_bytes > epi_bytes ? main_bytes : epi_bytes;
+  static constexpr size_t off_tokbits = off_tkv + sizeof(float) * kRouteTokens * kMaxK;
+  static constexpr size_t endB = off_tokbits + sizeof(unsigned) * 2 * kMaxN;
+  static_assert(endB <= regionB, "per-token scratch must fit in region B");
+  static constexpr size_t bytes = endC;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
@@ -74,139 +103,164 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int sr
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// d = a * b + d on two fp32 lanes at once (sm_100 paired FMA).
-__device__ __forceinline__ void ffma2(float2& d, float2 a, float2 b) {
-  unsigned long long dd = *reinterpret_cast<unsigned long long*>(&d);
-  const unsigned long long aa = *reinterpret_cast<const unsigned long long*>(&a);
-  const unsigned long long bb = *reinterpret_cast<const unsigned long long*>(&b);
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(dd) : "l"(aa), "l"(bb));
-  d = *reinterpret_cast<float2*>(&dd);
-}
+__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // (value desc, index asc) order: true if (va, ia) precedes (vb, ib).
 __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
-// One CTA: 32 tokens x all N+1 logits. Main loop: 128 threads as 8 token
-// groups x 16 logit groups; a thread owns 4 tokens (stride 8) x RPT reals
-// (stride 16) and 2 of every 32 d-columns of the null logit. Epilogue: 4
-// threads per token (reals i = q, q+4, ...), combined with 4-lane shuffles.
-template <int RPT>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
-  constexpr int NPAD = 16 * RPT;
+// One CTA: 64 tokens x all N+1 logits, 256 threads. Main loop: thread
+// (s, lg, tg) owns tokens {4tg..4tg+3, 32+4tg..32+4tg+3} and reals
+// {4lg..4lg+3, 4LG+4lg..4LG+4lg+3} over the d-columns [s*KS, (s+1)*KS) of
+// every staged tile; the null logit of token tid & 63 over the 8 d-columns it stages.
+// Epilogue: 4 threads per token.
+template <int LG>
+__global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
+  using G = RouteGeo<LG>;
+  constexpr int NPAD = G::NPAD, S = G::S, KS = G::KS, LS = G::LS, WT = G::WT;
   constexpr int NQ = NPAD / 4;  // reals per epilogue thread
-  using SM = RouteSmem<NPAD>;
-  constexpr int LS = SM::LS;
   extern __shared__ __align__(16) unsigned char smem[];
-  float* xst = reinterpret_cast<float*>(smem);              // [2][32][kXS]
-  float* wst = xst + 2 * kRouteTokens * kXS;                // [2][NPAD+1][kXS]
+  float* xsT = reinterpret_cast<float*>(smem);       // [2][BK][kXT]
+  float* wsT = xsT + 2 * kRouteBK * kXT;             // [2][BK][WT]
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tg = lane & 7;                  // token group 0..7
-  const int lg = warp * 4 + (lane >> 3);    // logit group 0..15
+  const int tid = threadIdx.x;
+  const int tg = tid % G::TG;
+  const int lg = (tid / G::TG) % LG;
+  const int sl = tid / (G::TG * LG);
   const int b = blockIdx.x;
   const int T = a.T, d = a.d, N = a.N, M = a.M, K = a.K;
   const int tok0 = b * kRouteTokens;
   const int nvalid = min(kRouteTokens, T - tok0);
   const int nkt = d / kRouteBK;
 
-  // Paired fp32 FMAs (fma.rn.f32x2): .x accumulates the even d-columns, .y the
-  // odd ones; the two partial sums are added once at the end.
-  float2 acc[4][RPT];
-  float2 accn[4];
+  float acc[kTileT][kTileR];
+  float accn = 0.f;  // null logit of token tid & 63 over d-columns (tid >> 6) * 8 .. +8 of each tile
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    accn[i] = make_float2(0.f, 0.f);
+  for (int i = 0; i < kTileT; ++i)
 #pragma unroll
-    for (int j = 0; j < RPT; ++j) acc[i][j] = make_float2(0.f, 0.f);
-  }
+    for (int j = 0; j < kTileR; ++j) acc[i][j] = 0.f;
 
-  // x tile: 32 rows x 32 bf16 = 128 16-byte chunks, one per thread
-  const int xrow = tid >> 2, xcol8 = (tid & 3) * 8;
+  // Staging, two tiles ahead: every thread copies its own pieces of tile kt+2
+  // by cp.async into its own landing slot (x: token tid & 63, 8 d-columns from
+  // (tid >> 6) * 8; W: chunk c = tid + 256 q -> row c % (NPAD+1), 8 d-columns
+  // from (c / (NPAD+1)) * 8) while tile kt is multiplied; after its own wait it
+  // writes tile kt+1 transposed into the free stage buffer. No registers are
+  // held across the multiply and no extra barrier is needed.
+  const int xrow = tid & 63, xkc = (tid >> 6) * 8;
   const bool xok = tok0 + xrow < T;
-  const uint16_t* xsrc = a.x + (size_t)(tok0 + xrow) * d + xcol8;
-  uint4 xr = make_uint4(0u, 0u, 0u, 0u);
-  auto load_x = [&](int kt) {
-    if (xok) xr = __ldg(reinterpret_cast<const uint4*>(xsrc + (size_t)kt * kRouteBK));
-  };
-  auto store_x = [&](int buf) {
-    float4* dst = reinterpret_cast<float4*>(xst + buf * kRouteTokens * kXS + xrow * kXS + xcol8);
-    dst[0] = make_float4(bf16lo(xr.x), bf16hi(xr.x), bf16lo(xr.y), bf16hi(xr.y));
-    dst[1] = make_float4(bf16lo(xr.z), bf16hi(xr.z), bf16lo(xr.w), bf16hi(xr.w));
-  };
-  auto load_w = [&](int kt, int buf) {
-    float* wb = wst + buf * (NPAD + 1) * kXS;
-    for (int c = tid; c < (NPAD + 1) * 8; c += kRouteThreads) {
-      const int r = c >> 3, col4 = (c & 7) * 4;
-      const int src_row = (r < N) ? r : (r == NPAD ? N : -1);
-      const float* src = a.w + (size_t)(src_row < 0 ? 0 : src_row) * d + (size_t)kt * kRouteBK + col4;
-      cp_async16(smem_u32(wb + r * kXS + col4), src, src_row < 0 ? 0 : 16);
-    }
-    cp_async_commit();
-  };
-
-  load_x(0);
-  load_w(0, 0);
-  for (int kt = 0; kt < nkt; ++kt) {
-    const int buf = kt & 1;
-    store_x(buf);
-    cp_async_wait_all();
-    __syncthreads();
-    if (kt + 1 < nkt) {
-      load_x(kt + 1);
-      load_w(kt + 1, buf ^ 1);
-    }
-    const float* xb = xst + buf * kRouteTokens * kXS;
-    const float* wb = wst + buf * (NPAD + 1) * kXS;
+  const uint16_t* xsrc = a.x + (size_t)(tok0 + (xok ? xrow : 0)) * d + xkc;
+  float* land0 = wsT + 2 * kRouteBK * WT + tid * G::LAND;
+  auto land = [&](int slot) { return land0 + slot * kRouteThreads * G::LAND; };
+  auto load_tiles = [&](int kt, int slot) {
+    if (kt < nkt) {
+      float* L = land(slot);
+      cp_async16(smem_u32(L), xsrc + (size_t)kt * kRouteBK, xok ? 16 : 0);
 #pragma unroll
-    for (int kk = 0; kk < kRouteBK / 4; ++kk) {
-      float4 xv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(xb + (tg + 8 * i) * kXS + kk * 4);
-#pragma unroll
-      for (int jj = 0; jj < RPT; ++jj) {
-        const float4 wv = *reinterpret_cast<const float4*>(wb + (lg + 16 * jj) * kXS + kk * 4);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          ffma2(acc[i][jj], make_float2(xv[i].x, xv[i].y), make_float2(wv.x, wv.y));
-          ffma2(acc[i][jj], make_float2(xv[i].z, xv[i].w), make_float2(wv.z, wv.w));
+      for (int q = 0; q < G::WPT; ++q) {
+        const int c = tid + kRouteThreads * q;
+        if (c < G::WCH) {
+          const int r = c % (NPAD + 1), kc = (c / (NPAD + 1)) * 8;
+          const int src_row = (r < N) ? r : (r == NPAD ? N : -1);
+          const float* src = a.w + (size_t)(src_row < 0 ? 0 : src_row) * d + (size_t)kt * kRouteBK + kc;
+          cp_async16(smem_u32(L + 4 + q * 8), src, src_row < 0 ? 0 : 16);
+          cp_async16(smem_u32(L + 8 + q * 8), src + 4, src_row < 0 ? 0 : 16);
         }
       }
     }
-    {  // the null logit: this logit group's 2 columns of the d-tile
-      const float2 wn = *reinterpret_cast<const float2*>(wb + NPAD * kXS + lg * 2);
+    cp_async_commit();  // one group per call, possibly empty
+  };
+  auto store_tiles = [&](int buf, int slot) {
+    const float* L = land(slot);
+    const uint4 xr = *reinterpret_cast<const uint4*>(L);
+    float* xb = xsT + buf * kRouteBK * kXT;
+    const float xv[8] = {bf16lo(xr.x), bf16hi(xr.x), bf16lo(xr.y), bf16hi(xr.y),
+                         bf16lo(xr.z), bf16hi(xr.z), bf16lo(xr.w), bf16hi(xr.w)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 xv = *reinterpret_cast<const float2*>(xb + (tg + 8 * i) * kXS + lg * 2);
-        ffma2(accn[i], xv, wn);
+    for (int u = 0; u < 8; ++u) xb[(xkc + u) * kXT + xrow] = xv[u];
+    float* wb = wsT + buf * kRouteBK * WT;
+#pragma unroll
+    for (int q = 0; q < G::WPT; ++q) {
+      const int c = tid + kRouteThreads * q;
+      if (c < G::WCH) {
+        const int r = c % (NPAD + 1), kc = (c / (NPAD + 1)) * 8;
+        const float4 w0 = *reinterpret_cast<const float4*>(L + 4 + q * 8);
+        const float4 w1 = *reinterpret_cast<const float4*>(L + 8 + q * 8);
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) wb[(kc + u) * WT + r] = wv[u];
       }
+    }
+  };
+
+  load_tiles(0, 0);
+  load_tiles(1, 1);
+  cp_async_wait_group1();  // this thread's copies of tile 0
+  store_tiles(0, 0);
+  for (int kt = 0; kt < nkt; ++kt) {
+    const int buf = kt & 1;
+    __syncthreads();
+    load_tiles(kt + 2, buf);  // slot `buf` held tile kt, already written out
+    const float* xb = xsT + buf * kRouteBK * kXT + (sl * KS) * kXT;
+    const float* wb = wsT + buf * kRouteBK * WT + (sl * KS) * WT;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      const float4 xa = *reinterpret_cast<const float4*>(xb + kk * kXT + 4 * tg);
+      const float4 xc = *reinterpret_cast<const float4*>(xb + kk * kXT + 32 + 4 * tg);
+      const float4 wa = *reinterpret_cast<const float4*>(wb + kk * WT + 4 * lg);
+      const float4 wc = *reinterpret_cast<const float4*>(wb + kk * WT + 4 * LG + 4 * lg);
+      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xc.x, xc.y, xc.z, xc.w};
+      const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wc.x, wc.y, wc.z, wc.w};
+#pragma unroll
+      for (int i = 0; i < kTileT; ++i)
+#pragma unroll
+        for (int jj = 0; jj < kTileR; ++jj) acc[i][jj] = fmaf(xv[i], wv[jj], acc[i][jj]);
+    }
+    {  // the null logit: token xrow over the 8 d-columns this thread stages
+      const float* xn = xsT + buf * kRouteBK * kXT + xkc * kXT + xrow;
+      const float* wn = wsT + buf * kRouteBK * WT + xkc * WT + NPAD;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) accn = fmaf(xn[u * kXT], wn[u * WT], accn);
+    }
+    if (kt + 1 < nkt) {
+      cp_async_wait_group1();    // this thread's copies of tile kt+1 (tile kt+2 may be in flight)
+      store_tiles(buf ^ 1, buf ^ 1);  // that stage buffer was last read before this iteration's barrier
     }
   }
   __syncthreads();  // main-loop buffers are reused below
 
-  float* s_l = reinterpret_cast<float*>(smem + SM::off_s);
-  float* p_s = reinterpret_cast<float*>(smem + SM::off_p);
-  float* npart = reinterpret_cast<float*>(smem + SM::off_npart);
-  float* lse2 = reinterpret_cast<float*>(smem + SM::off_lse2);
-  int* nul = reinterpret_cast<int*>(smem + SM::off_nul);
-  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem + SM::off_mask);
-  int* tk = reinterpret_cast<int*>(smem + SM::off_tk);
-  float* tkv = reinterpret_cast<float*>(smem + SM::off_tkv);
-  unsigned char* rtab = smem + SM::off_rtab;
-
+  float* red = reinterpret_cast<float*>(smem);  // [S][64][NPAD+1]
+  float* npart = reinterpret_cast<float*>(smem + G::off_npart);
+  float* s_l = reinterpret_cast<float*>(smem + G::off_s);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = tg + 8 * i;
+  for (int i = 0; i < kTileT; ++i) {
+    const int t = 4 * tg + (i & 3) + 32 * (i >> 2);
 #pragma unroll
-    for (int jj = 0; jj < RPT; ++jj) {
-      const int j = lg + 16 * jj;
-      if (j < N) s_l[t * LS + j] = (acc[i][jj].x + acc[i][jj].y) + (a.bias ? __ldg(a.bias + j) : 0.f);
+    for (int jj = 0; jj < kTileR; ++jj) {
+      const int r = 4 * lg + (jj & 3) + 4 * LG * (jj >> 2);
+      red[(sl * kRouteTokens + t) * (NPAD + 1) + r] = acc[i][jj];
     }
-    npart[lg * kRouteTokens + t] = accn[i].x + accn[i].y;
   }
+  npart[(tid >> 6) * kRouteTokens + (tid & 63)] = accn;
   __syncthreads();
+  for (int o = tid; o < kRouteTokens * NPAD; o += kRouteThreads) {
+    const int t = o / NPAD, j = o - t * NPAD;
+    if (j < N) {
+      float v = 0.f;
+#pragma unroll
+      for (int q = 0; q < S; ++q) v += red[(q * kRouteTokens + t) * (NPAD + 1) + j];
+      s_l[t * LS + j] = v + (a.bias ? __ldg(a.bias + j) : 0.f);
+    }
+  }
+  __syncthreads();  // region B is free from here on
+
+  float* p_s = reinterpret_cast<float*>(smem + G::off_p);
+  float* lse2 = reinterpret_cast<float*>(smem + G::off_lse2);
+  int* nul = reinterpret_cast<int*>(smem + G::off_nul);
+  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem + G::off_mask);
+  int* tk = reinterpret_cast<int*>(smem + G::off_tk);
+  float* tkv = reinterpret_cast<float*>(smem + G::off_tkv);
+  unsigned* tokbits = reinterpret_cast<unsigned*>(smem + G::off_tokbits);  // [2][kMaxN]
 
   {
     // ---- per-token routing, 4 lanes per token (all lanes take part in the shuffles)
@@ -215,7 +269,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
     const int tok = tok0 + t;
     float sn = 0.f;
 #pragma unroll
-    for (int l = 0; l < 16; ++l) sn += npart[l * kRouteTokens + t];
+    for (int l = 0; l < G::NNP; ++l) sn += npart[l * kRouteTokens + t];
     if (a.bias) sn += __ldg(a.bias + N);
     if (a.tnb && valid) sn += __ldg(a.tnb + tok);
     float v[NQ];
@@ -330,40 +384,54 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   }
   __syncthreads();
 
-  // Per-block ranks and counts (ascending token order inside an expert), P sums.
-  if (tid < N) {
-    const int e = tid;
-    int cnt = 0;
-    for (int t = 0; t < nvalid; ++t) {
-      if ((mask[t] >> e) & 1ull) rtab[t * NPAD + e] = (unsigned char)(cnt++);
+  // Per-block ranks and counts (ascending token order inside an expert): for
+  // each expert e, warps 0 and 1 ballot bit e of their 32 tokens' selection
+  // masks, giving the block's tokens that chose e as a 64-bit set; a slot's
+  // rank is the number of earlier tokens in that set.
+  const int lane = tid & 31, warp = tid >> 5;
+  if (warp < 2) {
+    const int t = 32 * warp + lane;
+    const unsigned long long m = (t < nvalid) ? mask[t] : 0ull;
+    for (int e = 0; e < N; ++e) {
+      const unsigned bits = __ballot_sync(0xffffffffu, (m >> e) & 1ull);
+      if (lane == 0) tokbits[warp * kMaxN + e] = bits;
     }
-    a.counts_blk[(size_t)e * a.nblk + b] = cnt;
-    if (cnt) atomicAdd(a.tot + e, cnt);
   }
-  if (tid <= N) {
-    const int col = (tid < N) ? tid : NPAD;
+  if (tid >= 64 && tid <= 64 + N) {  // probability sums of the block, one column per thread
+    const int i = tid - 64;
+    const int col = (i < N) ? i : NPAD;
     float s = 0.f;
     for (int t = 0; t < nvalid; ++t) s += p_s[t * LS + col];
-    a.ppart[(size_t)b * (N + 1) + tid] = s;
+    a.ppart[(size_t)b * (N + 1) + i] = s;
   }
-  __syncthreads();
-  if (tid <= K) {
+  if (tid >= 160 && tid <= 160 + K) {
+    const int c = tid - 160;
     int cnt = 0;
-    for (int t = 0; t < nvalid; ++t) cnt += (nul[t] == tid);
-    a.hist[(size_t)b * (K + 1) + tid] = cnt;
+    for (int t = 0; t < nvalid; ++t) cnt += (nul[t] == c);
+    a.hist[(size_t)b * (K + 1) + c] = cnt;
   }
-  if (tid == 32) {
+  if (tid == 192) {
     float s = 0.f;
     for (int t = 0; t < nvalid; ++t) s += lse2[t];
     a.lsq[b] = s;
+  }
+  __syncthreads();
+  if (tid < N) {
+    const int cnt = __popc(tokbits[tid]) + __popc(tokbits[kMaxN + tid]);
+    a.counts_blk[(size_t)tid * a.nblk + b] = cnt;
+    if (cnt) atomicAdd(a.tot + tid, cnt);
   }
   if (tid < nvalid * 4) {
     // lrank for (token, slot): 4 threads per token, slots k = q, q+4, ...
     const int t = tid >> 2, q = tid & 3;
     const int tok = tok0 + t;
+    const int w = t >> 5;
+    const unsigned below = (1u << (t & 31)) - 1u;
     for (int k = q; k < K; k += 4) {
       const int id = tk[t * kMaxK + k];
-      a.lrank[(size_t)tok * K + k] = (id < N) ? (int)rtab[t * NPAD + id] : -1;
+      int rank = -1;
+      if (id < N) rank = __popc(tokbits[w * kMaxN + id] & below) + (w ? __popc(tokbits[id]) : 0);
+      a.lrank[(size_t)tok * K + k] = rank;
     }
   }
 }
@@ -461,19 +529,19 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
   }
 }
 
-template <int RPT>
+template <int LG>
 static int launch_route_t(const RouteArgs& a, cudaStream_t st) {
-  using SM = RouteSmem<16 * RPT>;
+  using SM = RouteGeo<LG>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<LG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM::bytes);
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
   }
-  route_kernel<RPT><<<a.nblk, kRouteThreads, SM::bytes, st>>>(a);
+  route_kernel<LG><<<a.nblk, kRouteThreads, SM::bytes, st>>>(a);
   return cuda_status(cudaGetLastError());
 }
 
@@ -510,9 +578,10 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   cudaError_t e = cudaMemsetAsync(a.hdr, 0, kHdrTotOffset + sizeof(int32_t) * d.N, st);
   if (e != cudaSuccess) return cuda_status(e);
   int r;
-  if (d.N <= 16) r = launch_route_t<1>(a, st);
-  else if (d.N <= 32) r = launch_route_t<2>(a, st);
-  else r = launch_route_t<4>(a, st);
+  if (d.N <= 8) r = launch_route_t<1>(a, st);
+  else if (d.N <= 16) r = launch_route_t<2>(a, st);
+  else if (d.N <= 32) r = launch_route_t<4>(a, st);
+  else r = launch_route_t<8>(a, st);
   if (r != MOE_OK) return r;
   ScanArgs sa{};
   sa.counts_blk = a.counts_blk;
