@@ -48,7 +48,6 @@ struct RouteArgs {
   int T, d, N, M, K, nblk;
 };
 
-constexpr int kXS = kRouteBK + 4;  // padded fp32 row stride of staged tiles
 
 // Thread tile of the router product: 8 tokens x 8 reals. Shared memory, not
 // the FMA pipe, bounds an fp32 CUDA-core GEMM: an a x b register tile loads
