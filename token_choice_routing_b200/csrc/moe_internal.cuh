@@ -45,6 +45,7 @@ struct WsLayout {
   size_t sums;       // double [aux sums count]
   int nparts;        // first-level aux partials = min(kAuxParts, nblk)
   size_t auxp;       // double [nparts][aux_part_cols]
+  size_t wt;         // float [d][route_npad(N) + 4]: W_r transposed for the route kernel
   size_t total;
 };
 
@@ -54,6 +55,9 @@ constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // contiguous slice of route blocks in fp64: [sum p (N+1) | null hist (K+1) | sum lse^2].
 constexpr int kAuxParts = 64;
 inline int aux_part_cols(const moe_dims_t& d) { return (d.N + 1) + (d.K + 1) + 1; }
+
+// Real-logit count the route kernel pads N to (8, 16, 32 or 64).
+inline int route_npad(int N) { return N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : 64; }
 
 inline size_t aux_sums_count(const moe_dims_t& d) {
   return (size_t)d.N + (size_t)(d.K + 1) + (size_t)(d.N + 1) + 2;
@@ -75,6 +79,7 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   L.sums = o; o = align_up(o + sizeof(double) * aux_sums_count(d), 256);
   L.nparts = L.nblk < kAuxParts ? L.nblk : kAuxParts;
   L.auxp = o; o = align_up(o + sizeof(double) * (size_t)L.nparts * aux_part_cols(d), 256);
+  L.wt = o; o = align_up(o + sizeof(float) * (size_t)d.d * (route_npad(d.N) + 4), 256);
   L.total = o;
   return L;
 }

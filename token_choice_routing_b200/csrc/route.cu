@@ -28,6 +28,7 @@ namespace moe {
 struct RouteArgs {
   const uint16_t* x;
   const float* w;     // [N+1, d]
+  const float* wt;    // [d][NPAD+4] W^T of this call (workspace)
   const float* bias;  // [N+1] or null
   const float* tnb;   // [T] or null
   float* logits;      // [T, N+1] or null
@@ -67,14 +68,13 @@ struct RouteGeo {
   static constexpr int S = kRouteThreads / (TG * LG); // d-slices per staged tile
   static constexpr int KS = kRouteBK / S;             // d-columns per slice per tile (= LG)
   static_assert(S * KS == kRouteBK, "slices must tile the staged d-range");
-  static constexpr int WT = NPAD + 4;                 // row stride of the staged W^T tile (null at NPAD)
-  static constexpr int WCH = (NPAD + 1) * (kRouteBK / 8);  // 8-float chunks of a W tile
+  static constexpr int WT = NPAD + 4;                 // row stride of W^T (null at column NPAD)
+  static constexpr int WCH = kRouteBK * WT / 4;       // 16-byte chunks of a staged W^T tile
   static constexpr int WPT = (WCH + kRouteThreads - 1) / kRouteThreads;  // chunks per thread
   static constexpr int LS = NPAD + 1;                 // odd row stride
-  // per-thread cp.async landing slot: 16 B of x (8 bf16) then WPT 8-float W chunks
-  static constexpr int LAND = WPT * 8 + 4;
+  // x^T: 2 stages; W^T: 3 stages (loaded two tiles ahead); x landing: 2 slots of 16 B per thread
   static constexpr size_t main_bytes =
-      sizeof(float) * (2 * kRouteBK * (kXT + WT) + 2 * (size_t)kRouteThreads * LAND);
+      sizeof(float) * (2 * kRouteBK * kXT + 3 * kRouteBK * WT + 2 * (size_t)kRouteThreads * 4);
   // slice partial sums [S][64][NPAD+1] alias the main-loop buffers
   static constexpr size_t red_bytes = sizeof(float) * S * kRouteTokens * (NPAD + 1);
   static constexpr size_t regionB = align_up(main_bytes > red_bytes ? main_bytes : red_bytes, 16);
@@ -109,6 +109,28 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return va > vb || (va == vb && ia < ib);
 }
 
+// W^T for one call: wt[k][j] = W_r[j][k] for real j < N, wt[k][NPAD] = W_r[N][k]
+// (the null row), zero for the padding columns; row stride NPAD + 4. One CTA
+// per 32 d-columns, through a shared tile so both sides are coalesced.
+template <int LG>
+__global__ void __launch_bounds__(256) router_transpose_kernel(const float* __restrict__ w, float* __restrict__ wt,
+                                                               int N, int d) {
+  using G = RouteGeo<LG>;
+  constexpr int NPAD = G::NPAD, WT = G::WT;
+  __shared__ float tile[NPAD + 1][33];
+  const int k0 = blockIdx.x * 32;
+  for (int i = threadIdx.x; i < (NPAD + 1) * 32; i += blockDim.x) {
+    const int r = i >> 5, kk = i & 31;
+    const int src = (r < N) ? r : (r == NPAD ? N : -1);
+    tile[r][kk] = (src >= 0) ? w[(size_t)src * d + k0 + kk] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 32 * WT; i += blockDim.x) {
+    const int kk = i / WT, j = i - kk * WT;
+    wt[(size_t)(k0 + kk) * WT + j] = (j <= NPAD) ? tile[j][kk] : 0.f;
+  }
+}
+
 // One CTA: 64 tokens x all N+1 logits, 256 threads. Main loop: thread
 // (s, lg, tg) owns tokens {4tg..4tg+3, 32+4tg..32+4tg+3} and reals
 // {4lg..4lg+3, 4LG+4lg..4LG+4lg+3} over the d-columns [s*KS, (s+1)*KS) of
@@ -121,7 +143,6 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
   constexpr int NQ = NPAD / 4;  // reals per epilogue thread
   extern __shared__ __align__(16) unsigned char smem[];
   float* xsT = reinterpret_cast<float*>(smem);       // [2][BK][kXT]
-  float* wsT = xsT + 2 * kRouteBK * kXT;             // [2][BK][WT]
 
   const int tid = threadIdx.x;
   const int tg = tid % G::TG;
@@ -134,74 +155,61 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
   const int nkt = d / kRouteBK;
 
   float acc[kTileT][kTileR];
-  float accn = 0.f;  // null logit of token tid & 63 over d-columns (tid >> 6) * 8 .. +8 of each tile
 #pragma unroll
   for (int i = 0; i < kTileT; ++i)
 #pragma unroll
     for (int j = 0; j < kTileR; ++j) acc[i][j] = 0.f;
 
-  // Staging, two tiles ahead: every thread copies its own pieces of tile kt+2
-  // by cp.async into its own landing slot (x: token tid & 63, 8 d-columns from
-  // (tid >> 6) * 8; W: chunk c = tid + 256 q -> row c % (NPAD+1), 8 d-columns
-  // from (c / (NPAD+1)) * 8) while tile kt is multiplied; after its own wait it
-  // writes tile kt+1 transposed into the free stage buffer. No registers are
-  // held across the multiply and no extra barrier is needed.
+  // Staging, two tiles ahead. W^T tile kt+2 is copied by cp.async straight
+  // into its slot of a 3-deep ring (rows of NPAD+4 floats, already transposed
+  // by router_transpose_kernel). x: thread copies token tid & 63, 8 d-columns
+  // from (tid >> 6) * 8, into its own landing slot; after its own wait it
+  // widens them into the x^T stage of tile kt+1 and adds their share of the
+  // null logit (null weights from global, cached). No registers are held
+  // across the multiply.
+  float* wsT = xsT + 2 * kRouteBK * kXT;                       // [3][BK][WT]
+  float* land0 = wsT + 3 * kRouteBK * WT;                      // [2][256][4]
   const int xrow = tid & 63, xkc = (tid >> 6) * 8;
   const bool xok = tok0 + xrow < T;
   const uint16_t* xsrc = a.x + (size_t)(tok0 + (xok ? xrow : 0)) * d + xkc;
-  float* land0 = wsT + 2 * kRouteBK * WT + tid * G::LAND;
-  auto land = [&](int slot) { return land0 + slot * kRouteThreads * G::LAND; };
-  auto load_tiles = [&](int kt, int slot) {
+  const float* wnull = a.w + (size_t)N * d + xkc;
+  float accn = 0.f;  // null logit of token xrow over its staged columns
+  auto load_tiles = [&](int kt) {
     if (kt < nkt) {
-      float* L = land(slot);
-      cp_async16(smem_u32(L), xsrc + (size_t)kt * kRouteBK, xok ? 16 : 0);
+      cp_async16(smem_u32(land0 + ((kt & 1) * kRouteThreads + tid) * 4), xsrc + (size_t)kt * kRouteBK, xok ? 16 : 0);
+      float* wb = wsT + (kt % 3) * kRouteBK * WT;
+      const float* src = a.wt + (size_t)kt * kRouteBK * WT;
 #pragma unroll
       for (int q = 0; q < G::WPT; ++q) {
         const int c = tid + kRouteThreads * q;
-        if (c < G::WCH) {
-          const int r = c % (NPAD + 1), kc = (c / (NPAD + 1)) * 8;
-          const int src_row = (r < N) ? r : (r == NPAD ? N : -1);
-          const float* src = a.w + (size_t)(src_row < 0 ? 0 : src_row) * d + (size_t)kt * kRouteBK + kc;
-          cp_async16(smem_u32(L + 4 + q * 8), src, src_row < 0 ? 0 : 16);
-          cp_async16(smem_u32(L + 8 + q * 8), src + 4, src_row < 0 ? 0 : 16);
-        }
+        if (c < G::WCH) cp_async16(smem_u32(wb + 4 * c), src + 4 * c, 16);
       }
     }
     cp_async_commit();  // one group per call, possibly empty
   };
-  auto store_tiles = [&](int buf, int slot) {
-    const float* L = land(slot);
-    const uint4 xr = *reinterpret_cast<const uint4*>(L);
-    float* xb = xsT + buf * kRouteBK * kXT;
+  auto store_x = [&](int kt) {
+    const uint4 xr = *reinterpret_cast<const uint4*>(land0 + ((kt & 1) * kRouteThreads + tid) * 4);
+    float* xb = xsT + (kt & 1) * kRouteBK * kXT;
     const float xv[8] = {bf16lo(xr.x), bf16hi(xr.x), bf16lo(xr.y), bf16hi(xr.y),
                          bf16lo(xr.z), bf16hi(xr.z), bf16lo(xr.w), bf16hi(xr.w)};
 #pragma unroll
     for (int u = 0; u < 8; ++u) xb[(xkc + u) * kXT + xrow] = xv[u];
-    float* wb = wsT + buf * kRouteBK * WT;
+    const float4 w0 = __ldg(reinterpret_cast<const float4*>(wnull + (size_t)kt * kRouteBK));
+    const float4 w1 = __ldg(reinterpret_cast<const float4*>(wnull + (size_t)kt * kRouteBK + 4));
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int q = 0; q < G::WPT; ++q) {
-      const int c = tid + kRouteThreads * q;
-      if (c < G::WCH) {
-        const int r = c % (NPAD + 1), kc = (c / (NPAD + 1)) * 8;
-        const float4 w0 = *reinterpret_cast<const float4*>(L + 4 + q * 8);
-        const float4 w1 = *reinterpret_cast<const float4*>(L + 8 + q * 8);
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int u = 0; u < 8; ++u) wb[(kc + u) * WT + r] = wv[u];
-      }
-    }
+    for (int u = 0; u < 8; ++u) accn = fmaf(xv[u], wv[u], accn);
   };
 
-  load_tiles(0, 0);
-  load_tiles(1, 1);
+  load_tiles(0);
+  load_tiles(1);
   cp_async_wait_group1();  // this thread's copies of tile 0
-  store_tiles(0, 0);
+  store_x(0);
   for (int kt = 0; kt < nkt; ++kt) {
-    const int buf = kt & 1;
     __syncthreads();
-    load_tiles(kt + 2, buf);  // slot `buf` held tile kt, already written out
-    const float* xb = xsT + buf * kRouteBK * kXT + (sl * KS) * kXT;
-    const float* wb = wsT + buf * kRouteBK * WT + (sl * KS) * WT;
+    load_tiles(kt + 2);  // its W^T slot was last read at iteration kt-1; its x slot was written out
+    const float* xb = xsT + (kt & 1) * kRouteBK * kXT + (sl * KS) * kXT;
+    const float* wb = wsT + (kt % 3) * kRouteBK * WT + (sl * KS) * WT;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       const float4 xa = *reinterpret_cast<const float4*>(xb + kk * kXT + 4 * tg);
@@ -215,17 +223,12 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
 #pragma unroll
         for (int jj = 0; jj < kTileR; ++jj) acc[i][jj] = fmaf(xv[i], wv[jj], acc[i][jj]);
     }
-    {  // the null logit: token xrow over the 8 d-columns this thread stages
-      const float* xn = xsT + buf * kRouteBK * kXT + xkc * kXT + xrow;
-      const float* wn = wsT + buf * kRouteBK * WT + xkc * WT + NPAD;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) accn = fmaf(xn[u * kXT], wn[u * WT], accn);
-    }
     if (kt + 1 < nkt) {
-      cp_async_wait_group1();    // this thread's copies of tile kt+1 (tile kt+2 may be in flight)
-      store_tiles(buf ^ 1, buf ^ 1);  // that stage buffer was last read before this iteration's barrier
+      cp_async_wait_group1();  // this thread's copies of tile kt+1 (tile kt+2 may be in flight)
+      store_x(kt + 1);         // x^T stage (kt+1)&1 was last read before this iteration's barrier
     }
   }
+  cp_async_wait_all();
   __syncthreads();  // main-loop buffers are reused below
 
   float* red = reinterpret_cast<float*>(smem);  // [S][64][NPAD+1]
@@ -531,6 +534,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
 template <int LG>
 static int launch_route_t(const RouteArgs& a, cudaStream_t st) {
   using SM = RouteGeo<LG>;
+  router_transpose_kernel<LG><<<a.d / 32, 256, 0, st>>>(a.w, const_cast<float*>(a.wt), a.N, a.d);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -558,6 +562,7 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.topk_gate = topk_gate;
   a.n_real = n_real;
   a.hdr = ws_ptr<uint32_t>(ws, L.hdr);
+  a.wt = ws_ptr<float>(ws, L.wt);
   a.tot = ws_ptr<int32_t>(ws, L.hdr + kHdrTotOffset);
   a.counts_blk = ws_ptr<int32_t>(ws, L.counts_blk);
   a.bases = ws_ptr<int32_t>(ws, L.bases);
