@@ -10,39 +10,52 @@ namespace moe {
 
 constexpr int kCombineThreads = 256;
 
-__global__ void __launch_bounds__(kCombineThreads)
+// One warp per token, two 16-byte chunks per lane per pass. In each pass the
+// shared row's chunks and the chunks of the first four slots are loaded
+// together before any is used (null slots load nothing); the next token's slot
+// list is fetched while this one is combined. Sum order: shared, then slots in
+// rank order.
+__global__ void __launch_bounds__(kCombineThreads, 3)
 combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
                const float* __restrict__ gate, const int32_t* __restrict__ slot_row,
                uint16_t* __restrict__ y, int T, int d, int K, long long rcap, uint32_t* status) {
   const int lane = threadIdx.x & 31;
   const int wpb = kCombineThreads / 32;
   const int nch = d >> 3;
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
-    int row = -1;
-    float g = 0.f;
-    if (lane < K) {
-      row = __ldg(slot_row + (size_t)t * K + lane);
-      g = __ldg(gate + (size_t)t * K + lane);
+  const int stride = gridDim.x * wpb;
+  int t = blockIdx.x * wpb + (threadIdx.x >> 5);
+  auto load_slot = [&](int tt, int& row, float& g) {
+    row = -1;
+    g = 0.f;
+    if (tt < T && lane < K) {
+      row = __ldg(slot_row + (size_t)tt * K + lane);
+      g = __ldg(gate + (size_t)tt * K + lane);
       if (row >= rcap) {
         if (status) atomicOr(status, kStatusBounds);
         row = -1;
       }
     }
-    for (int c0 = 0; c0 < nch; c0 += 64) {  // two 16-byte chunks per lane per pass
-      float acc[2][8];
-      bool ok[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int c = c0 + 32 * h + lane;
-        ok[h] = c < nch;
-        const uint4 v = ok[h] ? __ldg(reinterpret_cast<const uint4*>(sh + (size_t)t * d) + c)
-                              : make_uint4(0u, 0u, 0u, 0u);
-        acc[h][0] = bf16lo(v.x); acc[h][1] = bf16hi(v.x); acc[h][2] = bf16lo(v.y); acc[h][3] = bf16hi(v.y);
-        acc[h][4] = bf16lo(v.z); acc[h][5] = bf16hi(v.z); acc[h][6] = bf16lo(v.w); acc[h][7] = bf16hi(v.w);
-      }
-      // slots in rank order, four at a time: issue the real rows' loads before using any
+  };
+  auto fma8 = [](float (&a)[8], float gk, const uint4& v) {
+    a[0] = fmaf(gk, bf16lo(v.x), a[0]); a[1] = fmaf(gk, bf16hi(v.x), a[1]);
+    a[2] = fmaf(gk, bf16lo(v.y), a[2]); a[3] = fmaf(gk, bf16hi(v.y), a[3]);
+    a[4] = fmaf(gk, bf16lo(v.z), a[4]); a[5] = fmaf(gk, bf16hi(v.z), a[5]);
+    a[6] = fmaf(gk, bf16lo(v.w), a[6]); a[7] = fmaf(gk, bf16hi(v.w), a[7]);
+  };
+  int row, rown;
+  float g, gn;
+  load_slot(t, row, g);
+  for (; t < T; t += stride) {
+    load_slot(t + stride, rown, gn);  // next token's slots, in flight during this one
+    for (int c0 = 0; c0 < nch; c0 += 64) {
+      const int ca = c0 + lane, cb = c0 + 32 + lane;
+      const bool oka = ca < nch, okb = cb < nch;
+      const uint4* shr = reinterpret_cast<const uint4*>(sh + (size_t)t * d);
+      const uint4 sa = oka ? __ldg(shr + ca) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 sb = okb ? __ldg(shr + cb) : make_uint4(0u, 0u, 0u, 0u);
+      float acc_a[8], acc_b[8];
       for (int k0 = 0; k0 < K; k0 += 4) {
-        uint4 v[4][2];
+        uint4 va[4], vb[4];
         float gq[4];
         int rq[4];
 #pragma unroll
@@ -51,38 +64,35 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
           rq[u] = __shfl_sync(0xffffffffu, row, k & 31);
           gq[u] = __shfl_sync(0xffffffffu, g, k & 31);
           if (k >= K) rq[u] = -1;
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            v[u][h] = (rq[u] >= 0 && ok[h])
-                          ? __ldg(reinterpret_cast<const uint4*>(ys + (size_t)rq[u] * d) + c0 + 32 * h + lane)
-                          : make_uint4(0u, 0u, 0u, 0u);
+          const uint4* src = reinterpret_cast<const uint4*>(ys + (size_t)(rq[u] < 0 ? 0 : rq[u]) * d);
+          va[u] = (rq[u] >= 0 && oka) ? __ldg(src + ca) : make_uint4(0u, 0u, 0u, 0u);
+          vb[u] = (rq[u] >= 0 && okb) ? __ldg(src + cb) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (k0 == 0) {
+          acc_a[0] = bf16lo(sa.x); acc_a[1] = bf16hi(sa.x); acc_a[2] = bf16lo(sa.y); acc_a[3] = bf16hi(sa.y);
+          acc_a[4] = bf16lo(sa.z); acc_a[5] = bf16hi(sa.z); acc_a[6] = bf16lo(sa.w); acc_a[7] = bf16hi(sa.w);
+          acc_b[0] = bf16lo(sb.x); acc_b[1] = bf16hi(sb.x); acc_b[2] = bf16lo(sb.y); acc_b[3] = bf16hi(sb.y);
+          acc_b[4] = bf16lo(sb.z); acc_b[5] = bf16hi(sb.z); acc_b[6] = bf16lo(sb.w); acc_b[7] = bf16hi(sb.w);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (rq[u] >= 0) {
-            const float gk = gq[u];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              acc[h][0] = fmaf(gk, bf16lo(v[u][h].x), acc[h][0]); acc[h][1] = fmaf(gk, bf16hi(v[u][h].x), acc[h][1]);
-              acc[h][2] = fmaf(gk, bf16lo(v[u][h].y), acc[h][2]); acc[h][3] = fmaf(gk, bf16hi(v[u][h].y), acc[h][3]);
-              acc[h][4] = fmaf(gk, bf16lo(v[u][h].z), acc[h][4]); acc[h][5] = fmaf(gk, bf16hi(v[u][h].z), acc[h][5]);
-              acc[h][6] = fmaf(gk, bf16lo(v[u][h].w), acc[h][6]); acc[h][7] = fmaf(gk, bf16hi(v[u][h].w), acc[h][7]);
-            }
+            fma8(acc_a, gq[u], va[u]);
+            fma8(acc_b, gq[u], vb[u]);
           }
         }
       }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (ok[h]) {
-          uint4 o;
-          o.x = pack_bf16x2(acc[h][0], acc[h][1]);
-          o.y = pack_bf16x2(acc[h][2], acc[h][3]);
-          o.z = pack_bf16x2(acc[h][4], acc[h][5]);
-          o.w = pack_bf16x2(acc[h][6], acc[h][7]);
-          reinterpret_cast<uint4*>(y + (size_t)t * d)[c0 + 32 * h + lane] = o;
-        }
-      }
+      if (oka)
+        reinterpret_cast<uint4*>(y + (size_t)t * d)[ca] =
+            make_uint4(pack_bf16x2(acc_a[0], acc_a[1]), pack_bf16x2(acc_a[2], acc_a[3]),
+                       pack_bf16x2(acc_a[4], acc_a[5]), pack_bf16x2(acc_a[6], acc_a[7]));
+      if (okb)
+        reinterpret_cast<uint4*>(y + (size_t)t * d)[cb] =
+            make_uint4(pack_bf16x2(acc_b[0], acc_b[1]), pack_bf16x2(acc_b[2], acc_b[3]),
+                       pack_bf16x2(acc_b[4], acc_b[5]), pack_bf16x2(acc_b[6], acc_b[7]));
     }
+    row = rown;
+    g = gn;
   }
 }
 
