@@ -326,7 +326,8 @@ def main():
     breakdown["gate_up"]["frac"] = breakdown["gate_up"]["TFLOP/s"] / bf16_peak
     breakdown["down"]["frac"] = breakdown["down"]["TFLOP/s"] / bf16_peak
     ffn_ms = kms["gate_up"] + kms["down"]
-    routed_tflops = 6.0 * d * F * R / (ffn_ms * 1e9)
+    # FFN FLOP/s over real rows only: routed (token, expert) slots plus the shared expert's T rows
+    ffn_tflops = (6.0 * d * F * R + 6.0 * d * Fs * T) / (ffn_ms * 1e9)
 
     achieved = breakdown["gate_up"]["TFLOP/s"]
     roofline = {"kernel": "grouped gate/up SwiGLU GEMM (tcgen05)", "bound": "tensor", "achieved": achieved,
@@ -378,7 +379,7 @@ def main():
             "data": "synthetic (seeded N(0,1) bf16 tokens, N(0,1/fan_in) bf16 weights, fp32 router)",
             "config": workload_config(cfg, args),
             "real_slots_per_step": R, "tokens_per_s": world * T * args.steps / (total_ms * 1e-3),
-            "routed_ffn_tflops_real_rows": routed_tflops,
+            "ffn_tflops_real_rows": ffn_tflops, "ffn_frac_of_bf16_peak": ffn_tflops / bf16_peak,
             "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk.summary(),
