@@ -185,6 +185,7 @@ def workload_config(cfg, args):
                         f"F_shared={cfg.F_shared} K={cfg.K} M={cfg.M} rho={cfg.rho:.3g}",
             "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "K": cfg.K, "F": cfg.F, "F_shared": cfg.F_shared,
             "global_batch_tokens": cfg.T * args.gpus, "parallelism": f"dp{args.gpus}",
+            "router": getattr(args, "router", "tensor"),
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
@@ -198,6 +199,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="qwen3_0p6b")
+    ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"],
+                    help="router product on the tensor cores (default) or the fp32 CUDA cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")
@@ -225,7 +228,7 @@ def main():
 
     cfg = I.CONFIGS[args.config]
     inp = I.make_inputs(cfg)
-    layer = MoENullLayer.from_inputs(inp, dev)
+    layer = MoENullLayer.from_inputs(inp, dev, router=args.router)
     x = bf16_tensor(inp.x, dev)
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
     T = cfg.T
@@ -313,7 +316,8 @@ def main():
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     fp32_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
     breakdown = {
-        "route": {"ms": kms["route"], "bound": "alu", "TFLOP/s": 2.0 * (N + 1) * d * T / (kms["route"] * 1e9),
+        "route": {"ms": kms["route"], "bound": "alu" if args.router == "fp32_cores" else "hbm",
+                  "TFLOP/s": 2.0 * (N + 1) * d * T / (kms["route"] * 1e9),
                   "GB/s": bytes_route / (kms["route"] * 1e6)},
         "dispatch": {"ms": kms["dispatch"], "bound": "hbm", "GB/s": bytes_dispatch / (kms["dispatch"] * 1e6)},
         "gate_up": {"ms": kms["gate_up"], "bound": "tensor", "TFLOP/s": flops_gu / (kms["gate_up"] * 1e9)},
@@ -321,6 +325,7 @@ def main():
         "combine": {"ms": kms["combine"], "bound": "hbm", "GB/s": bytes_combine / (kms["combine"] * 1e6)},
     }
     breakdown["route"]["frac_fp32_alu"] = breakdown["route"]["TFLOP/s"] / fp32_peak
+    breakdown["route"]["frac_hbm"] = breakdown["route"]["GB/s"] / hbm_peak
     breakdown["dispatch"]["frac"] = breakdown["dispatch"]["GB/s"] / hbm_peak
     breakdown["combine"]["frac"] = breakdown["combine"]["GB/s"] / hbm_peak
     breakdown["gate_up"]["frac"] = breakdown["gate_up"]["TFLOP/s"] / bf16_peak

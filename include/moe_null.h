@@ -70,7 +70,14 @@ typedef enum {
 } moe_status_t;
 
 /* Layer sizes. T tokens, model width d, N real experts, M null copies, top-K,
- * routed expert ffn width F, shared expert ffn width F_shared. flags: 0. */
+ * routed expert ffn width F, shared expert ffn width F_shared. flags: 0 or
+ * MOE_FLAG_ROUTER_FP32_CORES. Every call of one layer (route, dispatch,
+ * workspace sizing, ...) must see the same flags. */
+/* Router product on the fp32 CUDA cores instead of the tensor cores (see
+ * moe_route). Both give logits within the fp32 dot-product error bound; this
+ * path is several times slower on the router product. */
+#define MOE_FLAG_ROUTER_FP32_CORES 1u
+
 typedef struct moe_dims {
   int32_t T, d, N, M, K, F, F_shared;
   uint32_t flags;
@@ -135,7 +142,12 @@ MOE_API int moe_pack_gate_up(const moe_dims_t* dims, const uint16_t* w_gate, con
 
 /* Routing (section 三: Null Expert 机制, 阈值解释, 负载均衡损失, Z-Loss).
  *  s[t, j] = sum_c fp32(x[t,c]) * w_router[j,c] + bias[j] (+ tok_null_bias[t]
- *  for j = N), computed in fp32 on CUDA cores. Over the pool [s_0..s_{N-1},
+ *  for j = N), to fp32 accuracy: by default on the tensor cores, with each
+ *  fp32 weight split exactly into three bf16 terms (hi + mid + lo; bf16
+ *  products are exact, accumulation is fp32, the three partial sums are added
+ *  in fp32), or, with MOE_FLAG_ROUTER_FP32_CORES, as an fp32 FMA product on the
+ *  CUDA cores. x and w_router must be 16-byte aligned (x is read by TMA).
+ *  Over the pool [s_0..s_{N-1},
  *  s_N x M]: lse_t, p_{t,i}; top-K in (value desc, index asc) order -- a real
  *  logit equal to the null logit precedes every copy, copies fill N, N+1, ...;
  *  gates = softmax over the selected real logits (0 for nulls, all 0 if none).

@@ -29,17 +29,21 @@ def bf16_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().float().numpy().astype(np.float64)
 
 
-def make_layer(inp, device="cuda"):
+# Both router paths of the library: tensor cores (default) and fp32 CUDA cores.
+ROUTERS = ("tensor", "fp32_cores")
+
+
+def make_layer(inp, device="cuda", router="tensor"):
     from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
-    layer = MoENullLayer.from_inputs(inp, device)
+    layer = MoENullLayer.from_inputs(inp, device, router=router)
     x = bf16_tensor(inp.x, device)
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(device)
     return layer, x, tnb
 
 
-def run_forward(inp, device="cuda"):
+def run_forward(inp, device="cuda", router="tensor"):
     from token_choice_routing_b200 import binding as B
-    layer, x, tnb = make_layer(inp, device)
+    layer, x, tnb = make_layer(inp, device, router)
     out = layer.forward(x, tnb)
     torch.cuda.synchronize()
     st = B.get_device_status(out["workspace"])

@@ -64,8 +64,27 @@ def test_check_dims(lib):
         v.update(kw)
         assert B.check_dims(B.dims(**v)) == B.ERR_UNSUPPORTED, kw
     dm = good()
-    dm.flags = 1
-    assert B.check_dims(dm) == B.ERR_INVALID_ARG
+    dm.flags = B.FLAG_ROUTER_FP32_CORES
+    assert B.check_dims(dm) == B.OK
+    for f in (2, 4, 0x80000000, B.FLAG_ROUTER_FP32_CORES | 2):
+        dm.flags = f
+        assert B.check_dims(dm) == B.ERR_INVALID_ARG, f
+
+
+def test_workspace_depends_on_router_path(lib):
+    """The fp32 CUDA-core route keeps per-block statistics over 64-token blocks
+    and a transposed fp32 W_r; the tensor-core route over 128-token blocks and
+    a bf16 three-term split of W_r. Both layouts are sized by the library."""
+    B = lib
+    for T, d, N, K in ((1, 128, 1, 1), (16384, 1024, 64, 4), (131072, 2048, 64, 8), (777, 256, 15, 3)):
+        tc = B.workspace_bytes(B.dims(T, d, N, 64, K, 64, 64))
+        fp = B.workspace_bytes(B.dims(T, d, N, 64, K, 64, 64, B.FLAG_ROUTER_FP32_CORES))
+        assert tc > 0 and fp > 0 and tc % 256 == 0 and fp % 256 == 0
+        npw = (N + 1 + 15) // 16 * 16
+        npad = 8 if N <= 8 else 16 if N <= 16 else 32 if N <= 32 else 64
+        # the weight buffers alone differ by exactly this much (both 256-aligned regions)
+        al = lambda v: (v + 255) // 256 * 256
+        assert tc - al(2 * 3 * npw * d) >= 0 and fp - al(4 * d * (npad + 4)) >= 0
 
 
 def test_workspace_and_sizes(lib):

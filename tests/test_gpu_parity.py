@@ -30,13 +30,14 @@ SMALL = {
 }
 
 
+@pytest.mark.parametrize("router", H.ROUTERS)
 @pytest.mark.parametrize("name", list(SMALL))
-def test_small_layer_full_parity(name):
+def test_small_layer_full_parity(name, router):
     cfg = SMALL[name]
     inp = I.make_inputs(cfg)
     if cfg.name.startswith("ragged") or cfg.name in ("k1", "n64_k16", "t1"):
         inp.bias[cfg.N] = np.float32(0.3)
-    layer, x, tnb, out = H.run_forward(inp)
+    layer, x, tnb, out = H.run_forward(inp, router=router)
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -64,11 +65,12 @@ def test_small_layer_full_parity(name):
     H.check_layer_output(inp, out, r)
 
 
-@pytest.mark.parametrize("name", ["qwen3_0p6b", "qwen3_1p7b"])
-def test_full_size_layer_parity_sampled(name):
+@pytest.mark.parametrize("name,router", [("qwen3_0p6b", "tensor"), ("qwen3_1p7b", "tensor"),
+                                         ("qwen3_0p6b", "fp32_cores")])
+def test_full_size_layer_parity_sampled(name, router):
     cfg = I.CONFIGS[name]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, out = H.run_forward(inp)
+    layer, x, tnb, out = H.run_forward(inp, router=router)
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -106,7 +108,51 @@ def test_all_null_tokens_get_only_the_shared_expert():
     H.check_layer_output(inp, out, r)
 
 
-def test_exact_ties_break_by_index():
+@pytest.mark.parametrize("router", H.ROUTERS)
+@pytest.mark.parametrize("N", [8, 15, 64])
+def test_one_hot_tokens_read_back_router_weights_exactly(N, router):
+    """x_t = 2^k e_{c_t} gives s_tj = 2^k W_r[j, c_t] exactly: a single exact
+    product per logit. On the tensor-core path this holds only if the three
+    bf16 terms of every fp32 weight add back to it exactly and each term's
+    product lands in the right output column (hi, mid and lo side by side)."""
+    T, d = 300, 256
+    cfg = I.small_config("onehot", T=T, d=d, N=N, F=64, F_shared=64, K=2, M=4, config_id=913)
+    inp = I.make_inputs(cfg)
+    rng = np.random.default_rng(913)
+    c = rng.integers(0, d, size=T)
+    k = rng.integers(-3, 4, size=T)
+    x = np.zeros((T, d), dtype=np.float32)
+    x[np.arange(T), c] = np.ldexp(1.0, k)
+    inp.x = I.bf16_round(x)
+    # weights spanning many binades, with all 24 significant bits in use
+    w = (rng.standard_normal((N + 1, d)) * np.exp2(rng.integers(-20, 4, size=(N + 1, d)))).astype(np.float32)
+    inp.w_router = w
+    inp.bias[:] = 0
+    layer, xt, tnb, out = H.run_forward(inp, router=router)
+    lg = out["logits"].cpu().numpy()
+    want = (w[:, c].T * np.ldexp(1.0, k)[:, None]).astype(np.float32)
+    assert np.array_equal(lg, want), np.argwhere(lg != want)[:5]
+    H.check_routing(inp, out)
+
+
+def test_router_paths_agree_within_twice_the_bound():
+    """Tensor-core and fp32 CUDA-core logits on the same full-size inputs: each
+    is within the fp32 dot-product bound of the exact value, so they differ by
+    at most twice that bound; both route exactly as the oracle does on them."""
+    inp = I.make_inputs(I.CONFIGS["qwen3_0p6b"])
+    outs = {}
+    for router in H.ROUTERS:
+        layer, x, tnb, out = H.run_forward(inp, router=router)
+        H.check_routing(inp, out)
+        outs[router] = out["logits"].cpu().numpy().astype(np.float64)
+        del layer, out
+        torch.cuda.empty_cache()
+    diff = np.abs(outs["tensor"] - outs["fp32_cores"])
+    assert np.all(diff <= 2 * H.logit_bound(inp))
+
+
+@pytest.mark.parametrize("router", H.ROUTERS)
+def test_exact_ties_break_by_index(router):
     # Integer-valued x and multiples of 1/8 in W_r make every router logit an
     # exact fp32 value whatever the summation order, so equal rows give equal
     # logits: many real-real ties, and the null row is a copy of real row 2, so
@@ -121,7 +167,7 @@ def test_exact_ties_break_by_index():
     w[cfg.N] = w[2]
     inp.w_router = w
     inp.bias[:] = 0
-    layer, x, tnb, out = H.run_forward(inp)
+    layer, x, tnb, out = H.run_forward(inp, router=router)
     lg = out["logits"].cpu().numpy()
     assert np.array_equal(lg, H.oracle_logits(inp).astype(np.float32))
     assert np.array_equal(lg[:, 3], lg[:, 1]) and np.array_equal(lg[:, cfg.N], lg[:, 2])
@@ -147,7 +193,8 @@ def _subset(inp, cfg, rows):
                                tok_null_bias=None if inp.tok_null_bias is None else inp.tok_null_bias[rows])
 
 
-def test_k4_half_reproduces_k2_dense_bitwise():
+@pytest.mark.parametrize("router", H.ROUTERS)
+def test_k4_half_reproduces_k2_dense_bitwise(router):
     """Solution-space preservation (review page, section 三 / 解决方案空间保持):
     with each token's null logit strictly between its 2nd and 3rd real logit,
     K=4/M=64 selects the same two reals as K=2/M=0 and gives the same y."""
@@ -165,8 +212,8 @@ def test_k4_half_reproduces_k2_dense_bitwise():
     inp4 = _subset(inp, cfg4, rows)
     inp4.tok_null_bias = (0.5 * (srt[rows, 1] + srt[rows, 2]) - s[rows, N]).astype(np.float32)
     inp2 = _subset(inp, cfg2, rows)
-    layer4, _, _, out4 = H.run_forward(inp4)
-    layer2, _, _, out2 = H.run_forward(inp2)
+    layer4, _, _, out4 = H.run_forward(inp4, router=router)
+    layer2, _, _, out2 = H.run_forward(inp2, router=router)
     assert np.all(out4["n_real"].cpu().numpy() == 2)
     H.check_routing(inp4, out4)
     H.check_routing(inp2, out2)

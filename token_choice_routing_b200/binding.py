@@ -109,8 +109,12 @@ def _check(fn: str, code: int):
         raise MoEError(fn, code)
 
 
-def dims(T, d, N, M, K, F, F_shared) -> Dims:
-    return Dims(int(T), int(d), int(N), int(M), int(K), int(F), int(F_shared), 0)
+# moe_dims_t.flags: router product on the fp32 CUDA cores instead of the tensor cores
+FLAG_ROUTER_FP32_CORES = 1
+
+
+def dims(T, d, N, M, K, F, F_shared, flags=0) -> Dims:
+    return Dims(int(T), int(d), int(N), int(M), int(K), int(F), int(F_shared), int(flags))
 
 
 def check_dims(dm: Dims) -> int:

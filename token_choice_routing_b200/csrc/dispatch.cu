@@ -118,7 +118,7 @@ struct DispatchArgs {
   float* P;
   float* losses;
   int fuse_aux;
-  int T, d, N, M, K, nblk;
+  int T, d, N, M, K, nblk, blk_tokens;
 };
 
 constexpr int kDispatchThreads = 256;
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
     if (lane < K) {
       const int id = __ldg(a.topk_idx + (size_t)t * K + lane);
       if (id >= 0 && id < N) {
-        dest = __ldg(a.bases + (size_t)id * a.nblk + t / kRouteTokens) + __ldg(a.lrank + (size_t)t * K + lane);
+        dest = __ldg(a.bases + (size_t)id * a.nblk + t / a.blk_tokens) + __ldg(a.lrank + (size_t)t * K + lane);
         if (dest < 0 || dest >= rcap) {
           atomicOr(a.status, kStatusBounds);
           dest = -1;
@@ -220,6 +220,7 @@ int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_
   a.M = d.M;
   a.K = d.K;
   a.nblk = L.nblk;
+  a.blk_tokens = L.blk_tokens;
   const int wpb = kDispatchThreads / 32;
   int grid = (d.T + wpb - 1) / wpb;
   const int cap = sm_count() * 8;

@@ -378,7 +378,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D bf16 tensor [rows, cols] (cols contiguous), box = box_rows x 64 cols, 128B swizzle.
-static bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -460,8 +460,10 @@ int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, c
   FfnPlan p = plan_ffn(d, offsets, ws);
   const long long rcap = (long long)d.T * d.K;
   CUtensorMap ar, br, as_, bs;
-  if (!(make_tmap(&ar, xs, rcap, d.d, kBM) && make_tmap(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, p.BN1) &&
-        make_tmap(&as_, x, d.T, d.d, kBM) && make_tmap(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, p.BN1)))
+  if (!(make_tmap_bf16(&ar, xs, rcap, d.d, kBM) &&
+        make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, p.BN1) &&
+        make_tmap_bf16(&as_, x, d.T, d.d, kBM) &&
+        make_tmap_bf16(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, p.BN1)))
     return MOE_ERR_CUDA;
   p.g1.out_r = h;
   p.g1.out_s = h_shared;
@@ -475,8 +477,10 @@ int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, 
   FfnPlan p = plan_ffn(d, offsets, ws);
   const long long rcap = (long long)d.T * d.K;
   CUtensorMap ar, br, as_, bs;
-  if (!(make_tmap(&ar, h, rcap, d.F, kBM) && make_tmap(&br, w_down, (uint64_t)d.N * d.d, d.F, p.BN2) &&
-        make_tmap(&as_, h_shared, d.T, d.F_shared, kBM) && make_tmap(&bs, sdown, d.d, d.F_shared, p.BN2)))
+  if (!(make_tmap_bf16(&ar, h, rcap, d.F, kBM) &&
+        make_tmap_bf16(&br, w_down, (uint64_t)d.N * d.d, d.F, p.BN2) &&
+        make_tmap_bf16(&as_, h_shared, d.T, d.F_shared, kBM) &&
+        make_tmap_bf16(&bs, sdown, d.d, d.F_shared, p.BN2)))
     return MOE_ERR_CUDA;
   p.g2.out_r = ys;
   p.g2.out_s = shared_out;

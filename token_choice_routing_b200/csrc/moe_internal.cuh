@@ -5,6 +5,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -13,10 +14,12 @@
 namespace moe {
 
 // ------------------------------------------------------------------------------------
-// Tiling constants of the route kernel (fp32 CUDA-core router GEMM + routing).
-constexpr int kRouteTokens = 64;    // tokens per route CTA
-constexpr int kRouteBK = 32;        // d-slice per pipeline stage
-constexpr int kRouteThreads = 256;  // 8 token groups x logit groups x d-slices
+// Tiling constants of the route kernel (router product on tcgen05 + routing).
+constexpr int kRouteTokens = 128;                          // tokens per route CTA (one M=128 tile)
+constexpr int kRouteBK = 64;                               // d-columns per pipeline stage
+constexpr int kRouteEpiThreads = 256;                      // 8 epilogue warps
+constexpr int kRouteThreads = 64 + kRouteEpiThreads;       // + TMA warp + MMA warp
+constexpr int kFp32RouteTokens = 64;                       // tokens per CTA of the fp32 CUDA-core route
 constexpr int kMaxN = 64;
 constexpr int kMaxK = 16;
 
@@ -32,7 +35,8 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // Workspace layout, computed identically on the host for every entry point.
 struct WsLayout {
-  int nblk;          // route CTAs = ceil(T / kRouteTokens)
+  int blk_tokens;    // tokens per route block (route_block_tokens)
+  int nblk;          // route CTAs = ceil(T / blk_tokens)
   size_t hdr;        // uint32 status at 0; int32 per-expert totals at kHdrTotOffset (512 B)
   size_t counts_blk; // int32 [N][nblk]
   size_t bases;      // int32 [N][nblk]
@@ -45,7 +49,8 @@ struct WsLayout {
   size_t sums;       // double [aux sums count]
   int nparts;        // first-level aux partials = min(kAuxParts, nblk)
   size_t auxp;       // double [nparts][aux_part_cols]
-  size_t wt;         // float [d][route_npad(N) + 4]: W_r transposed for the route kernel
+  size_t wprep;      // router weight prepared for this call: bf16 [3 * route_npw(N)][d] (three
+                     // terms hi, mid, lo) or, for the fp32 CUDA-core route, W_r^T fp32 [d][npad + 4]
   size_t total;
 };
 
@@ -56,8 +61,19 @@ constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 constexpr int kAuxParts = 64;
 inline int aux_part_cols(const moe_dims_t& d) { return (d.N + 1) + (d.K + 1) + 1; }
 
-// Real-logit count the route kernel pads N to (8, 16, 32 or 64).
-inline int route_npad(int N) { return N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : 64; }
+// Rows per bf16 term of the split router weight: the N+1 logits padded to a
+// multiple of 16 (16 .. 80), so the three terms together are one MMA of N <= 240.
+inline int route_npw(int N) { return (N + 1 + 15) / 16 * 16; }
+
+// Real-logit count the fp32 CUDA-core route pads N to (8, 16, 32 or 64).
+inline int route_fp32_npad(int N) { return N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : 64; }
+
+inline bool route_fp32_cores(const moe_dims_t& d) { return (d.flags & MOE_FLAG_ROUTER_FP32_CORES) != 0u; }
+
+// Tokens per route block: the unit of the per-block statistics and ranks.
+inline int route_block_tokens(const moe_dims_t& d) {
+  return route_fp32_cores(d) ? kFp32RouteTokens : kRouteTokens;
+}
 
 inline size_t aux_sums_count(const moe_dims_t& d) {
   return (size_t)d.N + (size_t)(d.K + 1) + (size_t)(d.N + 1) + 2;
@@ -65,7 +81,8 @@ inline size_t aux_sums_count(const moe_dims_t& d) {
 
 inline WsLayout ws_layout(const moe_dims_t& d) {
   WsLayout L{};
-  L.nblk = (d.T + kRouteTokens - 1) / kRouteTokens;
+  L.blk_tokens = route_block_tokens(d);
+  L.nblk = (d.T + L.blk_tokens - 1) / L.blk_tokens;
   size_t o = 0;
   L.hdr = o; o += 512;
   L.counts_blk = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N * L.nblk, 256);
@@ -79,7 +96,10 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   L.sums = o; o = align_up(o + sizeof(double) * aux_sums_count(d), 256);
   L.nparts = L.nblk < kAuxParts ? L.nblk : kAuxParts;
   L.auxp = o; o = align_up(o + sizeof(double) * (size_t)L.nparts * aux_part_cols(d), 256);
-  L.wt = o; o = align_up(o + sizeof(float) * (size_t)d.d * (route_npad(d.N) + 4), 256);
+  L.wprep = o;
+  o = align_up(o + (route_fp32_cores(d) ? sizeof(float) * (size_t)d.d * (route_fp32_npad(d.N) + 4)
+                                        : sizeof(uint16_t) * 3 * (size_t)route_npw(d.N) * d.d),
+               256);
   L.total = o;
   return L;
 }
@@ -96,11 +116,21 @@ int check_dims(const moe_dims_t* d);
 int sm_count();
 int cuda_status(cudaError_t e);
 
+// 2-D bf16 tensor map [rows, cols] (cols contiguous) with a box of box_rows x 64
+// columns and the 128-byte swizzle (implemented in expert_ffn.cu).
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
 // Launchers (each returns a moe_status_t after enqueuing).
 int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router,
                  const float* bias, const float* tok_null_bias, float* logits_out,
                  int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* ws,
                  cudaStream_t st);
+// The fp32 CUDA-core route (route_fp32.cu) and the per-expert scan both routes end with.
+int launch_route_fp32(const moe_dims_t& d, const uint16_t* x, const float* w_router,
+                      const float* bias, const float* tok_null_bias, float* logits_out,
+                      int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* ws,
+                      cudaStream_t st);
+int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st);
 int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_idx, void* ws,
                     int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* slot_row,
                     uint16_t* xs, int32_t* counts_ext, float* P, float* losses,
@@ -252,6 +282,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+// 32 lanes x 32 bit, 8 consecutive columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");

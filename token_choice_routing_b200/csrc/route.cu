@@ -1,4 +1,4 @@
-// moe_route: router GEMM (fp32, CUDA cores) fused with the expanded-pool
+// moe_route: router product on the tensor cores, fused with the expanded-pool
 // softmax statistics, top-K over the pool, renormalised gates and the
 // per-block statistics that dispatch and the aux losses need.
 //
@@ -14,11 +14,22 @@
 //  * renormalisation over the selected reals: gates = softmax over their
 //    logits; null slots weigh 0.
 //  * Z-Loss / 负载均衡损失: lse_t over the N+M pool and p_{t,i} are reduced per
-//    block here (fp32 over 64 tokens) and across blocks in fp64 later.
+//    block here (fp32 over 128 tokens) and across blocks in fp64 later.
 //
-// Layout: one CTA = 64 tokens x all N+1 logits (see route_kernel). x (bf16) is
-// widened to fp32 once when staged in shared memory; W_r slices arrive by
-// cp.async, double-buffered.
+// The router is an fp32 linear layer over bf16 tokens. Its product runs on the
+// tcgen05 tensor cores at fp32 accuracy: every fp32 weight w is the exact sum
+// of three bf16 numbers hi + mid + lo (each term takes the next 8 significant
+// bits), a bf16 x bf16 product is exact, and the MMA accumulates in fp32. So
+// s_j = sum_c x_c (hi_jc + mid_jc + lo_jc) is evaluated as three fp32
+// accumulations (one MMA with the three terms side by side in N) added in
+// fp32: the same error bound as an fp32 dot product of length d, with two
+// more roundings.
+//
+// Layout: one CTA = 128 tokens x all N+1 logits (one M=128 tile). Warp 0
+// issues TMA loads of the x tile (128 x 64 bf16) and the split weight tile
+// (3*NPW x 64 bf16) into a 4-stage ring; warp 1 issues the MMAs (M=128,
+// N=3*NPW, K=16) from one thread into TMEM; warps 2-9 add the three terms per
+// logit, then route the 128 tokens with 4 lanes per token.
 #include "moe_internal.cuh"
 
 #include <climits>
@@ -26,9 +37,6 @@
 namespace moe {
 
 struct RouteArgs {
-  const uint16_t* x;
-  const float* w;     // [N+1, d]
-  const float* wt;    // [d][NPAD+4] W^T of this call (workspace)
   const float* bias;  // [N+1] or null
   const float* tnb;   // [T] or null
   float* logits;      // [T, N+1] or null
@@ -46,398 +54,453 @@ struct RouteArgs {
   int32_t* lrank;
   int32_t* counts;
   int32_t* offsets;
+  unsigned long long limit_ns;
   int T, d, N, M, K, nblk;
 };
 
-
-// Thread tile of the router product: 8 tokens x 8 reals. Shared memory, not
-// the FMA pipe, bounds an fp32 CUDA-core GEMM: an a x b register tile loads
-// (a + b) / (a b) floats per FMA, and 8 x 8 keeps that at 1/4, the balance
-// point of an SM. Staged tiles are stored k-major (x^T and W^T) so a thread
-// fetches its 8 tokens and 8 reals at one d-column with four 16-byte loads.
-// To keep enough warps, the d-columns of each staged tile are split over S
-// thread slices whose partial sums are added once at the end.
-constexpr int kTileT = 8;  // tokens per thread
-constexpr int kTileR = 8;  // reals per thread
-constexpr int kXT = kRouteTokens + 4;  // row stride of the staged x^T tile
-
-template <int LG>
-struct RouteGeo {
-  static constexpr int NPAD = kTileR * LG;            // padded real count
-  static constexpr int TG = kRouteTokens / kTileT;    // token groups (8)
-  static constexpr int S = kRouteThreads / (TG * LG); // d-slices per staged tile
-  static constexpr int KS = kRouteBK / S;             // d-columns per slice per tile (= LG)
-  static_assert(S * KS == kRouteBK, "slices must tile the staged d-range");
-  static constexpr int WT = NPAD + 4;                 // row stride of W^T (null at column NPAD)
-  static constexpr int WCH = kRouteBK * WT / 4;       // 16-byte chunks of a staged W^T tile
-  static constexpr int WPT = (WCH + kRouteThreads - 1) / kRouteThreads;  // chunks per thread
-  static constexpr int LS = NPAD + 1;                 // odd row stride
-  // x^T: 2 stages; W^T: 3 stages (loaded two tiles ahead); x landing: 2 slots of 16 B per thread
-  static constexpr size_t main_bytes =
-      sizeof(float) * (2 * kRouteBK * kXT + 3 * kRouteBK * WT + 2 * (size_t)kRouteThreads * 4);
-  // slice partial sums [S][64][NPAD+1] alias the main-loop buffers
-  static constexpr size_t red_bytes = sizeof(float) * S * kRouteTokens * (NPAD + 1);
-  static constexpr size_t regionB = align_up(main_bytes > red_bytes ? main_bytes : red_bytes, 16);
-  // region C (after B): null partials and the logits
-  static constexpr int NNP = kRouteThreads / kRouteTokens;  // null partial sums per token (4)
-  static constexpr size_t off_npart = regionB;
-  static constexpr size_t off_s = off_npart + sizeof(float) * NNP * kRouteTokens;
-  static constexpr size_t endC = off_s + sizeof(float) * kRouteTokens * LS;
-  // per-token scratch reuses region B once the partial sums are folded
-  static constexpr size_t off_p = 0;
-  static constexpr size_t off_lse2 = off_p + sizeof(float) * kRouteTokens * LS;
-  static constexpr size_t off_nul = off_lse2 + sizeof(float) * kRouteTokens;
-  static constexpr size_t off_mask = align_up(off_nul + sizeof(int) * kRouteTokens, 16);
-  static constexpr size_t off_tk = off_mask + sizeof(unsigned long long) * kRouteTokens;
-  static constexpr size_t off_tkv = off_tk + sizeof(int) * kRouteTokens * kMaxK;
-  static constexpr size_t off_tokbits = off_tkv + sizeof(float) * kRouteTokens * kMaxK;
-  static constexpr size_t endB = off_tokbits + sizeof(unsigned) * 2 * kMaxN;
-  static_assert(endB <= regionB, "per-token scratch must fit in region B");
-  static constexpr size_t bytes = endC;
-};
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
+// ---------------------------------------------------------------------------------------
+// W_r (fp32 [N+1][d]) -> three bf16 terms, rows t*NPW + j (t = 0 hi, 1 mid, 2 lo),
+// zero rows for N < j < NPW. With w = m 2^e (24-bit m): hi = RN8(w) leaves a
+// remainder of at most 16 significant bits, mid = RN8(remainder) leaves at most
+// 8, and lo holds those exactly; both subtractions are exact in fp32.
+__device__ __forceinline__ void split3(float w, uint16_t& h, uint16_t& m, uint16_t& l) {
+  const __nv_bfloat16 bh = __float2bfloat16_rn(w);
+  const float r1 = w - __bfloat162float(bh);
+  const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(bm);
+  const __nv_bfloat16 bl = __float2bfloat16_rn(r2);
+  h = __bfloat16_as_ushort(bh);
+  m = __bfloat16_as_ushort(bm);
+  l = __bfloat16_as_ushort(bl);
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// One thread per 8 d-columns of one padded row.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, uint16_t* __restrict__ w3,
+                                                           int N, int npw, int d) {
+  const int nch = d >> 3;
+  const long long total = (long long)npw * nch;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int j = (int)(i / nch), c = (int)(i - (long long)j * nch);
+    uint16_t hv[8], mv[8], lv[8];
+    if (j <= N) {
+      const float4* src = reinterpret_cast<const float4*>(w + (size_t)j * d + (size_t)c * 8);
+      const float4 p0 = __ldg(src), p1 = __ldg(src + 1);
+      const float v[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) split3(v[e], hv[e], mv[e], lv[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) hv[e] = mv[e] = lv[e] = 0;
+    }
+    auto pack = [](const uint16_t (&u)[8]) {
+      return make_uint4(u[0] | ((uint32_t)u[1] << 16), u[2] | ((uint32_t)u[3] << 16),
+                        u[4] | ((uint32_t)u[5] << 16), u[6] | ((uint32_t)u[7] << 16));
+    };
+    const size_t col = (size_t)c * 8;
+    *reinterpret_cast<uint4*>(w3 + (size_t)j * d + col) = pack(hv);
+    *reinterpret_cast<uint4*>(w3 + (size_t)(npw + j) * d + col) = pack(mv);
+    *reinterpret_cast<uint4*>(w3 + (size_t)(2 * npw + j) * d + col) = pack(lv);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Shared memory of the route kernel. The routing scratch aliases the staging
+// ring: it is written only after the last MMA has completed (its commit is
+// what releases the epilogue), and every issued TMA copy was consumed by an MMA.
+template <int NPW>
+struct RouteSmem {
+  static constexpr int STAGES = 4;
+  static constexpr int BROWS = 3 * NPW;
+  static constexpr int A_BYTES = kRouteTokens * kRouteBK * 2;
+  static constexpr int B_BYTES = BROWS * kRouteBK * 2;
+  static constexpr size_t off_a = 0;
+  static constexpr size_t off_b = off_a + (size_t)STAGES * A_BYTES;
+  static constexpr size_t ring_end = off_b + (size_t)STAGES * B_BYTES;
+  // routing scratch
+  static constexpr int LS = NPW + 1;  // odd row stride of the logit rows
+  static constexpr size_t off_s = 0;  // float [128][LS]: logits, then p in place
+  static constexpr size_t off_pn = off_s + sizeof(float) * kRouteTokens * LS;  // float [128] null p
+  static constexpr size_t off_lse2 = off_pn + sizeof(float) * kRouteTokens;    // float [128]
+  static constexpr size_t off_nul = off_lse2 + sizeof(float) * kRouteTokens;   // int [128]
+  static constexpr size_t off_mask = align_up(off_nul + sizeof(int) * kRouteTokens, 16);  // u64 [128]
+  static constexpr size_t off_tk = off_mask + sizeof(unsigned long long) * kRouteTokens;  // int [128][kMaxK]
+  static constexpr size_t off_tkv = off_tk + sizeof(int) * kRouteTokens * kMaxK;          // float [128][kMaxK]
+  static constexpr size_t off_tokbits = off_tkv + sizeof(float) * kRouteTokens * kMaxK;  // u32 [4][kMaxN]
+  static constexpr size_t scratch_end = off_tokbits + sizeof(unsigned) * 4 * kMaxN;
+  static_assert(scratch_end <= ring_end, "routing scratch must fit in the staging ring");
+  static constexpr size_t off_bar = ring_end;  // full[STAGES], empty[STAGES], tfull
+  static constexpr size_t off_misc = off_bar + 8 * (2 * STAGES + 1);  // [0] TMEM base, [1] abort
+  static constexpr size_t bytes = off_misc + 16 + 1024;  // + slack for 1024-byte alignment
+};
 
 // (value desc, index asc) order: true if (va, ia) precedes (vb, ib).
 __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
-// W^T for one call: wt[k][j] = W_r[j][k] for real j < N, wt[k][NPAD] = W_r[N][k]
-// (the null row), zero for the padding columns; row stride NPAD + 4. One CTA
-// per 32 d-columns, through a shared tile so both sides are coalesced.
-template <int LG>
-__global__ void __launch_bounds__(256) router_transpose_kernel(const float* __restrict__ w, float* __restrict__ wt,
-                                                               int N, int d) {
-  using G = RouteGeo<LG>;
-  constexpr int NPAD = G::NPAD, WT = G::WT;
-  __shared__ float tile[NPAD + 1][33];
-  const int k0 = blockIdx.x * 32;
-  for (int i = threadIdx.x; i < (NPAD + 1) * 32; i += blockDim.x) {
-    const int r = i >> 5, kk = i & 31;
-    const int src = (r < N) ? r : (r == NPAD ? N : -1);
-    tile[r][kk] = (src >= 0) ? w[(size_t)src * d + k0 + kk] : 0.f;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 32 * WT; i += blockDim.x) {
-    const int kk = i / WT, j = i - kk * WT;
-    wt[(size_t)(k0 + kk) * WT + j] = (j <= NPAD) ? tile[j][kk] : 0.f;
-  }
+// bar.red.and over a named barrier: every participating thread gets the AND
+// of all their predicates (a CTA-uniform decision among those threads).
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
-// One CTA: 64 tokens x all N+1 logits, 256 threads. Main loop: thread
-// (s, lg, tg) owns tokens {4tg..4tg+3, 32+4tg..32+4tg+3} and reals
-// {4lg..4lg+3, 4LG+4lg..4LG+4lg+3} over the d-columns [s*KS, (s+1)*KS) of
-// every staged tile; the null logit of token tid & 63 over the 8 d-columns it stages.
-// Epilogue: 4 threads per token.
-template <int LG>
-__global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
-  using G = RouteGeo<LG>;
-  constexpr int NPAD = G::NPAD, S = G::S, KS = G::KS, LS = G::LS, WT = G::WT;
-  constexpr int NQ = NPAD / 4;  // reals per epilogue thread
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* xsT = reinterpret_cast<float*>(smem);       // [2][BK][kXT]
+// ---------------------------------------------------------------------------------------
+// One CTA: tokens [128 b, 128 b + 128) x all N+1 logits, 320 threads.
+template <int NPW>
+__global__ void __launch_bounds__(kRouteThreads, 1)
+    route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 const RouteArgs a) {
+  using SM = RouteSmem<NPW>;
+  constexpr int STAGES = SM::STAGES;
+  constexpr int LS = SM::LS;
+  constexpr int NQ = (NPW < kMaxN ? NPW : kMaxN) / 4;  // reals per lane, 4 lanes per token
+  constexpr uint32_t TCOLS = SM::BROWS <= 64 ? 64u : SM::BROWS <= 128 ? 128u : 256u;
+  constexpr uint32_t IDESC = idesc_bf16_f32(kRouteTokens, SM::BROWS);
+  constexpr uint32_t TX = SM::A_BYTES + SM::B_BYTES;
 
-  const int tid = threadIdx.x;
-  const int tg = tid % G::TG;
-  const int lg = (tid / G::TG) % LG;
-  const int sl = tid / (G::TG * LG);
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base + SM::off_a;
+  unsigned char* sB = base + SM::off_b;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + SM::off_bar);
+  volatile int* misc = reinterpret_cast<volatile int*>(base + SM::off_misc);
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  const uint32_t tfull_bar = smem_u32(bars + 2 * STAGES);
+  volatile int* abort_flag = misc + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
-  const int T = a.T, d = a.d, N = a.N, M = a.M, K = a.K;
+  const int T = a.T, N = a.N, M = a.M, K = a.K;
   const int tok0 = b * kRouteTokens;
   const int nvalid = min(kRouteTokens, T - tok0);
-  const int nkt = d / kRouteBK;
+  const int nkb = a.d / kRouteBK;
 
-  float acc[kTileT][kTileR];
-#pragma unroll
-  for (int i = 0; i < kTileT; ++i)
-#pragma unroll
-    for (int j = 0; j < kTileR; ++j) acc[i][j] = 0.f;
-
-  // Staging, two tiles ahead. W^T tile kt+2 is copied by cp.async straight
-  // into its slot of a 3-deep ring (rows of NPAD+4 floats, already transposed
-  // by router_transpose_kernel). x: thread copies token tid & 63, 8 d-columns
-  // from (tid >> 6) * 8, into its own landing slot; after its own wait it
-  // widens them into the x^T stage of tile kt+1 and adds their share of the
-  // null logit (null weights from global, cached). No registers are held
-  // across the multiply.
-  float* wsT = xsT + 2 * kRouteBK * kXT;                       // [3][BK][WT]
-  float* land0 = wsT + 3 * kRouteBK * WT;                      // [2][256][4]
-  const int xrow = tid & 63, xkc = (tid >> 6) * 8;
-  const bool xok = tok0 + xrow < T;
-  const uint16_t* xsrc = a.x + (size_t)(tok0 + (xok ? xrow : 0)) * d + xkc;
-  const float* wnull = a.w + (size_t)N * d + xkc;
-  float accn = 0.f;  // null logit of token xrow over its staged columns
-  auto load_tiles = [&](int kt) {
-    if (kt < nkt) {
-      cp_async16(smem_u32(land0 + ((kt & 1) * kRouteThreads + tid) * 4), xsrc + (size_t)kt * kRouteBK, xok ? 16 : 0);
-      float* wb = wsT + (kt % 3) * kRouteBK * WT;
-      const float* src = a.wt + (size_t)kt * kRouteBK * WT;
-#pragma unroll
-      for (int q = 0; q < G::WPT; ++q) {
-        const int c = tid + kRouteThreads * q;
-        if (c < G::WCH) cp_async16(smem_u32(wb + 4 * c), src + 4 * c, 16);
-      }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmW);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
     }
-    cp_async_commit();  // one group per call, possibly empty
-  };
-  auto store_x = [&](int kt) {
-    const uint4 xr = *reinterpret_cast<const uint4*>(land0 + ((kt & 1) * kRouteThreads + tid) * 4);
-    float* xb = xsT + (kt & 1) * kRouteBK * kXT;
-    const float xv[8] = {bf16lo(xr.x), bf16hi(xr.x), bf16lo(xr.y), bf16hi(xr.y),
-                         bf16lo(xr.z), bf16hi(xr.z), bf16lo(xr.w), bf16hi(xr.w)};
-#pragma unroll
-    for (int u = 0; u < 8; ++u) xb[(xkc + u) * kXT + xrow] = xv[u];
-    const float4 w0 = __ldg(reinterpret_cast<const float4*>(wnull + (size_t)kt * kRouteBK));
-    const float4 w1 = __ldg(reinterpret_cast<const float4*>(wnull + (size_t)kt * kRouteBK + 4));
-    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-    for (int u = 0; u < 8; ++u) accn = fmaf(xv[u], wv[u], accn);
-  };
-
-  load_tiles(0);
-  load_tiles(1);
-  cp_async_wait_group1();  // this thread's copies of tile 0
-  store_x(0);
-  for (int kt = 0; kt < nkt; ++kt) {
-    __syncthreads();
-    load_tiles(kt + 2);  // its W^T slot was last read at iteration kt-1; its x slot was written out
-    const float* xb = xsT + (kt & 1) * kRouteBK * kXT + (sl * KS) * kXT;
-    const float* wb = wsT + (kt % 3) * kRouteBK * WT + (sl * KS) * WT;
-#pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
-      const float4 xa = *reinterpret_cast<const float4*>(xb + kk * kXT + 4 * tg);
-      const float4 xc = *reinterpret_cast<const float4*>(xb + kk * kXT + 32 + 4 * tg);
-      const float4 wa = *reinterpret_cast<const float4*>(wb + kk * WT + 4 * lg);
-      const float4 wc = *reinterpret_cast<const float4*>(wb + kk * WT + 4 * LG + 4 * lg);
-      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xc.x, xc.y, xc.z, xc.w};
-      const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wc.x, wc.y, wc.z, wc.w};
-#pragma unroll
-      for (int i = 0; i < kTileT; ++i)
-#pragma unroll
-        for (int jj = 0; jj < kTileR; ++jj) acc[i][jj] = fmaf(xv[i], wv[jj], acc[i][jj]);
-    }
-    if (kt + 1 < nkt) {
-      cp_async_wait_group1();  // this thread's copies of tile kt+1 (tile kt+2 may be in flight)
-      store_x(kt + 1);         // x^T stage (kt+1)&1 was last read before this iteration's barrier
-    }
+    mbar_init(tfull_bar, 1);
+    misc[1] = 0;
+    fence_mbar_init();
   }
-  cp_async_wait_all();
-  __syncthreads();  // main-loop buffers are reused below
-
-  float* red = reinterpret_cast<float*>(smem);  // [S][64][NPAD+1]
-  float* npart = reinterpret_cast<float*>(smem + G::off_npart);
-  float* s_l = reinterpret_cast<float*>(smem + G::off_s);
-#pragma unroll
-  for (int i = 0; i < kTileT; ++i) {
-    const int t = 4 * tg + (i & 3) + 32 * (i >> 2);
-#pragma unroll
-    for (int jj = 0; jj < kTileR; ++jj) {
-      const int r = 4 * lg + (jj & 3) + 4 * LG * (jj >> 2);
-      red[(sl * kRouteTokens + t) * (NPAD + 1) + r] = acc[i][jj];
-    }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<int*>(misc)), TCOLS);
+    tmem_relinquish();
   }
-  npart[(tid >> 6) * kRouteTokens + (tid & 63)] = accn;
+  tc_fence_before();
   __syncthreads();
-  for (int o = tid; o < kRouteTokens * NPAD; o += kRouteThreads) {
-    const int t = o / NPAD, j = o - t * NPAD;
-    if (j < N) {
-      float v = 0.f;
-#pragma unroll
-      for (int q = 0; q < S; ++q) v += red[(q * kRouteTokens + t) * (NPAD + 1) + j];
-      s_l[t * LS + j] = v + (a.bias ? __ldg(a.bias + j) : 0.f);
-    }
-  }
-  __syncthreads();  // region B is free from here on
+  tc_fence_after();
+  const uint32_t tmem_base = (uint32_t)misc[0];
 
-  float* p_s = reinterpret_cast<float*>(smem + G::off_p);
-  float* lse2 = reinterpret_cast<float*>(smem + G::off_lse2);
-  int* nul = reinterpret_cast<int*>(smem + G::off_nul);
-  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem + G::off_mask);
-  int* tk = reinterpret_cast<int*>(smem + G::off_tk);
-  float* tkv = reinterpret_cast<float*>(smem + G::off_tkv);
-  unsigned* tokbits = reinterpret_cast<unsigned*>(smem + G::off_tokbits);  // [2][kMaxN]
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------ TMA producer
+      uint32_t armed = 0, armed_par = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, a.limit_ns, abort_flag, a.hdr)) break;
+        mbar_arrive_expect_tx(full_bar(s), TX);
+        tma_load_2d(smem_u32(sA + s * SM::A_BYTES), &tmX, full_bar(s), kb * kRouteBK, tok0);
+        tma_load_2d(smem_u32(sB + s * SM::B_BYTES), &tmW, full_bar(s), kb * kRouteBK, 0);
+        armed |= 1u << s;
+        armed_par = (armed_par & ~(1u << s)) | (ph << s);
+      }
+      if (*abort_flag) {
+        // let every issued copy land before the CTA can exit
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s))
+            (void)mbar_wait_bounded(full_bar(s), (armed_par >> s) & 1u, a.limit_ns, nullptr, a.hdr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------ MMA issuer (single thread)
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait_bounded(full_bar(s), ph, a.limit_ns, abort_flag, a.hdr)) break;
+        tc_fence_after();
+        const uint64_t adesc = smem_desc_sw128(smem_u32(sA + s * SM::A_BYTES));
+        const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * SM::B_BYTES));
+#pragma unroll
+        for (int k = 0; k < kRouteBK / 16; ++k)
+          tc_mma_f16(tmem_base, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
+                     (kb | k) != 0 ? 1u : 0u);
+        tc_commit(empty_bar(s));
+      }
+      // fires once every MMA issued above has completed (also after an abort)
+      tc_commit(tfull_bar);
+      (void)mbar_wait_bounded(tfull_bar, 0, a.limit_ns, nullptr, a.hdr);
+    }
+  } else {
+    // ------------------------------ epilogue warps 2..9
+    const int etid = threadIdx.x - 64;
+    const int ew = warp - 2;
+    float* s_l = reinterpret_cast<float*>(base + SM::off_s);
+    float* pn = reinterpret_cast<float*>(base + SM::off_pn);
+    float* lse2 = reinterpret_cast<float*>(base + SM::off_lse2);
+    int* nul = reinterpret_cast<int*>(base + SM::off_nul);
+    unsigned long long* mask = reinterpret_cast<unsigned long long*>(base + SM::off_mask);
+    int* tk = reinterpret_cast<int*>(base + SM::off_tk);
+    float* tkv = reinterpret_cast<float*>(base + SM::off_tkv);
+    unsigned* tokbits = reinterpret_cast<unsigned*>(base + SM::off_tokbits);  // [4][kMaxN]
 
-  {
-    // ---- per-token routing, 4 lanes per token (all lanes take part in the shuffles)
-    const int t = tid >> 2, q = tid & 3;
-    const bool valid = t < nvalid;
-    const int tok = tok0 + t;
-    float sn = 0.f;
+    const bool ok = mbar_wait_bounded(tfull_bar, 0, a.limit_ns, abort_flag, a.hdr) && *abort_flag == 0;
+    const bool run = named_bar_and(1, kRouteEpiThreads, ok);
+    if (run) {
+      // ---- logits from TMEM: warp reads lane quarter q (tokens 32q..32q+31) and
+      // one half of the NPW columns; s_j = (hi_j + mid_j) + lo_j (+ bias)
+      tc_fence_after();
+      const int q = warp & 3, hh = ew >> 2;
+      const int t = q * 32 + lane;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
+      const float tn = (a.tnb != nullptr && t < nvalid) ? __ldg(a.tnb + tok0 + t) : 0.f;
+#pragma unroll 1
+      for (int c0 = hh * (NPW / 2); c0 < (hh + 1) * (NPW / 2); c0 += 8) {
+        uint32_t rh[8], rm[8], rl[8];
+        tmem_ld8(tb + (uint32_t)c0, rh);
+        tmem_ld8(tb + (uint32_t)(NPW + c0), rm);
+        tmem_ld8(tb + (uint32_t)(2 * NPW + c0), rl);
+        tmem_ld_wait();
 #pragma unroll
-    for (int l = 0; l < G::NNP; ++l) sn += npart[l * kRouteTokens + t];
-    if (a.bias) sn += __ldg(a.bias + N);
-    if (a.tnb && valid) sn += __ldg(a.tnb + tok);
-    float v[NQ];
-#pragma unroll
-    for (int u = 0; u < NQ; ++u) {
-      const int i = q + 4 * u;
-      v[u] = (i < N) ? s_l[t * LS + i] : -INFINITY;
-    }
-    // softmax statistics over the pool (M copies of the null logit)
-    float m = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < NQ; ++u) m = fmaxf(m, v[u]);
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    if (M > 0) m = fmaxf(m, sn);
-    float z = 0.f;
-#pragma unroll
-    for (int u = 0; u < NQ; ++u)
-      if (q + 4 * u < N) z += expf(v[u] - m);
-    z += __shfl_xor_sync(0xffffffffu, z, 1);
-    z += __shfl_xor_sync(0xffffffffu, z, 2);
-    const float Z = (M > 0) ? z + (float)M * expf(sn - m) : z;
-    const float lse = m + logf(Z);
-    // p_i = e^{s_i - lse} evaluated as e^{s_i - m} / Z: no cancellation when |m| is large
-#pragma unroll
-    for (int u = 0; u < NQ; ++u) {
-      const int i = q + 4 * u;
-      if (i < N) p_s[t * LS + i] = expf(v[u] - m) / Z;
-    }
-    if (q == 0) {
-      p_s[t * LS + NPAD] = (M > 0) ? expf(sn - m) / Z : 0.f;
-      lse2[t] = lse * lse;
-    }
-
-    // top-K over the pool, in rank order: K rounds of "best remaining real"
-    // against the null logit (a real equal to it wins: lower index)
-    unsigned sel = 0u;
-    int used = 0, r = 0;
-    unsigned long long msk = 0ull;
-    for (int k = 0; k < K; ++k) {
-      float bv = -INFINITY;
-      int bi = INT_MAX;
-#pragma unroll
-      for (int u = 0; u < NQ; ++u) {
-        const int i = q + 4 * u;
-        if (i < N && !((sel >> u) & 1u) && ranks_before(v[u], i, bv, bi)) {
-          bv = v[u];
-          bi = i;
-        }
-      }
-#pragma unroll
-      for (int off = 1; off <= 2; off <<= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (ranks_before(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      const bool take_null = (used < M) && (bi == INT_MAX || bv < sn);
-      int id;
-      if (take_null) {
-        id = N + used;
-        ++used;
-      } else {
-        id = bi;
-        ++r;
-        msk |= 1ull << bi;
-        if ((bi & 3) == q) sel |= 1u << (bi >> 2);
-      }
-      if (q == 0) {
-        tk[t * kMaxK + k] = id;
-        tkv[t * kMaxK + k] = bv;
-      }
-    }
-    __syncwarp();
-    if (valid) {
-      if (q == 0) {
-        // gates: softmax over the selected real logits (rank order: first real is the max)
-        float smax = 0.f, gsum = 0.f;
-        bool first = true;
-        for (int k = 0; k < K; ++k) {
-          if (tk[t * kMaxK + k] < N) {
-            const float sv = tkv[t * kMaxK + k];
-            if (first) {
-              smax = sv;
-              first = false;
-            }
-            gsum += expf(sv - smax);
+        for (int j = 0; j < 8; ++j) {
+          const int col = c0 + j;
+          if (col <= N) {
+            float s = (__uint_as_float(rh[j]) + __uint_as_float(rm[j])) + __uint_as_float(rl[j]);
+            if (a.bias) s += __ldg(a.bias + col);
+            if (col == N) s += tn;
+            s_l[t * LS + col] = s;
           }
         }
-        for (int k = 0; k < K; ++k) {
-          const int id = tk[t * kMaxK + k];
-          const float g = (id < N) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
-          a.topk_idx[(size_t)tok * K + k] = id;
-          a.topk_gate[(size_t)tok * K + k] = g;
-        }
-        a.n_real[tok] = r;
-        nul[t] = K - r;
-        mask[t] = msk;
       }
-      if (a.logits) {
-        float* lo = a.logits + (size_t)tok * (N + 1);
+    }
+    named_bar_sync(1, kRouteEpiThreads);
+
+    if (run) {
+      // ---- per-token routing, 4 lanes per token, two passes of 64 tokens
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int t = pass * 64 + (etid >> 2), q = etid & 3;
+        const bool valid = t < nvalid;
+        const int tok = tok0 + t;
+        float* row = s_l + t * LS;
+        const float sn = row[N];
+        float v[NQ];
 #pragma unroll
         for (int u = 0; u < NQ; ++u) {
           const int i = q + 4 * u;
-          if (i < N) lo[i] = v[u];
+          v[u] = (i < N) ? row[i] : -INFINITY;
         }
-        if (q == 0) lo[N] = sn;
+        // softmax statistics over the pool (M copies of the null logit)
+        float m = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < NQ; ++u) m = fmaxf(m, v[u]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        if (M > 0) m = fmaxf(m, sn);
+        float z = 0.f;
+#pragma unroll
+        for (int u = 0; u < NQ; ++u)
+          if (q + 4 * u < N) z += expf(v[u] - m);
+        z += __shfl_xor_sync(0xffffffffu, z, 1);
+        z += __shfl_xor_sync(0xffffffffu, z, 2);
+        const float Z = (M > 0) ? z + (float)M * expf(sn - m) : z;
+        const float lse = m + logf(Z);
+        // p_i = e^{s_i - lse} evaluated as e^{s_i - m} / Z (no cancellation when |m| is
+        // large), written over this lane's own logits
+#pragma unroll
+        for (int u = 0; u < NQ; ++u) {
+          const int i = q + 4 * u;
+          if (i < N) row[i] = expf(v[u] - m) / Z;
+        }
+        if (q == 0) {
+          pn[t] = (M > 0) ? expf(sn - m) / Z : 0.f;
+          lse2[t] = lse * lse;
+        }
+
+        // top-K over the pool, in rank order: K rounds of "best remaining real"
+        // against the null logit (a real equal to it wins: lower index)
+        unsigned sel = 0u;
+        int used = 0, r = 0;
+        unsigned long long msk = 0ull;
+        for (int k = 0; k < K; ++k) {
+          float bv = -INFINITY;
+          int bi = INT_MAX;
+#pragma unroll
+          for (int u = 0; u < NQ; ++u) {
+            const int i = q + 4 * u;
+            if (i < N && !((sel >> u) & 1u) && ranks_before(v[u], i, bv, bi)) {
+              bv = v[u];
+              bi = i;
+            }
+          }
+#pragma unroll
+          for (int off = 1; off <= 2; off <<= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ranks_before(ov, oi, bv, bi)) {
+              bv = ov;
+              bi = oi;
+            }
+          }
+          const bool take_null = (used < M) && (bi == INT_MAX || bv < sn);
+          int id;
+          if (take_null) {
+            id = N + used;
+            ++used;
+          } else {
+            id = bi;
+            ++r;
+            msk |= 1ull << bi;
+            if ((bi & 3) == q) sel |= 1u << (bi >> 2);
+          }
+          if (q == 0) {
+            tk[t * kMaxK + k] = id;
+            tkv[t * kMaxK + k] = bv;
+          }
+        }
+        __syncwarp();
+        if (valid) {
+          if (q == 0) {
+            // gates: softmax over the selected real logits (rank order: first real is the max)
+            float smax = 0.f, gsum = 0.f;
+            bool first = true;
+            for (int k = 0; k < K; ++k) {
+              if (tk[t * kMaxK + k] < N) {
+                const float sv = tkv[t * kMaxK + k];
+                if (first) {
+                  smax = sv;
+                  first = false;
+                }
+                gsum += expf(sv - smax);
+              }
+            }
+            for (int k = 0; k < K; ++k) {
+              const int id = tk[t * kMaxK + k];
+              const float g = (id < N) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
+              a.topk_idx[(size_t)tok * K + k] = id;
+              a.topk_gate[(size_t)tok * K + k] = g;
+            }
+            a.n_real[tok] = r;
+            nul[t] = K - r;
+            mask[t] = msk;
+          }
+          if (a.logits) {
+            float* lo = a.logits + (size_t)tok * (N + 1);
+#pragma unroll
+            for (int u = 0; u < NQ; ++u) {
+              const int i = q + 4 * u;
+              if (i < N) lo[i] = v[u];
+            }
+            if (q == 0) lo[N] = sn;
+          }
+        }
+      }
+    }
+    named_bar_sync(1, kRouteEpiThreads);
+
+    if (run) {
+      // ---- block statistics. Warps 2..5: for each expert e, ballot bit e of the
+      // selection masks of 32 tokens, giving the block's tokens that chose e as a
+      // 128-bit set (a slot's rank is the number of earlier tokens in that set).
+      // Warps 6..9: probability column sums, the null-count histogram and the
+      // sum of lse^2 over the block, each in a fixed order.
+      if (ew < 4) {
+        const int t = 32 * ew + lane;
+        const unsigned long long mk = (t < nvalid) ? mask[t] : 0ull;
+        for (int e = 0; e < N; ++e) {
+          const unsigned bits = __ballot_sync(0xffffffffu, (mk >> e) & 1ull);
+          if (lane == 0) tokbits[ew * kMaxN + e] = bits;
+        }
+      } else {
+        const int c = etid - 128;
+        if (c <= N) {
+          const float* col = (c < N) ? s_l + c : pn;
+          const int stride = (c < N) ? LS : 1;
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+          int t = 0;
+          for (; t + 4 <= nvalid; t += 4) {
+            s0 += col[t * stride];
+            s1 += col[(t + 1) * stride];
+            s2 += col[(t + 2) * stride];
+            s3 += col[(t + 3) * stride];
+          }
+          for (; t < nvalid; ++t) s0 += col[t * stride];
+          a.ppart[(size_t)b * (N + 1) + c] = (s0 + s1) + (s2 + s3);
+        } else if (c <= N + K + 1) {
+          const int h = c - N - 1;
+          int cnt = 0;
+          for (int t = 0; t < nvalid; ++t) cnt += (nul[t] == h);
+          a.hist[(size_t)b * (K + 1) + h] = cnt;
+        } else if (c == N + K + 2) {
+          float s0 = 0.f, s1 = 0.f;
+          int t = 0;
+          for (; t + 2 <= nvalid; t += 2) {
+            s0 += lse2[t];
+            s1 += lse2[t + 1];
+          }
+          if (t < nvalid) s0 += lse2[t];
+          a.lsq[b] = s0 + s1;
+        }
+      }
+    }
+    named_bar_sync(1, kRouteEpiThreads);
+
+    if (run) {
+      if (etid < N) {
+        int cnt = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) cnt += __popc(tokbits[w * kMaxN + etid]);
+        a.counts_blk[(size_t)etid * a.nblk + b] = cnt;
+        if (cnt) atomicAdd(a.tot + etid, cnt);
+      }
+      // lrank for (token, slot): 4 threads per token, slots k = q, q+4, ...
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int t = pass * 64 + (etid >> 2), q = etid & 3;
+        if (t < nvalid) {
+          const int w = t >> 5;
+          const unsigned below = (1u << (t & 31)) - 1u;
+          for (int k = q; k < K; k += 4) {
+            const int id = tk[t * kMaxK + k];
+            int rank = -1;
+            if (id < N) {
+              rank = __popc(tokbits[w * kMaxN + id] & below);
+              for (int w2 = 0; w2 < w; ++w2) rank += __popc(tokbits[w2 * kMaxN + id]);
+            }
+            a.lrank[(size_t)(tok0 + t) * K + k] = rank;
+          }
+        }
       }
     }
   }
-  __syncthreads();
 
-  // Per-block ranks and counts (ascending token order inside an expert): for
-  // each expert e, warps 0 and 1 ballot bit e of their 32 tokens' selection
-  // masks, giving the block's tokens that chose e as a 64-bit set; a slot's
-  // rank is the number of earlier tokens in that set.
-  const int lane = tid & 31, warp = tid >> 5;
-  if (warp < 2) {
-    const int t = 32 * warp + lane;
-    const unsigned long long m = (t < nvalid) ? mask[t] : 0ull;
-    for (int e = 0; e < N; ++e) {
-      const unsigned bits = __ballot_sync(0xffffffffu, (m >> e) & 1ull);
-      if (lane == 0) tokbits[warp * kMaxN + e] = bits;
-    }
-  }
-  if (tid >= 64 && tid <= 64 + N) {  // probability sums of the block, one column per thread
-    const int i = tid - 64;
-    const int col = (i < N) ? i : NPAD;
-    float s = 0.f;
-    for (int t = 0; t < nvalid; ++t) s += p_s[t * LS + col];
-    a.ppart[(size_t)b * (N + 1) + i] = s;
-  }
-  if (tid >= 160 && tid <= 160 + K) {
-    const int c = tid - 160;
-    int cnt = 0;
-    for (int t = 0; t < nvalid; ++t) cnt += (nul[t] == c);
-    a.hist[(size_t)b * (K + 1) + c] = cnt;
-  }
-  if (tid == 192) {
-    float s = 0.f;
-    for (int t = 0; t < nvalid; ++t) s += lse2[t];
-    a.lsq[b] = s;
-  }
+  tc_fence_before();
   __syncthreads();
-  if (tid < N) {
-    const int cnt = __popc(tokbits[tid]) + __popc(tokbits[kMaxN + tid]);
-    a.counts_blk[(size_t)tid * a.nblk + b] = cnt;
-    if (cnt) atomicAdd(a.tot + tid, cnt);
-  }
-  if (tid < nvalid * 4) {
-    // lrank for (token, slot): 4 threads per token, slots k = q, q+4, ...
-    const int t = tid >> 2, q = tid & 3;
-    const int tok = tok0 + t;
-    const int w = t >> 5;
-    const unsigned below = (1u << (t & 31)) - 1u;
-    for (int k = q; k < K; k += 4) {
-      const int id = tk[t * kMaxK + k];
-      int rank = -1;
-      if (id < N) rank = __popc(tokbits[w * kMaxN + id] & below) + (w ? __popc(tokbits[id]) : 0);
-      a.lrank[(size_t)tok * K + k] = rank;
-    }
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TCOLS);
   }
 }
 
+// ---------------------------------------------------------------------------------------
 // Per-expert scan over route blocks: bases[e][b] = offsets[e] + sum_{b' < b}
 // counts_blk[e][b'] (ascending token order inside an expert's segment), with
 // offsets[e] = sum_{e' < e} tot[e'] from the route blocks' integer atomics.
@@ -531,30 +594,50 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
   }
 }
 
-template <int LG>
-static int launch_route_t(const RouteArgs& a, cudaStream_t st) {
-  using SM = RouteGeo<LG>;
-  router_transpose_kernel<LG><<<a.d / 32, 256, 0, st>>>(a.w, const_cast<float*>(a.wt), a.N, a.d);
+template <int NPW>
+static int launch_route_t(const CUtensorMap& tx, const CUtensorMap& tw, const RouteArgs& a, cudaStream_t st) {
+  using SM = RouteSmem<NPW>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<LG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<NPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM::bytes);
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
   }
-  route_kernel<LG><<<a.nblk, kRouteThreads, SM::bytes, st>>>(a);
+  route_kernel<NPW><<<a.nblk, kRouteThreads, SM::bytes, st>>>(tx, tw, a);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(d);
+  ScanArgs sa{};
+  sa.counts_blk = ws_ptr<int32_t>(ws, L.counts_blk);
+  sa.tot = ws_ptr<int32_t>(ws, L.hdr + kHdrTotOffset);
+  sa.bases = ws_ptr<int32_t>(ws, L.bases);
+  sa.counts = ws_ptr<int32_t>(ws, L.counts);
+  sa.offsets = ws_ptr<int32_t>(ws, L.offsets);
+  sa.ppart = ws_ptr<float>(ws, L.ppart);
+  sa.hist = ws_ptr<int32_t>(ws, L.hist);
+  sa.lsq = ws_ptr<float>(ws, L.lsq);
+  sa.auxp = ws_ptr<double>(ws, L.auxp);
+  sa.N = d.N;
+  sa.K = d.K;
+  sa.nblk = L.nblk;
+  sa.nparts = L.nparts;
+  scan_kernel<<<d.N + L.nparts, kScanThreads, 0, st>>>(sa);
   return cuda_status(cudaGetLastError());
 }
 
 int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, const float* bias,
                  const float* tok_null_bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
                  int32_t* n_real, void* ws, cudaStream_t st) {
+  if (route_fp32_cores(d))
+    return launch_route_fp32(d, x, w_router, bias, tok_null_bias, logits_out, topk_idx, topk_gate, n_real,
+                             ws, st);
   const WsLayout L = ws_layout(d);
   RouteArgs a{};
-  a.x = x;
-  a.w = w_router;
   a.bias = bias;
   a.tnb = tok_null_bias;
   a.logits = logits_out;
@@ -562,7 +645,6 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.topk_gate = topk_gate;
   a.n_real = n_real;
   a.hdr = ws_ptr<uint32_t>(ws, L.hdr);
-  a.wt = ws_ptr<float>(ws, L.wt);
   a.tot = ws_ptr<int32_t>(ws, L.hdr + kHdrTotOffset);
   a.counts_blk = ws_ptr<int32_t>(ws, L.counts_blk);
   a.bases = ws_ptr<int32_t>(ws, L.bases);
@@ -572,6 +654,7 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.lrank = ws_ptr<int32_t>(ws, L.lrank);
   a.counts = ws_ptr<int32_t>(ws, L.counts);
   a.offsets = ws_ptr<int32_t>(ws, L.offsets);
+  a.limit_ns = kWaitLimitNs;
   a.T = d.T;
   a.d = d.d;
   a.N = d.N;
@@ -581,28 +664,32 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   // the status word and the per-expert totals start at zero for every layer call
   cudaError_t e = cudaMemsetAsync(a.hdr, 0, kHdrTotOffset + sizeof(int32_t) * d.N, st);
   if (e != cudaSuccess) return cuda_status(e);
+
+  // the split router weight for this call, then tensor maps over x and it
+  const int npw = route_npw(d.N);
+  uint16_t* w3 = ws_ptr<uint16_t>(ws, L.wprep);
+  {
+    const long long work = (long long)npw * (d.d / 8);
+    long long grid = (work + 255) / 256;
+    if (grid > (long long)sm_count() * 8) grid = (long long)sm_count() * 8;
+    router_split_kernel<<<(int)grid, 256, 0, st>>>(w_router, w3, d.N, npw, d.d);
+    const int r = cuda_status(cudaGetLastError());
+    if (r != MOE_OK) return r;
+  }
+  CUtensorMap tx, tw;
+  if (!make_tmap_bf16(&tx, x, (uint64_t)d.T, (uint64_t)d.d, kRouteTokens) ||
+      !make_tmap_bf16(&tw, w3, (uint64_t)3 * npw, (uint64_t)d.d, (uint32_t)(3 * npw)))
+    return MOE_ERR_CUDA;
   int r;
-  if (d.N <= 8) r = launch_route_t<1>(a, st);
-  else if (d.N <= 16) r = launch_route_t<2>(a, st);
-  else if (d.N <= 32) r = launch_route_t<4>(a, st);
-  else r = launch_route_t<8>(a, st);
+  switch (npw) {
+    case 16: r = launch_route_t<16>(tx, tw, a, st); break;
+    case 32: r = launch_route_t<32>(tx, tw, a, st); break;
+    case 48: r = launch_route_t<48>(tx, tw, a, st); break;
+    case 64: r = launch_route_t<64>(tx, tw, a, st); break;
+    default: r = launch_route_t<80>(tx, tw, a, st); break;
+  }
   if (r != MOE_OK) return r;
-  ScanArgs sa{};
-  sa.counts_blk = a.counts_blk;
-  sa.tot = a.tot;
-  sa.bases = a.bases;
-  sa.counts = a.counts;
-  sa.offsets = a.offsets;
-  sa.ppart = a.ppart;
-  sa.hist = a.hist;
-  sa.lsq = a.lsq;
-  sa.auxp = ws_ptr<double>(ws, L.auxp);
-  sa.N = d.N;
-  sa.K = d.K;
-  sa.nblk = L.nblk;
-  sa.nparts = L.nparts;
-  scan_kernel<<<d.N + L.nparts, kScanThreads, 0, st>>>(sa);
-  return cuda_status(cudaGetLastError());
+  return launch_route_scan(d, ws, st);
 }
 
 }  // namespace moe

@@ -28,8 +28,8 @@
 namespace moe {
 
 // 8 MiB (MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES in the header). A shape needs
-// moe_workspace_bytes(dims) of it: about 0.5 MB for T = 16384, K = 4, N = 64,
-// about 5.9 MB for T = 131072, K = 8, N = 64.
+// moe_workspace_bytes(dims) of it: about 0.9 MB for T = 16384, d = 1024, K = 4,
+// N = 64, about 6.1 MB for T = 131072, d = 2048, K = 8, N = 64.
 constexpr size_t kNoAllocScratchBytes = MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES;
 
 static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];

@@ -24,8 +24,15 @@ class MoENullLayer:
     def __init__(self, d: int, N: int, M: int, K: int, F: int, F_shared: int, *,
                  w_router: torch.Tensor, router_bias: Optional[torch.Tensor],
                  w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
-                 ws_gate: torch.Tensor, ws_up: torch.Tensor, ws_down: torch.Tensor):
+                 ws_gate: torch.Tensor, ws_up: torch.Tensor, ws_down: torch.Tensor,
+                 router: str = "tensor"):
+        """router: "tensor" (router product on the tensor cores, fp32 weights split
+        exactly into three bf16 terms) or "fp32_cores" (fp32 FMA on the CUDA cores)."""
+        if router not in ("tensor", "fp32_cores"):
+            raise ValueError(f"router must be 'tensor' or 'fp32_cores', not {router!r}")
         self.d, self.N, self.M, self.K, self.F, self.F_shared = d, N, M, K, F, F_shared
+        self.router = router
+        self.flags = B.FLAG_ROUTER_FP32_CORES if router == "fp32_cores" else 0
         dev = w_router.device
         self.device = dev
         self.w_router = w_router.contiguous()
@@ -46,17 +53,18 @@ class MoENullLayer:
                                   self.shared_gate_up.data_ptr(), self.shared_down.data_ptr())
 
     @classmethod
-    def from_inputs(cls, inp, device="cuda") -> "MoENullLayer":
+    def from_inputs(cls, inp, device="cuda", router: str = "tensor") -> "MoENullLayer":
         c = inp.cfg
         f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         return cls(c.d, c.N, c.M, c.K, c.F, c.F_shared,
                    w_router=f32(inp.w_router), router_bias=f32(inp.bias),
                    w_gate=bf16_tensor(inp.w_gate, device), w_up=bf16_tensor(inp.w_up, device),
                    w_down=bf16_tensor(inp.w_down, device), ws_gate=bf16_tensor(inp.ws_gate, device),
-                   ws_up=bf16_tensor(inp.ws_up, device), ws_down=bf16_tensor(inp.ws_down, device))
+                   ws_up=bf16_tensor(inp.ws_up, device), ws_down=bf16_tensor(inp.ws_down, device),
+                   router=router)
 
     def dims(self, T: int) -> B.Dims:
-        return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared)
+        return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags)
 
     def alloc(self, T: int, logits: bool = True) -> Dict[str, torch.Tensor]:
         """Caller-owned buffers for a T-token call (R_cap = T*K rows)."""
