@@ -185,7 +185,7 @@ def workload_config(cfg, args):
                         f"F_shared={cfg.F_shared} K={cfg.K} M={cfg.M} rho={cfg.rho:.3g}",
             "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "K": cfg.K, "F": cfg.F, "F_shared": cfg.F_shared,
             "global_batch_tokens": cfg.T * args.gpus, "parallelism": f"dp{args.gpus}",
-            "router": getattr(args, "router", "tensor"),
+            "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "pair"),
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
@@ -201,6 +201,8 @@ def main():
     ap.add_argument("--config", default="qwen3_0p6b")
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"],
                     help="router product on the tensor cores (default) or the fp32 CUDA cores")
+    ap.add_argument("--ffn", default="pair", choices=["pair", "single"],
+                    help="expert GEMMs on CTA pairs where the shape allows (default) or single-CTA tiles")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")
@@ -228,7 +230,7 @@ def main():
 
     cfg = I.CONFIGS[args.config]
     inp = I.make_inputs(cfg)
-    layer = MoENullLayer.from_inputs(inp, dev, router=args.router)
+    layer = MoENullLayer.from_inputs(inp, dev, router=args.router, ffn=args.ffn)
     x = bf16_tensor(inp.x, dev)
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
     T = cfg.T
@@ -335,7 +337,9 @@ def main():
     ffn_tflops = (6.0 * d * F * R + 6.0 * d * Fs * T) / (ffn_ms * 1e9)
 
     achieved = breakdown["gate_up"]["TFLOP/s"]
-    roofline = {"kernel": "grouped gate/up SwiGLU GEMM (tcgen05)", "bound": "tensor", "achieved": achieved,
+    pair = args.ffn == "pair" and cfg.F % 128 == 0 and cfg.F_shared % 128 == 0
+    roofline = {"kernel": "grouped gate/up SwiGLU GEMM (tcgen05, %s)" % ("CTA pairs" if pair else "single CTA"),
+                "bound": "tensor", "achieved": achieved,
                 "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
                 "peak_kind": f"{peak_kind} bf16 burst", "traffic": None,
                 "flops_per_launch": flops_gu, "ms_per_launch": kms["gate_up"]}

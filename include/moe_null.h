@@ -70,13 +70,20 @@ typedef enum {
 } moe_status_t;
 
 /* Layer sizes. T tokens, model width d, N real experts, M null copies, top-K,
- * routed expert ffn width F, shared expert ffn width F_shared. flags: 0 or
- * MOE_FLAG_ROUTER_FP32_CORES. Every call of one layer (route, dispatch,
- * workspace sizing, ...) must see the same flags. */
+ * routed expert ffn width F, shared expert ffn width F_shared. flags: 0 or a
+ * combination of the MOE_FLAG_* bits below. Every call of one layer (route,
+ * dispatch, workspace sizing, ...) must see the same flags. */
 /* Router product on the fp32 CUDA cores instead of the tensor cores (see
  * moe_route). Both give logits within the fp32 dot-product error bound; this
  * path is several times slower on the router product. */
 #define MOE_FLAG_ROUTER_FP32_CORES 1u
+
+/* Expert GEMMs on single-CTA 128 x 256 tiles instead of CTA pairs (256 x 256
+ * tiles, one tcgen05 MMA shared by the two CTAs of a cluster, which the library
+ * uses where the column tiles are 256 wide: F and F_shared multiples of 128 for
+ * gate/up, d a multiple of 256 for down). Same results up to fp32 accumulation
+ * order; for comparisons and measurement. */
+#define MOE_FLAG_FFN_SINGLE_CTA 2u
 
 typedef struct moe_dims {
   int32_t T, d, N, M, K, F, F_shared;

@@ -33,17 +33,21 @@ def bf16_f64(t: torch.Tensor) -> np.ndarray:
 ROUTERS = ("tensor", "fp32_cores")
 
 
-def make_layer(inp, device="cuda", router="tensor"):
+# Both expert GEMM variants: CTA pairs (default where the shape allows) and single-CTA tiles.
+FFNS = ("pair", "single")
+
+
+def make_layer(inp, device="cuda", router="tensor", ffn="pair"):
     from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
-    layer = MoENullLayer.from_inputs(inp, device, router=router)
+    layer = MoENullLayer.from_inputs(inp, device, router=router, ffn=ffn)
     x = bf16_tensor(inp.x, device)
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(device)
     return layer, x, tnb
 
 
-def run_forward(inp, device="cuda", router="tensor"):
+def run_forward(inp, device="cuda", router="tensor", ffn="pair"):
     from token_choice_routing_b200 import binding as B
-    layer, x, tnb = make_layer(inp, device, router)
+    layer, x, tnb = make_layer(inp, device, router, ffn)
     out = layer.forward(x, tnb)
     torch.cuda.synchronize()
     st = B.get_device_status(out["workspace"])

@@ -64,9 +64,10 @@ def test_check_dims(lib):
         v.update(kw)
         assert B.check_dims(B.dims(**v)) == B.ERR_UNSUPPORTED, kw
     dm = good()
-    dm.flags = B.FLAG_ROUTER_FP32_CORES
-    assert B.check_dims(dm) == B.OK
-    for f in (2, 4, 0x80000000, B.FLAG_ROUTER_FP32_CORES | 2):
+    for f in (B.FLAG_ROUTER_FP32_CORES, B.FLAG_FFN_SINGLE_CTA, B.FLAG_ROUTER_FP32_CORES | B.FLAG_FFN_SINGLE_CTA):
+        dm.flags = f
+        assert B.check_dims(dm) == B.OK, f
+    for f in (4, 8, 0x80000000, B.FLAG_ROUTER_FP32_CORES | 4):
         dm.flags = f
         assert B.check_dims(dm) == B.ERR_INVALID_ARG, f
 

@@ -30,14 +30,15 @@ SMALL = {
 }
 
 
+@pytest.mark.parametrize("ffn", H.FFNS)
 @pytest.mark.parametrize("router", H.ROUTERS)
 @pytest.mark.parametrize("name", list(SMALL))
-def test_small_layer_full_parity(name, router):
+def test_small_layer_full_parity(name, router, ffn):
     cfg = SMALL[name]
     inp = I.make_inputs(cfg)
     if cfg.name.startswith("ragged") or cfg.name in ("k1", "n64_k16", "t1"):
         inp.bias[cfg.N] = np.float32(0.3)
-    layer, x, tnb, out = H.run_forward(inp, router=router)
+    layer, x, tnb, out = H.run_forward(inp, router=router, ffn=ffn)
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -65,12 +66,13 @@ def test_small_layer_full_parity(name, router):
     H.check_layer_output(inp, out, r)
 
 
-@pytest.mark.parametrize("name,router", [("qwen3_0p6b", "tensor"), ("qwen3_1p7b", "tensor"),
-                                         ("qwen3_0p6b", "fp32_cores")])
-def test_full_size_layer_parity_sampled(name, router):
+@pytest.mark.parametrize("name,router,ffn", [("qwen3_0p6b", "tensor", "pair"), ("qwen3_1p7b", "tensor", "pair"),
+                                             ("qwen3_0p6b", "fp32_cores", "pair"),
+                                             ("qwen3_0p6b", "tensor", "single")])
+def test_full_size_layer_parity_sampled(name, router, ffn):
     cfg = I.CONFIGS[name]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, out = H.run_forward(inp, router=router)
+    layer, x, tnb, out = H.run_forward(inp, router=router, ffn=ffn)
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)

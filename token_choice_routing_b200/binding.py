@@ -109,8 +109,10 @@ def _check(fn: str, code: int):
         raise MoEError(fn, code)
 
 
-# moe_dims_t.flags: router product on the fp32 CUDA cores instead of the tensor cores
+# moe_dims_t.flags: router product on the fp32 CUDA cores instead of the tensor cores;
+# expert GEMMs on single-CTA tiles instead of CTA pairs
 FLAG_ROUTER_FP32_CORES = 1
+FLAG_FFN_SINGLE_CTA = 2
 
 
 def dims(T, d, N, M, K, F, F_shared, flags=0) -> Dims:

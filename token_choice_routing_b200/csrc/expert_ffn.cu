@@ -457,6 +457,7 @@ static FfnPlan plan_ffn(const moe_dims_t& d, const int32_t* offsets, void* ws) {
 int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
                    const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
                    void* ws, cudaStream_t st) {
+  if (ffn_pair_gate_up_ok(d)) return launch_gate_up_pair(d, xs, x, offsets, gate_up, sgate_up, h, h_shared, ws, st);
   FfnPlan p = plan_ffn(d, offsets, ws);
   const long long rcap = (long long)d.T * d.K;
   CUtensorMap ar, br, as_, bs;
@@ -474,6 +475,7 @@ int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, c
 int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
                 const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys, uint16_t* shared_out, void* ws,
                 cudaStream_t st) {
+  if (ffn_pair_down_ok(d)) return launch_down_pair(d, offsets, h, h_shared, w_down, sdown, ys, shared_out, ws, st);
   FfnPlan p = plan_ffn(d, offsets, ws);
   const long long rcap = (long long)d.T * d.K;
   CUtensorMap ar, br, as_, bs;

@@ -17,7 +17,7 @@ namespace moe {
 // Tiling constants of the route kernel (router product on tcgen05 + routing).
 constexpr int kRouteTokens = 128;                          // tokens per route CTA (one M=128 tile)
 constexpr int kRouteBK = 64;                               // d-columns per pipeline stage
-constexpr int kRouteEpiThreads = 256;                      // 8 epilogue warps
+constexpr int kRouteEpiThreads = 512;                      // 16 epilogue warps: 4 lanes per token
 constexpr int kRouteThreads = 64 + kRouteEpiThreads;       // + TMA warp + MMA warp
 constexpr int kFp32RouteTokens = 64;                       // tokens per CTA of the fp32 CUDA-core route
 constexpr int kMaxN = 64;
@@ -131,6 +131,15 @@ int launch_route_fp32(const moe_dims_t& d, const uint16_t* x, const float* w_rou
                       int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* ws,
                       cudaStream_t st);
 int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st);
+// The expert GEMMs on CTA pairs (expert_ffn_pair.cu), for shapes with 256-wide column tiles.
+bool ffn_pair_gate_up_ok(const moe_dims_t& d);
+bool ffn_pair_down_ok(const moe_dims_t& d);
+int launch_gate_up_pair(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                        const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
+                        void* ws, cudaStream_t st);
+int launch_down_pair(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
+                     const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys, uint16_t* shared_out, void* ws,
+                     cudaStream_t st);
 int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_idx, void* ws,
                     int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* slot_row,
                     uint16_t* xs, int32_t* counts_ext, float* P, float* losses,
@@ -311,6 +320,72 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// ---- thread-block clusters of two CTAs (a CTA pair sharing one tcgen05 MMA)
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier that may live in the other CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA tile load into this CTA's shared memory whose completion is counted on a
+// barrier that may live in the other CTA of the pair (the pair's leader).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cluster, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem] (+)= A * B^T over the pair: M = 256 (128 rows of A in each CTA), N
+// from idesc with N/2 rows of B in each CTA; each CTA's TMEM holds its 128 rows.
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on a barrier (own or peer CTA) when this thread's prior pair MMAs finish.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }

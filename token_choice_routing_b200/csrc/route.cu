@@ -28,7 +28,7 @@
 // Layout: one CTA = 128 tokens x all N+1 logits (one M=128 tile). Warp 0
 // issues TMA loads of the x tile (128 x 64 bf16) and the split weight tile
 // (3*NPW x 64 bf16) into a 4-stage ring; warp 1 issues the MMAs (M=128,
-// N=3*NPW, K=16) from one thread into TMEM; warps 2-9 add the three terms per
+// N=3*NPW, K=16) from one thread into TMEM; warps 2-17 add the three terms per
 // logit, then route the 128 tokens with 4 lanes per token.
 #include "moe_internal.cuh"
 
@@ -74,9 +74,13 @@ __device__ __forceinline__ void split3(float w, uint16_t& h, uint16_t& m, uint16
   l = __bfloat16_as_ushort(bl);
 }
 
-// One thread per 8 d-columns of one padded row.
+// One thread per 8 d-columns of one padded row. Block 0 also clears the first
+// `nclear` words of the workspace header (status word and per-expert totals),
+// which must start at zero for every layer call.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, uint16_t* __restrict__ w3,
-                                                           int N, int npw, int d) {
+                                                           int N, int npw, int d, uint32_t* hdr, int nclear) {
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nclear; i += blockDim.x) hdr[i] = 0u;
   const int nch = d >> 3;
   const long long total = (long long)npw * nch;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
@@ -122,12 +126,12 @@ struct RouteSmem {
   static constexpr size_t off_s = 0;  // float [128][LS]: logits, then p in place
   static constexpr size_t off_pn = off_s + sizeof(float) * kRouteTokens * LS;  // float [128] null p
   static constexpr size_t off_lse2 = off_pn + sizeof(float) * kRouteTokens;    // float [128]
-  static constexpr size_t off_nul = off_lse2 + sizeof(float) * kRouteTokens;   // int [128]
-  static constexpr size_t off_mask = align_up(off_nul + sizeof(int) * kRouteTokens, 16);  // u64 [128]
+  static constexpr size_t off_mask = align_up(off_lse2 + sizeof(float) * kRouteTokens, 16);  // u64 [128]
   static constexpr size_t off_tk = off_mask + sizeof(unsigned long long) * kRouteTokens;  // int [128][kMaxK]
   static constexpr size_t off_tkv = off_tk + sizeof(int) * kRouteTokens * kMaxK;          // float [128][kMaxK]
   static constexpr size_t off_tokbits = off_tkv + sizeof(float) * kRouteTokens * kMaxK;  // u32 [4][kMaxN]
-  static constexpr size_t scratch_end = off_tokbits + sizeof(unsigned) * 4 * kMaxN;
+  static constexpr size_t off_hist = off_tokbits + sizeof(unsigned) * 4 * kMaxN;         // int [kMaxK+1]
+  static constexpr size_t scratch_end = off_hist + sizeof(int) * (kMaxK + 1);
   static_assert(scratch_end <= ring_end, "routing scratch must fit in the staging ring");
   static constexpr size_t off_bar = ring_end;  // full[STAGES], empty[STAGES], tfull
   static constexpr size_t off_misc = off_bar + 8 * (2 * STAGES + 1);  // [0] TMEM base, [1] abort
@@ -155,7 +159,7 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
 }
 
 // ---------------------------------------------------------------------------------------
-// One CTA: tokens [128 b, 128 b + 128) x all N+1 logits, 320 threads.
+// One CTA: tokens [128 b, 128 b + 128) x all N+1 logits, 576 threads.
 template <int NPW>
 __global__ void __launch_bounds__(kRouteThreads, 1)
     route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -249,30 +253,31 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       (void)mbar_wait_bounded(tfull_bar, 0, a.limit_ns, nullptr, a.hdr);
     }
   } else {
-    // ------------------------------ epilogue warps 2..9
-    const int etid = threadIdx.x - 64;
-    const int ew = warp - 2;
+    // ------------------------------ epilogue warps 2..17
+    const int etid = threadIdx.x - 64;  // 0..511
+    const int ew = warp - 2;            // 0..15
     float* s_l = reinterpret_cast<float*>(base + SM::off_s);
     float* pn = reinterpret_cast<float*>(base + SM::off_pn);
     float* lse2 = reinterpret_cast<float*>(base + SM::off_lse2);
-    int* nul = reinterpret_cast<int*>(base + SM::off_nul);
     unsigned long long* mask = reinterpret_cast<unsigned long long*>(base + SM::off_mask);
     int* tk = reinterpret_cast<int*>(base + SM::off_tk);
     float* tkv = reinterpret_cast<float*>(base + SM::off_tkv);
     unsigned* tokbits = reinterpret_cast<unsigned*>(base + SM::off_tokbits);  // [4][kMaxN]
+    int* s_hist = reinterpret_cast<int*>(base + SM::off_hist);                // [kMaxK+1]
 
     const bool ok = mbar_wait_bounded(tfull_bar, 0, a.limit_ns, abort_flag, a.hdr) && *abort_flag == 0;
     const bool run = named_bar_and(1, kRouteEpiThreads, ok);
     if (run) {
       // ---- logits from TMEM: warp reads lane quarter q (tokens 32q..32q+31) and
-      // one half of the NPW columns; s_j = (hi_j + mid_j) + lo_j (+ bias)
+      // every fourth 8-column chunk; s_j = (hi_j + mid_j) + lo_j (+ bias)
       tc_fence_after();
-      const int q = warp & 3, hh = ew >> 2;
+      const int q = warp & 3, part = ew >> 2;
       const int t = q * 32 + lane;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
       const float tn = (a.tnb != nullptr && t < nvalid) ? __ldg(a.tnb + tok0 + t) : 0.f;
+      if (etid <= kMaxK) s_hist[etid] = 0;  // the staging ring is free from here on
 #pragma unroll 1
-      for (int c0 = hh * (NPW / 2); c0 < (hh + 1) * (NPW / 2); c0 += 8) {
+      for (int c0 = part * 8; c0 < NPW; c0 += 32) {
         uint32_t rh[8], rm[8], rl[8];
         tmem_ld8(tb + (uint32_t)c0, rh);
         tmem_ld8(tb + (uint32_t)(NPW + c0), rm);
@@ -293,176 +298,168 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     named_bar_sync(1, kRouteEpiThreads);
 
     if (run) {
-      // ---- per-token routing, 4 lanes per token, two passes of 64 tokens
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        const int t = pass * 64 + (etid >> 2), q = etid & 3;
-        const bool valid = t < nvalid;
-        const int tok = tok0 + t;
-        float* row = s_l + t * LS;
-        const float sn = row[N];
-        float v[NQ];
+      // ---- per-token routing, 4 lanes per token (lane q holds reals q, q+4, ...)
+      const int t = etid >> 2, q = etid & 3;
+      const bool valid = t < nvalid;
+      const int tok = tok0 + t;
+      float* row = s_l + t * LS;
+      const float sn = row[N];
+      float v[NQ];
+#pragma unroll
+      for (int u = 0; u < NQ; ++u) {
+        const int i = q + 4 * u;
+        v[u] = (i < N) ? row[i] : -INFINITY;
+      }
+      // softmax statistics over the pool (M copies of the null logit)
+      float m = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < NQ; ++u) m = fmaxf(m, v[u]);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      if (M > 0) m = fmaxf(m, sn);
+      float e[NQ];
+      float z = 0.f;
+#pragma unroll
+      for (int u = 0; u < NQ; ++u) {
+        e[u] = (q + 4 * u < N) ? expf(v[u] - m) : 0.f;
+        z += e[u];
+      }
+      z += __shfl_xor_sync(0xffffffffu, z, 1);
+      z += __shfl_xor_sync(0xffffffffu, z, 2);
+      const float en = (M > 0) ? expf(sn - m) : 0.f;
+      const float Z = (M > 0) ? z + (float)M * en : z;
+      const float lse = m + logf(Z);
+      // p_i = e^{s_i - lse} evaluated as e^{s_i - m} / Z (no cancellation when |m| is
+      // large), written over this lane's own logits
+#pragma unroll
+      for (int u = 0; u < NQ; ++u) {
+        const int i = q + 4 * u;
+        if (i < N) row[i] = e[u] / Z;
+      }
+      if (q == 0) {
+        pn[t] = (M > 0) ? en / Z : 0.f;
+        lse2[t] = lse * lse;
+      }
+
+      // top-K over the pool, in rank order: K rounds of "best remaining real"
+      // against the null logit (a real equal to it wins: lower index)
+      unsigned sel = 0u;
+      int used = 0, r = 0;
+      unsigned long long msk = 0ull;
+      for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY;
+        int bi = INT_MAX;
 #pragma unroll
         for (int u = 0; u < NQ; ++u) {
           const int i = q + 4 * u;
-          v[u] = (i < N) ? row[i] : -INFINITY;
+          if (i < N && !((sel >> u) & 1u) && ranks_before(v[u], i, bv, bi)) {
+            bv = v[u];
+            bi = i;
+          }
         }
-        // softmax statistics over the pool (M copies of the null logit)
-        float m = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < NQ; ++u) m = fmaxf(m, v[u]);
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        if (M > 0) m = fmaxf(m, sn);
-        float z = 0.f;
-#pragma unroll
-        for (int u = 0; u < NQ; ++u)
-          if (q + 4 * u < N) z += expf(v[u] - m);
-        z += __shfl_xor_sync(0xffffffffu, z, 1);
-        z += __shfl_xor_sync(0xffffffffu, z, 2);
-        const float Z = (M > 0) ? z + (float)M * expf(sn - m) : z;
-        const float lse = m + logf(Z);
-        // p_i = e^{s_i - lse} evaluated as e^{s_i - m} / Z (no cancellation when |m| is
-        // large), written over this lane's own logits
-#pragma unroll
-        for (int u = 0; u < NQ; ++u) {
-          const int i = q + 4 * u;
-          if (i < N) row[i] = expf(v[u] - m) / Z;
+        for (int off = 1; off <= 2; off <<= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ranks_before(ov, oi, bv, bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        const bool take_null = (used < M) && (bi == INT_MAX || bv < sn);
+        int id;
+        if (take_null) {
+          id = N + used;
+          ++used;
+        } else {
+          id = bi;
+          ++r;
+          msk |= 1ull << bi;
+          if ((bi & 3) == q) sel |= 1u << (bi >> 2);
         }
         if (q == 0) {
-          pn[t] = (M > 0) ? expf(sn - m) / Z : 0.f;
-          lse2[t] = lse * lse;
+          tk[t * kMaxK + k] = id;
+          tkv[t * kMaxK + k] = bv;
         }
-
-        // top-K over the pool, in rank order: K rounds of "best remaining real"
-        // against the null logit (a real equal to it wins: lower index)
-        unsigned sel = 0u;
-        int used = 0, r = 0;
-        unsigned long long msk = 0ull;
-        for (int k = 0; k < K; ++k) {
-          float bv = -INFINITY;
-          int bi = INT_MAX;
+      }
+      __syncwarp();
+      if (valid) {
+        if (q == 0) {
+          // gates: softmax over the selected real logits (rank order: first real is the max)
+          float smax = 0.f, gsum = 0.f;
+          bool first = true;
+          for (int k = 0; k < K; ++k) {
+            if (tk[t * kMaxK + k] < N) {
+              const float sv = tkv[t * kMaxK + k];
+              if (first) {
+                smax = sv;
+                first = false;
+              }
+              gsum += expf(sv - smax);
+            }
+          }
+          for (int k = 0; k < K; ++k) {
+            const int id = tk[t * kMaxK + k];
+            const float g = (id < N) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
+            a.topk_idx[(size_t)tok * K + k] = id;
+            a.topk_gate[(size_t)tok * K + k] = g;
+          }
+          a.n_real[tok] = r;
+          atomicAdd(s_hist + (K - r), 1);  // integer: the histogram does not depend on the order
+        }
+        mask[t] = msk;  // identical on the token's four lanes
+        if (a.logits) {
+          float* lo = a.logits + (size_t)tok * (N + 1);
 #pragma unroll
           for (int u = 0; u < NQ; ++u) {
             const int i = q + 4 * u;
-            if (i < N && !((sel >> u) & 1u) && ranks_before(v[u], i, bv, bi)) {
-              bv = v[u];
-              bi = i;
-            }
+            if (i < N) lo[i] = v[u];
           }
-#pragma unroll
-          for (int off = 1; off <= 2; off <<= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ranks_before(ov, oi, bv, bi)) {
-              bv = ov;
-              bi = oi;
-            }
-          }
-          const bool take_null = (used < M) && (bi == INT_MAX || bv < sn);
-          int id;
-          if (take_null) {
-            id = N + used;
-            ++used;
-          } else {
-            id = bi;
-            ++r;
-            msk |= 1ull << bi;
-            if ((bi & 3) == q) sel |= 1u << (bi >> 2);
-          }
-          if (q == 0) {
-            tk[t * kMaxK + k] = id;
-            tkv[t * kMaxK + k] = bv;
-          }
-        }
-        __syncwarp();
-        if (valid) {
-          if (q == 0) {
-            // gates: softmax over the selected real logits (rank order: first real is the max)
-            float smax = 0.f, gsum = 0.f;
-            bool first = true;
-            for (int k = 0; k < K; ++k) {
-              if (tk[t * kMaxK + k] < N) {
-                const float sv = tkv[t * kMaxK + k];
-                if (first) {
-                  smax = sv;
-                  first = false;
-                }
-                gsum += expf(sv - smax);
-              }
-            }
-            for (int k = 0; k < K; ++k) {
-              const int id = tk[t * kMaxK + k];
-              const float g = (id < N) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
-              a.topk_idx[(size_t)tok * K + k] = id;
-              a.topk_gate[(size_t)tok * K + k] = g;
-            }
-            a.n_real[tok] = r;
-            nul[t] = K - r;
-            mask[t] = msk;
-          }
-          if (a.logits) {
-            float* lo = a.logits + (size_t)tok * (N + 1);
-#pragma unroll
-            for (int u = 0; u < NQ; ++u) {
-              const int i = q + 4 * u;
-              if (i < N) lo[i] = v[u];
-            }
-            if (q == 0) lo[N] = sn;
-          }
+          if (q == 0) lo[N] = sn;
         }
       }
     }
     named_bar_sync(1, kRouteEpiThreads);
 
     if (run) {
-      // ---- block statistics. Warps 2..5: for each expert e, ballot bit e of the
-      // selection masks of 32 tokens, giving the block's tokens that chose e as a
-      // 128-bit set (a slot's rank is the number of earlier tokens in that set).
-      // Warps 6..9: probability column sums, the null-count histogram and the
-      // sum of lse^2 over the block, each in a fixed order.
-      if (ew < 4) {
-        const int t = 32 * ew + lane;
-        const unsigned long long mk = (t < nvalid) ? mask[t] : 0ull;
-        for (int e = 0; e < N; ++e) {
+      // ---- block statistics. Ballots: warp ew takes the 32 tokens of group ew & 3
+      // and experts [16 (ew >> 2), +16); bit e of the selection masks gives the
+      // block's tokens that chose e as a 128-bit set (a slot's rank is the number
+      // of earlier tokens in it). Column sums of p and the sum of lse^2: lane l
+      // adds tokens l, l+32, l+64, l+96 in that order, then a butterfly over the
+      // warp (every lane ends with the same, order-fixed total).
+      {
+        const int g = ew & 3;
+        const int tt = 32 * g + lane;
+        const unsigned long long mk = (tt < nvalid) ? mask[tt] : 0ull;
+        const int e1 = min(N, 16 * (ew >> 2) + 16);
+        for (int e = 16 * (ew >> 2); e < e1; ++e) {
           const unsigned bits = __ballot_sync(0xffffffffu, (mk >> e) & 1ull);
-          if (lane == 0) tokbits[ew * kMaxN + e] = bits;
+          if (lane == 0) tokbits[g * kMaxN + e] = bits;
         }
-      } else {
-        const int c = etid - 128;
-        if (c <= N) {
-          const float* col = (c < N) ? s_l + c : pn;
-          const int stride = (c < N) ? LS : 1;
-          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-          int t = 0;
-          for (; t + 4 <= nvalid; t += 4) {
-            s0 += col[t * stride];
-            s1 += col[(t + 1) * stride];
-            s2 += col[(t + 2) * stride];
-            s3 += col[(t + 3) * stride];
-          }
-          for (; t < nvalid; ++t) s0 += col[t * stride];
-          a.ppart[(size_t)b * (N + 1) + c] = (s0 + s1) + (s2 + s3);
-        } else if (c <= N + K + 1) {
-          const int h = c - N - 1;
-          int cnt = 0;
-          for (int t = 0; t < nvalid; ++t) cnt += (nul[t] == h);
-          a.hist[(size_t)b * (K + 1) + h] = cnt;
-        } else if (c == N + K + 2) {
-          float s0 = 0.f, s1 = 0.f;
-          int t = 0;
-          for (; t + 2 <= nvalid; t += 2) {
-            s0 += lse2[t];
-            s1 += lse2[t + 1];
-          }
-          if (t < nvalid) s0 += lse2[t];
-          a.lsq[b] = s0 + s1;
+      }
+      for (int c = ew; c <= N + 1; c += 16) {
+        // c < N: real column c; c == N: the null probability; c == N + 1: lse^2
+        const float* col = (c < N) ? s_l + c : (c == N) ? pn : lse2;
+        const int stride = (c < N) ? LS : 1;
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tt = lane + 32 * i;
+          if (tt < nvalid) sum += col[tt * stride];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) {
+          if (c <= N) a.ppart[(size_t)b * (N + 1) + c] = sum;
+          else a.lsq[b] = sum;
         }
       }
     }
     named_bar_sync(1, kRouteEpiThreads);
 
     if (run) {
+      if (etid <= K) a.hist[(size_t)b * (K + 1) + etid] = s_hist[etid];
       if (etid < N) {
         int cnt = 0;
 #pragma unroll
@@ -471,21 +468,18 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         if (cnt) atomicAdd(a.tot + etid, cnt);
       }
       // lrank for (token, slot): 4 threads per token, slots k = q, q+4, ...
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        const int t = pass * 64 + (etid >> 2), q = etid & 3;
-        if (t < nvalid) {
-          const int w = t >> 5;
-          const unsigned below = (1u << (t & 31)) - 1u;
-          for (int k = q; k < K; k += 4) {
-            const int id = tk[t * kMaxK + k];
-            int rank = -1;
-            if (id < N) {
-              rank = __popc(tokbits[w * kMaxN + id] & below);
-              for (int w2 = 0; w2 < w; ++w2) rank += __popc(tokbits[w2 * kMaxN + id]);
-            }
-            a.lrank[(size_t)(tok0 + t) * K + k] = rank;
+      const int t = etid >> 2, q = etid & 3;
+      if (t < nvalid) {
+        const int w = t >> 5;
+        const unsigned below = (1u << (t & 31)) - 1u;
+        for (int k = q; k < K; k += 4) {
+          const int id = tk[t * kMaxK + k];
+          int rank = -1;
+          if (id < N) {
+            rank = __popc(tokbits[w * kMaxN + id] & below);
+            for (int w2 = 0; w2 < w; ++w2) rank += __popc(tokbits[w2 * kMaxN + id]);
           }
+          a.lrank[(size_t)(tok0 + t) * K + k] = rank;
         }
       }
     }
@@ -661,18 +655,16 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.M = d.M;
   a.K = d.K;
   a.nblk = L.nblk;
-  // the status word and the per-expert totals start at zero for every layer call
-  cudaError_t e = cudaMemsetAsync(a.hdr, 0, kHdrTotOffset + sizeof(int32_t) * d.N, st);
-  if (e != cudaSuccess) return cuda_status(e);
-
-  // the split router weight for this call, then tensor maps over x and it
+  // the split router weight for this call (its block 0 also clears the status word
+  // and the per-expert totals), then tensor maps over x and it
   const int npw = route_npw(d.N);
   uint16_t* w3 = ws_ptr<uint16_t>(ws, L.wprep);
   {
     const long long work = (long long)npw * (d.d / 8);
     long long grid = (work + 255) / 256;
     if (grid > (long long)sm_count() * 8) grid = (long long)sm_count() * 8;
-    router_split_kernel<<<(int)grid, 256, 0, st>>>(w_router, w3, d.N, npw, d.d);
+    const int nclear = (int)((kHdrTotOffset + sizeof(int32_t) * d.N) / sizeof(uint32_t));
+    router_split_kernel<<<(int)grid, 256, 0, st>>>(w_router, w3, d.N, npw, d.d, a.hdr, nclear);
     const int r = cuda_status(cudaGetLastError());
     if (r != MOE_OK) return r;
   }

@@ -25,14 +25,19 @@ class MoENullLayer:
                  w_router: torch.Tensor, router_bias: Optional[torch.Tensor],
                  w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
                  ws_gate: torch.Tensor, ws_up: torch.Tensor, ws_down: torch.Tensor,
-                 router: str = "tensor"):
+                 router: str = "tensor", ffn: str = "pair"):
         """router: "tensor" (router product on the tensor cores, fp32 weights split
-        exactly into three bf16 terms) or "fp32_cores" (fp32 FMA on the CUDA cores)."""
+        exactly into three bf16 terms) or "fp32_cores" (fp32 FMA on the CUDA cores).
+        ffn: "pair" (expert GEMMs on CTA pairs where the shape allows) or "single"
+        (single-CTA tiles everywhere)."""
         if router not in ("tensor", "fp32_cores"):
             raise ValueError(f"router must be 'tensor' or 'fp32_cores', not {router!r}")
+        if ffn not in ("pair", "single"):
+            raise ValueError(f"ffn must be 'pair' or 'single', not {ffn!r}")
         self.d, self.N, self.M, self.K, self.F, self.F_shared = d, N, M, K, F, F_shared
-        self.router = router
-        self.flags = B.FLAG_ROUTER_FP32_CORES if router == "fp32_cores" else 0
+        self.router, self.ffn = router, ffn
+        self.flags = ((B.FLAG_ROUTER_FP32_CORES if router == "fp32_cores" else 0) |
+                      (B.FLAG_FFN_SINGLE_CTA if ffn == "single" else 0))
         dev = w_router.device
         self.device = dev
         self.w_router = w_router.contiguous()
@@ -53,7 +58,7 @@ class MoENullLayer:
                                   self.shared_gate_up.data_ptr(), self.shared_down.data_ptr())
 
     @classmethod
-    def from_inputs(cls, inp, device="cuda", router: str = "tensor") -> "MoENullLayer":
+    def from_inputs(cls, inp, device="cuda", router: str = "tensor", ffn: str = "pair") -> "MoENullLayer":
         c = inp.cfg
         f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         return cls(c.d, c.N, c.M, c.K, c.F, c.F_shared,
@@ -61,7 +66,7 @@ class MoENullLayer:
                    w_gate=bf16_tensor(inp.w_gate, device), w_up=bf16_tensor(inp.w_up, device),
                    w_down=bf16_tensor(inp.w_down, device), ws_gate=bf16_tensor(inp.ws_gate, device),
                    ws_up=bf16_tensor(inp.ws_up, device), ws_down=bf16_tensor(inp.ws_down, device),
-                   router=router)
+                   router=router, ffn=ffn)
 
     def dims(self, T: int) -> B.Dims:
         return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags)

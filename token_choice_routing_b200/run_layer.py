@@ -1,7 +1,7 @@
 """Run a few forwards of one seeded workload through the C ABI.
 
     python -m token_choice_routing_b200.run_layer [--config qwen3_0p6b] [--forwards 3]
-        [--router tensor|fp32_cores]
+        [--router tensor|fp32_cores] [--ffn pair|single]
 
 Used as the target of profiler captures (ncu -k <kernel> -s/-c selects the
 launch). Exits non-zero if the device status word reports an error.
@@ -21,9 +21,10 @@ def main(argv=None) -> int:
     ap.add_argument("--config", default="qwen3_0p6b", choices=sorted(I.CONFIGS))
     ap.add_argument("--forwards", type=int, default=3)
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"])
+    ap.add_argument("--ffn", default="pair", choices=["pair", "single"])
     a = ap.parse_args(argv)
     inp = I.make_inputs(I.CONFIGS[a.config])
-    layer = MoENullLayer.from_inputs(inp, "cuda", router=a.router)
+    layer = MoENullLayer.from_inputs(inp, "cuda", router=a.router, ffn=a.ffn)
     x = bf16_tensor(inp.x, "cuda")
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).cuda()
     out = layer.alloc(inp.cfg.T, logits=False)
