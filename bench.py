@@ -185,7 +185,7 @@ def workload_config(cfg, args):
                         f"F_shared={cfg.F_shared} K={cfg.K} M={cfg.M} rho={cfg.rho:.3g}",
             "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "K": cfg.K, "F": cfg.F, "F_shared": cfg.F_shared,
             "global_batch_tokens": cfg.T * args.gpus, "parallelism": f"dp{args.gpus}",
-            "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "pair"),
+            "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "single"),
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
@@ -201,8 +201,8 @@ def main():
     ap.add_argument("--config", default="qwen3_0p6b")
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"],
                     help="router product on the tensor cores (default) or the fp32 CUDA cores")
-    ap.add_argument("--ffn", default="pair", choices=["pair", "single"],
-                    help="expert GEMMs on CTA pairs where the shape allows (default) or single-CTA tiles")
+    ap.add_argument("--ffn", default="single", choices=["single", "pair"],
+                    help="expert GEMMs on single-CTA tiles (default) or CTA pairs where the shape allows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")

@@ -78,12 +78,14 @@ typedef enum {
  * path is several times slower on the router product. */
 #define MOE_FLAG_ROUTER_FP32_CORES 1u
 
-/* Expert GEMMs on single-CTA 128 x 256 tiles instead of CTA pairs (256 x 256
- * tiles, one tcgen05 MMA shared by the two CTAs of a cluster, which the library
- * uses where the column tiles are 256 wide: F and F_shared multiples of 128 for
- * gate/up, d a multiple of 256 for down). Same results up to fp32 accumulation
- * order; for comparisons and measurement. */
-#define MOE_FLAG_FFN_SINGLE_CTA 2u
+/* Expert GEMMs on CTA pairs: 256 x 256 tiles, one tcgen05 MMA shared by the
+ * two CTAs of a cluster, where the column tiles are 256 wide (F and F_shared
+ * multiples of 128 for gate/up, d a multiple of 256 for down); otherwise, and
+ * by default, single-CTA 128 x 256 tiles. A pair loads a third less operand
+ * data per flop but rounds each expert's rows up to 256 instead of 128; on
+ * this part it is ahead only when experts hold thousands of rows. Same results
+ * up to fp32 accumulation order. */
+#define MOE_FLAG_FFN_CTA_PAIR 2u
 
 typedef struct moe_dims {
   int32_t T, d, N, M, K, F, F_shared;

@@ -33,11 +33,11 @@ def bf16_f64(t: torch.Tensor) -> np.ndarray:
 ROUTERS = ("tensor", "fp32_cores")
 
 
-# Both expert GEMM variants: CTA pairs (default where the shape allows) and single-CTA tiles.
-FFNS = ("pair", "single")
+# Both expert GEMM variants: single-CTA tiles (default) and CTA pairs.
+FFNS = ("single", "pair")
 
 
-def make_layer(inp, device="cuda", router="tensor", ffn="pair"):
+def make_layer(inp, device="cuda", router="tensor", ffn="single"):
     from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
     layer = MoENullLayer.from_inputs(inp, device, router=router, ffn=ffn)
     x = bf16_tensor(inp.x, device)
@@ -45,7 +45,7 @@ def make_layer(inp, device="cuda", router="tensor", ffn="pair"):
     return layer, x, tnb
 
 
-def run_forward(inp, device="cuda", router="tensor", ffn="pair"):
+def run_forward(inp, device="cuda", router="tensor", ffn="single"):
     from token_choice_routing_b200 import binding as B
     layer, x, tnb = make_layer(inp, device, router, ffn)
     out = layer.forward(x, tnb)

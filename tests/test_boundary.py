@@ -64,7 +64,7 @@ def test_check_dims(lib):
         v.update(kw)
         assert B.check_dims(B.dims(**v)) == B.ERR_UNSUPPORTED, kw
     dm = good()
-    for f in (B.FLAG_ROUTER_FP32_CORES, B.FLAG_FFN_SINGLE_CTA, B.FLAG_ROUTER_FP32_CORES | B.FLAG_FFN_SINGLE_CTA):
+    for f in (B.FLAG_ROUTER_FP32_CORES, B.FLAG_FFN_CTA_PAIR, B.FLAG_ROUTER_FP32_CORES | B.FLAG_FFN_CTA_PAIR):
         dm.flags = f
         assert B.check_dims(dm) == B.OK, f
     for f in (4, 8, 0x80000000, B.FLAG_ROUTER_FP32_CORES | 4):

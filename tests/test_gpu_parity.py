@@ -66,9 +66,9 @@ def test_small_layer_full_parity(name, router, ffn):
     H.check_layer_output(inp, out, r)
 
 
-@pytest.mark.parametrize("name,router,ffn", [("qwen3_0p6b", "tensor", "pair"), ("qwen3_1p7b", "tensor", "pair"),
-                                             ("qwen3_0p6b", "fp32_cores", "pair"),
-                                             ("qwen3_0p6b", "tensor", "single")])
+@pytest.mark.parametrize("name,router,ffn", [("qwen3_0p6b", "tensor", "single"), ("qwen3_1p7b", "tensor", "single"),
+                                             ("qwen3_0p6b", "fp32_cores", "single"),
+                                             ("qwen3_0p6b", "tensor", "pair")])
 def test_full_size_layer_parity_sampled(name, router, ffn):
     cfg = I.CONFIGS[name]
     inp = I.make_inputs(cfg)

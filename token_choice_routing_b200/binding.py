@@ -110,9 +110,9 @@ def _check(fn: str, code: int):
 
 
 # moe_dims_t.flags: router product on the fp32 CUDA cores instead of the tensor cores;
-# expert GEMMs on single-CTA tiles instead of CTA pairs
+# expert GEMMs on CTA pairs instead of single-CTA tiles
 FLAG_ROUTER_FP32_CORES = 1
-FLAG_FFN_SINGLE_CTA = 2
+FLAG_FFN_CTA_PAIR = 2
 
 
 def dims(T, d, N, M, K, F, F_shared, flags=0) -> Dims:

@@ -19,6 +19,7 @@ __global__ void __launch_bounds__(kCombineThreads, 3)
 combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
                const float* __restrict__ gate, const int32_t* __restrict__ slot_row,
                uint16_t* __restrict__ y, int T, int d, int K, long long rcap, uint32_t* status) {
+  pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const int wpb = kCombineThreads / 32;
   const int nch = d >> 3;
@@ -113,9 +114,8 @@ int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shar
   int grid = (d.T + wpb - 1) / wpb;
   const int cap = sm_count() * occ;
   if (grid > cap) grid = cap;
-  combine_kernel<<<grid, kCombineThreads, 0, st>>>(ys, shared_out, topk_gate, slot_row, y, d.T, d.d, d.K,
-                                                   (long long)d.T * d.K, nullptr);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(combine_kernel, dim3(grid), dim3(kCombineThreads), 0, st, ys, shared_out, topk_gate, slot_row,
+                    y, d.T, d.d, d.K, (long long)d.T * d.K, nullptr);
 }
 
 }  // namespace moe

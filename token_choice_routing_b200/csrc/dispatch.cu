@@ -85,6 +85,7 @@ __device__ void aux_finalize_block(const double* sums, int N, int M, int K, int3
 
 __global__ void __launch_bounds__(256) aux_kernel(AuxPtrs p, double* sums_out, const double* sums_in,
                                                   int32_t* counts_ext, float* P, float* losses) {
+  pdl_wait_then_release();
   __shared__ double s_sums[kMaxN + kMaxK + 1 + kMaxN + 1 + 2];
   const int n = p.N + (p.K + 1) + (p.N + 1) + 2;
   if (sums_in == nullptr) {
@@ -124,6 +125,7 @@ struct DispatchArgs {
 constexpr int kDispatchThreads = 256;
 
 __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs a) {
+  pdl_wait_then_release();
   int blk = blockIdx.x;
   if (a.fuse_aux) {
     if (blk == 0) {  // scheduled first, so the reduction overlaps the gather
@@ -225,14 +227,13 @@ int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_
   int grid = (d.T + wpb - 1) / wpb;
   const int cap = sm_count() * 8;
   if (grid > cap) grid = cap;
-  dispatch_kernel<<<grid + 1, kDispatchThreads, 0, st>>>(a);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(dispatch_kernel, dim3(grid + 1), dim3(kDispatchThreads), 0, st, a);
 }
 
 int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const double* sums_in,
                int32_t* counts_ext, float* P, float* losses, cudaStream_t st) {
-  aux_kernel<<<1, 256, 0, st>>>(aux_ptrs(d, ws), sums_out, sums_in, counts_ext, P, losses);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(aux_kernel, dim3(1), dim3(256), 0, st, aux_ptrs(d, ws), sums_out, sums_in, counts_ext, P,
+                    losses);
 }
 
 // ---------------------------------------------------------------------------------------

@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
                     const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s,
                     const GemmArgs a) {
+  pdl_wait_then_release();
   using SM = GemmSmem<BN>;
   constexpr int OUTC = SWIGLU ? BN / 2 : BN;  // output columns per tile
   constexpr int NCHUNK = OUTC / 64;
@@ -330,6 +331,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
 // Gate/up packing: 64-row panels, gate panel then the matching up panel.
 __global__ void pack_gate_up_kernel(const uint16_t* __restrict__ wg, const uint16_t* __restrict__ wu,
                                     uint16_t* __restrict__ out, int groups, int F, int d) {
+  pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const long long rows = (long long)groups * 2 * F;
   const int nch = d >> 3;
@@ -349,13 +351,12 @@ int launch_pack_gate_up(const moe_dims_t& d, const uint16_t* w_gate, const uint1
                         uint16_t* sgate_up, cudaStream_t st) {
   const int grid = sm_count() * 8;
   if (gate_up) {
-    pack_gate_up_kernel<<<grid, 256, 0, st>>>(w_gate, w_up, gate_up, d.N, d.F, d.d);
-    int r = cuda_status(cudaGetLastError());
+    int r = launch_pdl(pack_gate_up_kernel, dim3(grid), dim3(256), 0, st, w_gate, w_up, gate_up, d.N, d.F, d.d);
     if (r != MOE_OK) return r;
   }
   if (sgate_up) {
-    pack_gate_up_kernel<<<grid, 256, 0, st>>>(ws_gate, ws_up, sgate_up, 1, d.F_shared, d.d);
-    int r = cuda_status(cudaGetLastError());
+    int r = launch_pdl(pack_gate_up_kernel, dim3(grid), dim3(256), 0, st, ws_gate, ws_up, sgate_up, 1, d.F_shared,
+                       d.d);
     if (r != MOE_OK) return r;
   }
   return MOE_OK;
@@ -407,8 +408,8 @@ static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   long long grid = sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid < 1) grid = 1;
-  grouped_gemm_kernel<BN, SWIGLU><<<(int)grid, kGemmThreads, SM::bytes, st>>>(ar, br, as_, bs, a);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(grouped_gemm_kernel<BN, SWIGLU>, dim3((unsigned)grid), dim3(kGemmThreads), SM::bytes, st, ar, br,
+                    as_, bs, a);
 }
 
 struct FfnPlan {

@@ -19,6 +19,11 @@
 // or a plain conversion, bf16 rows staged in shared memory, coalesced stores
 // masked at the expert's last row (rows past it are computed, never stored).
 //
+// Selected with MOE_FLAG_FFN_CTA_PAIR. Measured on the 16K-token workloads it
+// is not faster than the 1-CTA kernel: both are held by the L2 output rate,
+// which the 1-CTA kernel's concurrent reads of the same tiles already share,
+// and pair tiles round each expert up to 256 rows.
+//
 // Roles (192 threads per CTA, both CTAs): warp 0 lane 0 issues TMA loads into
 // its own CTA's 6-stage ring and counts them on the leader's full barrier;
 // warp 1 allocates TMEM (cta_group::2, 2 x 256 columns) and, in the leader only,
@@ -74,6 +79,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
                              const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s,
                              const PairArgs a) {
+  pdl_wait_then_release();
   using SM = PairSmem;
   constexpr int OUTC = SWIGLU ? kQN / 2 : kQN;  // output columns per tile
   constexpr int NCHUNK = OUTC / 64;
@@ -345,16 +351,18 @@ static int launch_pair(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   cudaGetDevice(&dev);
   auto kern = grouped_gemm_pair_kernel<SWIGLU>;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = PairSmem::bytes;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
   if (dev >= 0 && dev < 64 && clusters[dev] == 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PairSmem::bytes);
     if (e != cudaSuccess) return cuda_status(e);
@@ -368,6 +376,7 @@ static int launch_pair(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   if (max_tiles < np) np = max_tiles;
   if (np < 1) np = 1;
   cfg.gridDim = dim3((unsigned)(2 * np), 1, 1);
+  cfg.numAttrs = 2;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, ar, br, as_, bs, a));
 }
 
@@ -385,9 +394,9 @@ static PairArgs pair_common(const moe_dims_t& d, const int32_t* offsets, void* w
 }
 
 bool ffn_pair_gate_up_ok(const moe_dims_t& d) {
-  return !(d.flags & MOE_FLAG_FFN_SINGLE_CTA) && d.F % 128 == 0 && d.F_shared % 128 == 0;
+  return (d.flags & MOE_FLAG_FFN_CTA_PAIR) && d.F % 128 == 0 && d.F_shared % 128 == 0;
 }
-bool ffn_pair_down_ok(const moe_dims_t& d) { return !(d.flags & MOE_FLAG_FFN_SINGLE_CTA) && d.d % 256 == 0; }
+bool ffn_pair_down_ok(const moe_dims_t& d) { return (d.flags & MOE_FLAG_FFN_CTA_PAIR) && d.d % 256 == 0; }
 
 int launch_gate_up_pair(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
                         const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,

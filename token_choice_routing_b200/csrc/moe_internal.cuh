@@ -116,6 +116,29 @@ int check_dims(const moe_dims_t* d);
 int sm_count();
 int cuda_status(cudaError_t e);
 
+// Programmatic dependent launch. The layer's kernels are launched with
+// programmatic stream serialization (launch_pdl): the GPU may start launching a
+// kernel while its predecessor in the stream is still running, which hides the
+// launch latency between the layer's kernels. Every kernel first waits in
+// pdl_wait() until its predecessor has completed and its writes are visible (a
+// no-op when the kernel was launched the ordinary way), and only then lets its
+// own successor start launching, so no kernel ever runs ahead of earlier work.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, args...));
+}
+
 // 2-D bf16 tensor map [rows, cols] (cols contiguous) with a box of box_rows x 64
 // columns and the 128-byte swizzle (implemented in expert_ffn.cu).
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
@@ -171,6 +194,13 @@ int launch_selftest_wait(void* ws, unsigned long long limit_ns, cudaStream_t st)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Wait for the predecessor kernel in the stream (see launch_pdl), then allow the
+// successor to begin launching.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {

@@ -79,6 +79,7 @@ __device__ __forceinline__ void split3(float w, uint16_t& h, uint16_t& m, uint16
 // which must start at zero for every layer call.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, uint16_t* __restrict__ w3,
                                                            int N, int npw, int d, uint32_t* hdr, int nclear) {
+  pdl_wait_then_release();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nclear; i += blockDim.x) hdr[i] = 0u;
   const int nch = d >> 3;
@@ -164,6 +165,7 @@ template <int NPW>
 __global__ void __launch_bounds__(kRouteThreads, 1)
     route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const RouteArgs a) {
+  pdl_wait_then_release();
   using SM = RouteSmem<NPW>;
   constexpr int STAGES = SM::STAGES;
   constexpr int LS = SM::LS;
@@ -516,6 +518,7 @@ struct ScanArgs {
 };
 
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
+  pdl_wait_then_release();
   __shared__ int s_warp[kScanThreads / 32];
   __shared__ int s_off;
   __shared__ double s_ph[kScanThreads];
@@ -600,8 +603,7 @@ static int launch_route_t(const CUtensorMap& tx, const CUtensorMap& tw, const Ro
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
   }
-  route_kernel<NPW><<<a.nblk, kRouteThreads, SM::bytes, st>>>(tx, tw, a);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(route_kernel<NPW>, dim3(a.nblk), dim3(kRouteThreads), SM::bytes, st, tx, tw, a);
 }
 
 int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
@@ -620,8 +622,7 @@ int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
   sa.K = d.K;
   sa.nblk = L.nblk;
   sa.nparts = L.nparts;
-  scan_kernel<<<d.N + L.nparts, kScanThreads, 0, st>>>(sa);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(scan_kernel, dim3(d.N + L.nparts), dim3(kScanThreads), 0, st, sa);
 }
 
 int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, const float* bias,
@@ -664,8 +665,8 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
     long long grid = (work + 255) / 256;
     if (grid > (long long)sm_count() * 8) grid = (long long)sm_count() * 8;
     const int nclear = (int)((kHdrTotOffset + sizeof(int32_t) * d.N) / sizeof(uint32_t));
-    router_split_kernel<<<(int)grid, 256, 0, st>>>(w_router, w3, d.N, npw, d.d, a.hdr, nclear);
-    const int r = cuda_status(cudaGetLastError());
+    const int r = launch_pdl(router_split_kernel, dim3((unsigned)grid), dim3(256), 0, st, w_router, w3, d.N, npw,
+                             d.d, a.hdr, nclear);
     if (r != MOE_OK) return r;
   }
   CUtensorMap tx, tw;

@@ -124,6 +124,7 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
 template <int LG>
 __global__ void __launch_bounds__(256) router_transpose_kernel(const float* __restrict__ w, float* __restrict__ wt,
                                                                int N, int d) {
+  pdl_wait_then_release();
   using G = RouteGeo<LG>;
   constexpr int NPAD = G::NPAD, WT = G::WT;
   __shared__ float tile[NPAD + 1][33];
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(256) router_transpose_kernel(const float* __re
 // Epilogue: 4 threads per token.
 template <int LG>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
+  pdl_wait_then_release();
   using G = RouteGeo<LG>;
   constexpr int NPAD = G::NPAD, S = G::S, KS = G::KS, LS = G::LS, WT = G::WT;
   constexpr int NQ = NPAD / 4;  // reals per epilogue thread
@@ -450,7 +452,9 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
 template <int LG>
 static int launch_route_t(const RouteArgs& a, cudaStream_t st) {
   using SM = RouteGeo<LG>;
-  router_transpose_kernel<LG><<<a.d / 32, 256, 0, st>>>(a.w, const_cast<float*>(a.wt), a.N, a.d);
+  const int rt = launch_pdl(router_transpose_kernel<LG>, dim3(a.d / 32), dim3(256), 0, st, a.w,
+                            const_cast<float*>(a.wt), a.N, a.d);
+  if (rt != MOE_OK) return rt;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -460,8 +464,7 @@ static int launch_route_t(const RouteArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
   }
-  route_kernel<LG><<<a.nblk, kRouteThreads, SM::bytes, st>>>(a);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(route_kernel<LG>, dim3(a.nblk), dim3(kRouteThreads), SM::bytes, st, a);
 }
 
 }  // namespace fp32route

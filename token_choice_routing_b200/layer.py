@@ -25,11 +25,11 @@ class MoENullLayer:
                  w_router: torch.Tensor, router_bias: Optional[torch.Tensor],
                  w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
                  ws_gate: torch.Tensor, ws_up: torch.Tensor, ws_down: torch.Tensor,
-                 router: str = "tensor", ffn: str = "pair"):
+                 router: str = "tensor", ffn: str = "single"):
         """router: "tensor" (router product on the tensor cores, fp32 weights split
         exactly into three bf16 terms) or "fp32_cores" (fp32 FMA on the CUDA cores).
-        ffn: "pair" (expert GEMMs on CTA pairs where the shape allows) or "single"
-        (single-CTA tiles everywhere)."""
+        ffn: "single" (single-CTA tiles) or "pair" (expert GEMMs on CTA pairs where
+        the shape allows)."""
         if router not in ("tensor", "fp32_cores"):
             raise ValueError(f"router must be 'tensor' or 'fp32_cores', not {router!r}")
         if ffn not in ("pair", "single"):
@@ -37,7 +37,7 @@ class MoENullLayer:
         self.d, self.N, self.M, self.K, self.F, self.F_shared = d, N, M, K, F, F_shared
         self.router, self.ffn = router, ffn
         self.flags = ((B.FLAG_ROUTER_FP32_CORES if router == "fp32_cores" else 0) |
-                      (B.FLAG_FFN_SINGLE_CTA if ffn == "single" else 0))
+                      (B.FLAG_FFN_CTA_PAIR if ffn == "pair" else 0))
         dev = w_router.device
         self.device = dev
         self.w_router = w_router.contiguous()
@@ -58,7 +58,7 @@ class MoENullLayer:
                                   self.shared_gate_up.data_ptr(), self.shared_down.data_ptr())
 
     @classmethod
-    def from_inputs(cls, inp, device="cuda", router: str = "tensor", ffn: str = "pair") -> "MoENullLayer":
+    def from_inputs(cls, inp, device="cuda", router: str = "tensor", ffn: str = "single") -> "MoENullLayer":
         c = inp.cfg
         f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         return cls(c.d, c.N, c.M, c.K, c.F, c.F_shared,

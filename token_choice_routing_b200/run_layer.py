@@ -1,7 +1,7 @@
 """Run a few forwards of one seeded workload through the C ABI.
 
     python -m token_choice_routing_b200.run_layer [--config qwen3_0p6b] [--forwards 3]
-        [--router tensor|fp32_cores] [--ffn pair|single]
+        [--router tensor|fp32_cores] [--ffn single|pair]
 
 Used as the target of profiler captures (ncu -k <kernel> -s/-c selects the
 launch). Exits non-zero if the device status word reports an error.
@@ -21,7 +21,7 @@ def main(argv=None) -> int:
     ap.add_argument("--config", default="qwen3_0p6b", choices=sorted(I.CONFIGS))
     ap.add_argument("--forwards", type=int, default=3)
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"])
-    ap.add_argument("--ffn", default="pair", choices=["pair", "single"])
+    ap.add_argument("--ffn", default="single", choices=["single", "pair"])
     a = ap.parse_args(argv)
     inp = I.make_inputs(I.CONFIGS[a.config])
     layer = MoENullLayer.from_inputs(inp, "cuda", router=a.router, ffn=a.ffn)
