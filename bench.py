@@ -186,6 +186,8 @@ def workload_config(cfg, args):
             "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "K": cfg.K, "F": cfg.F, "F_shared": cfg.F_shared,
             "global_batch_tokens": cfg.T * args.gpus, "parallelism": f"dp{args.gpus}",
             "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "single"),
+            "routed_rows": "gathered from x inside gate/up (TMA tile::gather4)" if getattr(args, "gather", False)
+            else "copied into xs by dispatch",
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
@@ -203,6 +205,8 @@ def main():
                     help="router product on the tensor cores (default) or the fp32 CUDA cores")
     ap.add_argument("--ffn", default="single", choices=["single", "pair"],
                     help="expert GEMMs on single-CTA tiles (default) or CTA pairs where the shape allows")
+    ap.add_argument("--gather", action="store_true",
+                    help="no xs copy: gate/up gathers the routed rows of x by TMA (default: dispatch copies them)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")
@@ -234,7 +238,7 @@ def main():
     x = bf16_tensor(inp.x, dev)
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
     T = cfg.T
-    out = layer.alloc(T, logits=False)
+    out = layer.alloc(T, logits=False, xs=not args.gather)
     dm = layer.dims(T)
     nsum = B.aux_sums_count(dm)
     sums = torch.zeros(nsum, dtype=torch.float64, device=dev)
@@ -294,8 +298,12 @@ def main():
         B.dispatch(dm, x, out["topk_idx"], out["workspace"], out["counts"], out["offsets"], out["perm_tok"],
                    out["slot_row"], out["xs"])  # the aux reduction rides in this launch, as in moe_forward
         ev[2].record()
-        B.expert_gate_up(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, out["h"],
-                         out["h_shared"], out["workspace"])
+        if out["xs"] is None:
+            B.expert_gate_up_gather(dm, x, out["perm_tok"], out["offsets"], layer.gate_up, layer.shared_gate_up,
+                                    out["h"], out["h_shared"], out["workspace"])
+        else:
+            B.expert_gate_up(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, out["h"],
+                             out["h_shared"], out["workspace"])
         ev[3].record()
         B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down, out["ys"],
                       out["shared_out"], out["workspace"])
@@ -312,7 +320,9 @@ def main():
     flops_gu = 4.0 * d * F * R + 4.0 * d * Fs * T
     flops_dn = 2.0 * d * F * R + 2.0 * d * Fs * T
     bytes_route = 2.0 * d * T + (8.0 * K + 4.0) * T
-    bytes_dispatch = 4.0 * d * R + 4.0 * K * T
+    # dispatch: topk_idx and in-block ranks read, slot_row written (4 B each per slot), perm_tok per real
+    # slot; plus, when it copies rows into xs, 2d B read and 2d B written per real slot
+    bytes_dispatch = 12.0 * K * T + 4.0 * R + (0.0 if args.gather else 4.0 * d * R)
     bytes_combine = 2.0 * d * R + 4.0 * d * T
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))

@@ -112,7 +112,8 @@ typedef struct moe_outputs {
   int32_t* offsets;     /* [N+1] exclusive scan of counts; offsets[N] = R        */
   int32_t* perm_tok;    /* [R_cap] token of each expert-contiguous row (first R) */
   int32_t* slot_row;    /* [T, K] row of each slot in xs/h/ys, -1 for nulls      */
-  uint16_t* xs;         /* [R_cap, d] bf16 gathered rows                         */
+  uint16_t* xs;         /* [R_cap, d] bf16 gathered rows, or NULL: gate/up then
+                           gathers the rows of x by TMA and no copies are written */
   uint16_t* h;          /* [R_cap, F] bf16 routed SwiGLU activations             */
   uint16_t* h_shared;   /* [T, F_shared] bf16 shared SwiGLU activations          */
   uint16_t* ys;         /* [R_cap, d] bf16 routed expert outputs                 */
@@ -193,8 +194,10 @@ MOE_API int moe_route_noalloc(const moe_dims_t* dims, const uint16_t* x, const f
  * moe_route with the same workspace. counts [N], offsets [N+1]; the real slots
  * are laid out expert by expert, tokens ascending inside an expert: perm_tok
  * [T*K] (first offsets[N] entries valid), slot_row [T, K] (-1 for nulls), and
- * xs [T*K, d] bf16 with xs[slot_row[t,k]] = x[t]. Null slots cause no memory
- * traffic. Also reduces the aux statistics into the workspace (see moe_aux). */
+ * xs [T*K, d] bf16 with xs[slot_row[t,k]] = x[t], or xs = NULL to write no row
+ * copies (moe_expert_gate_up_gather then reads the rows of x through
+ * perm_tok). Null slots cause no memory traffic. Also reduces the aux
+ * statistics into the workspace (see moe_aux). */
 MOE_API int moe_dispatch(const moe_dims_t* dims, const uint16_t* x, const int32_t* topk_idx,
                  void* workspace, int32_t* counts, int32_t* offsets, int32_t* perm_tok,
                  int32_t* slot_row, uint16_t* xs, moe_stream_t stream);
@@ -219,6 +222,15 @@ MOE_API int moe_expert_gate_up(const moe_dims_t* dims, const uint16_t* xs, const
                        const int32_t* offsets, const uint16_t* gate_up,
                        const uint16_t* shared_gate_up, uint16_t* h, uint16_t* h_shared,
                        void* workspace, moe_stream_t stream);
+/* moe_expert_gate_up without the gathered copy xs: the routed rows are fetched
+ * from x by TMA row gathers (tile::gather4) through perm_tok, the row -> token
+ * map of moe_dispatch (row r of expert e's segment is token perm_tok[r]). Same
+ * h and h_shared as moe_expert_gate_up on the xs that moe_dispatch would write.
+ * x must be 16-byte aligned. */
+MOE_API int moe_expert_gate_up_gather(const moe_dims_t* dims, const uint16_t* x, const int32_t* perm_tok,
+                                      const int32_t* offsets, const uint16_t* gate_up,
+                                      const uint16_t* shared_gate_up, uint16_t* h, uint16_t* h_shared,
+                                      void* workspace, moe_stream_t stream);
 MOE_API int moe_expert_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* h,
                     const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* shared_down,
                     uint16_t* ys, uint16_t* shared_out, void* workspace, moe_stream_t stream);
@@ -250,7 +262,9 @@ MOE_API int moe_aux_finalize(const moe_dims_t* dims, const double* sums, int32_t
 MOE_API int moe_aux(const moe_dims_t* dims, const void* workspace, int32_t* counts_ext, float* P,
             float* losses, moe_stream_t stream);
 
-/* The whole forward: route, dispatch (+aux), expert FFNs, combine. */
+/* The whole forward: route, dispatch (+aux), expert FFNs, combine. With
+ * out->xs == NULL the routed rows are never copied: dispatch writes only the
+ * permutation and gate/up gathers rows of x (moe_expert_gate_up_gather). */
 MOE_API int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* x,
                 const float* tok_null_bias, const moe_outputs_t* out, void* workspace,
                 moe_stream_t stream);

@@ -45,10 +45,11 @@ def make_layer(inp, device="cuda", router="tensor", ffn="single"):
     return layer, x, tnb
 
 
-def run_forward(inp, device="cuda", router="tensor", ffn="single"):
+def run_forward(inp, device="cuda", router="tensor", ffn="single", xs=True):
+    """xs=False: no gathered copy of the routed rows; gate/up gathers rows of x."""
     from token_choice_routing_b200 import binding as B
     layer, x, tnb = make_layer(inp, device, router, ffn)
-    out = layer.forward(x, tnb)
+    out = layer.forward(x, tnb, layer.alloc(inp.cfg.T, xs=xs))
     torch.cuda.synchronize()
     st = B.get_device_status(out["workspace"])
     assert st == B.OK, B.status_string(st)
@@ -96,8 +97,9 @@ def check_dispatch(inp, out, r):
     R = int(offsets[-1])
     assert np.array_equal(out["perm_tok"][:R].cpu().numpy(), perm)
     assert np.array_equal(out["slot_row"].cpu().numpy(), slot_row)
-    xs = t2bits(out["xs"][:R])
-    assert np.array_equal(xs, inp.x[perm])
+    if out.get("xs") is not None:  # None: the forward gathered rows of x instead of copying them
+        xs = t2bits(out["xs"][:R])
+        assert np.array_equal(xs, inp.x[perm])
     return counts, offsets, perm, slot_row
 
 

@@ -30,15 +30,19 @@ SMALL = {
 }
 
 
-@pytest.mark.parametrize("ffn", H.FFNS)
-@pytest.mark.parametrize("router", H.ROUTERS)
+# (router, expert GEMM kernel, routed rows copied into xs or gathered inside gate/up)
+VARIANTS = [("tensor", "single", False), ("tensor", "single", True), ("fp32_cores", "single", True),
+            ("tensor", "pair", True), ("fp32_cores", "pair", False)]
+
+
+@pytest.mark.parametrize("router,ffn,xs", VARIANTS)
 @pytest.mark.parametrize("name", list(SMALL))
-def test_small_layer_full_parity(name, router, ffn):
+def test_small_layer_full_parity(name, router, ffn, xs):
     cfg = SMALL[name]
     inp = I.make_inputs(cfg)
     if cfg.name.startswith("ragged") or cfg.name in ("k1", "n64_k16", "t1"):
         inp.bias[cfg.N] = np.float32(0.3)
-    layer, x, tnb, out = H.run_forward(inp, router=router, ffn=ffn)
+    layer, x, tnb, out = H.run_forward(inp, router=router, ffn=ffn, xs=xs)
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -66,13 +70,15 @@ def test_small_layer_full_parity(name, router, ffn):
     H.check_layer_output(inp, out, r)
 
 
-@pytest.mark.parametrize("name,router,ffn", [("qwen3_0p6b", "tensor", "single"), ("qwen3_1p7b", "tensor", "single"),
-                                             ("qwen3_0p6b", "fp32_cores", "single"),
-                                             ("qwen3_0p6b", "tensor", "pair")])
-def test_full_size_layer_parity_sampled(name, router, ffn):
+@pytest.mark.parametrize("name,router,ffn,xs", [("qwen3_0p6b", "tensor", "single", False),
+                                                ("qwen3_1p7b", "tensor", "single", False),
+                                                ("qwen3_0p6b", "tensor", "single", True),
+                                                ("qwen3_0p6b", "fp32_cores", "single", True),
+                                                ("qwen3_0p6b", "tensor", "pair", True)])
+def test_full_size_layer_parity_sampled(name, router, ffn, xs):
     cfg = I.CONFIGS[name]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, out = H.run_forward(inp, router=router, ffn=ffn)
+    layer, x, tnb, out = H.run_forward(inp, router=router, ffn=ffn, xs=xs)
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -95,6 +101,26 @@ def test_large_configs_routing_and_sampled_output(name):
     rng = np.random.default_rng(1)
     tokens = np.sort(rng.choice(cfg.T, size=192, replace=False))
     H.check_layer_output(inp, out, r, tokens=tokens)
+
+
+@pytest.mark.parametrize("name", ["qwen3_0p6b", "ragged_b", "skew_small", "t1"])
+def test_row_gather_matches_row_copy_bitwise(name):
+    """Gate/up reading the routed rows of x through TMA row gathers feeds the
+    tensor cores exactly the rows dispatch would have copied, so h, ys and y
+    are bit-identical to the copy path."""
+    cfg = I.CONFIGS[name] if name in I.CONFIGS else SMALL[name]
+    inp = I.make_inputs(cfg)
+    layer, x, tnb = H.make_layer(inp)
+    outs = []
+    for xs in (True, False):
+        out = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs))
+        torch.cuda.synchronize()
+        outs.append(out)
+    R = int(outs[0]["offsets"][-1])
+    for k in ("perm_tok", "h", "ys"):
+        assert torch.equal(outs[0][k][:R], outs[1][k][:R]), k
+    for k in ("h_shared", "shared_out", "y", "losses", "counts_ext"):
+        assert torch.equal(outs[0][k], outs[1][k]), k
 
 
 def test_all_null_tokens_get_only_the_shared_expert():

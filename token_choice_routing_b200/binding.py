@@ -62,6 +62,7 @@ def _load() -> C.CDLL:
         "moe_dispatch": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_ffn": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_gate_up_gather": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_combine": (i32, [pd, vp, vp, vp, vp, vp, vp]),
         "moe_aux_sums_count": (sz, [pd]),
@@ -165,6 +166,12 @@ def expert_gate_up(dm, xs, x, offsets, gate_up, shared_gate_up, h, h_shared, ws,
     _check("moe_expert_gate_up", LIB.moe_expert_gate_up(C.byref(dm), _p(xs), _p(x), _p(offsets), _p(gate_up),
                                                         _p(shared_gate_up), _p(h), _p(h_shared), _p(ws),
                                                         _stream(stream)))
+
+
+def expert_gate_up_gather(dm, x, perm_tok, offsets, gate_up, shared_gate_up, h, h_shared, ws, stream=None):
+    _check("moe_expert_gate_up_gather",
+           LIB.moe_expert_gate_up_gather(C.byref(dm), _p(x), _p(perm_tok), _p(offsets), _p(gate_up),
+                                         _p(shared_gate_up), _p(h), _p(h_shared), _p(ws), _stream(stream)))
 
 
 def expert_down(dm, offsets, h, h_shared, w_down, shared_down, ys, shared_out, ws, stream=None):

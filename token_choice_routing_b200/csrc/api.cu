@@ -106,8 +106,7 @@ int moe_dispatch(const moe_dims_t* dims, const uint16_t* x, const int32_t* topk_
                  moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));
   if (dims->T == 0) return MOE_OK;
-  if (!x || !topk_idx || !workspace || !counts || !offsets || !perm_tok || !slot_row || !xs)
-    return MOE_ERR_INVALID_ARG;
+  if (!x || !topk_idx || !workspace || !counts || !offsets || !perm_tok || !slot_row) return MOE_ERR_INVALID_ARG;
   return launch_dispatch(*dims, x, topk_idx, workspace, counts, offsets, perm_tok, slot_row, xs, nullptr,
                          nullptr, nullptr, S(stream));
 }
@@ -133,6 +132,17 @@ int moe_expert_gate_up(const moe_dims_t* dims, const uint16_t* xs, const uint16_
   if (!xs || !x || !offsets || !gate_up || !shared_gate_up || !h || !h_shared || !workspace)
     return MOE_ERR_INVALID_ARG;
   return launch_gate_up(*dims, xs, x, offsets, gate_up, shared_gate_up, h, h_shared, workspace, S(stream));
+}
+
+int moe_expert_gate_up_gather(const moe_dims_t* dims, const uint16_t* x, const int32_t* perm_tok,
+                              const int32_t* offsets, const uint16_t* gate_up, const uint16_t* shared_gate_up,
+                              uint16_t* h, uint16_t* h_shared, void* workspace, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (dims->T == 0) return MOE_OK;
+  if (!x || !perm_tok || !offsets || !gate_up || !shared_gate_up || !h || !h_shared || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  return launch_gate_up_perm(*dims, nullptr, x, offsets, perm_tok, gate_up, shared_gate_up, h, h_shared, workspace,
+                             S(stream));
 }
 
 int moe_expert_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
@@ -183,7 +193,7 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
   if (!w->w_router || !w->gate_up || !w->w_down || !w->shared_gate_up || !w->shared_down)
     return MOE_ERR_INVALID_ARG;
   if (!out->topk_idx || !out->topk_gate || !out->n_real || !out->counts || !out->offsets || !out->perm_tok ||
-      !out->slot_row || !out->xs || !out->h || !out->h_shared || !out->ys || !out->shared_out || !out->y ||
+      !out->slot_row || !out->h || !out->h_shared || !out->ys || !out->shared_out || !out->y ||
       !out->counts_ext || !out->P || !out->losses)
     return MOE_ERR_INVALID_ARG;
   const cudaStream_t st = S(stream);
@@ -191,8 +201,11 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
                          out->topk_gate, out->n_real, workspace, st));
   MOE_CHECK(launch_dispatch(*dims, x, out->topk_idx, workspace, out->counts, out->offsets, out->perm_tok,
                             out->slot_row, out->xs, out->counts_ext, out->P, out->losses, st));
-  MOE_CHECK(launch_expert_ffn(*dims, out->xs, x, out->offsets, w->gate_up, w->w_down, w->shared_gate_up,
-                              w->shared_down, out->h, out->h_shared, out->ys, out->shared_out, workspace, st));
+  // xs == NULL: gate/up gathers the routed rows of x by TMA (no copies written by dispatch)
+  MOE_CHECK(launch_gate_up_perm(*dims, out->xs, x, out->offsets, out->xs ? nullptr : out->perm_tok, w->gate_up,
+                                w->shared_gate_up, out->h, out->h_shared, workspace, st));
+  MOE_CHECK(launch_down(*dims, out->offsets, out->h, out->h_shared, w->w_down, w->shared_down, out->ys,
+                        out->shared_out, workspace, st));
   return launch_combine(*dims, out->ys, out->shared_out, out->topk_gate, out->slot_row, out->y, st);
 }
 

@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
       }
       a.slot_row[(size_t)t * K + lane] = dest;
     }
+    if (a.xs == nullptr) continue;  // no row copies: gate/up gathers the rows of x itself
     const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * d);
     for (int c0 = 0; c0 < nch; c0 += 32) {  // warp-uniform trip count (shuffles below)
       const int c = c0 + lane;

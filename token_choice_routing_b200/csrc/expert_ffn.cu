@@ -20,6 +20,16 @@
 // coalesced, row-masked 16-byte stores (a tile may run past its expert's last
 // row; those rows are computed but never stored). Tiles are handed out
 // round-robin (all tiles of a GEMM have the same cost). Every wait is bounded.
+//
+// Row gather (gate/up with a token permutation): instead of reading routed rows
+// from a gathered copy xs, the producer warp gathers them from x with TMA
+// tile::gather4 loads (four rows each, one per lane and k-block, into the same
+// 128B-swizzled tile a 2-D load writes); rows past the expert's end read token 0
+// and are never stored. Dispatch then writes no row copies at all. Measured on
+// the 0.6B workload the gathers are ~2.3x slower for gate/up than reading the
+// copy (32 gather4 per tile and k-block hold the TMA unit), against ~10 us saved
+// in dispatch, so the copy stays the default and gathering is the option that
+// needs no R_cap x d buffer.
 #include "moe_internal.cuh"
 
 #include <cudaTypedefs.h>
@@ -35,6 +45,7 @@ constexpr int kStgRow = 64 * 2 + 16;  // staging row: 64 bf16 + 16 B pad
 
 struct GemmArgs {
   const int32_t* offsets;  // [N+1]
+  const int32_t* perm;     // token of each routed row, or null (routed A read from xs)
   int N, T;
   int kb_r, kb_s;          // 64-wide k-blocks per tile: routed, shared
   int nt_r, nt_s;          // n-tiles per group: routed, shared
@@ -179,39 +190,55 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
   };
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------ TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0, armed_par = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const TileInfo ti = decode(tile);
-        const void* ta = (ti.g < N) ? (const void*)&tmA_r : (const void*)&tmA_s;
-        const void* tb = (ti.g < N) ? (const void*)&tmB_r : (const void*)&tmB_s;
-        bool ok = true;
-        for (int kb = 0; kb < ti.nkb; ++kb) {
-          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, a.limit_ns, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(full_bar(stage), TX_BYTES);
-          tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), ta, full_bar(stage), kb * kBK, ti.arow);
-          tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), tb, full_bar(stage), kb * kBK, ti.brow);
-          armed |= 1u << stage;
-          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+    // ------------------------------ TMA producer (lane 0; every lane gathers 4 rows)
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_par = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileInfo ti = decode(tile);
+      const void* ta = (ti.g < N) ? (const void*)&tmA_r : (const void*)&tmA_s;
+      const void* tb = (ti.g < N) ? (const void*)&tmB_r : (const void*)&tmB_s;
+      const bool gather = a.perm != nullptr && ti.g < N;
+      int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+      if (gather) {
+        const int i0 = 4 * lane;  // tile rows i0 .. i0 + 3 of this lane
+        const int32_t* pp = a.perm + ti.arow + i0;
+        if (i0 + 0 < ti.mvalid) r0 = __ldg(pp + 0);
+        if (i0 + 1 < ti.mvalid) r1 = __ldg(pp + 1);
+        if (i0 + 2 < ti.mvalid) r2 = __ldg(pp + 2);
+        if (i0 + 3 < ti.mvalid) r3 = __ldg(pp + 3);
+      }
+      bool ok = true;
+      for (int kb = 0; kb < ti.nkb; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, a.limit_ns, abort_flag, a.status);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
         }
-        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(full_bar(stage), TX_BYTES);
+          if (!gather) tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), ta, full_bar(stage), kb * kBK, ti.arow);
+          tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), tb, full_bar(stage), kb * kBK, ti.brow);
+        }
+        __syncwarp();
+        if (gather)
+          tma_gather4(smem_u32(sA + stage * SM::A_BYTES + lane * 512), ta, full_bar(stage), kb * kBK, r0, r1, r2,
+                      r3);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-      if (*abort_flag) {
-        // let every issued copy land before the CTA can exit
-        for (int s = 0; s < kStages; ++s)
-          if (armed & (1u << s))
-            (void)mbar_wait_bounded(full_bar(s), (armed_par >> s) & 1u, a.limit_ns, nullptr, a.status);
-      }
+      if (!ok) break;
+    }
+    if (lane == 0 && *abort_flag) {
+      // let every issued copy land before the CTA can exit
+      for (int s = 0; s < kStages; ++s)
+        if (armed & (1u << s))
+          (void)mbar_wait_bounded(full_bar(s), (armed_par >> s) & 1u, a.limit_ns, nullptr, a.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -458,17 +485,27 @@ static FfnPlan plan_ffn(const moe_dims_t& d, const int32_t* offsets, void* ws) {
 int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
                    const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
                    void* ws, cudaStream_t st) {
-  if (ffn_pair_gate_up_ok(d)) return launch_gate_up_pair(d, xs, x, offsets, gate_up, sgate_up, h, h_shared, ws, st);
+  return launch_gate_up_perm(d, xs, x, offsets, nullptr, gate_up, sgate_up, h, h_shared, ws, st);
+}
+
+int launch_gate_up_perm(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                        const int32_t* perm, const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h,
+                        uint16_t* h_shared, void* ws, cudaStream_t st) {
+  if (perm == nullptr && ffn_pair_gate_up_ok(d))
+    return launch_gate_up_pair(d, xs, x, offsets, gate_up, sgate_up, h, h_shared, ws, st);
   FfnPlan p = plan_ffn(d, offsets, ws);
   const long long rcap = (long long)d.T * d.K;
   CUtensorMap ar, br, as_, bs;
-  if (!(make_tmap_bf16(&ar, xs, rcap, d.d, kBM) &&
+  // routed A: the gathered copy xs (128-row boxes), or x itself for row gathers (1-row boxes)
+  const bool ok_a = perm ? make_tmap_bf16(&ar, x, d.T, d.d, 1) : make_tmap_bf16(&ar, xs, rcap, d.d, kBM);
+  if (!(ok_a &&
         make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, p.BN1) &&
         make_tmap_bf16(&as_, x, d.T, d.d, kBM) &&
         make_tmap_bf16(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, p.BN1)))
     return MOE_ERR_CUDA;
   p.g1.out_r = h;
   p.g1.out_s = h_shared;
+  p.g1.perm = perm;
   return (p.BN1 == 256) ? launch_gemm<256, true>(ar, br, as_, bs, p.g1, p.max1, st)
                         : launch_gemm<128, true>(ar, br, as_, bs, p.g1, p.max1, st);
 }

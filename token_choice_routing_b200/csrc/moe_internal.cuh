@@ -172,6 +172,11 @@ int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const doub
 int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
                    const float* topk_gate, const int32_t* slot_row, uint16_t* y,
                    cudaStream_t st);
+// perm (optional): token of each routed row; when given, gate/up gathers the
+// routed rows of x by TMA instead of reading a gathered copy xs (xs unused).
+int launch_gate_up_perm(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                        const int32_t* perm, const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h,
+                        uint16_t* h_shared, void* ws, cudaStream_t st);
 int launch_expert_ffn(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x,
                       const int32_t* offsets, const uint16_t* gate_up, const uint16_t* w_down,
                       const uint16_t* sgate_up, const uint16_t* sdown, uint16_t* h,
@@ -350,6 +355,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// TMA row gather: four rows (y0..y3) of a 2-D tensor map whose box is one row
+// high, columns [x, x + box width), written as four consecutive rows at dst.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint32_t bar, int x, int y0, int y1,
+                                            int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+      : "memory");
 }
 
 // ---- thread-block clusters of two CTAs (a CTA pair sharing one tcgen05 MMA)

@@ -549,18 +549,33 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
     return;
   }
   const int e = blockIdx.x;
-  if (tid == 0) {
-    int o = 0;
-    for (int q = 0; q < e; ++q) o += a.tot[q];
-    s_off = o;
-    if (e == 0) {
-      int run = 0;
-      for (int q = 0; q < N; ++q) {
-        a.offsets[q] = run;
-        a.counts[q] = a.tot[q];
-        run += a.tot[q];
+  if (warp == 0) {
+    // exclusive prefix of the per-expert totals (N <= 64: two per lane), by shuffles
+    const int t0 = (lane < N) ? a.tot[lane] : 0;
+    const int t1 = (lane + 32 < N) ? a.tot[lane + 32] : 0;
+    int i0 = t0, i1 = t1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u0 = __shfl_up_sync(0xffffffffu, i0, o);
+      const int u1 = __shfl_up_sync(0xffffffffu, i1, o);
+      if (lane >= o) {
+        i0 += u0;
+        i1 += u1;
       }
-      a.offsets[N] = run;
+    }
+    const int low_total = __shfl_sync(0xffffffffu, i0, 31);
+    const int ex0 = i0 - t0, ex1 = low_total + i1 - t1;  // exclusive prefixes of experts lane, lane + 32
+    if (lane == (e & 31)) s_off = (e < 32) ? ex0 : ex1;
+    if (e == 0) {
+      if (lane < N) {
+        a.offsets[lane] = ex0;
+        a.counts[lane] = t0;
+      }
+      if (lane + 32 < N) {
+        a.offsets[lane + 32] = ex1;
+        a.counts[lane + 32] = t1;
+      }
+      if (lane == 31) a.offsets[N] = low_total + i1;
     }
   }
   const int per = (nblk + kScanThreads - 1) / kScanThreads;

@@ -53,9 +53,15 @@ def dp_forward(layer, x, tok_null_bias, out, sums, group=None):
     B.aux_sums(dm, ws, sums)
     allreduce_aux_sums(sums, group)
     B.aux_finalize(dm, sums, out["counts_ext"], out["P"], out["losses"])
-    B.dispatch(dm, x, out["topk_idx"], ws, out["counts"], out["offsets"], out["perm_tok"], out["slot_row"],
-               out["xs"])
-    B.expert_ffn(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.w_down, layer.shared_gate_up,
-                 layer.shared_down, out["h"], out["h_shared"], out["ys"], out["shared_out"], ws)
+    xs = out.get("xs")
+    B.dispatch(dm, x, out["topk_idx"], ws, out["counts"], out["offsets"], out["perm_tok"], out["slot_row"], xs)
+    if xs is None:  # gate/up gathers the routed rows of x itself
+        B.expert_gate_up_gather(dm, x, out["perm_tok"], out["offsets"], layer.gate_up, layer.shared_gate_up,
+                                out["h"], out["h_shared"], ws)
+        B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down, out["ys"],
+                      out["shared_out"], ws)
+    else:
+        B.expert_ffn(dm, xs, x, out["offsets"], layer.gate_up, layer.w_down, layer.shared_gate_up,
+                     layer.shared_down, out["h"], out["h_shared"], out["ys"], out["shared_out"], ws)
     B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"])
     return out

@@ -71,8 +71,10 @@ class MoENullLayer:
     def dims(self, T: int) -> B.Dims:
         return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags)
 
-    def alloc(self, T: int, logits: bool = True) -> Dict[str, torch.Tensor]:
-        """Caller-owned buffers for a T-token call (R_cap = T*K rows)."""
+    def alloc(self, T: int, logits: bool = True, xs: bool = True) -> Dict[str, torch.Tensor]:
+        """Caller-owned buffers for a T-token call (R_cap = T*K rows). xs=False
+        leaves out the gathered copy of the routed rows: the forward then gathers
+        rows of x inside the gate/up GEMM and dispatch writes no copies."""
         dev, d, N, M, K, F, Fs = self.device, self.d, self.N, self.M, self.K, self.F, self.F_shared
         R = T * K
         i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
@@ -85,7 +87,7 @@ class MoENullLayer:
             offsets=torch.empty((N + 1,), dtype=i32, device=dev),
             perm_tok=torch.empty((max(R, 1),), dtype=i32, device=dev),
             slot_row=torch.empty((T, K), dtype=i32, device=dev),
-            xs=torch.empty((max(R, 1), d), dtype=bf, device=dev),
+            xs=torch.empty((max(R, 1), d), dtype=bf, device=dev) if xs else None,
             h=torch.empty((max(R, 1), F), dtype=bf, device=dev),
             h_shared=torch.empty((max(T, 1), Fs), dtype=bf, device=dev),
             ys=torch.empty((max(R, 1), d), dtype=bf, device=dev),
