@@ -49,6 +49,38 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Sources whose change invalidates a recorded ncu traffic figure of the grouped GEMM.
+GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
+GEMM_PROFILE = "profiles/grouped_gemm_qwen3_0p6b.md"
+
+
+def gemm_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_gate_up_traffic(workload: str):
+    """DRAM bytes (read + write) of one gate/up launch from the committed ncu summary:
+    its line 'traffic-record: workload=W kernel=gate_up dram_bytes_per_launch=B
+    source_sha256=H'. None unless it was taken on this workload from the current
+    kernel sources."""
+    try:
+        with open(os.path.join(ROOT, GEMM_PROFILE)) as f:
+            lines = [l.strip() for l in f if l.strip().startswith("traffic-record:")]
+    except OSError:
+        return None
+    digest = gemm_source_digest()
+    for l in lines:
+        kv = dict(p.split("=", 1) for p in l.split()[1:] if "=" in p)
+        if kv.get("workload") == workload and kv.get("kernel") == "gate_up" and kv.get("source_sha256") == digest:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
 class ClockSampler:
     """Samples the GPU's SM clock and clock-event (throttle) reasons through NVML
     from a background thread while the timed region runs."""
@@ -351,7 +383,9 @@ def main():
     roofline = {"kernel": "grouped gate/up SwiGLU GEMM (tcgen05, %s)" % ("CTA pairs" if pair else "single CTA"),
                 "bound": "tensor", "achieved": achieved,
                 "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
-                "peak_kind": f"{peak_kind} bf16 burst", "traffic": None,
+                "peak_kind": f"{peak_kind} bf16 burst",
+                "traffic": recorded_gate_up_traffic(cfg.name) if not (args.gather or pair) else None,
+                "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "flops_per_launch": flops_gu, "ms_per_launch": kms["gate_up"]}
 
     # ---- end to end through the C ABI with host buffers

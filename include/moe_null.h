@@ -113,7 +113,7 @@ typedef struct moe_outputs {
   int32_t* perm_tok;    /* [R_cap] token of each expert-contiguous row (first R) */
   int32_t* slot_row;    /* [T, K] row of each slot in xs/h/ys, -1 for nulls      */
   uint16_t* xs;         /* [R_cap, d] bf16 gathered rows, or NULL: gate/up then
-                           gathers the rows of x by TMA and no copies are written */
+                           gathers the rows of x itself and no copies are written */
   uint16_t* h;          /* [R_cap, F] bf16 routed SwiGLU activations             */
   uint16_t* h_shared;   /* [T, F_shared] bf16 shared SwiGLU activations          */
   uint16_t* ys;         /* [R_cap, d] bf16 routed expert outputs                 */
@@ -223,7 +223,7 @@ MOE_API int moe_expert_gate_up(const moe_dims_t* dims, const uint16_t* xs, const
                        const uint16_t* shared_gate_up, uint16_t* h, uint16_t* h_shared,
                        void* workspace, moe_stream_t stream);
 /* moe_expert_gate_up without the gathered copy xs: the routed rows are fetched
- * from x by TMA row gathers (tile::gather4) through perm_tok, the row -> token
+ * from x by 16-byte asynchronous copies (cp.async) through perm_tok, the row -> token
  * map of moe_dispatch (row r of expert e's segment is token perm_tok[r]). Same
  * h and h_shared as moe_expert_gate_up on the xs that moe_dispatch would write.
  * x must be 16-byte aligned. */

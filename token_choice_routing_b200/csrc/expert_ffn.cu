@@ -22,14 +22,13 @@
 // round-robin (all tiles of a GEMM have the same cost). Every wait is bounded.
 //
 // Row gather (gate/up with a token permutation): instead of reading routed rows
-// from a gathered copy xs, the producer warp gathers them from x with TMA
-// tile::gather4 loads (four rows each, one per lane and k-block, into the same
-// 128B-swizzled tile a 2-D load writes); rows past the expert's end read token 0
-// and are never stored. Dispatch then writes no row copies at all. Measured on
-// the 0.6B workload the gathers are ~2.3x slower for gate/up than reading the
-// copy (32 gather4 per tile and k-block hold the TMA unit), against ~10 us saved
-// in dispatch, so the copy stays the default and gathering is the option that
-// needs no R_cap x d buffer.
+// from a gathered copy xs, the producer warp copies them from x with 16-byte
+// cp.async loads (4 rows per pass, 8 lanes per row) straight into the
+// 128B-swizzled tile a 2-D TMA load would write; each lane's copies signal the
+// stage's full barrier on completion (cp.async.mbarrier.arrive.noinc) and the
+// MMA thread fences them into the async proxy before issuing. Rows past the
+// expert's end read token 0 and are never stored. Dispatch then writes no row
+// copies at all.
 #include "moe_internal.cuh"
 
 #include <cudaTypedefs.h>
@@ -46,6 +45,8 @@ constexpr int kStgRow = 64 * 2 + 16;  // staging row: 64 bf16 + 16 B pad
 struct GemmArgs {
   const int32_t* offsets;  // [N+1]
   const int32_t* perm;     // token of each routed row, or null (routed A read from xs)
+  const uint16_t* x;       // [T, ld_x]: the rows perm refers to
+  int ld_x;
   int N, T;
   int kb_r, kb_s;          // 64-wide k-blocks per tile: routed, shared
   int nt_r, nt_s;          // n-tiles per group: routed, shared
@@ -71,7 +72,8 @@ struct GemmSmem {
   static constexpr int n_bar = 2 * kStages + 5;  // full, empty, tfull[2], tempty[2], drain
   static constexpr size_t off_misc = off_bar + 8 * n_bar;
   static constexpr size_t off_tab = off_misc + 16;
-  static constexpr size_t end = off_tab + sizeof(int) * 3 * (kMaxN + 2);
+  static constexpr size_t off_perm = off_tab + sizeof(int) * 3 * (kMaxN + 2);  // int [128]: tokens of a tile
+  static constexpr size_t end = off_perm + sizeof(int) * kBM;
   static constexpr size_t bytes = end + 1024;  // slack for 1024-byte alignment
 };
 
@@ -79,7 +81,7 @@ struct TileInfo {
   int g, arow, mvalid, brow, nkb, col0;
 };
 
-template <int BN, bool SWIGLU>
+template <int BN, bool SWIGLU, bool GATHER>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
                     const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s,
@@ -121,7 +123,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       prefetch_tmap(&tmB_s);
     }
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), 1);
+      // producer lane 0's expect_tx arrival (+ with row gathers, 32 copy-completion arrivals)
+      mbar_init(full_bar(s), GATHER ? 1 + 32 : 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -189,8 +192,45 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     return ti;
   };
 
-  if (warp == 0) {
-    // ------------------------------ TMA producer (lane 0; every lane gathers 4 rows)
+  if (warp == 0 && !GATHER) {
+    if (lane == 0) {
+      // ------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo ti = decode(tile);
+        const void* ta = (ti.g < N) ? (const void*)&tmA_r : (const void*)&tmA_s;
+        const void* tb = (ti.g < N) ? (const void*)&tmB_r : (const void*)&tmB_s;
+        bool ok = true;
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, a.limit_ns, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), TX_BYTES);
+          tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), ta, full_bar(stage), kb * kBK, ti.arow);
+          tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), tb, full_bar(stage), kb * kBK, ti.brow);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // let every issued copy land before the CTA can exit
+        for (int s = 0; s < kStages; ++s)
+          if (armed & (1u << s))
+            (void)mbar_wait_bounded(full_bar(s), (armed_par >> s) & 1u, a.limit_ns, nullptr, a.status);
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------ producer warp with row gathers: TMA loads (lane 0),
+    // routed A rows by cp.async (all lanes)
+    int* s_perm = reinterpret_cast<int*>(base + SM::off_perm);
     int stage = 0;
     uint32_t phase = 0;
     uint32_t armed = 0, armed_par = 0;
@@ -198,15 +238,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       const TileInfo ti = decode(tile);
       const void* ta = (ti.g < N) ? (const void*)&tmA_r : (const void*)&tmA_s;
       const void* tb = (ti.g < N) ? (const void*)&tmB_r : (const void*)&tmB_s;
-      const bool gather = a.perm != nullptr && ti.g < N;
-      int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+      const bool gather = ti.g < N;
       if (gather) {
-        const int i0 = 4 * lane;  // tile rows i0 .. i0 + 3 of this lane
-        const int32_t* pp = a.perm + ti.arow + i0;
-        if (i0 + 0 < ti.mvalid) r0 = __ldg(pp + 0);
-        if (i0 + 1 < ti.mvalid) r1 = __ldg(pp + 1);
-        if (i0 + 2 < ti.mvalid) r2 = __ldg(pp + 2);
-        if (i0 + 3 < ti.mvalid) r3 = __ldg(pp + 3);
+        // the token of each tile row; rows past the expert's end read token 0 (never stored)
+        __syncwarp();  // the previous tile's copies have all been issued
+#pragma unroll
+        for (int j = 0; j < kBM / 32; ++j) {
+          const int i = j * 32 + lane;
+          s_perm[i] = (i < ti.mvalid) ? __ldg(a.perm + ti.arow + i) : 0;
+        }
+        __syncwarp();
       }
       bool ok = true;
       for (int kb = 0; kb < ti.nkb; ++kb) {
@@ -217,14 +258,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(full_bar(stage), TX_BYTES);
+          mbar_arrive_expect_tx(full_bar(stage), gather ? (uint32_t)SM::B_BYTES : TX_BYTES);
           if (!gather) tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), ta, full_bar(stage), kb * kBK, ti.arow);
           tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), tb, full_bar(stage), kb * kBK, ti.brow);
         }
-        __syncwarp();
-        if (gather)
-          tma_gather4(smem_u32(sA + stage * SM::A_BYTES + lane * 512), ta, full_bar(stage), kb * kBK, r0, r1, r2,
-                      r3);
+        if (gather) {
+          // 128 rows x 128 B: 4 rows per pass, 8 lanes per row, 16 B per lane, into the
+          // 128B-swizzled layout a 2-D TMA load would write (chunk c of row r at c ^ (r & 7))
+          const int chunk = lane & 7;
+          const uint32_t dst0 = smem_u32(sA + stage * SM::A_BYTES);
+          const uint16_t* src0 = a.x + (size_t)kb * kBK + chunk * 8;
+#pragma unroll 8
+          for (int p = 0; p < kBM / 4; ++p) {
+            const int r = p * 4 + (lane >> 3);
+            const int tok = s_perm[r];
+            cp_async_16(dst0 + (uint32_t)(r * 128 + ((chunk ^ (r & 7)) << 4)), src0 + (size_t)tok * a.ld_x);
+          }
+        }
+        cp_async_mbar_arrive_noinc(full_bar(stage));  // fires when this lane's copies so far have landed
         armed |= 1u << stage;
         armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages) {
@@ -234,6 +285,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       }
       if (!ok) break;
     }
+    cp_async_wait_all_copies();
     if (lane == 0 && *abort_flag) {
       // let every issued copy land before the CTA can exit
       for (int s = 0; s < kStages; ++s)
@@ -260,6 +312,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             break;
           }
           tc_fence_after();
+          if constexpr (GATHER) fence_proxy_async_shared();  // gathered rows -> async proxy (tensor cores)
           const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * SM::A_BYTES));
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * SM::B_BYTES));
 #pragma unroll
@@ -419,7 +472,7 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU>
+template <int BN, bool SWIGLU, bool GATHER>
 static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUtensorMap& as_,
                        const CUtensorMap& bs, const GemmArgs& a, long long max_tiles, cudaStream_t st) {
   using SM = GemmSmem<BN>;
@@ -427,7 +480,7 @@ static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, SWIGLU>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, SWIGLU, GATHER>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::bytes);
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
@@ -435,7 +488,7 @@ static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   long long grid = sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(grouped_gemm_kernel<BN, SWIGLU>, dim3((unsigned)grid), dim3(kGemmThreads), SM::bytes, st, ar, br,
+  return launch_pdl(grouped_gemm_kernel<BN, SWIGLU, GATHER>, dim3((unsigned)grid), dim3(kGemmThreads), SM::bytes, st, ar, br,
                     as_, bs, a);
 }
 
@@ -497,7 +550,8 @@ int launch_gate_up_perm(const moe_dims_t& d, const uint16_t* xs, const uint16_t*
   const long long rcap = (long long)d.T * d.K;
   CUtensorMap ar, br, as_, bs;
   // routed A: the gathered copy xs (128-row boxes), or x itself for row gathers (1-row boxes)
-  const bool ok_a = perm ? make_tmap_bf16(&ar, x, d.T, d.d, 1) : make_tmap_bf16(&ar, xs, rcap, d.d, kBM);
+  // (with perm the routed rows are gathered by cp.async and the map is not used)
+  const bool ok_a = make_tmap_bf16(&ar, perm ? x : xs, perm ? (uint64_t)d.T : (uint64_t)rcap, d.d, kBM);
   if (!(ok_a &&
         make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, p.BN1) &&
         make_tmap_bf16(&as_, x, d.T, d.d, kBM) &&
@@ -506,8 +560,13 @@ int launch_gate_up_perm(const moe_dims_t& d, const uint16_t* xs, const uint16_t*
   p.g1.out_r = h;
   p.g1.out_s = h_shared;
   p.g1.perm = perm;
-  return (p.BN1 == 256) ? launch_gemm<256, true>(ar, br, as_, bs, p.g1, p.max1, st)
-                        : launch_gemm<128, true>(ar, br, as_, bs, p.g1, p.max1, st);
+  p.g1.x = x;
+  p.g1.ld_x = d.d;
+  if (perm)
+    return (p.BN1 == 256) ? launch_gemm<256, true, true>(ar, br, as_, bs, p.g1, p.max1, st)
+                          : launch_gemm<128, true, true>(ar, br, as_, bs, p.g1, p.max1, st);
+  return (p.BN1 == 256) ? launch_gemm<256, true, false>(ar, br, as_, bs, p.g1, p.max1, st)
+                        : launch_gemm<128, true, false>(ar, br, as_, bs, p.g1, p.max1, st);
 }
 
 int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
@@ -524,8 +583,8 @@ int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, 
     return MOE_ERR_CUDA;
   p.g2.out_r = ys;
   p.g2.out_s = shared_out;
-  return (p.BN2 == 256) ? launch_gemm<256, false>(ar, br, as_, bs, p.g2, p.max2, st)
-                        : launch_gemm<128, false>(ar, br, as_, bs, p.g2, p.max2, st);
+  return (p.BN2 == 256) ? launch_gemm<256, false, false>(ar, br, as_, bs, p.g2, p.max2, st)
+                        : launch_gemm<128, false, false>(ar, br, as_, bs, p.g2, p.max2, st);
 }
 
 int launch_expert_ffn(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,

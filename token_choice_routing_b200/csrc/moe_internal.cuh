@@ -357,15 +357,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-// TMA row gather: four rows (y0..y3) of a 2-D tensor map whose box is one row
-// high, columns [x, x + box width), written as four consecutive rows at dst.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint32_t bar, int x, int y0, int y1,
-                                            int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
-      : "memory");
+// 16-byte asynchronous copy global -> shared (L2 only), completion tracked per thread.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on an mbarrier once all of this thread's earlier cp.async copies have
+// landed (the arrival is counted in the barrier's initial count: .noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all_copies() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Make generic-proxy writes to shared memory (cp.async) visible to the async
+// proxy (tcgen05 operand reads) for this thread's subsequent operations.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---- thread-block clusters of two CTAs (a CTA pair sharing one tcgen05 MMA)
