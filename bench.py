@@ -388,6 +388,17 @@ def main():
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "flops_per_launch": flops_gu, "ms_per_launch": kms["gate_up"]}
 
+    if cfg.name.startswith("decode"):
+        # a few rows per expert: the gate/up GEMM streams the weights of the experts that some
+        # token chose (the others are never read), so its bound is HBM on those bytes
+        used = int((out["counts"] > 0).sum().item())
+        bytes_gu = (2.0 * 2 * F * d * used + 2.0 * 2 * Fs * d + 2.0 * d * (R + T) + 2.0 * F * R + 2.0 * Fs * T)
+        gbs = bytes_gu / (kms["gate_up"] * 1e6)
+        roofline = {"kernel": "grouped gate/up SwiGLU GEMM (weight streaming, tcgen05)", "bound": "hbm",
+                    "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                    "peak_kind": f"{peak_kind} HBM copy", "traffic": None, "bytes_per_launch": bytes_gu,
+                    "experts_used": used, "ms_per_launch": kms["gate_up"]}
+
     # ---- end to end through the C ABI with host buffers
     x_pin = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).view(torch.bfloat16).pin_memory()
     loss_pin = torch.empty(2, dtype=torch.float32).pin_memory()

@@ -123,6 +123,23 @@ def test_row_gather_matches_row_copy_bitwise(name):
         assert torch.equal(outs[0][k], outs[1][k]), k
 
 
+@pytest.mark.parametrize("name,T", [("decode_0p6b", 1), ("decode_0p6b", 8), ("decode_0p6b", 64),
+                                    ("decode_0p6b", 256), ("decode_1p7b", 64)])
+def test_decode_sized_forward_parity(name, T):
+    """Small-batch forwards with a full-size layer's weights (a few rows per expert; the
+    expert GEMMs only read the weights of experts that some token chose)."""
+    import dataclasses
+    cfg = dataclasses.replace(I.CONFIGS[name], T=T)
+    inp = I.make_inputs(cfg)
+    layer, x, tnb, out = H.run_forward(inp)
+    r = H.check_routing(inp, out)
+    counts, offsets, perm, slot_row = H.check_dispatch(inp, out, r)
+    H.check_aux(inp, out, r)
+    H.check_layer_output(inp, out, r)
+    assert int(offsets[-1]) == int(r["n_real"].sum())
+    assert (counts == 0).sum() >= cfg.N - int(r["n_real"].sum())  # unchosen experts have empty segments
+
+
 def test_all_null_tokens_get_only_the_shared_expert():
     cfg = I.small_config("allnull", T=100, d=256, N=8, F=64, F_shared=128, K=4, M=8, config_id=910)
     inp = I.make_inputs(cfg, null_bias=1000.0)

@@ -319,27 +319,30 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
       if (M > 0) m = fmaxf(m, sn);
+      // (these feed only the aux statistics P and L_z, kept to ~1e-6 relative: the
+      // fast exponential and one reciprocal are within that)
       float e[NQ];
       float z = 0.f;
 #pragma unroll
       for (int u = 0; u < NQ; ++u) {
-        e[u] = (q + 4 * u < N) ? expf(v[u] - m) : 0.f;
+        e[u] = (q + 4 * u < N) ? __expf(v[u] - m) : 0.f;
         z += e[u];
       }
       z += __shfl_xor_sync(0xffffffffu, z, 1);
       z += __shfl_xor_sync(0xffffffffu, z, 2);
-      const float en = (M > 0) ? expf(sn - m) : 0.f;
+      const float en = (M > 0) ? __expf(sn - m) : 0.f;
       const float Z = (M > 0) ? z + (float)M * en : z;
       const float lse = m + logf(Z);
+      const float rz = 1.f / Z;
       // p_i = e^{s_i - lse} evaluated as e^{s_i - m} / Z (no cancellation when |m| is
       // large), written over this lane's own logits
 #pragma unroll
       for (int u = 0; u < NQ; ++u) {
         const int i = q + 4 * u;
-        if (i < N) row[i] = e[u] / Z;
+        if (i < N) row[i] = e[u] * rz;
       }
       if (q == 0) {
-        pn[t] = (M > 0) ? en / Z : 0.f;
+        pn[t] = (M > 0) ? en * rz : 0.f;
         lse2[t] = lse * lse;
       }
 
@@ -348,6 +351,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       unsigned sel = 0u;
       int used = 0, r = 0;
       unsigned long long msk = 0ull;
+      float smax = 0.f;  // the first real taken is the largest real logit
       for (int k = 0; k < K; ++k) {
         float bv = -INFINITY;
         int bi = INT_MAX;
@@ -375,37 +379,31 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           ++used;
         } else {
           id = bi;
+          if (r == 0) smax = bv;
           ++r;
           msk |= 1ull << bi;
           if ((bi & 3) == q) sel |= 1u << (bi >> 2);
         }
-        if (q == 0) {
+        if ((k & 3) == q) {  // slot k belongs to lane k mod 4 from here on
           tk[t * kMaxK + k] = id;
           tkv[t * kMaxK + k] = bv;
         }
       }
-      __syncwarp();
+      // gates: softmax over the selected real logits; each lane takes slots q, q+4, ...
+      // and the four partial sums are added in a fixed order
+      float gsum = 0.f;
+      for (int k = q; k < K; k += 4)
+        if (tk[t * kMaxK + k] < N) gsum += expf(tkv[t * kMaxK + k] - smax);
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
       if (valid) {
+        for (int k = q; k < K; k += 4) {
+          const int id = tk[t * kMaxK + k];
+          const float g = (id < N) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
+          a.topk_idx[(size_t)tok * K + k] = id;
+          a.topk_gate[(size_t)tok * K + k] = g;
+        }
         if (q == 0) {
-          // gates: softmax over the selected real logits (rank order: first real is the max)
-          float smax = 0.f, gsum = 0.f;
-          bool first = true;
-          for (int k = 0; k < K; ++k) {
-            if (tk[t * kMaxK + k] < N) {
-              const float sv = tkv[t * kMaxK + k];
-              if (first) {
-                smax = sv;
-                first = false;
-              }
-              gsum += expf(sv - smax);
-            }
-          }
-          for (int k = 0; k < K; ++k) {
-            const int id = tk[t * kMaxK + k];
-            const float g = (id < N) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
-            a.topk_idx[(size_t)tok * K + k] = id;
-            a.topk_gate[(size_t)tok * K + k] = g;
-          }
           a.n_real[tok] = r;
           atomicAdd(s_hist + (K - r), 1);  // integer: the histogram does not depend on the order
         }

@@ -58,6 +58,7 @@ class LayerConfig:
     M: int
     skew: bool = False
     seqs: int = 1
+    bias_from: Optional[str] = None  # workload whose calibrated null bias this one uses
 
     @property
     def rho(self) -> float:
@@ -78,6 +79,12 @@ CONFIGS: Dict[str, LayerConfig] = {c.name: c for c in [
     LayerConfig("sweep_k4_m64", 32, T=65536, d=2048, N=64, F=1536, F_shared=1536, K=4, M=64, seqs=8),
     LayerConfig("sweep_k8_m192", 33, T=65536, d=2048, N=64, F=1536, F_shared=1536, K=8, M=192, seqs=8),
     LayerConfig("skew", 4, T=131072, d=2048, N=64, F=1536, F_shared=1536, K=8, M=64, skew=True, seqs=16),
+    # Small-batch (decode-sized) forwards with the 0.6B and 1.7B layers' weights: same
+    # config ids, so the router and expert weights are the same draws; ~T rho K / N rows
+    # per expert, so the expert GEMMs stream weights (experts no token chose are skipped).
+    LayerConfig("decode_0p6b", 1, T=64, d=1024, N=64, F=768, F_shared=768, K=4, M=64, bias_from="qwen3_0p6b"),
+    LayerConfig("decode_1p7b", 2, T=64, d=2048, N=64, F=1536, F_shared=1536, K=8, M=192,
+                bias_from="qwen3_1p7b"),
 ]}
 
 # Null-logit bias per workload, from tests/golden/calibrate_null_bias.py (oracle
@@ -92,6 +99,7 @@ NULL_BIAS: Dict[str, float] = {
     "sweep_k8_m192": 2.3533687591552734,
     "tiny": 0.7090700268745422,
 }
+
 
 SKEW_LOW_INFO_FRACTION = 0.6
 SKEW_LOW_INFO_SCALE = 0.3
@@ -208,7 +216,7 @@ def make_inputs(cfg: LayerConfig, *, T: Optional[int] = None, weights: bool = Tr
     if cfg.skew:
         bias[:N] = (-SKEW_ZIPF_S * np.log(np.arange(N, dtype=np.float64) + 1.0)).astype(np.float32)
     elif cfg.M > 0:
-        nb = NULL_BIAS.get(cfg.name, 0.0) if null_bias is None else null_bias
+        nb = NULL_BIAS.get(cfg.bias_from or cfg.name, 0.0) if null_bias is None else null_bias
         bias[N] = np.float32(nb)
 
     if weights:
