@@ -23,7 +23,9 @@ Sources (cited by page title and section):
       (aux loss alpha*E*sum f_i P_i), section 4.3 (router z-loss).
 [MPP] MoE++ explainer page, section "Gating 机制与残差门控": topk over all
       logits, softmax over the k, zero the zero-compute experts' weights,
-      divide by the remaining sum.
+      divide by the remaining sum; section "核心创新：三种零计算专家": the zero
+      expert outputs nothing, the copy expert returns its input, the constant
+      expert replaces it with a learned vector (one per expert, hidden size).
 
 Readings where the pages are silent (each is listed in the design notes):
 * pool = N real slots followed by M null copies (indices N..N+M-1); with M = 0
@@ -49,17 +51,20 @@ __all__ = [
     "router_logits", "expanded_pool", "pool_logsumexp", "pool_probs", "topk_pool",
     "threshold_real_count", "renormalised_gates", "dispatch", "swiglu",
     "layer_output", "aux_stats", "aux_partial_sums", "aux_finalize", "route",
-    "bf16_round_f64",
+    "bf16_round_f64", "expanded_pool_pp", "pool_kinds", "renormalised_gates_pp",
+    "layer_output_pp", "route_pp",
 ]
 
 
-def router_logits(x, w_router, bias=None, tok_null_bias=None):
+def router_logits(x, w_router, bias=None, tok_null_bias=None, null_col=None):
     """Router logits s[t, j], j = 0..N (N real experts, then the null logit).
 
     [KR] 三/Null Expert 机制: the router is widened to N+1 logits, the last one
     belonging to the null expert. [T44] 三: the router is a linear map of the
     token's hidden state. ``bias`` [N+1] is added to every logit; the optional
-    per-token ``tok_null_bias`` [T] is added to the null logit only.
+    per-token ``tok_null_bias`` [T] is added to the null logit only (column
+    ``null_col``, by default the last; with MoE++ experts the null logit is
+    column N and the copy and constant experts' logits follow it).
     """
     x = np.asarray(x, dtype=np.float64)
     w = np.asarray(w_router, dtype=np.float64)
@@ -67,7 +72,7 @@ def router_logits(x, w_router, bias=None, tok_null_bias=None):
     if bias is not None:
         s = s + np.asarray(bias, dtype=np.float64)[None, :]
     if tok_null_bias is not None:
-        s[:, -1] += np.asarray(tok_null_bias, dtype=np.float64)
+        s[:, -1 if null_col is None else null_col] += np.asarray(tok_null_bias, dtype=np.float64)
     return s
 
 
@@ -240,7 +245,8 @@ def aux_stats(idx, p, lse, N, M):
     """
     idx = np.asarray(idx)
     T = idx.shape[0]
-    counts_ext = np.bincount(idx.reshape(-1), minlength=N + M)[:N + M].astype(np.int64)
+    pool = np.asarray(p).shape[1]  # N + M (+ MoE++ copy and constant experts)
+    counts_ext = np.bincount(idx.reshape(-1), minlength=pool)[:pool].astype(np.int64)
     f = counts_ext / float(T)
     P = np.asarray(p, dtype=np.float64).mean(axis=0)
     L_bal = N * float(np.sum(f * P))
@@ -257,7 +263,8 @@ def aux_partial_sums(idx, p, lse, N, M):
     over all tokens ([KR] 三/负载均衡损失).
     """
     idx = np.asarray(idx)
-    counts_ext = np.bincount(idx.reshape(-1), minlength=N + M)[:N + M].astype(np.int64)
+    pool = np.asarray(p).shape[1]
+    counts_ext = np.bincount(idx.reshape(-1), minlength=pool)[:pool].astype(np.int64)
     psum = np.asarray(p, dtype=np.float64).sum(axis=0)
     lsq = float(np.sum(np.asarray(lse, dtype=np.float64) ** 2))
     return counts_ext, psum, lsq, int(idx.shape[0])
@@ -284,4 +291,84 @@ def route(s, M, K):
     idx = topk_pool(v, K)
     n_real = (idx < N).sum(axis=1)
     gates = renormalised_gates(s, idx, N)
+    return dict(v=v, lse=lse, p=p, idx=idx, n_real=n_real, gates=gates)
+
+
+# ---------------------------------------------------------------------------------------
+# MoE++ zero-computation experts next to the null expert ([MPP] 核心创新).
+#
+# Router rows: N real experts, the null logit (column N), C copy experts, V constant
+# experts (columns N+1 .. N+C+V). Pool (what top-K ranks): the N reals, the M null
+# copies, then the copy and the constant experts (pool indices N+M .. N+M+C+V-1), so
+# on equal logits a null copy precedes a copy or constant expert. Gates: softmax over
+# the selected slots that are not null copies ([MPP] zeroes only the zero expert's
+# weight before renormalising). Outputs: a copy expert returns x, constant expert j
+# the vector c_j, a null copy nothing. With C = V = 0 every function below equals its
+# null-only counterpart above.
+
+
+def pool_kinds(N, M, C, V):
+    """Kind of each pool slot (0 real, 1 null copy, 2 copy, 3 constant) and the
+    router column its logit comes from. Returns two int64 arrays [N+M+C+V]."""
+    kind = np.concatenate([np.zeros(N), np.ones(M), np.full(C, 2), np.full(V, 3)]).astype(np.int64)
+    col = np.concatenate([np.arange(N), np.full(M, N), N + 1 + np.arange(C + V)]).astype(np.int64)
+    return kind, col
+
+
+def expanded_pool_pp(s, N, M, C, V):
+    """The MoE++ pool [s_0..s_{N-1}, s_N x M, s_{N+1}..s_{N+C+V}] from logits [T, N+1+C+V]."""
+    s = np.asarray(s, dtype=np.float64)
+    _, col = pool_kinds(N, M, C, V)
+    return s[:, col]
+
+
+def renormalised_gates_pp(v, idx, N, M):
+    """Gates over the pool: softmax of the selected slots that are not null copies
+    (pool index < N or >= N+M); null copies get 0; all 0 if every slot is null."""
+    v = np.asarray(v, dtype=np.float64)
+    idx = np.asarray(idx)
+    T, K = idx.shape
+    g = np.zeros((T, K), dtype=np.float64)
+    for t in range(T):
+        sel = [k for k in range(K) if idx[t, k] < N or idx[t, k] >= N + M]
+        if not sel:
+            continue
+        vals = np.array([v[t, idx[t, k]] for k in sel])
+        e = np.exp(vals - vals.max())
+        g[t, sel] = e / e.sum()
+    return g
+
+
+def layer_output_pp(x, idx, gates, N, M, C, V, experts, shared, const_vectors, tokens=None,
+                    round_h=False):
+    """y_t = E_shared(x_t) + sum of g E_i(x_t) over selected reals + g x_t over
+    selected copy experts + g c_j over selected constant experts j ([KR] 三/核心公式
+    with the [MPP] experts' outputs). ``const_vectors`` [V, d]."""
+    x = np.asarray(x, dtype=np.float64)
+    idx = np.asarray(idx)
+    gates = np.asarray(gates, dtype=np.float64)
+    if tokens is None:
+        tokens = np.arange(x.shape[0])
+    tokens = np.asarray(tokens)
+    y = layer_output(x, idx, gates, N, experts, shared, tokens=tokens, round_h=round_h)
+    xt = x[tokens]
+    sub_idx = idx[tokens]
+    sub_g = np.where((sub_idx >= N + M) & (sub_idx < N + M + C), gates[tokens], 0.0)
+    y += sub_g.sum(axis=1)[:, None] * xt
+    cv = np.asarray(const_vectors, dtype=np.float64).reshape(V, -1) if V else None
+    for j in range(V):
+        rows, ks = np.nonzero(sub_idx == N + M + C + j)
+        if rows.size:
+            np.add.at(y, rows, gates[tokens][rows, ks][:, None] * cv[j][None, :])
+    return y
+
+
+def route_pp(s, N, M, C, V, K):
+    """All routing outputs of the MoE++ pool from logits s [T, N+1+C+V]."""
+    v = expanded_pool_pp(s, N, M, C, V)
+    lse = pool_logsumexp(v)
+    p = pool_probs(v, lse)
+    idx = topk_pool(v, K)
+    n_real = (idx < N).sum(axis=1)
+    gates = renormalised_gates_pp(v, idx, N, M)
     return dict(v=v, lse=lse, p=p, idx=idx, n_real=n_real, gates=gates)

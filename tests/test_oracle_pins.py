@@ -346,3 +346,119 @@ def test_bf16_rounding_matches_torch():
     a = rng.standard_normal(10000) * 10
     ref = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(O.bf16_round_f64(a.astype(np.float32)), ref)
+
+
+# --- MoE++ copy and constant experts next to the null expert ----------------------------
+
+def _pp_case(seed, T, d, N, M, C, V, F=16, Fs=12):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, d))
+    experts = (rng.standard_normal((N, F, d)) / math.sqrt(d), rng.standard_normal((N, F, d)) / math.sqrt(d),
+               rng.standard_normal((N, d, F)) / math.sqrt(F))
+    shared = (rng.standard_normal((Fs, d)) / math.sqrt(d), rng.standard_normal((Fs, d)) / math.sqrt(d),
+              rng.standard_normal((d, Fs)) / math.sqrt(Fs))
+    cv = rng.standard_normal((V, d))
+    return rng, x, experts, shared, cv
+
+
+def test_pp_without_copy_or_constant_experts_is_the_null_only_layer():
+    rng, x, ex, sh, cv = _pp_case(401, 40, 8, 5, 3, 0, 0)
+    s = rng.standard_normal((40, 6))
+    for K in (1, 3, 5):
+        a, b = O.route(s, 3, K), O.route_pp(s, 5, 3, 0, 0, K)
+        for k in ("v", "idx", "n_real"):
+            np.testing.assert_array_equal(a[k], b[k])
+        for k in ("lse", "p", "gates"):  # same values, NumPy may sum them in another order
+            np.testing.assert_allclose(a[k], b[k], rtol=1e-14, atol=1e-300)
+        np.testing.assert_allclose(O.layer_output(x, a["idx"], a["gates"], 5, ex, sh),
+                                   O.layer_output_pp(x, b["idx"], b["gates"], 5, 3, 0, 0, ex, sh, cv),
+                                   rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("N,M,C,V", [(2, 1, 1, 1), (3, 2, 2, 0), (2, 0, 1, 2), (1, 2, 1, 1)])
+def test_pp_topk_matches_bruteforce_with_ties(N, M, C, V):
+    """Quantised logits tie null copies with copy/constant experts and with reals:
+    the pool order (reals, null copies, copy, constant) decides them."""
+    rng = np.random.default_rng(500 + N + 10 * M + 100 * C + 1000 * V)
+    T = 40
+    s = rng.integers(-2, 3, size=(T, N + 1 + C + V)).astype(np.float64) / 2.0
+    kind, col = O.pool_kinds(N, M, C, V)
+    assert kind.tolist() == [0] * N + [1] * M + [2] * C + [3] * V
+    for K in range(1, min(4, N + M + C + V) + 1):
+        v = O.expanded_pool_pp(s, N, M, C, V)
+        for t in range(T):
+            assert [v[t, i] for i in range(v.shape[1])] == [s[t, c] for c in col]
+        idx = O.topk_pool(v, K)
+        for t in range(T):
+            assert idx[t].tolist() == _brute_topk(list(v[t]), K), (t, K, v[t])
+
+
+def test_pp_gates_match_the_masked_topk_procedure():
+    """[MPP] Gating: softmax over the K selected logits, zero the zero expert's
+    weight, divide by the remaining sum. The direct softmax over the selected
+    non-null slots must give the same gates."""
+    N, M, C, V, K = 4, 3, 2, 2, 5
+    rng = np.random.default_rng(601)
+    s = rng.standard_normal((200, N + 1 + C + V))
+    s[:, N] += 0.8  # plenty of null slots
+    r = O.route_pp(s, N, M, C, V, K)
+    sel = np.take_along_axis(r["v"], r["idx"], axis=1)
+    g = scipy.special.softmax(sel, axis=1)
+    g[(r["idx"] >= N) & (r["idx"] < N + M)] = 0.0
+    tot = g.sum(axis=1, keepdims=True)
+    g = np.divide(g, tot, out=np.zeros_like(g), where=tot > 0)
+    np.testing.assert_allclose(r["gates"], g, rtol=1e-12, atol=1e-15)
+
+
+def test_pp_copy_and_constant_outputs():
+    """A token whose slots are all copy experts gets E_shared(x) + x; all on
+    constant expert j (with K = 1), E_shared(x) + c_j; all null, E_shared(x)."""
+    N, M, C, V, K = 3, 2, 2, 2, 2
+    rng, x, ex, sh, cv = _pp_case(602, 6, 8, N, M, C, V)
+    s = np.full((6, N + 1 + C + V), -50.0)
+    s[0, N + 1] = s[0, N + 2] = 3.0  # token 0: both copy experts
+    s[1, N + 3] = 4.0                # token 1: constant expert 0 (K = 1 below)
+    s[2, N] = 5.0                    # token 2: null copies only
+    s[3, N + 4] = 2.0                # token 3: constant 1 and one copy
+    s[3, N + 1] = 1.0
+    ys = O.swiglu(x, *sh)
+    r = O.route_pp(s, N, M, C, V, K)
+    y = O.layer_output_pp(x, r["idx"], r["gates"], N, M, C, V, ex, sh, cv)
+    np.testing.assert_allclose(y[0], ys[0] + x[0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y[2], ys[2], rtol=1e-12, atol=1e-12)
+    g3 = scipy.special.softmax([2.0, 1.0])
+    np.testing.assert_allclose(y[3], ys[3] + g3[0] * cv[1] + g3[1] * x[3], rtol=1e-12, atol=1e-12)
+    r1 = O.route_pp(s, N, M, C, V, 1)
+    y1 = O.layer_output_pp(x, r1["idx"], r1["gates"], N, M, C, V, ex, sh, cv)
+    np.testing.assert_allclose(y1[1], ys[1] + cv[0], rtol=1e-12, atol=1e-12)
+
+
+def test_pp_copy_expert_mixes_input_and_dense_output():
+    """Review page, 为什么用零专家而非复制专家: with copy experts the MoE output is
+    (1 - rho) x + rho y_dense. With r reals and c copies selected on equal logits,
+    the real gates sum to rho = r/(r+c) and y_dense is the reals' mean output."""
+    N, M, C, V, K = 4, 0, 3, 0, 5
+    rng, x, ex, sh, cv = _pp_case(603, 5, 8, N, M, C, V)
+    s = np.full((5, N + 1 + C + V), -30.0)
+    s[:, [0, 2]] = 1.0          # r = 2 reals
+    s[:, N + 1:N + 1 + C] = 1.0  # c = 3 copies
+    r = O.route_pp(s, N, M, C, V, K)
+    y = O.layer_output_pp(x, r["idx"], r["gates"], N, M, C, V, ex, sh, cv) - O.swiglu(x, *sh)
+    rho = 2 / 5
+    y_dense = (O.swiglu(x, ex[0][0], ex[1][0], ex[2][0]) + O.swiglu(x, ex[0][2], ex[1][2], ex[2][2])) / 2
+    np.testing.assert_allclose(y, (1 - rho) * x + rho * y_dense, rtol=1e-12, atol=1e-12)
+
+
+def test_pp_aux_invariants():
+    N, M, C, V, K, T = 6, 4, 2, 3, 4, 300
+    rng = np.random.default_rng(604)
+    s = rng.standard_normal((T, N + 1 + C + V))
+    r = O.route_pp(s, N, M, C, V, K)
+    counts, f, P, L_bal, L_z = O.aux_stats(r["idx"], r["p"], r["lse"], N, M)
+    assert counts.shape == (N + M + C + V,) and counts.sum() == T * K
+    assert abs(P.sum() - 1.0) < 1e-12 and abs(f.sum() - K) < 1e-12
+    # null copies still fill in index order; copy/constant counts are plain counts
+    assert np.all(np.diff(counts[N:N + M]) <= 0)
+    for j in range(C + V):
+        assert counts[N + M + j] == int((r["idx"] == N + M + j).sum())
+    np.testing.assert_allclose(L_z, np.mean(scipy.special.logsumexp(r["v"], axis=1) ** 2), rtol=1e-12)
