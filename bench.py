@@ -213,12 +213,14 @@ def run_reference(args):
 
 
 def workload_config(cfg, args):
+    pp = f" C={cfg.C} V={cfg.V}" if cfg.C + cfg.V else ""
     return {"workload": f"{cfg.name}: MoE layer fwd T={cfg.T} d={cfg.d} N={cfg.N} F={cfg.F} "
-                        f"F_shared={cfg.F_shared} K={cfg.K} M={cfg.M} rho={cfg.rho:.3g}",
+                        f"F_shared={cfg.F_shared} K={cfg.K} M={cfg.M}{pp} rho={cfg.rho:.3g}",
             "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "K": cfg.K, "F": cfg.F, "F_shared": cfg.F_shared,
+            "C": cfg.C, "V": cfg.V,
             "global_batch_tokens": cfg.T * args.gpus, "parallelism": f"dp{args.gpus}",
             "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "single"),
-            "routed_rows": "gathered from x inside gate/up (TMA tile::gather4)" if getattr(args, "gather", False)
+            "routed_rows": "gathered from x inside gate/up (cp.async row gathers)" if getattr(args, "gather", False)
             else "copied into xs by dispatch",
             "l2": "flushed between timed steps (256 MiB write)"}
 
@@ -340,7 +342,8 @@ def main():
         B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down, out["ys"],
                       out["shared_out"], out["workspace"])
         ev[4].record()
-        B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"])
+        B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
+                  topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
         ev[5].record()
         torch.cuda.synchronize()
         for i, n in enumerate(names):
@@ -356,6 +359,8 @@ def main():
     # slot; plus, when it copies rows into xs, 2d B read and 2d B written per real slot
     bytes_dispatch = 12.0 * K * T + 4.0 * R + (0.0 if args.gather else 4.0 * d * R)
     bytes_combine = 2.0 * d * R + 4.0 * d * T
+    if cfg.C + cfg.V > 0:  # MoE++ copy/constant slots read a row of x or a constant vector
+        bytes_combine += 2.0 * d * float(out["counts_ext"][cfg.N + cfg.M:].sum().item())
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     fp32_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
@@ -402,7 +407,7 @@ def main():
     # ---- end to end through the C ABI with host buffers
     x_pin = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).view(torch.bfloat16).pin_memory()
     loss_pin = torch.empty(2, dtype=torch.float32).pin_memory()
-    cext_pin = torch.empty(N + cfg.M, dtype=torch.int32).pin_memory()
+    cext_pin = torch.empty(out["counts_ext"].numel(), dtype=torch.int32).pin_memory()
     xin = torch.empty_like(x)
     e2e_ms = []
     for i in range(args.warmup + args.steps):
@@ -423,7 +428,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_total = float(t.item())
     e2e = {"value": world * R * args.steps / (e2e_total * 1e-3), "unit": UNIT,
-           "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(8 + 4 * (N + cfg.M)),
+           "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(8 + 4 * cext_pin.numel()),
            "ms_per_step": e2e_total / args.steps}
 
     cpu = None

@@ -14,6 +14,15 @@
  * load-balance statistics L_bal = N * sum_{i<N+M} f_i P_i (负载均衡损失) and the
  * Z-loss L_z = mean_t (log sum_{i<N+M} e^{s_i})^2 (Z-Loss).
  *
+ * Optionally the pool also holds MoE++'s other zero-computation experts (MoE++
+ * explainer page, 核心创新：三种零计算专家): C copy experts (output x) and V
+ * constant experts (output a learned vector c_j), each with its own router row
+ * after the null logit. Pool order: reals 0..N-1, null copies N..N+M-1, copy
+ * experts N+M..N+M+C-1, constant experts N+M+C..N+M+C+V-1. They take gates like
+ * real experts (renormalisation runs over every selected slot except null
+ * copies) and cost no GEMM work: combine adds g x and g c_j. C = V = 0 is the
+ * paper's layer.
+ *
  * Conventions shared by every entry point:
  *  - All pointers except `dims`, `w` and `out` (host structs) are DEVICE
  *    pointers on the current CUDA device. bf16 tensors are passed as uint16_t
@@ -30,8 +39,10 @@
  *    word inside the workspace; read it with moe_get_device_status.
  *  - T = 0 is a no-op that returns MOE_OK.
  *  - Non-finite inputs give undefined routing.
- *  - Limits: 1 <= N <= 64, 0 <= M, 1 <= K <= 16, K <= N + M, d a multiple of
- *    128 (128..8192), F and F_shared multiples of 64 (64..16384), T*K < 2^31.
+ *  - Limits: 1 <= N <= 64, 0 <= M, 1 <= K <= 16, K <= N + M + C + V, d a
+ *    multiple of 128 (128..8192), F and F_shared multiples of 64 (64..16384),
+ *    T*K < 2^31; with C + V > 0 also N + 1 + C + V <= 80 (and the tensor-core
+ *    router).
  *    Outside them: MOE_ERR_UNSUPPORTED (or MOE_ERR_INVALID_ARG for values that
  *    are never valid, e.g. K < 1, M < 0, T < 0).
  *
@@ -56,7 +67,7 @@
 extern "C" {
 #endif
 
-#define MOE_NULL_ABI_VERSION 1
+#define MOE_NULL_ABI_VERSION 2
 
 typedef void* moe_stream_t; /* a cudaStream_t */
 
@@ -90,16 +101,20 @@ typedef enum {
 typedef struct moe_dims {
   int32_t T, d, N, M, K, F, F_shared;
   uint32_t flags;
+  int32_t C, V;  /* MoE++ copy and constant experts (0, 0: null experts only) */
 } moe_dims_t;
 
 /* Weights of one layer (device pointers). */
 typedef struct moe_weights {
-  const float* w_router;        /* [N+1, d] fp32; row N is the null logit       */
-  const float* router_bias;     /* [N+1] fp32 or NULL (added to every logit)    */
+  const float* w_router;        /* [N+1+C+V, d] fp32; row N is the null logit,
+                                   rows N+1.. the copy, then constant experts   */
+  const float* router_bias;     /* [N+1+C+V] fp32 or NULL (added to each logit) */
   const uint16_t* gate_up;      /* [N, 2F, d] bf16, from moe_pack_gate_up       */
   const uint16_t* w_down;       /* [N, d, F] bf16                               */
   const uint16_t* shared_gate_up; /* [2F_shared, d] bf16, from moe_pack_gate_up */
   const uint16_t* shared_down;  /* [d, F_shared] bf16                           */
+  const uint16_t* const_vectors; /* [V, d] bf16 constant experts' outputs, or
+                                    NULL when V = 0                             */
 } moe_weights_t;
 
 /* Outputs and intermediates of moe_forward (device pointers). R_cap = T*K. */
@@ -119,8 +134,8 @@ typedef struct moe_outputs {
   uint16_t* ys;         /* [R_cap, d] bf16 routed expert outputs                 */
   uint16_t* shared_out; /* [T, d] bf16 shared expert output                      */
   uint16_t* y;          /* [T, d] bf16 layer output                              */
-  int32_t* counts_ext;  /* [N+M] tokens per pool slot                            */
-  float* P;             /* [N+M] mean routing probability per pool slot          */
+  int32_t* counts_ext;  /* [N+M+C+V] tokens per pool slot                        */
+  float* P;             /* [N+M+C+V] mean routing probability per pool slot      */
   float* losses;        /* [2] = {L_bal, L_z}                                    */
 } moe_outputs_t;
 
@@ -157,14 +172,17 @@ MOE_API int moe_pack_gate_up(const moe_dims_t* dims, const uint16_t* w_gate, con
  *  products are exact, accumulation is fp32, the three partial sums are added
  *  in fp32), or, with MOE_FLAG_ROUTER_FP32_CORES, as an fp32 FMA product on the
  *  CUDA cores. x and w_router must be 16-byte aligned (x is read by TMA).
- *  Over the pool [s_0..s_{N-1},
- *  s_N x M]: lse_t, p_{t,i}; top-K in (value desc, index asc) order -- a real
- *  logit equal to the null logit precedes every copy, copies fill N, N+1, ...;
- *  gates = softmax over the selected real logits (0 for nulls, all 0 if none).
+ *  Over the pool [s_0..s_{N-1}, s_N x M, s_{N+1}..s_{N+C+V}] (pool indices:
+ *  reals, null copies, copy experts, constant experts): lse_t, p_{t,i}; top-K
+ *  in (value desc, pool index asc) order -- a real logit equal to the null
+ *  logit precedes every null copy, null copies fill N, N+1, ... and precede a
+ *  copy or constant expert of equal logit; gates = softmax over the selected
+ *  slots that are not null copies (0 for null copies, all 0 if only nulls).
  *  With M = 0 the null logit takes no part in anything.
- *  x [T, d] bf16; tok_null_bias [T] or NULL; logits_out [T, N+1] or NULL;
- *  topk_idx [T, K]; topk_gate [T, K]; n_real [T]. Also fills the workspace
- *  with per-block statistics and the dispatch scan (counts, offsets). */
+ *  x [T, d] bf16; tok_null_bias [T] or NULL (added to the null logit);
+ *  logits_out [T, N+1+C+V] or NULL; topk_idx [T, K] (pool indices); topk_gate
+ *  [T, K]; n_real [T] (real experts only). Also fills the workspace with
+ *  per-block statistics and the dispatch scan (counts, offsets). */
 MOE_API int moe_route(const moe_dims_t* dims, const uint16_t* x, const float* w_router,
               const float* router_bias, const float* tok_null_bias, float* logits_out,
               int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* workspace,
@@ -235,15 +253,20 @@ MOE_API int moe_expert_down(const moe_dims_t* dims, const int32_t* offsets, cons
                     const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* shared_down,
                     uint16_t* ys, uint16_t* shared_out, void* workspace, moe_stream_t stream);
 
-/* Combine (section 三 / 核心公式): y[t] = bf16(shared_out[t] + sum over real
- * slots k, in rank order, of topk_gate[t,k] * ys[slot_row[t,k]]), fp32
- * accumulation, one rounding. y [T, d]. */
+/* Combine (section 三 / 核心公式): y[t] = bf16(shared_out[t] + sum over the
+ * token's slots k, in rank order, of topk_gate[t,k] * out_k), out_k =
+ * ys[slot_row[t,k]] for a real expert, x[t] for a copy expert, const_vectors[j]
+ * for constant expert j, nothing for a null copy; fp32 accumulation, one
+ * rounding. y [T, d]. topk_idx, x and const_vectors are read only when C + V >
+ * 0 (they may be NULL otherwise). */
 MOE_API int moe_combine(const moe_dims_t* dims, const uint16_t* ys, const uint16_t* shared_out,
-                const float* topk_gate, const int32_t* slot_row, uint16_t* y,
-                moe_stream_t stream);
+                const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx,
+                const uint16_t* x, const uint16_t* const_vectors, uint16_t* y, moe_stream_t stream);
 
 /* Number of doubles in the additive aux statistics of a token shard:
- * [counts_real (N) | null histogram (K+1) | sum_t p (N+1) | sum_t lse^2 | T]. */
+ * [counts_real (N) | null histogram (K+1), then the C+V copy/constant expert
+ * counts | sum_t p (N+1+C+V: reals, the null logit, copy/constant experts) |
+ * sum_t lse^2 | T]. */
 MOE_API size_t moe_aux_sums_count(const moe_dims_t* dims);
 
 /* Additive aux statistics of this call's tokens (layout above), for a
@@ -252,9 +275,9 @@ MOE_API int moe_aux_sums(const moe_dims_t* dims, const void* workspace, double* 
                  moe_stream_t stream);
 
 /* L_bal / L_z from (possibly all-reduced) sums (section 三 / 负载均衡损失,
- * Z-Loss): counts_ext [N+M] (copy j counts the tokens with more than j null
- * slots), P [N+M] (copies share the null probability), losses [2] =
- * {L_bal = N * sum_i f_i P_i with f_i = counts_ext_i / T_total, L_z}. */
+ * Z-Loss): counts_ext [N+M+C+V] (null copy j counts the tokens with more than j
+ * null slots), P [N+M+C+V] (null copies share the null probability), losses [2]
+ * = {L_bal = N * sum_i f_i P_i with f_i = counts_ext_i / T_total, L_z}. */
 MOE_API int moe_aux_finalize(const moe_dims_t* dims, const double* sums, int32_t* counts_ext,
                      float* P, float* losses, moe_stream_t stream);
 

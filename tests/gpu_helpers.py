@@ -64,12 +64,12 @@ def logit_bound(inp):
     w = np.abs(inp.w_router.astype(np.float64))
     mag = x @ w.T + np.abs(inp.bias.astype(np.float64))[None, :]
     if inp.tok_null_bias is not None:
-        mag[:, -1] += np.abs(inp.tok_null_bias.astype(np.float64))
+        mag[:, inp.cfg.N] += np.abs(inp.tok_null_bias.astype(np.float64))
     return (inp.cfg.d + 3) * 2.0 ** -24 * mag + 1e-30
 
 
 def oracle_logits(inp):
-    return O.router_logits(f64(inp.x), inp.w_router, inp.bias, inp.tok_null_bias)
+    return O.router_logits(f64(inp.x), inp.w_router, inp.bias, inp.tok_null_bias, null_col=inp.cfg.N)
 
 
 def check_routing(inp, out, full_gates=True):
@@ -80,7 +80,7 @@ def check_routing(inp, out, full_gates=True):
     s_ref = oracle_logits(inp)
     err = np.abs(s_gpu - s_ref)
     assert np.all(err <= logit_bound(inp)), float((err / logit_bound(inp)).max())
-    r = O.route(s_gpu, M, K)
+    r = O.route_pp(s_gpu, N, M, cfg.C, cfg.V, K)  # = O.route when C = V = 0
     idx = out["topk_idx"].cpu().numpy()
     assert np.array_equal(idx, r["idx"]), np.argwhere(idx != r["idx"])[:5]
     assert np.array_equal(out["n_real"].cpu().numpy(), r["n_real"])
@@ -128,7 +128,12 @@ def check_y(y_gpu, y_ref):
 def check_layer_output(inp, out, r, tokens=None):
     ex, sh = expert_weights(inp)
     x = f64(inp.x)
-    y_ref = O.layer_output(x, r["idx"], r["gates"], inp.cfg.N, ex, sh, tokens=tokens)
+    c = inp.cfg
+    if c.C + c.V > 0:
+        cv = f64(inp.const_vectors) if c.V else None
+        y_ref = O.layer_output_pp(x, r["idx"], r["gates"], c.N, c.M, c.C, c.V, ex, sh, cv, tokens=tokens)
+    else:
+        y_ref = O.layer_output(x, r["idx"], r["gates"], c.N, ex, sh, tokens=tokens)
     y_gpu = bf16_f64(out["y"][:inp.cfg.T])
     if tokens is not None:
         y_gpu = y_gpu[tokens]

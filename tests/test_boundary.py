@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.LIB.moe_abi_version() == 1
+    assert lib.LIB.moe_abi_version() == 2
     for code in (0, -1, -2, -3, -4, -5, 7):
         assert isinstance(lib.status_string(code), str) and lib.status_string(code)
 
@@ -63,6 +63,16 @@ def test_check_dims(lib):
         v = dict(T=256, d=128, N=8, M=8, K=4, F=64, F_shared=64)
         v.update(kw)
         assert B.check_dims(B.dims(**v)) == B.ERR_UNSUPPORTED, kw
+    # MoE++ copy/constant experts: at most 16 of them and 80 router rows, tensor-core router only
+    ok = dict(T=256, d=128, N=8, M=8, K=4, F=64, F_shared=64)
+    assert B.check_dims(B.dims(**ok, C=2, V=3)) == B.OK
+    assert B.check_dims(B.dims(**dict(ok, N=64, M=0, K=4), C=10, V=5)) == B.OK  # 80 rows
+    assert B.check_dims(B.dims(**dict(ok, N=64), C=10, V=6)) == B.ERR_UNSUPPORTED  # 81 rows
+    assert B.check_dims(B.dims(**ok, C=9, V=8)) == B.ERR_UNSUPPORTED  # 17 > 16
+    assert B.check_dims(B.dims(**ok, flags=B.FLAG_ROUTER_FP32_CORES, C=1)) == B.ERR_UNSUPPORTED
+    assert B.check_dims(B.dims(**ok, C=-1)) == B.ERR_INVALID_ARG
+    assert B.check_dims(B.dims(**dict(ok, M=0, K=9), C=0, V=0)) == B.ERR_INVALID_ARG  # K > N+M
+    assert B.check_dims(B.dims(**dict(ok, M=0, K=9), C=1, V=0)) == B.OK  # K <= N+M+C+V
     dm = good()
     for f in (B.FLAG_ROUTER_FP32_CORES, B.FLAG_FFN_CTA_PAIR, B.FLAG_ROUTER_FP32_CORES | B.FLAG_FFN_CTA_PAIR):
         dm.flags = f
@@ -96,6 +106,8 @@ def test_workspace_and_sizes(lib):
     big = B.workspace_bytes(B.dims(100000, 1024, 64, 64, 4, 768, 768))
     assert big > small and big % 256 == 0
     assert B.aux_sums_count(good()) == 8 + 5 + 9 + 2
+    # with C + V = 5: five more slot counts and five more probability sums
+    assert B.aux_sums_count(B.dims(256, 128, 8, 8, 4, 64, 64, C=2, V=3)) == 8 + 10 + 14 + 2
     assert B.packed_gate_up_elems(good(), False) == 8 * 2 * 64 * 128
     assert B.packed_gate_up_elems(good(), True) == 2 * 64 * 128
 
@@ -108,7 +120,7 @@ def test_host_side_rejections_touch_no_device(lib):
     # null pointers with valid dims -> INVALID_ARG before any CUDA call
     assert L.moe_route(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_dispatch(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
-    assert L.moe_combine(C.byref(dm), nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_combine(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_aux(C.byref(dm), nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_forward(C.byref(dm), nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_get_device_status(nul, nul) == B.ERR_INVALID_ARG

@@ -110,3 +110,6 @@ def test_sums_layout_matches_library_count():
     from token_choice_routing_b200 import binding as B
     for N, M, K in ((8, 4, 4), (64, 8, 8), (5, 16, 16)):
         assert aux_sums_slices(N, K)["T"].stop == B.aux_sums_count(B.dims(10, 128, N, M, K, 64, 64))
+    for N, M, K, Cc, V in ((8, 4, 4, 2, 3), (60, 0, 8, 10, 5)):
+        assert aux_sums_slices(N, K, Cc + V)["T"].stop == B.aux_sums_count(B.dims(10, 128, N, M, K, 64, 64,
+                                                                                C=Cc, V=V))

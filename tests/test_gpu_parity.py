@@ -27,6 +27,8 @@ SMALL = {
     "t1": I.small_config("t1", T=1, d=128, N=8, F=64, F_shared=64, K=4, M=8, config_id=906),
     "skew_small": I.small_config("skew_small", T=512, d=256, N=64, F=128, F_shared=128, K=8, M=64,
                                  config_id=907, skew=True, seqs=2),
+    # T K > 128 N: the expert GEMMs take their 256-wide column tiles (ragged expert tails)
+    "bn256": I.small_config("bn256", T=600, d=256, N=4, F=256, F_shared=128, K=2, M=2, config_id=908),
 }
 
 
@@ -138,6 +140,65 @@ def test_decode_sized_forward_parity(name, T):
     H.check_layer_output(inp, out, r)
     assert int(offsets[-1]) == int(r["n_real"].sum())
     assert (counts == 0).sum() >= cfg.N - int(r["n_real"].sum())  # unchosen experts have empty segments
+
+
+# MoE++ copy and constant experts next to the null expert
+PP = {
+    "pp_a": I.small_config("pp_a", T=300, d=256, N=8, F=128, F_shared=128, K=4, M=4, C=2, V=2, config_id=920),
+    "pp_b": I.small_config("pp_b", T=200, d=384, N=13, F=64, F_shared=192, K=5, M=0, C=3, V=1, config_id=921),
+    "pp_80rows": I.small_config("pp_80rows", T=256, d=256, N=64, F=128, F_shared=128, K=8, M=8, C=10, V=5,
+                                config_id=922),
+    "pp_copy_only": I.small_config("pp_copy_only", T=130, d=128, N=4, F=64, F_shared=64, K=3, M=2, C=3, V=0,
+                                   config_id=923),
+    # 65 router rows with a constant expert in logit column 64
+    "pp_65rows": I.small_config("pp_65rows", T=200, d=128, N=60, F=64, F_shared=64, K=6, M=4, C=2, V=2,
+                                config_id=925),
+}
+
+
+@pytest.mark.parametrize("name", list(PP))
+def test_moepp_copy_and_constant_experts_parity(name):
+    cfg = PP[name]
+    inp = I.make_inputs(cfg)
+    inp.bias[cfg.N] = np.float32(0.4)
+    inp.bias[cfg.N + 1:] = np.float32(0.6)  # copy/constant experts chosen often enough
+    layer, x, tnb, out = H.run_forward(inp)
+    r = H.check_routing(inp, out)
+    H.check_dispatch(inp, out, r)
+    H.check_aux(inp, out, r)
+    idx = out["topk_idx"].cpu().numpy()
+    assert np.any(idx >= cfg.N + cfg.M)  # some copy/constant slots were taken
+    H.check_layer_output(inp, out, r)
+
+
+def test_moepp_null_copies_precede_copy_and_constant_experts_on_ties():
+    """Integer-valued x and 1/8-multiple weights give exact logits: the null row
+    equals copy expert 0's and constant expert 0's rows, so on equal logits the
+    null copies (pool indices N..N+M-1) must come first."""
+    cfg = I.small_config("pp_ties", T=150, d=256, N=6, F=64, F_shared=64, K=5, M=2, C=2, V=2, config_id=924)
+    inp = I.make_inputs(cfg)
+    rng = np.random.default_rng(924)
+    inp.x = I.bf16_round(rng.integers(-3, 4, size=(cfg.T, cfg.d)).astype(np.float32))
+    w = (rng.integers(-4, 5, size=(cfg.router_rows, cfg.d)) / 8.0).astype(np.float32)
+    w[cfg.N + 1] = w[cfg.N]  # copy expert 0 ties the null logit
+    w[cfg.N + 3] = w[cfg.N]  # constant expert 0 ties it too
+    inp.w_router = w
+    inp.bias[:] = 0
+    layer, x, tnb, out = H.run_forward(inp)
+    lg = out["logits"].cpu().numpy()
+    assert np.array_equal(lg, H.oracle_logits(inp).astype(np.float32))
+    r = H.check_routing(inp, out)
+    H.check_aux(inp, out, r)
+    idx = out["topk_idx"].cpu().numpy()
+    n_tie = 0
+    for t in range(cfg.T):
+        row = idx[t].tolist()
+        for sp in (cfg.N + cfg.M, cfg.N + cfg.M + cfg.C):  # copy 0, constant 0
+            if sp in row:
+                assert all(cfg.N + j in row[:row.index(sp)] for j in range(cfg.M)), row
+                n_tie += 1
+    assert n_tie > 0
+    H.check_layer_output(inp, out, r)
 
 
 def test_all_null_tokens_get_only_the_shared_expert():

@@ -27,12 +27,13 @@ class MoEError(RuntimeError):
 
 class Dims(C.Structure):
     _fields_ = [("T", C.c_int32), ("d", C.c_int32), ("N", C.c_int32), ("M", C.c_int32),
-                ("K", C.c_int32), ("F", C.c_int32), ("F_shared", C.c_int32), ("flags", C.c_uint32)]
+                ("K", C.c_int32), ("F", C.c_int32), ("F_shared", C.c_int32), ("flags", C.c_uint32),
+                ("C", C.c_int32), ("V", C.c_int32)]
 
 
 class Weights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("w_router", "router_bias", "gate_up", "w_down",
-                                           "shared_gate_up", "shared_down")]
+                                           "shared_gate_up", "shared_down", "const_vectors")]
 
 
 OUTPUT_FIELDS = ("logits", "topk_idx", "topk_gate", "n_real", "counts", "offsets", "perm_tok",
@@ -64,7 +65,7 @@ def _load() -> C.CDLL:
         "moe_expert_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_gate_up_gather": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
-        "moe_combine": (i32, [pd, vp, vp, vp, vp, vp, vp]),
+        "moe_combine": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_aux_sums_count": (sz, [pd]),
         "moe_aux_sums": (i32, [pd, vp, vp, vp]),
         "moe_aux_finalize": (i32, [pd, vp, vp, vp, vp, vp]),
@@ -78,7 +79,7 @@ def _load() -> C.CDLL:
         f = getattr(lib, name)
         f.restype = res
         f.argtypes = args
-    if lib.moe_abi_version() != 1:
+    if lib.moe_abi_version() != 2:
         raise ImportError("libmoe_null ABI version mismatch")
     return lib
 
@@ -116,8 +117,8 @@ FLAG_ROUTER_FP32_CORES = 1
 FLAG_FFN_CTA_PAIR = 2
 
 
-def dims(T, d, N, M, K, F, F_shared, flags=0) -> Dims:
-    return Dims(int(T), int(d), int(N), int(M), int(K), int(F), int(F_shared), int(flags))
+def dims(T, d, N, M, K, F, F_shared, flags=0, C=0, V=0) -> Dims:
+    return Dims(int(T), int(d), int(N), int(M), int(K), int(F), int(F_shared), int(flags), int(C), int(V))
 
 
 def check_dims(dm: Dims) -> int:
@@ -180,9 +181,11 @@ def expert_down(dm, offsets, h, h_shared, w_down, shared_down, ys, shared_out, w
                                                   _stream(stream)))
 
 
-def combine(dm, ys, shared_out, topk_gate, slot_row, y, stream=None):
-    _check("moe_combine", LIB.moe_combine(C.byref(dm), _p(ys), _p(shared_out), _p(topk_gate),
-                                          _p(slot_row), _p(y), _stream(stream)))
+def combine(dm, ys, shared_out, topk_gate, slot_row, y, stream=None, topk_idx=None, x=None,
+            const_vectors=None):
+    """topk_idx, x and const_vectors are needed only with MoE++ copy/constant experts."""
+    _check("moe_combine", LIB.moe_combine(C.byref(dm), _p(ys), _p(shared_out), _p(topk_gate), _p(slot_row),
+                                          _p(topk_idx), _p(x), _p(const_vectors), _p(y), _stream(stream)))
 
 
 def aux(dm, ws, counts_ext, P, losses, stream=None):

@@ -27,7 +27,12 @@ int check_dims(const moe_dims_t* d) {
   if ((d->flags & ~(MOE_FLAG_ROUTER_FP32_CORES | MOE_FLAG_FFN_CTA_PAIR)) != 0u) return MOE_ERR_INVALID_ARG;
   if (d->T < 0 || d->d <= 0 || d->N < 1 || d->M < 0 || d->K < 1 || d->F <= 0 || d->F_shared <= 0)
     return MOE_ERR_INVALID_ARG;
-  if ((long long)d->K > (long long)d->N + d->M) return MOE_ERR_INVALID_ARG;
+  if (d->C < 0 || d->V < 0) return MOE_ERR_INVALID_ARG;
+  if ((long long)d->K > (long long)d->N + d->M + d->C + d->V) return MOE_ERR_INVALID_ARG;
+  if (d->C + d->V > 0) {  // MoE++ copy/constant experts: tensor-core router, one 80-row router tile
+    if (d->C + d->V > kMaxPP || router_rows(*d) > kMaxRows) return MOE_ERR_UNSUPPORTED;
+    if (route_fp32_cores(*d)) return MOE_ERR_UNSUPPORTED;
+  }
   if (d->N > kMaxN || d->K > kMaxK) return MOE_ERR_UNSUPPORTED;
   if (d->d % 128 != 0 || d->d > 8192) return MOE_ERR_UNSUPPORTED;
   if (d->F % 64 != 0 || d->F > 16384 || d->F_shared % 64 != 0 || d->F_shared > 16384)
@@ -156,11 +161,14 @@ int moe_expert_down(const moe_dims_t* dims, const int32_t* offsets, const uint16
 }
 
 int moe_combine(const moe_dims_t* dims, const uint16_t* ys, const uint16_t* shared_out, const float* topk_gate,
-                const int32_t* slot_row, uint16_t* y, moe_stream_t stream) {
+                const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x, const uint16_t* const_vectors,
+                uint16_t* y, moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));
   if (dims->T == 0) return MOE_OK;
   if (!ys || !shared_out || !topk_gate || !slot_row || !y) return MOE_ERR_INVALID_ARG;
-  return launch_combine(*dims, ys, shared_out, topk_gate, slot_row, y, S(stream));
+  if (dims->C + dims->V > 0 && (!topk_idx || (dims->C > 0 && !x) || (dims->V > 0 && !const_vectors)))
+    return MOE_ERR_INVALID_ARG;
+  return launch_combine(*dims, ys, shared_out, topk_gate, slot_row, topk_idx, x, const_vectors, y, S(stream));
 }
 
 int moe_aux_sums(const moe_dims_t* dims, const void* workspace, double* sums, moe_stream_t stream) {
@@ -192,6 +200,7 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
   if (!w || !out || !x || !workspace) return MOE_ERR_INVALID_ARG;
   if (!w->w_router || !w->gate_up || !w->w_down || !w->shared_gate_up || !w->shared_down)
     return MOE_ERR_INVALID_ARG;
+  if (dims->V > 0 && !w->const_vectors) return MOE_ERR_INVALID_ARG;
   if (!out->topk_idx || !out->topk_gate || !out->n_real || !out->counts || !out->offsets || !out->perm_tok ||
       !out->slot_row || !out->h || !out->h_shared || !out->ys || !out->shared_out || !out->y ||
       !out->counts_ext || !out->P || !out->losses)
@@ -206,7 +215,8 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
                                 w->shared_gate_up, out->h, out->h_shared, workspace, st));
   MOE_CHECK(launch_down(*dims, out->offsets, out->h, out->h_shared, w->w_down, w->shared_down, out->ys,
                         out->shared_out, workspace, st));
-  return launch_combine(*dims, out->ys, out->shared_out, out->topk_gate, out->slot_row, out->y, st);
+  return launch_combine(*dims, out->ys, out->shared_out, out->topk_gate, out->slot_row, out->topk_idx, x,
+                        w->const_vectors, out->y, st);
 }
 
 int moe_get_device_status(const void* workspace, moe_stream_t stream) {

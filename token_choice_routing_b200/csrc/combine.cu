@@ -1,7 +1,9 @@
 // moe_combine: y[t] = E_shared(x_t) + sum over the token's real slots of
 // g_{t,k} * E_e(x_t) (Kilian et al., "Improving MoE Compute Efficiency by
 // Composing Weight and Data Sparsity", review page, section 三 / 核心公式).
-// Null experts output zero, so null slots (slot_row = -1) are skipped.
+// Null experts output zero, so null slots (slot_row = -1) are skipped. MoE++
+// copy experts add g x_t and constant expert j adds g c_j (MoE++ explainer page,
+// 三种零计算专家); they have no ys row either, and are told apart by topk_idx.
 // Written as a gather (each token reads its own rows of ys) so it is
 // deterministic: fp32 accumulation in rank order, one bf16 rounding.
 #include "moe_internal.cuh"
@@ -14,11 +16,14 @@ constexpr int kCombineThreads = 256;
 // shared row's chunks and the chunks of the first four slots are loaded
 // together before any is used (null slots load nothing); the next token's slot
 // list is fetched while this one is combined. Sum order: shared, then slots in
-// rank order.
+// rank order. A slot's source row is coded as: >= 0 a row of ys, -1 nothing
+// (null copy), -2 the token's row of x (copy expert), -3 - j constant vector j.
 __global__ void __launch_bounds__(kCombineThreads, 3)
 combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
                const float* __restrict__ gate, const int32_t* __restrict__ slot_row,
-               uint16_t* __restrict__ y, int T, int d, int K, long long rcap, uint32_t* status) {
+               const int32_t* __restrict__ topk_idx, const uint16_t* __restrict__ x,
+               const uint16_t* __restrict__ cv, uint16_t* __restrict__ y, int T, int d, int K, long long rcap,
+               int NM, int C, int V, uint32_t* status) {
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const int wpb = kCombineThreads / 32;
@@ -34,6 +39,11 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
       if (row >= rcap) {
         if (status) atomicOr(status, kStatusBounds);
         row = -1;
+      }
+      if (row < 0 && C + V > 0) {
+        const int id = __ldg(topk_idx + (size_t)tt * K + lane) - NM;  // position among copy/constant
+        if (id >= 0 && id < C) row = -2;
+        else if (id >= C && id < C + V) row = -3 - (id - C);
       }
     }
   };
@@ -65,9 +75,13 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
           rq[u] = __shfl_sync(0xffffffffu, row, k & 31);
           gq[u] = __shfl_sync(0xffffffffu, g, k & 31);
           if (k >= K) rq[u] = -1;
-          const uint4* src = reinterpret_cast<const uint4*>(ys + (size_t)(rq[u] < 0 ? 0 : rq[u]) * d);
-          va[u] = (rq[u] >= 0 && oka) ? __ldg(src + ca) : make_uint4(0u, 0u, 0u, 0u);
-          vb[u] = (rq[u] >= 0 && okb) ? __ldg(src + cb) : make_uint4(0u, 0u, 0u, 0u);
+          const uint16_t* srow = (rq[u] >= 0)    ? ys + (size_t)rq[u] * d
+                                 : (rq[u] == -2) ? x + (size_t)t * d
+                                 : (rq[u] <= -3) ? cv + (size_t)(-3 - rq[u]) * d
+                                                 : ys;
+          const uint4* src = reinterpret_cast<const uint4*>(srow);
+          va[u] = (rq[u] != -1 && oka) ? __ldg(src + ca) : make_uint4(0u, 0u, 0u, 0u);
+          vb[u] = (rq[u] != -1 && okb) ? __ldg(src + cb) : make_uint4(0u, 0u, 0u, 0u);
         }
         if (k0 == 0) {
           acc_a[0] = bf16lo(sa.x); acc_a[1] = bf16hi(sa.x); acc_a[2] = bf16lo(sa.y); acc_a[3] = bf16hi(sa.y);
@@ -77,7 +91,7 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          if (rq[u] >= 0) {
+          if (rq[u] != -1) {
             fma8(acc_a, gq[u], va[u]);
             fma8(acc_b, gq[u], vb[u]);
           }
@@ -98,7 +112,8 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
 }
 
 int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
-                   const float* topk_gate, const int32_t* slot_row, uint16_t* y, cudaStream_t st) {
+                   const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st) {
   // one wave of resident CTAs; each warp then loops over tokens
   static int per_sm[64] = {0};
   int dev = 0;
@@ -115,7 +130,8 @@ int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shar
   const int cap = sm_count() * occ;
   if (grid > cap) grid = cap;
   return launch_pdl(combine_kernel, dim3(grid), dim3(kCombineThreads), 0, st, ys, shared_out, topk_gate, slot_row,
-                    y, d.T, d.d, d.K, (long long)d.T * d.K, nullptr);
+                    topk_idx, x, const_vectors, y, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, d.V,
+                    nullptr);
 }
 
 }  // namespace moe

@@ -10,31 +10,36 @@
 // which is the stable (expert, token) order. Null slots are skipped before any
 // load, so they cost no memory traffic.
 //
-// Aux (same page, 负载均衡损失 and Z-Loss): L_bal = N * sum_{i<N+M} f_i P_i with
-// f_i = count_i / T and P_i = mean_t p_{t,i}; L_z = mean_t lse_t^2. Per-block
-// fp32 partials from the route kernel are summed in fp64, first over fixed
-// slices of blocks (in the scan launch), then over the slices here.
+// Aux (same page, 负载均衡损失 and Z-Loss): L_bal = N * sum_i f_i P_i over the pool
+// (reals, null copies, and MoE++ copy/constant experts when present) with f_i =
+// count_i / T and P_i = mean_t p_{t,i}; L_z = mean_t lse_t^2. Per-block fp32
+// partials from the route kernel are summed in fp64, first over fixed slices of
+// blocks (in the scan launch), then over the slices here.
 #include "moe_internal.cuh"
 
 namespace moe {
 
 struct AuxPtrs {
   const int32_t* counts;  // [N] real counts (route scan)
-  const double* auxp;     // [nparts][(N+1) + (K+1) + 1] fp64 partials (scan launch)
-  int nparts, N, M, K, T;
+  const double* auxp;     // [nparts][(N+1+C+V) + (K+1+C+V) + 1] fp64 partials (scan launch)
+  int nparts, N, M, K, T, C, V;
 };
 
-// sums layout: [counts_real N | hist K+1 | psum N+1 | lsq | T]. The first-level
-// partials (at most kAuxParts = 64 of them) are combined one column per warp:
-// lane l adds partials l and l+32, then a fixed shuffle tree (deterministic).
+// Most doubles the sums of one layer can take (see aux_sums_count).
+constexpr int kMaxSums = kMaxN + (kMaxK + 1 + kMaxPP) + kMaxRows + 2;
+
+// sums layout: [counts_real N | hist K+1+C+V (null slots per token, then per copy /
+// constant expert) | psum N+1+C+V (per router row) | lsq | T]. The first-level partials
+// (at most kAuxParts = 64 of them) are combined one column per warp: lane l adds
+// partials l and l+32, then a fixed shuffle tree (deterministic).
 __device__ void aux_sums_block(const AuxPtrs& p, double* sums) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-  const int N = p.N, K = p.K;
+  const int N = p.N, K = p.K, PP = p.C + p.V;
   double* s_cnt = sums;
   double* s_hist = sums + N;
-  double* s_psum = s_hist + (K + 1);
-  double* s_lsq = s_psum + (N + 1);
-  const int c1 = N + 1, c2 = c1 + K + 1, cols = c2 + 1;
+  double* s_psum = s_hist + (K + 1 + PP);
+  double* s_lsq = s_psum + (N + 1 + PP);
+  const int c1 = N + 1 + PP, c2 = c1 + K + 1 + PP, cols = c2 + 1;
   for (int e = tid; e < N; e += blockDim.x) s_cnt[e] = (double)p.counts[e];
   for (int c = warp; c < cols; c += nwarps) {
     double acc = 0.0;
@@ -52,24 +57,29 @@ __device__ void aux_sums_block(const AuxPtrs& p, double* sums) {
   __syncthreads();
 }
 
-__device__ void aux_finalize_block(const double* sums, int N, int M, int K, int32_t* counts_ext,
+__device__ void aux_finalize_block(const double* sums, int N, int M, int K, int PP, int32_t* counts_ext,
                                    float* P, float* losses) {
   const int tid = threadIdx.x;
   const double* s_cnt = sums;
   const double* s_hist = sums + N;
-  const double* s_psum = s_hist + (K + 1);
-  const double Tt = s_psum[N + 1 + 1];
+  const double* s_psum = s_hist + (K + 1 + PP);
+  const double lsq = s_psum[N + 1 + PP];
+  const double Tt = s_psum[N + 1 + PP + 1];
   const double inv = Tt > 0.0 ? 1.0 / Tt : 0.0;
-  for (int i = tid; i < N + M; i += blockDim.x) {
+  for (int i = tid; i < N + M + PP; i += blockDim.x) {
     if (i < N) {
       if (counts_ext) counts_ext[i] = (int32_t)s_cnt[i];
       if (P) P[i] = (float)(s_psum[i] * inv);
-    } else {
-      const int j = i - N;  // copy j is taken by tokens with more than j null slots
+    } else if (i < N + M) {
+      const int j = i - N;  // null copy j is taken by tokens with more than j null slots
       double c = 0.0;
       for (int q = j + 1; q <= K; ++q) c += s_hist[q];
       if (counts_ext) counts_ext[i] = (int32_t)c;
       if (P) P[i] = (float)(s_psum[N] * inv);
+    } else {
+      const int j = i - N - M;  // copy or constant expert j: its own count and probability
+      if (counts_ext) counts_ext[i] = (int32_t)s_hist[K + 1 + j];
+      if (P) P[i] = (float)(s_psum[N + 1 + j] * inv);
     }
   }
   if (tid == 0 && losses) {
@@ -78,16 +88,17 @@ __device__ void aux_finalize_block(const double* sums, int N, int M, int K, int3
     double nulls = 0.0;
     for (int q = 1; q <= K; ++q) nulls += (double)q * s_hist[q];
     acc += nulls * s_psum[N];
+    for (int j = 0; j < PP; ++j) acc += s_hist[K + 1 + j] * s_psum[N + 1 + j];
     losses[0] = (float)((double)N * acc * inv * inv);
-    losses[1] = (float)(s_psum[N + 1] * inv);
+    losses[1] = (float)(lsq * inv);
   }
 }
 
 __global__ void __launch_bounds__(256) aux_kernel(AuxPtrs p, double* sums_out, const double* sums_in,
                                                   int32_t* counts_ext, float* P, float* losses) {
   pdl_wait_then_release();
-  __shared__ double s_sums[kMaxN + kMaxK + 1 + kMaxN + 1 + 2];
-  const int n = p.N + (p.K + 1) + (p.N + 1) + 2;
+  __shared__ double s_sums[kMaxSums];
+  const int n = p.N + (p.K + 1 + p.C + p.V) + (p.N + 1 + p.C + p.V) + 2;
   if (sums_in == nullptr) {
     aux_sums_block(p, s_sums);
     if (sums_out)
@@ -96,7 +107,7 @@ __global__ void __launch_bounds__(256) aux_kernel(AuxPtrs p, double* sums_out, c
     for (int i = threadIdx.x; i < n; i += blockDim.x) s_sums[i] = sums_in[i];
     __syncthreads();
   }
-  if (counts_ext || P || losses) aux_finalize_block(s_sums, p.N, p.M, p.K, counts_ext, P, losses);
+  if (counts_ext || P || losses) aux_finalize_block(s_sums, p.N, p.M, p.K, p.C + p.V, counts_ext, P, losses);
 }
 
 struct DispatchArgs {
@@ -129,11 +140,12 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
   int blk = blockIdx.x;
   if (a.fuse_aux) {
     if (blk == 0) {  // scheduled first, so the reduction overlaps the gather
-      __shared__ double s_sums[kMaxN + kMaxK + 1 + kMaxN + 1 + 2];
+      __shared__ double s_sums[kMaxSums];
       aux_sums_block(a.aux, s_sums);
       if (a.sums)
-        for (int i = threadIdx.x; i < a.N + a.K + 1 + a.N + 1 + 2; i += blockDim.x) a.sums[i] = s_sums[i];
-      aux_finalize_block(s_sums, a.N, a.M, a.K, a.counts_ext, a.P, a.losses);
+        for (int i = threadIdx.x; i < a.N + 2 * (a.aux.C + a.aux.V) + a.K + 1 + a.N + 1 + 2; i += blockDim.x)
+          a.sums[i] = s_sums[i];
+      aux_finalize_block(s_sums, a.N, a.M, a.K, a.aux.C + a.aux.V, a.counts_ext, a.P, a.losses);
       return;
     }
     --blk;
@@ -162,7 +174,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
         } else {
           a.perm_tok[dest] = t;
         }
-      } else if (id < 0 || id >= N + a.M) {
+      } else if (id < 0 || id >= N + a.M + a.aux.C + a.aux.V) {
         atomicOr(a.status, kStatusBounds);
       }
       a.slot_row[(size_t)t * K + lane] = dest;
@@ -191,6 +203,8 @@ static AuxPtrs aux_ptrs(const moe_dims_t& d, const void* ws) {
   p.M = d.M;
   p.K = d.K;
   p.T = d.T;
+  p.C = d.C;
+  p.V = d.V;
   return p;
 }
 

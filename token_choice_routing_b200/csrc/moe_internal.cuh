@@ -22,6 +22,8 @@ constexpr int kRouteThreads = 64 + kRouteEpiThreads;       // + TMA warp + MMA w
 constexpr int kFp32RouteTokens = 64;                       // tokens per CTA of the fp32 CUDA-core route
 constexpr int kMaxN = 64;
 constexpr int kMaxK = 16;
+constexpr int kMaxPP = 16;     // MoE++ copy + constant experts
+constexpr int kMaxRows = 80;   // router rows N + 1 + C + V (one tensor-core tile of three terms)
 
 // Status bits recorded on the device (the host maps them to moe_status_t).
 constexpr uint32_t kStatusTimeout = 1u;
@@ -40,16 +42,16 @@ struct WsLayout {
   size_t hdr;        // uint32 status at 0; int32 per-expert totals at kHdrTotOffset (512 B)
   size_t counts_blk; // int32 [N][nblk]
   size_t bases;      // int32 [N][nblk]
-  size_t ppart;      // float [nblk][N+1]
+  size_t ppart;      // float [nblk][N+1+C+V]
   size_t lsq;        // float [nblk]
-  size_t hist;       // int32 [nblk][K+1]
+  size_t hist;       // int32 [nblk][K+1+C+V]: null histogram, then copy/constant expert counts
   size_t lrank;      // int32 [T][K]
   size_t counts;     // int32 [N]
   size_t offsets;    // int32 [N+1]
   size_t sums;       // double [aux sums count]
   int nparts;        // first-level aux partials = min(kAuxParts, nblk)
   size_t auxp;       // double [nparts][aux_part_cols]
-  size_t wprep;      // router weight prepared for this call: bf16 [3 * route_npw(N)][d] (three
+  size_t wprep;      // router weight prepared for this call: bf16 [3 * route_npw][d] (three
                      // terms hi, mid, lo) or, for the fp32 CUDA-core route, W_r^T fp32 [d][npad + 4]
   size_t total;
 };
@@ -59,11 +61,17 @@ constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // First-level aux partials: each of up to kAuxParts CTAs reduces a fixed,
 // contiguous slice of route blocks in fp64: [sum p (N+1) | null hist (K+1) | sum lse^2].
 constexpr int kAuxParts = 64;
-inline int aux_part_cols(const moe_dims_t& d) { return (d.N + 1) + (d.K + 1) + 1; }
+// MoE++ copy + constant experts, and the column counts that follow from them: router
+// rows / logits (N real, the null logit, C + V), per-block probability sums (one per
+// router row) and per-block slot counts (null histogram K+1, then one per C/V expert).
+inline int pp_experts(const moe_dims_t& d) { return d.C + d.V; }
+inline int router_rows(const moe_dims_t& d) { return d.N + 1 + pp_experts(d); }
+inline int hist_cols(const moe_dims_t& d) { return d.K + 1 + pp_experts(d); }
+inline int aux_part_cols(const moe_dims_t& d) { return router_rows(d) + hist_cols(d) + 1; }
 
-// Rows per bf16 term of the split router weight: the N+1 logits padded to a
+// Rows per bf16 term of the split router weight: the router rows padded to a
 // multiple of 16 (16 .. 80), so the three terms together are one MMA of N <= 240.
-inline int route_npw(int N) { return (N + 1 + 15) / 16 * 16; }
+inline int route_npw(const moe_dims_t& d) { return (router_rows(d) + 15) / 16 * 16; }
 
 // Real-logit count the fp32 CUDA-core route pads N to (8, 16, 32 or 64).
 inline int route_fp32_npad(int N) { return N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : 64; }
@@ -75,8 +83,9 @@ inline int route_block_tokens(const moe_dims_t& d) {
   return route_fp32_cores(d) ? kFp32RouteTokens : kRouteTokens;
 }
 
+// [counts_real (N) | slot counts (hist_cols) | probability sums (router_rows) | lse^2 | T]
 inline size_t aux_sums_count(const moe_dims_t& d) {
-  return (size_t)d.N + (size_t)(d.K + 1) + (size_t)(d.N + 1) + 2;
+  return (size_t)d.N + (size_t)hist_cols(d) + (size_t)router_rows(d) + 2;
 }
 
 inline WsLayout ws_layout(const moe_dims_t& d) {
@@ -87,9 +96,9 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   L.hdr = o; o += 512;
   L.counts_blk = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N * L.nblk, 256);
   L.bases = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N * L.nblk, 256);
-  L.ppart = o; o = align_up(o + sizeof(float) * (size_t)(d.N + 1) * L.nblk, 256);
+  L.ppart = o; o = align_up(o + sizeof(float) * (size_t)router_rows(d) * L.nblk, 256);
   L.lsq = o; o = align_up(o + sizeof(float) * (size_t)L.nblk, 256);
-  L.hist = o; o = align_up(o + sizeof(int32_t) * (size_t)(d.K + 1) * L.nblk, 256);
+  L.hist = o; o = align_up(o + sizeof(int32_t) * (size_t)hist_cols(d) * L.nblk, 256);
   L.lrank = o; o = align_up(o + sizeof(int32_t) * (size_t)d.T * d.K, 256);
   L.counts = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N, 256);
   L.offsets = o; o = align_up(o + sizeof(int32_t) * (size_t)(d.N + 1), 256);
@@ -98,7 +107,7 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   L.auxp = o; o = align_up(o + sizeof(double) * (size_t)L.nparts * aux_part_cols(d), 256);
   L.wprep = o;
   o = align_up(o + (route_fp32_cores(d) ? sizeof(float) * (size_t)d.d * (route_fp32_npad(d.N) + 4)
-                                        : sizeof(uint16_t) * 3 * (size_t)route_npw(d.N) * d.d),
+                                        : sizeof(uint16_t) * 3 * (size_t)route_npw(d) * d.d),
                256);
   L.total = o;
   return L;
@@ -170,8 +179,8 @@ int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_
 int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const double* sums_in,
                int32_t* counts_ext, float* P, float* losses, cudaStream_t st);
 int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
-                   const float* topk_gate, const int32_t* slot_row, uint16_t* y,
-                   cudaStream_t st);
+                   const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st);
 // perm (optional): token of each routed row; when given, gate/up gathers the
 // routed rows of x by TMA instead of reading a gathered copy xs (xs unused).
 int launch_gate_up_perm(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,

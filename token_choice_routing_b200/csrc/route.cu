@@ -56,11 +56,12 @@ struct RouteArgs {
   int32_t* offsets;
   unsigned long long limit_ns;
   int T, d, N, M, K, nblk;
+  int ncols;  // router rows N + 1 + C + V (MoE++ copy and constant experts after the null logit)
 };
 
 // ---------------------------------------------------------------------------------------
-// W_r (fp32 [N+1][d]) -> three bf16 terms, rows t*NPW + j (t = 0 hi, 1 mid, 2 lo),
-// zero rows for N < j < NPW. With w = m 2^e (24-bit m): hi = RN8(w) leaves a
+// W_r (fp32 [rows][d], rows = N+1+C+V) -> three bf16 terms, rows t*NPW + j (t = 0 hi,
+// 1 mid, 2 lo), zero rows for rows <= j < NPW. With w = m 2^e (24-bit m): hi = RN8(w) leaves a
 // remainder of at most 16 significant bits, mid = RN8(remainder) leaves at most
 // 8, and lo holds those exactly; both subtractions are exact in fp32.
 __device__ __forceinline__ void split3(float w, uint16_t& h, uint16_t& m, uint16_t& l) {
@@ -78,7 +79,7 @@ __device__ __forceinline__ void split3(float w, uint16_t& h, uint16_t& m, uint16
 // `nclear` words of the workspace header (status word and per-expert totals),
 // which must start at zero for every layer call.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, uint16_t* __restrict__ w3,
-                                                           int N, int npw, int d, uint32_t* hdr, int nclear) {
+                                                           int rows, int npw, int d, uint32_t* hdr, int nclear) {
   pdl_wait_then_release();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nclear; i += blockDim.x) hdr[i] = 0u;
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
        i += (long long)gridDim.x * blockDim.x) {
     const int j = (int)(i / nch), c = (int)(i - (long long)j * nch);
     uint16_t hv[8], mv[8], lv[8];
-    if (j <= N) {
+    if (j < rows) {
       const float4* src = reinterpret_cast<const float4*>(w + (size_t)j * d + (size_t)c * 8);
       const float4 p0 = __ldg(src), p1 = __ldg(src + 1);
       const float v[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -131,8 +132,9 @@ struct RouteSmem {
   static constexpr size_t off_tk = off_mask + sizeof(unsigned long long) * kRouteTokens;  // int [128][kMaxK]
   static constexpr size_t off_tkv = off_tk + sizeof(int) * kRouteTokens * kMaxK;          // float [128][kMaxK]
   static constexpr size_t off_tokbits = off_tkv + sizeof(float) * kRouteTokens * kMaxK;  // u32 [4][kMaxN]
-  static constexpr size_t off_hist = off_tokbits + sizeof(unsigned) * 4 * kMaxN;         // int [kMaxK+1]
-  static constexpr size_t scratch_end = off_hist + sizeof(int) * (kMaxK + 1);
+  static constexpr int HIST = kMaxK + 1 + kMaxPP;  // null histogram + copy/constant counts
+  static constexpr size_t off_hist = off_tokbits + sizeof(unsigned) * 4 * kMaxN;         // int [HIST]
+  static constexpr size_t scratch_end = off_hist + sizeof(int) * HIST;
   static_assert(scratch_end <= ring_end, "routing scratch must fit in the staging ring");
   static constexpr size_t off_bar = ring_end;  // full[STAGES], empty[STAGES], tfull
   static constexpr size_t off_misc = off_bar + 8 * (2 * STAGES + 1);  // [0] TMEM base, [1] abort
@@ -161,7 +163,9 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
 
 // ---------------------------------------------------------------------------------------
 // One CTA: tokens [128 b, 128 b + 128) x all N+1 logits, 576 threads.
-template <int NPW>
+// NQ: logit columns per lane (4 lanes per token): NPW / 4, or 16 when NPW = 80 and
+// there are no copy/constant experts (the candidates are then the reals, columns < 64).
+template <int NPW, int NQ>
 __global__ void __launch_bounds__(kRouteThreads, 1)
     route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const RouteArgs a) {
@@ -169,7 +173,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   using SM = RouteSmem<NPW>;
   constexpr int STAGES = SM::STAGES;
   constexpr int LS = SM::LS;
-  constexpr int NQ = (NPW < kMaxN ? NPW : kMaxN) / 4;  // reals per lane, 4 lanes per token
   constexpr uint32_t TCOLS = SM::BROWS <= 64 ? 64u : SM::BROWS <= 128 ? 128u : 256u;
   constexpr uint32_t IDESC = idesc_bf16_f32(kRouteTokens, SM::BROWS);
   constexpr uint32_t TX = SM::A_BYTES + SM::B_BYTES;
@@ -277,7 +280,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       const int t = q * 32 + lane;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
       const float tn = (a.tnb != nullptr && t < nvalid) ? __ldg(a.tnb + tok0 + t) : 0.f;
-      if (etid <= kMaxK) s_hist[etid] = 0;  // the staging ring is free from here on
+      if (etid < SM::HIST) s_hist[etid] = 0;  // the staging ring is free from here on
 #pragma unroll 1
       for (int c0 = part * 8; c0 < NPW; c0 += 32) {
         uint32_t rh[8], rm[8], rl[8];
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int col = c0 + j;
-          if (col <= N) {
+          if (col < a.ncols) {
             float s = (__uint_as_float(rh[j]) + __uint_as_float(rm[j])) + __uint_as_float(rl[j]);
             if (a.bias) s += __ldg(a.bias + col);
             if (col == N) s += tn;
@@ -300,17 +303,22 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     named_bar_sync(1, kRouteEpiThreads);
 
     if (run) {
-      // ---- per-token routing, 4 lanes per token (lane q holds reals q, q+4, ...)
+      // ---- per-token routing, 4 lanes per token. Lane q holds the distinct candidates
+      // in logit columns i = q, q+4, ...: reals (i < N, pool index i) and MoE++ copy and
+      // constant experts (N < i < ncols, pool index i - 1 + M); column N is the null logit.
       const int t = etid >> 2, q = etid & 3;
       const bool valid = t < nvalid;
       const int tok = tok0 + t;
+      const int ncols = a.ncols;
+      auto is_cand = [&](int i) { return i < ncols && i != N; };
+      auto pool_of = [&](int i) { return i < N ? i : i - 1 + M; };
       float* row = s_l + t * LS;
       const float sn = row[N];
       float v[NQ];
 #pragma unroll
       for (int u = 0; u < NQ; ++u) {
         const int i = q + 4 * u;
-        v[u] = (i < N) ? row[i] : -INFINITY;
+        v[u] = is_cand(i) ? row[i] : -INFINITY;
       }
       // softmax statistics over the pool (M copies of the null logit)
       float m = -INFINITY;
@@ -325,7 +333,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       float z = 0.f;
 #pragma unroll
       for (int u = 0; u < NQ; ++u) {
-        e[u] = (q + 4 * u < N) ? __expf(v[u] - m) : 0.f;
+        e[u] = is_cand(q + 4 * u) ? __expf(v[u] - m) : 0.f;
         z += e[u];
       }
       z += __shfl_xor_sync(0xffffffffu, z, 1);
@@ -339,28 +347,29 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 #pragma unroll
       for (int u = 0; u < NQ; ++u) {
         const int i = q + 4 * u;
-        if (i < N) row[i] = e[u] * rz;
+        if (is_cand(i)) row[i] = e[u] * rz;
       }
       if (q == 0) {
         pn[t] = (M > 0) ? en * rz : 0.f;
         lse2[t] = lse * lse;
       }
 
-      // top-K over the pool, in rank order: K rounds of "best remaining real"
-      // against the null logit (a real equal to it wins: lower index)
+      // top-K over the pool, in rank order: K rounds of "best remaining candidate"
+      // against the next null copy, compared by (value desc, pool index asc): a real
+      // equal to the null logit wins, a copy or constant expert equal to it loses
       unsigned sel = 0u;
-      int used = 0, r = 0;
+      int used = 0, r = 0, rpp = 0;
       unsigned long long msk = 0ull;
-      float smax = 0.f;  // the first real taken is the largest real logit
+      float smax = 0.f;  // the first non-null slot taken holds the largest gated logit
       for (int k = 0; k < K; ++k) {
         float bv = -INFINITY;
         int bi = INT_MAX;
 #pragma unroll
         for (int u = 0; u < NQ; ++u) {
           const int i = q + 4 * u;
-          if (i < N && !((sel >> u) & 1u) && ranks_before(v[u], i, bv, bi)) {
+          if (is_cand(i) && !((sel >> u) & 1u) && ranks_before(v[u], pool_of(i), bv, bi)) {
             bv = v[u];
-            bi = i;
+            bi = pool_of(i);
           }
         }
 #pragma unroll
@@ -372,48 +381,55 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
             bi = oi;
           }
         }
-        const bool take_null = (used < M) && (bi == INT_MAX || bv < sn);
+        const bool take_null = (used < M) && (bi == INT_MAX || ranks_before(sn, N + used, bv, bi));
         int id;
         if (take_null) {
           id = N + used;
           ++used;
         } else {
           id = bi;
-          if (r == 0) smax = bv;
-          ++r;
-          msk |= 1ull << bi;
-          if ((bi & 3) == q) sel |= 1u << (bi >> 2);
+          if (r + rpp == 0) smax = bv;
+          if (bi < N) {
+            ++r;
+            msk |= 1ull << bi;
+          } else {
+            ++rpp;
+          }
+          const int ci = (bi < N) ? bi : bi - M + 1;  // logit column of the candidate taken
+          if ((ci & 3) == q) sel |= 1u << (ci >> 2);
         }
         if ((k & 3) == q) {  // slot k belongs to lane k mod 4 from here on
           tk[t * kMaxK + k] = id;
           tkv[t * kMaxK + k] = bv;
         }
       }
-      // gates: softmax over the selected real logits; each lane takes slots q, q+4, ...
-      // and the four partial sums are added in a fixed order
+      // gates: softmax over the selected slots that are not null copies; each lane takes
+      // slots q, q+4, ... and the four partial sums are added in a fixed order
+      auto gated = [&](int id) { return id < N || id >= N + M; };
       float gsum = 0.f;
       for (int k = q; k < K; k += 4)
-        if (tk[t * kMaxK + k] < N) gsum += expf(tkv[t * kMaxK + k] - smax);
+        if (gated(tk[t * kMaxK + k])) gsum += expf(tkv[t * kMaxK + k] - smax);
       gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
       gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
       if (valid) {
         for (int k = q; k < K; k += 4) {
           const int id = tk[t * kMaxK + k];
-          const float g = (id < N) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
+          const float g = gated(id) ? expf(tkv[t * kMaxK + k] - smax) / gsum : 0.f;
           a.topk_idx[(size_t)tok * K + k] = id;
           a.topk_gate[(size_t)tok * K + k] = g;
+          if (id >= N + M) atomicAdd(s_hist + (K + 1) + (id - N - M), 1);  // copy/constant counts
         }
         if (q == 0) {
           a.n_real[tok] = r;
-          atomicAdd(s_hist + (K - r), 1);  // integer: the histogram does not depend on the order
+          atomicAdd(s_hist + (K - r - rpp), 1);  // null slots; integer: order does not matter
         }
         mask[t] = msk;  // identical on the token's four lanes
         if (a.logits) {
-          float* lo = a.logits + (size_t)tok * (N + 1);
+          float* lo = a.logits + (size_t)tok * ncols;
 #pragma unroll
           for (int u = 0; u < NQ; ++u) {
             const int i = q + 4 * u;
-            if (i < N) lo[i] = v[u];
+            if (is_cand(i)) lo[i] = v[u];
           }
           if (q == 0) lo[N] = sn;
         }
@@ -438,10 +454,12 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           if (lane == 0) tokbits[g * kMaxN + e] = bits;
         }
       }
-      for (int c = ew; c <= N + 1; c += 16) {
-        // c < N: real column c; c == N: the null probability; c == N + 1: lse^2
-        const float* col = (c < N) ? s_l + c : (c == N) ? pn : lse2;
-        const int stride = (c < N) ? LS : 1;
+      const int ncols = a.ncols;
+      for (int c = ew; c <= ncols; c += 16) {
+        // c < ncols: probability of logit column c (real, the null logit for c == N, copy
+        // or constant expert); c == ncols: lse^2
+        const float* col = (c == N) ? pn : (c < ncols) ? s_l + c : lse2;
+        const int stride = (c == N || c == ncols) ? 1 : LS;
         float sum = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -451,7 +469,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane == 0) {
-          if (c <= N) a.ppart[(size_t)b * (N + 1) + c] = sum;
+          if (c < ncols) a.ppart[(size_t)b * ncols + c] = sum;
           else a.lsq[b] = sum;
         }
       }
@@ -459,7 +477,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     named_bar_sync(1, kRouteEpiThreads);
 
     if (run) {
-      if (etid <= K) a.hist[(size_t)b * (K + 1) + etid] = s_hist[etid];
+      const int hc = K + 1 + (a.ncols - N - 1);  // null histogram, then copy/constant counts
+      if (etid < hc) a.hist[(size_t)b * hc + etid] = s_hist[etid];
       if (etid < N) {
         int cnt = 0;
 #pragma unroll
@@ -508,11 +527,12 @@ struct ScanArgs {
   int32_t* counts;
   int32_t* offsets;
   // first-level aux reduction (CTAs N .. N+nparts-1)
-  const float* ppart;   // [nblk][N+1]
-  const int32_t* hist;  // [nblk][K+1]
+  const float* ppart;   // [nblk][ncols]
+  const int32_t* hist;  // [nblk][hcols]
   const float* lsq;     // [nblk]
-  double* auxp;         // [nparts][cols]
+  double* auxp;         // [nparts][ncols + hcols + 1]
   int N, K, nblk, nparts;
+  int ncols, hcols;     // router rows; null histogram + copy/constant expert counts
 };
 
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
@@ -526,14 +546,14 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
     // fp64 partial sums of the aux statistics over a fixed slice of route blocks
     const int g = blockIdx.x - N;
     const int b0 = (int)((long long)g * nblk / a.nparts), b1 = (int)((long long)(g + 1) * nblk / a.nparts);
-    const int c1 = N + 1, c2 = c1 + a.K + 1, cols = c2 + 1;
+    const int c1 = a.ncols, c2 = c1 + a.hcols, cols = c2 + 1;
     const int nph = kScanThreads / cols;
     const int col = tid % cols, ph = tid / cols;
     double acc = 0.0;
     if (ph < nph) {
       for (int b = b0 + ph; b < b1; b += nph) {
         if (col < c1) acc += (double)a.ppart[(size_t)b * c1 + col];
-        else if (col < c2) acc += (double)a.hist[(size_t)b * (a.K + 1) + (col - c1)];
+        else if (col < c2) acc += (double)a.hist[(size_t)b * a.hcols + (col - c1)];
         else acc += (double)a.lsq[b];
       }
     }
@@ -604,19 +624,19 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
   }
 }
 
-template <int NPW>
+template <int NPW, int NQ>
 static int launch_route_t(const CUtensorMap& tx, const CUtensorMap& tw, const RouteArgs& a, cudaStream_t st) {
   using SM = RouteSmem<NPW>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<NPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<NPW, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM::bytes);
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
   }
-  return launch_pdl(route_kernel<NPW>, dim3(a.nblk), dim3(kRouteThreads), SM::bytes, st, tx, tw, a);
+  return launch_pdl(route_kernel<NPW, NQ>, dim3(a.nblk), dim3(kRouteThreads), SM::bytes, st, tx, tw, a);
 }
 
 int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
@@ -635,6 +655,8 @@ int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
   sa.K = d.K;
   sa.nblk = L.nblk;
   sa.nparts = L.nparts;
+  sa.ncols = router_rows(d);
+  sa.hcols = hist_cols(d);
   return launch_pdl(scan_kernel, dim3(d.N + L.nparts), dim3(kScanThreads), 0, st, sa);
 }
 
@@ -669,17 +691,18 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.M = d.M;
   a.K = d.K;
   a.nblk = L.nblk;
+  a.ncols = router_rows(d);
   // the split router weight for this call (its block 0 also clears the status word
   // and the per-expert totals), then tensor maps over x and it
-  const int npw = route_npw(d.N);
+  const int npw = route_npw(d);
   uint16_t* w3 = ws_ptr<uint16_t>(ws, L.wprep);
   {
     const long long work = (long long)npw * (d.d / 8);
     long long grid = (work + 255) / 256;
     if (grid > (long long)sm_count() * 8) grid = (long long)sm_count() * 8;
     const int nclear = (int)((kHdrTotOffset + sizeof(int32_t) * d.N) / sizeof(uint32_t));
-    const int r = launch_pdl(router_split_kernel, dim3((unsigned)grid), dim3(256), 0, st, w_router, w3, d.N, npw,
-                             d.d, a.hdr, nclear);
+    const int r = launch_pdl(router_split_kernel, dim3((unsigned)grid), dim3(256), 0, st, w_router, w3,
+                             router_rows(d), npw, d.d, a.hdr, nclear);
     if (r != MOE_OK) return r;
   }
   CUtensorMap tx, tw;
@@ -688,11 +711,13 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
     return MOE_ERR_CUDA;
   int r;
   switch (npw) {
-    case 16: r = launch_route_t<16>(tx, tw, a, st); break;
-    case 32: r = launch_route_t<32>(tx, tw, a, st); break;
-    case 48: r = launch_route_t<48>(tx, tw, a, st); break;
-    case 64: r = launch_route_t<64>(tx, tw, a, st); break;
-    default: r = launch_route_t<80>(tx, tw, a, st); break;
+    case 16: r = launch_route_t<16, 4>(tx, tw, a, st); break;
+    case 32: r = launch_route_t<32, 8>(tx, tw, a, st); break;
+    case 48: r = launch_route_t<48, 12>(tx, tw, a, st); break;
+    case 64: r = launch_route_t<64, 16>(tx, tw, a, st); break;
+    default:  // 80 rows: without copy/constant experts the candidates are the reals, columns < 64
+      r = (pp_experts(d) == 0) ? launch_route_t<80, 16>(tx, tw, a, st) : launch_route_t<80, 20>(tx, tw, a, st);
+      break;
   }
   if (r != MOE_OK) return r;
   return launch_route_scan(d, ws, st);

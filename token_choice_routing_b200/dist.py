@@ -21,10 +21,12 @@ import torch
 import torch.distributed as dist
 
 
-def aux_sums_slices(N: int, K: int) -> Dict[str, slice]:
+def aux_sums_slices(N: int, K: int, PP: int = 0) -> Dict[str, slice]:
+    """Layout of moe_aux_sums' vector; PP = MoE++ copy + constant experts (their slot
+    counts follow the null histogram, their probability sums follow the null logit's)."""
     o = 0
     out = {}
-    for name, n in (("counts_real", N), ("null_hist", K + 1), ("psum", N + 1), ("lse2", 1), ("T", 1)):
+    for name, n in (("counts_real", N), ("null_hist", K + 1 + PP), ("psum", N + 1 + PP), ("lse2", 1), ("T", 1)):
         out[name] = slice(o, o + n)
         o += n
     return out
@@ -63,5 +65,6 @@ def dp_forward(layer, x, tok_null_bias, out, sums, group=None):
     else:
         B.expert_ffn(dm, xs, x, out["offsets"], layer.gate_up, layer.w_down, layer.shared_gate_up,
                      layer.shared_down, out["h"], out["h_shared"], out["ys"], out["shared_out"], ws)
-    B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"])
+    B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
+              topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
     return out

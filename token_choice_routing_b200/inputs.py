@@ -40,9 +40,10 @@ import numpy as np
 
 SEED_BASE = 20260000
 
-# Order of the per-tensor sub-streams; never reorder (it would change inputs).
+# Order of the per-tensor sub-streams; never reorder (it would change inputs). New
+# streams go at the end: the earlier ones keep their draws.
 _STREAMS = ("x", "w_router", "w_gate", "w_up", "w_down",
-            "ws_gate", "ws_up", "ws_down", "spans")
+            "ws_gate", "ws_up", "ws_down", "spans", "const_vectors")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -59,10 +60,16 @@ class LayerConfig:
     skew: bool = False
     seqs: int = 1
     bias_from: Optional[str] = None  # workload whose calibrated null bias this one uses
+    C: int = 0  # MoE++ copy experts (router rows N+1 .. N+C)
+    V: int = 0  # MoE++ constant experts (router rows N+C+1 .. N+C+V)
 
     @property
     def rho(self) -> float:
         return self.N / float(self.N + self.M)
+
+    @property
+    def router_rows(self) -> int:
+        return self.N + 1 + self.C + self.V
 
     @property
     def seed(self) -> int:
@@ -85,6 +92,10 @@ CONFIGS: Dict[str, LayerConfig] = {c.name: c for c in [
     LayerConfig("decode_0p6b", 1, T=64, d=1024, N=64, F=768, F_shared=768, K=4, M=64, bias_from="qwen3_0p6b"),
     LayerConfig("decode_1p7b", 2, T=64, d=2048, N=64, F=1536, F_shared=1536, K=8, M=192,
                 bias_from="qwen3_1p7b"),
+    # The 0.6B layer with MoE++ copy and constant experts beside the null expert: the same
+    # draws for x, the expert weights and the first N+1 router rows (rows are drawn in order).
+    LayerConfig("moepp_0p6b", 1, T=16384, d=1024, N=64, F=768, F_shared=768, K=4, M=64, seqs=8,
+                bias_from="qwen3_0p6b", C=4, V=4),
 ]}
 
 # Null-logit bias per workload, from tests/golden/calibrate_null_bias.py (oracle
@@ -182,6 +193,7 @@ class LayerInputs:
     ws_gate: np.ndarray        # [F_s, d] bf16 bits
     ws_up: np.ndarray          # [F_s, d] bf16 bits
     ws_down: np.ndarray        # [d, F_s] bf16 bits
+    const_vectors: Optional[np.ndarray] = None  # [V, d] bf16 bits (MoE++ constant experts)
 
 
 def make_inputs(cfg: LayerConfig, *, T: Optional[int] = None, weights: bool = True,
@@ -210,9 +222,9 @@ def make_inputs(cfg: LayerConfig, *, T: Optional[int] = None, weights: bool = Tr
         x = _normal_bf16(s["x"], (T, d), 1.0)
 
     g_r = np.random.Generator(np.random.PCG64(s["w_router"]))
-    w_router = (g_r.standard_normal((N + 1, d)) / math.sqrt(d)).astype(np.float32)
+    w_router = (g_r.standard_normal((cfg.router_rows, d)) / math.sqrt(d)).astype(np.float32)
 
-    bias = np.zeros(N + 1, dtype=np.float32)
+    bias = np.zeros(cfg.router_rows, dtype=np.float32)
     if cfg.skew:
         bias[:N] = (-SKEW_ZIPF_S * np.log(np.arange(N, dtype=np.float64) + 1.0)).astype(np.float32)
     elif cfg.M > 0:
@@ -230,13 +242,14 @@ def make_inputs(cfg: LayerConfig, *, T: Optional[int] = None, weights: bool = Tr
         e = np.zeros((0,), dtype=np.uint16)
         w_gate = w_up = w_down = ws_gate = ws_up = ws_down = e
 
+    const_vectors = _normal_bf16(s["const_vectors"], (cfg.V, d), 0.5) if cfg.V else None
     return LayerInputs(cfg, x, w_router, bias, tok_null_bias,
-                       w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+                       w_gate, w_up, w_down, ws_gate, ws_up, ws_down, const_vectors)
 
 
 def small_config(name: str = "small", *, T: int, d: int, N: int, F: int, F_shared: int,
                  K: int, M: int, config_id: int = 900, skew: bool = False,
-                 seqs: int = 1) -> LayerConfig:
+                 seqs: int = 1, C: int = 0, V: int = 0) -> LayerConfig:
     """An ad-hoc configuration for tests (edge cases, ragged sizes)."""
     return LayerConfig(name, config_id, T=T, d=d, N=N, F=F, F_shared=F_shared, K=K, M=M,
-                       skew=skew, seqs=seqs)
+                       skew=skew, seqs=seqs, C=C, V=V)

@@ -25,17 +25,23 @@ class MoENullLayer:
                  w_router: torch.Tensor, router_bias: Optional[torch.Tensor],
                  w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
                  ws_gate: torch.Tensor, ws_up: torch.Tensor, ws_down: torch.Tensor,
-                 router: str = "tensor", ffn: str = "single"):
+                 router: str = "tensor", ffn: str = "single", C: int = 0, V: int = 0,
+                 const_vectors: Optional[torch.Tensor] = None):
         """router: "tensor" (router product on the tensor cores, fp32 weights split
         exactly into three bf16 terms) or "fp32_cores" (fp32 FMA on the CUDA cores).
         ffn: "single" (single-CTA tiles) or "pair" (expert GEMMs on CTA pairs where
-        the shape allows)."""
+        the shape allows). C, V: MoE++ copy and constant experts (router rows
+        N+1 .. N+C+V after the null logit; const_vectors [V, d] bf16)."""
         if router not in ("tensor", "fp32_cores"):
             raise ValueError(f"router must be 'tensor' or 'fp32_cores', not {router!r}")
         if ffn not in ("pair", "single"):
             raise ValueError(f"ffn must be 'pair' or 'single', not {ffn!r}")
         self.d, self.N, self.M, self.K, self.F, self.F_shared = d, N, M, K, F, F_shared
+        self.C, self.V = C, V
         self.router, self.ffn = router, ffn
+        if V > 0 and (const_vectors is None or tuple(const_vectors.shape) != (V, d)):
+            raise ValueError("const_vectors [V, d] bf16 is required when V > 0")
+        self.const_vectors = None if V == 0 else const_vectors.contiguous()
         self.flags = ((B.FLAG_ROUTER_FP32_CORES if router == "fp32_cores" else 0) |
                       (B.FLAG_FFN_CTA_PAIR if ffn == "pair" else 0))
         dev = w_router.device
@@ -55,21 +61,23 @@ class MoENullLayer:
         self._weights = B.Weights(self.w_router.data_ptr(),
                                   None if self.router_bias is None else self.router_bias.data_ptr(),
                                   self.gate_up.data_ptr(), self.w_down.data_ptr(),
-                                  self.shared_gate_up.data_ptr(), self.shared_down.data_ptr())
+                                  self.shared_gate_up.data_ptr(), self.shared_down.data_ptr(),
+                                  None if self.const_vectors is None else self.const_vectors.data_ptr())
 
     @classmethod
     def from_inputs(cls, inp, device="cuda", router: str = "tensor", ffn: str = "single") -> "MoENullLayer":
         c = inp.cfg
         f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        cv = None if c.V == 0 else bf16_tensor(inp.const_vectors, device)
         return cls(c.d, c.N, c.M, c.K, c.F, c.F_shared,
                    w_router=f32(inp.w_router), router_bias=f32(inp.bias),
                    w_gate=bf16_tensor(inp.w_gate, device), w_up=bf16_tensor(inp.w_up, device),
                    w_down=bf16_tensor(inp.w_down, device), ws_gate=bf16_tensor(inp.ws_gate, device),
                    ws_up=bf16_tensor(inp.ws_up, device), ws_down=bf16_tensor(inp.ws_down, device),
-                   router=router, ffn=ffn)
+                   router=router, ffn=ffn, C=c.C, V=c.V, const_vectors=cv)
 
     def dims(self, T: int) -> B.Dims:
-        return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags)
+        return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags, self.C, self.V)
 
     def alloc(self, T: int, logits: bool = True, xs: bool = True) -> Dict[str, torch.Tensor]:
         """Caller-owned buffers for a T-token call (R_cap = T*K rows). xs=False
@@ -79,7 +87,7 @@ class MoENullLayer:
         R = T * K
         i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
         out = dict(
-            logits=torch.empty((T, N + 1), dtype=f32, device=dev) if logits else None,
+            logits=torch.empty((T, N + 1 + self.C + self.V), dtype=f32, device=dev) if logits else None,
             topk_idx=torch.empty((T, K), dtype=i32, device=dev),
             topk_gate=torch.empty((T, K), dtype=f32, device=dev),
             n_real=torch.empty((T,), dtype=i32, device=dev),
@@ -93,8 +101,8 @@ class MoENullLayer:
             ys=torch.empty((max(R, 1), d), dtype=bf, device=dev),
             shared_out=torch.empty((max(T, 1), d), dtype=bf, device=dev),
             y=torch.empty((max(T, 1), d), dtype=bf, device=dev),
-            counts_ext=torch.empty((N + M,), dtype=i32, device=dev),
-            P=torch.empty((N + M,), dtype=f32, device=dev),
+            counts_ext=torch.empty((N + M + self.C + self.V,), dtype=i32, device=dev),
+            P=torch.empty((N + M + self.C + self.V,), dtype=f32, device=dev),
             losses=torch.empty((2,), dtype=f32, device=dev),
         )
         out["workspace"] = torch.empty((max(B.workspace_bytes(self.dims(T)), 256),), dtype=torch.uint8, device=dev)
