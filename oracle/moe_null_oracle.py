@@ -1,4 +1,5 @@
-"""CPU oracle: forward pass of a token-choice MoE layer with zero-compute null experts.
+"""CPU oracle: forward and backward pass of a token-choice MoE layer with zero-compute
+null experts.
 
 TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's
 CPU-baseline leg may import this module. The CUDA library never calls it, and it
@@ -39,9 +40,11 @@ Readings where the pages are silent (each is listed in the design notes):
 * f_i = count_i / T, so sum_i f_i = K; P_i = mean_t p_{t,i} over the pool;
 * rows within an expert's segment are in ascending token order (stable argsort).
 
-Parity status: every function below is pinned by the CPU tests in
+Parity status: every forward function below is pinned by the CPU tests in
 tests/test_oracle_pins.py (brute force, closed forms, textbook reductions,
-library routines); none is "parity unpinned".
+library routines); every backward function by tests/test_oracle_backward_pins.py
+(central finite differences of the forward objective, shift-invariance closed
+forms); none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -52,7 +55,8 @@ __all__ = [
     "threshold_real_count", "renormalised_gates", "dispatch", "swiglu",
     "layer_output", "aux_stats", "aux_partial_sums", "aux_finalize", "route",
     "bf16_round_f64", "expanded_pool_pp", "pool_kinds", "renormalised_gates_pp",
-    "layer_output_pp", "route_pp",
+    "layer_output_pp", "route_pp", "swiglu_backward", "gate_backward", "aux_backward",
+    "pool_grad_to_logits", "router_backward", "layer_backward", "layer_objective",
 ]
 
 
@@ -372,3 +376,171 @@ def route_pp(s, N, M, C, V, K):
     n_real = (idx < N).sum(axis=1)
     gates = renormalised_gates_pp(v, idx, N, M)
     return dict(v=v, lse=lse, p=p, idx=idx, n_real=n_real, gates=gates)
+
+
+# ---------------------------------------------------------------------------------------
+# Backward pass of the layer.
+#
+# The objective differentiated is  L = <y, dy> + alpha * L_bal + beta * L_z, with dy the
+# upstream gradient of the layer output ([KR] 四 实验结果/训练配置 trains with the load-balance
+# and Z losses added at fixed weights, 2e-2 and 1e-3; here the weights are arguments). The
+# routing choice (top-K indices) and the load fractions f_i = count_i / T are piecewise
+# constant in the logits, so they carry no gradient: the gradient reaches the logits
+# through the renormalised gates, through P_i (the pool softmax) in L_bal, and through
+# lse in L_z. Every product below is the chain rule written out for one of those terms.
+
+
+def swiglu_backward(z, w_gate, w_up, w_down, dout):
+    """Gradients of E(z) = (silu(z W_g^T) * (z W_u^T)) W_d^T for an upstream dE.
+
+    With a = z W_g^T, b = z W_u^T, sigma = 1/(1+e^{-a}), h = a sigma b:
+      dW_d = dE^T h, dh = dE W_d, db = dh * a sigma,
+      da = dh * b * sigma (1 + a (1 - sigma))   (derivative of a sigma(a)),
+      dW_g = da^T z, dW_u = db^T z, dz = da W_g + db W_u.
+    Returns dz [R, d], dW_g [F, d], dW_u [F, d], dW_d [d, F].
+    """
+    z = np.asarray(z, dtype=np.float64)
+    wg = np.asarray(w_gate, dtype=np.float64)
+    wu = np.asarray(w_up, dtype=np.float64)
+    wd = np.asarray(w_down, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    a = z @ wg.T
+    b = z @ wu.T
+    sig = 1.0 / (1.0 + np.exp(-a))
+    h = a * sig * b
+    dwd = dout.T @ h
+    dh = dout @ wd
+    db = dh * a * sig
+    da = dh * b * sig * (1.0 + a * (1.0 - sig))
+    return da @ wg + db @ wu, da.T @ z, db.T @ z, dwd
+
+
+def gate_backward(v, idx, gates, dg, N, M):
+    """Pool-logit gradient of the renormalised gates, from dL/dg [T, K].
+
+    The gates of a token are a softmax over the logits of its selected slots that are
+    not null copies ([KR] 三/Null Expert 机制; [MPP] for copy and constant experts), so
+    for a selected slot i: dL/dv_i = g_i (dL/dg_i - sum_j g_j dL/dg_j). Other slots get 0.
+    Returns float64 [T, P].
+    """
+    v = np.asarray(v, dtype=np.float64)
+    idx = np.asarray(idx)
+    g = np.asarray(gates, dtype=np.float64)
+    dg = np.asarray(dg, dtype=np.float64)
+    T, K = idx.shape
+    dv = np.zeros(v.shape, dtype=np.float64)
+    for t in range(T):
+        sel = [k for k in range(K) if idx[t, k] < N or idx[t, k] >= N + M]
+        if not sel:
+            continue
+        mean = sum(g[t, k] * dg[t, k] for k in sel)
+        for k in sel:
+            dv[t, idx[t, k]] += g[t, k] * (dg[t, k] - mean)
+    return dv
+
+
+def aux_backward(idx, p, lse, N, alpha, beta):
+    """Pool-logit gradient of alpha * L_bal + beta * L_z.
+
+    [KR] 三/负载均衡损失 and 三/Z-Loss. With f fixed and P_i = mean_t p_{t,i},
+    dL_bal/dv_{t,j} = (N/T) p_{t,j} (f_j - sum_i f_i p_{t,i}); with
+    L_z = mean_t lse_t^2, dL_z/dv_{t,j} = (2/T) lse_t p_{t,j}. Returns [T, P].
+    """
+    idx = np.asarray(idx)
+    p = np.asarray(p, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    T, P = p.shape
+    f = np.bincount(idx.reshape(-1), minlength=P)[:P] / float(T)
+    fp = (p * f[None, :]).sum(axis=1)
+    d_bal = (N / T) * p * (f[None, :] - fp[:, None])
+    d_z = (2.0 / T) * lse[:, None] * p
+    return alpha * d_bal + beta * d_z
+
+
+def pool_grad_to_logits(dv, N, M, C=0, V=0):
+    """Fold a pool gradient [T, N+M+C+V] onto the router's logit columns [T, N+1+C+V]:
+    the M null copies all read column N, so their gradients add up there."""
+    dv = np.asarray(dv, dtype=np.float64)
+    _, col = pool_kinds(N, M, C, V)
+    ds = np.zeros((dv.shape[0], N + 1 + C + V), dtype=np.float64)
+    for i, c in enumerate(col):
+        ds[:, c] += dv[:, i]
+    return ds
+
+
+def router_backward(x, w_router, ds):
+    """Gradients of the router's linear map s = x W_r^T + bias (+ per-token null offset).
+
+    Returns dx [T, d] = ds W_r, dW_r [rows, d] = ds^T x, dbias [rows] = sum_t ds and the
+    per-token null-offset gradient ds[:, N] is the caller's (column N of ds).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_router, dtype=np.float64)
+    ds = np.asarray(ds, dtype=np.float64)
+    return ds @ w, ds.T @ x, ds.sum(axis=0)
+
+
+def layer_backward(x, s, w_router, N, M, K, experts, shared, dy, alpha, beta,
+                   C=0, V=0, const_vectors=None):
+    """All gradients of L = <y, dy> + alpha L_bal + beta L_z for one layer.
+
+    ``s`` are the forward logits [T, N+1+C+V] (the routing is taken from them, so a
+    parity test passes the logits the GPU computed). Returns a dict with dx [T, d],
+    dg [T, K] (gradient of each slot's gate), ds [T, N+1+C+V] (logit gradient),
+    dW_r, dbias, dtnb [T] (null-offset gradient), dW_gate/dW_up [N, F, d],
+    dW_down [N, d, F], the shared expert's (dWs_gate, dWs_up, dWs_down) and
+    dconst [V, d].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    T, d = x.shape
+    r = route_pp(s, N, M, C, V, K)
+    idx, gates = r["idx"], r["gates"]
+    wg, wu, wd = (np.asarray(w, dtype=np.float64) for w in experts)
+    dx, dwsg, dwsu, dwsd = swiglu_backward(x, *shared, dy)
+    dwg = np.zeros_like(wg)
+    dwu = np.zeros_like(wu)
+    dwd = np.zeros_like(wd)
+    dg = np.zeros((T, K), dtype=np.float64)
+    for e in range(N):
+        rows, ks = np.nonzero(idx == e)
+        if rows.size == 0:
+            continue
+        z = x[rows]
+        ye = swiglu(z, wg[e], wu[e], wd[e])
+        dg[rows, ks] = (dy[rows] * ye).sum(axis=1)
+        dz, dwg[e], dwu[e], dwd[e] = swiglu_backward(z, wg[e], wu[e], wd[e],
+                                                     gates[rows, ks][:, None] * dy[rows])
+        np.add.at(dx, rows, dz)
+    cv = np.asarray(const_vectors, dtype=np.float64).reshape(V, d) if V else np.zeros((0, d))
+    dconst = np.zeros((V, d), dtype=np.float64)
+    for j in range(C + V):
+        rows, ks = np.nonzero(idx == N + M + j)
+        if rows.size == 0:
+            continue
+        if j < C:  # copy expert: output x_t
+            dg[rows, ks] = (dy[rows] * x[rows]).sum(axis=1)
+            np.add.at(dx, rows, gates[rows, ks][:, None] * dy[rows])
+        else:      # constant expert: output c_j
+            dg[rows, ks] = dy[rows] @ cv[j - C]
+            dconst[j - C] = (gates[rows, ks][:, None] * dy[rows]).sum(axis=0)
+    dv = gate_backward(r["v"], idx, gates, dg, N, M) + aux_backward(idx, r["p"], r["lse"], N,
+                                                                   alpha, beta)
+    ds = pool_grad_to_logits(dv, N, M, C, V)
+    dx_r, dw_r, dbias = router_backward(x, w_router, ds)
+    return dict(dx=dx + dx_r, dg=dg, ds=ds, dW_r=dw_r, dbias=dbias, dtnb=ds[:, N].copy(),
+                dW_gate=dwg, dW_up=dwu, dW_down=dwd, dWs_gate=dwsg, dWs_up=dwsu,
+                dWs_down=dwsd, dconst=dconst, idx=idx, gates=gates)
+
+
+def layer_objective(x, w_router, bias, tok_null_bias, N, M, K, experts, shared, dy, alpha,
+                    beta, C=0, V=0, const_vectors=None):
+    """The scalar L = <y, dy> + alpha L_bal + beta L_z that :func:`layer_backward`
+    differentiates, computed by the forward functions alone (for finite differences)."""
+    null_col = N if (C + V) else None
+    s = router_logits(x, w_router, bias, tok_null_bias, null_col=null_col)
+    r = route_pp(s, N, M, C, V, K)
+    y = layer_output_pp(x, r["idx"], r["gates"], N, M, C, V, experts, shared,
+                        const_vectors if V else np.zeros((0, np.asarray(x).shape[1])))
+    _, _, _, L_bal, L_z = aux_stats(r["idx"], r["p"], r["lse"], N, M)
+    return float(np.sum(y * np.asarray(dy, dtype=np.float64))) + alpha * L_bal + beta * L_z
