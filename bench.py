@@ -212,6 +212,131 @@ def run_reference(args):
     return 0
 
 
+BWD_ALPHA, BWD_BETA = 2e-2, 1e-3  # load-balance and Z-loss weights of the paper's training runs
+
+
+def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
+    """Backward pass of the same layer: gradients of <y, dy> + alpha L_bal + beta L_z with a
+    seeded dy, the forward's tensors resident. The timed step is one moe_backward call (L2
+    flushed before each); the stages are then timed one by one through their entry points."""
+    import numpy as np
+    import torch
+    from token_choice_routing_b200 import binding as B
+    from token_choice_routing_b200 import inputs as I
+    from token_choice_routing_b200.layer import bf16_tensor
+
+    dev = x.device
+    T, d, F, Fs, N, K = cfg.T, cfg.d, cfg.F, cfg.F_shared, cfg.N, cfg.K
+    rows = N + 1 + cfg.C + cfg.V
+    bout = layer.alloc(T, logits=True, xs=True)
+    layer.forward(x, tnb, bout)
+    dy = bf16_tensor(I.upstream_grad(cfg), dev)
+    grads = layer.alloc_grads(T)
+    bws = grads["workspace"]
+
+    def bstep():
+        layer.backward(x, bout, dy, BWD_ALPHA, BWD_BETA, grads=grads)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        bstep()
+    torch.cuda.synchronize()
+    st = B.get_device_status(bws)
+    if st != B.OK:
+        raise SystemExit(f"backward device status: {B.status_string(st)}")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record()
+        bstep()
+        e1.record()
+    torch.cuda.synchronize()
+    total_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    R = int(bout["offsets"][-1].item())
+
+    # stages one by one, CUDA events between them
+    dm = layer.dims(T)
+    Rc = T * K
+    dys = torch.empty((Rc, d), dtype=torch.bfloat16, device=dev)
+    dg = torch.empty((T, K), dtype=torch.float32, device=dev)
+    ds = torch.empty((T, rows), dtype=torch.float32, device=dev)
+    dxs = torch.empty((Rc, d), dtype=torch.bfloat16, device=dev)
+    dxsh = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    o = bout
+    stages = [
+        ("combine_bwd", lambda: B.combine_backward(dm, dy, o["ys"], o["topk_gate"], o["slot_row"], dys, dg, bws,
+                                                   topk_idx=o["topk_idx"], x=x, const_vectors=layer.const_vectors)),
+        ("router_bwd", lambda: B.router_backward(dm, o["logits"], o["topk_idx"], o["topk_gate"], dg, o["counts_ext"],
+                                                 T, BWD_ALPHA, BWD_BETA, ds, grads["dtok_null_bias"])),
+        ("router_wgrad", lambda: B.router_weight_grad(dm, x, ds, grads["dw_router"], grads["dbias"], bws)),
+        ("preact", lambda: B.expert_preact(dm, o["xs"], x, o["offsets"], layer.gate_up, layer.shared_gate_up, bws)),
+        ("dgrad_down", lambda: B.expert_dgrad_down(dm, o["offsets"], dys, dy, layer.w_down, layer.shared_down, bws)),
+        ("wgrad_down", lambda: B.expert_wgrad_down(dm, o["offsets"], dys, dy, o["h"], o["h_shared"],
+                                                   grads["dw_down"], grads["dws_down"], bws)),
+        ("dgrad_gate_up", lambda: B.expert_dgrad_gate_up(dm, o["offsets"], layer.gate_up, layer.shared_gate_up, dxs,
+                                                         dxsh, bws)),
+        ("wgrad_gate_up", lambda: B.expert_wgrad_gate_up(dm, o["offsets"], o["xs"], x, grads["dw_gate"],
+                                                         grads["dw_up"], grads["dws_gate"], grads["dws_up"], bws)),
+        ("input_grad", lambda: B.input_grad(dm, dxsh, dxs, o["slot_row"], o["topk_idx"], o["topk_gate"], dy, ds,
+                                            layer.w_router, grads["dx"], bws)),
+    ]
+    acc = {n: 0.0 for n, _ in stages}
+    nb = max(3, min(args.steps, 10))
+    for _ in range(nb):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+        ev[0].record()
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            ev[i + 1].record()
+        torch.cuda.synchronize()
+        for i, (n, _) in enumerate(stages):
+            acc[n] += ev[i].elapsed_time(ev[i + 1])
+    st = B.get_device_status(bws)
+    if st != B.OK:
+        raise SystemExit(f"backward device status: {B.status_string(st)}")
+    kms = {n: acc[n] / nb for n in acc}
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fl = {"preact": 4.0 * d * (F * R + Fs * T), "dgrad_down": 2.0 * d * (F * R + Fs * T),
+          "wgrad_down": 2.0 * d * (F * R + Fs * T), "dgrad_gate_up": 4.0 * d * (F * R + Fs * T),
+          "wgrad_gate_up": 4.0 * d * (F * R + Fs * T),
+          "router_wgrad": 2.0 * rows * d * T, "input_grad": 2.0 * rows * d * T}
+    by = {"combine_bwd": 2.0 * d * T + 4.0 * d * R + 12.0 * K * T,
+          "router_bwd": 8.0 * rows * T + 12.0 * K * T,
+          "input_grad": 4.0 * d * T + 2.0 * d * R + 4.0 * rows * T + 4.0 * K * T}
+    kernels = {}
+    for n, ms in kms.items():
+        k = {"ms": ms}
+        if n in ("preact", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"):
+            k.update(bound="tensor", **{"TFLOP/s": fl[n] / (ms * 1e9)})
+            k["frac"] = k["TFLOP/s"] / bf16_peak
+        elif n in by:
+            k.update(bound="hbm", **{"GB/s": by[n] / (ms * 1e6)})
+            k["frac"] = k["GB/s"] / hbm_peak
+        else:
+            k.update(bound="alu", **{"TFLOP/s": fl[n] / (ms * 1e9)})
+        kernels[n] = k
+    gemm = ["preact", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"]
+    top = max(gemm, key=lambda n: kms[n])
+    gemm_ms = sum(kms[n] for n in gemm)
+    gemm_flops = sum(fl[n] for n in gemm)
+    split = 2 if (T + 63) // 64 > 32 else 0  # shared-expert K-chunk reductions of the two weight gradients
+    return {
+        "metric": "real-slot tokens/s per MoE layer bwd", "value": R * args.steps / (total_ms * 1e-3),
+        "unit": UNIT, "ms_per_step": total_ms / args.steps, "steps": args.steps,
+        "objective": f"<y, dy> + {BWD_ALPHA} L_bal + {BWD_BETA} L_z (dy seeded N(0,1) bf16)",
+        "preactivations": "recomputed by the gate/up GEMM without its SwiGLU epilogue",
+        "ffn_tflops_real_rows": gemm_flops / (gemm_ms * 1e9),
+        "roofline": {"kernel": f"{top} grouped GEMM (tcgen05)", "bound": "tensor",
+                     "achieved": fl[top] / (kms[top] * 1e9), "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": fl[top] / (kms[top] * 1e9) / bf16_peak, "peak_kind": f"{peak_kind} bf16 burst",
+                     "traffic": None, "flops_per_launch": fl[top], "ms_per_launch": kms[top]},
+        "kernels": kernels,
+        "gpu_launches": (11 + split + (1 if cfg.V else 0)) * args.steps,
+    }
+
+
 def workload_config(cfg, args):
     pp = f" C={cfg.C} V={cfg.V}" if cfg.C + cfg.V else ""
     return {"workload": f"{cfg.name}: MoE layer fwd T={cfg.T} d={cfg.d} N={cfg.N} F={cfg.F} "
@@ -242,6 +367,7 @@ def main():
     ap.add_argument("--gather", action="store_true",
                     help="no xs copy: gate/up gathers the routed rows of x by TMA (default: dispatch copies them)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")
     args = ap.parse_args()
@@ -431,6 +557,10 @@ def main():
            "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(8 + 4 * cext_pin.numel()),
            "ms_per_step": e2e_total / args.steps}
 
+    backward = None
+    if not args.no_backward and world == 1 and not args.gather:
+        backward = measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         S = calibrate_sample(inp, args.cpu_seconds)
@@ -452,6 +582,7 @@ def main():
             "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk.summary(),
+            "backward": backward,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

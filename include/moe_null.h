@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define MOE_NULL_ABI_VERSION 2
+#define MOE_NULL_ABI_VERSION 3
 
 typedef void* moe_stream_t; /* a cudaStream_t */
 
@@ -304,6 +304,137 @@ MOE_API int moe_clear_device_status(void* workspace, moe_stream_t stream);
  * after `limit_ns` nanoseconds (1e3..1e10), records MOE_ERR_TIMEOUT in the
  * workspace status word and returns. The context stays usable. */
 MOE_API int moe_selftest_bounded_wait(void* workspace, uint64_t limit_ns, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Backward pass.
+ *
+ * The paper trains the layer end to end with the load-balance and Z losses added at
+ * fixed weights (paper-review page, section 四 实验结果 / 训练配置: 2e-2 and 1e-3).
+ * The backward differentiates the objective <y, dy> + alpha L_bal + beta L_z, dy the
+ * upstream gradient of y. Top-K choices and the load fractions f_i are piecewise
+ * constant in the logits and carry no gradient; the logits receive gradient through
+ * the renormalised gates, through P_i in L_bal and through lse in L_z. As in the
+ * forward, null slots cost nothing: the expert gradients run on the real rows only.
+ * Each expert is SwiGLU; its gate/up pre-activations are recomputed from xs with the
+ * forward's gate/up GEMM (no SwiGLU epilogue) rather than stored by the forward.
+ *
+ * Requirements: the forward ran with out->logits and out->xs non-NULL (the copy
+ * path). Weight gradients of the experts are bf16; router, bias and constant-vector
+ * gradients are fp32. Every gradient is written (not accumulated).
+ *
+ * Backward workspace: moe_backward_workspace_bytes(dims) bytes, 256-byte aligned,
+ * separate from the forward workspace; its first word is a status word like the
+ * forward workspace's (moe_get_device_status / moe_clear_device_status accept it).
+ * moe_backward clears it. */
+
+/* Forward tensors the backward reads (device pointers, all from moe_forward). */
+typedef struct moe_saved {
+  const uint16_t* x;          /* [T, d] bf16 layer input                              */
+  const float* logits;        /* [T, N+1+C+V] fp32 router logits                      */
+  const int32_t* topk_idx;    /* [T, K]                                               */
+  const float* topk_gate;     /* [T, K]                                               */
+  const int32_t* offsets;     /* [N+1]                                                */
+  const int32_t* slot_row;    /* [T, K]                                               */
+  const uint16_t* xs;         /* [R_cap, d] gathered routed rows                      */
+  const uint16_t* h;          /* [R_cap, F] routed SwiGLU activations                 */
+  const uint16_t* h_shared;   /* [T, F_shared]                                        */
+  const uint16_t* ys;         /* [R_cap, d] routed expert outputs                     */
+  const int32_t* counts_ext;  /* [N+M+C+V] slot counts over every data-parallel rank  */
+  int64_t t_total;            /* tokens over every data-parallel rank (>= T)          */
+} moe_saved_t;
+
+/* Gradients (device pointers). */
+typedef struct moe_grads {
+  uint16_t* dx;               /* [T, d] bf16                                          */
+  float* dw_router;           /* [N+1+C+V, d] fp32                                    */
+  float* dbias;               /* [N+1+C+V] fp32, or NULL                              */
+  float* dtok_null_bias;      /* [T] fp32 gradient of the per-token null offset, or NULL */
+  uint16_t* dw_gate;          /* [N, F, d] bf16                                       */
+  uint16_t* dw_up;            /* [N, F, d] bf16                                       */
+  uint16_t* dw_down;          /* [N, d, F] bf16                                       */
+  uint16_t* dws_gate;         /* [F_shared, d] bf16                                   */
+  uint16_t* dws_up;           /* [F_shared, d] bf16                                   */
+  uint16_t* dws_down;         /* [d, F_shared] bf16                                   */
+  float* dconst;              /* [V, d] fp32 (V > 0), else NULL                       */
+} moe_grads_t;
+
+/* Backward workspace size in bytes (0 if dims are invalid). */
+MOE_API size_t moe_backward_workspace_bytes(const moe_dims_t* dims);
+
+/* Combine backward (核心公式): for each selected slot, dg[t,k] = <dy_t, out> where out
+ * is the slot's expert output (its row of ys, x_t for a copy expert, c_j for a
+ * constant expert; 0 for a null copy), and for a real slot dys[row] = bf16(g dy_t).
+ * dy [T, d] bf16; dys [R_cap, d] bf16 (rows of real slots written); dg [T, K] fp32.
+ * topk_idx, x and const_vectors are read only when C + V > 0. */
+MOE_API int moe_combine_backward(const moe_dims_t* dims, const uint16_t* dy, const uint16_t* ys,
+                                 const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx,
+                                 const uint16_t* x, const uint16_t* const_vectors, uint16_t* dys, float* dg,
+                                 void* bwd_workspace, moe_stream_t stream);
+
+/* Router backward (Null Expert 机制, 负载均衡损失, Z-Loss): the logit gradient
+ * ds [T, N+1+C+V] fp32 from the gate gradients dg, the forward logits and the global
+ * slot counts: gates g = softmax over the selected non-null slots give
+ * g_k (dg_k - sum_l g_l dg_l); alpha L_bal gives alpha (N/t_total) p_i (f_i - sum_l f_l p_l)
+ * over the pool; beta L_z gives beta (2/t_total) lse_t p_i. The null logit's entry sums
+ * its M copies. dtok_null_bias (optional, [T]) receives column N. */
+MOE_API int moe_router_backward(const moe_dims_t* dims, const float* logits, const int32_t* topk_idx,
+                                const float* topk_gate, const float* dg, const int32_t* counts_ext,
+                                int64_t t_total, float alpha, float beta, float* ds, float* dtok_null_bias,
+                                moe_stream_t stream);
+
+/* dw_router = ds^T x ([N+1+C+V, d] fp32) and dbias = sum_t ds (optional), summed in
+ * a fixed order (deterministic). */
+MOE_API int moe_router_weight_grad(const moe_dims_t* dims, const uint16_t* x, const float* ds, float* dw_router,
+                                   float* dbias, void* bwd_workspace, moe_stream_t stream);
+
+/* Expert FFN backward (实现: grouped GEMMs over the real rows only): recomputes the
+ * gate/up pre-activations, then dgrad of the down projection fused with the SwiGLU
+ * derivative, the down weight gradient, dgrad of gate/up and the gate/up weight
+ * gradient, for the routed experts (rows of xs, upstream dys) and the shared expert
+ * (rows of x, upstream dy). Writes dxs [R_cap, d] and dx_shared [T, d] (bf16) and
+ * g->dw_gate/up/down and g->dws_gate/up/down. */
+MOE_API int moe_expert_ffn_backward(const moe_dims_t* dims, const moe_weights_t* w, const moe_saved_t* saved,
+                                    const uint16_t* dys, const uint16_t* dy, uint16_t* dxs, uint16_t* dx_shared,
+                                    const moe_grads_t* g, void* bwd_workspace, moe_stream_t stream);
+
+/* The five stages of moe_expert_ffn_backward, one GEMM launch each, for callers that
+ * schedule or time them separately. The pre-activations z and their gradients dz live in
+ * the backward workspace; call the stages in this order:
+ *   moe_expert_preact        z = [xs W_g^T | xs W_u^T] (packed order), shared from x
+ *   moe_expert_dgrad_down    dh = dys W_d, then dz from dh and z (SwiGLU derivative)
+ *   moe_expert_wgrad_down    dw_down[e] = dys_e^T h_e, dws_down = dy^T h_shared
+ *   moe_expert_dgrad_gate_up dxs = dz W_gu, dx_shared = dz_shared W_sgu
+ *   moe_expert_wgrad_gate_up dw_gate/dw_up[e] = dz_e^T xs_e (unpacked), shared from x */
+MOE_API int moe_expert_preact(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x,
+                              const int32_t* offsets, const uint16_t* gate_up, const uint16_t* shared_gate_up,
+                              void* bwd_workspace, moe_stream_t stream);
+MOE_API int moe_expert_dgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys,
+                                  const uint16_t* dy, const uint16_t* w_down, const uint16_t* shared_down,
+                                  void* bwd_workspace, moe_stream_t stream);
+MOE_API int moe_expert_wgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys,
+                                  const uint16_t* dy, const uint16_t* h, const uint16_t* h_shared,
+                                  uint16_t* dw_down, uint16_t* dws_down, void* bwd_workspace,
+                                  moe_stream_t stream);
+MOE_API int moe_expert_dgrad_gate_up(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* gate_up,
+                                     const uint16_t* shared_gate_up, uint16_t* dxs, uint16_t* dx_shared,
+                                     void* bwd_workspace, moe_stream_t stream);
+MOE_API int moe_expert_wgrad_gate_up(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* xs,
+                                     const uint16_t* x, uint16_t* dw_gate, uint16_t* dw_up, uint16_t* dws_gate,
+                                     uint16_t* dws_up, void* bwd_workspace, moe_stream_t stream);
+
+/* Input gradient: dx[t] = dx_shared[t] + sum over the token's real slots of
+ * dxs[slot_row] + sum over its copy-expert slots of g dy[t] + sum_j ds[t, j] W_r[j, :],
+ * accumulated in fp32 and rounded once to bf16. */
+MOE_API int moe_input_grad(const moe_dims_t* dims, const uint16_t* dx_shared, const uint16_t* dxs,
+                           const int32_t* slot_row, const int32_t* topk_idx, const float* topk_gate,
+                           const uint16_t* dy, const float* ds, const float* w_router, uint16_t* dx,
+                           void* bwd_workspace, moe_stream_t stream);
+
+/* The whole backward: combine, router, router weight gradient, expert FFNs, input
+ * gradient and (V > 0) the constant experts' gradient. */
+MOE_API int moe_backward(const moe_dims_t* dims, const moe_weights_t* w, const moe_saved_t* saved,
+                         const uint16_t* dy, float alpha, float beta, const moe_grads_t* g, void* bwd_workspace,
+                         moe_stream_t stream);
 
 #ifdef __cplusplus
 }

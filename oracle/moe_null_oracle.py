@@ -439,18 +439,25 @@ def gate_backward(v, idx, gates, dg, N, M):
     return dv
 
 
-def aux_backward(idx, p, lse, N, alpha, beta):
+def aux_backward(idx, p, lse, N, alpha, beta, counts=None, t_total=None):
     """Pool-logit gradient of alpha * L_bal + beta * L_z.
 
     [KR] 三/负载均衡损失 and 三/Z-Loss. With f fixed and P_i = mean_t p_{t,i},
     dL_bal/dv_{t,j} = (N/T) p_{t,j} (f_j - sum_i f_i p_{t,i}); with
-    L_z = mean_t lse_t^2, dL_z/dv_{t,j} = (2/T) lse_t p_{t,j}. Returns [T, P].
+    L_z = mean_t lse_t^2, dL_z/dv_{t,j} = (2/T) lse_t p_{t,j}. Returns [T, P] for the
+    rows given. For one shard of a data-parallel batch, ``counts`` (slot counts over
+    the whole batch) and ``t_total`` (its token count) replace this shard's own:
+    f and both means run over the whole batch.
     """
     idx = np.asarray(idx)
     p = np.asarray(p, dtype=np.float64)
     lse = np.asarray(lse, dtype=np.float64)
     T, P = p.shape
-    f = np.bincount(idx.reshape(-1), minlength=P)[:P] / float(T)
+    if counts is None:
+        counts = np.bincount(idx.reshape(-1), minlength=P)[:P]
+    if t_total is not None:
+        T = int(t_total)
+    f = np.asarray(counts, dtype=np.float64) / float(T)
     fp = (p * f[None, :]).sum(axis=1)
     d_bal = (N / T) * p * (f[None, :] - fp[:, None])
     d_z = (2.0 / T) * lse[:, None] * p

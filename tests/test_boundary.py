@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.LIB.moe_abi_version() == 2
+    assert lib.LIB.moe_abi_version() == 3
     for code in (0, -1, -2, -3, -4, -5, 7):
         assert isinstance(lib.status_string(code), str) and lib.status_string(code)
 
@@ -132,3 +132,35 @@ def test_host_side_rejections_touch_no_device(lib):
     # T = 0 is a no-op
     zero = B.dims(0, 128, 8, 8, 4, 64, 64)
     assert L.moe_route(C.byref(zero), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.OK
+
+
+def test_backward_workspace_and_host_side_rejections(lib):
+    B = lib
+    L = B.LIB
+    dm = good()
+    T, d, K, F, Fs = 256, 128, 4, 64, 64
+    bw = B.backward_workspace_bytes(dm)
+    assert bw > 0 and bw % 256 == 0
+    # holds at least the gate/up pre-activations and their gradients (routed and shared),
+    # the routed rows' upstream and input gradients and the shared expert's input gradient
+    assert bw >= 2 * (2 * (T * K * 2 * F + T * 2 * Fs)) + 2 * 2 * T * K * d + 2 * T * d
+    assert B.backward_workspace_bytes(B.dims(-1, 128, 8, 8, 4, 64, 64)) == 0
+    big = B.backward_workspace_bytes(B.dims(16384, 1024, 64, 64, 4, 768, 768))
+    assert big > bw
+    nul = None
+    inv = B.ERR_INVALID_ARG
+    assert L.moe_combine_backward(C.byref(dm), *([nul] * 11)) == inv
+    assert L.moe_router_backward(C.byref(dm), nul, nul, nul, nul, nul, T, 0.02, 0.001, nul, nul, nul) == inv
+    assert L.moe_router_weight_grad(C.byref(dm), nul, nul, nul, nul, nul, nul) == inv
+    assert L.moe_expert_ffn_backward(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul) == inv
+    assert L.moe_input_grad(C.byref(dm), *([nul] * 11)) == inv
+    assert L.moe_backward(C.byref(dm), nul, nul, nul, 0.02, 0.001, nul, nul, nul) == inv
+    # a token total smaller than this call's tokens is never valid (pointers set to a dummy value)
+    fake = C.c_void_p(256)
+    assert L.moe_router_backward(C.byref(dm), fake, fake, fake, fake, fake, T - 1, 0.02, 0.001, fake, nul,
+                                 nul) == inv
+    # invalid dims first; T = 0 is a no-op
+    bad = B.dims(256, 100, 8, 8, 4, 64, 64)
+    assert L.moe_backward(C.byref(bad), nul, nul, nul, 0.02, 0.001, nul, nul, nul) == B.ERR_UNSUPPORTED
+    zero = B.dims(0, 128, 8, 8, 4, 64, 64)
+    assert L.moe_backward(C.byref(zero), nul, nul, nul, 0.02, 0.001, nul, nul, nul) == B.OK

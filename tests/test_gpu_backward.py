@@ -1,0 +1,196 @@
+"""GPU parity of the backward pass: the CUDA path (through the C ABI) against the
+oracle's layer_backward, run on the GPU's own fp32 logits so both sides take the
+same routing.
+
+Tolerances: every gradient to relative Frobenius error 1e-2 (bf16 activations and
+bf16 weight gradients, fp32 accumulation; the oracle is fp64 without rounding), each
+routed expert's weight gradients to 2e-2, and experts that received no rows exactly
+zero. With dy = 0 only the load-balance and Z-loss terms act: the logit, router-weight
+and bias gradients then follow from fp32 softmax arithmetic alone and are held to 1e-4,
+and every expert gradient is exactly zero.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from token_choice_routing_b200 import inputs as I
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+ALPHA, BETA = 2e-2, 1e-3   # the paper's loss weights (review page, 四 / 训练配置)
+REL = 1e-2
+REL_EXPERT = 2e-2
+
+CASES = {
+    "tiny": I.CONFIGS["tiny"],
+    # ragged: several 128-row tiles per expert with tails, N not a power of two
+    "ragged": I.small_config("bwd_ragged", T=300, d=256, N=12, F=192, F_shared=128, K=3, M=4, config_id=930),
+    # F and F_shared multiples of 128 and d a multiple of 256: the wide tiles of every GEMM
+    "wide": I.small_config("bwd_wide", T=700, d=512, N=6, F=256, F_shared=384, K=2, M=2, config_id=931),
+    # T > 2048: the shared expert's weight gradients are split into K chunks and reduced
+    "split": I.small_config("bwd_split", T=4500, d=256, N=8, F=128, F_shared=128, K=4, M=8, config_id=932),
+    # M = 0 (plain top-K) and K = 1
+    "m0": I.small_config("bwd_m0", T=130, d=128, N=16, F=64, F_shared=64, K=2, M=0, config_id=933),
+    "k1": I.small_config("bwd_k1", T=257, d=128, N=32, F=64, F_shared=64, K=1, M=32, config_id=934),
+    "t1": I.small_config("bwd_t1", T=1, d=128, N=8, F=64, F_shared=64, K=4, M=8, config_id=935),
+    # skewed routing: experts with many rows next to experts with none
+    "skew": I.small_config("bwd_skew", T=512, d=256, N=64, F=128, F_shared=128, K=8, M=64, config_id=936,
+                           skew=True, seqs=2),
+}
+
+PP_CASES = {
+    "pp": I.small_config("bwd_pp", T=300, d=256, N=8, F=128, F_shared=128, K=4, M=4, C=2, V=2, config_id=937),
+    "pp_copy": I.small_config("bwd_pp_copy", T=160, d=128, N=4, F=64, F_shared=64, K=3, M=2, C=3, V=0,
+                              config_id=938),
+}
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def run(cfg, dy_scale=1.0, alpha=ALPHA, beta=BETA):
+    inp = I.make_inputs(cfg)
+    layer, x, tnb, out = H.run_forward(inp)
+    dy_bits = I.upstream_grad(cfg, scale=dy_scale) if dy_scale else np.zeros((cfg.T, cfg.d), np.uint16)
+    from token_choice_routing_b200.layer import bf16_tensor
+    from token_choice_routing_b200 import binding as B
+    dy = bf16_tensor(dy_bits, "cuda")
+    g = layer.backward(x, out, dy, alpha, beta)
+    torch.cuda.synchronize()
+    st = B.get_device_status(g["workspace"])
+    assert st == B.OK, B.status_string(st)
+    return inp, layer, x, out, dy, dy_bits, g
+
+
+def oracle_backward(inp, out, dy_bits, alpha, beta):
+    c = inp.cfg
+    s = out["logits"].cpu().numpy().astype(np.float64)
+    experts = (H.f64(inp.w_gate), H.f64(inp.w_up), H.f64(inp.w_down))
+    shared = (H.f64(inp.ws_gate), H.f64(inp.ws_up), H.f64(inp.ws_down))
+    cv = H.f64(inp.const_vectors) if c.V else None
+    return O.layer_backward(H.f64(inp.x), s, inp.w_router.astype(np.float64), c.N, c.M, c.K, experts, shared,
+                            H.f64(dy_bits), alpha, beta, C=c.C, V=c.V, const_vectors=cv)
+
+
+def check_all(inp, out, g, ref, counts):
+    c = inp.cfg
+    assert np.array_equal(out["topk_idx"].cpu().numpy(), ref["idx"])
+    assert rel(f64(g["dx"]), ref["dx"]) < REL
+    assert rel(f64(g["dw_router"]), ref["dW_r"]) < REL
+    assert rel(f64(g["dbias"]), ref["dbias"]) < REL
+    if c.M > 0:
+        assert rel(f64(g["dtok_null_bias"]), ref["dtnb"]) < REL
+    for k_gpu, k_ref in (("dws_gate", "dWs_gate"), ("dws_up", "dWs_up"), ("dws_down", "dWs_down")):
+        assert rel(f64(g[k_gpu]), ref[k_ref]) < REL, k_gpu
+    for k_gpu, k_ref in (("dw_gate", "dW_gate"), ("dw_up", "dW_up"), ("dw_down", "dW_down")):
+        G, R = f64(g[k_gpu]), ref[k_ref]
+        assert rel(G, R) < REL, k_gpu
+        for e in range(c.N):
+            if counts[e] == 0:
+                assert not np.any(G[e]), f"{k_gpu}[{e}] must be zero (expert without rows)"
+            else:
+                assert rel(G[e], R[e]) < REL_EXPERT, (k_gpu, e, counts[e])
+    if c.V:
+        assert rel(f64(g["dconst"]), ref["dconst"]) < REL
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_parity(name):
+    inp, layer, x, out, dy, dy_bits, g = run(CASES[name])
+    ref = oracle_backward(inp, out, dy_bits, ALPHA, BETA)
+    counts = out["counts"].cpu().numpy()
+    check_all(inp, out, g, ref, counts)
+
+
+@pytest.mark.parametrize("name", list(PP_CASES))
+def test_backward_parity_moepp(name):
+    inp, layer, x, out, dy, dy_bits, g = run(PP_CASES[name])
+    ref = oracle_backward(inp, out, dy_bits, ALPHA, BETA)
+    idx = out["topk_idx"].cpu().numpy()
+    c = inp.cfg
+    assert (idx >= c.N + c.M).any(), "the case must select copy or constant experts"
+    check_all(inp, out, g, ref, out["counts"].cpu().numpy())
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "skew"])
+def test_backward_loss_terms_only(name):
+    """dy = 0: only alpha L_bal + beta L_z act (weights 1 and 0.5 to make them large)."""
+    inp, layer, x, out, dy, dy_bits, g = run(CASES[name], dy_scale=0.0, alpha=1.0, beta=0.5)
+    ref = oracle_backward(inp, out, dy_bits, 1.0, 0.5)
+    for k in ("dw_gate", "dw_up", "dw_down", "dws_gate", "dws_up", "dws_down"):
+        assert not torch.any(g[k].float() != 0), k
+    assert rel(f64(g["dw_router"]), ref["dW_r"]) < 1e-4
+    assert rel(f64(g["dbias"]), ref["dbias"]) < 1e-4
+    assert rel(f64(g["dx"]), ref["dx"]) < REL  # router part only, rounded to bf16
+
+
+def test_backward_step_entry_points_match_the_whole_call():
+    """combine, router, router weight, expert FFN and input-gradient entry points called one
+    by one give bit-identical gradients to moe_backward."""
+    from token_choice_routing_b200 import binding as B
+    cfg = CASES["ragged"]
+    inp, layer, x, out, dy, dy_bits, g = run(cfg)
+    T, c = cfg.T, cfg
+    dm = layer.dims(T)
+    g2 = layer.alloc_grads(T)
+    bws = g2["workspace"]
+    dev = "cuda"
+    R = T * c.K
+    dys = torch.empty((R, c.d), dtype=torch.bfloat16, device=dev)
+    dg = torch.empty((T, c.K), dtype=torch.float32, device=dev)
+    ds = torch.empty((T, c.N + 1), dtype=torch.float32, device=dev)
+    dxs = torch.empty((R, c.d), dtype=torch.bfloat16, device=dev)
+    dxsh = torch.empty((T, c.d), dtype=torch.bfloat16, device=dev)
+    B.clear_device_status(bws)
+    B.combine_backward(dm, dy, out["ys"], out["topk_gate"], out["slot_row"], dys, dg, bws)
+    B.router_backward(dm, out["logits"], out["topk_idx"], out["topk_gate"], dg, out["counts_ext"], T, ALPHA, BETA,
+                      ds, g2["dtok_null_bias"])
+    B.router_weight_grad(dm, x, ds, g2["dw_router"], g2["dbias"], bws)
+    sv = layer.saved(x, out)
+    gr = B.Grads(*[None if g2.get(n) is None else g2[n].data_ptr() for n in B.GRAD_FIELDS])
+    B.expert_ffn_backward(dm, layer._weights, sv, dys, dy, dxs, dxsh, gr, bws)
+    B.input_grad(dm, dxsh, dxs, out["slot_row"], out["topk_idx"], out["topk_gate"], dy, ds, layer.w_router,
+                 g2["dx"], bws)
+    torch.cuda.synchronize()
+    assert B.get_device_status(bws) == B.OK
+    for k in ("dx", "dw_router", "dbias", "dtok_null_bias", "dw_gate", "dw_up", "dw_down", "dws_gate", "dws_up",
+              "dws_down"):
+        assert torch.equal(g[k], g2[k]), k
+
+
+def test_backward_is_deterministic():
+    cfg = CASES["split"]
+    inp, layer, x, out, dy, dy_bits, g = run(cfg)
+    g2 = layer.backward(x, out, dy, ALPHA, BETA)
+    torch.cuda.synchronize()
+    for k in ("dx", "dw_router", "dbias", "dw_gate", "dw_down", "dws_gate", "dws_up", "dws_down"):
+        assert torch.equal(g[k], g2[k]), k
+
+
+def test_backward_data_parallel_statistics():
+    """With counts and a token total from several ranks (here a made-up global total), the
+    load-balance gradient uses the global f_i and 1/T_total: compare with the oracle's
+    aux_backward evaluated on those statistics."""
+    from token_choice_routing_b200 import binding as B
+    cfg = CASES["tiny"]
+    inp, layer, x, out, dy, dy_bits, g = run(cfg, dy_scale=0.0, alpha=1.0, beta=0.5)
+    T, c = cfg.T, cfg
+    ce = (out["counts_ext"] * 3).contiguous()  # as if three ranks had routed alike
+    g3 = layer.backward(x, out, dy, 1.0, 0.5, counts_ext=ce, t_total=3 * T)
+    torch.cuda.synchronize()
+    s = out["logits"].cpu().numpy().astype(np.float64)
+    r = O.route(s, c.M, c.K)
+    dv = O.aux_backward(r["idx"], r["p"], r["lse"], c.N, 1.0, 0.5, counts=ce.cpu().numpy(), t_total=3 * T)
+    ds = O.pool_grad_to_logits(dv, c.N, c.M)
+    assert rel(f64(g3["dbias"]), ds.sum(axis=0)) < 1e-4
+    assert rel(f64(g3["dw_router"]), ds.T @ H.f64(inp.x)) < 1e-4

@@ -171,3 +171,25 @@ def test_gate_gradient_of_single_real_expert_is_zero():
     assert ((g["idx"] < 4).sum(axis=1) == 1).all()
     np.testing.assert_allclose(g["ds"], 0.0, atol=1e-15)
     assert np.abs(g["dg"][:, 0]).min() > 0
+
+
+def test_aux_backward_of_a_shard_equals_the_rows_of_the_whole_batch():
+    """Data parallel: with the whole batch's slot counts and token total, the loss-term
+    gradient of one shard's tokens equals those tokens' rows of the whole-batch gradient
+    (f and both means are whole-batch quantities; each token's row depends on no other
+    token's logits)."""
+    rng = np.random.default_rng(21)
+    T, N, M, K = 40, 6, 5, 3
+    s = rng.standard_normal((T, N + 1))
+    v = o.expanded_pool(s, M)
+    lse = o.pool_logsumexp(v)
+    p = o.pool_probs(v, lse)
+    idx = o.topk_pool(v, K)
+    whole = o.aux_backward(idx, p, lse, N, 0.7, 0.3)
+    counts = np.bincount(idx.reshape(-1), minlength=N + M)
+    for rows in (np.arange(0, 17), np.arange(17, 40)):
+        part = o.aux_backward(idx[rows], p[rows], lse[rows], N, 0.7, 0.3, counts=counts, t_total=T)
+        np.testing.assert_allclose(part, whole[rows], rtol=1e-13, atol=1e-16)
+    # and a shard's own statistics give something else
+    own = o.aux_backward(idx[:17], p[:17], lse[:17], N, 0.7, 0.3)
+    assert not np.allclose(own, whole[:17])

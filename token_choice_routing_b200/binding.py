@@ -45,6 +45,22 @@ class Outputs(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in OUTPUT_FIELDS]
 
 
+SAVED_FIELDS = ("x", "logits", "topk_idx", "topk_gate", "offsets", "slot_row", "xs", "h", "h_shared", "ys",
+                "counts_ext")
+
+
+class Saved(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in SAVED_FIELDS] + [("t_total", C.c_int64)]
+
+
+GRAD_FIELDS = ("dx", "dw_router", "dbias", "dtok_null_bias", "dw_gate", "dw_up", "dw_down", "dws_gate",
+               "dws_up", "dws_down", "dconst")
+
+
+class Grads(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in GRAD_FIELDS]
+
+
 def _load() -> C.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
@@ -74,12 +90,26 @@ def _load() -> C.CDLL:
         "moe_get_device_status": (i32, [vp, vp]),
         "moe_clear_device_status": (i32, [vp, vp]),
         "moe_selftest_bounded_wait": (i32, [vp, C.c_uint64, vp]),
+        "moe_backward_workspace_bytes": (sz, [pd]),
+        "moe_combine_backward": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_router_backward": (i32, [pd, vp, vp, vp, vp, vp, C.c_int64, C.c_float, C.c_float, vp, vp, vp]),
+        "moe_router_weight_grad": (i32, [pd, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_ffn_backward": (i32, [pd, C.POINTER(Weights), C.POINTER(Saved), vp, vp, vp, vp,
+                                          C.POINTER(Grads), vp, vp]),
+        "moe_input_grad": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_preact": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_dgrad_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_wgrad_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_dgrad_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_wgrad_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_backward": (i32, [pd, C.POINTER(Weights), C.POINTER(Saved), vp, C.c_float, C.c_float,
+                               C.POINTER(Grads), vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
         f.restype = res
         f.argtypes = args
-    if lib.moe_abi_version() != 2:
+    if lib.moe_abi_version() != 3:
         raise ImportError("libmoe_null ABI version mismatch")
     return lib
 
@@ -216,3 +246,78 @@ def clear_device_status(ws, stream=None):
 
 def selftest_bounded_wait(ws, limit_ns: int, stream=None):
     _check("moe_selftest_bounded_wait", LIB.moe_selftest_bounded_wait(_p(ws), int(limit_ns), _stream(stream)))
+
+
+# ------------------------------------------------------------------------------ backward
+
+
+def backward_workspace_bytes(dm: Dims) -> int:
+    return int(LIB.moe_backward_workspace_bytes(C.byref(dm)))
+
+
+def combine_backward(dm, dy, ys, topk_gate, slot_row, dys, dg, bws, stream=None, topk_idx=None, x=None,
+                     const_vectors=None):
+    _check("moe_combine_backward",
+           LIB.moe_combine_backward(C.byref(dm), _p(dy), _p(ys), _p(topk_gate), _p(slot_row), _p(topk_idx), _p(x),
+                                    _p(const_vectors), _p(dys), _p(dg), _p(bws), _stream(stream)))
+
+
+def router_backward(dm, logits, topk_idx, topk_gate, dg, counts_ext, t_total, alpha, beta, ds,
+                    dtok_null_bias=None, stream=None):
+    _check("moe_router_backward",
+           LIB.moe_router_backward(C.byref(dm), _p(logits), _p(topk_idx), _p(topk_gate), _p(dg), _p(counts_ext),
+                                   int(t_total), float(alpha), float(beta), _p(ds), _p(dtok_null_bias),
+                                   _stream(stream)))
+
+
+def router_weight_grad(dm, x, ds, dw_router, dbias, bws, stream=None):
+    _check("moe_router_weight_grad",
+           LIB.moe_router_weight_grad(C.byref(dm), _p(x), _p(ds), _p(dw_router), _p(dbias), _p(bws),
+                                      _stream(stream)))
+
+
+def expert_ffn_backward(dm, weights: Weights, saved: Saved, dys, dy, dxs, dx_shared, grads: Grads, bws,
+                        stream=None):
+    _check("moe_expert_ffn_backward",
+           LIB.moe_expert_ffn_backward(C.byref(dm), C.byref(weights), C.byref(saved), _p(dys), _p(dy), _p(dxs),
+                                       _p(dx_shared), C.byref(grads), _p(bws), _stream(stream)))
+
+
+def input_grad(dm, dx_shared, dxs, slot_row, topk_idx, topk_gate, dy, ds, w_router, dx, bws, stream=None):
+    _check("moe_input_grad",
+           LIB.moe_input_grad(C.byref(dm), _p(dx_shared), _p(dxs), _p(slot_row), _p(topk_idx), _p(topk_gate),
+                              _p(dy), _p(ds), _p(w_router), _p(dx), _p(bws), _stream(stream)))
+
+
+def backward(dm, weights: Weights, saved: Saved, dy, alpha, beta, grads: Grads, bws, stream=None):
+    _check("moe_backward", LIB.moe_backward(C.byref(dm), C.byref(weights), C.byref(saved), _p(dy), float(alpha),
+                                            float(beta), C.byref(grads), _p(bws), _stream(stream)))
+
+
+def expert_preact(dm, xs, x, offsets, gate_up, shared_gate_up, bws, stream=None):
+    _check("moe_expert_preact", LIB.moe_expert_preact(C.byref(dm), _p(xs), _p(x), _p(offsets), _p(gate_up),
+                                                      _p(shared_gate_up), _p(bws), _stream(stream)))
+
+
+def expert_dgrad_down(dm, offsets, dys, dy, w_down, shared_down, bws, stream=None):
+    _check("moe_expert_dgrad_down", LIB.moe_expert_dgrad_down(C.byref(dm), _p(offsets), _p(dys), _p(dy),
+                                                              _p(w_down), _p(shared_down), _p(bws),
+                                                              _stream(stream)))
+
+
+def expert_wgrad_down(dm, offsets, dys, dy, h, h_shared, dw_down, dws_down, bws, stream=None):
+    _check("moe_expert_wgrad_down", LIB.moe_expert_wgrad_down(C.byref(dm), _p(offsets), _p(dys), _p(dy), _p(h),
+                                                              _p(h_shared), _p(dw_down), _p(dws_down), _p(bws),
+                                                              _stream(stream)))
+
+
+def expert_dgrad_gate_up(dm, offsets, gate_up, shared_gate_up, dxs, dx_shared, bws, stream=None):
+    _check("moe_expert_dgrad_gate_up",
+           LIB.moe_expert_dgrad_gate_up(C.byref(dm), _p(offsets), _p(gate_up), _p(shared_gate_up), _p(dxs),
+                                        _p(dx_shared), _p(bws), _stream(stream)))
+
+
+def expert_wgrad_gate_up(dm, offsets, xs, x, dw_gate, dw_up, dws_gate, dws_up, bws, stream=None):
+    _check("moe_expert_wgrad_gate_up",
+           LIB.moe_expert_wgrad_gate_up(C.byref(dm), _p(offsets), _p(xs), _p(x), _p(dw_gate), _p(dw_up),
+                                        _p(dws_gate), _p(dws_up), _p(bws), _stream(stream)))

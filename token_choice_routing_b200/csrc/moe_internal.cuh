@@ -113,6 +113,51 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   return L;
 }
 
+// Backward-pass workspace (moe_backward_workspace_bytes). R_cap = T*K rows.
+int router_wgrad_chunks(const moe_dims_t& d, int* chunk_tokens);
+int bwd_shared_split(const moe_dims_t& d, int* chunk_kb);
+size_t bwd_split_partial_floats(const moe_dims_t& d);
+
+struct BwdLayout {
+  size_t hdr;    // uint32 status at 0 (256 B)
+  size_t z;      // bf16 [R_cap, 2F] gate/up pre-activations (packed column order)
+  size_t zs;     // bf16 [T, 2F_shared]
+  size_t dz;     // bf16 [R_cap, 2F] their gradients
+  size_t dzs;    // bf16 [T, 2F_shared]
+  size_t dys;    // bf16 [R_cap, d] upstream gradient of each routed row: g * dy
+  size_t dxs;    // bf16 [R_cap, d] input gradient of each routed row
+  size_t dxsh;   // bf16 [T, d] input gradient through the shared expert
+  size_t dg;     // fp32 [T, K] gate gradients
+  size_t ds;     // fp32 [T, N+1+C+V] logit gradients
+  size_t rpart;  // fp32 [chunks, rows, d] router weight-gradient partials
+  size_t bpart;  // fp32 [chunks, rows] router bias-gradient partials
+  size_t spart;  // fp32 shared-expert weight-gradient K-chunk partials
+  size_t total;
+};
+
+inline BwdLayout bwd_layout(const moe_dims_t& d) {
+  BwdLayout L{};
+  const size_t rcap = (size_t)d.T * d.K, T = (size_t)d.T;
+  const size_t rows = (size_t)router_rows(d);
+  const int nch = router_wgrad_chunks(d, nullptr);
+  size_t o = 0;
+  L.hdr = o; o += 256;
+  L.z = o; o = align_up(o + 2 * rcap * 2 * d.F, 256);
+  L.zs = o; o = align_up(o + 2 * T * 2 * d.F_shared, 256);
+  L.dz = o; o = align_up(o + 2 * rcap * 2 * d.F, 256);
+  L.dzs = o; o = align_up(o + 2 * T * 2 * d.F_shared, 256);
+  L.dys = o; o = align_up(o + 2 * rcap * d.d, 256);
+  L.dxs = o; o = align_up(o + 2 * rcap * d.d, 256);
+  L.dxsh = o; o = align_up(o + 2 * T * d.d, 256);
+  L.dg = o; o = align_up(o + 4 * T * d.K, 256);
+  L.ds = o; o = align_up(o + 4 * T * rows, 256);
+  L.rpart = o; o = align_up(o + 4 * (size_t)nch * rows * d.d, 256);
+  L.bpart = o; o = align_up(o + 4 * (size_t)nch * rows, 256);
+  L.spart = o; o = align_up(o + 4 * bwd_split_partial_floats(d), 256);
+  L.total = o;
+  return L;
+}
+
 template <typename T>
 inline T* ws_ptr(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
 template <typename T>
@@ -201,6 +246,36 @@ int launch_pack_gate_up(const moe_dims_t& d, const uint16_t* w_gate, const uint1
                         const uint16_t* ws_gate, const uint16_t* ws_up, uint16_t* gate_up,
                         uint16_t* sgate_up, cudaStream_t st);
 int launch_selftest_wait(void* ws, unsigned long long limit_ns, cudaStream_t st);
+
+// Backward pass (backward.cu, expert_ffn_bwd.cu, expert_ffn.cu).
+int launch_gate_up_preact(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                          const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* z, uint16_t* zs,
+                          uint32_t* status, cudaStream_t st);
+int launch_dgrad_down_swiglu(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
+                             const uint16_t* w_down, const uint16_t* sdown, const uint16_t* z, const uint16_t* zs,
+                             uint16_t* dz, uint16_t* dzs, uint32_t* status, cudaStream_t st);
+int launch_dgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dz, const uint16_t* dzs,
+                         const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* dxs, uint16_t* dx_shared,
+                         uint32_t* status, cudaStream_t st);
+int launch_wgrad_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
+                      const uint16_t* h, const uint16_t* h_shared, uint16_t* dw_down, uint16_t* dws_down,
+                      float* partials, uint32_t* status, cudaStream_t st);
+int launch_wgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dz, const uint16_t* dzs,
+                         const uint16_t* xs, const uint16_t* x, uint16_t* dw_gate, uint16_t* dw_up,
+                         uint16_t* dws_gate, uint16_t* dws_up, float* partials, uint32_t* status, cudaStream_t st);
+int launch_combine_bwd(const moe_dims_t& d, const uint16_t* dy, const uint16_t* ys, const float* topk_gate,
+                       const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                       const uint16_t* const_vectors, uint16_t* dys, float* dg, uint32_t* status, cudaStream_t st);
+int launch_router_bwd(const moe_dims_t& d, const float* logits, const int32_t* topk_idx, const float* topk_gate,
+                      const float* dg, const int32_t* counts_ext, long long t_total, float alpha, float beta,
+                      float* ds, float* dtnb, cudaStream_t st);
+int launch_router_wgrad(const moe_dims_t& d, const float* ds, const uint16_t* x, float* part, float* bpart,
+                        float* dw_router, float* dbias, cudaStream_t st);
+int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint16_t* dxs, const int32_t* slot_row,
+                      const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, const float* ds,
+                      const float* w_router, uint16_t* dx, uint32_t* status, cudaStream_t st);
+int launch_const_grad(const moe_dims_t& d, const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy,
+                      float* dconst, cudaStream_t st);
 
 // ------------------------------------------------------------------------------------
 // Device helpers.

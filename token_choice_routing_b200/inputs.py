@@ -43,7 +43,7 @@ SEED_BASE = 20260000
 # Order of the per-tensor sub-streams; never reorder (it would change inputs). New
 # streams go at the end: the earlier ones keep their draws.
 _STREAMS = ("x", "w_router", "w_gate", "w_up", "w_down",
-            "ws_gate", "ws_up", "ws_down", "spans", "const_vectors")
+            "ws_gate", "ws_up", "ws_down", "spans", "const_vectors", "dy")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -245,6 +245,13 @@ def make_inputs(cfg: LayerConfig, *, T: Optional[int] = None, weights: bool = Tr
     const_vectors = _normal_bf16(s["const_vectors"], (cfg.V, d), 0.5) if cfg.V else None
     return LayerInputs(cfg, x, w_router, bias, tok_null_bias,
                        w_gate, w_up, w_down, ws_gate, ws_up, ws_down, const_vectors)
+
+
+def upstream_grad(cfg: LayerConfig, *, T: Optional[int] = None, scale: float = 1.0) -> np.ndarray:
+    """Seeded upstream gradient dy of the layer output for the backward pass: N(0, scale^2)
+    bf16 bits [T, d], from the config's own "dy" stream."""
+    T = cfg.T if T is None else T
+    return _normal_bf16(_streams(cfg.seed)["dy"], (T, cfg.d), scale)
 
 
 def small_config(name: str = "small", *, T: int, d: int, N: int, F: int, F_shared: int,

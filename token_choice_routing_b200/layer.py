@@ -108,6 +108,54 @@ class MoENullLayer:
         out["workspace"] = torch.empty((max(B.workspace_bytes(self.dims(T)), 256),), dtype=torch.uint8, device=dev)
         return out
 
+    def alloc_grads(self, T: int) -> Dict[str, torch.Tensor]:
+        """Gradient buffers and the backward workspace for a T-token backward."""
+        dev, d, N, F, Fs = self.device, self.d, self.N, self.F, self.F_shared
+        rows = N + 1 + self.C + self.V
+        bf, f32 = torch.bfloat16, torch.float32
+        g = dict(
+            dx=torch.empty((max(T, 1), d), dtype=bf, device=dev),
+            dw_router=torch.empty((rows, d), dtype=f32, device=dev),
+            dbias=torch.empty((rows,), dtype=f32, device=dev),
+            dtok_null_bias=torch.empty((max(T, 1),), dtype=f32, device=dev),
+            dw_gate=torch.empty((N, F, d), dtype=bf, device=dev),
+            dw_up=torch.empty((N, F, d), dtype=bf, device=dev),
+            dw_down=torch.empty((N, d, F), dtype=bf, device=dev),
+            dws_gate=torch.empty((Fs, d), dtype=bf, device=dev),
+            dws_up=torch.empty((Fs, d), dtype=bf, device=dev),
+            dws_down=torch.empty((d, Fs), dtype=bf, device=dev),
+            dconst=torch.empty((self.V, d), dtype=f32, device=dev) if self.V else None,
+        )
+        g["workspace"] = torch.empty((max(B.backward_workspace_bytes(self.dims(T)), 256),), dtype=torch.uint8,
+                                     device=dev)
+        return g
+
+    def saved(self, x: torch.Tensor, out: Dict[str, torch.Tensor], counts_ext: Optional[torch.Tensor] = None,
+              t_total: Optional[int] = None) -> B.Saved:
+        """The forward tensors the backward reads. counts_ext and t_total default to this
+        call's own (one data-parallel rank); pass the all-reduced ones otherwise."""
+        if out.get("logits") is None or out.get("xs") is None:
+            raise ValueError("the backward needs the forward's logits and xs")
+        ce = out["counts_ext"] if counts_ext is None else counts_ext
+        ptr = lambda t: t.data_ptr()
+        return B.Saved(ptr(x), ptr(out["logits"]), ptr(out["topk_idx"]), ptr(out["topk_gate"]),
+                       ptr(out["offsets"]), ptr(out["slot_row"]), ptr(out["xs"]), ptr(out["h"]),
+                       ptr(out["h_shared"]), ptr(out["ys"]), ptr(ce),
+                       int(x.shape[0] if t_total is None else t_total))
+
+    def backward(self, x: torch.Tensor, out: Dict[str, torch.Tensor], dy: torch.Tensor, alpha: float = 2e-2,
+                 beta: float = 1e-3, grads: Optional[Dict[str, torch.Tensor]] = None,
+                 counts_ext: Optional[torch.Tensor] = None, t_total: Optional[int] = None,
+                 stream=None) -> Dict[str, torch.Tensor]:
+        """Gradients of <y, dy> + alpha L_bal + beta L_z through ``moe_backward``."""
+        T = x.shape[0]
+        if grads is None:
+            grads = self.alloc_grads(T)
+        sv = self.saved(x, out, counts_ext, t_total)
+        g = B.Grads(*[None if grads.get(n) is None else grads[n].data_ptr() for n in B.GRAD_FIELDS])
+        B.backward(self.dims(T), self._weights, sv, dy, alpha, beta, g, grads["workspace"], stream)
+        return grads
+
     def forward(self, x: torch.Tensor, tok_null_bias: Optional[torch.Tensor] = None,
                 out: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
         T = x.shape[0]
