@@ -267,18 +267,19 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         ("combine_bwd", lambda: B.combine_backward(dm, dy, o["ys"], o["topk_gate"], o["slot_row"], dys, dg, bws,
                                                    topk_idx=o["topk_idx"], x=x, const_vectors=layer.const_vectors)),
         ("router_bwd", lambda: B.router_backward(dm, o["logits"], o["topk_idx"], o["topk_gate"], dg, o["counts_ext"],
-                                                 T, BWD_ALPHA, BWD_BETA, ds, grads["dtok_null_bias"])),
-        ("router_wgrad", lambda: B.router_weight_grad(dm, x, ds, grads["dw_router"], grads["dbias"], bws)),
-        ("preact", lambda: B.expert_preact(dm, o["xs"], x, o["offsets"], layer.gate_up, layer.shared_gate_up, bws)),
+                                                 T, BWD_ALPHA, BWD_BETA, ds, bws, grads["dtok_null_bias"])),
+        ("router_wgrad", lambda: B.router_weight_grad(dm, x, grads["dw_router"], grads["dbias"], bws)),
         ("dgrad_down", lambda: B.expert_dgrad_down(dm, o["offsets"], dys, dy, layer.w_down, layer.shared_down, bws)),
+        ("swiglu_bwd", lambda: B.expert_swiglu_backward(dm, o["xs"], x, o["offsets"], layer.gate_up,
+                                                        layer.shared_gate_up, bws)),
         ("wgrad_down", lambda: B.expert_wgrad_down(dm, o["offsets"], dys, dy, o["h"], o["h_shared"],
                                                    grads["dw_down"], grads["dws_down"], bws)),
-        ("dgrad_gate_up", lambda: B.expert_dgrad_gate_up(dm, o["offsets"], layer.gate_up, layer.shared_gate_up, dxs,
-                                                         dxsh, bws)),
+        ("dgrad_gate_up", lambda: B.expert_dgrad_gate_up(dm, o["offsets"], layer.gate_up, layer.shared_gate_up,
+                                                         layer.w_router, dxs, dxsh, bws)),
         ("wgrad_gate_up", lambda: B.expert_wgrad_gate_up(dm, o["offsets"], o["xs"], x, grads["dw_gate"],
                                                          grads["dw_up"], grads["dws_gate"], grads["dws_up"], bws)),
-        ("input_grad", lambda: B.input_grad(dm, dxsh, dxs, o["slot_row"], o["topk_idx"], o["topk_gate"], dy, ds,
-                                            layer.w_router, grads["dx"], bws)),
+        ("input_grad", lambda: B.input_grad(dm, dxsh, dxs, o["slot_row"], o["topk_idx"], o["topk_gate"], dy,
+                                            grads["dx"], bws)),
     ]
     acc = {n: 0.0 for n, _ in stages}
     nb = max(3, min(args.steps, 10))
@@ -298,17 +299,17 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     kms = {n: acc[n] / nb for n in acc}
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    fl = {"preact": 4.0 * d * (F * R + Fs * T), "dgrad_down": 2.0 * d * (F * R + Fs * T),
-          "wgrad_down": 2.0 * d * (F * R + Fs * T), "dgrad_gate_up": 4.0 * d * (F * R + Fs * T),
-          "wgrad_gate_up": 4.0 * d * (F * R + Fs * T),
-          "router_wgrad": 2.0 * rows * d * T, "input_grad": 2.0 * rows * d * T}
+    # the router's input gradient ds W_r rides in dgrad_gate_up (extra k-blocks of the shared tiles)
+    fl = {"swiglu_bwd": 4.0 * d * (F * R + Fs * T), "dgrad_down": 2.0 * d * (F * R + Fs * T),
+          "wgrad_down": 2.0 * d * (F * R + Fs * T), "dgrad_gate_up": 4.0 * d * (F * R + Fs * T) + 2.0 * rows * d * T,
+          "wgrad_gate_up": 4.0 * d * (F * R + Fs * T), "router_wgrad": 2.0 * rows * d * T}
     by = {"combine_bwd": 2.0 * d * T + 4.0 * d * R + 12.0 * K * T,
           "router_bwd": 8.0 * rows * T + 12.0 * K * T,
-          "input_grad": 4.0 * d * T + 2.0 * d * R + 4.0 * rows * T + 4.0 * K * T}
+          "input_grad": 4.0 * d * T + 2.0 * d * R + 8.0 * K * T}
     kernels = {}
     for n, ms in kms.items():
         k = {"ms": ms}
-        if n in ("preact", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"):
+        if n in ("swiglu_bwd", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up", "router_wgrad"):
             k.update(bound="tensor", **{"TFLOP/s": fl[n] / (ms * 1e9)})
             k["frac"] = k["TFLOP/s"] / bf16_peak
         elif n in by:
@@ -317,23 +318,26 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         else:
             k.update(bound="alu", **{"TFLOP/s": fl[n] / (ms * 1e9)})
         kernels[n] = k
-    gemm = ["preact", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"]
+    gemm = ["swiglu_bwd", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"]
     top = max(gemm, key=lambda n: kms[n])
     gemm_ms = sum(kms[n] for n in gemm)
     gemm_flops = sum(fl[n] for n in gemm)
     split = 2 if (T + 63) // 64 > 32 else 0  # shared-expert K-chunk reductions of the two weight gradients
+    # combine_bwd, router_bwd, router wgrad (+ reduce), W_r split, preact, dgrad/wgrad down, dgrad/wgrad
+    # gate/up, input_grad
+    launches = 11 + split + (1 if cfg.V else 0)
     return {
         "metric": "real-slot tokens/s per MoE layer bwd", "value": R * args.steps / (total_ms * 1e-3),
         "unit": UNIT, "ms_per_step": total_ms / args.steps, "steps": args.steps,
         "objective": f"<y, dy> + {BWD_ALPHA} L_bal + {BWD_BETA} L_z (dy seeded N(0,1) bf16)",
-        "preactivations": "recomputed by the gate/up GEMM without its SwiGLU epilogue",
+        "preactivations": "recomputed in fp32 on the tensor cores; the SwiGLU derivative in that GEMM's epilogue",
         "ffn_tflops_real_rows": gemm_flops / (gemm_ms * 1e9),
         "roofline": {"kernel": f"{top} grouped GEMM (tcgen05)", "bound": "tensor",
                      "achieved": fl[top] / (kms[top] * 1e9), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": fl[top] / (kms[top] * 1e9) / bf16_peak, "peak_kind": f"{peak_kind} bf16 burst",
                      "traffic": None, "flops_per_launch": fl[top], "ms_per_launch": kms[top]},
         "kernels": kernels,
-        "gpu_launches": (11 + split + (1 if cfg.V else 0)) * args.steps,
+        "gpu_launches": launches * args.steps,
     }
 
 

@@ -315,8 +315,9 @@ MOE_API int moe_selftest_bounded_wait(void* workspace, uint64_t limit_ns, moe_st
  * constant in the logits and carry no gradient; the logits receive gradient through
  * the renormalised gates, through P_i in L_bal and through lse in L_z. As in the
  * forward, null slots cost nothing: the expert gradients run on the real rows only.
- * Each expert is SwiGLU; its gate/up pre-activations are recomputed from xs with the
- * forward's gate/up GEMM (no SwiGLU epilogue) rather than stored by the forward.
+ * Each expert is SwiGLU; its gate/up pre-activations are recomputed from xs on the tensor
+ * cores (fp32 in TMEM) rather than stored by the forward, and the SwiGLU derivative is
+ * taken in that GEMM's epilogue.
  *
  * Requirements: the forward ran with out->logits and out->xs non-NULL (the copy
  * path). Weight gradients of the experts are bf16; router, bias and constant-vector
@@ -376,59 +377,69 @@ MOE_API int moe_combine_backward(const moe_dims_t* dims, const uint16_t* dy, con
  * slot counts: gates g = softmax over the selected non-null slots give
  * g_k (dg_k - sum_l g_l dg_l); alpha L_bal gives alpha (N/t_total) p_i (f_i - sum_l f_l p_l)
  * over the pool; beta L_z gives beta (2/t_total) lse_t p_i. The null logit's entry sums
- * its M copies. dtok_null_bias (optional, [T]) receives column N. */
+ * its M copies. dtok_null_bias (optional, [T]) receives column N. The call also leaves in
+ * the backward workspace ds as two bf16 terms (hi = bf16(ds), lo = bf16(ds - hi)) and
+ * per-warp column sums of ds, which moe_router_weight_grad and the router term of
+ * moe_expert_dgrad_gate_up read. */
 MOE_API int moe_router_backward(const moe_dims_t* dims, const float* logits, const int32_t* topk_idx,
                                 const float* topk_gate, const float* dg, const int32_t* counts_ext,
                                 int64_t t_total, float alpha, float beta, float* ds, float* dtok_null_bias,
-                                moe_stream_t stream);
+                                void* bwd_workspace, moe_stream_t stream);
 
-/* dw_router = ds^T x ([N+1+C+V, d] fp32) and dbias = sum_t ds (optional), summed in
+/* dw_router = ds^T x ([N+1+C+V, d] fp32) on the tensor cores from the two-term ds that
+ * moe_router_backward left in the workspace (x is bf16, so each product is exact; the
+ * terms carry ds to 2^-16 relative), and dbias = sum_t ds (optional). Both are summed in
  * a fixed order (deterministic). */
-MOE_API int moe_router_weight_grad(const moe_dims_t* dims, const uint16_t* x, const float* ds, float* dw_router,
-                                   float* dbias, void* bwd_workspace, moe_stream_t stream);
+MOE_API int moe_router_weight_grad(const moe_dims_t* dims, const uint16_t* x, float* dw_router, float* dbias,
+                                   void* bwd_workspace, moe_stream_t stream);
 
-/* Expert FFN backward (实现: grouped GEMMs over the real rows only): recomputes the
- * gate/up pre-activations, then dgrad of the down projection fused with the SwiGLU
- * derivative, the down weight gradient, dgrad of gate/up and the gate/up weight
+/* Expert FFN backward (实现: grouped GEMMs over the real rows only): dgrad of the down
+ * projection, the gate/up pre-activations recomputed with the SwiGLU derivative in the
+ * same GEMM's epilogue, the down weight gradient, dgrad of gate/up and the gate/up weight
  * gradient, for the routed experts (rows of xs, upstream dys) and the shared expert
  * (rows of x, upstream dy). Writes dxs [R_cap, d] and dx_shared [T, d] (bf16) and
- * g->dw_gate/up/down and g->dws_gate/up/down. */
+ * g->dw_gate/up/down and g->dws_gate/up/down. When w->w_router is set, dx_shared also
+ * receives the router's input gradient ds W_r (two-term products hi*hi + hi*lo + lo*hi
+ * on the tensor cores, as extra k-blocks of the shared expert's tiles), from the ds that
+ * moe_router_backward left in the workspace. */
 MOE_API int moe_expert_ffn_backward(const moe_dims_t* dims, const moe_weights_t* w, const moe_saved_t* saved,
                                     const uint16_t* dys, const uint16_t* dy, uint16_t* dxs, uint16_t* dx_shared,
                                     const moe_grads_t* g, void* bwd_workspace, moe_stream_t stream);
 
 /* The five stages of moe_expert_ffn_backward, one GEMM launch each, for callers that
- * schedule or time them separately. The pre-activations z and their gradients dz live in
- * the backward workspace; call the stages in this order:
- *   moe_expert_preact        z = [xs W_g^T | xs W_u^T] (packed order), shared from x
- *   moe_expert_dgrad_down    dh = dys W_d, then dz from dh and z (SwiGLU derivative)
- *   moe_expert_wgrad_down    dw_down[e] = dys_e^T h_e, dws_down = dy^T h_shared
- *   moe_expert_dgrad_gate_up dxs = dz W_gu, dx_shared = dz_shared W_sgu
+ * schedule or time them separately. dh and dz live in the backward workspace; call the
+ * stages in this order:
+ *   moe_expert_dgrad_down      dh = dys W_d (routed), dh_shared = dy W_sd
+ *   moe_expert_swiglu_backward z = [xs W_g^T | xs W_u^T] recomputed in fp32 on the tensor
+ *                              cores; its epilogue writes dz = [da | db] (packed order) with
+ *                              da = dh b sigma(a) (1 + a (1 - sigma(a))), db = dh a sigma(a)
+ *   moe_expert_wgrad_down      dw_down[e] = dys_e^T h_e, dws_down = dy^T h_shared
+ *   moe_expert_dgrad_gate_up dxs = dz W_gu, dx_shared = dz_shared W_sgu (+ ds W_r when
+ *                            w_router is not NULL)
  *   moe_expert_wgrad_gate_up dw_gate/dw_up[e] = dz_e^T xs_e (unpacked), shared from x */
-MOE_API int moe_expert_preact(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x,
-                              const int32_t* offsets, const uint16_t* gate_up, const uint16_t* shared_gate_up,
-                              void* bwd_workspace, moe_stream_t stream);
 MOE_API int moe_expert_dgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys,
                                   const uint16_t* dy, const uint16_t* w_down, const uint16_t* shared_down,
                                   void* bwd_workspace, moe_stream_t stream);
+MOE_API int moe_expert_swiglu_backward(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x,
+                                       const int32_t* offsets, const uint16_t* gate_up,
+                                       const uint16_t* shared_gate_up, void* bwd_workspace, moe_stream_t stream);
 MOE_API int moe_expert_wgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys,
                                   const uint16_t* dy, const uint16_t* h, const uint16_t* h_shared,
                                   uint16_t* dw_down, uint16_t* dws_down, void* bwd_workspace,
                                   moe_stream_t stream);
 MOE_API int moe_expert_dgrad_gate_up(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* gate_up,
-                                     const uint16_t* shared_gate_up, uint16_t* dxs, uint16_t* dx_shared,
-                                     void* bwd_workspace, moe_stream_t stream);
+                                     const uint16_t* shared_gate_up, const float* w_router, uint16_t* dxs,
+                                     uint16_t* dx_shared, void* bwd_workspace, moe_stream_t stream);
 MOE_API int moe_expert_wgrad_gate_up(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* xs,
                                      const uint16_t* x, uint16_t* dw_gate, uint16_t* dw_up, uint16_t* dws_gate,
                                      uint16_t* dws_up, void* bwd_workspace, moe_stream_t stream);
 
-/* Input gradient: dx[t] = dx_shared[t] + sum over the token's real slots of
- * dxs[slot_row] + sum over its copy-expert slots of g dy[t] + sum_j ds[t, j] W_r[j, :],
- * accumulated in fp32 and rounded once to bf16. */
+/* Input gradient: dx[t] = dx_shared[t] (the shared expert's and the router's input
+ * gradient) + sum over the token's real slots of dxs[slot_row] + sum over its copy-expert
+ * slots of g dy[t], accumulated in fp32 in rank order and rounded once to bf16. */
 MOE_API int moe_input_grad(const moe_dims_t* dims, const uint16_t* dx_shared, const uint16_t* dxs,
                            const int32_t* slot_row, const int32_t* topk_idx, const float* topk_gate,
-                           const uint16_t* dy, const float* ds, const float* w_router, uint16_t* dx,
-                           void* bwd_workspace, moe_stream_t stream);
+                           const uint16_t* dy, uint16_t* dx, void* bwd_workspace, moe_stream_t stream);
 
 /* The whole backward: combine, router, router weight gradient, expert FFNs, input
  * gradient and (V > 0) the constant experts' gradient. */

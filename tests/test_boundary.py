@@ -150,15 +150,20 @@ def test_backward_workspace_and_host_side_rejections(lib):
     nul = None
     inv = B.ERR_INVALID_ARG
     assert L.moe_combine_backward(C.byref(dm), *([nul] * 11)) == inv
-    assert L.moe_router_backward(C.byref(dm), nul, nul, nul, nul, nul, T, 0.02, 0.001, nul, nul, nul) == inv
-    assert L.moe_router_weight_grad(C.byref(dm), nul, nul, nul, nul, nul, nul) == inv
+    assert L.moe_router_backward(C.byref(dm), nul, nul, nul, nul, nul, T, 0.02, 0.001, nul, nul, nul, nul) == inv
+    assert L.moe_router_weight_grad(C.byref(dm), nul, nul, nul, nul, nul) == inv
     assert L.moe_expert_ffn_backward(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul) == inv
-    assert L.moe_input_grad(C.byref(dm), *([nul] * 11)) == inv
+    assert L.moe_input_grad(C.byref(dm), *([nul] * 9)) == inv
+    assert L.moe_expert_dgrad_down(C.byref(dm), *([nul] * 7)) == inv
+    assert L.moe_expert_swiglu_backward(C.byref(dm), *([nul] * 7)) == inv
+    assert L.moe_expert_wgrad_down(C.byref(dm), *([nul] * 9)) == inv
+    assert L.moe_expert_dgrad_gate_up(C.byref(dm), *([nul] * 8)) == inv
+    assert L.moe_expert_wgrad_gate_up(C.byref(dm), *([nul] * 9)) == inv
     assert L.moe_backward(C.byref(dm), nul, nul, nul, 0.02, 0.001, nul, nul, nul) == inv
     # a token total smaller than this call's tokens is never valid (pointers set to a dummy value)
     fake = C.c_void_p(256)
     assert L.moe_router_backward(C.byref(dm), fake, fake, fake, fake, fake, T - 1, 0.02, 0.001, fake, nul,
-                                 nul) == inv
+                                 fake, nul) == inv
     # invalid dims first; T = 0 is a no-op
     bad = B.dims(256, 100, 8, 8, 4, 64, 64)
     assert L.moe_backward(C.byref(bad), nul, nul, nul, 0.02, 0.001, nul, nul, nul) == B.ERR_UNSUPPORTED

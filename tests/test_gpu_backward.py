@@ -154,18 +154,35 @@ def test_backward_step_entry_points_match_the_whole_call():
     B.clear_device_status(bws)
     B.combine_backward(dm, dy, out["ys"], out["topk_gate"], out["slot_row"], dys, dg, bws)
     B.router_backward(dm, out["logits"], out["topk_idx"], out["topk_gate"], dg, out["counts_ext"], T, ALPHA, BETA,
-                      ds, g2["dtok_null_bias"])
-    B.router_weight_grad(dm, x, ds, g2["dw_router"], g2["dbias"], bws)
+                      ds, bws, g2["dtok_null_bias"])
+    B.router_weight_grad(dm, x, g2["dw_router"], g2["dbias"], bws)
     sv = layer.saved(x, out)
     gr = B.Grads(*[None if g2.get(n) is None else g2[n].data_ptr() for n in B.GRAD_FIELDS])
     B.expert_ffn_backward(dm, layer._weights, sv, dys, dy, dxs, dxsh, gr, bws)
-    B.input_grad(dm, dxsh, dxs, out["slot_row"], out["topk_idx"], out["topk_gate"], dy, ds, layer.w_router,
-                 g2["dx"], bws)
+    B.input_grad(dm, dxsh, dxs, out["slot_row"], out["topk_idx"], out["topk_gate"], dy, g2["dx"], bws)
     torch.cuda.synchronize()
     assert B.get_device_status(bws) == B.OK
     for k in ("dx", "dw_router", "dbias", "dtok_null_bias", "dw_gate", "dw_up", "dw_down", "dws_gate", "dws_up",
               "dws_down"):
         assert torch.equal(g[k], g2[k]), k
+    # and the five GEMM stages one by one give the same expert gradients and dx
+    g3 = layer.alloc_grads(T)
+    bws3 = g3["workspace"]
+    B.clear_device_status(bws3)
+    B.combine_backward(dm, dy, out["ys"], out["topk_gate"], out["slot_row"], dys, dg, bws3)
+    B.router_backward(dm, out["logits"], out["topk_idx"], out["topk_gate"], dg, out["counts_ext"], T, ALPHA, BETA,
+                      ds, bws3, g3["dtok_null_bias"])
+    B.expert_dgrad_down(dm, out["offsets"], dys, dy, layer.w_down, layer.shared_down, bws3)
+    B.expert_swiglu_backward(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, bws3)
+    B.expert_wgrad_down(dm, out["offsets"], dys, dy, out["h"], out["h_shared"], g3["dw_down"], g3["dws_down"], bws3)
+    B.expert_dgrad_gate_up(dm, out["offsets"], layer.gate_up, layer.shared_gate_up, layer.w_router, dxs, dxsh, bws3)
+    B.expert_wgrad_gate_up(dm, out["offsets"], out["xs"], x, g3["dw_gate"], g3["dw_up"], g3["dws_gate"],
+                           g3["dws_up"], bws3)
+    B.input_grad(dm, dxsh, dxs, out["slot_row"], out["topk_idx"], out["topk_gate"], dy, g3["dx"], bws3)
+    torch.cuda.synchronize()
+    assert B.get_device_status(bws3) == B.OK
+    for k in ("dx", "dw_gate", "dw_up", "dw_down", "dws_gate", "dws_up", "dws_down"):
+        assert torch.equal(g[k], g3[k]), k
 
 
 def test_backward_is_deterministic():

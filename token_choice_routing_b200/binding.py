@@ -92,15 +92,15 @@ def _load() -> C.CDLL:
         "moe_selftest_bounded_wait": (i32, [vp, C.c_uint64, vp]),
         "moe_backward_workspace_bytes": (sz, [pd]),
         "moe_combine_backward": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
-        "moe_router_backward": (i32, [pd, vp, vp, vp, vp, vp, C.c_int64, C.c_float, C.c_float, vp, vp, vp]),
-        "moe_router_weight_grad": (i32, [pd, vp, vp, vp, vp, vp, vp]),
+        "moe_router_backward": (i32, [pd, vp, vp, vp, vp, vp, C.c_int64, C.c_float, C.c_float, vp, vp, vp, vp]),
+        "moe_router_weight_grad": (i32, [pd, vp, vp, vp, vp, vp]),
         "moe_expert_ffn_backward": (i32, [pd, C.POINTER(Weights), C.POINTER(Saved), vp, vp, vp, vp,
                                           C.POINTER(Grads), vp, vp]),
-        "moe_input_grad": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
-        "moe_expert_preact": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_input_grad": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_swiglu_backward": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_dgrad_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_wgrad_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
-        "moe_expert_dgrad_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_dgrad_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_wgrad_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_backward": (i32, [pd, C.POINTER(Weights), C.POINTER(Saved), vp, C.c_float, C.c_float,
                                C.POINTER(Grads), vp, vp]),
@@ -262,18 +262,17 @@ def combine_backward(dm, dy, ys, topk_gate, slot_row, dys, dg, bws, stream=None,
                                     _p(const_vectors), _p(dys), _p(dg), _p(bws), _stream(stream)))
 
 
-def router_backward(dm, logits, topk_idx, topk_gate, dg, counts_ext, t_total, alpha, beta, ds,
+def router_backward(dm, logits, topk_idx, topk_gate, dg, counts_ext, t_total, alpha, beta, ds, bws,
                     dtok_null_bias=None, stream=None):
     _check("moe_router_backward",
            LIB.moe_router_backward(C.byref(dm), _p(logits), _p(topk_idx), _p(topk_gate), _p(dg), _p(counts_ext),
-                                   int(t_total), float(alpha), float(beta), _p(ds), _p(dtok_null_bias),
+                                   int(t_total), float(alpha), float(beta), _p(ds), _p(dtok_null_bias), _p(bws),
                                    _stream(stream)))
 
 
-def router_weight_grad(dm, x, ds, dw_router, dbias, bws, stream=None):
+def router_weight_grad(dm, x, dw_router, dbias, bws, stream=None):
     _check("moe_router_weight_grad",
-           LIB.moe_router_weight_grad(C.byref(dm), _p(x), _p(ds), _p(dw_router), _p(dbias), _p(bws),
-                                      _stream(stream)))
+           LIB.moe_router_weight_grad(C.byref(dm), _p(x), _p(dw_router), _p(dbias), _p(bws), _stream(stream)))
 
 
 def expert_ffn_backward(dm, weights: Weights, saved: Saved, dys, dy, dxs, dx_shared, grads: Grads, bws,
@@ -283,10 +282,10 @@ def expert_ffn_backward(dm, weights: Weights, saved: Saved, dys, dy, dxs, dx_sha
                                        _p(dx_shared), C.byref(grads), _p(bws), _stream(stream)))
 
 
-def input_grad(dm, dx_shared, dxs, slot_row, topk_idx, topk_gate, dy, ds, w_router, dx, bws, stream=None):
+def input_grad(dm, dx_shared, dxs, slot_row, topk_idx, topk_gate, dy, dx, bws, stream=None):
     _check("moe_input_grad",
            LIB.moe_input_grad(C.byref(dm), _p(dx_shared), _p(dxs), _p(slot_row), _p(topk_idx), _p(topk_gate),
-                              _p(dy), _p(ds), _p(w_router), _p(dx), _p(bws), _stream(stream)))
+                              _p(dy), _p(dx), _p(bws), _stream(stream)))
 
 
 def backward(dm, weights: Weights, saved: Saved, dy, alpha, beta, grads: Grads, bws, stream=None):
@@ -294,9 +293,10 @@ def backward(dm, weights: Weights, saved: Saved, dy, alpha, beta, grads: Grads, 
                                             float(beta), C.byref(grads), _p(bws), _stream(stream)))
 
 
-def expert_preact(dm, xs, x, offsets, gate_up, shared_gate_up, bws, stream=None):
-    _check("moe_expert_preact", LIB.moe_expert_preact(C.byref(dm), _p(xs), _p(x), _p(offsets), _p(gate_up),
-                                                      _p(shared_gate_up), _p(bws), _stream(stream)))
+def expert_swiglu_backward(dm, xs, x, offsets, gate_up, shared_gate_up, bws, stream=None):
+    _check("moe_expert_swiglu_backward",
+           LIB.moe_expert_swiglu_backward(C.byref(dm), _p(xs), _p(x), _p(offsets), _p(gate_up), _p(shared_gate_up),
+                                          _p(bws), _stream(stream)))
 
 
 def expert_dgrad_down(dm, offsets, dys, dy, w_down, shared_down, bws, stream=None):
@@ -311,10 +311,11 @@ def expert_wgrad_down(dm, offsets, dys, dy, h, h_shared, dw_down, dws_down, bws,
                                                               _stream(stream)))
 
 
-def expert_dgrad_gate_up(dm, offsets, gate_up, shared_gate_up, dxs, dx_shared, bws, stream=None):
+def expert_dgrad_gate_up(dm, offsets, gate_up, shared_gate_up, w_router, dxs, dx_shared, bws, stream=None):
+    """w_router (or None): add the router's input gradient ds W_r to dx_shared."""
     _check("moe_expert_dgrad_gate_up",
-           LIB.moe_expert_dgrad_gate_up(C.byref(dm), _p(offsets), _p(gate_up), _p(shared_gate_up), _p(dxs),
-                                        _p(dx_shared), _p(bws), _stream(stream)))
+           LIB.moe_expert_dgrad_gate_up(C.byref(dm), _p(offsets), _p(gate_up), _p(shared_gate_up), _p(w_router),
+                                        _p(dxs), _p(dx_shared), _p(bws), _stream(stream)))
 
 
 def expert_wgrad_gate_up(dm, offsets, xs, x, dw_gate, dw_up, dws_gate, dws_up, bws, stream=None):

@@ -17,25 +17,44 @@ static int check_pp_inputs(const moe_dims_t* d, const int32_t* topk_idx, const u
   return MOE_OK;
 }
 
+// The five expert GEMMs. With w->w_router set, the router's input gradient ds W_r (from the
+// split ds that the router backward left in the workspace) is added to dx_shared inside the
+// shared expert's gate/up dgrad.
 static int expert_ffn_bwd(const moe_dims_t& d, const moe_weights_t* w, const moe_saved_t* sv, const uint16_t* dys,
                           const uint16_t* dy, uint16_t* dxs, uint16_t* dx_shared, const moe_grads_t* g, void* ws,
                           cudaStream_t st) {
   const BwdLayout L = bwd_layout(d);
   uint32_t* status = ws_ptr<uint32_t>(ws, L.hdr);
-  uint16_t* z = ws_ptr<uint16_t>(ws, L.z);
-  uint16_t* zs = ws_ptr<uint16_t>(ws, L.zs);
+  uint16_t* dh = ws_ptr<uint16_t>(ws, L.dh);
+  uint16_t* dhs = ws_ptr<uint16_t>(ws, L.dhs);
   uint16_t* dz = ws_ptr<uint16_t>(ws, L.dz);
   uint16_t* dzs = ws_ptr<uint16_t>(ws, L.dzs);
   float* spart = ws_ptr<float>(ws, L.spart);
-  MOE_CHECK(launch_gate_up_preact(d, sv->xs, sv->x, sv->offsets, w->gate_up, w->shared_gate_up, z, zs, status, st));
-  MOE_CHECK(launch_dgrad_down_swiglu(d, sv->offsets, dys, dy, w->w_down, w->shared_down, z, zs, dz, dzs, status,
-                                     st));
+  uint16_t* dsplit = nullptr;
+  uint16_t* w2 = nullptr;
+  if (w->w_router) {
+    dsplit = ws_ptr<uint16_t>(ws, L.dsplit);
+    w2 = ws_ptr<uint16_t>(ws, L.w2);
+    MOE_CHECK(launch_router_split2(d, w->w_router, w2, st));
+  }
+  MOE_CHECK(launch_dgrad_down(d, sv->offsets, dys, dy, w->w_down, w->shared_down, dh, dhs, status, st));
+  MOE_CHECK(launch_swiglu_backward(d, sv->offsets, sv->xs, sv->x, w->gate_up, w->shared_gate_up, dh, dhs, dz, dzs,
+                                   status, st));
   MOE_CHECK(launch_wgrad_down(d, sv->offsets, dys, dy, sv->h, sv->h_shared, g->dw_down, g->dws_down, spart, status,
                               st));
-  MOE_CHECK(launch_dgrad_gate_up(d, sv->offsets, dz, dzs, w->gate_up, w->shared_gate_up, dxs, dx_shared, status,
-                                 st));
+  MOE_CHECK(launch_dgrad_gate_up(d, sv->offsets, dz, dzs, w->gate_up, w->shared_gate_up, dsplit, w2, dxs, dx_shared,
+                                 status, st));
   return launch_wgrad_gate_up(d, sv->offsets, dz, dzs, sv->xs, sv->x, g->dw_gate, g->dw_up, g->dws_gate, g->dws_up,
                               spart, status, st);
+}
+
+static int router_wgrad(const moe_dims_t& d, const uint16_t* x, float* dw_router, float* dbias, void* ws,
+                        cudaStream_t st) {
+  const BwdLayout L = bwd_layout(d);
+  float* part = ws_ptr<float>(ws, L.rpart);
+  MOE_CHECK(launch_router_wgrad_tc(d, ws_ptr<uint16_t>(ws, L.dsplit), x, part, ws_ptr<uint32_t>(ws, L.hdr), st));
+  return launch_router_wgrad_reduce(d, part, router_wgrad_split(d, nullptr), ws_ptr<float>(ws, L.bpart), dw_router,
+                                    dbias, st);
 }
 
 static bool saved_ok(const moe_saved_t* s, const moe_dims_t* d) {
@@ -69,17 +88,19 @@ int moe_combine_backward(const moe_dims_t* dims, const uint16_t* dy, const uint1
 
 int moe_router_backward(const moe_dims_t* dims, const float* logits, const int32_t* topk_idx, const float* topk_gate,
                         const float* dg, const int32_t* counts_ext, int64_t t_total, float alpha, float beta,
-                        float* ds, float* dtok_null_bias, moe_stream_t stream) {
+                        float* ds, float* dtok_null_bias, void* bwd_workspace, moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));
   if (dims->T == 0) return MOE_OK;
-  if (!logits || !topk_idx || !topk_gate || !dg || !counts_ext || !ds) return MOE_ERR_INVALID_ARG;
+  if (!logits || !topk_idx || !topk_gate || !dg || !counts_ext || !ds || !bwd_workspace) return MOE_ERR_INVALID_ARG;
   if (t_total < (int64_t)dims->T || t_total <= 0) return MOE_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(*dims);
   return launch_router_bwd(*dims, logits, topk_idx, topk_gate, dg, counts_ext, (long long)t_total, alpha, beta, ds,
-                           dtok_null_bias, S(stream));
+                           dtok_null_bias, ws_ptr<uint16_t>(bwd_workspace, L.dsplit),
+                           ws_ptr<float>(bwd_workspace, L.bpart), S(stream));
 }
 
-int moe_router_weight_grad(const moe_dims_t* dims, const uint16_t* x, const float* ds, float* dw_router,
-                           float* dbias, void* bwd_workspace, moe_stream_t stream) {
+int moe_router_weight_grad(const moe_dims_t* dims, const uint16_t* x, float* dw_router, float* dbias,
+                           void* bwd_workspace, moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));
   if (!dw_router) return MOE_ERR_INVALID_ARG;
   const size_t rows = (size_t)router_rows(*dims);
@@ -87,10 +108,8 @@ int moe_router_weight_grad(const moe_dims_t* dims, const uint16_t* x, const floa
     MOE_CHECK(cuda_status(cudaMemsetAsync(dw_router, 0, sizeof(float) * rows * dims->d, S(stream))));
     return dbias ? cuda_status(cudaMemsetAsync(dbias, 0, sizeof(float) * rows, S(stream))) : MOE_OK;
   }
-  if (!x || !ds || !bwd_workspace) return MOE_ERR_INVALID_ARG;
-  const BwdLayout L = bwd_layout(*dims);
-  return launch_router_wgrad(*dims, ds, x, ws_ptr<float>(bwd_workspace, L.rpart), ws_ptr<float>(bwd_workspace, L.bpart),
-                             dw_router, dbias, S(stream));
+  if (!x || !bwd_workspace) return MOE_ERR_INVALID_ARG;
+  return router_wgrad(*dims, x, dw_router, dbias, bwd_workspace, S(stream));
 }
 
 int moe_expert_ffn_backward(const moe_dims_t* dims, const moe_weights_t* w, const moe_saved_t* saved,
@@ -106,18 +125,6 @@ int moe_expert_ffn_backward(const moe_dims_t* dims, const moe_weights_t* w, cons
 
 // The five GEMM stages of moe_expert_ffn_backward, one launch each (the weight gradients
 // add the reduction of the shared expert's K chunks when T needs more than one).
-int moe_expert_preact(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
-                      const uint16_t* gate_up, const uint16_t* shared_gate_up, void* bwd_workspace,
-                      moe_stream_t stream) {
-  MOE_CHECK(check_dims(dims));
-  if (dims->T == 0) return MOE_OK;
-  if (!xs || !x || !offsets || !gate_up || !shared_gate_up || !bwd_workspace) return MOE_ERR_INVALID_ARG;
-  const BwdLayout L = bwd_layout(*dims);
-  void* ws = bwd_workspace;
-  return launch_gate_up_preact(*dims, xs, x, offsets, gate_up, shared_gate_up, ws_ptr<uint16_t>(ws, L.z),
-                               ws_ptr<uint16_t>(ws, L.zs), ws_ptr<uint32_t>(ws, L.hdr), S(stream));
-}
-
 int moe_expert_dgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
                           const uint16_t* w_down, const uint16_t* shared_down, void* bwd_workspace,
                           moe_stream_t stream) {
@@ -126,9 +133,21 @@ int moe_expert_dgrad_down(const moe_dims_t* dims, const int32_t* offsets, const 
   if (!offsets || !dys || !dy || !w_down || !shared_down || !bwd_workspace) return MOE_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(*dims);
   void* ws = bwd_workspace;
-  return launch_dgrad_down_swiglu(*dims, offsets, dys, dy, w_down, shared_down, ws_ptr<uint16_t>(ws, L.z),
-                                  ws_ptr<uint16_t>(ws, L.zs), ws_ptr<uint16_t>(ws, L.dz), ws_ptr<uint16_t>(ws, L.dzs),
-                                  ws_ptr<uint32_t>(ws, L.hdr), S(stream));
+  return launch_dgrad_down(*dims, offsets, dys, dy, w_down, shared_down, ws_ptr<uint16_t>(ws, L.dh),
+                           ws_ptr<uint16_t>(ws, L.dhs), ws_ptr<uint32_t>(ws, L.hdr), S(stream));
+}
+
+int moe_expert_swiglu_backward(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                               const uint16_t* gate_up, const uint16_t* shared_gate_up, void* bwd_workspace,
+                               moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (dims->T == 0) return MOE_OK;
+  if (!xs || !x || !offsets || !gate_up || !shared_gate_up || !bwd_workspace) return MOE_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(*dims);
+  void* ws = bwd_workspace;
+  return launch_swiglu_backward(*dims, offsets, xs, x, gate_up, shared_gate_up, ws_ptr<uint16_t>(ws, L.dh),
+                                ws_ptr<uint16_t>(ws, L.dhs), ws_ptr<uint16_t>(ws, L.dz), ws_ptr<uint16_t>(ws, L.dzs),
+                                ws_ptr<uint32_t>(ws, L.hdr), S(stream));
 }
 
 int moe_expert_wgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
@@ -145,15 +164,22 @@ int moe_expert_wgrad_down(const moe_dims_t* dims, const int32_t* offsets, const 
 }
 
 int moe_expert_dgrad_gate_up(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* gate_up,
-                             const uint16_t* shared_gate_up, uint16_t* dxs, uint16_t* dx_shared, void* bwd_workspace,
-                             moe_stream_t stream) {
+                             const uint16_t* shared_gate_up, const float* w_router, uint16_t* dxs,
+                             uint16_t* dx_shared, void* bwd_workspace, moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));
   if (dims->T == 0) return MOE_OK;
   if (!offsets || !gate_up || !shared_gate_up || !dxs || !dx_shared || !bwd_workspace) return MOE_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(*dims);
   void* ws = bwd_workspace;
+  uint16_t* dsplit = nullptr;
+  uint16_t* w2 = nullptr;
+  if (w_router) {
+    dsplit = ws_ptr<uint16_t>(ws, L.dsplit);
+    w2 = ws_ptr<uint16_t>(ws, L.w2);
+    MOE_CHECK(launch_router_split2(*dims, w_router, w2, S(stream)));
+  }
   return launch_dgrad_gate_up(*dims, offsets, ws_ptr<uint16_t>(ws, L.dz), ws_ptr<uint16_t>(ws, L.dzs), gate_up,
-                              shared_gate_up, dxs, dx_shared, ws_ptr<uint32_t>(ws, L.hdr), S(stream));
+                              shared_gate_up, dsplit, w2, dxs, dx_shared, ws_ptr<uint32_t>(ws, L.hdr), S(stream));
 }
 
 int moe_expert_wgrad_gate_up(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* xs, const uint16_t* x,
@@ -171,14 +197,14 @@ int moe_expert_wgrad_gate_up(const moe_dims_t* dims, const int32_t* offsets, con
 }
 
 int moe_input_grad(const moe_dims_t* dims, const uint16_t* dx_shared, const uint16_t* dxs, const int32_t* slot_row,
-                   const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, const float* ds,
-                   const float* w_router, uint16_t* dx, void* bwd_workspace, moe_stream_t stream) {
+                   const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, uint16_t* dx,
+                   void* bwd_workspace, moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));
   if (dims->T == 0) return MOE_OK;
-  if (!dx_shared || !dxs || !slot_row || !ds || !w_router || !dx || !bwd_workspace) return MOE_ERR_INVALID_ARG;
+  if (!dx_shared || !dxs || !slot_row || !dx || !bwd_workspace) return MOE_ERR_INVALID_ARG;
   if (dims->C > 0 && (!topk_idx || !topk_gate || !dy)) return MOE_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(*dims);
-  return launch_input_grad(*dims, dx_shared, dxs, slot_row, topk_idx, topk_gate, dy, ds, w_router, dx,
+  return launch_input_grad(*dims, dx_shared, dxs, slot_row, topk_idx, topk_gate, dy, dx,
                            ws_ptr<uint32_t>(bwd_workspace, L.hdr), S(stream));
 }
 
@@ -206,12 +232,12 @@ int moe_backward(const moe_dims_t* dims, const moe_weights_t* w, const moe_saved
   MOE_CHECK(launch_combine_bwd(d, dy, saved->ys, saved->topk_gate, saved->slot_row, saved->topk_idx, saved->x,
                                w->const_vectors, dys, dg, status, st));
   MOE_CHECK(launch_router_bwd(d, saved->logits, saved->topk_idx, saved->topk_gate, dg, saved->counts_ext,
-                              (long long)saved->t_total, alpha, beta, ds, g->dtok_null_bias, st));
-  MOE_CHECK(launch_router_wgrad(d, ds, saved->x, ws_ptr<float>(ws, L.rpart), ws_ptr<float>(ws, L.bpart),
-                                g->dw_router, g->dbias, st));
+                              (long long)saved->t_total, alpha, beta, ds, g->dtok_null_bias,
+                              ws_ptr<uint16_t>(ws, L.dsplit), ws_ptr<float>(ws, L.bpart), st));
+  MOE_CHECK(router_wgrad(d, saved->x, g->dw_router, g->dbias, ws, st));
   MOE_CHECK(expert_ffn_bwd(d, w, saved, dys, dy, dxs, dxsh, g, ws, st));
-  MOE_CHECK(launch_input_grad(d, dxsh, dxs, saved->slot_row, saved->topk_idx, saved->topk_gate, dy, ds, w->w_router,
-                              g->dx, status, st));
+  MOE_CHECK(launch_input_grad(d, dxsh, dxs, saved->slot_row, saved->topk_idx, saved->topk_gate, dy, g->dx, status,
+                              st));
   return launch_const_grad(d, saved->topk_idx, saved->topk_gate, dy, g->dconst, st);
 }
 

@@ -18,6 +18,9 @@ constexpr int kCombineThreads = 256;
 // list is fetched while this one is combined. Sum order: shared, then slots in
 // rank order. A slot's source row is coded as: >= 0 a row of ys, -1 nothing
 // (null copy), -2 the token's row of x (copy expert), -3 - j constant vector j.
+// UNIT_ROWS (the backward's input gradient): rows of ys enter with weight 1, the gate
+// having been applied upstream; copy slots still take g times their row of x.
+template <bool UNIT_ROWS>
 __global__ void __launch_bounds__(kCombineThreads, 3)
 combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
                const float* __restrict__ gate, const int32_t* __restrict__ slot_row,
@@ -75,6 +78,7 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
           rq[u] = __shfl_sync(0xffffffffu, row, k & 31);
           gq[u] = __shfl_sync(0xffffffffu, g, k & 31);
           if (k >= K) rq[u] = -1;
+          if (UNIT_ROWS && rq[u] >= 0) gq[u] = 1.f;
           const uint16_t* srow = (rq[u] >= 0)    ? ys + (size_t)rq[u] * d
                                  : (rq[u] == -2) ? x + (size_t)t * d
                                  : (rq[u] <= -3) ? cv + (size_t)(-3 - rq[u]) * d
@@ -111,16 +115,15 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
   }
 }
 
-int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
-                   const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
-                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st) {
-  // one wave of resident CTAs; each warp then loops over tokens
+// one wave of resident CTAs; each warp then loops over tokens
+static int combine_grid(const moe_dims_t& d) {
   static int per_sm[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   int occ = (dev >= 0 && dev < 64) ? per_sm[dev] : 0;
   if (occ == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_kernel, kCombineThreads, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_kernel<false>, kCombineThreads, 0) !=
+            cudaSuccess ||
         occ < 1)
       occ = 1;
     if (dev >= 0 && dev < 64) per_sm[dev] = occ;
@@ -129,9 +132,28 @@ int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shar
   int grid = (d.T + wpb - 1) / wpb;
   const int cap = sm_count() * occ;
   if (grid > cap) grid = cap;
-  return launch_pdl(combine_kernel, dim3(grid), dim3(kCombineThreads), 0, st, ys, shared_out, topk_gate, slot_row,
-                    topk_idx, x, const_vectors, y, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, d.V,
-                    nullptr);
+  return grid < 1 ? 1 : grid;
+}
+
+int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
+                   const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st) {
+  const int grid = combine_grid(d);
+  return launch_pdl(combine_kernel<false>, dim3(grid), dim3(kCombineThreads), 0, st, ys, shared_out, topk_gate,
+                    slot_row, topk_idx, x, const_vectors, y, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C,
+                    d.V, nullptr);
+}
+
+// Input gradient of the backward pass: dx[t] = dx_shared[t] (the shared expert's and the
+// router's input gradient) + sum over the token's real slots of dxs[slot_row] + sum over
+// its copy-expert slots of g dy[t]; the same gather as the forward combine.
+int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint16_t* dxs, const int32_t* slot_row,
+                      const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, uint16_t* dx,
+                      uint32_t* status, cudaStream_t st) {
+  const int grid = combine_grid(d);
+  return launch_pdl(combine_kernel<true>, dim3(grid), dim3(kCombineThreads), 0, st, dxs, dx_shared, topk_gate,
+                    slot_row, topk_idx, dy, (const uint16_t*)nullptr, dx, d.T, d.d, d.K, (long long)d.T * d.K,
+                    d.N + d.M, d.C, 0, status);
 }
 
 }  // namespace moe

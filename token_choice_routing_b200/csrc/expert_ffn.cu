@@ -587,40 +587,6 @@ int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, 
                         : launch_gemm<128, false, false>(ar, br, as_, bs, p.g2, p.max2, st);
 }
 
-// Gate/up pre-activations without the SwiGLU epilogue: z = [A W_g^T | A W_u^T] in the packed
-// column order (64 gate columns, then the matching 64 up columns). The backward pass
-// recomputes them for the SwiGLU derivative.
-int launch_gate_up_preact(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
-                          const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* z, uint16_t* zs,
-                          uint32_t* status, cudaStream_t st) {
-  const long long rcap = (long long)d.T * d.K;
-  const int BN = (d.F % 128 == 0 && d.F_shared % 128 == 0) ? 256 : 128;
-  GemmArgs g{};
-  g.offsets = offsets;
-  g.N = d.N;
-  g.T = d.T;
-  g.kb_r = g.kb_s = d.d / kBK;
-  g.nt_r = 2 * d.F / BN;
-  g.nt_s = 2 * d.F_shared / BN;
-  g.brows_r = 2 * d.F;
-  g.rows_cap = rcap;
-  g.out_r = z;
-  g.ld_r = 2 * d.F;
-  g.out_s = zs;
-  g.ld_s = 2 * d.F_shared;
-  g.status = status;
-  g.limit_ns = kWaitLimitNs;
-  g.has_shared = 1;
-  const long long max_tiles = (rcap / kBM + d.N) * g.nt_r + (long long)((d.T + kBM - 1) / kBM) * g.nt_s;
-  CUtensorMap ar, br, as_, bs;
-  if (!(make_tmap_bf16(&ar, xs, rcap, d.d, kBM) && make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, BN) &&
-        make_tmap_bf16(&as_, x, d.T, d.d, kBM) &&
-        make_tmap_bf16(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, BN)))
-    return MOE_ERR_CUDA;
-  return (BN == 256) ? launch_gemm<256, false, false>(ar, br, as_, bs, g, max_tiles, st)
-                     : launch_gemm<128, false, false>(ar, br, as_, bs, g, max_tiles, st);
-}
-
 int launch_expert_ffn(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
                       const uint16_t* gate_up, const uint16_t* w_down, const uint16_t* sgate_up,
                       const uint16_t* sdown, uint16_t* h, uint16_t* h_shared, uint16_t* ys,

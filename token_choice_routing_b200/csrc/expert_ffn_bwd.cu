@@ -14,9 +14,12 @@
 // so, as in the forward, nothing is computed for null slots.
 //
 // One kernel template serves the three GEMM shapes:
-//   kDgradPlain / kDgradSwiglu: C[row, n] = sum_k A[row, k] B[k, n]. A (activation rows,
-//     K contiguous) is K-major; B is the weight in its natural layout [K, n] (n contiguous)
-//     and is read MN-major: 64 x 64 TMA boxes, one per 64 output columns.
+//   kDgradPlain: C[row, n] = sum_k A[row, k] B[k, n]. A (activation rows, K contiguous) is
+//     K-major; B is the weight in its natural layout [K, n] (n contiguous) and is read
+//     MN-major: 64 x 64 TMA boxes, one per 64 output columns.
+//   kPreactSwiglu: the forward's gate/up product z = A W_gu^T (both K-major) recomputed
+//     into TMEM in fp32; its epilogue reads the matching tile of dh (TMA) and writes the
+//     SwiGLU derivative dz = [da | db] in the packed column order, with 8 epilogue warps.
 //   kWgrad: C[m, n] = sum_r A[r, m] B[r, n] over the rows r of one expert: both operands are
 //     activation rows read MN-major. The last k-block of an expert reads rows of the next
 //     expert (or unwritten rows); those rows are zeroed in shared memory before the MMA.
@@ -36,11 +39,17 @@ namespace bwd {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;  // producer, MMA, 4 epilogue warps (8 for kPreactSwiglu)
 constexpr int kStgRow = 64 * 2 + 16;
 constexpr int kBox = 64 * 64 * 2;  // one 64 x 64 bf16 box (8 KB)
 
-enum Mode { kDgradPlain = 0, kDgradSwiglu = 1, kWgrad = 2 };
+enum Mode { kDgradPlain = 0, kPreactSwiglu = 1, kWgrad = 2 };
+
+template <int MODE>
+struct Threads {
+  static constexpr int epi = (MODE == kPreactSwiglu) ? 256 : 128;  // epilogue threads
+  static constexpr int total = 64 + epi;
+};
 
 struct Args {
   const int32_t* offsets;  // [N+1]
@@ -58,6 +67,8 @@ struct Args {
   uint16_t* out_r2;        // wgrad of packed gate/up: destination of the up rows (else null)
   uint16_t* out_s2;
   float* part_s;           // wgrad, nsplit > 1: fp32 partials [nsplit, Mout_s, ld_s]
+  int part_only;           // wgrad: the shared group always writes fp32 partials
+  int kb_x, xrp;           // dgrad: extra k-blocks of the shared group (router term), term width
   uint32_t* status;
   unsigned long long limit_ns;
   int has_shared;
@@ -67,8 +78,8 @@ template <int BN, int MODE>
 struct Smem {
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN * kBK * 2;
-  static constexpr int Z_BYTES = (MODE == kDgradSwiglu) ? kBM * 2 * BN * 2 : 0;
-  static constexpr int STG_BYTES = (MODE == kDgradSwiglu) ? 0 : kBM * kStgRow;
+  static constexpr int Z_BYTES = (MODE == kPreactSwiglu) ? kBM * BN : 0;  // dh tile: 128 x BN/2 bf16
+  static constexpr int STG_BYTES = (MODE == kPreactSwiglu) ? 0 : kBM * kStgRow;
   static constexpr size_t off_a = 0;
   static constexpr size_t off_b = off_a + (size_t)kStages * A_BYTES;
   static constexpr size_t off_z = off_b + (size_t)kStages * B_BYTES;
@@ -79,6 +90,7 @@ struct Smem {
   static constexpr size_t off_tab = off_misc + 16;
   static constexpr size_t end = off_tab + sizeof(int) * 3 * (kMaxN + 2);
   static constexpr size_t bytes = end + 1024;
+  static_assert(bytes <= 232448, "shared memory per CTA");
 };
 
 struct Tile {
@@ -104,7 +116,7 @@ __host__ __device__ constexpr uint32_t idesc_t(int M, int N, bool a_mn, bool b_m
 }
 
 template <int BN, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Threads<MODE>::total, 1)
 bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
                 const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s,
                 const __grid_constant__ CUtensorMap tmZ_r, const __grid_constant__ CUtensorMap tmZ_s,
@@ -112,8 +124,10 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
   pdl_wait_then_release();
   using SM = Smem<BN, MODE>;
   constexpr bool WG = (MODE == kWgrad);
+  constexpr bool PRE = (MODE == kPreactSwiglu);
+  constexpr int EPI = Threads<MODE>::epi;
   constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-  constexpr uint32_t IDESC = idesc_t(kBM, BN, WG, true);
+  constexpr uint32_t IDESC = idesc_t(kBM, BN, WG, !PRE);
   constexpr uint32_t TX_BYTES = SM::A_BYTES + SM::B_BYTES;
   constexpr int NBOX_B = BN / 64;
 
@@ -153,7 +167,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(tfull_bar(s), 1);
-      mbar_init(tempty_bar(s), 128);
+      mbar_init(tempty_bar(s), EPI);
     }
     mbar_init(drain_bar, 1);
     mbar_init(z_bar, 1);
@@ -248,7 +262,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
       ti.mvalid = min(kBM, s_m[lo] - mt * kBM);
       ti.krows = 0;
       ti.chunk = 0;
-      ti.nkb = (lo < N) ? a.kb_r : a.kb_s;
+      ti.nkb = (lo < N) ? a.kb_r : a.kb_s + a.kb_x;
       ti.brow = (lo < N) ? lo * a.kdim_r : 0;
     }
     return ti;
@@ -280,6 +294,21 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
 #pragma unroll
             for (int j = 0; j < NBOX_B; ++j)
               tma_load_2d(dB + j * kBox, tb, full_bar(stage), ti.nt * BN + 64 * j, kr);
+          } else if (PRE) {
+            // K-major A and B (the packed gate/up rows of this n-tile), as in the forward
+            tma_load_2d(dA, ta, full_bar(stage), kb * kBK, ti.row0);
+            tma_load_2d(dB, tb, full_bar(stage), kb * kBK, ti.brow + ti.nt * BN);
+          } else if (ti.g == N && kb >= a.kb_s) {
+            // router term of the shared group: ds W_r = ds_hi W_hi + ds_hi W_lo + ds_lo W_hi, the
+            // two-term splits read from the maps in the pre-activation slots
+            const int e = kb - a.kb_s;
+            const int njb = a.xrp / kBK;
+            const int p = e / njb, jb = e - p * njb;
+            const int at = (p == 2) ? 1 : 0, bt = (p == 1) ? 1 : 0;
+            tma_load_2d(dA, &tmZ_r, full_bar(stage), at * a.xrp + jb * kBK, ti.row0);
+#pragma unroll
+            for (int j = 0; j < NBOX_B; ++j)
+              tma_load_2d(dB + j * kBox, &tmZ_s, full_bar(stage), ti.nt * BN + 64 * j, bt * a.xrp + jb * kBK);
           } else {
             tma_load_2d(dA, ta, full_bar(stage), kb * kBK, ti.row0);
 #pragma unroll
@@ -357,7 +386,10 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
               // K-major A: +32 bytes along K inside the 128-byte swizzle atom
               adesc = smem_desc_sw128(aS) + (uint64_t)(2 * k);
             }
-            bdesc = desc_mn_sw128(bS + (uint32_t)(k * 2048), kBox);
+            if constexpr (PRE)
+              bdesc = smem_desc_sw128(bS) + (uint64_t)(2 * k);
+            else
+              bdesc = desc_mn_sw128(bS + (uint32_t)(k * 2048), kBox);
             tc_mma_f16(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
           }
           tc_commit(empty_bar(stage));
@@ -378,22 +410,25 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
     }
     __syncwarp();
   } else {
-    // ------------------------------ epilogue warpgroup (warps 2..5)
-    const int q = warp & 3;
+    // ------------------------------ epilogue warps (2..5, or 2..9 for kPreactSwiglu)
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
     const int etid = (warp - 2) * 32 + lane;
+    const int ehalf = (warp - 2) >> 2;   // kPreactSwiglu: which half of the tile's columns
     int li = 0;
-    int z_inflight = -1;  // (etid 0) tile counter of a pre-activation load not yet waited for
-    if constexpr (MODE == kDgradSwiglu) {
-      // the first tile's pre-activations
+    int z_inflight = -1;  // (etid 0) tile counter of a dh-tile load not yet waited for
+    // dh tile of a tile: rows row0.., dh columns [nt BN/2, (nt+1) BN/2) in 64-column boxes
+    auto load_dh = [&](const Tile& t, uint32_t bar) {
+      const void* tz = (t.g < N) ? (const void*)&tmZ_r : (const void*)&tmZ_s;
+      mbar_arrive_expect_tx(bar, SM::Z_BYTES);
+#pragma unroll
+      for (int b = 0; b < BN / 128; ++b)
+        tma_load_2d(smem_u32(sZ + b * (kBM * 128)), tz, bar, t.nt * (BN / 2) + 64 * b, t.row0);
+    };
+    if constexpr (PRE) {
       if (etid == 0 && (int)blockIdx.x < total) {
         z_inflight = 0;
-        const Tile t0 = decode(blockIdx.x);
-        const void* tz = (t0.g < N) ? (const void*)&tmZ_r : (const void*)&tmZ_s;
-        mbar_arrive_expect_tx(z_bar, SM::Z_BYTES);
-#pragma unroll
-        for (int b = 0; b < 2 * BN / 64; ++b)
-          tma_load_2d(smem_u32(sZ + b * (kBM * 128)), tz, z_bar, 2 * t0.nt * BN + 64 * b, t0.row0);
+        load_dh(decode(blockIdx.x), z_bar);
       }
     }
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++li) {
@@ -403,76 +438,66 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
       if (!mbar_wait_bounded(tfull_bar(acc), ap, a.limit_ns, abort_flag, a.status)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if constexpr (MODE == kDgradSwiglu) {
+      if constexpr (PRE) {
         if (!mbar_wait_bounded(z_bar, (uint32_t)li & 1u, a.limit_ns, abort_flag, a.status)) break;
         z_inflight = -1;
-        // dh (TMEM) and the pre-activations a (gate) and b (up) of this row -> da, db in place
+        // z (fp32, TMEM: 64 gate then 64 up columns per panel) and dh (smem) of this row ->
+        // da = dh b sigma (1 + a (1 - sigma)), db = dh a sigma, stored as bf16 straight to dz
+        uint16_t* out = (ti.g < N) ? a.out_r : a.out_s;
+        const int ld = (ti.g < N) ? a.ld_r : a.ld_s;
+        const bool live = row < ti.mvalid;
+        uint16_t* orow = out + (size_t)(ti.row0 + row) * ld + ti.nt * BN;
 #pragma unroll 1
-        for (int g16 = 0; g16 < BN / 16; ++g16) {
-          uint32_t r[16];
-          tmem_ld16(tb + (uint32_t)(g16 * 16), r);
+        for (int g = 0; g < BN / 64; ++g) {
+          const int f0 = ehalf * (BN / 4) + g * 16;  // first of 16 dh columns in the tile
+          const int p = f0 >> 6, within = f0 & 63;
+          uint32_t zg[16], zu[16];
+          tmem_ld16(tb + (uint32_t)(p * 128 + within), zg);
+          tmem_ld16(tb + (uint32_t)(p * 128 + 64 + within), zu);
           tmem_ld_wait();
-          const int lp = g16 >> 2;  // 64-column panel of the tile
+          uint32_t og[8], ou[8];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const int ch = ((g16 & 3) << 1) + half;
-            unsigned char* pg = sZ + (2 * lp) * (kBM * 128) + row * 128 + ((ch ^ (row & 7)) << 4);
-            unsigned char* pu = pg + kBM * 128;
-            uint4 zg = *reinterpret_cast<const uint4*>(pg);
-            uint4 zu = *reinterpret_cast<const uint4*>(pu);
-            uint32_t* wg = reinterpret_cast<uint32_t*>(&zg);
-            uint32_t* wu = reinterpret_cast<uint32_t*>(&zu);
+            const int ch = (within >> 3) + half;
+            const uint4 hv = *reinterpret_cast<const uint4*>(sZ + p * (kBM * 128) + row * 128 + ((ch ^ (row & 7)) << 4));
+            const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               float dav[2], dbv[2];
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                const float av = h ? bf16hi(wg[j]) : bf16lo(wg[j]);
-                const float bv = h ? bf16hi(wu[j]) : bf16lo(wu[j]);
-                const float dh = __uint_as_float(r[half * 8 + 2 * j + h]);
+                const int c = half * 8 + 2 * j + h;
+                const float av = __uint_as_float(zg[c]);
+                const float bv = __uint_as_float(zu[c]);
+                const float dh = h ? bf16hi(hw[j]) : bf16lo(hw[j]);
                 const float sg = __fdividef(1.f, 1.f + __expf(-av));
                 dbv[h] = dh * av * sg;
                 dav[h] = dh * bv * sg * (1.f + av * (1.f - sg));
               }
-              wg[j] = pack_bf16x2(dav[0], dav[1]);
-              wu[j] = pack_bf16x2(dbv[0], dbv[1]);
+              og[half * 4 + j] = pack_bf16x2(dav[0], dav[1]);
+              ou[half * 4 + j] = pack_bf16x2(dbv[0], dbv[1]);
             }
-            *reinterpret_cast<uint4*>(pg) = zg;
-            *reinterpret_cast<uint4*>(pu) = zu;
+          }
+          if (live) {
+            uint4* dg4 = reinterpret_cast<uint4*>(orow + p * 128 + within);
+            uint4* du4 = reinterpret_cast<uint4*>(orow + p * 128 + 64 + within);
+            dg4[0] = make_uint4(og[0], og[1], og[2], og[3]);
+            dg4[1] = make_uint4(og[4], og[5], og[6], og[7]);
+            du4[0] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+            du4[1] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
           }
         }
         tc_fence_before();
         mbar_arrive(tempty_bar(acc));
-        named_bar_sync(1, 128);
-        // coalesced copy-out of the 128 x 2BN tile (rows past the expert's end are skipped)
-        uint16_t* out = (ti.g < N) ? a.out_r : a.out_s;
-        const int ld = (ti.g < N) ? a.ld_r : a.ld_s;
-        constexpr int CPR = 2 * BN / 8;  // 16-byte chunks per row
-#pragma unroll 4
-        for (int it = 0; it < kBM * CPR / 128; ++it) {
-          const int idx = it * 128 + etid;
-          const int r = idx / CPR, cc = idx % CPR;
-          const int box = cc >> 3, ch = cc & 7;
-          if (r < ti.mvalid) {
-            const uint4 v = *reinterpret_cast<const uint4*>(sZ + box * (kBM * 128) + r * 128 + ((ch ^ (r & 7)) << 4));
-            *reinterpret_cast<uint4*>(out + (size_t)(ti.row0 + r) * ld + 2 * ti.nt * BN + cc * 8) = v;
-          }
-        }
-        fence_proxy_async_shared();  // generic accesses to the z buffer before the next TMA write
-        named_bar_sync(1, 128);
-        // the next tile's pre-activations
+        fence_proxy_async_shared();  // generic reads of the dh tile before the next TMA write
+        named_bar_sync(1, EPI);
         if (etid == 0 && tile + (int)gridDim.x < total) {
           z_inflight = li + 1;
-          const Tile tn = decode(tile + gridDim.x);
-          const void* tz = (tn.g < N) ? (const void*)&tmZ_r : (const void*)&tmZ_s;
-          mbar_arrive_expect_tx(z_bar, SM::Z_BYTES);
-#pragma unroll
-          for (int b = 0; b < 2 * BN / 64; ++b)
-            tma_load_2d(smem_u32(sZ + b * (kBM * 128)), tz, z_bar, 2 * tn.nt * BN + 64 * b, tn.row0);
+          load_dh(decode(tile + gridDim.x), z_bar);
         }
       } else {
         // plain bf16 output (dgrad) or weight gradient (wgrad), staged 64 columns at a time
-        const bool partial = WG && ti.g == N && a.nsplit > 1;
+        const bool partial = WG && ti.g == N && (a.nsplit > 1 || a.part_only);
         const bool empty = WG && ti.nkb == 0;
         uint16_t* out;
         int ld;
@@ -547,7 +572,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
               tc_fence_before();
               mbar_arrive(tempty_bar(acc));
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, EPI);
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
               const int idx = it * 128 + etid;
@@ -562,7 +587,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
                 if (r < ti.mvalid) *reinterpret_cast<uint4*>(out + (size_t)(ti.row0 + r) * ld + col) = v;
               }
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, EPI);
           }
         }
       }
@@ -628,7 +653,7 @@ static int launch(const CUtensorMap& ar, const CUtensorMap& br, const CUtensorMa
   long long grid = sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(bwd_gemm_kernel<BN, MODE>, dim3((unsigned)grid), dim3(kThreads), SM::bytes, st, ar, br, as_, bs,
+  return launch_pdl(bwd_gemm_kernel<BN, MODE>, dim3((unsigned)grid), dim3(Threads<MODE>::total), SM::bytes, st, ar, br, as_, bs,
                     zr, zs, a);
 }
 
@@ -679,33 +704,70 @@ size_t bwd_split_partial_floats(const moe_dims_t& d) {
   return (size_t)ns * (a > b ? a : b);
 }
 
-int launch_dgrad_down_swiglu(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
-                             const uint16_t* w_down, const uint16_t* sdown, const uint16_t* z, const uint16_t* zs,
-                             uint16_t* dz, uint16_t* dzs, uint32_t* status, cudaStream_t st) {
+static int dgrad_bn(int a, int b) {
+  for (int bn = 256; bn >= 64; bn >>= 1)
+    if (a % bn == 0 && b % bn == 0) return bn;
+  return 0;
+}
+
+// dh = dys W_d (routed rows) and dh_shared = dy W_sd (all T rows).
+int launch_dgrad_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
+                      const uint16_t* w_down, const uint16_t* sdown, uint16_t* dh, uint16_t* dh_shared,
+                      uint32_t* status, cudaStream_t st) {
   const long long rcap = (long long)d.T * d.K;
-  const int BN = (d.F % 128 == 0 && d.F_shared % 128 == 0) ? 128 : 64;
+  const int BN = dgrad_bn(d.F, d.F_shared);
+  if (BN == 0) return MOE_ERR_UNSUPPORTED;
   Args a = base_args(d, offsets, status);
   a.kb_r = a.kb_s = d.d / kBK;
   a.nt_r = d.F / BN;
   a.nt_s = d.F_shared / BN;
   a.kdim_r = d.d;
+  a.out_r = dh;
+  a.ld_r = d.F;
+  a.out_s = dh_shared;
+  a.ld_s = d.F_shared;
+  CUtensorMap ar, br, as_, bs;
+  if (!(make_tmap_bf16(&ar, dys, rcap, d.d, kBM) && make_tmap_bf16(&br, w_down, (uint64_t)d.N * d.d, d.F, 64) &&
+        make_tmap_bf16(&as_, dy, d.T, d.d, kBM) && make_tmap_bf16(&bs, sdown, d.d, d.F_shared, 64)))
+    return MOE_ERR_CUDA;
+  const long long mt = dgrad_max_tiles(d, a.nt_r, a.nt_s);
+  switch (BN) {
+    case 256: return launch<256, kDgradPlain>(ar, br, as_, bs, ar, ar, a, mt, st);
+    case 128: return launch<128, kDgradPlain>(ar, br, as_, bs, ar, ar, a, mt, st);
+    default: return launch<64, kDgradPlain>(ar, br, as_, bs, ar, ar, a, mt, st);
+  }
+}
+
+// The gate/up pre-activations z recomputed in TMEM (fp32) and, in the epilogue, the SwiGLU
+// derivative dz = [da | db] (packed column order) from z and dh.
+int launch_swiglu_backward(const moe_dims_t& d, const int32_t* offsets, const uint16_t* xs, const uint16_t* x,
+                           const uint16_t* gate_up, const uint16_t* sgate_up, const uint16_t* dh,
+                           const uint16_t* dh_shared, uint16_t* dz, uint16_t* dzs, uint32_t* status,
+                           cudaStream_t st) {
+  const long long rcap = (long long)d.T * d.K;
+  const int BN = (d.F % 128 == 0 && d.F_shared % 128 == 0) ? 256 : 128;
+  Args a = base_args(d, offsets, status);
+  a.kb_r = a.kb_s = d.d / kBK;
+  a.nt_r = 2 * d.F / BN;
+  a.nt_s = 2 * d.F_shared / BN;
+  a.kdim_r = 2 * d.F;
   a.out_r = dz;
   a.ld_r = 2 * d.F;
   a.out_s = dzs;
   a.ld_s = 2 * d.F_shared;
-  CUtensorMap ar, br, as_, bs, zr, zsm;
-  if (!(make_tmap_bf16(&ar, dys, rcap, d.d, kBM) && make_tmap_bf16(&br, w_down, (uint64_t)d.N * d.d, d.F, 64) &&
-        make_tmap_bf16(&as_, dy, d.T, d.d, kBM) && make_tmap_bf16(&bs, sdown, d.d, d.F_shared, 64) &&
-        make_tmap_bf16(&zr, z, rcap, 2 * d.F, kBM) && make_tmap_bf16(&zsm, zs, d.T, 2 * d.F_shared, kBM)))
+  CUtensorMap ar, br, as_, bs, hr, hs;
+  if (!(make_tmap_bf16(&ar, xs, rcap, d.d, kBM) && make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, BN) &&
+        make_tmap_bf16(&as_, x, d.T, d.d, kBM) && make_tmap_bf16(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, BN) &&
+        make_tmap_bf16(&hr, dh, rcap, d.F, kBM) && make_tmap_bf16(&hs, dh_shared, d.T, d.F_shared, kBM)))
     return MOE_ERR_CUDA;
   const long long mt = dgrad_max_tiles(d, a.nt_r, a.nt_s);
-  return BN == 128 ? launch<128, kDgradSwiglu>(ar, br, as_, bs, zr, zsm, a, mt, st)
-                   : launch<64, kDgradSwiglu>(ar, br, as_, bs, zr, zsm, a, mt, st);
+  return BN == 256 ? launch<256, kPreactSwiglu>(ar, br, as_, bs, hr, hs, a, mt, st)
+                   : launch<128, kPreactSwiglu>(ar, br, as_, bs, hr, hs, a, mt, st);
 }
 
 int launch_dgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dz, const uint16_t* dzs,
-                         const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* dxs, uint16_t* dx_shared,
-                         uint32_t* status, cudaStream_t st) {
+                         const uint16_t* gate_up, const uint16_t* sgate_up, const uint16_t* dsplit,
+                         const uint16_t* w2, uint16_t* dxs, uint16_t* dx_shared, uint32_t* status, cudaStream_t st) {
   const long long rcap = (long long)d.T * d.K;
   const int BN = (d.d % 256 == 0) ? 256 : 128;
   Args a = base_args(d, offsets, status);
@@ -717,15 +779,24 @@ int launch_dgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint
   a.ld_r = d.d;
   a.out_s = dx_shared;
   a.ld_s = d.d;
-  CUtensorMap ar, br, as_, bs;
+  CUtensorMap ar, br, as_, bs, xr, xw;
   if (!(make_tmap_bf16(&ar, dz, rcap, 2 * d.F, kBM) &&
         make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, 64) &&
         make_tmap_bf16(&as_, dzs, d.T, 2 * d.F_shared, kBM) &&
         make_tmap_bf16(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, 64)))
     return MOE_ERR_CUDA;
+  xr = ar;
+  xw = ar;
+  if (dsplit && w2) {
+    const int rp = router_split_rows(d);
+    a.xrp = rp;
+    a.kb_x = 3 * (rp / kBK);  // (hi, hi), (hi, lo), (lo, hi) over RP/64 k-blocks each
+    if (!(make_tmap_bf16(&xr, dsplit, d.T, 2 * rp, kBM) && make_tmap_bf16(&xw, w2, (uint64_t)2 * rp, d.d, 64)))
+      return MOE_ERR_CUDA;
+  }
   const long long mt = dgrad_max_tiles(d, a.nt_r, a.nt_s);
-  return BN == 256 ? launch<256, kDgradPlain>(ar, br, as_, bs, ar, ar, a, mt, st)
-                   : launch<128, kDgradPlain>(ar, br, as_, bs, ar, ar, a, mt, st);
+  return BN == 256 ? launch<256, kDgradPlain>(ar, br, as_, bs, xr, xw, a, mt, st)
+                   : launch<128, kDgradPlain>(ar, br, as_, bs, xr, xw, a, mt, st);
 }
 
 static int launch_wgrad(const moe_dims_t& d, const Args& a0, int BN, const CUtensorMap& ar, const CUtensorMap& br,
@@ -794,6 +865,42 @@ int launch_wgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint
         make_tmap_bf16(&as_, dzs, d.T, 2 * d.F_shared, 64) && make_tmap_bf16(&bs, x, d.T, d.d, 64)))
     return MOE_ERR_CUDA;
   return launch_wgrad(d, a, BN, ar, br, as_, bs, 2 * d.F_shared, dws_gate, dws_up, st);
+}
+
+// K chunks of the router weight gradient dsplit^T x: at least 4 k-blocks each, at most 32
+// chunks.
+int router_wgrad_split(const moe_dims_t& d, int* chunk_kb) {
+  const int kb = (d.T + kBK - 1) / kBK;
+  int ck = 4;
+  if ((kb + ck - 1) / ck > 32) ck = (kb + 31) / 32;
+  if (chunk_kb) *chunk_kb = ck;
+  const int n = (kb + ck - 1) / ck;
+  return n < 1 ? 1 : n;
+}
+
+// Router weight gradient on the tensor cores: fp32 partials of dsplit^T x per K chunk
+// ([chunks, 2 RP, d]: hi-term rows, then lo-term rows), reduced by
+// launch_router_wgrad_reduce. The weight-gradient kernel runs with no routed group.
+int launch_router_wgrad_tc(const moe_dims_t& d, const uint16_t* dsplit, const uint16_t* x, float* part,
+                           uint32_t* status, cudaStream_t st) {
+  const int rp = router_split_rows(d);
+  const int BN = (d.d % 256 == 0) ? 256 : 128;
+  moe_dims_t d0 = d;
+  d0.N = 0;
+  Args a = base_args(d0, nullptr, status);
+  a.mt_r = a.nt_r = 0;
+  a.mt_s = 2 * rp / kBM;
+  a.nt_s = d.d / BN;
+  a.nsplit = router_wgrad_split(d, &a.chunk_kb);
+  a.part_only = 1;
+  a.part_s = part;
+  a.ld_s = d.d;
+  a.rows_cap = d.T;
+  CUtensorMap as_, bs;
+  if (!(make_tmap_bf16(&as_, dsplit, d.T, 2 * rp, 64) && make_tmap_bf16(&bs, x, d.T, d.d, 64))) return MOE_ERR_CUDA;
+  const long long tiles = (long long)a.nsplit * a.mt_s * a.nt_s;
+  return BN == 256 ? launch<256, kWgrad>(as_, bs, as_, bs, as_, as_, a, tiles, st)
+                   : launch<128, kWgrad>(as_, bs, as_, bs, as_, as_, a, tiles, st);
 }
 
 }  // namespace moe

@@ -114,23 +114,29 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
 }
 
 // Backward-pass workspace (moe_backward_workspace_bytes). R_cap = T*K rows.
-int router_wgrad_chunks(const moe_dims_t& d, int* chunk_tokens);
 int bwd_shared_split(const moe_dims_t& d, int* chunk_kb);
 size_t bwd_split_partial_floats(const moe_dims_t& d);
+int router_wgrad_split(const moe_dims_t& d, int* chunk_kb);
+int router_bwd_grid(const moe_dims_t& d);
+// Router rows padded to a multiple of 64: the width of each bf16 term of the split logit
+// gradients and router weights that the backward's tensor-core products read.
+inline int router_split_rows(const moe_dims_t& d) { return (router_rows(d) + 63) / 64 * 64; }
 
 struct BwdLayout {
   size_t hdr;    // uint32 status at 0 (256 B)
-  size_t z;      // bf16 [R_cap, 2F] gate/up pre-activations (packed column order)
-  size_t zs;     // bf16 [T, 2F_shared]
-  size_t dz;     // bf16 [R_cap, 2F] their gradients
+  size_t dh;     // bf16 [R_cap, F] gradient of the routed SwiGLU activations
+  size_t dhs;    // bf16 [T, F_shared] the shared expert's
+  size_t dz;     // bf16 [R_cap, 2F] gradients of the gate/up pre-activations (packed order)
   size_t dzs;    // bf16 [T, 2F_shared]
   size_t dys;    // bf16 [R_cap, d] upstream gradient of each routed row: g * dy
   size_t dxs;    // bf16 [R_cap, d] input gradient of each routed row
   size_t dxsh;   // bf16 [T, d] input gradient through the shared expert
   size_t dg;     // fp32 [T, K] gate gradients
   size_t ds;     // fp32 [T, N+1+C+V] logit gradients
-  size_t rpart;  // fp32 [chunks, rows, d] router weight-gradient partials
-  size_t bpart;  // fp32 [chunks, rows] router bias-gradient partials
+  size_t dsplit; // bf16 [T, 2 RP] logit gradients as two terms (hi | lo), RP = router_split_rows
+  size_t w2;     // bf16 [2 RP, d] router weights as two terms (hi rows, then lo rows)
+  size_t rpart;  // fp32 [chunks, 2 RP, d] partials of dsplit^T x
+  size_t bpart;  // fp32 [router_bwd CTAs, rows] column sums of ds
   size_t spart;  // fp32 shared-expert weight-gradient K-chunk partials
   size_t total;
 };
@@ -139,11 +145,12 @@ inline BwdLayout bwd_layout(const moe_dims_t& d) {
   BwdLayout L{};
   const size_t rcap = (size_t)d.T * d.K, T = (size_t)d.T;
   const size_t rows = (size_t)router_rows(d);
-  const int nch = router_wgrad_chunks(d, nullptr);
+  const int nch = router_wgrad_split(d, nullptr);
+  const size_t rp = (size_t)router_split_rows(d);
   size_t o = 0;
   L.hdr = o; o += 256;
-  L.z = o; o = align_up(o + 2 * rcap * 2 * d.F, 256);
-  L.zs = o; o = align_up(o + 2 * T * 2 * d.F_shared, 256);
+  L.dh = o; o = align_up(o + 2 * rcap * d.F, 256);
+  L.dhs = o; o = align_up(o + 2 * T * d.F_shared, 256);
   L.dz = o; o = align_up(o + 2 * rcap * 2 * d.F, 256);
   L.dzs = o; o = align_up(o + 2 * T * 2 * d.F_shared, 256);
   L.dys = o; o = align_up(o + 2 * rcap * d.d, 256);
@@ -151,8 +158,10 @@ inline BwdLayout bwd_layout(const moe_dims_t& d) {
   L.dxsh = o; o = align_up(o + 2 * T * d.d, 256);
   L.dg = o; o = align_up(o + 4 * T * d.K, 256);
   L.ds = o; o = align_up(o + 4 * T * rows, 256);
-  L.rpart = o; o = align_up(o + 4 * (size_t)nch * rows * d.d, 256);
-  L.bpart = o; o = align_up(o + 4 * (size_t)nch * rows, 256);
+  L.dsplit = o; o = align_up(o + 2 * T * 2 * rp, 256);
+  L.w2 = o; o = align_up(o + 2 * 2 * rp * d.d, 256);
+  L.rpart = o; o = align_up(o + 4 * (size_t)nch * 2 * rp * d.d, 256);
+  L.bpart = o; o = align_up(o + 4 * (size_t)router_bwd_grid(d) * rows, 256);
   L.spart = o; o = align_up(o + 4 * bwd_split_partial_floats(d), 256);
   L.total = o;
   return L;
@@ -248,32 +257,39 @@ int launch_pack_gate_up(const moe_dims_t& d, const uint16_t* w_gate, const uint1
 int launch_selftest_wait(void* ws, unsigned long long limit_ns, cudaStream_t st);
 
 // Backward pass (backward.cu, expert_ffn_bwd.cu, expert_ffn.cu).
-int launch_gate_up_preact(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
-                          const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* z, uint16_t* zs,
-                          uint32_t* status, cudaStream_t st);
-int launch_dgrad_down_swiglu(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
-                             const uint16_t* w_down, const uint16_t* sdown, const uint16_t* z, const uint16_t* zs,
-                             uint16_t* dz, uint16_t* dzs, uint32_t* status, cudaStream_t st);
+int launch_dgrad_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
+                      const uint16_t* w_down, const uint16_t* sdown, uint16_t* dh, uint16_t* dh_shared,
+                      uint32_t* status, cudaStream_t st);
+int launch_swiglu_backward(const moe_dims_t& d, const int32_t* offsets, const uint16_t* xs, const uint16_t* x,
+                           const uint16_t* gate_up, const uint16_t* sgate_up, const uint16_t* dh,
+                           const uint16_t* dh_shared, uint16_t* dz, uint16_t* dzs, uint32_t* status,
+                           cudaStream_t st);
+// dsplit/w2 (optional, both or neither): the router's input gradient ds W_r is added to
+// dx_shared as extra k-blocks of the shared expert's tiles
 int launch_dgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dz, const uint16_t* dzs,
-                         const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* dxs, uint16_t* dx_shared,
-                         uint32_t* status, cudaStream_t st);
+                         const uint16_t* gate_up, const uint16_t* sgate_up, const uint16_t* dsplit,
+                         const uint16_t* w2, uint16_t* dxs, uint16_t* dx_shared, uint32_t* status, cudaStream_t st);
 int launch_wgrad_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,
                       const uint16_t* h, const uint16_t* h_shared, uint16_t* dw_down, uint16_t* dws_down,
                       float* partials, uint32_t* status, cudaStream_t st);
 int launch_wgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dz, const uint16_t* dzs,
                          const uint16_t* xs, const uint16_t* x, uint16_t* dw_gate, uint16_t* dw_up,
                          uint16_t* dws_gate, uint16_t* dws_up, float* partials, uint32_t* status, cudaStream_t st);
+int launch_router_wgrad_tc(const moe_dims_t& d, const uint16_t* dsplit, const uint16_t* x, float* part,
+                           uint32_t* status, cudaStream_t st);
+int launch_router_split2(const moe_dims_t& d, const float* w_router, uint16_t* w2, cudaStream_t st);
+int launch_router_wgrad_reduce(const moe_dims_t& d, const float* part, int nchunk, const float* bpart, float* dw,
+                               float* dbias, cudaStream_t st);
 int launch_combine_bwd(const moe_dims_t& d, const uint16_t* dy, const uint16_t* ys, const float* topk_gate,
                        const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
                        const uint16_t* const_vectors, uint16_t* dys, float* dg, uint32_t* status, cudaStream_t st);
 int launch_router_bwd(const moe_dims_t& d, const float* logits, const int32_t* topk_idx, const float* topk_gate,
                       const float* dg, const int32_t* counts_ext, long long t_total, float alpha, float beta,
-                      float* ds, float* dtnb, cudaStream_t st);
-int launch_router_wgrad(const moe_dims_t& d, const float* ds, const uint16_t* x, float* part, float* bpart,
-                        float* dw_router, float* dbias, cudaStream_t st);
+                      float* ds, float* dtnb, uint16_t* dsplit, float* bpart, cudaStream_t st);
+// dx = dx_shared + sum over real slots of dxs rows + sum over copy slots of g dy (combine.cu)
 int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint16_t* dxs, const int32_t* slot_row,
-                      const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, const float* ds,
-                      const float* w_router, uint16_t* dx, uint32_t* status, cudaStream_t st);
+                      const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, uint16_t* dx,
+                      uint32_t* status, cudaStream_t st);
 int launch_const_grad(const moe_dims_t& d, const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy,
                       float* dconst, cudaStream_t st);
 

@@ -1,7 +1,10 @@
-"""Run a few forwards of one seeded workload through the C ABI.
+"""Run a few forwards (and backwards) of one seeded workload through the C ABI.
 
     python -m token_choice_routing_b200.run_layer [--config qwen3_0p6b] [--forwards 3]
-        [--router tensor|fp32_cores] [--ffn single|pair]
+        [--backwards 0] [--router tensor|fp32_cores] [--ffn single|pair]
+
+With --backwards N the forwards keep the logits and the gathered rows, and N backward
+passes of <y, dy> + 2e-2 L_bal + 1e-3 L_z (seeded dy) follow them.
 
 Used as the target of profiler captures (ncu -k <kernel> -s/-c selects the
 launch). Exits non-zero if the device status word reports an error.
@@ -22,17 +25,27 @@ def main(argv=None) -> int:
     ap.add_argument("--forwards", type=int, default=3)
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"])
     ap.add_argument("--ffn", default="single", choices=["single", "pair"])
+    ap.add_argument("--backwards", type=int, default=0)
     a = ap.parse_args(argv)
     inp = I.make_inputs(I.CONFIGS[a.config])
     layer = MoENullLayer.from_inputs(inp, "cuda", router=a.router, ffn=a.ffn)
     x = bf16_tensor(inp.x, "cuda")
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).cuda()
-    out = layer.alloc(inp.cfg.T, logits=False)
+    out = layer.alloc(inp.cfg.T, logits=a.backwards > 0)
     for _ in range(a.forwards):
         layer.forward(x, tnb, out)
     torch.cuda.synchronize()
     st = B.get_device_status(out["workspace"])
     print(f"{a.config}: {a.forwards} forwards, R={int(out['offsets'][-1])}, status={B.status_string(st)}")
+    if st != B.OK or a.backwards <= 0:
+        return 0 if st == B.OK else 1
+    dy = bf16_tensor(I.upstream_grad(inp.cfg), "cuda")
+    grads = layer.alloc_grads(inp.cfg.T)
+    for _ in range(a.backwards):
+        layer.backward(x, out, dy, 2e-2, 1e-3, grads=grads)
+    torch.cuda.synchronize()
+    st = B.get_device_status(grads["workspace"])
+    print(f"{a.config}: {a.backwards} backwards, status={B.status_string(st)}")
     return 0 if st == B.OK else 1
 
 
