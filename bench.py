@@ -322,10 +322,9 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     top = max(gemm, key=lambda n: kms[n])
     gemm_ms = sum(kms[n] for n in gemm)
     gemm_flops = sum(fl[n] for n in gemm)
-    split = 2 if (T + 63) // 64 > 32 else 0  # shared-expert K-chunk reductions of the two weight gradients
-    # combine_bwd, router_bwd, router wgrad (+ reduce), W_r split, preact, dgrad/wgrad down, dgrad/wgrad
-    # gate/up, input_grad
-    launches = 11 + split + (1 if cfg.V else 0)
+    # combine_bwd, router_bwd, router wgrad (+ its reduce), W_r split, dgrad down, SwiGLU backward,
+    # wgrad down, dgrad gate/up, wgrad gate/up, input_grad (+ the constant experts' gradient)
+    launches = 11 + (1 if cfg.V else 0)
     return {
         "metric": "real-slot tokens/s per MoE layer bwd", "value": R * args.steps / (total_ms * 1e-3),
         "unit": UNIT, "ms_per_step": total_ms / args.steps, "steps": args.steps,

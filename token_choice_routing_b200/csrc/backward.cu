@@ -46,7 +46,10 @@ __device__ __forceinline__ uint4 scale8(float g, const uint4& v) {
 // the slot's expert output (a row of ys, x_t for a copy expert, c_j for a constant
 // expert; 0 for a null copy), and for a real slot dys[row] = g[t,k] dy_t (bf16), the
 // upstream gradient of that expert row. The shared expert's upstream gradient is dy.
-// One warp per token; dot products in fp32, reduced across the warp in a fixed order.
+// One warp per token, slots in groups of four: for each group, passes of 64 16-byte
+// chunks (two per lane) load the dy chunks and the four slots' chunks together before any
+// is used; dot products accumulate in fp32 per lane and are reduced across the warp in a
+// fixed order.
 __global__ void __launch_bounds__(kBwdThreads)
 combine_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ ys,
                    const float* __restrict__ gate, const int32_t* __restrict__ slot_row,
@@ -75,23 +78,52 @@ combine_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__
     }
     const uint4* dyr = reinterpret_cast<const uint4*>(dy + (size_t)t * d);
     float mydg = 0.f;
-    for (int k = 0; k < K; ++k) {
-      const int rk = __shfl_sync(0xffffffffu, row, k);
-      const float gk = __shfl_sync(0xffffffffu, g, k);
-      if (rk == -1) continue;
-      const uint16_t* src = (rk >= 0) ? ys + (size_t)rk * d : (rk == -2) ? x + (size_t)t * d : cv + (size_t)(-3 - rk) * d;
-      const uint4* sr = reinterpret_cast<const uint4*>(src);
-      uint4* dst = (rk >= 0) ? reinterpret_cast<uint4*>(dys + (size_t)rk * d) : nullptr;
-      float s = 0.f;
-#pragma unroll 4
-      for (int c = lane; c < nch; c += 32) {
-        const uint4 a = __ldg(dyr + c);
-        const uint4 b = __ldg(sr + c);
-        s += dot8(a, b);
-        if (dst) dst[c] = scale8(gk, a);
+    for (int k0 = 0; k0 < K; k0 += 4) {
+      int rq[4];
+      float gq[4], dot[4];
+      const uint4* src[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = k0 + u;
+        rq[u] = __shfl_sync(0xffffffffu, row, k & 31);
+        gq[u] = __shfl_sync(0xffffffffu, g, k & 31);
+        if (k >= K) rq[u] = -1;
+        const uint16_t* sp = (rq[u] >= 0)    ? ys + (size_t)rq[u] * d
+                             : (rq[u] == -2) ? x + (size_t)t * d
+                             : (rq[u] <= -3) ? cv + (size_t)(-3 - rq[u]) * d
+                                             : ys;
+        src[u] = reinterpret_cast<const uint4*>(sp);
+        dot[u] = 0.f;
       }
-      s = warp_sum(s);
-      if (lane == k) mydg = s;
+      if (rq[0] == -1 && rq[1] == -1 && rq[2] == -1 && rq[3] == -1) continue;  // all null copies
+      for (int c0 = 0; c0 < nch; c0 += 64) {
+        const int ca = c0 + lane, cb = c0 + 32 + lane;
+        const bool oka = ca < nch, okb = cb < nch;
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 ya = oka ? __ldg(dyr + ca) : z4;
+        const uint4 yb = okb ? __ldg(dyr + cb) : z4;
+        uint4 va[4], vb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          va[u] = (rq[u] != -1 && oka) ? __ldg(src[u] + ca) : z4;
+          vb[u] = (rq[u] != -1 && okb) ? __ldg(src[u] + cb) : z4;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (rq[u] == -1) continue;
+          dot[u] += dot8(ya, va[u]) + dot8(yb, vb[u]);
+          if (rq[u] >= 0) {
+            uint4* dst = reinterpret_cast<uint4*>(dys + (size_t)rq[u] * d);
+            if (oka) dst[ca] = scale8(gq[u], ya);
+            if (okb) dst[cb] = scale8(gq[u], yb);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float sdot = warp_sum(dot[u]);
+        if (lane == k0 + u) mydg = sdot;
+      }
     }
     if (lane < K) dg[(size_t)t * K + lane] = mydg;
   }

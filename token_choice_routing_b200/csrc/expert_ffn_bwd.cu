@@ -268,13 +268,20 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
     return ti;
   };
 
+  // This CTA's r-th tile: round-robin, so neighbouring CTAs work on neighbouring tiles (the
+  // same expert's operands) at the same time. (Dealing weight-gradient tiles largest expert
+  // first in snake order measured 40-45% slower: it breaks that L2 sharing.)
+  auto tile_at = [&](int r) { return r * (int)gridDim.x + (int)blockIdx.x; };
+
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      for (int r = 0;; ++r) {
+        const int tile = tile_at(r);
+        if (tile >= total) break;
         const Tile ti = decode(tile);
         const void* ta = (ti.g < N) ? (const void*)&tmA_r : (const void*)&tmA_s;
         const void* tb = (ti.g < N) ? (const void*)&tmB_r : (const void*)&tmB_s;
@@ -335,7 +342,9 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
     int stage = 0;
     uint32_t phase = 0;
     int li = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++li) {
+    for (;; ++li) {
+      const int tile = tile_at(li);
+      if (tile >= total) break;
       const Tile ti = decode(tile);
       const int acc = li & 1;
       const uint32_t ap = (uint32_t)(li >> 1) & 1u;
@@ -431,7 +440,9 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
         load_dh(decode(blockIdx.x), z_bar);
       }
     }
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++li) {
+    for (;; ++li) {
+      const int tile = tile_at(li);
+      if (tile >= total) break;
       const Tile ti = decode(tile);
       const int acc = li & 1;
       const uint32_t ap = (uint32_t)(li >> 1) & 1u;
@@ -491,9 +502,9 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant
         mbar_arrive(tempty_bar(acc));
         fence_proxy_async_shared();  // generic reads of the dh tile before the next TMA write
         named_bar_sync(1, EPI);
-        if (etid == 0 && tile + (int)gridDim.x < total) {
+        if (etid == 0 && tile_at(li + 1) < total) {
           z_inflight = li + 1;
-          load_dh(decode(tile + gridDim.x), z_bar);
+          load_dh(decode(tile_at(li + 1)), z_bar);
         }
       } else {
         // plain bf16 output (dgrad) or weight gradient (wgrad), staged 64 columns at a time
@@ -803,6 +814,7 @@ static int launch_wgrad(const moe_dims_t& d, const Args& a0, int BN, const CUten
                         const CUtensorMap& as_, const CUtensorMap& bs, int mrows_s, uint16_t* out_s,
                         uint16_t* out_s2, cudaStream_t st) {
   Args a = a0;
+  if (a.nsplit > 1 && !a.part_s) return MOE_ERR_INVALID_ARG;
   const long long tiles = (long long)a.nsplit * a.mt_s * a.nt_s + (long long)d.N * a.mt_r * a.nt_r;
   int r;
   switch (BN) {
@@ -834,7 +846,6 @@ int launch_wgrad_down(const moe_dims_t& d, const int32_t* offsets, const uint16_
   a.out_s = dws_down;
   a.ld_s = d.F_shared;
   a.part_s = partials;
-  if (a.nsplit > 1 && partials == nullptr) return MOE_ERR_INVALID_ARG;
   CUtensorMap ar, br, as_, bs;
   if (!(make_tmap_bf16(&ar, dys, rcap, d.d, 64) && make_tmap_bf16(&br, h, rcap, d.F, 64) &&
         make_tmap_bf16(&as_, dy, d.T, d.d, 64) && make_tmap_bf16(&bs, h_shared, d.T, d.F_shared, 64)))
@@ -844,7 +855,8 @@ int launch_wgrad_down(const moe_dims_t& d, const int32_t* offsets, const uint16_
 
 int launch_wgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dz, const uint16_t* dzs,
                          const uint16_t* xs, const uint16_t* x, uint16_t* dw_gate, uint16_t* dw_up,
-                         uint16_t* dws_gate, uint16_t* dws_up, float* partials, uint32_t* status, cudaStream_t st) {
+                         uint16_t* dws_gate, uint16_t* dws_up, float* partials, uint32_t* status,
+                         cudaStream_t st) {
   const long long rcap = (long long)d.T * d.K;
   const int BN = (d.d % 256 == 0) ? 256 : 128;
   Args a = base_args(d, offsets, status);
@@ -859,7 +871,6 @@ int launch_wgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint
   a.out_s2 = dws_up;
   a.ld_s = d.d;
   a.part_s = partials;
-  if (a.nsplit > 1 && partials == nullptr) return MOE_ERR_INVALID_ARG;
   CUtensorMap ar, br, as_, bs;
   if (!(make_tmap_bf16(&ar, dz, rcap, 2 * d.F, 64) && make_tmap_bf16(&br, xs, rcap, d.d, 64) &&
         make_tmap_bf16(&as_, dzs, d.T, 2 * d.F_shared, 64) && make_tmap_bf16(&bs, x, d.T, d.d, 64)))

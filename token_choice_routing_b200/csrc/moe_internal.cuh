@@ -274,7 +274,8 @@ int launch_wgrad_down(const moe_dims_t& d, const int32_t* offsets, const uint16_
                       float* partials, uint32_t* status, cudaStream_t st);
 int launch_wgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint16_t* dz, const uint16_t* dzs,
                          const uint16_t* xs, const uint16_t* x, uint16_t* dw_gate, uint16_t* dw_up,
-                         uint16_t* dws_gate, uint16_t* dws_up, float* partials, uint32_t* status, cudaStream_t st);
+                         uint16_t* dws_gate, uint16_t* dws_up, float* partials, uint32_t* status,
+                         cudaStream_t st);
 int launch_router_wgrad_tc(const moe_dims_t& d, const uint16_t* dsplit, const uint16_t* x, float* part,
                            uint32_t* status, cudaStream_t st);
 int launch_router_split2(const moe_dims_t& d, const float* w_router, uint16_t* w2, cudaStream_t st);
