@@ -211,3 +211,22 @@ def test_backward_data_parallel_statistics():
     ds = O.pool_grad_to_logits(dv, c.N, c.M)
     assert rel(f64(g3["dbias"]), ds.sum(axis=0)) < 1e-4
     assert rel(f64(g3["dw_router"]), ds.T @ H.f64(inp.x)) < 1e-4
+
+
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_backward_decode_sized_with_full_weights(T):
+    """Small batches with the 0.6B-shaped layer's weights: most experts receive no rows
+    (their weight gradients must be exactly zero) and the shared expert's K is a few rows."""
+    base = I.CONFIGS["decode_0p6b"]
+    cfg = I.small_config("bwd_decode", T=T, d=base.d, N=base.N, F=base.F, F_shared=base.F_shared, K=base.K,
+                         M=base.M, config_id=939)
+    inp = I.make_inputs(cfg, null_bias=I.NULL_BIAS.get("qwen3_0p6b", 0.0))
+    layer, x, tnb, out = H.run_forward(inp)
+    from token_choice_routing_b200.layer import bf16_tensor
+    from token_choice_routing_b200 import binding as B
+    dy_bits = I.upstream_grad(cfg)
+    g = layer.backward(x, out, bf16_tensor(dy_bits, "cuda"), ALPHA, BETA)
+    torch.cuda.synchronize()
+    assert B.get_device_status(g["workspace"]) == B.OK
+    ref = oracle_backward(inp, out, dy_bits, ALPHA, BETA)
+    check_all(inp, out, g, ref, out["counts"].cpu().numpy())

@@ -300,6 +300,7 @@ router_wgrad_reduce_kernel(const float* __restrict__ part, int nchunk, int rp, c
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)dw_ctas * blockDim.x) {
     const long long e = i * 4;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
     for (int c = 0; c < nchunk; ++c) {
       const float4 h = __ldg(reinterpret_cast<const float4*>(part + c * slab + e));
       const float4 l = __ldg(reinterpret_cast<const float4*>(part + c * slab + (size_t)rp * d + e));
@@ -311,35 +312,54 @@ router_wgrad_reduce_kernel(const float* __restrict__ part, int nchunk, int rp, c
 
 // ---------------------------------------------------------------------------------------
 // Constant experts' gradient: dconst[j] = sum over the tokens that selected constant
-// expert j of g dy_t (fp32, token order). Grid: (d / 256 column tiles) x V.
+// expert j of g dy_t (fp32). Grid: (d / 256 column tiles) x V; 32 warps per CTA, each
+// taking every 32nd block of 32 tokens (lane: 8 columns), then the 32 warp sums added in warp
+// order, so the result is deterministic.
 constexpr int kConstCols = 256;
+constexpr int kConstWarps = 32;
 
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kConstWarps * 32)
 const_grad_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ gate,
                   const uint16_t* __restrict__ dy, float* __restrict__ dconst, int T, int d, int K, int pool_id0) {
   pdl_wait_then_release();
-  __shared__ float s_g[kBwdThreads];
+  __shared__ __align__(16) float s_acc[kConstWarps][kConstCols];
   const int j = blockIdx.y;
-  const int c = blockIdx.x * kConstCols + threadIdx.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c0 = blockIdx.x * kConstCols;
+  const int col = c0 + lane * 8;
+  const bool colok = col < d;
   const int target = pool_id0 + j;
-  float acc = 0.f;
-  for (int tb = 0; tb < T; tb += kBwdThreads) {
-    // gate of constant expert j for each of 256 tokens (0 if the token did not select it)
-    const int t = tb + threadIdx.x;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  // warp w takes blocks of 32 tokens (block index = w mod 32): each lane tests one token,
+  // then the tokens that chose expert j are visited in ascending order
+  for (int t0 = w * 32; t0 < T; t0 += kConstWarps * 32) {
+    const int t = t0 + lane;
     float gj = 0.f;
     if (t < T)
       for (int k = 0; k < K; ++k)
         if (__ldg(topk_idx + (size_t)t * K + k) == target) gj = __ldg(gate + (size_t)t * K + k);
-    __syncthreads();
-    s_g[threadIdx.x] = gj;
-    __syncthreads();
-    const int nt = min(kBwdThreads, T - tb);
-    for (int u = 0; u < nt; ++u) {
-      const float g = s_g[u];
-      if (g != 0.f && c < d) acc = fmaf(g, __uint_as_float((uint32_t)dy[(size_t)(tb + u) * d + c] << 16), acc);
+    unsigned m = __ballot_sync(0xffffffffu, gj != 0.f);
+    while (m) {
+      const int src = __ffs(m) - 1;
+      m &= m - 1;
+      const float g = __shfl_sync(0xffffffffu, gj, src);
+      if (colok) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(dy + (size_t)(t0 + src) * d + col));
+        acc[0] = fmaf(g, bf16lo(v.x), acc[0]); acc[1] = fmaf(g, bf16hi(v.x), acc[1]);
+        acc[2] = fmaf(g, bf16lo(v.y), acc[2]); acc[3] = fmaf(g, bf16hi(v.y), acc[3]);
+        acc[4] = fmaf(g, bf16lo(v.z), acc[4]); acc[5] = fmaf(g, bf16hi(v.z), acc[5]);
+        acc[6] = fmaf(g, bf16lo(v.w), acc[6]); acc[7] = fmaf(g, bf16hi(v.w), acc[7]);
+      }
     }
   }
-  if (c < d) dconst[(size_t)j * d + c] = acc;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) s_acc[w][lane * 8 + u] = acc[u];
+  __syncthreads();
+  if (threadIdx.x < kConstCols && c0 + (int)threadIdx.x < d) {
+    float sum = 0.f;
+    for (int ww = 0; ww < kConstWarps; ++ww) sum += s_acc[ww][threadIdx.x];
+    dconst[(size_t)j * d + c0 + threadIdx.x] = sum;
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -399,7 +419,7 @@ int launch_const_grad(const moe_dims_t& d, const int32_t* topk_idx, const float*
                       float* dconst, cudaStream_t st) {
   if (d.V == 0) return MOE_OK;
   const dim3 grid((d.d + kConstCols - 1) / kConstCols, d.V);
-  return launch_pdl(const_grad_kernel, grid, dim3(kConstCols), 0, st, topk_idx, topk_gate, dy, dconst, d.T, d.d, d.K,
+  return launch_pdl(const_grad_kernel, grid, dim3(kConstWarps * 32), 0, st, topk_idx, topk_gate, dy, dconst, d.T, d.d, d.K,
                     d.N + d.M + d.C);
 }
 

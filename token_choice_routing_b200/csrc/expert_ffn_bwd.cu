@@ -630,6 +630,7 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const float* __restri
     const int m = (int)(e0 / ncols);
     const int c = (int)(e0 - (long long)m * ncols);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int s = 0; s < nsplit; ++s) {
       const float4* p = reinterpret_cast<const float4*>(part + s * stride + e0);
       const float4 v0 = __ldg(p), v1 = __ldg(p + 1);
