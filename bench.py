@@ -52,33 +52,38 @@ def load_peaks():
 # Sources whose change invalidates a recorded ncu traffic figure of the grouped GEMM.
 GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
 GEMM_PROFILE = "profiles/grouped_gemm_qwen3_0p6b.md"
+BWD_GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn_bwd.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
+BWD_GEMM_PROFILE = "profiles/bwd_gemm_kernel_qwen3_0p6b.md"
 
 
-def gemm_source_digest() -> str:
+def gemm_source_digest(sources=GEMM_SOURCES) -> str:
     import hashlib
     h = hashlib.sha256()
-    for rel in GEMM_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def recorded_gate_up_traffic(workload: str):
-    """DRAM bytes (read + write) of one gate/up launch from the committed ncu summary:
-    its line 'traffic-record: workload=W kernel=gate_up dram_bytes_per_launch=B
-    source_sha256=H'. None unless it was taken on this workload from the current
-    kernel sources."""
+def recorded_traffic(workload: str, kernel: str, profile=GEMM_PROFILE, sources=GEMM_SOURCES):
+    """DRAM bytes (read + write) of one launch of `kernel` from a committed ncu summary:
+    its line 'traffic-record: workload=W kernel=K dram_bytes_per_launch=B source_sha256=H'.
+    None unless it was taken on this workload from the current kernel sources."""
     try:
-        with open(os.path.join(ROOT, GEMM_PROFILE)) as f:
+        with open(os.path.join(ROOT, profile)) as f:
             lines = [l.strip() for l in f if l.strip().startswith("traffic-record:")]
     except OSError:
         return None
-    digest = gemm_source_digest()
+    digest = gemm_source_digest(sources)
     for l in lines:
         kv = dict(p.split("=", 1) for p in l.split()[1:] if "=" in p)
-        if kv.get("workload") == workload and kv.get("kernel") == "gate_up" and kv.get("source_sha256") == digest:
+        if kv.get("workload") == workload and kv.get("kernel") == kernel and kv.get("source_sha256") == digest:
             return float(kv["dram_bytes_per_launch"])
     return None
+
+
+def recorded_gate_up_traffic(workload: str):
+    return recorded_traffic(workload, "gate_up")
 
 
 class ClockSampler:
@@ -334,7 +339,9 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         "roofline": {"kernel": f"{top} grouped GEMM (tcgen05)", "bound": "tensor",
                      "achieved": fl[top] / (kms[top] * 1e9), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": fl[top] / (kms[top] * 1e9) / bf16_peak, "peak_kind": f"{peak_kind} bf16 burst",
-                     "traffic": None, "flops_per_launch": fl[top], "ms_per_launch": kms[top]},
+                     "traffic": recorded_traffic(cfg.name, top, BWD_GEMM_PROFILE, BWD_GEMM_SOURCES),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                     "flops_per_launch": fl[top], "ms_per_launch": kms[top]},
         "kernels": kernels,
         "gpu_launches": launches * args.steps,
     }
