@@ -31,6 +31,8 @@ CASES = {
     "wide": I.small_config("bwd_wide", T=700, d=512, N=6, F=256, F_shared=384, K=2, M=2, config_id=931),
     # T > 2048: the shared expert's weight gradients are split into K chunks and reduced
     "split": I.small_config("bwd_split", T=4500, d=256, N=8, F=128, F_shared=128, K=4, M=8, config_id=932),
+    # d not a multiple of 256 and F not a multiple of 128: the 128- and 64-wide tiles
+    "odd": I.small_config("bwd_odd", T=333, d=384, N=13, F=192, F_shared=64, K=5, M=9, config_id=940),
     # M = 0 (plain top-K) and K = 1
     "m0": I.small_config("bwd_m0", T=130, d=128, N=16, F=64, F_shared=64, K=2, M=0, config_id=933),
     "k1": I.small_config("bwd_k1", T=257, d=128, N=32, F=64, F_shared=64, K=1, M=32, config_id=934),
@@ -58,9 +60,9 @@ def f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def run(cfg, dy_scale=1.0, alpha=ALPHA, beta=BETA):
+def run(cfg, dy_scale=1.0, alpha=ALPHA, beta=BETA, router="tensor", ffn="single"):
     inp = I.make_inputs(cfg)
-    layer, x, tnb, out = H.run_forward(inp)
+    layer, x, tnb, out = H.run_forward(inp, router=router, ffn=ffn)
     dy_bits = I.upstream_grad(cfg, scale=dy_scale) if dy_scale else np.zeros((cfg.T, cfg.d), np.uint16)
     from token_choice_routing_b200.layer import bf16_tensor
     from token_choice_routing_b200 import binding as B
@@ -110,6 +112,15 @@ def test_backward_parity(name):
     ref = oracle_backward(inp, out, dy_bits, ALPHA, BETA)
     counts = out["counts"].cpu().numpy()
     check_all(inp, out, g, ref, counts)
+
+
+@pytest.mark.parametrize("router,ffn", [("fp32_cores", "single"), ("tensor", "pair")])
+def test_backward_after_each_forward_path(router, ffn):
+    """The backward reads only the forward's outputs: after the fp32 CUDA-core router or the
+    CTA-pair expert GEMMs it matches the oracle the same way."""
+    inp, layer, x, out, dy, dy_bits, g = run(CASES["wide"], router=router, ffn=ffn)
+    ref = oracle_backward(inp, out, dy_bits, ALPHA, BETA)
+    check_all(inp, out, g, ref, out["counts"].cpu().numpy())
 
 
 @pytest.mark.parametrize("name", list(PP_CASES))
