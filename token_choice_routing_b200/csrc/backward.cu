@@ -142,7 +142,7 @@ combine_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__
 // lo = bf16(ds - hi), in dsplit [T, 2 RP] (columns j and RP + j, zero past the router
 // rows), the operand of the tensor-core products ds^T x and ds W_r, and per-warp column
 // sums of ds for the bias gradient.
-constexpr int kRouterBwdMaxGrid = 1184;
+constexpr int kRouterBwdMaxGrid = 1184;  // 8 CTAs per SM on 148 SMs; also sizes the bias partials
 
 __global__ void __launch_bounds__(kBwdThreads)
 router_bwd_kernel(const float* __restrict__ logits, const int32_t* __restrict__ topk_idx,

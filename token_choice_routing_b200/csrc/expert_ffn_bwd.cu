@@ -4,13 +4,14 @@
 // Kilian et al., "Improving MoE Compute Efficiency by Composing Weight and Data Sparsity"
 // (review page, section 四 实验结果 / 训练配置: the layer is trained end to end; section
 // 三 / 实现: the grouped matmul runs on the real rows only). With the SwiGLU expert
-// E(z) = W_d (silu(W_g z) * (W_u z)) and its gate/up pre-activations a, b (recomputed from
-// the forward's rows), the gradients of one expert's rows are
-//   dh   = dys W_d                      (dgrad of the down projection)
-//   da, db from dh, a, b                (SwiGLU backward, fused into that GEMM's epilogue)
-//   dW_d = dys^T h                      (wgrad, K = the expert's rows)
-//   dz   = [da | db] W_gu               (dgrad of gate/up)
-//   dW_gu = [da | db]^T z               (wgrad, K = the expert's rows)
+// E(x) = W_d (silu(W_g x) * (W_u x)), its gate/up pre-activations [a | b] = x W_gu^T
+// (recomputed from the forward's rows) and h = silu(a) * b, the gradients of one expert's
+// rows xs are
+//   dh    = dys W_d                     (dgrad of the down projection)
+//   dz    = [da | db] from dh, a, b     (SwiGLU backward, in the recomputing GEMM's epilogue)
+//   dW_d  = dys^T h                     (wgrad, K = the expert's rows)
+//   dxs   = dz W_gu                     (dgrad of gate/up)
+//   dW_gu = dz^T xs                     (wgrad, K = the expert's rows)
 // so, as in the forward, nothing is computed for null slots.
 //
 // One kernel template serves the three GEMM shapes:
@@ -39,7 +40,6 @@ namespace bwd {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 192;  // producer, MMA, 4 epilogue warps (8 for kPreactSwiglu)
 constexpr int kStgRow = 64 * 2 + 16;
 constexpr int kBox = 64 * 64 * 2;  // one 64 x 64 bf16 box (8 KB)
 
