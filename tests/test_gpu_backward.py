@@ -241,3 +241,17 @@ def test_backward_decode_sized_with_full_weights(T):
     assert B.get_device_status(g["workspace"]) == B.OK
     ref = oracle_backward(inp, out, dy_bits, ALPHA, BETA)
     check_all(inp, out, g, ref, out["counts"].cpu().numpy())
+
+
+def test_backward_empty_batch_is_a_no_op():
+    """T = 0: the forward and the backward return without touching any buffer."""
+    cfg = I.CONFIGS["tiny"]
+    inp = I.make_inputs(cfg)
+    layer = H.make_layer(inp)[0]
+    x0 = torch.empty((0, cfg.d), dtype=torch.bfloat16, device="cuda")
+    out = layer.forward(x0, None, layer.alloc(0))
+    g = layer.alloc_grads(0)
+    sentinel = g["dw_gate"].clone()
+    layer.backward(x0, out, torch.empty((0, cfg.d), dtype=torch.bfloat16, device="cuda"), ALPHA, BETA, grads=g)
+    torch.cuda.synchronize()
+    assert torch.equal(g["dw_gate"], sentinel)
