@@ -222,8 +222,11 @@ BWD_ALPHA, BWD_BETA = 2e-2, 1e-3  # load-balance and Z-loss weights of the paper
 
 def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     """Backward pass of the same layer: gradients of <y, dy> + alpha L_bal + beta L_z with a
-    seeded dy, the forward's tensors resident. The timed step is one moe_backward call (L2
-    flushed before each); the stages are then timed one by one through their entry points."""
+    seeded dy, the forward's tensors resident. Training mode: the forward keeps the gate/up
+    pre-activations (its time is reported as forward_training_ms) and the backward takes the
+    SwiGLU derivative from them. The timed step is one moe_backward call (L2 flushed before
+    each). The backward that recomputes the pre-activations instead is timed too
+    (backward_recompute_ms). The stages are then timed one by one through their entry points."""
     import numpy as np
     import torch
     from token_choice_routing_b200 import binding as B
@@ -233,30 +236,33 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     dev = x.device
     T, d, F, Fs, N, K = cfg.T, cfg.d, cfg.F, cfg.F_shared, cfg.N, cfg.K
     rows = N + 1 + cfg.C + cfg.V
-    bout = layer.alloc(T, logits=True, xs=True)
-    layer.forward(x, tnb, bout)
+    bout = layer.alloc(T, logits=True, xs=True, save_preact=True)   # training forward
+    rout = layer.alloc(T, logits=True, xs=True)                      # no saved pre-activations
+    layer.forward(x, tnb, rout)
     dy = bf16_tensor(I.upstream_grad(cfg), dev)
     grads = layer.alloc_grads(T)
     bws = grads["workspace"]
 
-    def bstep():
-        layer.backward(x, bout, dy, BWD_ALPHA, BWD_BETA, grads=grads)
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in evs)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        bstep()
-    torch.cuda.synchronize()
+    fwd_train_ms = timed(lambda: layer.forward(x, tnb, bout)) / args.steps
+    recompute_ms = timed(lambda: layer.backward(x, rout, dy, BWD_ALPHA, BWD_BETA, grads=grads)) / args.steps
+    total_ms = timed(lambda: layer.backward(x, bout, dy, BWD_ALPHA, BWD_BETA, grads=grads))
     st = B.get_device_status(bws)
     if st != B.OK:
         raise SystemExit(f"backward device status: {B.status_string(st)}")
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for e0, e1 in evs:
-        flush.zero_()
-        e0.record()
-        bstep()
-        e1.record()
-    torch.cuda.synchronize()
-    total_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
     R = int(bout["offsets"][-1].item())
 
     # stages one by one, CUDA events between them
@@ -275,8 +281,9 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
                                                  T, BWD_ALPHA, BWD_BETA, ds, bws, grads["dtok_null_bias"])),
         ("router_wgrad", lambda: B.router_weight_grad(dm, x, grads["dw_router"], grads["dbias"], bws)),
         ("dgrad_down", lambda: B.expert_dgrad_down(dm, o["offsets"], dys, dy, layer.w_down, layer.shared_down, bws)),
-        ("swiglu_bwd", lambda: B.expert_swiglu_backward(dm, o["xs"], x, o["offsets"], layer.gate_up,
-                                                        layer.shared_gate_up, bws)),
+        ("swiglu_bwd", lambda: B.expert_swiglu_backward_saved(dm, o["offsets"], o["z"], o["z_shared"], bws)),
+        ("swiglu_bwd_recompute", lambda: B.expert_swiglu_backward(dm, o["xs"], x, o["offsets"], layer.gate_up,
+                                                                  layer.shared_gate_up, bws)),
         ("wgrad_down", lambda: B.expert_wgrad_down(dm, o["offsets"], dys, dy, o["h"], o["h_shared"],
                                                    grads["dw_down"], grads["dws_down"], bws)),
         ("dgrad_gate_up", lambda: B.expert_dgrad_gate_up(dm, o["offsets"], layer.gate_up, layer.shared_gate_up,
@@ -305,16 +312,17 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     # the router's input gradient ds W_r rides in dgrad_gate_up (extra k-blocks of the shared tiles)
-    fl = {"swiglu_bwd": 4.0 * d * (F * R + Fs * T), "dgrad_down": 2.0 * d * (F * R + Fs * T),
+    fl = {"swiglu_bwd_recompute": 4.0 * d * (F * R + Fs * T), "dgrad_down": 2.0 * d * (F * R + Fs * T),
           "wgrad_down": 2.0 * d * (F * R + Fs * T), "dgrad_gate_up": 4.0 * d * (F * R + Fs * T) + 2.0 * rows * d * T,
           "wgrad_gate_up": 4.0 * d * (F * R + Fs * T), "router_wgrad": 2.0 * rows * d * T}
-    by = {"combine_bwd": 2.0 * d * T + 4.0 * d * R + 12.0 * K * T,
+    # the saved-pre-activation SwiGLU backward reads z (4F B) and dh (2F B) and writes dz (4F B) per row
+    by = {"swiglu_bwd": 10.0 * (F * R + Fs * T), "combine_bwd": 2.0 * d * T + 4.0 * d * R + 12.0 * K * T,
           "router_bwd": 8.0 * rows * T + 12.0 * K * T,
           "input_grad": 4.0 * d * T + 2.0 * d * R + 8.0 * K * T}
     kernels = {}
     for n, ms in kms.items():
         k = {"ms": ms}
-        if n in ("swiglu_bwd", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up", "router_wgrad"):
+        if n in ("swiglu_bwd_recompute", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up", "router_wgrad"):
             k.update(bound="tensor", **{"TFLOP/s": fl[n] / (ms * 1e9)})
             k["frac"] = k["TFLOP/s"] / bf16_peak
         elif n in by:
@@ -323,7 +331,7 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         else:
             k.update(bound="alu", **{"TFLOP/s": fl[n] / (ms * 1e9)})
         kernels[n] = k
-    gemm = ["swiglu_bwd", "dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"]
+    gemm = ["dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"]
     top = max(gemm, key=lambda n: kms[n])
     gemm_ms = sum(kms[n] for n in gemm)
     gemm_flops = sum(fl[n] for n in gemm)
@@ -334,7 +342,8 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         "metric": "real-slot tokens/s per MoE layer bwd", "value": R * args.steps / (total_ms * 1e-3),
         "unit": UNIT, "ms_per_step": total_ms / args.steps, "steps": args.steps,
         "objective": f"<y, dy> + {BWD_ALPHA} L_bal + {BWD_BETA} L_z (dy seeded N(0,1) bf16)",
-        "preactivations": "recomputed in fp32 on the tensor cores; the SwiGLU derivative in that GEMM's epilogue",
+        "preactivations": "saved by the forward (training mode); the SwiGLU derivative is an elementwise pass",
+        "forward_training_ms": fwd_train_ms, "backward_recompute_ms": recompute_ms,
         "ffn_tflops_real_rows": gemm_flops / (gemm_ms * 1e9),
         "roofline": {"kernel": f"{top} grouped GEMM (tcgen05)", "bound": "tensor",
                      "achieved": fl[top] / (kms[top] * 1e9), "peak": bf16_peak, "unit": "TFLOP/s",

@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define MOE_NULL_ABI_VERSION 3
+#define MOE_NULL_ABI_VERSION 4
 
 typedef void* moe_stream_t; /* a cudaStream_t */
 
@@ -137,6 +137,11 @@ typedef struct moe_outputs {
   int32_t* counts_ext;  /* [N+M+C+V] tokens per pool slot                        */
   float* P;             /* [N+M+C+V] mean routing probability per pool slot      */
   float* losses;        /* [2] = {L_bal, L_z}                                    */
+  uint16_t* z;          /* [R_cap, 2F] bf16 gate/up pre-activations (packed order:
+                           64-column panels of 64 gate then 64 up columns), or NULL.
+                           Training: with z and z_shared set (and xs), the forward also
+                           writes them and moe_backward skips their recomputation.     */
+  uint16_t* z_shared;   /* [T, 2F_shared] bf16, or NULL (set both or neither)        */
 } moe_outputs_t;
 
 /* ABI version (MOE_NULL_ABI_VERSION) of the loaded library. */
@@ -315,9 +320,10 @@ MOE_API int moe_selftest_bounded_wait(void* workspace, uint64_t limit_ns, moe_st
  * constant in the logits and carry no gradient; the logits receive gradient through
  * the renormalised gates, through P_i in L_bal and through lse in L_z. As in the
  * forward, null slots cost nothing: the expert gradients run on the real rows only.
- * Each expert is SwiGLU; its gate/up pre-activations are recomputed from xs on the tensor
- * cores (fp32 in TMEM) rather than stored by the forward, and the SwiGLU derivative is
- * taken in that GEMM's epilogue.
+ * Each expert is SwiGLU. Its gate/up pre-activations z either come from the forward
+ * (moe_outputs_t.z / z_shared: training mode; then the SwiGLU derivative is an elementwise
+ * pass over z and dh) or are recomputed from xs on the tensor cores (fp32 in TMEM), with the
+ * SwiGLU derivative taken in that GEMM's epilogue.
  *
  * Requirements: the forward ran with out->logits and out->xs non-NULL (the copy
  * path). Weight gradients of the experts are bf16; router, bias and constant-vector
@@ -342,6 +348,9 @@ typedef struct moe_saved {
   const uint16_t* ys;         /* [R_cap, d] routed expert outputs                     */
   const int32_t* counts_ext;  /* [N+M+C+V] slot counts over every data-parallel rank  */
   int64_t t_total;            /* tokens over every data-parallel rank (>= T)          */
+  const uint16_t* z;          /* [R_cap, 2F] pre-activations saved by the forward, or
+                                 NULL to recompute them on the tensor cores             */
+  const uint16_t* z_shared;   /* [T, 2F_shared], or NULL (set both or neither)          */
 } moe_saved_t;
 
 /* Gradients (device pointers). */
@@ -423,6 +432,10 @@ MOE_API int moe_expert_dgrad_down(const moe_dims_t* dims, const int32_t* offsets
 MOE_API int moe_expert_swiglu_backward(const moe_dims_t* dims, const uint16_t* xs, const uint16_t* x,
                                        const int32_t* offsets, const uint16_t* gate_up,
                                        const uint16_t* shared_gate_up, void* bwd_workspace, moe_stream_t stream);
+/* Training-mode alternative to moe_expert_swiglu_backward: dz from the pre-activations the
+ * forward saved (z [R_cap, 2F], z_shared [T, 2F_shared]) and the dh in the workspace. */
+MOE_API int moe_expert_swiglu_backward_saved(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* z,
+                                             const uint16_t* z_shared, void* bwd_workspace, moe_stream_t stream);
 MOE_API int moe_expert_wgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys,
                                   const uint16_t* dy, const uint16_t* h, const uint16_t* h_shared,
                                   uint16_t* dw_down, uint16_t* dws_down, void* bwd_workspace,

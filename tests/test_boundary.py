@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.LIB.moe_abi_version() == 3
+    assert lib.LIB.moe_abi_version() == 4
     for code in (0, -1, -2, -3, -4, -5, 7):
         assert isinstance(lib.status_string(code), str) and lib.status_string(code)
 
@@ -156,6 +156,7 @@ def test_backward_workspace_and_host_side_rejections(lib):
     assert L.moe_input_grad(C.byref(dm), *([nul] * 9)) == inv
     assert L.moe_expert_dgrad_down(C.byref(dm), *([nul] * 7)) == inv
     assert L.moe_expert_swiglu_backward(C.byref(dm), *([nul] * 7)) == inv
+    assert L.moe_expert_swiglu_backward_saved(C.byref(dm), *([nul] * 5)) == inv
     assert L.moe_expert_wgrad_down(C.byref(dm), *([nul] * 9)) == inv
     assert L.moe_expert_dgrad_gate_up(C.byref(dm), *([nul] * 8)) == inv
     assert L.moe_expert_wgrad_gate_up(C.byref(dm), *([nul] * 9)) == inv

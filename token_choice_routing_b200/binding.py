@@ -38,7 +38,7 @@ class Weights(C.Structure):
 
 OUTPUT_FIELDS = ("logits", "topk_idx", "topk_gate", "n_real", "counts", "offsets", "perm_tok",
                  "slot_row", "xs", "h", "h_shared", "ys", "shared_out", "y", "counts_ext", "P",
-                 "losses")
+                 "losses", "z", "z_shared")
 
 
 class Outputs(C.Structure):
@@ -50,7 +50,8 @@ SAVED_FIELDS = ("x", "logits", "topk_idx", "topk_gate", "offsets", "slot_row", "
 
 
 class Saved(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in SAVED_FIELDS] + [("t_total", C.c_int64)]
+    _fields_ = [(n, C.c_void_p) for n in SAVED_FIELDS] + [("t_total", C.c_int64), ("z", C.c_void_p),
+                                                          ("z_shared", C.c_void_p)]
 
 
 GRAD_FIELDS = ("dx", "dw_router", "dbias", "dtok_null_bias", "dw_gate", "dw_up", "dw_down", "dws_gate",
@@ -98,6 +99,7 @@ def _load() -> C.CDLL:
                                           C.POINTER(Grads), vp, vp]),
         "moe_input_grad": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_swiglu_backward": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_swiglu_backward_saved": (i32, [pd, vp, vp, vp, vp, vp]),
         "moe_expert_dgrad_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_wgrad_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_dgrad_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -109,7 +111,7 @@ def _load() -> C.CDLL:
         f = getattr(lib, name)
         f.restype = res
         f.argtypes = args
-    if lib.moe_abi_version() != 3:
+    if lib.moe_abi_version() != 4:
         raise ImportError("libmoe_null ABI version mismatch")
     return lib
 
@@ -322,3 +324,9 @@ def expert_wgrad_gate_up(dm, offsets, xs, x, dw_gate, dw_up, dws_gate, dws_up, b
     _check("moe_expert_wgrad_gate_up",
            LIB.moe_expert_wgrad_gate_up(C.byref(dm), _p(offsets), _p(xs), _p(x), _p(dw_gate), _p(dw_up),
                                         _p(dws_gate), _p(dws_up), _p(bws), _stream(stream)))
+
+
+def expert_swiglu_backward_saved(dm, offsets, z, z_shared, bws, stream=None):
+    _check("moe_expert_swiglu_backward_saved",
+           LIB.moe_expert_swiglu_backward_saved(C.byref(dm), _p(offsets), _p(z), _p(z_shared), _p(bws),
+                                                _stream(stream)))

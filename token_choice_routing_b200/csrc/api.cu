@@ -205,14 +205,22 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
       !out->slot_row || !out->h || !out->h_shared || !out->ys || !out->shared_out || !out->y ||
       !out->counts_ext || !out->P || !out->losses)
     return MOE_ERR_INVALID_ARG;
+  // saved pre-activations: both buffers or neither, and only with the gathered copy xs
+  if ((out->z != nullptr) != (out->z_shared != nullptr) || (out->z && !out->xs)) return MOE_ERR_INVALID_ARG;
   const cudaStream_t st = S(stream);
   MOE_CHECK(launch_route(*dims, x, w->w_router, w->router_bias, tok_null_bias, out->logits, out->topk_idx,
                          out->topk_gate, out->n_real, workspace, st));
   MOE_CHECK(launch_dispatch(*dims, x, out->topk_idx, workspace, out->counts, out->offsets, out->perm_tok,
                             out->slot_row, out->xs, out->counts_ext, out->P, out->losses, st));
-  // xs == NULL: gate/up gathers the routed rows of x by TMA (no copies written by dispatch)
-  MOE_CHECK(launch_gate_up_perm(*dims, out->xs, x, out->offsets, out->xs ? nullptr : out->perm_tok, w->gate_up,
-                                w->shared_gate_up, out->h, out->h_shared, workspace, st));
+  if (out->z) {
+    // training: the pre-activations are kept for the backward pass (copy path only)
+    MOE_CHECK(launch_gate_up_save(*dims, out->xs, x, out->offsets, w->gate_up, w->shared_gate_up, out->h,
+                                  out->h_shared, out->z, out->z_shared, workspace, st));
+  } else {
+    // xs == NULL: gate/up gathers the routed rows of x by TMA (no copies written by dispatch)
+    MOE_CHECK(launch_gate_up_perm(*dims, out->xs, x, out->offsets, out->xs ? nullptr : out->perm_tok, w->gate_up,
+                                  w->shared_gate_up, out->h, out->h_shared, workspace, st));
+  }
   MOE_CHECK(launch_down(*dims, out->offsets, out->h, out->h_shared, w->w_down, w->shared_down, out->ys,
                         out->shared_out, workspace, st));
   return launch_combine(*dims, out->ys, out->shared_out, out->topk_gate, out->slot_row, out->topk_idx, x,

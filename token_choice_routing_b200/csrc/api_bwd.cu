@@ -38,8 +38,11 @@ static int expert_ffn_bwd(const moe_dims_t& d, const moe_weights_t* w, const moe
     MOE_CHECK(launch_router_split2(d, w->w_router, w2, st));
   }
   MOE_CHECK(launch_dgrad_down(d, sv->offsets, dys, dy, w->w_down, w->shared_down, dh, dhs, status, st));
-  MOE_CHECK(launch_swiglu_backward(d, sv->offsets, sv->xs, sv->x, w->gate_up, w->shared_gate_up, dh, dhs, dz, dzs,
-                                   status, st));
+  if (sv->z && sv->z_shared)  // training mode: pre-activations saved by the forward
+    MOE_CHECK(launch_swiglu_bwd_saved(d, sv->offsets, sv->z, sv->z_shared, dh, dhs, dz, dzs, status, st));
+  else
+    MOE_CHECK(launch_swiglu_backward(d, sv->offsets, sv->xs, sv->x, w->gate_up, w->shared_gate_up, dh, dhs, dz, dzs,
+                                     status, st));
   MOE_CHECK(launch_wgrad_down(d, sv->offsets, dys, dy, sv->h, sv->h_shared, g->dw_down, g->dws_down, spart, status,
                               st));
   MOE_CHECK(launch_dgrad_gate_up(d, sv->offsets, dz, dzs, w->gate_up, w->shared_gate_up, dsplit, w2, dxs, dx_shared,
@@ -59,7 +62,8 @@ static int router_wgrad(const moe_dims_t& d, const uint16_t* x, float* dw_router
 
 static bool saved_ok(const moe_saved_t* s, const moe_dims_t* d) {
   return s && s->x && s->logits && s->topk_idx && s->topk_gate && s->offsets && s->slot_row && s->xs && s->h &&
-         s->h_shared && s->ys && s->counts_ext && s->t_total >= (int64_t)d->T && s->t_total > 0;
+         s->h_shared && s->ys && s->counts_ext && s->t_total >= (int64_t)d->T && s->t_total > 0 &&
+         ((s->z != nullptr) == (s->z_shared != nullptr));
 }
 
 static bool expert_grads_ok(const moe_grads_t* g) {
@@ -119,6 +123,7 @@ int moe_expert_ffn_backward(const moe_dims_t* dims, const moe_weights_t* w, cons
   if (dims->T == 0) return MOE_OK;
   if (!w || !w->gate_up || !w->w_down || !w->shared_gate_up || !w->shared_down) return MOE_ERR_INVALID_ARG;
   if (!saved || !saved->x || !saved->xs || !saved->offsets || !saved->h || !saved->h_shared) return MOE_ERR_INVALID_ARG;
+  if ((saved->z != nullptr) != (saved->z_shared != nullptr)) return MOE_ERR_INVALID_ARG;
   if (!dys || !dy || !dxs || !dx_shared || !expert_grads_ok(g) || !bwd_workspace) return MOE_ERR_INVALID_ARG;
   return expert_ffn_bwd(*dims, w, saved, dys, dy, dxs, dx_shared, g, bwd_workspace, S(stream));
 }
@@ -148,6 +153,18 @@ int moe_expert_swiglu_backward(const moe_dims_t* dims, const uint16_t* xs, const
   return launch_swiglu_backward(*dims, offsets, xs, x, gate_up, shared_gate_up, ws_ptr<uint16_t>(ws, L.dh),
                                 ws_ptr<uint16_t>(ws, L.dhs), ws_ptr<uint16_t>(ws, L.dz), ws_ptr<uint16_t>(ws, L.dzs),
                                 ws_ptr<uint32_t>(ws, L.hdr), S(stream));
+}
+
+int moe_expert_swiglu_backward_saved(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* z,
+                                     const uint16_t* z_shared, void* bwd_workspace, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (dims->T == 0) return MOE_OK;
+  if (!offsets || !z || !z_shared || !bwd_workspace) return MOE_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(*dims);
+  void* ws = bwd_workspace;
+  return launch_swiglu_bwd_saved(*dims, offsets, z, z_shared, ws_ptr<uint16_t>(ws, L.dh), ws_ptr<uint16_t>(ws, L.dhs),
+                                 ws_ptr<uint16_t>(ws, L.dz), ws_ptr<uint16_t>(ws, L.dzs), ws_ptr<uint32_t>(ws, L.hdr),
+                                 S(stream));
 }
 
 int moe_expert_wgrad_down(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* dys, const uint16_t* dy,

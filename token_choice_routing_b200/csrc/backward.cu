@@ -363,6 +363,59 @@ const_grad_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict_
 }
 
 // ---------------------------------------------------------------------------------------
+// SwiGLU backward from saved pre-activations (training mode): for every routed row below
+// offsets[N] and every shared row, dz = [da | db] with a, b the saved gate/up values (bf16,
+// packed order: 64-column panels of 64 gate then 64 up columns) and dh the gradient of h:
+// da = dh b sigma(a) (1 + a (1 - sigma(a))), db = dh a sigma(a). One item = 8 consecutive h
+// columns (one 16-byte chunk of dh, two of z, two of dz).
+__global__ void __launch_bounds__(kBwdThreads)
+swiglu_bwd_saved_kernel(const int32_t* __restrict__ offsets, int N, long long rcap, const uint16_t* __restrict__ z,
+                        const uint16_t* __restrict__ dh, uint16_t* __restrict__ dz, int F,
+                        const uint16_t* __restrict__ zs, const uint16_t* __restrict__ dhs, uint16_t* __restrict__ dzs,
+                        int Fs, int T, uint32_t* status) {
+  pdl_wait_then_release();
+  long long R = __ldg(offsets + N);
+  if (R < 0 || R > rcap) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, kStatusBounds);
+    R = 0;
+  }
+  const long long cr = F / 8, cs = Fs / 8;
+  const long long n_r = R * cr, n_all = n_r + (long long)T * cs;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_all; i += (long long)gridDim.x * blockDim.x) {
+    const bool routed = i < n_r;
+    const long long k = routed ? i : i - n_r;
+    const long long cpr = routed ? cr : cs;
+    const long long row = k / cpr;
+    const int f = (int)(k - row * cpr) * 8;
+    const int w = routed ? F : Fs;
+    const uint16_t* zr = (routed ? z : zs) + (size_t)row * 2 * w + (f >> 6) * 128 + (f & 63);
+    const uint4 hv = __ldg(reinterpret_cast<const uint4*>((routed ? dh : dhs) + (size_t)row * w + f));
+    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(zr));
+    const uint4 uv = __ldg(reinterpret_cast<const uint4*>(zr + 64));
+    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float da[2], db[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float a = h ? bf16hi(gw[j]) : bf16lo(gw[j]);
+        const float b = h ? bf16hi(uw[j]) : bf16lo(uw[j]);
+        const float g = h ? bf16hi(hw[j]) : bf16lo(hw[j]);
+        const float sg = __fdividef(1.f, 1.f + __expf(-a));
+        db[h] = g * a * sg;
+        da[h] = g * b * sg * (1.f + a * (1.f - sg));
+      }
+      og[j] = pack_bf16x2(da[0], da[1]);
+      ou[j] = pack_bf16x2(db[0], db[1]);
+    }
+    uint16_t* dr = (routed ? dz : dzs) + (size_t)row * 2 * w + (f >> 6) * 128 + (f & 63);
+    *reinterpret_cast<uint4*>(dr) = make_uint4(og[0], og[1], og[2], og[3]);
+    *reinterpret_cast<uint4*>(dr + 64) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // Host launchers.
 
 static int grid_warps(long long items, int occ_cap) {
@@ -421,6 +474,13 @@ int launch_const_grad(const moe_dims_t& d, const int32_t* topk_idx, const float*
   const dim3 grid((d.d + kConstCols - 1) / kConstCols, d.V);
   return launch_pdl(const_grad_kernel, grid, dim3(kConstWarps * 32), 0, st, topk_idx, topk_gate, dy, dconst, d.T, d.d, d.K,
                     d.N + d.M + d.C);
+}
+
+int launch_swiglu_bwd_saved(const moe_dims_t& d, const int32_t* offsets, const uint16_t* z, const uint16_t* zs,
+                            const uint16_t* dh, const uint16_t* dhs, uint16_t* dz, uint16_t* dzs, uint32_t* status,
+                            cudaStream_t st) {
+  return launch_pdl(swiglu_bwd_saved_kernel, dim3(sm_count() * 8), dim3(kBwdThreads), 0, st, offsets, d.N,
+                    (long long)d.T * d.K, z, dh, dz, d.F, zs, dhs, dzs, d.F_shared, d.T, status);
 }
 
 }  // namespace moe

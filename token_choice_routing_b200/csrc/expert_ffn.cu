@@ -59,6 +59,10 @@ struct GemmArgs {
   uint32_t* status;
   unsigned long long limit_ns;
   int has_shared;
+  uint16_t* zout_r;        // SAVEZ: gate/up pre-activations [rows_cap, 2F] (packed column order)
+  int ldz_r;
+  uint16_t* zout_s;        // SAVEZ: the shared expert's [T, 2F_shared]
+  int ldz_s;
 };
 
 template <int BN>
@@ -81,7 +85,7 @@ struct TileInfo {
   int g, arow, mvalid, brow, nkb, col0;
 };
 
-template <int BN, bool SWIGLU, bool GATHER>
+template <int BN, bool SWIGLU, bool GATHER, bool SAVEZ = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
                     const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s,
@@ -367,6 +371,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
               const float h1 = __fdividef(g1, 1.f + __expf(-g1)) * u1;
               packed[j] = pack_bf16x2(h0, h1);
             }
+            if constexpr (SAVEZ) {
+              // training: keep the pre-activations (bf16, packed order) for the backward pass
+              if (row < ti.mvalid) {
+                uint16_t* zo = (ti.g < N) ? a.zout_r : a.zout_s;
+                const int ldz = (ti.g < N) ? a.ldz_r : a.ldz_s;
+                uint16_t* zrow = zo + (size_t)(ti.arow + row) * ldz + 2 * ti.col0 + c * 128 + g16 * 16;
+                uint4* zg = reinterpret_cast<uint4*>(zrow);
+                uint4* zu = reinterpret_cast<uint4*>(zrow + 64);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                  zg[q] = make_uint4(pack_bf16x2(__uint_as_float(gr[8 * q + 0]), __uint_as_float(gr[8 * q + 1])),
+                                     pack_bf16x2(__uint_as_float(gr[8 * q + 2]), __uint_as_float(gr[8 * q + 3])),
+                                     pack_bf16x2(__uint_as_float(gr[8 * q + 4]), __uint_as_float(gr[8 * q + 5])),
+                                     pack_bf16x2(__uint_as_float(gr[8 * q + 6]), __uint_as_float(gr[8 * q + 7])));
+                  zu[q] = make_uint4(pack_bf16x2(__uint_as_float(ur[8 * q + 0]), __uint_as_float(ur[8 * q + 1])),
+                                     pack_bf16x2(__uint_as_float(ur[8 * q + 2]), __uint_as_float(ur[8 * q + 3])),
+                                     pack_bf16x2(__uint_as_float(ur[8 * q + 4]), __uint_as_float(ur[8 * q + 5])),
+                                     pack_bf16x2(__uint_as_float(ur[8 * q + 6]), __uint_as_float(ur[8 * q + 7])));
+                }
+              }
+            }
           } else {
             uint32_t r[16];
             tmem_ld16(tb + (uint32_t)(c * 64 + g16 * 16), r);
@@ -472,7 +497,7 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU, bool GATHER>
+template <int BN, bool SWIGLU, bool GATHER, bool SAVEZ = false>
 static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUtensorMap& as_,
                        const CUtensorMap& bs, const GemmArgs& a, long long max_tiles, cudaStream_t st) {
   using SM = GemmSmem<BN>;
@@ -480,7 +505,7 @@ static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, SWIGLU, GATHER>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, SWIGLU, GATHER, SAVEZ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::bytes);
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
@@ -488,7 +513,7 @@ static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   long long grid = sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(grouped_gemm_kernel<BN, SWIGLU, GATHER>, dim3((unsigned)grid), dim3(kGemmThreads), SM::bytes, st, ar, br,
+  return launch_pdl(grouped_gemm_kernel<BN, SWIGLU, GATHER, SAVEZ>, dim3((unsigned)grid), dim3(kGemmThreads), SM::bytes, st, ar, br,
                     as_, bs, a);
 }
 
@@ -567,6 +592,31 @@ int launch_gate_up_perm(const moe_dims_t& d, const uint16_t* xs, const uint16_t*
                           : launch_gemm<128, true, true>(ar, br, as_, bs, p.g1, p.max1, st);
   return (p.BN1 == 256) ? launch_gemm<256, true, false>(ar, br, as_, bs, p.g1, p.max1, st)
                         : launch_gemm<128, true, false>(ar, br, as_, bs, p.g1, p.max1, st);
+}
+
+// gate/up with the pre-activations also written (training): z [rows_cap, 2F] and zs [T, 2F_shared]
+// in the packed column order, bf16. Copy path (xs) only.
+int launch_gate_up_save(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                        const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
+                        uint16_t* z, uint16_t* zs, void* ws, cudaStream_t st) {
+  FfnPlan p = plan_ffn(d, offsets, ws);
+  const long long rcap = (long long)d.T * d.K;
+  CUtensorMap ar, br, as_, bs;
+  if (!(make_tmap_bf16(&ar, xs, (uint64_t)rcap, d.d, kBM) &&
+        make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, p.BN1) &&
+        make_tmap_bf16(&as_, x, d.T, d.d, kBM) &&
+        make_tmap_bf16(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, p.BN1)))
+    return MOE_ERR_CUDA;
+  p.g1.out_r = h;
+  p.g1.out_s = h_shared;
+  p.g1.x = x;
+  p.g1.ld_x = d.d;
+  p.g1.zout_r = z;
+  p.g1.ldz_r = 2 * d.F;
+  p.g1.zout_s = zs;
+  p.g1.ldz_s = 2 * d.F_shared;
+  return (p.BN1 == 256) ? launch_gemm<256, true, false, true>(ar, br, as_, bs, p.g1, p.max1, st)
+                        : launch_gemm<128, true, false, true>(ar, br, as_, bs, p.g1, p.max1, st);
 }
 
 int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,

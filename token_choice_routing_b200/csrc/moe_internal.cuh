@@ -245,6 +245,11 @@ int launch_expert_ffn(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x
                       const uint16_t* sgate_up, const uint16_t* sdown, uint16_t* h,
                       uint16_t* h_shared, uint16_t* ys, uint16_t* shared_out, void* ws,
                       cudaStream_t st);
+// gate/up that also writes the pre-activations z [T K, 2F] and zs [T, 2F_shared] (bf16, packed
+// column order) for the backward pass; copy path (xs) only
+int launch_gate_up_save(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
+                        const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
+                        uint16_t* z, uint16_t* zs, void* ws, cudaStream_t st);
 int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,
                    const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h, uint16_t* h_shared,
                    void* ws, cudaStream_t st);
@@ -293,6 +298,11 @@ int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint
                       uint32_t* status, cudaStream_t st);
 int launch_const_grad(const moe_dims_t& d, const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy,
                       float* dconst, cudaStream_t st);
+// dz from saved pre-activations and dh (elementwise, every routed row below offsets[N] and
+// every shared row)
+int launch_swiglu_bwd_saved(const moe_dims_t& d, const int32_t* offsets, const uint16_t* z, const uint16_t* zs,
+                            const uint16_t* dh, const uint16_t* dhs, uint16_t* dz, uint16_t* dzs, uint32_t* status,
+                            cudaStream_t st);
 
 // ------------------------------------------------------------------------------------
 // Device helpers.

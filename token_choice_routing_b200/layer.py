@@ -79,10 +79,12 @@ class MoENullLayer:
     def dims(self, T: int) -> B.Dims:
         return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags, self.C, self.V)
 
-    def alloc(self, T: int, logits: bool = True, xs: bool = True) -> Dict[str, torch.Tensor]:
+    def alloc(self, T: int, logits: bool = True, xs: bool = True, save_preact: bool = False) -> Dict[str, torch.Tensor]:
         """Caller-owned buffers for a T-token call (R_cap = T*K rows). xs=False
         leaves out the gathered copy of the routed rows: the forward then gathers
-        rows of x inside the gate/up GEMM and dispatch writes no copies."""
+        rows of x inside the gate/up GEMM and dispatch writes no copies.
+        save_preact=True (training) adds z/z_shared: the forward keeps the gate/up
+        pre-activations and the backward does not recompute them."""
         dev, d, N, M, K, F, Fs = self.device, self.d, self.N, self.M, self.K, self.F, self.F_shared
         R = T * K
         i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
@@ -104,6 +106,8 @@ class MoENullLayer:
             counts_ext=torch.empty((N + M + self.C + self.V,), dtype=i32, device=dev),
             P=torch.empty((N + M + self.C + self.V,), dtype=f32, device=dev),
             losses=torch.empty((2,), dtype=f32, device=dev),
+            z=torch.empty((max(R, 1), 2 * F), dtype=bf, device=dev) if save_preact else None,
+            z_shared=torch.empty((max(T, 1), 2 * Fs), dtype=bf, device=dev) if save_preact else None,
         )
         out["workspace"] = torch.empty((max(B.workspace_bytes(self.dims(T)), 256),), dtype=torch.uint8, device=dev)
         return out
@@ -138,10 +142,12 @@ class MoENullLayer:
             raise ValueError("the backward needs the forward's logits and xs")
         ce = out["counts_ext"] if counts_ext is None else counts_ext
         ptr = lambda t: t.data_ptr()
+        z, zs = out.get("z"), out.get("z_shared")
         return B.Saved(ptr(x), ptr(out["logits"]), ptr(out["topk_idx"]), ptr(out["topk_gate"]),
                        ptr(out["offsets"]), ptr(out["slot_row"]), ptr(out["xs"]), ptr(out["h"]),
                        ptr(out["h_shared"]), ptr(out["ys"]), ptr(ce),
-                       int(x.shape[0] if t_total is None else t_total))
+                       int(x.shape[0] if t_total is None else t_total),
+                       None if z is None else ptr(z), None if zs is None else ptr(zs))
 
     def backward(self, x: torch.Tensor, out: Dict[str, torch.Tensor], dy: torch.Tensor, alpha: float = 2e-2,
                  beta: float = 1e-3, grads: Optional[Dict[str, torch.Tensor]] = None,
