@@ -488,11 +488,13 @@ def router_backward(x, w_router, ds):
 
 
 def layer_backward(x, s, w_router, N, M, K, experts, shared, dy, alpha, beta,
-                   C=0, V=0, const_vectors=None):
+                   C=0, V=0, const_vectors=None, counts=None, t_total=None):
     """All gradients of L = <y, dy> + alpha L_bal + beta L_z for one layer.
 
     ``s`` are the forward logits [T, N+1+C+V] (the routing is taken from them, so a
-    parity test passes the logits the GPU computed). Returns a dict with dx [T, d],
+    parity test passes the logits the GPU computed). For one shard of a data-parallel
+    batch, ``counts`` and ``t_total`` are the whole batch's slot counts and token count
+    (see :func:`aux_backward`). Returns a dict with dx [T, d],
     dg [T, K] (gradient of each slot's gate), ds [T, N+1+C+V] (logit gradient),
     dW_r, dbias, dtnb [T] (null-offset gradient), dW_gate/dW_up [N, F, d],
     dW_down [N, d, F], the shared expert's (dWs_gate, dWs_up, dWs_down) and
@@ -532,7 +534,7 @@ def layer_backward(x, s, w_router, N, M, K, experts, shared, dy, alpha, beta,
             dg[rows, ks] = dy[rows] @ cv[j - C]
             dconst[j - C] = (gates[rows, ks][:, None] * dy[rows]).sum(axis=0)
     dv = gate_backward(r["v"], idx, gates, dg, N, M) + aux_backward(idx, r["p"], r["lse"], N,
-                                                                   alpha, beta)
+                                                                   alpha, beta, counts, t_total)
     ds = pool_grad_to_logits(dv, N, M, C, V)
     dx_r, dw_r, dbias = router_backward(x, w_router, ds)
     return dict(dx=dx + dx_r, dg=dg, ds=ds, dW_r=dw_r, dbias=dbias, dtnb=ds[:, N].copy(),

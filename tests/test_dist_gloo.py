@@ -113,3 +113,65 @@ def test_sums_layout_matches_library_count():
     for N, M, K, Cc, V in ((8, 4, 4, 2, 3), (60, 0, 8, 10, 5)):
         assert aux_sums_slices(N, K, Cc + V)["T"].stop == B.aux_sums_count(B.dims(10, 128, N, M, K, 64, 64,
                                                                                 C=Cc, V=V))
+
+
+def _bwd_case():
+    rng = np.random.default_rng(78)
+    T, d, N, M, K, F, Fs = 40, 8, 4, 3, 2, 6, 5
+    x = rng.standard_normal((T, d))
+    w_r = rng.standard_normal((N + 1, d)) / np.sqrt(d)
+    s = x @ w_r.T
+    s[:, N] += rng.choice([-4.0, 0.0, 4.0], size=T)
+    experts = (rng.standard_normal((N, F, d)), rng.standard_normal((N, F, d)), rng.standard_normal((N, d, F)))
+    shared = (rng.standard_normal((Fs, d)), rng.standard_normal((Fs, d)), rng.standard_normal((d, Fs)))
+    dy = rng.standard_normal((T, d))
+    return x, w_r, s, experts, shared, dy, N, M, K
+
+
+def _bwd_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from token_choice_routing_b200.dist import allreduce_grads, allreduce_token_total
+        x, w_r, s, experts, shared, dy, N, M, K = _bwd_case()
+        shard = np.array_split(np.arange(x.shape[0]), world)[rank]
+        # whole-batch statistics from the ranks: slot counts (the forward's all-reduce) and T
+        idx = O.route(s[shard], M, K)["idx"]
+        counts = torch.from_numpy(np.bincount(idx.reshape(-1), minlength=N + M).astype(np.int64))
+        dist.all_reduce(counts)
+        t_total = allreduce_token_total(len(shard))
+        g = O.layer_backward(x[shard], s[shard], w_r, N, M, K, experts, shared, dy[shard], 0.5, 0.25,
+                             counts=counts.numpy(), t_total=t_total)
+        grads = {"dw_router": torch.from_numpy(g["dW_r"]), "dbias": torch.from_numpy(g["dbias"]),
+                 "dw_gate": torch.from_numpy(g["dW_gate"]), "dws_down": torch.from_numpy(g["dWs_down"]),
+                 "dx": torch.from_numpy(g["dx"].copy())}
+        dx_before = grads["dx"].clone()
+        allreduce_grads(grads)
+        q.put((rank, t_total, {k: v.numpy() for k, v in grads.items()}, torch.equal(dx_before, grads["dx"])))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_backward_statistics_and_gradient_sum():
+    """Data-parallel backward plumbing on two CPU ranks: the token total and slot counts are
+    all-reduced, each rank differentiates its own tokens with them, and allreduce_grads sums the
+    weight gradients (not dx) into the whole batch's gradient."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    x, w_r, s, experts, shared, dy, N, M, K = _bwd_case()
+    whole = O.layer_backward(x, s, w_r, N, M, K, experts, shared, dy, 0.5, 0.25)
+    for rank, t_total, grads, dx_kept in res:
+        assert t_total == x.shape[0] and dx_kept
+        np.testing.assert_allclose(grads["dw_router"], whole["dW_r"], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(grads["dbias"], whole["dbias"], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(grads["dw_gate"], whole["dW_gate"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(grads["dws_down"], whole["dWs_down"], rtol=1e-12, atol=1e-12)

@@ -193,3 +193,22 @@ def test_aux_backward_of_a_shard_equals_the_rows_of_the_whole_batch():
     # and a shard's own statistics give something else
     own = o.aux_backward(idx[:17], p[:17], lse[:17], N, 0.7, 0.3)
     assert not np.allclose(own, whole[:17])
+
+
+def test_shard_gradients_sum_to_the_whole_batch_gradient():
+    """Data parallel: each shard's weight gradients, taken with the whole batch's slot counts
+    and token total, add up to the whole batch's weight gradients (the objective is a sum over
+    tokens of <y_t, dy_t> plus losses built from whole-batch means)."""
+    c = _case(T=18, d=6, N=4, M=3, K=2, F=4, Fs=3, seed=17)
+    s = o.router_logits(c["x"], c["w_r"], c["bias"], c["tnb"])
+    whole = o.layer_backward(c["x"], s, c["w_r"], 4, 3, 2, c["experts"], c["shared"], c["dy"], 0.7, 0.4)
+    counts = np.bincount(whole["idx"].reshape(-1), minlength=7)
+    acc = None
+    for rows in (np.arange(0, 7), np.arange(7, 18)):
+        part = o.layer_backward(c["x"][rows], s[rows], c["w_r"], 4, 3, 2, c["experts"], c["shared"], c["dy"][rows],
+                                0.7, 0.4, counts=counts, t_total=18)
+        np.testing.assert_allclose(part["dx"], whole["dx"][rows], rtol=1e-12, atol=1e-14)
+        acc = part if acc is None else {k: acc[k] + part[k] for k in ("dW_r", "dbias", "dW_gate", "dW_up", "dW_down",
+                                                                      "dWs_gate", "dWs_up", "dWs_down")}
+    for k in ("dW_r", "dbias", "dW_gate", "dW_up", "dW_down", "dWs_gate", "dWs_up", "dWs_down"):
+        np.testing.assert_allclose(acc[k], whole[k], rtol=1e-12, atol=1e-14, err_msg=k)

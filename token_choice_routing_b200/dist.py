@@ -68,3 +68,37 @@ def dp_forward(layer, x, tok_null_bias, out, sums, group=None):
     B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
               topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
     return out
+
+
+# Weight gradients summed over the ranks in data-parallel training. dx and the per-token
+# null-offset gradient belong to each rank's own tokens and are not reduced.
+GRAD_SUM_KEYS = ("dw_router", "dbias", "dw_gate", "dw_up", "dw_down", "dws_gate", "dws_up", "dws_down", "dconst")
+
+
+def allreduce_token_total(T_local: int, device="cpu", group=None) -> int:
+    """Tokens over all ranks (the denominator of f_i and of both losses' means)."""
+    t = torch.tensor([int(T_local)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    return int(t.item())
+
+
+def allreduce_grads(grads: Dict[str, torch.Tensor], keys=GRAD_SUM_KEYS, group=None) -> Dict[str, torch.Tensor]:
+    """In-place SUM all-reduce of the weight gradients. Each rank's backward differentiates
+    its own tokens' terms of <y, dy> + alpha L_bal + beta L_z with the whole-batch f_i and
+    token total, so the sum over ranks is the whole batch's gradient."""
+    for k in keys:
+        t = grads.get(k)
+        if t is not None and t.numel() > 0:
+            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    return grads
+
+
+def dp_backward(layer, x, out, dy, t_total: int, alpha: float = 2e-2, beta: float = 1e-3, grads=None, group=None,
+                reduce_grads: bool = True):
+    """Data-parallel backward after ``dp_forward``: ``out["counts_ext"]`` already holds the
+    all-reduced slot counts and ``t_total`` is ``allreduce_token_total`` of the ranks' T. The
+    weight gradients are then summed over the ranks (``reduce_grads``)."""
+    g = layer.backward(x, out, dy, alpha, beta, grads=grads, t_total=t_total)
+    if reduce_grads:
+        allreduce_grads(g, group=group)
+    return g
