@@ -879,12 +879,12 @@ int launch_wgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint
   return launch_wgrad(d, a, BN, ar, br, as_, bs, 2 * d.F_shared, dws_gate, dws_up, st);
 }
 
-// K chunks of the router weight gradient dsplit^T x: at least 4 k-blocks each, at most 32
-// chunks.
+// K chunks of the router weight gradient dsplit^T x: at least 16 k-blocks each, at most 16
+// chunks (on the 0.6B-shaped workload one round of 128 tiles, 16.8 MB of partials).
 int router_wgrad_split(const moe_dims_t& d, int* chunk_kb) {
   const int kb = (d.T + kBK - 1) / kBK;
-  int ck = 4;
-  if ((kb + ck - 1) / ck > 32) ck = (kb + 31) / 32;
+  int ck = 16;
+  if ((kb + ck - 1) / ck > 16) ck = (kb + 15) / 16;
   if (chunk_kb) *chunk_kb = ck;
   const int n = (kb + ck - 1) / ck;
   return n < 1 ? 1 : n;
