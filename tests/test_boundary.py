@@ -170,3 +170,41 @@ def test_backward_workspace_and_host_side_rejections(lib):
     assert L.moe_backward(C.byref(bad), nul, nul, nul, 0.02, 0.001, nul, nul, nul) == B.ERR_UNSUPPORTED
     zero = B.dims(0, 128, 8, 8, 4, 64, 64)
     assert L.moe_backward(C.byref(zero), nul, nul, nul, 0.02, 0.001, nul, nul, nul) == B.OK
+
+
+def test_struct_layouts_match_header(tmp_path, lib):
+    """The binding's ctypes structures have the C header's field offsets and sizes (compiled
+    with the host C compiler against include/moe_null.h)."""
+    import shutil
+    import subprocess
+    B = lib
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    structs = {
+        "moe_dims_t": (B.Dims, [f for f, _ in B.Dims._fields_]),
+        "moe_weights_t": (B.Weights, [f for f, _ in B.Weights._fields_]),
+        "moe_outputs_t": (B.Outputs, [f for f, _ in B.Outputs._fields_]),
+        "moe_saved_t": (B.Saved, [f for f, _ in B.Saved._fields_]),
+        "moe_grads_t": (B.Grads, [f for f, _ in B.Grads._fields_]),
+    }
+    src = ['#include <stdio.h>', '#include <stddef.h>', '#include "moe_null.h"', "int main(void) {"]
+    for name, (_, fields) in structs.items():
+        src.append(f'  printf("{name} sizeof %zu\\n", sizeof({name}));')
+        for f in fields:
+            src.append(f'  printf("{name} {f} %zu\\n", offsetof({name}, {f}));')
+    src += ["  return 0;", "}"]
+    c = tmp_path / "layout.c"
+    c.write_text("\n".join(src) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {}
+    for line in out:
+        if line.strip():
+            name, field, val = line.split()
+            got[(name, field)] = int(val)
+    for name, (cls, fields) in structs.items():
+        assert got[(name, "sizeof")] == C.sizeof(cls), name
+        for f in fields:
+            assert got[(name, f)] == getattr(cls, f).offset, (name, f)

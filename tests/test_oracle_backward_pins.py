@@ -212,3 +212,18 @@ def test_shard_gradients_sum_to_the_whole_batch_gradient():
                                                                       "dWs_gate", "dWs_up", "dWs_down")}
     for k in ("dW_r", "dbias", "dW_gate", "dW_up", "dW_down", "dWs_gate", "dWs_up", "dWs_down"):
         np.testing.assert_allclose(acc[k], whole[k], rtol=1e-12, atol=1e-14, err_msg=k)
+
+
+def test_gate_gradient_two_selected_experts_closed_form():
+    """Worked example: a token whose two selected slots are real with logits s1, s2 has gates
+    g1 = 1/(1+e^{s2-s1}), g2 = 1 - g1, so dL/ds1 = -dL/ds2 = g1 g2 (dg1 - dg2); the other
+    logits get nothing from the gates."""
+    s1, s2, dg1, dg2 = 0.7, -0.4, 1.3, -0.6
+    v = np.array([[s1, s2, -3.0, -2.5, -2.5]])  # 3 reals, then 2 copies of a null logit -2.5
+    idx = np.array([[0, 1]])
+    gates = o.renormalised_gates(np.array([[s1, s2, -3.0, -2.5]]), idx, 3)
+    g1 = 1.0 / (1.0 + np.exp(s2 - s1))
+    np.testing.assert_allclose(gates[0], [g1, 1 - g1], rtol=1e-15)
+    dv = o.gate_backward(v, idx, gates, np.array([[dg1, dg2]]), 3, 2)
+    expect = g1 * (1 - g1) * (dg1 - dg2)
+    np.testing.assert_allclose(dv[0], [expect, -expect, 0.0, 0.0, 0.0], rtol=1e-14, atol=1e-16)
