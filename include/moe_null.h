@@ -292,7 +292,10 @@ MOE_API int moe_aux(const moe_dims_t* dims, const void* workspace, int32_t* coun
 
 /* The whole forward: route, dispatch (+aux), expert FFNs, combine. With
  * out->xs == NULL the routed rows are never copied: dispatch writes only the
- * permutation and gate/up gathers rows of x (moe_expert_gate_up_gather). */
+ * permutation and gate/up gathers rows of x (moe_expert_gate_up_gather). With
+ * out->z and out->z_shared set (training; xs required) the gate/up GEMM also
+ * writes the pre-activations for moe_backward. z and z_shared must both be set or
+ * both NULL, else MOE_ERR_INVALID_ARG before anything is enqueued. */
 MOE_API int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* x,
                 const float* tok_null_bias, const moe_outputs_t* out, void* workspace,
                 moe_stream_t stream);
