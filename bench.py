@@ -598,6 +598,9 @@ def main():
             "config": workload_config(cfg, args),
             "real_slots_per_step": R, "tokens_per_s": world * T * args.steps / (total_ms * 1e-3),
             "ffn_tflops_real_rows": ffn_tflops, "ffn_frac_of_bf16_peak": ffn_tflops / bf16_peak,
+            # the FLOPs behind it: routed real slots and the shared expert's T rows (one launch each GEMM)
+            "ffn_gflop_per_step": {"routed": 6.0 * cfg.d * cfg.F * R / 1e9,
+                                   "shared": 6.0 * cfg.d * cfg.F_shared * cfg.T / 1e9},
             "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk.summary(),
