@@ -1,10 +1,12 @@
 """Run a few forwards (and backwards) of one seeded workload through the C ABI.
 
     python -m token_choice_routing_b200.run_layer [--config qwen3_0p6b] [--forwards 3]
-        [--backwards 0] [--router tensor|fp32_cores] [--ffn single|pair]
+        [--backwards 0] [--save-preact] [--router tensor|fp32_cores] [--ffn single|pair]
 
 With --backwards N the forwards keep the logits and the gathered rows, and N backward
-passes of <y, dy> + 2e-2 L_bal + 1e-3 L_z (seeded dy) follow them.
+passes of <y, dy> + 2e-2 L_bal + 1e-3 L_z (seeded dy) follow them. --save-preact runs the
+training mode: the forwards also save the gate/up pre-activations and the backwards take the
+SwiGLU derivative from them.
 
 Used as the target of profiler captures (ncu -k <kernel> -s/-c selects the
 launch). Exits non-zero if the device status word reports an error.
@@ -26,12 +28,13 @@ def main(argv=None) -> int:
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"])
     ap.add_argument("--ffn", default="single", choices=["single", "pair"])
     ap.add_argument("--backwards", type=int, default=0)
+    ap.add_argument("--save-preact", action="store_true")
     a = ap.parse_args(argv)
     inp = I.make_inputs(I.CONFIGS[a.config])
     layer = MoENullLayer.from_inputs(inp, "cuda", router=a.router, ffn=a.ffn)
     x = bf16_tensor(inp.x, "cuda")
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).cuda()
-    out = layer.alloc(inp.cfg.T, logits=a.backwards > 0)
+    out = layer.alloc(inp.cfg.T, logits=a.backwards > 0, save_preact=a.save_preact)
     for _ in range(a.forwards):
         layer.forward(x, tnb, out)
     torch.cuda.synchronize()
