@@ -175,3 +175,54 @@ def test_two_rank_backward_statistics_and_gradient_sum():
         np.testing.assert_allclose(grads["dbias"], whole["dbias"], rtol=1e-12, atol=1e-13)
         np.testing.assert_allclose(grads["dw_gate"], whole["dW_gate"], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(grads["dws_down"], whole["dWs_down"], rtol=1e-12, atol=1e-12)
+
+
+def _bf16_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from token_choice_routing_b200.dist import allreduce_grads
+        g = torch.from_numpy(_bf16_grads(rank)).to(torch.bfloat16)
+        grads = {"dw_down": g, "dw_router": torch.from_numpy(_bf16_grads(rank).astype(np.float32))}
+        allreduce_grads(grads)
+        q.put((rank, grads["dw_down"].float().numpy(), grads["dw_router"].numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _bf16_grads(rank):
+    """A rank's bf16-valued gradient: values spread over several binades, so that rounding
+    after each partial sum would differ from one rounding of the exact sum."""
+    rng = np.random.default_rng(500 + rank)
+    mant = rng.integers(128, 256, size=4096)          # 8 significant bits: exactly a bf16 value
+    sign = rng.choice([-1.0, 1.0], size=4096)
+    return (sign * mant * np.exp2(rng.integers(-3, 4, size=4096) - 7.0)).astype(np.float32)
+
+
+def test_bf16_gradients_are_summed_in_fp32_and_rounded_once():
+    """allreduce_grads over four ranks gives each bf16 weight gradient as bf16(the exact sum of
+    the ranks' values): at most one rounding, whatever the number of ranks. (Four bf16 values
+    within seven binades of each other add exactly in float32.)"""
+    world = 4
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bf16_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    exact = sum(_bf16_grads(r).astype(np.float64) for r in range(world))
+    once = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(exact.astype(np.float32).astype(np.float64), exact)  # the fp32 sum is exact
+    # a bf16 running sum (what an all-reduce in bf16 does) would not be: the case can tell them apart
+    run = torch.from_numpy(_bf16_grads(0)).to(torch.bfloat16)
+    for r in range(1, world):
+        run = (run + torch.from_numpy(_bf16_grads(r)).to(torch.bfloat16))
+    assert not np.array_equal(run.float().numpy(), once)
+    for rank, g, gr in res:
+        assert np.array_equal(g, once), rank
+        np.testing.assert_allclose(gr, exact, rtol=1e-6, atol=1e-6)

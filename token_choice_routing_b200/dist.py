@@ -85,10 +85,21 @@ def allreduce_token_total(T_local: int, device="cpu", group=None) -> int:
 def allreduce_grads(grads: Dict[str, torch.Tensor], keys=GRAD_SUM_KEYS, group=None) -> Dict[str, torch.Tensor]:
     """In-place SUM all-reduce of the weight gradients. Each rank's backward differentiates
     its own tokens' terms of <y, dy> + alpha L_bal + beta L_z with the whole-batch f_i and
-    token total, so the sum over ranks is the whole batch's gradient."""
+    token total, so the sum over ranks is the whole batch's gradient.
+
+    bf16 gradients (the expert weights') are summed in float32 and rounded to bf16 once:
+    each is widened into a float32 staging tensor, all-reduced, and written back. A bf16
+    all-reduce would round after every partial sum, so its error would grow with the
+    number of ranks; here it is one rounding of the float32 sum."""
     for k in keys:
         t = grads.get(k)
-        if t is not None and t.numel() > 0:
+        if t is None or t.numel() == 0:
+            continue
+        if t.dtype in (torch.bfloat16, torch.float16):
+            acc = t.to(torch.float32)
+            dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=group)
+            t.copy_(acc)
+        else:
             dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
     return grads
 
