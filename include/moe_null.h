@@ -132,7 +132,9 @@ typedef struct moe_outputs {
   uint16_t* h;          /* [R_cap, F] bf16 routed SwiGLU activations             */
   uint16_t* h_shared;   /* [T, F_shared] bf16 shared SwiGLU activations          */
   uint16_t* ys;         /* [R_cap, d] bf16 routed expert outputs                 */
-  uint16_t* shared_out; /* [T, d] bf16 shared expert output                      */
+  uint16_t* shared_out; /* [T, d] bf16 shared expert output, or NULL: the combine is
+                           then folded into the down GEMM (moe_expert_down_combine)
+                           and the shared expert's output is never written alone   */
   uint16_t* y;          /* [T, d] bf16 layer output                              */
   int32_t* counts_ext;  /* [N+M+C+V] tokens per pool slot                        */
   float* P;             /* [N+M+C+V] mean routing probability per pool slot      */
@@ -199,19 +201,32 @@ MOE_API int moe_route(const moe_dims_t* dims, const uint16_t* x, const float* w_
  * synchronise the device. The paper has no counterpart of this entry point; it
  * is a deployment convenience. Same inputs, outputs and results as moe_route.
  * Its internal scratch is a fixed MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES array in
- * the library's own device memory, held by every GPU that loads the library
- * until the process exits. Shapes whose moe_workspace_bytes exceeds that size
- * are rejected with MOE_ERR_UNSUPPORTED before anything is enqueued. The first
- * call on each device looks up the array's device address once; make that
- * first call before any stream capture. All calls on a device share the array
- * (each call clears what must start at zero): calls whose GPU work overlaps,
- * e.g. on two unordered streams, race and give wrong results. It allocates
- * nothing and does not fill a workspace for moe_dispatch. */
+ * the library's own device memory, held by every GPU that uses this entry
+ * point from its first call there until the process exits. Shapes whose
+ * moe_workspace_bytes exceeds that size are rejected with MOE_ERR_UNSUPPORTED
+ * before anything is enqueued. The first call on each device (and the first
+ * after the device's context was replaced, e.g. by cudaDeviceReset) looks up
+ * the array's device address; make that first call before any stream capture.
+ * All calls on a device share the array (each call clears what must start at
+ * zero): calls whose GPU work overlaps, e.g. on two unordered streams, race and
+ * give wrong results. It allocates nothing and does not fill a workspace for
+ * moe_dispatch. Device-side failures are recorded in the array's status word:
+ * read it with moe_route_noalloc_device_status. */
 #define MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES ((size_t)8 << 20)
 MOE_API int moe_route_noalloc(const moe_dims_t* dims, const uint16_t* x, const float* w_router,
                               const float* router_bias, const float* tok_null_bias, float* logits_out,
                               int32_t* topk_idx, float* topk_gate, int32_t* n_real,
                               moe_stream_t stream);
+
+/* Synchronises `stream`, then returns MOE_OK or the first device-side error that a
+ * moe_route_noalloc call on the current device recorded since the last call cleared
+ * it (MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_BOUNDS): the counterpart of
+ * moe_get_device_status for the entry point without a workspace. */
+MOE_API int moe_route_noalloc_device_status(moe_stream_t stream);
+
+/* Test aid, as moe_selftest_bounded_wait, recording into the status word that
+ * moe_route_noalloc_device_status reads; the next moe_route_noalloc call clears it. */
+MOE_API int moe_route_noalloc_selftest_bounded_wait(uint64_t limit_ns, moe_stream_t stream);
 
 /* Dispatch (section 三 / 实现: nulls sorted to the end and truncated). After
  * moe_route with the same workspace. counts [N], offsets [N+1]; the real slots
@@ -258,6 +273,51 @@ MOE_API int moe_expert_down(const moe_dims_t* dims, const int32_t* offsets, cons
                     const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* shared_down,
                     uint16_t* ys, uint16_t* shared_out, void* workspace, moe_stream_t stream);
 
+/* Expert parallelism (MoE tutorial page, 五、通信：All-to-All 为什么是成本中心: the
+ * experts are spread over the GPUs, a dispatch all-to-all sends each token's rows to
+ * the GPUs that hold its experts and a combine all-to-all brings the outputs back;
+ * MoE++ page, 局限性与开放问题 / 分布式部署复杂度: the zero-computation experts live on
+ * every GPU, so null slots are never sent). On the rank that holds a shard of the
+ * routed experts, these run the two grouped GEMMs over the rows it received:
+ *  - dims->N is the number of experts in the shard (the groups); dims->M and dims->K
+ *    play no part (pass 0 and 1);
+ *  - offsets [N+1] (device) delimit each expert's received rows, expert-contiguous;
+ *  - gate_up [N, 2F, d] (packed as by moe_pack_gate_up) and w_down [N, d, F] are the
+ *    shard's weights, e.g. pointers into the whole layer's at its first expert;
+ *  - rows_cap (>= 1) is the row count of xs, h and ys, independent of T*K: a rank can
+ *    receive up to world_size * T * K rows;
+ *  - the shared expert runs as usual over the rank's own dims->T tokens of x into
+ *    h_shared and shared_out (dims->T = 0: no shared expert, the routed rows still run).
+ * Same per-row results as moe_expert_gate_up / moe_expert_down (a row's output does
+ * not depend on which tile holds it). Single-CTA tiles. */
+MOE_API int moe_expert_gate_up_rows(const moe_dims_t* dims, int64_t rows_cap, const uint16_t* xs,
+                                    const uint16_t* x, const int32_t* offsets, const uint16_t* gate_up,
+                                    const uint16_t* shared_gate_up, uint16_t* h, uint16_t* h_shared,
+                                    void* workspace, moe_stream_t stream);
+MOE_API int moe_expert_down_rows(const moe_dims_t* dims, int64_t rows_cap, const int32_t* offsets,
+                                 const uint16_t* h, const uint16_t* h_shared, const uint16_t* w_down,
+                                 const uint16_t* shared_down, uint16_t* ys, uint16_t* shared_out,
+                                 void* workspace, moe_stream_t stream);
+
+/* moe_expert_down + moe_combine in one launch (section 三 / 核心公式): the down
+ * GEMM writes ys for the routed rows, and its shared-expert tiles, which come
+ * after every routed tile, write y[t] = bf16(bf16(shared[t]) + sum over the
+ * token's slots k, in rank order, of topk_gate[t,k] * out_k) with out_k as in
+ * moe_combine: the same arithmetic, so y is bit-identical to moe_expert_down
+ * followed by moe_combine, without the shared expert's output ever going to
+ * memory. A shared tile first waits (bounded; MOE_ERR_TIMEOUT in the status word
+ * if it runs out) until the launch's routed tiles have stored their rows, which
+ * relies on the persistent grid (one CTA per SM) being resident at once. The
+ * workspace must come from moe_route (which clears the two counters this call
+ * uses; the call leaves them cleared). Always single-CTA tiles. topk_idx, x and
+ * const_vectors are read only when C + V > 0. */
+MOE_API int moe_expert_down_combine(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* h,
+                                    const uint16_t* h_shared, const uint16_t* w_down,
+                                    const uint16_t* shared_down, uint16_t* ys, const float* topk_gate,
+                                    const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                                    const uint16_t* const_vectors, uint16_t* y, void* workspace,
+                                    moe_stream_t stream);
+
 /* Combine (section 三 / 核心公式): y[t] = bf16(shared_out[t] + sum over the
  * token's slots k, in rank order, of topk_gate[t,k] * out_k), out_k =
  * ys[slot_row[t,k]] for a real expert, x[t] for a copy expert, const_vectors[j]
@@ -291,6 +351,8 @@ MOE_API int moe_aux(const moe_dims_t* dims, const void* workspace, int32_t* coun
             float* losses, moe_stream_t stream);
 
 /* The whole forward: route, dispatch (+aux), expert FFNs, combine. With
+ * out->shared_out == NULL the combine runs inside the down GEMM
+ * (moe_expert_down_combine) and the forward is six launches. With
  * out->xs == NULL the routed rows are never copied: dispatch writes only the
  * permutation and gate/up gathers rows of x (moe_expert_gate_up_gather). With
  * out->z and out->z_shared set (training; xs required) the gate/up GEMM also

@@ -94,9 +94,10 @@ def test_full_size_layer_parity_sampled(name, router, ffn, xs):
 
 @pytest.mark.parametrize("name", ["sweep_k2_m0", "sweep_k3_m32", "sweep_k4_m64", "sweep_k8_m192", "skew"])
 def test_large_configs_routing_and_sampled_output(name):
+    """The combine inside the down GEMM, at the large workloads, against the oracle."""
     cfg = I.CONFIGS[name]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, out = H.run_forward(inp)
+    layer, x, tnb, out = H.run_forward(inp, shared_out=False)
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -115,7 +116,7 @@ def test_row_gather_matches_row_copy_bitwise(name):
     layer, x, tnb = H.make_layer(inp)
     outs = []
     for xs in (True, False):
-        out = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs))
+        out = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, shared_out=True))
         torch.cuda.synchronize()
         outs.append(out)
     R = int(outs[0]["offsets"][-1])
@@ -368,3 +369,58 @@ def test_repeated_calls_same_workspace_deterministic():
         layer.forward(x, tnb, out)
     torch.cuda.synchronize()
     assert torch.equal(out["y"], y1) and torch.equal(out["losses"], l1)
+
+
+# The combine folded into the down GEMM's shared-expert tiles (moe_expert_down_combine, what
+# the forward runs when no shared_out buffer is given) against the separate down GEMM and
+# combine launches: same arithmetic, so y must be bit-identical; every other output too.
+FUSED = [("tiny", "tensor", "single", True), ("ragged_b", "tensor", "single", True),
+         ("bn256", "tensor", "single", True), ("m0", "fp32_cores", "single", True),
+         ("n64_k16", "tensor", "single", False), ("skew_small", "tensor", "pair", True),
+         ("t1", "tensor", "single", True), ("pp_a", "tensor", "single", True), ("pp_b", "tensor", "single", True),
+         ("pp_80rows", "tensor", "single", True), ("qwen3_0p6b", "tensor", "single", True),
+         ("qwen3_1p7b", "tensor", "single", True), ("skew", "tensor", "single", True),
+         ("decode_0p6b", "tensor", "single", True)]
+
+
+@pytest.mark.parametrize("name,router,ffn,xs", FUSED)
+def test_combine_in_down_gemm_is_bitwise_the_separate_combine(name, router, ffn, xs):
+    cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP[name]
+    inp = I.make_inputs(cfg)
+    if cfg.C + cfg.V:
+        inp.bias[cfg.N] = np.float32(0.4)
+        inp.bias[cfg.N + 1:] = np.float32(0.6)
+    layer, x, tnb = H.make_layer(inp, router=router, ffn=ffn)
+    ref = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, shared_out=True))
+    outs = [layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, shared_out=False)) for _ in range(2)]  # counters reset
+    torch.cuda.synchronize()
+    from token_choice_routing_b200 import binding as B
+    R = int(ref["offsets"][-1])
+    for out in outs:
+        assert B.get_device_status(out["workspace"]) == B.OK
+        assert out["shared_out"] is None
+        for k in ("y", "topk_idx", "topk_gate", "counts", "offsets", "slot_row", "h_shared", "counts_ext", "P",
+                  "losses"):
+            assert torch.equal(out[k], ref[k]), k
+        for k in ("perm_tok", "h", "ys"):
+            assert torch.equal(out[k][:R], ref[k][:R]), k
+
+
+def test_down_combine_entry_point_called_alone_twice():
+    """moe_expert_down_combine on its own, twice in a row after one forward (its counters are
+    reset by the last CTA of each launch), gives the forward's y both times."""
+    from token_choice_routing_b200 import binding as B
+    cfg = I.CONFIGS["qwen3_0p6b"]
+    inp = I.make_inputs(cfg)
+    layer, x, tnb = H.make_layer(inp)
+    out = layer.forward(x, tnb, layer.alloc(cfg.T, shared_out=False))
+    torch.cuda.synchronize()
+    y0 = out["y"].clone()
+    dm = layer.dims(cfg.T)
+    for _ in range(2):
+        out["y"].zero_()
+        B.expert_down_combine(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down,
+                              out["ys"], out["topk_gate"], out["slot_row"], out["y"], out["workspace"])
+        torch.cuda.synchronize()
+        assert B.get_device_status(out["workspace"]) == B.OK
+        assert torch.equal(out["y"], y0)

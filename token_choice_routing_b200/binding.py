@@ -83,6 +83,9 @@ def _load() -> C.CDLL:
         "moe_expert_gate_up_gather": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_combine": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_down_combine": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_gate_up_rows": (i32, [pd, C.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_expert_down_rows": (i32, [pd, C.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_aux_sums_count": (sz, [pd]),
         "moe_aux_sums": (i32, [pd, vp, vp, vp]),
         "moe_aux_finalize": (i32, [pd, vp, vp, vp, vp, vp]),
@@ -91,6 +94,9 @@ def _load() -> C.CDLL:
         "moe_get_device_status": (i32, [vp, vp]),
         "moe_clear_device_status": (i32, [vp, vp]),
         "moe_selftest_bounded_wait": (i32, [vp, C.c_uint64, vp]),
+        "moe_route_noalloc": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_route_noalloc_device_status": (i32, [vp]),
+        "moe_route_noalloc_selftest_bounded_wait": (i32, [C.c_uint64, vp]),
         "moe_backward_workspace_bytes": (sz, [pd]),
         "moe_combine_backward": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_router_backward": (i32, [pd, vp, vp, vp, vp, vp, C.c_int64, C.c_float, C.c_float, vp, vp, vp, vp]),
@@ -211,6 +217,30 @@ def expert_down(dm, offsets, h, h_shared, w_down, shared_down, ys, shared_out, w
     _check("moe_expert_down", LIB.moe_expert_down(C.byref(dm), _p(offsets), _p(h), _p(h_shared), _p(w_down),
                                                   _p(shared_down), _p(ys), _p(shared_out), _p(ws),
                                                   _stream(stream)))
+
+
+def expert_gate_up_rows(dm, rows_cap, xs, x, offsets, gate_up, shared_gate_up, h, h_shared, ws, stream=None):
+    """Gate/up grouped GEMM of an expert shard over rows_cap received rows (expert parallelism)."""
+    _check("moe_expert_gate_up_rows",
+           LIB.moe_expert_gate_up_rows(C.byref(dm), int(rows_cap), _p(xs), _p(x), _p(offsets), _p(gate_up),
+                                       _p(shared_gate_up), _p(h), _p(h_shared), _p(ws), _stream(stream)))
+
+
+def expert_down_rows(dm, rows_cap, offsets, h, h_shared, w_down, shared_down, ys, shared_out, ws, stream=None):
+    """Down grouped GEMM of an expert shard over rows_cap received rows (expert parallelism)."""
+    _check("moe_expert_down_rows",
+           LIB.moe_expert_down_rows(C.byref(dm), int(rows_cap), _p(offsets), _p(h), _p(h_shared), _p(w_down),
+                                    _p(shared_down), _p(ys), _p(shared_out), _p(ws), _stream(stream)))
+
+
+def expert_down_combine(dm, offsets, h, h_shared, w_down, shared_down, ys, topk_gate, slot_row, y, ws,
+                        stream=None, topk_idx=None, x=None, const_vectors=None):
+    """Down GEMM with the combine in its shared-expert tiles (topk_idx, x and const_vectors
+    are needed only with MoE++ copy/constant experts)."""
+    _check("moe_expert_down_combine",
+           LIB.moe_expert_down_combine(C.byref(dm), _p(offsets), _p(h), _p(h_shared), _p(w_down), _p(shared_down),
+                                       _p(ys), _p(topk_gate), _p(slot_row), _p(topk_idx), _p(x),
+                                       _p(const_vectors), _p(y), _p(ws), _stream(stream)))
 
 
 def combine(dm, ys, shared_out, topk_gate, slot_row, y, stream=None, topk_idx=None, x=None,

@@ -160,6 +160,43 @@ int moe_expert_down(const moe_dims_t* dims, const int32_t* offsets, const uint16
   return launch_down(*dims, offsets, h, h_shared, w_down, shared_down, ys, shared_out, workspace, S(stream));
 }
 
+int moe_expert_gate_up_rows(const moe_dims_t* dims, int64_t rows_cap, const uint16_t* xs, const uint16_t* x,
+                            const int32_t* offsets, const uint16_t* gate_up, const uint16_t* shared_gate_up,
+                            uint16_t* h, uint16_t* h_shared, void* workspace, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (rows_cap < 1 || rows_cap >= (int64_t)INT_MAX) return rows_cap < 1 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
+  if (!xs || !offsets || !gate_up || !h || !workspace) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!x || !shared_gate_up || !h_shared)) return MOE_ERR_INVALID_ARG;
+  return launch_gate_up_rows(*dims, (long long)rows_cap, xs, x, offsets, gate_up, shared_gate_up, h, h_shared,
+                             workspace, S(stream));
+}
+
+int moe_expert_down_rows(const moe_dims_t* dims, int64_t rows_cap, const int32_t* offsets, const uint16_t* h,
+                         const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* shared_down, uint16_t* ys,
+                         uint16_t* shared_out, void* workspace, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (rows_cap < 1 || rows_cap >= (int64_t)INT_MAX) return rows_cap < 1 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
+  if (!offsets || !h || !w_down || !ys || !workspace) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!h_shared || !shared_down || !shared_out)) return MOE_ERR_INVALID_ARG;
+  return launch_down_rows(*dims, (long long)rows_cap, offsets, h, h_shared, w_down, shared_down, ys, shared_out,
+                          workspace, S(stream));
+}
+
+int moe_expert_down_combine(const moe_dims_t* dims, const int32_t* offsets, const uint16_t* h,
+                            const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* shared_down,
+                            uint16_t* ys, const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx,
+                            const uint16_t* x, const uint16_t* const_vectors, uint16_t* y, void* workspace,
+                            moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (dims->T == 0) return MOE_OK;
+  if (!offsets || !h || !h_shared || !w_down || !shared_down || !ys || !topk_gate || !slot_row || !y || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (dims->C + dims->V > 0 && (!topk_idx || (dims->C > 0 && !x) || (dims->V > 0 && !const_vectors)))
+    return MOE_ERR_INVALID_ARG;
+  return launch_down_combine(*dims, offsets, h, h_shared, w_down, shared_down, ys, topk_gate, slot_row, topk_idx, x,
+                             const_vectors, y, workspace, S(stream));
+}
+
 int moe_combine(const moe_dims_t* dims, const uint16_t* ys, const uint16_t* shared_out, const float* topk_gate,
                 const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x, const uint16_t* const_vectors,
                 uint16_t* y, moe_stream_t stream) {
@@ -202,8 +239,8 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
     return MOE_ERR_INVALID_ARG;
   if (dims->V > 0 && !w->const_vectors) return MOE_ERR_INVALID_ARG;
   if (!out->topk_idx || !out->topk_gate || !out->n_real || !out->counts || !out->offsets || !out->perm_tok ||
-      !out->slot_row || !out->h || !out->h_shared || !out->ys || !out->shared_out || !out->y ||
-      !out->counts_ext || !out->P || !out->losses)
+      !out->slot_row || !out->h || !out->h_shared || !out->ys || !out->y || !out->counts_ext || !out->P ||
+      !out->losses)
     return MOE_ERR_INVALID_ARG;
   // saved pre-activations: both buffers or neither, and only with the gathered copy xs
   if ((out->z != nullptr) != (out->z_shared != nullptr) || (out->z && !out->xs)) return MOE_ERR_INVALID_ARG;
@@ -221,6 +258,10 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
     MOE_CHECK(launch_gate_up_perm(*dims, out->xs, x, out->offsets, out->xs ? nullptr : out->perm_tok, w->gate_up,
                                   w->shared_gate_up, out->h, out->h_shared, workspace, st));
   }
+  if (out->shared_out == nullptr)  // the combine runs in the down GEMM's shared-expert tiles
+    return launch_down_combine(*dims, out->offsets, out->h, out->h_shared, w->w_down, w->shared_down, out->ys,
+                               out->topk_gate, out->slot_row, out->topk_idx, x, w->const_vectors, out->y,
+                               workspace, st);
   MOE_CHECK(launch_down(*dims, out->offsets, out->h, out->h_shared, w->w_down, w->shared_down, out->ys,
                         out->shared_out, workspace, st));
   return launch_combine(*dims, out->ys, out->shared_out, out->topk_gate, out->slot_row, out->topk_idx, x,

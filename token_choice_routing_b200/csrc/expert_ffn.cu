@@ -21,6 +21,17 @@
 // row; those rows are computed but never stored). Tiles are handed out
 // round-robin (all tiles of a GEMM have the same cost). Every wait is bounded.
 //
+// Combine folded into the down GEMM (COMBINE): the shared expert's tiles come after every
+// routed tile in the tile order, so their epilogue can finish the layer: y[t] =
+// bf16(shared[t]) + sum over the token's slots, in rank order, of g * ys[slot_row] (fp32,
+// one rounding; the same arithmetic as moe_combine, so y is bit-identical). Each routed
+// tile's epilogue publishes its stored rows with a release increment of a counter in the
+// workspace; before its first shared tile a CTA's epilogue waits (bounded) until the
+// counter holds every routed tile. The grid is persistent (one CTA per SM, at most one
+// per SM) and each CTA takes its tiles in increasing order, so the CTA that owns a routed
+// tile never waits before finishing it: the wait cannot deadlock while the grid is
+// resident. The last CTA to exit resets the counters for the next launch.
+//
 // Row gather (gate/up with a token permutation): instead of reading routed rows
 // from a gathered copy xs, the producer warp copies them from x with 16-byte
 // cp.async loads (4 rows per pass, 8 lanes per row) straight into the
@@ -63,6 +74,18 @@ struct GemmArgs {
   int ldz_r;
   uint16_t* zout_s;        // SAVEZ: the shared expert's [T, 2F_shared]
   int ldz_s;
+  // COMBINE: the shared tiles' epilogue writes y from the shared expert's output and the
+  // token's slots (source of slot k: slot_row >= 0 a row of out_r = ys; else, with MoE++
+  // experts, topk_idx tells a copy expert (row of cx) or constant expert j (row j of cv))
+  const int32_t* slot_row;  // [T, K]
+  const float* gate;        // [T, K]
+  const int32_t* topk_idx;  // [T, K] (read only when C + V > 0)
+  const uint16_t* cx;       // [T, d] the layer input (copy experts)
+  const uint16_t* cv;       // [V, d] constant experts' vectors
+  uint16_t* y;              // [T, d]
+  int K, NM, C, V;
+  uint32_t* tiles_done;     // routed tiles whose rows are stored (workspace header)
+  uint32_t* cta_exits;      // CTAs that have exited (the last resets both counters)
 };
 
 template <int BN>
@@ -85,7 +108,93 @@ struct TileInfo {
   int g, arow, mvalid, brow, nkb, col0;
 };
 
-template <int BN, bool SWIGLU, bool GATHER, bool SAVEZ = false>
+__device__ __forceinline__ void fma8(float (&acc)[8], float g, const uint4& v) {
+  acc[0] = fmaf(g, bf16lo(v.x), acc[0]); acc[1] = fmaf(g, bf16hi(v.x), acc[1]);
+  acc[2] = fmaf(g, bf16lo(v.y), acc[2]); acc[3] = fmaf(g, bf16hi(v.y), acc[3]);
+  acc[4] = fmaf(g, bf16lo(v.z), acc[4]); acc[5] = fmaf(g, bf16hi(v.z), acc[5]);
+  acc[6] = fmaf(g, bf16lo(v.w), acc[6]); acc[7] = fmaf(g, bf16hi(v.w), acc[7]);
+}
+
+// Combine in a shared tile (COMBINE), one thread per tile row (its TMEM lane), the token
+// t = arow + row. combine_sources: the token's slots in rank order, compacted to the ones
+// with an output (a row of ys, written by this launch's routed tiles; x for a copy expert;
+// a constant vector), coded as in moe_combine (>= 0 ys row, -2 x row, -3 - j constant j),
+// into this thread's own entries of src/gw. combine_chunk: 64 columns of the row: the
+// shared expert's bf16 values plus the sources' in rank order, fp32, one rounding.
+__device__ __forceinline__ int combine_sources(const GemmArgs& a, int t, int* src, float* gw) {
+  const int K = a.K;
+  int n = 0;
+  for (int k = 0; k < K; ++k) {
+    int r = __ldg(a.slot_row + (size_t)t * K + k);
+    const float g = __ldg(a.gate + (size_t)t * K + k);
+    if (r >= a.rows_cap) {
+      atomicOr(a.status, kStatusBounds);
+      r = -1;
+    }
+    if (r < 0 && a.C + a.V > 0) {
+      const int id = __ldg(a.topk_idx + (size_t)t * K + k) - a.NM;  // among copy/constant experts
+      if (id >= 0 && id < a.C) r = -2;
+      else if (id >= a.C && id < a.C + a.V) r = -3 - (id - a.C);
+    }
+    if (r != -1) {
+      src[n] = r;
+      gw[n] = g;
+      ++n;
+    }
+  }
+  return n;
+}
+
+__device__ __forceinline__ const uint4* combine_src_ptr(const GemmArgs& a, int code, int t, int col) {
+  const uint16_t* p = (code >= 0) ? a.out_r + (size_t)code * a.ld_r
+                      : (code == -2) ? a.cx + (size_t)t * a.ld_s
+                                     : a.cv + (size_t)(-3 - code) * a.ld_s;
+  return reinterpret_cast<const uint4*>(p + col);
+}
+
+__device__ __forceinline__ void combine_chunk(const GemmArgs& a, const uint32_t (&sh)[64], int t, int col, int n,
+                                              const int* src, const float* gw) {
+  float acc[64];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t p = pack_bf16x2(__uint_as_float(sh[2 * j]), __uint_as_float(sh[2 * j + 1]));
+    acc[2 * j] = bf16lo(p);
+    acc[2 * j + 1] = bf16hi(p);
+  }
+  // two sources per pass: all their 16-byte pieces are loaded before either is added
+#pragma unroll 1
+  for (int i = 0; i < n; i += 2) {
+    const bool two = i + 1 < n;
+    uint4 v0[8], v1[8];
+    const uint4* p0 = combine_src_ptr(a, src[i], t, col);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v0[j] = __ldcg(p0 + j);
+    if (two) {
+      const uint4* p1 = combine_src_ptr(a, src[i + 1], t, col);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v1[j] = __ldcg(p1 + j);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float (&c8)[8] = *reinterpret_cast<float(*)[8]>(acc + 8 * j);
+      fma8(c8, gw[i], v0[j]);
+    }
+    if (two) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float (&c8)[8] = *reinterpret_cast<float(*)[8]>(acc + 8 * j);
+        fma8(c8, gw[i + 1], v1[j]);
+      }
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)t * a.ld_s + col);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    dst[j] = make_uint4(pack_bf16x2(acc[8 * j + 0], acc[8 * j + 1]), pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
+                        pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]), pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
+}
+
+template <int BN, bool SWIGLU, bool GATHER, bool SAVEZ = false, bool COMBINE = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
                     const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s,
@@ -343,14 +452,53 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;      // tile row held by this thread
     const int etid = (warp - 2) * 32 + lane;
+    bool routed_done = false;
     int li = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++li) {
       const TileInfo ti = decode(tile);
       const int acc = li & 1;
       const uint32_t ap = (uint32_t)(li >> 1) & 1u;
       if (!mbar_wait_bounded(tfull_bar(acc), ap, a.limit_ns, abort_flag, a.status)) break;
+      const bool comb = COMBINE && ti.g == N;
+      if constexpr (COMBINE) {
+        if (comb && !routed_done) {
+          // every routed tile's ys rows must be stored before a shared tile combines them
+          int ok = 1;
+          if (etid == 0)
+            ok = counter_wait_bounded(a.tiles_done, (uint32_t)s_tstart[N], a.limit_ns, abort_flag, a.status);
+          if (!named_bar_and(1, 128, ok != 0)) break;
+          routed_done = true;
+        }
+      }
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      if constexpr (COMBINE && !SWIGLU) {
+        if (comb) {
+          // thread-per-row combine: no staging; the staging rows hold each thread's own
+          // compacted slot list instead (16 sources x 8 B per row fits in a 144-byte row)
+          int* src = reinterpret_cast<int*>(stg + row * kStgRow);
+          float* gw = reinterpret_cast<float*>(stg + row * kStgRow + 64);
+          const int t = ti.arow + row;
+          const bool live = row < ti.mvalid;
+          const int n = live ? combine_sources(a, t, src, gw) : 0;
+#pragma unroll 1
+          for (int c = 0; c < NCHUNK; ++c) {
+            uint32_t r[64];
+#pragma unroll
+            for (int g16 = 0; g16 < 4; ++g16) {
+              uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(r + 16 * g16);
+              tmem_ld16(tb + (uint32_t)(c * 64 + g16 * 16), r16);
+            }
+            tmem_ld_wait();
+            if (c == NCHUNK - 1) {
+              tc_fence_before();
+              mbar_arrive(tempty_bar(acc));  // TMEM buffer free for the next-but-one tile
+            }
+            if (live) combine_chunk(a, r, t, ti.col0 + c * 64, n, src, gw);
+          }
+          continue;
+        }
+      }
       uint16_t* out = (ti.g < N) ? a.out_r : a.out_s;
       const int ld = (ti.g < N) ? a.ld_r : a.ld_s;
 #pragma unroll 1
@@ -418,7 +566,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             *reinterpret_cast<uint4*>(out + (size_t)(ti.arow + r) * ld + ti.col0 + c * 64 + ch * 8) = v;
           }
         }
+        if (COMBINE && c == NCHUNK - 1) __threadfence();  // this routed tile's rows, before the release
         named_bar_sync(1, 128);
+      }
+      if (COMBINE && etid == 0) red_add_release_gpu(a.tiles_done, 1u);
+    }
+  }
+
+  if constexpr (COMBINE) {
+    // the last CTA out resets the counters for the next launch (every CTA has passed its
+    // waits by the time it exits)
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(a.cta_exits, 1u) == gridDim.x - 1) {
+        atomicExch(a.tiles_done, 0u);
+        atomicExch(a.cta_exits, 0u);
       }
     }
   }
@@ -497,7 +660,7 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU, bool GATHER, bool SAVEZ = false>
+template <int BN, bool SWIGLU, bool GATHER, bool SAVEZ = false, bool COMBINE = false>
 static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUtensorMap& as_,
                        const CUtensorMap& bs, const GemmArgs& a, long long max_tiles, cudaStream_t st) {
   using SM = GemmSmem<BN>;
@@ -505,16 +668,18 @@ static int launch_gemm(const CUtensorMap& ar, const CUtensorMap& br, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, SWIGLU, GATHER, SAVEZ>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, SWIGLU, GATHER, SAVEZ, COMBINE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::bytes);
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
   }
+  // persistent: at most one CTA per SM (the shared memory allows no second), so with COMBINE
+  // every CTA is resident at once and the shared tiles' wait on the routed tiles cannot stall
   long long grid = sm_count();
   if (max_tiles < grid) grid = max_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(grouped_gemm_kernel<BN, SWIGLU, GATHER, SAVEZ>, dim3((unsigned)grid), dim3(kGemmThreads), SM::bytes, st, ar, br,
-                    as_, bs, a);
+  return launch_pdl(grouped_gemm_kernel<BN, SWIGLU, GATHER, SAVEZ, COMBINE>, dim3((unsigned)grid),
+                    dim3(kGemmThreads), SM::bytes, st, ar, br, as_, bs, a);
 }
 
 struct FfnPlan {
@@ -523,10 +688,12 @@ struct FfnPlan {
   GemmArgs g1, g2;
 };
 
-static FfnPlan plan_ffn(const moe_dims_t& d, const int32_t* offsets, void* ws) {
+// rows_cap: rows of the routed A/output buffers; by default the layer's R_cap = T K (the
+// expert-parallel calls pass the rows a rank received instead)
+static FfnPlan plan_ffn(const moe_dims_t& d, const int32_t* offsets, void* ws, long long rows_cap = -1) {
   const WsLayout L = ws_layout(d);
   FfnPlan p{};
-  const long long rcap = (long long)d.T * d.K;
+  const long long rcap = rows_cap >= 0 ? rows_cap : (long long)d.T * d.K;
   p.BN1 = (d.F % 128 == 0 && d.F_shared % 128 == 0) ? 256 : 128;
   p.BN2 = (d.d % 256 == 0) ? 256 : 128;
   const long long mtiles_r = rcap / kBM + d.N;  // sum_e ceil(m_e/128) <= R/128 + N
@@ -631,6 +798,90 @@ int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, 
         make_tmap_bf16(&as_, h_shared, d.T, d.F_shared, kBM) &&
         make_tmap_bf16(&bs, sdown, d.d, d.F_shared, p.BN2)))
     return MOE_ERR_CUDA;
+  p.g2.out_r = ys;
+  p.g2.out_s = shared_out;
+  return (p.BN2 == 256) ? launch_gemm<256, false, false>(ar, br, as_, bs, p.g2, p.max2, st)
+                        : launch_gemm<128, false, false>(ar, br, as_, bs, p.g2, p.max2, st);
+}
+
+// The down GEMM with the combine folded into its shared-expert tiles: ys for the routed
+// rows, and y = bf16(shared) + sum_k g ys (and the MoE++ copy / constant terms) for every
+// token; shared_out is not written. Single-CTA tiles (the CTA-pair flag does not apply).
+int launch_down_combine(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
+                        const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys, const float* topk_gate,
+                        const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                        const uint16_t* const_vectors, uint16_t* y, void* ws, cudaStream_t st) {
+  FfnPlan p = plan_ffn(d, offsets, ws);
+  const long long rcap = (long long)d.T * d.K;
+  CUtensorMap ar, br, as_, bs;
+  if (!(make_tmap_bf16(&ar, h, rcap, d.F, kBM) &&
+        make_tmap_bf16(&br, w_down, (uint64_t)d.N * d.d, d.F, p.BN2) &&
+        make_tmap_bf16(&as_, h_shared, d.T, d.F_shared, kBM) &&
+        make_tmap_bf16(&bs, sdown, d.d, d.F_shared, p.BN2)))
+    return MOE_ERR_CUDA;
+  const WsLayout L = ws_layout(d);
+  GemmArgs& g = p.g2;
+  g.out_r = ys;
+  g.out_s = nullptr;
+  g.slot_row = slot_row;
+  g.gate = topk_gate;
+  g.topk_idx = topk_idx;
+  g.cx = x;
+  g.cv = const_vectors;
+  g.y = y;
+  g.K = d.K;
+  g.NM = d.N + d.M;
+  g.C = d.C;
+  g.V = d.V;
+  g.tiles_done = ws_ptr<uint32_t>(ws, L.hdr + kHdrCombineOffset);
+  g.cta_exits = g.tiles_done + 1;
+  return (p.BN2 == 256) ? launch_gemm<256, false, false, false, true>(ar, br, as_, bs, g, p.max2, st)
+                        : launch_gemm<128, false, false, false, true>(ar, br, as_, bs, g, p.max2, st);
+}
+
+// Expert parallelism: the grouped GEMMs of one rank's expert shard over the rows it
+// received (rows_cap of them at most, expert-contiguous by offsets[0..N]), with the shared
+// expert over this rank's own T tokens. Single-CTA tiles.
+int launch_gate_up_rows(const moe_dims_t& d, long long rows_cap, const uint16_t* xs, const uint16_t* x,
+                        const int32_t* offsets, const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h,
+                        uint16_t* h_shared, void* ws, cudaStream_t st) {
+  FfnPlan p = plan_ffn(d, offsets, ws, rows_cap);
+  CUtensorMap ar, br, as_, bs;
+  if (!(make_tmap_bf16(&ar, xs, (uint64_t)rows_cap, d.d, kBM) &&
+        make_tmap_bf16(&br, gate_up, (uint64_t)d.N * 2 * d.F, d.d, p.BN1)))
+    return MOE_ERR_CUDA;
+  if (d.T == 0) {  // a rank without tokens of its own: routed rows only (the shared maps go unused)
+    p.g1.has_shared = 0;
+    as_ = ar;
+    bs = br;
+  } else if (!(make_tmap_bf16(&as_, x, d.T, d.d, kBM) &&
+               make_tmap_bf16(&bs, sgate_up, (uint64_t)2 * d.F_shared, d.d, p.BN1))) {
+    return MOE_ERR_CUDA;
+  }
+  p.g1.out_r = h;
+  p.g1.out_s = h_shared;
+  p.g1.x = x;
+  p.g1.ld_x = d.d;
+  return (p.BN1 == 256) ? launch_gemm<256, true, false>(ar, br, as_, bs, p.g1, p.max1, st)
+                        : launch_gemm<128, true, false>(ar, br, as_, bs, p.g1, p.max1, st);
+}
+
+int launch_down_rows(const moe_dims_t& d, long long rows_cap, const int32_t* offsets, const uint16_t* h,
+                     const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys,
+                     uint16_t* shared_out, void* ws, cudaStream_t st) {
+  FfnPlan p = plan_ffn(d, offsets, ws, rows_cap);
+  CUtensorMap ar, br, as_, bs;
+  if (!(make_tmap_bf16(&ar, h, (uint64_t)rows_cap, d.F, kBM) &&
+        make_tmap_bf16(&br, w_down, (uint64_t)d.N * d.d, d.F, p.BN2)))
+    return MOE_ERR_CUDA;
+  if (d.T == 0) {
+    p.g2.has_shared = 0;
+    as_ = ar;
+    bs = br;
+  } else if (!(make_tmap_bf16(&as_, h_shared, d.T, d.F_shared, kBM) &&
+               make_tmap_bf16(&bs, sdown, d.d, d.F_shared, p.BN2))) {
+    return MOE_ERR_CUDA;
+  }
   p.g2.out_r = ys;
   p.g2.out_s = shared_out;
   return (p.BN2 == 256) ? launch_gemm<256, false, false>(ar, br, as_, bs, p.g2, p.max2, st)

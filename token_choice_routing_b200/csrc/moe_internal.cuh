@@ -31,6 +31,12 @@ constexpr uint32_t kStatusBounds = 2u;
 
 // Byte offset of the per-expert row totals inside the workspace header.
 constexpr size_t kHdrTotOffset = 16;
+// Byte offset of the two counters of the down GEMM with the combine folded in: routed
+// tiles whose ys rows are stored, and CTAs that have exited (the last one resets both).
+constexpr size_t kHdrCombineOffset = 448;
+// Bytes of the header that every route call clears: status word, per-expert totals and
+// the down GEMM's counters.
+constexpr size_t kHdrClearBytes = kHdrCombineOffset + 8;
 
 // Default limit of every device-side wait, in ns of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -256,6 +262,16 @@ int launch_gate_up(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, c
 int launch_down(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
                 const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys, uint16_t* shared_out, void* ws,
                 cudaStream_t st);
+int launch_gate_up_rows(const moe_dims_t& d, long long rows_cap, const uint16_t* xs, const uint16_t* x,
+                        const int32_t* offsets, const uint16_t* gate_up, const uint16_t* sgate_up, uint16_t* h,
+                        uint16_t* h_shared, void* ws, cudaStream_t st);
+int launch_down_rows(const moe_dims_t& d, long long rows_cap, const int32_t* offsets, const uint16_t* h,
+                     const uint16_t* h_shared, const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys,
+                     uint16_t* shared_out, void* ws, cudaStream_t st);
+int launch_down_combine(const moe_dims_t& d, const int32_t* offsets, const uint16_t* h, const uint16_t* h_shared,
+                        const uint16_t* w_down, const uint16_t* sdown, uint16_t* ys, const float* topk_gate,
+                        const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                        const uint16_t* const_vectors, uint16_t* y, void* ws, cudaStream_t st);
 int launch_pack_gate_up(const moe_dims_t& d, const uint16_t* w_gate, const uint16_t* w_up,
                         const uint16_t* ws_gate, const uint16_t* ws_up, uint16_t* gate_up,
                         uint16_t* sgate_up, cudaStream_t st);
@@ -376,6 +392,36 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Release / acquire accesses of a counter in global memory (gpu scope).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait until the counter *p reaches `target` (acquire). Returns false (and records
+// a timeout in *status) if `limit_ns` passed, or if *abort became non-zero meanwhile.
+__device__ __forceinline__ bool counter_wait_bounded(const uint32_t* p, uint32_t target,
+                                                     unsigned long long limit_ns, volatile int* abort,
+                                                     uint32_t* status) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      if (status) atomicOr(status, kStatusTimeout);
+      if (abort) *abort = 1;
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x,
                                             int y) {
   asm volatile(
@@ -451,6 +497,21 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// bar.red.and over a named barrier: every participating thread gets the AND
+// of all their predicates (a CTA-uniform decision among those threads).
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // Shared-memory matrix descriptor (tcgen05) for a K-major tile whose rows are

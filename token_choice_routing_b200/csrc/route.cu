@@ -25,11 +25,14 @@
 // fp32: the same error bound as an fp32 dot product of length d, with two
 // more roundings.
 //
-// Layout: one CTA = 128 tokens x all N+1 logits (one M=128 tile). Warp 0
-// issues TMA loads of the x tile (128 x 64 bf16) and the split weight tile
-// (3*NPW x 64 bf16) into a 4-stage ring; warp 1 issues the MMAs (M=128,
-// N=3*NPW, K=16) from one thread into TMEM; warps 2-17 add the three terms per
-// logit, then route the 128 tokens with 4 lanes per token.
+// Layout: a persistent CTA per SM takes tiles of 128 tokens x all N+1 logits (one
+// M=128 MMA tile each) in turn. Warp 0 issues TMA loads of the x tile (128 x 64
+// bf16) and the split weight tile (3*NPW x 64 bf16) into a 3-stage ring, running
+// ahead across tiles; warp 1 issues the MMAs (M=128, N=3*NPW, K=16) from one
+// thread into one of two TMEM accumulators; warps 2-17 add the three terms per
+// logit into shared memory (which frees the accumulator for the tile after next),
+// then route the 128 tokens with 4 lanes per token while the next tile's product
+// is already running.
 #include "moe_internal.cuh"
 
 #include <climits>
@@ -76,8 +79,9 @@ __device__ __forceinline__ void split3(float w, uint16_t& h, uint16_t& m, uint16
 }
 
 // One thread per 8 d-columns of one padded row. Block 0 also clears the first
-// `nclear` words of the workspace header (status word and per-expert totals),
-// which must start at zero for every layer call.
+// `nclear` words of the workspace header (status word, per-expert totals and the
+// counters of the down GEMM with the combine folded in), which must start at zero
+// for every layer call.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, uint16_t* __restrict__ w3,
                                                            int rows, int npw, int d, uint32_t* hdr, int nclear) {
   pdl_wait_then_release();
@@ -111,12 +115,12 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
 }
 
 // ---------------------------------------------------------------------------------------
-// Shared memory of the route kernel. The routing scratch aliases the staging
-// ring: it is written only after the last MMA has completed (its commit is
-// what releases the epilogue), and every issued TMA copy was consumed by an MMA.
+// Shared memory of the route kernel: a 3-stage ring of x and split-weight tiles, and the
+// routing scratch of the epilogue beside it (not aliased: the epilogue of one tile runs
+// while the ring already fills for the next).
 template <int NPW>
 struct RouteSmem {
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 3;
   static constexpr int BROWS = 3 * NPW;
   static constexpr int A_BYTES = kRouteTokens * kRouteBK * 2;
   static constexpr int B_BYTES = BROWS * kRouteBK * 2;
@@ -125,7 +129,7 @@ struct RouteSmem {
   static constexpr size_t ring_end = off_b + (size_t)STAGES * B_BYTES;
   // routing scratch
   static constexpr int LS = NPW + 1;  // odd row stride of the logit rows
-  static constexpr size_t off_s = 0;  // float [128][LS]: logits, then p in place
+  static constexpr size_t off_s = ring_end;  // float [128][LS]: logits, then p in place
   static constexpr size_t off_pn = off_s + sizeof(float) * kRouteTokens * LS;  // float [128] null p
   static constexpr size_t off_lse2 = off_pn + sizeof(float) * kRouteTokens;    // float [128]
   static constexpr size_t off_mask = align_up(off_lse2 + sizeof(float) * kRouteTokens, 16);  // u64 [128]
@@ -135,10 +139,11 @@ struct RouteSmem {
   static constexpr int HIST = kMaxK + 1 + kMaxPP;  // null histogram + copy/constant counts
   static constexpr size_t off_hist = off_tokbits + sizeof(unsigned) * 4 * kMaxN;         // int [HIST]
   static constexpr size_t scratch_end = off_hist + sizeof(int) * HIST;
-  static_assert(scratch_end <= ring_end, "routing scratch must fit in the staging ring");
-  static constexpr size_t off_bar = ring_end;  // full[STAGES], empty[STAGES], tfull
-  static constexpr size_t off_misc = off_bar + 8 * (2 * STAGES + 1);  // [0] TMEM base, [1] abort
+  // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  static constexpr size_t off_bar = align_up(scratch_end, 8);
+  static constexpr size_t off_misc = off_bar + 8 * (2 * STAGES + 5);  // [0] TMEM base, [1] abort
   static constexpr size_t bytes = off_misc + 16 + 1024;  // + slack for 1024-byte alignment
+  static_assert(bytes <= 227 * 1024, "route kernel shared memory");
 };
 
 // (value desc, index asc) order: true if (va, ia) precedes (vb, ib).
@@ -146,23 +151,10 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return va > vb || (va == vb && ia < ib);
 }
 
-// bar.red.and over a named barrier: every participating thread gets the AND
-// of all their predicates (a CTA-uniform decision among those threads).
-__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 // ---------------------------------------------------------------------------------------
-// One CTA: tokens [128 b, 128 b + 128) x all N+1 logits, 576 threads.
+// Persistent: one CTA per SM (at most), 576 threads, taking 128-token tiles b = blockIdx.x,
+// blockIdx.x + gridDim.x, ... (tokens [128 b, 128 b + 128) x all router rows each). Two
+// TMEM accumulators: the MMA of tile i+1 runs while the epilogue routes tile i.
 // NQ: logit columns per lane (4 lanes per token): NPW / 4, or 16 when NPW = 80 and
 // there are no copy/constant experts (the candidates are then the reals, columns < 64).
 template <int NPW, int NQ>
@@ -173,7 +165,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   using SM = RouteSmem<NPW>;
   constexpr int STAGES = SM::STAGES;
   constexpr int LS = SM::LS;
-  constexpr uint32_t TCOLS = SM::BROWS <= 64 ? 64u : SM::BROWS <= 128 ? 128u : 256u;
+  constexpr uint32_t ACOLS = SM::BROWS <= 64 ? 64u : SM::BROWS <= 128 ? 128u : 256u;  // per accumulator
+  constexpr uint32_t TCOLS = 2 * ACOLS;
   constexpr uint32_t IDESC = idesc_bf16_f32(kRouteTokens, SM::BROWS);
   constexpr uint32_t TX = SM::A_BYTES + SM::B_BYTES;
 
@@ -186,15 +179,15 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   volatile int* misc = reinterpret_cast<volatile int*>(base + SM::off_misc);
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
-  const uint32_t tfull_bar = smem_u32(bars + 2 * STAGES);
+  auto tfull_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + s); };
+  auto tempty_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + 2 + s); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * STAGES + 4);
   volatile int* abort_flag = misc + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x;
   const int T = a.T, N = a.N, M = a.M, K = a.K;
-  const int tok0 = b * kRouteTokens;
-  const int nvalid = min(kRouteTokens, T - tok0);
   const int nkb = a.d / kRouteBK;
+  const int ntile = a.nblk;
 
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmX);
@@ -203,7 +196,11 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    mbar_init(tfull_bar, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(tfull_bar(s), 1);
+      mbar_init(tempty_bar(s), kRouteEpiThreads);
+    }
+    mbar_init(drain_bar, 1);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -218,17 +215,27 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------ TMA producer
+      // ------------------------------ TMA producer (runs ahead across tiles)
+      int stage = 0;
+      uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, a.limit_ns, abort_flag, a.hdr)) break;
-        mbar_arrive_expect_tx(full_bar(s), TX);
-        tma_load_2d(smem_u32(sA + s * SM::A_BYTES), &tmX, full_bar(s), kb * kRouteBK, tok0);
-        tma_load_2d(smem_u32(sB + s * SM::B_BYTES), &tmW, full_bar(s), kb * kRouteBK, 0);
-        armed |= 1u << s;
-        armed_par = (armed_par & ~(1u << s)) | (ph << s);
+      bool ok = true;
+      for (int b = blockIdx.x; b < ntile && ok; b += gridDim.x) {
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, a.limit_ns, abort_flag, a.hdr)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), TX);
+          tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), &tmX, full_bar(stage), kb * kRouteBK, b * kRouteTokens);
+          tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), &tmW, full_bar(stage), kb * kRouteBK, 0);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
       }
       if (*abort_flag) {
         // let every issued copy land before the CTA can exit
@@ -240,25 +247,42 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------ MMA issuer (single thread)
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait_bounded(full_bar(s), ph, a.limit_ns, abort_flag, a.hdr)) break;
+      int stage = 0;
+      uint32_t phase = 0;
+      int li = 0;
+      bool ok = true;
+      for (int b = blockIdx.x; b < ntile && ok; b += gridDim.x, ++li) {
+        const int acc = li & 1;
+        const uint32_t ap = (uint32_t)(li >> 1) & 1u;
+        if (!mbar_wait_bounded(tempty_bar(acc), ap ^ 1u, a.limit_ns, abort_flag, a.hdr)) break;
         tc_fence_after();
-        const uint64_t adesc = smem_desc_sw128(smem_u32(sA + s * SM::A_BYTES));
-        const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * SM::B_BYTES));
+        const uint32_t d_tmem = tmem_base + (uint32_t)acc * ACOLS;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, a.limit_ns, abort_flag, a.hdr)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * SM::A_BYTES));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * SM::B_BYTES));
 #pragma unroll
-        for (int k = 0; k < kRouteBK / 16; ++k)
-          tc_mma_f16(tmem_base, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
-                     (kb | k) != 0 ? 1u : 0u);
-        tc_commit(empty_bar(s));
+          for (int k = 0; k < kRouteBK / 16; ++k)
+            tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
+                       (kb | k) != 0 ? 1u : 0u);
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit(tfull_bar(acc));
       }
       // fires once every MMA issued above has completed (also after an abort)
-      tc_commit(tfull_bar);
-      (void)mbar_wait_bounded(tfull_bar, 0, a.limit_ns, nullptr, a.hdr);
+      tc_commit(drain_bar);
+      (void)mbar_wait_bounded(drain_bar, 0, a.limit_ns, nullptr, a.hdr);
     }
   } else {
-    // ------------------------------ epilogue warps 2..17
+    // ------------------------------ epilogue warps 2..17, one tile after another
     const int etid = threadIdx.x - 64;  // 0..511
     const int ew = warp - 2;            // 0..15
     float* s_l = reinterpret_cast<float*>(base + SM::off_s);
@@ -269,18 +293,23 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     float* tkv = reinterpret_cast<float*>(base + SM::off_tkv);
     unsigned* tokbits = reinterpret_cast<unsigned*>(base + SM::off_tokbits);  // [4][kMaxN]
     int* s_hist = reinterpret_cast<int*>(base + SM::off_hist);                // [kMaxK+1]
-
-    const bool ok = mbar_wait_bounded(tfull_bar, 0, a.limit_ns, abort_flag, a.hdr) && *abort_flag == 0;
-    const bool run = named_bar_and(1, kRouteEpiThreads, ok);
-    if (run) {
+    int li = 0;
+    for (int b = blockIdx.x; b < ntile; b += gridDim.x, ++li) {
+    const int acc = li & 1;
+    const uint32_t ap = (uint32_t)(li >> 1) & 1u;
+    const int tok0 = b * kRouteTokens;
+    const int nvalid = min(kRouteTokens, T - tok0);
+    const bool ok = mbar_wait_bounded(tfull_bar(acc), ap, a.limit_ns, abort_flag, a.hdr) && *abort_flag == 0;
+    if (!named_bar_and(1, kRouteEpiThreads, ok)) break;
+    {
       // ---- logits from TMEM: warp reads lane quarter q (tokens 32q..32q+31) and
       // every fourth 8-column chunk; s_j = (hi_j + mid_j) + lo_j (+ bias)
       tc_fence_after();
       const int q = warp & 3, part = ew >> 2;
       const int t = q * 32 + lane;
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACOLS;
       const float tn = (a.tnb != nullptr && t < nvalid) ? __ldg(a.tnb + tok0 + t) : 0.f;
-      if (etid < SM::HIST) s_hist[etid] = 0;  // the staging ring is free from here on
+      if (etid < SM::HIST) s_hist[etid] = 0;
 #pragma unroll 1
       for (int c0 = part * 8; c0 < NPW; c0 += 32) {
         uint32_t rh[8], rm[8], rl[8];
@@ -299,10 +328,12 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           }
         }
       }
+      // the accumulator is free for the tile after next
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
     }
     named_bar_sync(1, kRouteEpiThreads);
-
-    if (run) {
+    {
       // ---- per-token routing, 4 lanes per token. Lane q holds the distinct candidates
       // in logit columns i = q, q+4, ...: reals (i < N, pool index i) and MoE++ copy and
       // constant experts (N < i < ncols, pool index i - 1 + M); column N is the null logit.
@@ -437,7 +468,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     }
     named_bar_sync(1, kRouteEpiThreads);
 
-    if (run) {
+    {
       // ---- block statistics. Ballots: warp ew takes the 32 tokens of group ew & 3
       // and experts [16 (ew >> 2), +16); bit e of the selection masks gives the
       // block's tokens that chose e as a 128-bit set (a slot's rank is the number
@@ -476,7 +507,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     }
     named_bar_sync(1, kRouteEpiThreads);
 
-    if (run) {
+    {
       const int hc = K + 1 + (a.ncols - N - 1);  // null histogram, then copy/constant counts
       if (etid < hc) a.hist[(size_t)b * hc + etid] = s_hist[etid];
       if (etid < N) {
@@ -501,6 +532,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           a.lrank[(size_t)(tok0 + t) * K + k] = rank;
         }
       }
+    }
+    named_bar_sync(1, kRouteEpiThreads);  // scratch free for the next tile
     }
   }
 
@@ -636,7 +669,9 @@ static int launch_route_t(const CUtensorMap& tx, const CUtensorMap& tw, const Ro
     if (e != cudaSuccess) return cuda_status(e);
     attr_set[dev] = true;
   }
-  return launch_pdl(route_kernel<NPW, NQ>, dim3(a.nblk), dim3(kRouteThreads), SM::bytes, st, tx, tw, a);
+  // persistent: one CTA per SM at most (its shared memory allows no second), tiles round robin
+  const int grid = a.nblk < sm_count() ? a.nblk : sm_count();
+  return launch_pdl(route_kernel<NPW, NQ>, dim3((unsigned)grid), dim3(kRouteThreads), SM::bytes, st, tx, tw, a);
 }
 
 int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
@@ -700,7 +735,7 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
     const long long work = (long long)npw * (d.d / 8);
     long long grid = (work + 255) / 256;
     if (grid > (long long)sm_count() * 8) grid = (long long)sm_count() * 8;
-    const int nclear = (int)((kHdrTotOffset + sizeof(int32_t) * d.N) / sizeof(uint32_t));
+    const int nclear = (int)(kHdrClearBytes / sizeof(uint32_t));
     const int r = launch_pdl(router_split_kernel, dim3((unsigned)grid), dim3(256), 0, st, w_router, w3,
                              router_rows(d), npw, d.d, a.hdr, nclear);
     if (r != MOE_OK) return r;

@@ -500,8 +500,9 @@ int launch_route_fp32(const moe_dims_t& d, const uint16_t* x, const float* w_rou
   a.M = d.M;
   a.K = d.K;
   a.nblk = L.nblk;
-  // the status word and the per-expert totals start at zero for every layer call
-  cudaError_t e = cudaMemsetAsync(a.hdr, 0, kHdrTotOffset + sizeof(int32_t) * d.N, st);
+  // the status word, the per-expert totals and the down GEMM's counters start at zero for
+  // every layer call
+  cudaError_t e = cudaMemsetAsync(a.hdr, 0, kHdrClearBytes, st);
   if (e != cudaSuccess) return cuda_status(e);
   int r;
   if (d.N <= 8) r = launch_route_t<1>(a, st);

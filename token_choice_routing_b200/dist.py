@@ -60,13 +60,18 @@ def dp_forward(layer, x, tok_null_bias, out, sums, group=None):
     if xs is None:  # gate/up gathers the routed rows of x itself
         B.expert_gate_up_gather(dm, x, out["perm_tok"], out["offsets"], layer.gate_up, layer.shared_gate_up,
                                 out["h"], out["h_shared"], ws)
+    else:
+        B.expert_gate_up(dm, xs, x, out["offsets"], layer.gate_up, layer.shared_gate_up, out["h"], out["h_shared"],
+                         ws)
+    if out.get("shared_out") is None:  # the combine inside the down GEMM's shared-expert tiles
+        B.expert_down_combine(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down,
+                              out["ys"], out["topk_gate"], out["slot_row"], out["y"], ws, topk_idx=out["topk_idx"],
+                              x=x, const_vectors=layer.const_vectors)
+    else:
         B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down, out["ys"],
                       out["shared_out"], ws)
-    else:
-        B.expert_ffn(dm, xs, x, out["offsets"], layer.gate_up, layer.w_down, layer.shared_gate_up,
-                     layer.shared_down, out["h"], out["h_shared"], out["ys"], out["shared_out"], ws)
-    B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
-              topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
+        B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
+                  topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
     return out
 
 

@@ -79,12 +79,17 @@ class MoENullLayer:
     def dims(self, T: int) -> B.Dims:
         return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags, self.C, self.V)
 
-    def alloc(self, T: int, logits: bool = True, xs: bool = True, save_preact: bool = False) -> Dict[str, torch.Tensor]:
+    def alloc(self, T: int, logits: bool = True, xs: bool = True, save_preact: bool = False,
+              shared_out: bool = True) -> Dict[str, torch.Tensor]:
         """Caller-owned buffers for a T-token call (R_cap = T*K rows). xs=False
         leaves out the gathered copy of the routed rows: the forward then gathers
         rows of x inside the gate/up GEMM and dispatch writes no copies.
         save_preact=True (training) adds z/z_shared: the forward keeps the gate/up
-        pre-activations and the backward does not recompute them."""
+        pre-activations and the backward does not recompute them.
+        shared_out=True (default) keeps the shared expert's output as a buffer of its
+        own and runs the combine as a separate launch; shared_out=False folds the
+        combine into the down GEMM's shared-expert tiles (moe_expert_down_combine), so
+        that output never goes to memory."""
         dev, d, N, M, K, F, Fs = self.device, self.d, self.N, self.M, self.K, self.F, self.F_shared
         R = T * K
         i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
@@ -101,7 +106,7 @@ class MoENullLayer:
             h=torch.empty((max(R, 1), F), dtype=bf, device=dev),
             h_shared=torch.empty((max(T, 1), Fs), dtype=bf, device=dev),
             ys=torch.empty((max(R, 1), d), dtype=bf, device=dev),
-            shared_out=torch.empty((max(T, 1), d), dtype=bf, device=dev),
+            shared_out=torch.empty((max(T, 1), d), dtype=bf, device=dev) if shared_out else None,
             y=torch.empty((max(T, 1), d), dtype=bf, device=dev),
             counts_ext=torch.empty((N + M + self.C + self.V,), dtype=i32, device=dev),
             P=torch.empty((N + M + self.C + self.V,), dtype=f32, device=dev),
