@@ -2,7 +2,7 @@
 """Benchmark of the null-expert MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config qwen3_0p6b]
+                    [--config skew] [--no-backward] [--no-per-config] [--no-cpu-baseline]
 
 A step is one full forward of the layer (route -> dispatch + aux -> grouped
 gate/up SwiGLU GEMM -> grouped down GEMM -> combine) over one batch of T
@@ -10,13 +10,23 @@ synthetic tokens that is already resident in HBM. L2 is flushed (a 256 MiB
 write) between timed steps; each step is timed with CUDA events on the
 launching stream. Prints one JSON line (rank 0).
 
+The default workload is the largest single-GPU one: the skewed batch of
+16 x 8192 tokens on the 1.7B-shaped layer (d=2048, N=64, F=1536, K=8, M=64).
+Beside it, one GPU also measures the training-mode backward on the same
+workload (`backward`) and forward-only steps of the 0.6B- and 1.7B-shaped layers
+and of the four points of the matched E[K]=2 sparsity sweep (`per_config`).
+
 Metric: real (token, expert) slots per second for the layer forward, i.e. R /
 t_step summed over ranks (null slots are not counted). Multi-GPU runs are data
 parallel (each rank its own T tokens, weak scaling) with one NCCL all-reduce
 of the additive aux statistics per step, the layer's only exchange.
 
+`e2e` is the same metric through the layer's public forward with host buffers:
+every step copies x in from pinned host memory and y, the losses and the slot
+counts back to pinned host memory, inside the timed region.
+
 --impl reference times the CPU oracle (the float64 NumPy restatement used by
-the tests) on a bounded token sample of the same workload, on the host cores.
+the tests) on a bounded sample of the same workload's tokens, on the host cores.
 """
 from __future__ import annotations
 
@@ -52,6 +62,7 @@ def load_peaks():
 # Sources whose change invalidates a recorded ncu traffic figure of the grouped GEMM.
 GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
 GEMM_PROFILE = "profiles/grouped_gemm_qwen3_0p6b.md"
+GEMM_PROFILES = (GEMM_PROFILE, "profiles/grouped_gemm_skew.md")
 BWD_GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn_bwd.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
 BWD_GEMM_PROFILE = "profiles/bwd_gemm_kernel_qwen3_0p6b.md"
 
@@ -68,11 +79,16 @@ def gemm_source_digest(sources=GEMM_SOURCES) -> str:
 def recorded_traffic(workload: str, kernel: str, profile=GEMM_PROFILE, sources=GEMM_SOURCES):
     """DRAM bytes (read + write) of one launch of `kernel` from a committed ncu summary:
     its line 'traffic-record: workload=W kernel=K dram_bytes_per_launch=B source_sha256=H'.
-    None unless it was taken on this workload from the current kernel sources."""
-    try:
-        with open(os.path.join(ROOT, profile)) as f:
-            lines = [l.strip() for l in f if l.strip().startswith("traffic-record:")]
-    except OSError:
+    None unless it was taken on this workload from the current kernel sources. `profile`
+    is one summary file or a tuple of them."""
+    lines = []
+    for prof in ((profile,) if isinstance(profile, str) else profile):
+        try:
+            with open(os.path.join(ROOT, prof)) as f:
+                lines += [l.strip() for l in f if l.strip().startswith("traffic-record:")]
+        except OSError:
+            pass
+    if not lines:
         return None
     digest = gemm_source_digest(sources)
     for l in lines:
@@ -83,7 +99,7 @@ def recorded_traffic(workload: str, kernel: str, profile=GEMM_PROFILE, sources=G
 
 
 def recorded_gate_up_traffic(workload: str):
-    return recorded_traffic(workload, "gate_up")
+    return recorded_traffic(workload, "gate_up", GEMM_PROFILES)
 
 
 class ClockSampler:
@@ -148,24 +164,58 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline object)
 
+def sample_tokens(T: int, S: int):
+    """S token indices spread evenly over the batch, so that a sample of a workload with
+    token spans of different kinds (the skewed one) holds each kind in its proportion."""
+    import numpy as np
+    S = max(1, min(T, S))
+    return np.unique(np.linspace(0, T - 1, S).round().astype(np.int64))
+
+
+_F64_WEIGHTS = {}
+
+
+def f64_weights(inp):
+    """The expert weights widened to float64 once per workload (outside the timed region, as
+    the GPU arm's weights are resident before its timing starts)."""
+    import numpy as np
+    from token_choice_routing_b200 import inputs as I
+    key = inp.cfg.name
+    if key not in _F64_WEIGHTS:
+        _F64_WEIGHTS.clear()
+        f = lambda b: I.bf16_to_f32(b).astype(np.float64)
+        _F64_WEIGHTS[key] = ((f(inp.w_gate), f(inp.w_up), f(inp.w_down)),
+                             (f(inp.ws_gate), f(inp.ws_up), f(inp.ws_down)))
+    return _F64_WEIGHTS[key]
+
+
 def oracle_sample_run(inp, S):
-    """Full oracle forward on the first S tokens; returns (seconds, real slots)."""
+    """Full oracle forward on S tokens spread over the batch, stage by stage.
+    Returns (seconds, real slots, {stage: seconds}); the stages are the oracle's own
+    functions: route (router logits, pool, top-K, gates), dispatch, experts (the SwiGLU
+    experts and the gated sum, one oracle function) and aux."""
     import numpy as np
     import oracle as O
     from token_choice_routing_b200 import inputs as I
     cfg = inp.cfg
     f = lambda b: I.bf16_to_f32(b).astype(np.float64)
+    experts, shared = f64_weights(inp)
+    tok = sample_tokens(cfg.T, S)
+    st = {}
     t0 = time.perf_counter()
-    x = f(inp.x[:S])
-    tnb = None if inp.tok_null_bias is None else inp.tok_null_bias[:S]
+    x = f(inp.x[tok])
+    tnb = None if inp.tok_null_bias is None else inp.tok_null_bias[tok]
     s = O.router_logits(x, inp.w_router, inp.bias, tnb)
     r = O.route(s, cfg.M, cfg.K)
+    t1 = time.perf_counter()
     O.dispatch(r["idx"], cfg.N)
-    O.layer_output(x, r["idx"], r["gates"], cfg.N, (f(inp.w_gate), f(inp.w_up), f(inp.w_down)),
-                   (f(inp.ws_gate), f(inp.ws_up), f(inp.ws_down)))
+    t2 = time.perf_counter()
+    O.layer_output(x, r["idx"], r["gates"], cfg.N, experts, shared)
+    t3 = time.perf_counter()
     O.aux_stats(r["idx"], r["p"], r["lse"], cfg.N, cfg.M)
-    dt = time.perf_counter() - t0
-    return dt, int(r["n_real"].sum())
+    t4 = time.perf_counter()
+    st = {"route": t1 - t0, "dispatch": t2 - t1, "experts_and_combine": t3 - t2, "aux": t4 - t3}
+    return t4 - t0, int(r["n_real"].sum()), st
 
 
 def blas_threads():
@@ -181,9 +231,21 @@ def blas_threads():
 
 def calibrate_sample(inp, target_s):
     S0 = min(inp.cfg.T, 512)
-    dt, _ = oracle_sample_run(inp, S0)
+    dt, _, _ = oracle_sample_run(inp, S0)
     S = int(S0 * target_s / max(dt, 1e-3))
     return max(64, min(inp.cfg.T, S))
+
+
+def oracle_steps(inp, S, steps):
+    """`steps` oracle forwards of the same S-token sample; per-step seconds, per-stage medians."""
+    per_step, stages, tot_r = [], {}, 0
+    for _ in range(steps):
+        dt, R, st = oracle_sample_run(inp, S)
+        per_step.append(dt)
+        tot_r += R
+        for k, v in st.items():
+            stages.setdefault(k, []).append(v)
+    return per_step, tot_r, {k: statistics.median(v) for k, v in stages.items()}
 
 
 def run_reference(args):
@@ -196,21 +258,20 @@ def run_reference(args):
     S = calibrate_sample(inp, args.ref_step_seconds)
     for _ in range(args.warmup):
         oracle_sample_run(inp, S)
-    tot_t, tot_r = 0.0, 0
-    for _ in range(args.steps):
-        dt, R = oracle_sample_run(inp, S)
-        tot_t += dt
-        tot_r += R
+    per_step, tot_r, stages = oracle_steps(inp, S, args.steps)
+    tot_t = sum(per_step)
     value = tot_r / tot_t
     cores = blas_threads()
-    sample = f"first {S} of {cfg.T} tokens per step (full oracle forward: route, dispatch, experts, aux)"
+    sample = (f"{len(sample_tokens(cfg.T, S))} of {cfg.T} tokens per step, spread evenly over the batch "
+              "(full oracle forward: route, dispatch, experts, aux)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) tokens, N(0,1/fan_in) weights)",
         "config": workload_config(cfg, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         "stage_s_median": stages, "step_s": per_step},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -366,28 +427,193 @@ def workload_config(cfg, args):
             "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "single"),
             "routed_rows": "gathered from x inside gate/up (cp.async row gathers)" if getattr(args, "gather", False)
             else "copied into xs by dispatch",
+            "combine": "inside the down GEMM's shared-expert tiles" if getattr(args, "fused_combine", False)
+            else "separate launch",
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
 # ----------------------------------------------------------------------------------------
 # GPU arm
 
+# Forward-only workloads measured beside the headline (the per_config object): the 0.6B- and
+# 1.7B-shaped layers and the four points of the matched E[K] = 2 data-sparsity sweep.
+PER_CONFIG = ("qwen3_0p6b", "qwen3_1p7b", "sweep_k2_m0", "sweep_k3_m32", "sweep_k4_m64", "sweep_k8_m192")
+
+# launches of one forward: router weight split, route, scan, dispatch(+aux), gate/up, down, combine
+# (with --fused-combine the combine runs inside the down GEMM: one launch fewer)
+FWD_LAUNCHES = 7
+
+
+def timed_events(fn, steps, warmup, flush, sync_before=None):
+    """Per-step device milliseconds of `fn` (CUDA events on the current stream, L2 flushed
+    by a 256 MiB write before every step, warm-up steps untimed)."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    if sync_before is not None:
+        sync_before()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record()
+        fn()
+        e1.record()
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in evs]
+
+
+def forward_stage_ms(layer, dm, x, tnb, out, flush, nb):
+    """Mean device ms of the forward's stages, each launched through its own entry point in
+    the forward's order with CUDA events between them (L2 flushed before each pass). With no
+    shared_out buffer the combine runs inside the down GEMM ("down_combine"), as in the
+    forward; otherwise "down" and "combine" are separate launches."""
+    import torch
+    from token_choice_routing_b200 import binding as B
+    fused = out.get("shared_out") is None
+    names = ["route", "dispatch", "gate_up"] + (["down_combine"] if fused else ["down", "combine"])
+    acc = {n: 0.0 for n in names}
+    for _ in range(nb):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        ev[0].record()
+        # "route" = router weight split + route + scan launches
+        B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, out["topk_idx"], out["topk_gate"],
+                out["n_real"], out["workspace"])
+        ev[1].record()
+        B.dispatch(dm, x, out["topk_idx"], out["workspace"], out["counts"], out["offsets"], out["perm_tok"],
+                   out["slot_row"], out["xs"])  # the aux reduction rides in this launch, as in moe_forward
+        ev[2].record()
+        if out["xs"] is None:
+            B.expert_gate_up_gather(dm, x, out["perm_tok"], out["offsets"], layer.gate_up, layer.shared_gate_up,
+                                    out["h"], out["h_shared"], out["workspace"])
+        else:
+            B.expert_gate_up(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, out["h"],
+                             out["h_shared"], out["workspace"])
+        ev[3].record()
+        if fused:
+            B.expert_down_combine(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down,
+                                  out["ys"], out["topk_gate"], out["slot_row"], out["y"], out["workspace"],
+                                  topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
+            ev[4].record()
+        else:
+            B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down,
+                          out["ys"], out["shared_out"], out["workspace"])
+            ev[4].record()
+            B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
+                      topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
+            ev[5].record()
+        torch.cuda.synchronize()
+        for i, n in enumerate(names):
+            acc[n] += ev[i].elapsed_time(ev[i + 1])
+    return {n: acc[n] / nb for n in names}
+
+
+def forward_figures(cfg, R, kms, peaks, args, out):
+    """Per-kernel throughput and roofline fractions of one forward from its stage times.
+    GEMM FLOPs count real rows only (routed real slots and the shared expert's T rows);
+    route, dispatch and combine count the bytes the method must move. The down GEMM with
+    the combine inside it is reported against the tensor peak (its FLOPs) and, beside
+    that, the combine's own bytes over the same time."""
+    T, d, F, Fs, N, K = cfg.T, cfg.d, cfg.F, cfg.F_shared, cfg.N, cfg.K
+    flops_gu = 4.0 * d * F * R + 4.0 * d * Fs * T
+    flops_dn = 2.0 * d * F * R + 2.0 * d * Fs * T
+    bytes_route = 2.0 * d * T + (8.0 * K + 4.0) * T
+    # dispatch: topk_idx and in-block ranks read, slot_row written (4 B each per slot), perm_tok per real
+    # slot; plus, when it copies rows into xs, 2d B read and 2d B written per real slot
+    bytes_dispatch = 12.0 * K * T + 4.0 * R + (0.0 if args.gather else 4.0 * d * R)
+    bytes_combine = 2.0 * d * R + 4.0 * d * T
+    if cfg.C + cfg.V > 0:  # MoE++ copy/constant slots read a row of x or a constant vector
+        bytes_combine += 2.0 * d * float(out["counts_ext"][cfg.N + cfg.M:].sum().item())
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fp32_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+    b = {
+        "route": {"ms": kms["route"], "bound": "alu" if args.router == "fp32_cores" else "hbm",
+                  "TFLOP/s": 2.0 * (N + 1) * d * T / (kms["route"] * 1e9),
+                  "GB/s": bytes_route / (kms["route"] * 1e6)},
+        "dispatch": {"ms": kms["dispatch"], "bound": "hbm", "GB/s": bytes_dispatch / (kms["dispatch"] * 1e6)},
+        "gate_up": {"ms": kms["gate_up"], "bound": "tensor", "TFLOP/s": flops_gu / (kms["gate_up"] * 1e9)},
+    }
+    b["route"]["frac_fp32_alu"] = b["route"]["TFLOP/s"] / fp32_peak
+    b["route"]["frac_hbm"] = b["route"]["GB/s"] / hbm_peak
+    b["dispatch"]["frac"] = b["dispatch"]["GB/s"] / hbm_peak
+    b["gate_up"]["frac"] = b["gate_up"]["TFLOP/s"] / bf16_peak
+    if "down_combine" in kms:
+        ms = kms["down_combine"]
+        # the fused launch writes y (2d B per token) instead of the shared output, and reads each
+        # real slot's ys row (2d B) from L2 or HBM: those are the combine's bytes inside it
+        b["down_combine"] = {"ms": ms, "bound": "tensor", "TFLOP/s": flops_dn / (ms * 1e9),
+                             "frac": flops_dn / (ms * 1e9) / bf16_peak,
+                             "combine_bytes": 2.0 * d * R + 2.0 * d * T}
+        ffn_ms = kms["gate_up"] + ms
+    else:
+        b["down"] = {"ms": kms["down"], "bound": "tensor", "TFLOP/s": flops_dn / (kms["down"] * 1e9)}
+        b["down"]["frac"] = b["down"]["TFLOP/s"] / bf16_peak
+        b["combine"] = {"ms": kms["combine"], "bound": "hbm", "GB/s": bytes_combine / (kms["combine"] * 1e6)}
+        b["combine"]["frac"] = b["combine"]["GB/s"] / hbm_peak
+        ffn_ms = kms["gate_up"] + kms["down"]
+    ffn_tflops = (6.0 * d * F * R + 6.0 * d * Fs * T) / (ffn_ms * 1e9)
+    return b, ffn_tflops, flops_gu
+
+
+def measure_per_config(args, names, dev, flush, peaks):
+    """Forward-only measurement of further workloads (one at a time, buffers freed between):
+    median step time over `steps` timed forwards, real slots per second, stage times."""
+    import torch
+    from token_choice_routing_b200 import inputs as I
+    from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
+    res = {}
+    steps, warmup = max(3, min(args.steps, 10)), max(3, min(args.warmup, 5))
+    for name in names:
+        cfg = I.CONFIGS[name]
+        inp = I.make_inputs(cfg)
+        layer = MoENullLayer.from_inputs(inp, dev, router=args.router, ffn=args.ffn)
+        x = bf16_tensor(inp.x, dev)
+        tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
+        out = layer.alloc(cfg.T, logits=False, xs=not args.gather, shared_out=not args.fused_combine)
+        ms = timed_events(lambda: layer.forward(x, tnb, out), steps, warmup, flush)
+        R = int(out["offsets"][-1].item())
+        kms = forward_stage_ms(layer, layer.dims(cfg.T), x, tnb, out, flush, 3)
+        b, ffn_tflops, _ = forward_figures(cfg, R, kms, peaks, args, out)
+        med = statistics.median(ms)
+        res[name] = {"T": cfg.T, "K": cfg.K, "M": cfg.M, "rho": cfg.rho, "real_slots_per_step": R,
+                     "ms_per_step_median": med, "ms_per_step_mean": sum(ms) / len(ms), "steps": steps,
+                     "value": R / (med * 1e-3), "tokens_per_s": cfg.T / (med * 1e-3),
+                     "ffn_tflops_real_rows": ffn_tflops,
+                     "kernels": {k: {kk: vv for kk, vv in v.items() if kk in ("ms", "frac", "frac_hbm", "GB/s")}
+                                 for k, v in b.items()}}
+        del layer, out, x, tnb, inp
+        torch.cuda.empty_cache()
+    sw = [n for n in names if n.startswith("sweep_")]
+    if len(sw) > 1:
+        base = res[sw[0]]["ms_per_step_median"]
+        res["sweep_time_vs_rho1"] = {n: res[n]["ms_per_step_median"] / base for n in sw}
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="qwen3_0p6b")
+    ap.add_argument("--config", default="skew",
+                    help="headline workload (default: skew, the largest single-GPU workload)")
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"],
                     help="router product on the tensor cores (default) or the fp32 CUDA cores")
     ap.add_argument("--ffn", default="single", choices=["single", "pair"],
                     help="expert GEMMs on single-CTA tiles (default) or CTA pairs where the shape allows")
     ap.add_argument("--gather", action="store_true",
                     help="no xs copy: gate/up gathers the routed rows of x by TMA (default: dispatch copies them)")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="combine inside the down GEMM's shared-expert tiles (default: its own launch)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the forward-only per_config workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
+    ap.add_argument("--cpu-steps", type=int, default=3, help="oracle steps of the cpu_baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -417,7 +643,7 @@ def main():
     x = bf16_tensor(inp.x, dev)
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
     T = cfg.T
-    out = layer.alloc(T, logits=False, xs=not args.gather)
+    out = layer.alloc(T, logits=False, xs=not args.gather, shared_out=not args.fused_combine)
     dm = layer.dims(T)
     nsum = B.aux_sums_count(dm)
     sums = torch.zeros(nsum, dtype=torch.float64, device=dev)
@@ -429,8 +655,8 @@ def main():
         else:
             dp_forward(layer, x, tnb, out, sums)
 
-    # route, scan, dispatch(+aux), gate_up, down, combine (+ aux sums and finalize when data parallel)
-    kernels_per_step = 6 if world == 1 else 8
+    # one forward, plus the aux sums and their finalize when data parallel
+    kernels_per_step = FWD_LAUNCHES - (1 if args.fused_combine else 0) + (2 if world > 1 else 0)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -440,93 +666,27 @@ def main():
     if st != B.OK:
         raise SystemExit(f"device status after warm-up: {B.status_string(st)}")
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for e0, e1 in evs:
-            flush.zero_()
-            e0.record()
-            step()
-            e1.record()
-        torch.cuda.synchronize()
-    step_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+        step_ms = timed_events(step, args.steps, 0, flush, sync_before=dist.barrier if world > 1 else None)
     total_ms = sum(step_ms)
+    med_ms = statistics.median(step_ms)
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([total_ms, med_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms, med_ms = float(t[0].item()), float(t[1].item())
     R = int(out["offsets"][-1].item())
     value = world * R * args.steps / (total_ms * 1e-3)
     st = B.get_device_status(out["workspace"])
     if st != B.OK:
         raise SystemExit(f"device status after timing: {B.status_string(st)}")
 
-    # ---- per-kernel breakdown (separately timed steps, same launches, CUDA events between them)
-    names = ["route", "dispatch", "gate_up", "down", "combine"]  # "route" = route + scan launches
-    acc = {n: 0.0 for n in names}
-    nb = max(3, min(args.steps, 10))
-    for _ in range(nb):
-        flush.zero_()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-        ev[0].record()
-        B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, out["topk_idx"], out["topk_gate"],
-                out["n_real"], out["workspace"])
-        ev[1].record()
-        B.dispatch(dm, x, out["topk_idx"], out["workspace"], out["counts"], out["offsets"], out["perm_tok"],
-                   out["slot_row"], out["xs"])  # the aux reduction rides in this launch, as in moe_forward
-        ev[2].record()
-        if out["xs"] is None:
-            B.expert_gate_up_gather(dm, x, out["perm_tok"], out["offsets"], layer.gate_up, layer.shared_gate_up,
-                                    out["h"], out["h_shared"], out["workspace"])
-        else:
-            B.expert_gate_up(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, out["h"],
-                             out["h_shared"], out["workspace"])
-        ev[3].record()
-        B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down, out["ys"],
-                      out["shared_out"], out["workspace"])
-        ev[4].record()
-        B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
-                  topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
-        ev[5].record()
-        torch.cuda.synchronize()
-        for i, n in enumerate(names):
-            acc[n] += ev[i].elapsed_time(ev[i + 1])
-    kms = {n: acc[n] / nb for n in names}
-
+    # ---- per-kernel breakdown (separately timed passes, same launches, CUDA events between them)
+    kms = forward_stage_ms(layer, dm, x, tnb, out, flush, max(3, min(args.steps, 10)))
     peaks, peak_kind = load_peaks()
-    d, F, Fs, N, K = cfg.d, cfg.F, cfg.F_shared, cfg.N, cfg.K
-    flops_gu = 4.0 * d * F * R + 4.0 * d * Fs * T
-    flops_dn = 2.0 * d * F * R + 2.0 * d * Fs * T
-    bytes_route = 2.0 * d * T + (8.0 * K + 4.0) * T
-    # dispatch: topk_idx and in-block ranks read, slot_row written (4 B each per slot), perm_tok per real
-    # slot; plus, when it copies rows into xs, 2d B read and 2d B written per real slot
-    bytes_dispatch = 12.0 * K * T + 4.0 * R + (0.0 if args.gather else 4.0 * d * R)
-    bytes_combine = 2.0 * d * R + 4.0 * d * T
-    if cfg.C + cfg.V > 0:  # MoE++ copy/constant slots read a row of x or a constant vector
-        bytes_combine += 2.0 * d * float(out["counts_ext"][cfg.N + cfg.M:].sum().item())
+    breakdown, ffn_tflops, flops_gu = forward_figures(cfg, R, kms, peaks, args, out)
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    fp32_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
-    breakdown = {
-        "route": {"ms": kms["route"], "bound": "alu" if args.router == "fp32_cores" else "hbm",
-                  "TFLOP/s": 2.0 * (N + 1) * d * T / (kms["route"] * 1e9),
-                  "GB/s": bytes_route / (kms["route"] * 1e6)},
-        "dispatch": {"ms": kms["dispatch"], "bound": "hbm", "GB/s": bytes_dispatch / (kms["dispatch"] * 1e6)},
-        "gate_up": {"ms": kms["gate_up"], "bound": "tensor", "TFLOP/s": flops_gu / (kms["gate_up"] * 1e9)},
-        "down": {"ms": kms["down"], "bound": "tensor", "TFLOP/s": flops_dn / (kms["down"] * 1e9)},
-        "combine": {"ms": kms["combine"], "bound": "hbm", "GB/s": bytes_combine / (kms["combine"] * 1e6)},
-    }
-    breakdown["route"]["frac_fp32_alu"] = breakdown["route"]["TFLOP/s"] / fp32_peak
-    breakdown["route"]["frac_hbm"] = breakdown["route"]["GB/s"] / hbm_peak
-    breakdown["dispatch"]["frac"] = breakdown["dispatch"]["GB/s"] / hbm_peak
-    breakdown["combine"]["frac"] = breakdown["combine"]["GB/s"] / hbm_peak
-    breakdown["gate_up"]["frac"] = breakdown["gate_up"]["TFLOP/s"] / bf16_peak
-    breakdown["down"]["frac"] = breakdown["down"]["TFLOP/s"] / bf16_peak
-    ffn_ms = kms["gate_up"] + kms["down"]
-    # FFN FLOP/s over real rows only: routed (token, expert) slots plus the shared expert's T rows
-    ffn_tflops = (6.0 * d * F * R + 6.0 * d * Fs * T) / (ffn_ms * 1e9)
+    d, F, Fs = cfg.d, cfg.F, cfg.F_shared
 
     achieved = breakdown["gate_up"]["TFLOP/s"]
     pair = args.ffn == "pair" and cfg.F % 128 == 0 and cfg.F_shared % 128 == 0
@@ -549,50 +709,61 @@ def main():
                     "peak_kind": f"{peak_kind} HBM copy", "traffic": None, "bytes_per_launch": bytes_gu,
                     "experts_used": used, "ms_per_launch": kms["gate_up"]}
 
-    # ---- end to end through the C ABI with host buffers
+    # ---- end to end through the public API with host buffers: every step copies x in from pinned
+    # host memory, runs the forward, and copies y, the two losses and the slot counts back
     x_pin = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
     loss_pin = torch.empty(2, dtype=torch.float32).pin_memory()
     cext_pin = torch.empty(out["counts_ext"].numel(), dtype=torch.int32).pin_memory()
     xin = torch.empty_like(x)
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+
+    def e2e_step():
         xin.copy_(x_pin, non_blocking=True)
         layer.forward(xin, tnb, out)
+        y_pin.copy_(out["y"][:T], non_blocking=True)
         loss_pin.copy_(out["losses"], non_blocking=True)
         cext_pin.copy_(out["counts_ext"], non_blocking=True)
-        e1.record()
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(e0.elapsed_time(e1))
+
+    e2e_ms = timed_events(e2e_step, args.steps, args.warmup, flush)
     e2e_total = sum(e2e_ms)
     if world > 1:
         t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_total = float(t.item())
+    if not torch.equal(y_pin.to(dev), out["y"][:T]):
+        raise SystemExit("e2e: the y copied back differs from the device y")
     e2e = {"value": world * R * args.steps / (e2e_total * 1e-3), "unit": UNIT,
-           "h2d_bytes_per_step": int(x_pin.numel() * 2), "d2h_bytes_per_step": int(8 + 4 * cext_pin.numel()),
-           "ms_per_step": e2e_total / args.steps}
+           "h2d_bytes_per_step": int(x_pin.numel() * 2),
+           "d2h_bytes_per_step": int(y_pin.numel() * 2 + 4 * loss_pin.numel() + 4 * cext_pin.numel()),
+           "ms_per_step": e2e_total / args.steps, "ms_per_step_median": statistics.median(e2e_ms)}
+    del x_pin, y_pin, xin
 
     backward = None
     if not args.no_backward and world == 1 and not args.gather:
         backward = measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind)
 
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        del layer, out, x, tnb
+        torch.cuda.empty_cache()
+        per_config = measure_per_config(args, [n for n in PER_CONFIG if n != cfg.name], dev, flush, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        S = calibrate_sample(inp, args.cpu_seconds)
-        dt, Rs = oracle_sample_run(inp, S)
-        cpu = {"value": Rs / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"first {S} of {T} tokens, one full oracle forward ({dt:.1f} s)"}
+        S = calibrate_sample(inp, args.cpu_seconds / max(1, args.cpu_steps))
+        per_step, Rs, stages = oracle_steps(inp, S, max(1, args.cpu_steps))
+        cpu = {"value": Rs / sum(per_step), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{len(sample_tokens(T, S))} of {T} tokens spread evenly over the batch, "
+                         f"{len(per_step)} full oracle forwards ({sum(per_step):.1f} s)",
+               "step_s": per_step, "stage_s_median": stages}
 
     if world > 1:
         dist.barrier()
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "ms_per_step_median": med_ms,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 tokens, N(0,1/fan_in) bf16 weights, fp32 router)",
             "config": workload_config(cfg, args),
@@ -605,6 +776,7 @@ def main():
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk.summary(),
             "backward": backward,
+            "per_config": per_config,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -28,14 +28,27 @@ def test_traffic_record_is_used_only_with_matching_sources(tmp_path, monkeypatch
 
 
 def test_committed_records_parse():
-    """The committed profiles carry well-formed records for the headline workload."""
-    for prof in (bench.GEMM_PROFILE, bench.BWD_GEMM_PROFILE):
+    """The committed profiles carry well-formed records of known workloads."""
+    from token_choice_routing_b200 import inputs as I
+    for prof in (*bench.GEMM_PROFILES, bench.BWD_GEMM_PROFILE):
+        if not os.path.exists(os.path.join(ROOT, prof)):
+            continue
         lines = [l for l in open(os.path.join(ROOT, prof)) if l.startswith("traffic-record:")]
         assert lines, prof
         for l in lines:
             kv = dict(p.split("=", 1) for p in l.split()[1:])
-            assert kv["workload"] == "qwen3_0p6b" and int(kv["dram_bytes_per_launch"]) > 0
+            assert kv["workload"] in I.CONFIGS and int(kv["dram_bytes_per_launch"]) > 0
             assert len(kv["source_sha256"]) == 64
+
+
+def test_token_sample_spreads_over_the_batch():
+    """The oracle's timing sample takes tokens from every part of the batch (the skewed
+    workload's low-information and dense spans alike)."""
+    tok = bench.sample_tokens(131072, 1000)
+    assert tok[0] == 0 and tok[-1] == 131071 and len(tok) == 1000
+    low = (tok % 8192) < round(0.6 * 8192)   # the skewed workload's low-information spans
+    assert abs(low.mean() - 0.6) < 0.01
+    assert bench.sample_tokens(10, 50).tolist() == list(range(10))
 
 
 def test_reference_arm_json_line():
