@@ -427,8 +427,9 @@ def workload_config(cfg, args):
             "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "single"),
             "routed_rows": "gathered from x inside gate/up (cp.async row gathers)" if getattr(args, "gather", False)
             else "copied into xs by dispatch",
-            "combine": "inside the down GEMM's shared-expert tiles" if getattr(args, "fused_combine", False)
-            else "separate launch",
+            "combine": {"inplace": "shared expert written into y, routed rows added in place",
+                        "separate": "shared expert output in its own buffer, then the combine launch",
+                        "fused": "inside the down GEMM's shared-expert tiles"}[getattr(args, "combine", "inplace")],
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
@@ -440,7 +441,7 @@ def workload_config(cfg, args):
 PER_CONFIG = ("qwen3_0p6b", "qwen3_1p7b", "sweep_k2_m0", "sweep_k3_m32", "sweep_k4_m64", "sweep_k8_m192")
 
 # launches of one forward: router weight split, route, scan, dispatch(+aux), gate/up, down, combine
-# (with --fused-combine the combine runs inside the down GEMM: one launch fewer)
+# (with --combine fused the combine runs inside the down GEMM: one launch fewer)
 FWD_LAUNCHES = 7
 
 
@@ -523,7 +524,13 @@ def forward_figures(cfg, R, kms, peaks, args, out):
     # dispatch: topk_idx and in-block ranks read, slot_row written (4 B each per slot), perm_tok per real
     # slot; plus, when it copies rows into xs, 2d B read and 2d B written per real slot
     bytes_dispatch = 12.0 * K * T + 4.0 * R + (0.0 if args.gather else 4.0 * d * R)
-    bytes_combine = 2.0 * d * R + 4.0 * d * T
+    # combine: each real slot's row of ys (2d B); the shared expert's row read and y written (4d B)
+    # for every token, or in place only for the tokens that have a source at all
+    if getattr(args, "combine", "separate") == "inplace":
+        t_src = int((out["n_real"][:T] > 0).sum().item()) if cfg.C + cfg.V == 0 else T
+        bytes_combine = 2.0 * d * R + 4.0 * d * t_src
+    else:
+        bytes_combine = 2.0 * d * R + 4.0 * d * T
     if cfg.C + cfg.V > 0:  # MoE++ copy/constant slots read a row of x or a constant vector
         bytes_combine += 2.0 * d * float(out["counts_ext"][cfg.N + cfg.M:].sum().item())
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -572,7 +579,7 @@ def measure_per_config(args, names, dev, flush, peaks):
         layer = MoENullLayer.from_inputs(inp, dev, router=args.router, ffn=args.ffn)
         x = bf16_tensor(inp.x, dev)
         tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
-        out = layer.alloc(cfg.T, logits=False, xs=not args.gather, shared_out=not args.fused_combine)
+        out = layer.alloc(cfg.T, logits=False, xs=not args.gather, combine=args.combine)
         ms = timed_events(lambda: layer.forward(x, tnb, out), steps, warmup, flush)
         R = int(out["offsets"][-1].item())
         kms = forward_stage_ms(layer, layer.dims(cfg.T), x, tnb, out, flush, 3)
@@ -607,8 +614,10 @@ def main():
                     help="expert GEMMs on single-CTA tiles (default) or CTA pairs where the shape allows")
     ap.add_argument("--gather", action="store_true",
                     help="no xs copy: gate/up gathers the routed rows of x by TMA (default: dispatch copies them)")
-    ap.add_argument("--fused-combine", action="store_true",
-                    help="combine inside the down GEMM's shared-expert tiles (default: its own launch)")
+    ap.add_argument("--combine", default="inplace", choices=["inplace", "separate", "fused"],
+                    help="inplace (default): the down GEMM writes the shared expert's output into y and "
+                         "the combine adds the routed rows there; separate: its own buffer; fused: the "
+                         "combine inside the down GEMM's shared-expert tiles")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--no-per-config", action="store_true", help="skip the forward-only per_config workloads")
@@ -643,7 +652,7 @@ def main():
     x = bf16_tensor(inp.x, dev)
     tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).to(dev)
     T = cfg.T
-    out = layer.alloc(T, logits=False, xs=not args.gather, shared_out=not args.fused_combine)
+    out = layer.alloc(T, logits=False, xs=not args.gather, combine=args.combine)
     dm = layer.dims(T)
     nsum = B.aux_sums_count(dm)
     sums = torch.zeros(nsum, dtype=torch.float64, device=dev)
@@ -656,7 +665,7 @@ def main():
             dp_forward(layer, x, tnb, out, sums)
 
     # one forward, plus the aux sums and their finalize when data parallel
-    kernels_per_step = FWD_LAUNCHES - (1 if args.fused_combine else 0) + (2 if world > 1 else 0)
+    kernels_per_step = FWD_LAUNCHES - (1 if args.combine == "fused" else 0) + (2 if world > 1 else 0)
 
     for _ in range(args.warmup):
         flush.zero_()

@@ -132,9 +132,11 @@ typedef struct moe_outputs {
   uint16_t* h;          /* [R_cap, F] bf16 routed SwiGLU activations             */
   uint16_t* h_shared;   /* [T, F_shared] bf16 shared SwiGLU activations          */
   uint16_t* ys;         /* [R_cap, d] bf16 routed expert outputs                 */
-  uint16_t* shared_out; /* [T, d] bf16 shared expert output, or NULL: the combine is
-                           then folded into the down GEMM (moe_expert_down_combine)
-                           and the shared expert's output is never written alone   */
+  uint16_t* shared_out; /* [T, d] bf16 shared expert output; or y itself: the down
+                           GEMM then writes it into y and the combine adds the routed
+                           rows in place, skipping tokens that have none; or NULL:
+                           the combine is folded into the down GEMM
+                           (moe_expert_down_combine). y is the same in all three.   */
   uint16_t* y;          /* [T, d] bf16 layer output                              */
   int32_t* counts_ext;  /* [N+M+C+V] tokens per pool slot                        */
   float* P;             /* [N+M+C+V] mean routing probability per pool slot      */
@@ -323,7 +325,8 @@ MOE_API int moe_expert_down_combine(const moe_dims_t* dims, const int32_t* offse
  * ys[slot_row[t,k]] for a real expert, x[t] for a copy expert, const_vectors[j]
  * for constant expert j, nothing for a null copy; fp32 accumulation, one
  * rounding. y [T, d]. topk_idx, x and const_vectors are read only when C + V >
- * 0 (they may be NULL otherwise). */
+ * 0 (they may be NULL otherwise). shared_out may be y itself (in place): a
+ * token with no slot that has an output is then left as it is. */
 MOE_API int moe_combine(const moe_dims_t* dims, const uint16_t* ys, const uint16_t* shared_out,
                 const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx,
                 const uint16_t* x, const uint16_t* const_vectors, uint16_t* y, moe_stream_t stream);

@@ -45,14 +45,15 @@ def make_layer(inp, device="cuda", router="tensor", ffn="single"):
     return layer, x, tnb
 
 
-def run_forward(inp, device="cuda", router="tensor", ffn="single", xs=True, shared_out=True):
+def run_forward(inp, device="cuda", router="tensor", ffn="single", xs=True, combine="separate"):
     """xs=False: no gathered copy of the routed rows; gate/up gathers rows of x.
-    shared_out=True (the default): the shared expert's output gets a buffer of its own
-    (checked by the GEMM tests) and the combine is its own launch; False: the combine runs
+    combine="separate" (the default here): the shared expert's output gets a buffer of its
+    own (checked by the GEMM tests) and the combine reads it; "inplace": the down GEMM
+    writes it into y and the combine adds the routed rows there; "fused": the combine runs
     in the down GEMM's shared-expert tiles."""
     from token_choice_routing_b200 import binding as B
     layer, x, tnb = make_layer(inp, device, router, ffn)
-    out = layer.forward(x, tnb, layer.alloc(inp.cfg.T, xs=xs, shared_out=shared_out))
+    out = layer.forward(x, tnb, layer.alloc(inp.cfg.T, xs=xs, combine=combine))
     torch.cuda.synchronize()
     st = B.get_device_status(out["workspace"])
     assert st == B.OK, B.status_string(st)

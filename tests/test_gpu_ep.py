@@ -26,7 +26,7 @@ def test_expert_parallel_forward_matches_one_gpu(name, world):
     cfg = I.CONFIGS[name] if name in I.CONFIGS else cfgs[name]
     inp = I.make_inputs(cfg)
     layer, x, tnb = H.make_layer(inp)
-    ref = layer.forward(x, tnb, layer.alloc(cfg.T))  # the separate combine, as the ranks run it
+    ref = layer.forward(x, tnb, layer.alloc(cfg.T))
     torch.cuda.synchronize()
     bounds = np.linspace(0, cfg.T, world + 1).astype(int)
     fabric = ep.LocalFabric(world)
@@ -35,7 +35,7 @@ def test_expert_parallel_forward_matches_one_gpu(name, world):
     def rank_fn(rank, tr):
         a, b = int(bounds[rank]), int(bounds[rank + 1])
         shard = ep.ExpertShard(layer, rank, world)
-        out = layer.alloc(b - a, shared_out=True)
+        out = layer.alloc(b - a)
         sums = torch.zeros(nsum, dtype=torch.float64, device="cuda")
         ep.ep_forward(shard, x[a:b], None if tnb is None else tnb[a:b], out, tr, sums)
         torch.cuda.synchronize()

@@ -79,8 +79,8 @@ def test_dp_statistics_of_a_split_batch_match_the_whole_batch():
     np.testing.assert_allclose(losses.cpu().numpy(), out["losses"].cpu().numpy(), rtol=1e-6)
 
 
-@pytest.mark.parametrize("shared_out", [False, True])
-def test_dp_forward_in_a_one_rank_group_equals_forward_bitwise(shared_out):
+@pytest.mark.parametrize("combine", ["inplace", "separate", "fused"])
+def test_dp_forward_in_a_one_rank_group_equals_forward_bitwise(combine):
     """dp_forward's sequence (route, aux sums, NCCL all-reduce, finalize, dispatch, expert GEMMs,
     combine in the down GEMM or on its own) with one rank is moe_forward, bit for bit."""
     import torch.distributed as dist
@@ -88,11 +88,11 @@ def test_dp_forward_in_a_one_rank_group_equals_forward_bitwise(shared_out):
     from token_choice_routing_b200.dist import dp_forward
     cfg = I.CONFIGS["qwen3_0p6b"]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, ref = H.run_forward(inp, shared_out=shared_out)
+    layer, x, tnb, ref = H.run_forward(inp, combine=combine)
     dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1,
                             timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
     try:
-        out = layer.alloc(cfg.T, shared_out=shared_out)
+        out = layer.alloc(cfg.T, combine=combine)
         sums = torch.zeros(B.aux_sums_count(layer.dims(cfg.T)), dtype=torch.float64, device="cuda")
         dp_forward(layer, x, tnb, out, sums)
         torch.cuda.synchronize()
@@ -102,7 +102,7 @@ def test_dp_forward_in_a_one_rank_group_equals_forward_bitwise(shared_out):
     assert st == B.OK, B.status_string(st)
     R = int(ref["offsets"][-1])
     keys = ["logits", "topk_idx", "topk_gate", "n_real", "counts", "offsets", "slot_row", "h_shared", "y",
-            "counts_ext", "P", "losses"] + (["shared_out"] if shared_out else [])
+            "counts_ext", "P", "losses"] + (["shared_out"] if combine == "separate" else [])
     for k in keys:
         assert torch.equal(out[k], ref[k]), k
     for k in ("perm_tok", "xs", "h", "ys"):

@@ -94,10 +94,11 @@ def test_full_size_layer_parity_sampled(name, router, ffn, xs):
 
 @pytest.mark.parametrize("name", ["sweep_k2_m0", "sweep_k3_m32", "sweep_k4_m64", "sweep_k8_m192", "skew"])
 def test_large_configs_routing_and_sampled_output(name):
-    """The combine inside the down GEMM, at the large workloads, against the oracle."""
+    """The forward as the benchmark runs it (the shared expert written into y, the combine in
+    place), at the large workloads, against the oracle."""
     cfg = I.CONFIGS[name]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, out = H.run_forward(inp, shared_out=False)
+    layer, x, tnb, out = H.run_forward(inp, combine="inplace")
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -116,7 +117,7 @@ def test_row_gather_matches_row_copy_bitwise(name):
     layer, x, tnb = H.make_layer(inp)
     outs = []
     for xs in (True, False):
-        out = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, shared_out=True))
+        out = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, combine="separate"))
         torch.cuda.synchronize()
         outs.append(out)
     R = int(outs[0]["offsets"][-1])
@@ -391,14 +392,13 @@ def test_combine_in_down_gemm_is_bitwise_the_separate_combine(name, router, ffn,
         inp.bias[cfg.N] = np.float32(0.4)
         inp.bias[cfg.N + 1:] = np.float32(0.6)
     layer, x, tnb = H.make_layer(inp, router=router, ffn=ffn)
-    ref = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, shared_out=True))
-    outs = [layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, shared_out=False)) for _ in range(2)]  # counters reset
+    ref = layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, combine="separate"))
+    outs = [layer.forward(x, tnb, layer.alloc(cfg.T, xs=xs, combine=c)) for c in ("fused", "fused", "inplace")]
     torch.cuda.synchronize()
     from token_choice_routing_b200 import binding as B
     R = int(ref["offsets"][-1])
     for out in outs:
         assert B.get_device_status(out["workspace"]) == B.OK
-        assert out["shared_out"] is None
         for k in ("y", "topk_idx", "topk_gate", "counts", "offsets", "slot_row", "h_shared", "counts_ext", "P",
                   "losses"):
             assert torch.equal(out[k], ref[k]), k
@@ -413,7 +413,7 @@ def test_down_combine_entry_point_called_alone_twice():
     cfg = I.CONFIGS["qwen3_0p6b"]
     inp = I.make_inputs(cfg)
     layer, x, tnb = H.make_layer(inp)
-    out = layer.forward(x, tnb, layer.alloc(cfg.T, shared_out=False))
+    out = layer.forward(x, tnb, layer.alloc(cfg.T, combine="fused"))
     torch.cuda.synchronize()
     y0 = out["y"].clone()
     dm = layer.dims(cfg.T)

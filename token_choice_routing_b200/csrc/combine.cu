@@ -12,21 +12,23 @@ namespace moe {
 
 constexpr int kCombineThreads = 256;
 
-// One warp per token, two 16-byte chunks per lane per pass. In each pass the
-// shared row's chunks and the chunks of the first four slots are loaded
-// together before any is used (null slots load nothing); the next token's slot
-// list is fetched while this one is combined. Sum order: shared, then slots in
-// rank order. A slot's source row is coded as: >= 0 a row of ys, -1 nothing
-// (null copy), -2 the token's row of x (copy expert), -3 - j constant vector j.
+// One warp per token, two 16-byte chunks per lane per pass. A slot's source row is coded
+// as: >= 0 a row of ys, -1 nothing (null copy), -2 the token's row of x (copy expert),
+// -3 - j constant vector j. The token's slots with a source are compacted (in rank order)
+// and taken four at a time: in each pass the shared row's chunks and those slots' chunks
+// are loaded together before any is used, so a token with up to four sources costs one
+// round of loads per pass whatever K is; the next token's slot list is fetched while this
+// one is combined. Sum order: shared, then the sources in rank order; fp32, one rounding.
 // UNIT_ROWS (the backward's input gradient): rows of ys enter with weight 1, the gate
 // having been applied upstream; copy slots still take g times their row of x.
-template <bool UNIT_ROWS>
+// INPLACE (sh == y, the shared expert's output written into y by the down GEMM): a token
+// without a source already holds its result, bf16(shared), and is skipped.
+template <bool UNIT_ROWS, bool INPLACE>
 __global__ void __launch_bounds__(kCombineThreads, 3)
-combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
-               const float* __restrict__ gate, const int32_t* __restrict__ slot_row,
-               const int32_t* __restrict__ topk_idx, const uint16_t* __restrict__ x,
-               const uint16_t* __restrict__ cv, uint16_t* __restrict__ y, int T, int d, int K, long long rcap,
-               int NM, int C, int V, uint32_t* status) {
+combine_kernel(const uint16_t* ys, const uint16_t* sh, const float* __restrict__ gate,
+               const int32_t* __restrict__ slot_row, const int32_t* __restrict__ topk_idx,
+               const uint16_t* __restrict__ x, const uint16_t* __restrict__ cv, uint16_t* y, int T, int d, int K,
+               long long rcap, int NM, int C, int V, uint32_t* status) {
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const int wpb = kCombineThreads / 32;
@@ -61,6 +63,12 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
   load_slot(t, row, g);
   for (; t < T; t += stride) {
     load_slot(t + stride, rown, gn);  // next token's slots, in flight during this one
+    const unsigned srcs = __ballot_sync(0xffffffffu, row != -1);  // lanes >= K hold -1
+    if (INPLACE && srcs == 0u) {
+      row = rown;
+      g = gn;
+      continue;
+    }
     for (int c0 = 0; c0 < nch; c0 += 64) {
       const int ca = c0 + lane, cb = c0 + 32 + lane;
       const bool oka = ca < nch, okb = cb < nch;
@@ -68,16 +76,19 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
       const uint4 sa = oka ? __ldg(shr + ca) : make_uint4(0u, 0u, 0u, 0u);
       const uint4 sb = okb ? __ldg(shr + cb) : make_uint4(0u, 0u, 0u, 0u);
       float acc_a[8], acc_b[8];
-      for (int k0 = 0; k0 < K; k0 += 4) {
+      bool first = true;
+      unsigned m = srcs;
+      do {
         uint4 va[4], vb[4];
         float gq[4];
         int rq[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int k = k0 + u;
-          rq[u] = __shfl_sync(0xffffffffu, row, k & 31);
-          gq[u] = __shfl_sync(0xffffffffu, g, k & 31);
-          if (k >= K) rq[u] = -1;
+          const int k = m ? __ffs(m) - 1 : 0;
+          rq[u] = __shfl_sync(0xffffffffu, row, k);
+          gq[u] = __shfl_sync(0xffffffffu, g, k);
+          if (m == 0u) rq[u] = -1;
+          m &= m - 1u;
           if (UNIT_ROWS && rq[u] >= 0) gq[u] = 1.f;
           const uint16_t* srow = (rq[u] >= 0)    ? ys + (size_t)rq[u] * d
                                  : (rq[u] == -2) ? x + (size_t)t * d
@@ -87,11 +98,12 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
           va[u] = (rq[u] != -1 && oka) ? __ldg(src + ca) : make_uint4(0u, 0u, 0u, 0u);
           vb[u] = (rq[u] != -1 && okb) ? __ldg(src + cb) : make_uint4(0u, 0u, 0u, 0u);
         }
-        if (k0 == 0) {
+        if (first) {
           acc_a[0] = bf16lo(sa.x); acc_a[1] = bf16hi(sa.x); acc_a[2] = bf16lo(sa.y); acc_a[3] = bf16hi(sa.y);
           acc_a[4] = bf16lo(sa.z); acc_a[5] = bf16hi(sa.z); acc_a[6] = bf16lo(sa.w); acc_a[7] = bf16hi(sa.w);
           acc_b[0] = bf16lo(sb.x); acc_b[1] = bf16hi(sb.x); acc_b[2] = bf16lo(sb.y); acc_b[3] = bf16hi(sb.y);
           acc_b[4] = bf16lo(sb.z); acc_b[5] = bf16hi(sb.z); acc_b[6] = bf16lo(sb.w); acc_b[7] = bf16hi(sb.w);
+          first = false;
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -100,7 +112,7 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* __restrict__ sh,
             fma8(acc_b, gq[u], vb[u]);
           }
         }
-      }
+      } while (m != 0u);
       if (oka)
         reinterpret_cast<uint4*>(y + (size_t)t * d)[ca] =
             make_uint4(pack_bf16x2(acc_a[0], acc_a[1]), pack_bf16x2(acc_a[2], acc_a[3]),
@@ -122,7 +134,7 @@ static int combine_grid(const moe_dims_t& d) {
   cudaGetDevice(&dev);
   int occ = (dev >= 0 && dev < 64) ? per_sm[dev] : 0;
   if (occ == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_kernel<false>, kCombineThreads, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_kernel<false, false>, kCombineThreads, 0) !=
             cudaSuccess ||
         occ < 1)
       occ = 1;
@@ -139,9 +151,10 @@ int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shar
                    const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
                    const uint16_t* const_vectors, uint16_t* y, cudaStream_t st) {
   const int grid = combine_grid(d);
-  return launch_pdl(combine_kernel<false>, dim3(grid), dim3(kCombineThreads), 0, st, ys, shared_out, topk_gate,
-                    slot_row, topk_idx, x, const_vectors, y, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C,
-                    d.V, nullptr);
+  // shared_out == y: the shared expert's output is already in y; tokens without a source keep it
+  auto kern = (shared_out == y) ? combine_kernel<false, true> : combine_kernel<false, false>;
+  return launch_pdl(kern, dim3(grid), dim3(kCombineThreads), 0, st, ys, shared_out, topk_gate, slot_row, topk_idx, x,
+                    const_vectors, y, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, d.V, nullptr);
 }
 
 // Input gradient of the backward pass: dx[t] = dx_shared[t] (the shared expert's and the
@@ -151,7 +164,7 @@ int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint
                       const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, uint16_t* dx,
                       uint32_t* status, cudaStream_t st) {
   const int grid = combine_grid(d);
-  return launch_pdl(combine_kernel<true>, dim3(grid), dim3(kCombineThreads), 0, st, dxs, dx_shared, topk_gate,
+  return launch_pdl(combine_kernel<true, false>, dim3(grid), dim3(kCombineThreads), 0, st, dxs, dx_shared, topk_gate,
                     slot_row, topk_idx, dy, (const uint16_t*)nullptr, dx, d.T, d.d, d.K, (long long)d.T * d.K,
                     d.N + d.M, d.C, 0, status);
 }

@@ -162,34 +162,56 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
   const long long rcap = (long long)a.T * K;
   const int nch = d >> 3;  // 16-byte chunks per row
   const int wpb = kDispatchThreads / 32;
-  for (int t = blk * wpb + (tid >> 5); t < a.T; t += nblocks * wpb) {
+  const int stride = nblocks * wpb;
+  // lane k < K: the destination row of the token's slot k (-1: null or out of range)
+  auto slot_dest = [&](int t) {
     int dest = -1;
-    if (lane < K) {
+    if (t < a.T && lane < K) {
       const int id = __ldg(a.topk_idx + (size_t)t * K + lane);
       if (id >= 0 && id < N) {
         dest = __ldg(a.bases + (size_t)id * a.nblk + t / a.blk_tokens) + __ldg(a.lrank + (size_t)t * K + lane);
         if (dest < 0 || dest >= rcap) {
           atomicOr(a.status, kStatusBounds);
           dest = -1;
-        } else {
-          a.perm_tok[dest] = t;
         }
       } else if (id < 0 || id >= N + a.M + a.aux.C + a.aux.V) {
         atomicOr(a.status, kStatusBounds);
       }
-      a.slot_row[(size_t)t * K + lane] = dest;
     }
-    if (a.xs == nullptr) continue;  // no row copies: gate/up gathers the rows of x itself
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * d);
-    for (int c0 = 0; c0 < nch; c0 += 32) {  // warp-uniform trip count (shuffles below)
-      const int c = c0 + lane;
-      const bool ok = c < nch;
-      const uint4 v = ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-      for (int k = 0; k < K; ++k) {
-        const int dk = __shfl_sync(0xffffffffu, dest, k);
-        if (dk >= 0 && ok) reinterpret_cast<uint4*>(a.xs + (size_t)dk * d)[c] = v;
+    return dest;
+  };
+  int t = blk * wpb + (tid >> 5);
+  int dest = slot_dest(t);
+  for (; t < a.T; t += stride) {
+    const int dest_next = slot_dest(t + stride);  // the next token's rows, looked up meanwhile
+    if (lane < K) {
+      a.slot_row[(size_t)t * K + lane] = dest;
+      if (dest >= 0) a.perm_tok[dest] = t;
+    }
+    const unsigned real = __ballot_sync(0xffffffffu, dest >= 0);
+    if (a.xs != nullptr && real != 0u) {
+      // the whole row is loaded (8 x 16 B per lane for d <= 2048) before any copy is stored
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * d);
+      for (int c0 = 0; c0 < nch; c0 += 256) {  // warp-uniform trip count
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = c0 + j * 32 + lane;
+          v[j] = (c < nch) ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (unsigned m = real; m != 0u; m &= m - 1u) {
+          const int k = __ffs(m) - 1;
+          const int dk = __shfl_sync(0xffffffffu, dest, k);
+          uint4* dst = reinterpret_cast<uint4*>(a.xs + (size_t)dk * d);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int c = c0 + j * 32 + lane;
+            if (c < nch) dst[c] = v[j];
+          }
+        }
       }
     }
+    dest = dest_next;
   }
 }
 

@@ -242,8 +242,8 @@ class ExpertShard:
 def ep_forward(shard: ExpertShard, x: torch.Tensor, tok_null_bias: Optional[torch.Tensor], out: Dict,
                transport, sums: torch.Tensor) -> Dict:
     """One expert-parallel layer step on this rank's tokens (see the module docstring).
-    ``out`` comes from ``shard.layer.alloc(T, shared_out=True)`` (the combine runs after the
-    return exchange, so the shared expert's output needs its own buffer); ``sums`` is a
+    ``out`` comes from ``shard.layer.alloc(T)`` with the combine "inplace" or "separate" (it
+    runs after the return exchange, not inside the down GEMM); ``sums`` is a
     float64 device tensor of ``aux_sums_count`` elements. Adds ``out["ep_plan"]``."""
     from . import binding as B
     layer = shard.layer
@@ -251,7 +251,7 @@ def ep_forward(shard: ExpertShard, x: torch.Tensor, tok_null_bias: Optional[torc
     dm = layer.dims(T)
     ws = out["workspace"]
     if out.get("shared_out") is None or out.get("xs") is None:
-        raise ValueError("expert parallelism needs the xs and shared_out buffers")
+        raise ValueError("expert parallelism needs xs and a shared-expert output buffer (or y)")
     B.route(dm, x, layer.w_router, layer.router_bias, tok_null_bias, out.get("logits"), out["topk_idx"],
             out["topk_gate"], out["n_real"], ws)
     B.aux_sums(dm, ws, sums)

@@ -80,16 +80,22 @@ class MoENullLayer:
         return B.dims(T, self.d, self.N, self.M, self.K, self.F, self.F_shared, self.flags, self.C, self.V)
 
     def alloc(self, T: int, logits: bool = True, xs: bool = True, save_preact: bool = False,
-              shared_out: bool = True) -> Dict[str, torch.Tensor]:
+              combine: str = "inplace") -> Dict[str, torch.Tensor]:
         """Caller-owned buffers for a T-token call (R_cap = T*K rows). xs=False
         leaves out the gathered copy of the routed rows: the forward then gathers
         rows of x inside the gate/up GEMM and dispatch writes no copies.
         save_preact=True (training) adds z/z_shared: the forward keeps the gate/up
         pre-activations and the backward does not recompute them.
-        shared_out=True (default) keeps the shared expert's output as a buffer of its
-        own and runs the combine as a separate launch; shared_out=False folds the
-        combine into the down GEMM's shared-expert tiles (moe_expert_down_combine), so
-        that output never goes to memory."""
+        combine: where the shared expert's output goes and how the routed outputs are
+        added to it.
+          "inplace" (default): the down GEMM writes it into y and the combine adds the
+            gated routed rows in place, skipping tokens without any (their y is done);
+          "separate": a buffer of its own (out["shared_out"]), read by the combine;
+          "fused": the combine runs in the down GEMM's shared-expert tiles
+            (moe_expert_down_combine) and that output never goes to memory.
+        All three give bit-identical y."""
+        if combine not in ("inplace", "separate", "fused"):
+            raise ValueError(f"combine must be 'inplace', 'separate' or 'fused', not {combine!r}")
         dev, d, N, M, K, F, Fs = self.device, self.d, self.N, self.M, self.K, self.F, self.F_shared
         R = T * K
         i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
@@ -106,7 +112,7 @@ class MoENullLayer:
             h=torch.empty((max(R, 1), F), dtype=bf, device=dev),
             h_shared=torch.empty((max(T, 1), Fs), dtype=bf, device=dev),
             ys=torch.empty((max(R, 1), d), dtype=bf, device=dev),
-            shared_out=torch.empty((max(T, 1), d), dtype=bf, device=dev) if shared_out else None,
+            shared_out=torch.empty((max(T, 1), d), dtype=bf, device=dev) if combine == "separate" else None,
             y=torch.empty((max(T, 1), d), dtype=bf, device=dev),
             counts_ext=torch.empty((N + M + self.C + self.V,), dtype=i32, device=dev),
             P=torch.empty((N + M + self.C + self.V,), dtype=f32, device=dev),
@@ -114,6 +120,8 @@ class MoENullLayer:
             z=torch.empty((max(R, 1), 2 * F), dtype=bf, device=dev) if save_preact else None,
             z_shared=torch.empty((max(T, 1), 2 * Fs), dtype=bf, device=dev) if save_preact else None,
         )
+        if combine == "inplace":
+            out["shared_out"] = out["y"]
         out["workspace"] = torch.empty((max(B.workspace_bytes(self.dims(T)), 256),), dtype=torch.uint8, device=dev)
         return out
 
