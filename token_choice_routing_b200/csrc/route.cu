@@ -118,12 +118,13 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
 // Shared memory of the route kernel: a 3-stage ring of x and split-weight tiles, and the
 // routing scratch of the epilogue beside it (not aliased: the epilogue of one tile runs
 // while the ring already fills for the next).
-template <int NPW>
+template <int NPW, bool PAIR>
 struct RouteSmem {
-  static constexpr int STAGES = 3;
-  static constexpr int BROWS = 3 * NPW;
+  static constexpr int STAGES = PAIR ? 4 : 3;
+  static constexpr int BROWS = 3 * NPW;                   // rows of the split weight (the MMA's N)
+  static constexpr int BROWS_CTA = PAIR ? BROWS / 2 : BROWS;  // rows this CTA loads
   static constexpr int A_BYTES = kRouteTokens * kRouteBK * 2;
-  static constexpr int B_BYTES = BROWS * kRouteBK * 2;
+  static constexpr int B_BYTES = BROWS_CTA * kRouteBK * 2;
   static constexpr size_t off_a = 0;
   static constexpr size_t off_b = off_a + (size_t)STAGES * A_BYTES;
   static constexpr size_t ring_end = off_b + (size_t)STAGES * B_BYTES;
@@ -152,23 +153,28 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
 }
 
 // ---------------------------------------------------------------------------------------
-// Persistent: one CTA per SM (at most), 576 threads, taking 128-token tiles b = blockIdx.x,
-// blockIdx.x + gridDim.x, ... (tokens [128 b, 128 b + 128) x all router rows each). Two
-// TMEM accumulators: the MMA of tile i+1 runs while the epilogue routes tile i.
+// Persistent: one CTA per SM (at most), 576 threads, taking 128-token tiles in turn
+// (tokens [128 b, 128 b + 128) x all router rows each). Two TMEM accumulators: the MMA of
+// tile i+1 runs while the epilogue routes tile i.
+// PAIR: the two CTAs of a cluster share one MMA of M = 256 (tcgen05 cta_group::2) over a
+// unit of two consecutive tiles: each CTA loads its own 128 tokens and half of the split
+// weight's rows, so the weight, which every tile reads whole, crosses from L2 once per 256
+// tokens instead of once per 128. Each CTA's TMEM then holds its own tokens x all logits,
+// and the epilogue is unchanged. Without PAIR a unit is one tile.
 // NQ: logit columns per lane (4 lanes per token): NPW / 4, or 16 when NPW = 80 and
 // there are no copy/constant experts (the candidates are then the reals, columns < 64).
-template <int NPW, int NQ>
+template <int NPW, int NQ, bool PAIR>
 __global__ void __launch_bounds__(kRouteThreads, 1)
     route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const RouteArgs a) {
   pdl_wait_then_release();
-  using SM = RouteSmem<NPW>;
+  using SM = RouteSmem<NPW, PAIR>;
   constexpr int STAGES = SM::STAGES;
   constexpr int LS = SM::LS;
   constexpr uint32_t ACOLS = SM::BROWS <= 64 ? 64u : SM::BROWS <= 128 ? 128u : 256u;  // per accumulator
   constexpr uint32_t TCOLS = 2 * ACOLS;
-  constexpr uint32_t IDESC = idesc_bf16_f32(kRouteTokens, SM::BROWS);
-  constexpr uint32_t TX = SM::A_BYTES + SM::B_BYTES;
+  constexpr uint32_t IDESC = idesc_bf16_f32(PAIR ? 2 * kRouteTokens : kRouteTokens, SM::BROWS);
+  constexpr uint32_t TX = (PAIR ? 2 : 1) * (SM::A_BYTES + SM::B_BYTES);  // one stage, both CTAs
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base =
@@ -187,7 +193,15 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = a.T, N = a.N, M = a.M, K = a.K;
   const int nkb = a.d / kRouteBK;
-  const int ntile = a.nblk;
+  const uint32_t crank = PAIR ? cluster_rank() : 0u;
+  const bool leader = crank == 0u;
+  // units (a tile, or two tiles for a pair) u = unit0, unit0 + ustep, ...; this CTA's tile of
+  // unit u is tile_of(u) (with an odd tile count the last pair's second CTA has none: its
+  // tokens are past T, loaded as zeros and never written)
+  const int unit0 = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int ustep = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
+  const int nunit = PAIR ? (a.nblk + 1) / 2 : a.nblk;
+  auto tile_of = [&](int u) { return PAIR ? 2 * u + (int)crank : u; };
 
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmX);
@@ -198,18 +212,24 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(tfull_bar(s), 1);
-      mbar_init(tempty_bar(s), kRouteEpiThreads);
+      mbar_init(tempty_bar(s), (PAIR ? 2 : 1) * (kRouteEpiThreads / 32));  // one arrival per epilogue warp
     }
     mbar_init(drain_bar, 1);
     misc[1] = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(const_cast<int*>(misc)), TCOLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(const_cast<int*>(misc)), TCOLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(const_cast<int*>(misc)), TCOLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = (uint32_t)misc[0];
 
@@ -220,15 +240,26 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
       bool ok = true;
-      for (int b = blockIdx.x; b < ntile && ok; b += gridDim.x) {
+      for (int u = unit0; u < nunit && ok; u += ustep) {
+        const int b = tile_of(u);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, a.limit_ns, abort_flag, a.hdr)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(stage), TX);
-          tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), &tmX, full_bar(stage), kb * kRouteBK, b * kRouteTokens);
-          tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), &tmW, full_bar(stage), kb * kRouteBK, 0);
+          if constexpr (PAIR) {
+            // both CTAs' copies of a stage complete on the leader's barrier
+            const uint32_t fb = map_to_rank(full_bar(stage), 0);
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), TX);
+            tma_load_2d_pair(smem_u32(sA + stage * SM::A_BYTES), &tmX, fb, kb * kRouteBK, b * kRouteTokens);
+            tma_load_2d_pair(smem_u32(sB + stage * SM::B_BYTES), &tmW, fb, kb * kRouteBK,
+                             (int)crank * SM::BROWS_CTA);
+          } else {
+            mbar_arrive_expect_tx(full_bar(stage), TX);
+            tma_load_2d(smem_u32(sA + stage * SM::A_BYTES), &tmX, full_bar(stage), kb * kRouteBK,
+                        b * kRouteTokens);
+            tma_load_2d(smem_u32(sB + stage * SM::B_BYTES), &tmW, full_bar(stage), kb * kRouteBK, 0);
+          }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -237,21 +268,22 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           }
         }
       }
-      if (*abort_flag) {
-        // let every issued copy land before the CTA can exit
+      if (*abort_flag && leader) {
+        // let every issued copy land before the CTA can exit (a pair's copies all count on
+        // the leader's barriers)
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s))
             (void)mbar_wait_bounded(full_bar(s), (armed_par >> s) & 1u, a.limit_ns, nullptr, a.hdr);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------ MMA issuer (single thread)
+    if (lane == 0 && leader) {
+      // ------------------------------ MMA issuer (single thread; the leader's, for a pair)
       int stage = 0;
       uint32_t phase = 0;
       int li = 0;
       bool ok = true;
-      for (int b = blockIdx.x; b < ntile && ok; b += gridDim.x, ++li) {
+      for (int u = unit0; u < nunit && ok; u += ustep, ++li) {
         const int acc = li & 1;
         const uint32_t ap = (uint32_t)(li >> 1) & 1u;
         if (!mbar_wait_bounded(tempty_bar(acc), ap ^ 1u, a.limit_ns, abort_flag, a.hdr)) break;
@@ -266,19 +298,37 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * SM::A_BYTES));
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * SM::B_BYTES));
 #pragma unroll
-          for (int k = 0; k < kRouteBK / 16; ++k)
-            tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
-                       (kb | k) != 0 ? 1u : 0u);
-          tc_commit(empty_bar(stage));
+          for (int k = 0; k < kRouteBK / 16; ++k) {
+            if constexpr (PAIR)
+              tc_mma_pair(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
+                          (kb | k) != 0 ? 1u : 0u);
+            else
+              tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
+                         (kb | k) != 0 ? 1u : 0u);
+          }
+          if constexpr (PAIR) {  // free this stage in both CTAs
+            tc_commit_pair(empty_bar(stage));
+            tc_commit_pair(map_to_rank(empty_bar(stage), 1));
+          } else {
+            tc_commit(empty_bar(stage));
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) tc_commit(tfull_bar(acc));
+        if (ok) {
+          if constexpr (PAIR) {
+            tc_commit_pair(tfull_bar(acc));
+            tc_commit_pair(map_to_rank(tfull_bar(acc), 1));
+          } else {
+            tc_commit(tfull_bar(acc));
+          }
+        }
       }
       // fires once every MMA issued above has completed (also after an abort)
-      tc_commit(drain_bar);
+      if constexpr (PAIR) tc_commit_pair(drain_bar);
+      else tc_commit(drain_bar);
       (void)mbar_wait_bounded(drain_bar, 0, a.limit_ns, nullptr, a.hdr);
     }
   } else {
@@ -294,11 +344,13 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     unsigned* tokbits = reinterpret_cast<unsigned*>(base + SM::off_tokbits);  // [4][kMaxN]
     int* s_hist = reinterpret_cast<int*>(base + SM::off_hist);                // [kMaxK+1]
     int li = 0;
-    for (int b = blockIdx.x; b < ntile; b += gridDim.x, ++li) {
+    for (int u = unit0; u < nunit; u += ustep, ++li) {
+    const int b = tile_of(u);
+    const bool live = b < a.nblk;  // false: the empty second tile of an odd tile count
     const int acc = li & 1;
     const uint32_t ap = (uint32_t)(li >> 1) & 1u;
     const int tok0 = b * kRouteTokens;
-    const int nvalid = min(kRouteTokens, T - tok0);
+    const int nvalid = max(0, min(kRouteTokens, T - tok0));
     const bool ok = mbar_wait_bounded(tfull_bar(acc), ap, a.limit_ns, abort_flag, a.hdr) && *abort_flag == 0;
     if (!named_bar_and(1, kRouteEpiThreads, ok)) break;
     {
@@ -328,9 +380,13 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
           }
         }
       }
-      // the accumulator is free for the tile after next
+      // the accumulator is free for the tile after next (for a pair, once both CTAs say so)
       tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));
+        else mbar_arrive(tempty_bar(acc));
+      }
     }
     named_bar_sync(1, kRouteEpiThreads);
     {
@@ -499,7 +555,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) {
+        if (lane == 0 && live) {
           if (c < ncols) a.ppart[(size_t)b * ncols + c] = sum;
           else a.lsq[b] = sum;
         }
@@ -509,8 +565,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 
     {
       const int hc = K + 1 + (a.ncols - N - 1);  // null histogram, then copy/constant counts
-      if (etid < hc) a.hist[(size_t)b * hc + etid] = s_hist[etid];
-      if (etid < N) {
+      if (live && etid < hc) a.hist[(size_t)b * hc + etid] = s_hist[etid];
+      if (live && etid < N) {
         int cnt = 0;
 #pragma unroll
         for (int w = 0; w < 4; ++w) cnt += __popc(tokbits[w * kMaxN + etid]);
@@ -538,11 +594,13 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // the leader's MMAs read both CTAs' shared memory
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TCOLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TCOLS);
+    else tmem_dealloc(tmem_base, TCOLS);
   }
 }
 
@@ -657,21 +715,57 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a) {
   }
 }
 
-template <int NPW, int NQ>
+template <int NPW, int NQ, bool PAIR>
 static int launch_route_t(const CUtensorMap& tx, const CUtensorMap& tw, const RouteArgs& a, cudaStream_t st) {
-  using SM = RouteSmem<NPW>;
-  static bool attr_set[64] = {false};
+  using SM = RouteSmem<NPW, PAIR>;
+  auto kern = route_kernel<NPW, NQ, PAIR>;
+  static int max_units[64] = {0};  // resident CTAs (or pairs) per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<NPW, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SM::bytes);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(kRouteThreads, 1, 1);
+  cfg.dynamicSmemBytes = SM::bytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (dev >= 0 && dev < 64 && max_units[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::bytes);
     if (e != cudaSuccess) return cuda_status(e);
-    attr_set[dev] = true;
+    int n = PAIR ? sm_count() / 2 : sm_count();
+    if (PAIR) {
+      int c = 0;
+      cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+      if (cudaOccupancyMaxActiveClusters(&c, kern, &cfg) == cudaSuccess && c >= 1) n = c;
+    }
+    max_units[dev] = n;
   }
-  // persistent: one CTA per SM at most (its shared memory allows no second), tiles round robin
-  const int grid = a.nblk < sm_count() ? a.nblk : sm_count();
-  return launch_pdl(route_kernel<NPW, NQ>, dim3((unsigned)grid), dim3(kRouteThreads), SM::bytes, st, tx, tw, a);
+  // persistent: at most one CTA per SM (the shared memory allows no second), units round robin
+  const int units = PAIR ? (a.nblk + 1) / 2 : a.nblk;
+  int grid_units = (dev >= 0 && dev < 64) ? max_units[dev] : (PAIR ? sm_count() / 2 : sm_count());
+  if (units < grid_units) grid_units = units;
+  if (grid_units < 1) grid_units = 1;
+  cfg.gridDim = dim3((unsigned)((PAIR ? 2 : 1) * grid_units), 1, 1);
+  cfg.attrs = PAIR ? attr : attr + 1;
+  cfg.numAttrs = PAIR ? 2 : 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tx, tw, a));
+}
+
+// CTA pairs when the tiles outnumber the SMs (each CTA then takes several tiles and the
+// weight's L2 stream is what the pair halves); with one wave of tiles or less the single-CTA
+// kernel starts every tile at once and measured slightly faster.
+static bool route_pairs(int nblk) { return nblk > sm_count(); }
+
+template <int NPW, int NQ>
+static int launch_route_np(const CUtensorMap& tx, const CUtensorMap& tw, const RouteArgs& a, cudaStream_t st) {
+  return route_pairs(a.nblk) ? launch_route_t<NPW, NQ, true>(tx, tw, a, st)
+                             : launch_route_t<NPW, NQ, false>(tx, tw, a, st);
 }
 
 int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
@@ -740,18 +834,20 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
                              router_rows(d), npw, d.d, a.hdr, nclear);
     if (r != MOE_OK) return r;
   }
+  // the weight's box: all 3 npw rows, or half of them for each CTA of a pair
+  const uint32_t wbox = (uint32_t)(route_pairs(L.nblk) ? 3 * npw / 2 : 3 * npw);
   CUtensorMap tx, tw;
   if (!make_tmap_bf16(&tx, x, (uint64_t)d.T, (uint64_t)d.d, kRouteTokens) ||
-      !make_tmap_bf16(&tw, w3, (uint64_t)3 * npw, (uint64_t)d.d, (uint32_t)(3 * npw)))
+      !make_tmap_bf16(&tw, w3, (uint64_t)3 * npw, (uint64_t)d.d, wbox))
     return MOE_ERR_CUDA;
   int r;
   switch (npw) {
-    case 16: r = launch_route_t<16, 4>(tx, tw, a, st); break;
-    case 32: r = launch_route_t<32, 8>(tx, tw, a, st); break;
-    case 48: r = launch_route_t<48, 12>(tx, tw, a, st); break;
-    case 64: r = launch_route_t<64, 16>(tx, tw, a, st); break;
+    case 16: r = launch_route_np<16, 4>(tx, tw, a, st); break;
+    case 32: r = launch_route_np<32, 8>(tx, tw, a, st); break;
+    case 48: r = launch_route_np<48, 12>(tx, tw, a, st); break;
+    case 64: r = launch_route_np<64, 16>(tx, tw, a, st); break;
     default:  // 80 rows: without copy/constant experts the candidates are the reals, columns < 64
-      r = (pp_experts(d) == 0) ? launch_route_t<80, 16>(tx, tw, a, st) : launch_route_t<80, 20>(tx, tw, a, st);
+      r = (pp_experts(d) == 0) ? launch_route_np<80, 16>(tx, tw, a, st) : launch_route_np<80, 20>(tx, tw, a, st);
       break;
   }
   if (r != MOE_OK) return r;
