@@ -61,6 +61,8 @@ def load_peaks():
 
 # Sources whose change invalidates a recorded ncu traffic figure of the grouped GEMM.
 GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
+PAIR_GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn_pair.cu",
+                     "token_choice_routing_b200/csrc/moe_internal.cuh")
 GEMM_PROFILE = "profiles/grouped_gemm_qwen3_0p6b.md"
 GEMM_PROFILES = (GEMM_PROFILE, "profiles/grouped_gemm_skew.md")
 BWD_GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn_bwd.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
@@ -98,7 +100,11 @@ def recorded_traffic(workload: str, kernel: str, profile=GEMM_PROFILE, sources=G
     return None
 
 
-def recorded_gate_up_traffic(workload: str):
+def recorded_gate_up_traffic(workload: str, pair: bool = False):
+    """The gate/up launch's recorded DRAM bytes: the single-CTA kernel ("gate_up") or the
+    CTA-pair kernel ("gate_up_pair"), each pinned to its own sources."""
+    if pair:
+        return recorded_traffic(workload, "gate_up_pair", GEMM_PROFILES, PAIR_GEMM_SOURCES)
     return recorded_traffic(workload, "gate_up", GEMM_PROFILES)
 
 
@@ -424,7 +430,7 @@ def workload_config(cfg, args):
             "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "K": cfg.K, "F": cfg.F, "F_shared": cfg.F_shared,
             "C": cfg.C, "V": cfg.V,
             "global_batch_tokens": cfg.T * args.gpus, "parallelism": f"dp{args.gpus}",
-            "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "single"),
+            "router": getattr(args, "router", "tensor"), "ffn": getattr(args, "ffn", "auto"),
             "routed_rows": "gathered from x inside gate/up (cp.async row gathers)" if getattr(args, "gather", False)
             else "copied into xs by dispatch",
             "combine": {"inplace": "shared expert written into y, routed rows added in place",
@@ -610,8 +616,9 @@ def main():
                     help="headline workload (default: skew, the largest single-GPU workload)")
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"],
                     help="router product on the tensor cores (default) or the fp32 CUDA cores")
-    ap.add_argument("--ffn", default="single", choices=["single", "pair"],
-                    help="expert GEMMs on single-CTA tiles (default) or CTA pairs where the shape allows")
+    ap.add_argument("--ffn", default="auto", choices=["auto", "single", "pair"],
+                    help="expert GEMMs on single-CTA tiles, CTA pairs where the shape allows, or auto "
+                         "(default: pairs from 65536 tokens per call)")
     ap.add_argument("--gather", action="store_true",
                     help="no xs copy: gate/up gathers the routed rows of x by TMA (default: dispatch copies them)")
     ap.add_argument("--combine", default="inplace", choices=["inplace", "separate", "fused"],
@@ -621,6 +628,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--no-per-config", action="store_true", help="skip the forward-only per_config workloads")
+    ap.add_argument("--e2e-chunk", type=int, default=16384,
+                    help="tokens per chunk of the host-buffer forward that e2e times")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time of the cpu_baseline")
     ap.add_argument("--cpu-steps", type=int, default=3, help="oracle steps of the cpu_baseline")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0, help="oracle seconds per reference step")
@@ -698,12 +707,13 @@ def main():
     d, F, Fs = cfg.d, cfg.F, cfg.F_shared
 
     achieved = breakdown["gate_up"]["TFLOP/s"]
-    pair = args.ffn == "pair" and cfg.F % 128 == 0 and cfg.F_shared % 128 == 0
+    pair = (args.ffn == "pair" or (args.ffn == "auto" and T >= MoENullLayer.PAIR_MIN_TOKENS)) \
+        and cfg.F % 128 == 0 and cfg.F_shared % 128 == 0
     roofline = {"kernel": "grouped gate/up SwiGLU GEMM (tcgen05, %s)" % ("CTA pairs" if pair else "single CTA"),
                 "bound": "tensor", "achieved": achieved,
                 "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
                 "peak_kind": f"{peak_kind} bf16 burst",
-                "traffic": recorded_gate_up_traffic(cfg.name) if not (args.gather or pair) else None,
+                "traffic": None if args.gather else recorded_gate_up_traffic(cfg.name, pair),
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "flops_per_launch": flops_gu, "ms_per_launch": kms["gate_up"]}
 
@@ -718,20 +728,22 @@ def main():
                     "peak_kind": f"{peak_kind} HBM copy", "traffic": None, "bytes_per_launch": bytes_gu,
                     "experts_used": used, "ms_per_launch": kms["gate_up"]}
 
-    # ---- end to end through the public API with host buffers: every step copies x in from pinned
-    # host memory, runs the forward, and copies y, the two losses and the slot counts back
+    # ---- end to end through the public API with host buffers: every step copies x (and the
+    # per-token null offsets) in from pinned host memory and y, the losses and the slot counts back
+    # to pinned host memory; the layer's host forward runs in token chunks so the copies in and
+    # out overlap each other and the compute
     x_pin = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    tnb_pin = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).pin_memory()
     y_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
     loss_pin = torch.empty(2, dtype=torch.float32).pin_memory()
     cext_pin = torch.empty(out["counts_ext"].numel(), dtype=torch.int32).pin_memory()
-    xin = torch.empty_like(x)
+    chunk = min(T, args.e2e_chunk)
+    pipe = layer.alloc_host_pipeline(chunk)
 
     def e2e_step():
-        xin.copy_(x_pin, non_blocking=True)
-        layer.forward(xin, tnb, out)
-        y_pin.copy_(out["y"][:T], non_blocking=True)
-        loss_pin.copy_(out["losses"], non_blocking=True)
-        cext_pin.copy_(out["counts_ext"], non_blocking=True)
+        st = layer.forward_host(x_pin, y_pin, pipe, tnb_pin)
+        loss_pin.copy_(st["losses"], non_blocking=True)
+        cext_pin.copy_(st["counts_ext"], non_blocking=True)
 
     e2e_ms = timed_events(e2e_step, args.steps, args.warmup, flush)
     e2e_total = sum(e2e_ms)
@@ -739,13 +751,17 @@ def main():
         t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_total = float(t.item())
+    torch.cuda.synchronize()
     if not torch.equal(y_pin.to(dev), out["y"][:T]):
-        raise SystemExit("e2e: the y copied back differs from the device y")
+        raise SystemExit("e2e: the y copied back differs from the device forward's y")
+    h2d = x_pin.numel() * 2 + (0 if tnb_pin is None else tnb_pin.numel() * 4)
     e2e = {"value": world * R * args.steps / (e2e_total * 1e-3), "unit": UNIT,
-           "h2d_bytes_per_step": int(x_pin.numel() * 2),
+           "h2d_bytes_per_step": int(h2d),
            "d2h_bytes_per_step": int(y_pin.numel() * 2 + 4 * loss_pin.numel() + 4 * cext_pin.numel()),
-           "ms_per_step": e2e_total / args.steps, "ms_per_step_median": statistics.median(e2e_ms)}
-    del x_pin, y_pin, xin
+           "ms_per_step": e2e_total / args.steps, "ms_per_step_median": statistics.median(e2e_ms),
+           "chunk_tokens": chunk,
+           "launches_per_step": (FWD_LAUNCHES + 1) * ((T + chunk - 1) // chunk) + 1}
+    del x_pin, y_pin, pipe
 
     backward = None
     if not args.no_backward and world == 1 and not args.gather:

@@ -342,6 +342,11 @@ MOE_API size_t moe_aux_sums_count(const moe_dims_t* dims);
 MOE_API int moe_aux_sums(const moe_dims_t* dims, const void* workspace, double* sums,
                  moe_stream_t stream);
 
+/* moe_aux_sums added into `sums` (+=) instead of written over it: the statistics of
+ * a batch processed in several calls (token chunks), summed on the device. */
+MOE_API int moe_aux_sums_accumulate(const moe_dims_t* dims, const void* workspace, double* sums,
+                                    moe_stream_t stream);
+
 /* L_bal / L_z from (possibly all-reduced) sums (section 三 / 负载均衡损失,
  * Z-Loss): counts_ext [N+M+C+V] (null copy j counts the tokens with more than j
  * null slots), P [N+M+C+V] (null copies share the null probability), losses [2]

@@ -92,13 +92,15 @@ def test_full_size_layer_parity_sampled(name, router, ffn, xs):
     assert abs(out["n_real"].float().mean().item() - cfg.rho * cfg.K) < 0.02
 
 
-@pytest.mark.parametrize("name", ["sweep_k2_m0", "sweep_k3_m32", "sweep_k4_m64", "sweep_k8_m192", "skew"])
-def test_large_configs_routing_and_sampled_output(name):
+@pytest.mark.parametrize("name,ffn", [("sweep_k2_m0", "single"), ("sweep_k3_m32", "single"),
+                                      ("sweep_k4_m64", "single"), ("sweep_k8_m192", "auto"), ("skew", "single"),
+                                      ("skew", "auto")])
+def test_large_configs_routing_and_sampled_output(name, ffn):
     """The forward as the benchmark runs it (the shared expert written into y, the combine in
-    place), at the large workloads, against the oracle."""
+    place; with ffn="auto" these sizes take the CTA-pair GEMMs), against the oracle."""
     cfg = I.CONFIGS[name]
     inp = I.make_inputs(cfg)
-    layer, x, tnb, out = H.run_forward(inp, combine="inplace")
+    layer, x, tnb, out = H.run_forward(inp, ffn=ffn, combine="inplace")
     r = H.check_routing(inp, out)
     H.check_dispatch(inp, out, r)
     H.check_aux(inp, out, r)
@@ -424,3 +426,29 @@ def test_down_combine_entry_point_called_alone_twice():
         torch.cuda.synchronize()
         assert B.get_device_status(out["workspace"]) == B.OK
         assert torch.equal(out["y"], y0)
+
+
+@pytest.mark.parametrize("name,chunk", [("qwen3_0p6b", 4096), ("qwen3_0p6b", 5000), ("skew_small", 200),
+                                        ("tiny", 256), ("pp_a", 128)])
+def test_forward_from_host_memory_in_chunks(name, chunk):
+    """MoENullLayer.forward_host: the batch in token chunks from and to pinned host memory,
+    copies overlapping the chunks' compute. y is bit-identical to one forward over the whole
+    batch; the batch's statistics (summed over the chunks) give its counts exactly and P and
+    the losses to fp64 summation order."""
+    cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP[name]
+    inp = I.make_inputs(cfg)
+    layer, x, tnb = H.make_layer(inp)
+    ref = layer.forward(x, tnb, layer.alloc(cfg.T))
+    torch.cuda.synchronize()
+    x_pin = x.cpu().pin_memory()
+    y_pin = torch.empty_like(x_pin).pin_memory()
+    tnb_pin = None if tnb is None else tnb.cpu().pin_memory()
+    pipe = layer.alloc_host_pipeline(chunk)
+    for _ in range(2):  # twice: the pipeline's buffers are reused
+        y_pin.zero_()
+        st = layer.forward_host(x_pin, y_pin, pipe, tnb_pin)
+        torch.cuda.synchronize()
+        assert torch.equal(y_pin, ref["y"][:cfg.T].cpu())
+        assert torch.equal(st["counts_ext"], ref["counts_ext"])
+        np.testing.assert_allclose(st["P"].cpu().numpy(), ref["P"].cpu().numpy(), rtol=1e-6, atol=1e-12)
+        np.testing.assert_allclose(st["losses"].cpu().numpy(), ref["losses"].cpu().numpy(), rtol=1e-6)

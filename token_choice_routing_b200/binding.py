@@ -88,6 +88,7 @@ def _load() -> C.CDLL:
         "moe_expert_down_rows": (i32, [pd, C.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_aux_sums_count": (sz, [pd]),
         "moe_aux_sums": (i32, [pd, vp, vp, vp]),
+        "moe_aux_sums_accumulate": (i32, [pd, vp, vp, vp]),
         "moe_aux_finalize": (i32, [pd, vp, vp, vp, vp, vp]),
         "moe_aux": (i32, [pd, vp, vp, vp, vp, vp]),
         "moe_forward": (i32, [pd, C.POINTER(Weights), vp, vp, C.POINTER(Outputs), vp, vp]),
@@ -256,6 +257,10 @@ def aux(dm, ws, counts_ext, P, losses, stream=None):
 
 def aux_sums(dm, ws, sums, stream=None):
     _check("moe_aux_sums", LIB.moe_aux_sums(C.byref(dm), _p(ws), _p(sums), _stream(stream)))
+
+
+def aux_sums_accumulate(dm, ws, sums, stream=None):
+    _check("moe_aux_sums_accumulate", LIB.moe_aux_sums_accumulate(C.byref(dm), _p(ws), _p(sums), _stream(stream)))
 
 
 def aux_finalize(dm, sums, counts_ext, P, losses, stream=None):

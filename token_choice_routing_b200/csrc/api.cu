@@ -215,6 +215,13 @@ int moe_aux_sums(const moe_dims_t* dims, const void* workspace, double* sums, mo
   return launch_aux(*dims, workspace, sums, nullptr, nullptr, nullptr, nullptr, S(stream));
 }
 
+int moe_aux_sums_accumulate(const moe_dims_t* dims, const void* workspace, double* sums, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (!workspace || !sums) return MOE_ERR_INVALID_ARG;
+  if (dims->T == 0) return MOE_OK;
+  return launch_aux(*dims, workspace, sums, nullptr, nullptr, nullptr, nullptr, S(stream), true);
+}
+
 int moe_aux_finalize(const moe_dims_t* dims, const double* sums, int32_t* counts_ext, float* P, float* losses,
                      moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));

@@ -95,14 +95,14 @@ __device__ void aux_finalize_block(const double* sums, int N, int M, int K, int 
 }
 
 __global__ void __launch_bounds__(256) aux_kernel(AuxPtrs p, double* sums_out, const double* sums_in,
-                                                  int32_t* counts_ext, float* P, float* losses) {
+                                                  int32_t* counts_ext, float* P, float* losses, int accumulate) {
   pdl_wait_then_release();
   __shared__ double s_sums[kMaxSums];
   const int n = p.N + (p.K + 1 + p.C + p.V) + (p.N + 1 + p.C + p.V) + 2;
   if (sums_in == nullptr) {
     aux_sums_block(p, s_sums);
     if (sums_out)
-      for (int i = threadIdx.x; i < n; i += blockDim.x) sums_out[i] = s_sums[i];
+      for (int i = threadIdx.x; i < n; i += blockDim.x) sums_out[i] = accumulate ? sums_out[i] + s_sums[i] : s_sums[i];
   } else {
     for (int i = threadIdx.x; i < n; i += blockDim.x) s_sums[i] = sums_in[i];
     __syncthreads();
@@ -268,9 +268,9 @@ int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_
 }
 
 int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const double* sums_in,
-               int32_t* counts_ext, float* P, float* losses, cudaStream_t st) {
+               int32_t* counts_ext, float* P, float* losses, cudaStream_t st, bool accumulate) {
   return launch_pdl(aux_kernel, dim3(1), dim3(256), 0, st, aux_ptrs(d, ws), sums_out, sums_in, counts_ext, P,
-                    losses);
+                    losses, accumulate ? 1 : 0);
 }
 
 // ---------------------------------------------------------------------------------------

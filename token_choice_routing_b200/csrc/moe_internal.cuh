@@ -237,7 +237,8 @@ int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_
                     uint16_t* xs, int32_t* counts_ext, float* P, float* losses,
                     cudaStream_t st);
 int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const double* sums_in,
-               int32_t* counts_ext, float* P, float* losses, cudaStream_t st);
+               int32_t* counts_ext, float* P, float* losses, cudaStream_t st,
+               bool accumulate = false);
 int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
                    const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
                    const uint16_t* const_vectors, uint16_t* y, cudaStream_t st);

@@ -443,38 +443,54 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 
       // top-K over the pool, in rank order: K rounds of "best remaining candidate"
       // against the next null copy, compared by (value desc, pool index asc): a real
-      // equal to the null logit wins, a copy or constant expert equal to it loses
+      // equal to the null logit wins, a copy or constant expert equal to it loses.
+      // Taking a null copy leaves the best remaining candidate as it was, and the null
+      // keeps beating it while copies remain (a real's index is below every copy's, a
+      // copy or constant expert's above), so the candidates are scanned again only after
+      // one of them was taken: about r + 1 scans instead of K. The four lanes of a token
+      // take the same decisions; the shuffles run within them (tokens diverge).
+      const unsigned gmask = 0xFu << (lane & ~3);
       unsigned sel = 0u;
       int used = 0, r = 0, rpp = 0;
       unsigned long long msk = 0ull;
       float smax = 0.f;  // the first non-null slot taken holds the largest gated logit
+      float bv = -INFINITY;
+      int bi = INT_MAX;
+      bool have_best = false;
       for (int k = 0; k < K; ++k) {
-        float bv = -INFINITY;
-        int bi = INT_MAX;
+        if (!have_best) {
+          bv = -INFINITY;
+          bi = INT_MAX;
 #pragma unroll
-        for (int u = 0; u < NQ; ++u) {
-          const int i = q + 4 * u;
-          if (is_cand(i) && !((sel >> u) & 1u) && ranks_before(v[u], pool_of(i), bv, bi)) {
-            bv = v[u];
-            bi = pool_of(i);
+          for (int u = 0; u < NQ; ++u) {
+            const int i = q + 4 * u;
+            if (is_cand(i) && !((sel >> u) & 1u) && ranks_before(v[u], pool_of(i), bv, bi)) {
+              bv = v[u];
+              bi = pool_of(i);
+            }
           }
-        }
 #pragma unroll
-        for (int off = 1; off <= 2; off <<= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (ranks_before(ov, oi, bv, bi)) {
-            bv = ov;
-            bi = oi;
+          for (int off = 1; off <= 2; off <<= 1) {
+            const float ov = __shfl_xor_sync(gmask, bv, off);
+            const int oi = __shfl_xor_sync(gmask, bi, off);
+            if (ranks_before(ov, oi, bv, bi)) {
+              bv = ov;
+              bi = oi;
+            }
           }
+          have_best = true;
         }
         const bool take_null = (used < M) && (bi == INT_MAX || ranks_before(sn, N + used, bv, bi));
         int id;
+        float idv;
         if (take_null) {
           id = N + used;
+          idv = sn;
           ++used;
         } else {
           id = bi;
+          idv = bv;
+          have_best = false;  // taken: the next round scans the remaining candidates
           if (r + rpp == 0) smax = bv;
           if (bi < N) {
             ++r;
@@ -487,7 +503,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         }
         if ((k & 3) == q) {  // slot k belongs to lane k mod 4 from here on
           tk[t * kMaxK + k] = id;
-          tkv[t * kMaxK + k] = bv;
+          tkv[t * kMaxK + k] = idv;
         }
       }
       // gates: softmax over the selected slots that are not null copies; each lane takes
