@@ -446,8 +446,9 @@ def workload_config(cfg, args):
 # 1.7B-shaped layers and the four points of the matched E[K] = 2 data-sparsity sweep.
 PER_CONFIG = ("qwen3_0p6b", "qwen3_1p7b", "sweep_k2_m0", "sweep_k3_m32", "sweep_k4_m64", "sweep_k8_m192")
 
-# launches of one forward: router weight split, route, scan, dispatch(+aux), gate/up, down, combine
-# (with --combine fused the combine runs inside the down GEMM: one launch fewer)
+# launches of one forward: header clear (the router weight itself is split once, when the layer
+# is built), route, scan, dispatch(+aux), gate/up, down, combine (with --combine fused the combine
+# runs inside the down GEMM: one launch fewer)
 FWD_LAUNCHES = 7
 
 
@@ -485,9 +486,14 @@ def forward_stage_ms(layer, dm, x, tnb, out, flush, nb):
         flush.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         ev[0].record()
-        # "route" = router weight split + route + scan launches
-        B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, out["topk_idx"], out["topk_gate"],
-                out["n_real"], out["workspace"])
+        # "route" = header clear + route + scan launches from the prepared router weight, as in the
+        # forward (the fp32 CUDA-core router transposes its weight per call instead)
+        if layer.router_split is not None:
+            B.route_prepared(dm, x, layer.router_split, layer.router_bias, tnb, None, out["topk_idx"],
+                             out["topk_gate"], out["n_real"], out["workspace"])
+        else:
+            B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, out["topk_idx"], out["topk_gate"],
+                    out["n_real"], out["workspace"])
         ev[1].record()
         B.dispatch(dm, x, out["topk_idx"], out["workspace"], out["counts"], out["offsets"], out["perm_tok"],
                    out["slot_row"], out["xs"])  # the aux reduction rides in this launch, as in moe_forward
@@ -674,6 +680,7 @@ def main():
             dp_forward(layer, x, tnb, out, sums)
 
     # one forward, plus the aux sums and their finalize when data parallel
+    # (with the fp32 CUDA-core router its per-call weight transpose takes the header clear's place)
     kernels_per_step = FWD_LAUNCHES - (1 if args.combine == "fused" else 0) + (2 if world > 1 else 0)
 
     for _ in range(args.warmup):

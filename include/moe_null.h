@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define MOE_NULL_ABI_VERSION 4
+#define MOE_NULL_ABI_VERSION 5
 
 typedef void* moe_stream_t; /* a cudaStream_t */
 
@@ -115,6 +115,9 @@ typedef struct moe_weights {
   const uint16_t* shared_down;  /* [d, F_shared] bf16                           */
   const uint16_t* const_vectors; /* [V, d] bf16 constant experts' outputs, or
                                     NULL when V = 0                             */
+  const uint16_t* router_split;  /* [3 * P, d] bf16 from moe_prepare_router, or
+                                    NULL: moe_forward then splits w_router for
+                                    each call (tensor-core router only)         */
 } moe_weights_t;
 
 /* Outputs and intermediates of moe_forward (device pointers). R_cap = T*K. */
@@ -174,6 +177,18 @@ MOE_API int moe_pack_gate_up(const moe_dims_t* dims, const uint16_t* w_gate, con
                      const uint16_t* ws_gate, const uint16_t* ws_up, uint16_t* gate_up,
                      uint16_t* shared_gate_up, moe_stream_t stream);
 
+/* Element count (bf16) of the router weight split into three bf16 terms for the
+ * tensor-core router: 3 * P * d with P = N+1+C+V rounded up to a multiple of 16. */
+MOE_API size_t moe_router_split_elems(const moe_dims_t* dims);
+
+/* One-time preparation of the router weight for the tensor-core router (like
+ * moe_pack_gate_up for the expert weights): router_split [3 * P, d] receives the
+ * exact three-term bf16 split of w_router [N+1+C+V, d] (hi, mid and lo rows, zero
+ * rows past N+1+C+V; see moe_route). Passed as moe_weights_t.router_split, it spares
+ * moe_forward the split of every call. Redo it whenever w_router changes. */
+MOE_API int moe_prepare_router(const moe_dims_t* dims, const float* w_router, uint16_t* router_split,
+                               moe_stream_t stream);
+
 /* Routing (section 三: Null Expert 机制, 阈值解释, 负载均衡损失, Z-Loss).
  *  s[t, j] = sum_c fp32(x[t,c]) * w_router[j,c] + bias[j] (+ tok_null_bias[t]
  *  for j = N), to fp32 accuracy: by default on the tensor cores, with each
@@ -196,6 +211,14 @@ MOE_API int moe_route(const moe_dims_t* dims, const uint16_t* x, const float* w_
               const float* router_bias, const float* tok_null_bias, float* logits_out,
               int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* workspace,
               moe_stream_t stream);
+
+/* moe_route for the tensor-core router with its weight already split by
+ * moe_prepare_router (router_split [3 * P, d] bf16): one launch fewer per call.
+ * Same results as moe_route. Not for MOE_FLAG_ROUTER_FP32_CORES (MOE_ERR_INVALID_ARG). */
+MOE_API int moe_route_prepared(const moe_dims_t* dims, const uint16_t* x, const uint16_t* router_split,
+                               const float* router_bias, const float* tok_null_bias, float* logits_out,
+                               int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* workspace,
+                               moe_stream_t stream);
 
 /* moe_route without a workspace argument, for callers that cannot allocate
  * device memory: plugin-style interfaces that receive only their input and

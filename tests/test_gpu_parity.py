@@ -452,3 +452,42 @@ def test_forward_from_host_memory_in_chunks(name, chunk):
         assert torch.equal(st["counts_ext"], ref["counts_ext"])
         np.testing.assert_allclose(st["P"].cpu().numpy(), ref["P"].cpu().numpy(), rtol=1e-6, atol=1e-12)
         np.testing.assert_allclose(st["losses"].cpu().numpy(), ref["losses"].cpu().numpy(), rtol=1e-6)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_b", "pp_80rows", "skew"])
+def test_route_from_the_prepared_router_weight_is_bitwise_moe_route(name):
+    """moe_route_prepared (the weight split once by moe_prepare_router, as the layer's forward
+    uses it) gives exactly what moe_route (splitting per call) gives; the fp32 CUDA-core
+    router has no prepared form and is refused."""
+    from token_choice_routing_b200 import binding as B
+    cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP[name]
+    inp = I.make_inputs(cfg, weights=False)
+    from token_choice_routing_b200.layer import bf16_tensor
+    x = bf16_tensor(inp.x, "cuda")
+    w = torch.from_numpy(inp.w_router).cuda()
+    b = torch.from_numpy(inp.bias).cuda()
+    tnb = None if inp.tok_null_bias is None else torch.from_numpy(inp.tok_null_bias).cuda()
+    dm = B.dims(cfg.T, cfg.d, cfg.N, cfg.M, cfg.K, cfg.F, cfg.F_shared, 0, cfg.C, cfg.V)
+    split = torch.empty(B.router_split_elems(dm), dtype=torch.bfloat16, device="cuda")
+    B.prepare_router(dm, w, split)
+    outs = []
+    for prepared in (False, True):
+        ws = torch.empty(B.workspace_bytes(dm), dtype=torch.uint8, device="cuda")
+        o = [torch.empty((cfg.T, cfg.router_rows), dtype=torch.float32, device="cuda"),
+             torch.empty((cfg.T, cfg.K), dtype=torch.int32, device="cuda"),
+             torch.empty((cfg.T, cfg.K), dtype=torch.float32, device="cuda"),
+             torch.empty((cfg.T,), dtype=torch.int32, device="cuda")]
+        if prepared:
+            B.route_prepared(dm, x, split, b, tnb, *o, ws)
+        else:
+            B.route(dm, x, w, b, tnb, *o, ws)
+        torch.cuda.synchronize()
+        assert B.get_device_status(ws) == B.OK
+        outs.append(o)
+    for a, c in zip(*outs):
+        assert torch.equal(a, c)
+    dm32 = B.dims(cfg.T, cfg.d, cfg.N, cfg.M, cfg.K, cfg.F, cfg.F_shared, B.FLAG_ROUTER_FP32_CORES, cfg.C, cfg.V)
+    if cfg.C + cfg.V == 0:
+        ws = torch.empty(B.workspace_bytes(dm32), dtype=torch.uint8, device="cuda")
+        with pytest.raises(B.MoEError):
+            B.route_prepared(dm32, x, split, b, tnb, *outs[0], ws)

@@ -33,7 +33,7 @@ class Dims(C.Structure):
 
 class Weights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("w_router", "router_bias", "gate_up", "w_down",
-                                           "shared_gate_up", "shared_down", "const_vectors")]
+                                           "shared_gate_up", "shared_down", "const_vectors", "router_split")]
 
 
 OUTPUT_FIELDS = ("logits", "topk_idx", "topk_gate", "n_real", "counts", "offsets", "perm_tok",
@@ -76,7 +76,10 @@ def _load() -> C.CDLL:
         "moe_workspace_bytes": (sz, [pd]),
         "moe_packed_gate_up_elems": (sz, [pd, i32]),
         "moe_pack_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_router_split_elems": (sz, [pd]),
+        "moe_prepare_router": (i32, [pd, vp, vp, vp]),
         "moe_route": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_route_prepared": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_dispatch": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_ffn": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_gate_up": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -118,7 +121,7 @@ def _load() -> C.CDLL:
         f = getattr(lib, name)
         f.restype = res
         f.argtypes = args
-    if lib.moe_abi_version() != 4:
+    if lib.moe_abi_version() != 5:
         raise ImportError("libmoe_null ABI version mismatch")
     return lib
 
@@ -182,10 +185,25 @@ def pack_gate_up(dm, w_gate, w_up, ws_gate, ws_up, gate_up, shared_gate_up, stre
                                                      _stream(stream)))
 
 
+def router_split_elems(dm: Dims) -> int:
+    return int(LIB.moe_router_split_elems(C.byref(dm)))
+
+
+def prepare_router(dm, w_router, router_split, stream=None):
+    _check("moe_prepare_router", LIB.moe_prepare_router(C.byref(dm), _p(w_router), _p(router_split),
+                                                         _stream(stream)))
+
+
 def route(dm, x, w_router, bias, tok_null_bias, logits, topk_idx, topk_gate, n_real, ws, stream=None):
     _check("moe_route", LIB.moe_route(C.byref(dm), _p(x), _p(w_router), _p(bias), _p(tok_null_bias),
                                       _p(logits), _p(topk_idx), _p(topk_gate), _p(n_real), _p(ws),
                                       _stream(stream)))
+
+
+def route_prepared(dm, x, router_split, bias, tok_null_bias, logits, topk_idx, topk_gate, n_real, ws, stream=None):
+    _check("moe_route_prepared",
+           LIB.moe_route_prepared(C.byref(dm), _p(x), _p(router_split), _p(bias), _p(tok_null_bias), _p(logits),
+                                  _p(topk_idx), _p(topk_gate), _p(n_real), _p(ws), _stream(stream)))
 
 
 def dispatch(dm, x, topk_idx, ws, counts, offsets, perm_tok, slot_row, xs, stream=None):

@@ -96,6 +96,18 @@ int moe_pack_gate_up(const moe_dims_t* dims, const uint16_t* w_gate, const uint1
   return launch_pack_gate_up(*dims, w_gate, w_up, ws_gate, ws_up, gate_up, shared_gate_up, S(stream));
 }
 
+size_t moe_router_split_elems(const moe_dims_t* dims) {
+  if (check_dims(dims) != MOE_OK) return 0;
+  return (size_t)3 * route_npw(*dims) * dims->d;
+}
+
+int moe_prepare_router(const moe_dims_t* dims, const float* w_router, uint16_t* router_split,
+                       moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (!w_router || !router_split) return MOE_ERR_INVALID_ARG;
+  return launch_router_split(*dims, w_router, router_split, S(stream), nullptr);
+}
+
 int moe_route(const moe_dims_t* dims, const uint16_t* x, const float* w_router, const float* router_bias,
               const float* tok_null_bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
               int32_t* n_real, void* workspace, moe_stream_t stream) {
@@ -104,6 +116,17 @@ int moe_route(const moe_dims_t* dims, const uint16_t* x, const float* w_router, 
   if (!x || !w_router || !topk_idx || !topk_gate || !n_real || !workspace) return MOE_ERR_INVALID_ARG;
   return launch_route(*dims, x, w_router, router_bias, tok_null_bias, logits_out, topk_idx, topk_gate,
                       n_real, workspace, S(stream));
+}
+
+int moe_route_prepared(const moe_dims_t* dims, const uint16_t* x, const uint16_t* router_split,
+                       const float* router_bias, const float* tok_null_bias, float* logits_out, int32_t* topk_idx,
+                       float* topk_gate, int32_t* n_real, void* workspace, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (route_fp32_cores(*dims)) return MOE_ERR_INVALID_ARG;
+  if (dims->T == 0) return MOE_OK;
+  if (!x || !router_split || !topk_idx || !topk_gate || !n_real || !workspace) return MOE_ERR_INVALID_ARG;
+  return launch_route(*dims, x, nullptr, router_bias, tok_null_bias, logits_out, topk_idx, topk_gate, n_real,
+                      workspace, S(stream), router_split);
 }
 
 int moe_dispatch(const moe_dims_t* dims, const uint16_t* x, const int32_t* topk_idx, void* workspace,
@@ -253,7 +276,7 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
   if ((out->z != nullptr) != (out->z_shared != nullptr) || (out->z && !out->xs)) return MOE_ERR_INVALID_ARG;
   const cudaStream_t st = S(stream);
   MOE_CHECK(launch_route(*dims, x, w->w_router, w->router_bias, tok_null_bias, out->logits, out->topk_idx,
-                         out->topk_gate, out->n_real, workspace, st));
+                         out->topk_gate, out->n_real, workspace, st, w->router_split));
   MOE_CHECK(launch_dispatch(*dims, x, out->topk_idx, workspace, out->counts, out->offsets, out->perm_tok,
                             out->slot_row, out->xs, out->counts_ext, out->P, out->losses, st));
   if (out->z) {

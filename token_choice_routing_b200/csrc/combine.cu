@@ -25,7 +25,7 @@ constexpr int kCombineThreads = 256;
 // without a source already holds its result, bf16(shared), and is skipped.
 template <bool UNIT_ROWS, bool INPLACE>
 __global__ void __launch_bounds__(kCombineThreads, 3)
-combine_kernel(const uint16_t* ys, const uint16_t* sh, const float* __restrict__ gate,
+combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* sh, const float* __restrict__ gate,
                const int32_t* __restrict__ slot_row, const int32_t* __restrict__ topk_idx,
                const uint16_t* __restrict__ x, const uint16_t* __restrict__ cv, uint16_t* y, int T, int d, int K,
                long long rcap, int NM, int C, int V, uint32_t* status) {
@@ -69,12 +69,15 @@ combine_kernel(const uint16_t* ys, const uint16_t* sh, const float* __restrict__
       g = gn;
       continue;
     }
+    // the shared row's pieces of the next pass are loaded before this pass's stores (in place
+    // they are the same buffer, so the compiler would not move them above the stores itself)
+    const uint4* shr = reinterpret_cast<const uint4*>(sh + (size_t)t * d);
+    uint4 sa_n = (lane < nch) ? shr[lane] : make_uint4(0u, 0u, 0u, 0u);
+    uint4 sb_n = (32 + lane < nch) ? shr[32 + lane] : make_uint4(0u, 0u, 0u, 0u);
     for (int c0 = 0; c0 < nch; c0 += 64) {
       const int ca = c0 + lane, cb = c0 + 32 + lane;
       const bool oka = ca < nch, okb = cb < nch;
-      const uint4* shr = reinterpret_cast<const uint4*>(sh + (size_t)t * d);
-      const uint4 sa = oka ? __ldg(shr + ca) : make_uint4(0u, 0u, 0u, 0u);
-      const uint4 sb = okb ? __ldg(shr + cb) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 sa = sa_n, sb = sb_n;
       float acc_a[8], acc_b[8];
       bool first = true;
       unsigned m = srcs;
@@ -113,6 +116,11 @@ combine_kernel(const uint16_t* ys, const uint16_t* sh, const float* __restrict__
           }
         }
       } while (m != 0u);
+      if (c0 + 64 < nch) {
+        const int na = c0 + 64 + lane, nb = c0 + 96 + lane;
+        sa_n = (na < nch) ? shr[na] : make_uint4(0u, 0u, 0u, 0u);
+        sb_n = (nb < nch) ? shr[nb] : make_uint4(0u, 0u, 0u, 0u);
+      }
       if (oka)
         reinterpret_cast<uint4*>(y + (size_t)t * d)[ca] =
             make_uint4(pack_bf16x2(acc_a[0], acc_a[1]), pack_bf16x2(acc_a[2], acc_a[3]),

@@ -45,7 +45,8 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 struct WsLayout {
   int blk_tokens;    // tokens per route block (route_block_tokens)
   int nblk;          // route CTAs = ceil(T / blk_tokens)
-  size_t hdr;        // uint32 status at 0; int32 per-expert totals at kHdrTotOffset (512 B)
+  size_t hdr;        // uint32 status at 0; int32 per-expert totals at kHdrTotOffset; the down
+                     // GEMM's counters at kHdrCombineOffset (512 B)
   size_t counts_blk; // int32 [N][nblk]
   size_t bases;      // int32 [N][nblk]
   size_t ppart;      // float [nblk][N+1+C+V]
@@ -213,10 +214,17 @@ inline int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Launchers (each returns a moe_status_t after enqueuing).
+// w_split: the three-term bf16 router weight prepared by moe_prepare_router, or null to
+// split w_router into the workspace for this call (the tensor-core route; the fp32 route
+// ignores it).
 int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router,
                  const float* bias, const float* tok_null_bias, float* logits_out,
                  int32_t* topk_idx, float* topk_gate, int32_t* n_real, void* ws,
-                 cudaStream_t st);
+                 cudaStream_t st, const uint16_t* w_split = nullptr);
+// W_r fp32 [rows, d] -> the three bf16 terms [3 route_npw, d] (hi, mid, lo rows); with ws
+// set, the same launch also clears the workspace header; with w3 null it only does that.
+int launch_router_split(const moe_dims_t& d, const float* w_router, uint16_t* w3, cudaStream_t st,
+                        void* ws = nullptr);
 // The fp32 CUDA-core route (route_fp32.cu) and the per-expert scan both routes end with.
 int launch_route_fp32(const moe_dims_t& d, const uint16_t* x, const float* w_router,
                       const float* bias, const float* tok_null_bias, float* logits_out,

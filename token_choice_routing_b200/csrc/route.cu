@@ -40,6 +40,7 @@
 namespace moe {
 
 struct RouteArgs {
+  int32_t* tot;       // [N] rows per expert (integer atomics; zero at the start of every call)
   const float* bias;  // [N+1] or null
   const float* tnb;   // [T] or null
   float* logits;      // [T, N+1] or null
@@ -48,7 +49,6 @@ struct RouteArgs {
   int32_t* n_real;
   // workspace
   uint32_t* hdr;  // [0] status
-  int32_t* tot;   // [N] rows per expert (integer atomics)
   int32_t* counts_blk;
   int32_t* bases;
   float* ppart;
@@ -78,14 +78,14 @@ __device__ __forceinline__ void split3(float w, uint16_t& h, uint16_t& m, uint16
   l = __bfloat16_as_ushort(bl);
 }
 
-// One thread per 8 d-columns of one padded row. Block 0 also clears the first
-// `nclear` words of the workspace header (status word, per-expert totals and the
-// counters of the down GEMM with the combine folded in), which must start at zero
-// for every layer call.
+// One thread per 8 d-columns of one padded row. With hdr set, block 0 also clears the
+// first `nclear` words of the workspace header (status word, per-expert totals and the
+// counters of the down GEMM with the combine folded in), which must start at zero for
+// every layer call; with npw = 0 that is all it does (the weight was split beforehand).
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, uint16_t* __restrict__ w3,
                                                            int rows, int npw, int d, uint32_t* hdr, int nclear) {
   pdl_wait_then_release();
-  if (blockIdx.x == 0)
+  if (hdr != nullptr && blockIdx.x == 0)
     for (int i = threadIdx.x; i < nclear; i += blockDim.x) hdr[i] = 0u;
   const int nch = d >> 3;
   const long long total = (long long)npw * nch;
@@ -805,9 +805,21 @@ int launch_route_scan(const moe_dims_t& d, void* ws, cudaStream_t st) {
   return launch_pdl(scan_kernel, dim3(d.N + L.nparts), dim3(kScanThreads), 0, st, sa);
 }
 
+int launch_router_split(const moe_dims_t& d, const float* w_router, uint16_t* w3, cudaStream_t st, void* ws) {
+  const int npw = (w3 != nullptr) ? route_npw(d) : 0;  // no weight: only the header is cleared
+  const long long work = (long long)npw * (d.d / 8);
+  long long grid = (work + 255) / 256;
+  if (grid > (long long)sm_count() * 8) grid = (long long)sm_count() * 8;
+  if (grid < 1) grid = 1;
+  uint32_t* hdr = (ws != nullptr) ? ws_ptr<uint32_t>(ws, ws_layout(d).hdr) : nullptr;
+  const int nclear = (int)(kHdrClearBytes / sizeof(uint32_t));
+  return launch_pdl(router_split_kernel, dim3((unsigned)grid), dim3(256), 0, st, w_router, w3, router_rows(d), npw,
+                    d.d, hdr, nclear);
+}
+
 int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, const float* bias,
                  const float* tok_null_bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
-                 int32_t* n_real, void* ws, cudaStream_t st) {
+                 int32_t* n_real, void* ws, cudaStream_t st, const uint16_t* w_split) {
   if (route_fp32_cores(d))
     return launch_route_fp32(d, x, w_router, bias, tok_null_bias, logits_out, topk_idx, topk_gate, n_real,
                              ws, st);
@@ -837,18 +849,16 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.K = d.K;
   a.nblk = L.nblk;
   a.ncols = router_rows(d);
-  // the split router weight for this call (its block 0 also clears the status word
-  // and the per-expert totals), then tensor maps over x and it
+  // the split router weight: prepared once by the caller (moe_prepare_router), or split
+  // here into the workspace for this call; the same launch clears the workspace header (with
+  // a prepared weight that is all it does, in one block); then tensor maps over x and it
   const int npw = route_npw(d);
-  uint16_t* w3 = ws_ptr<uint16_t>(ws, L.wprep);
+  const uint16_t* w3 = w_split;
   {
-    const long long work = (long long)npw * (d.d / 8);
-    long long grid = (work + 255) / 256;
-    if (grid > (long long)sm_count() * 8) grid = (long long)sm_count() * 8;
-    const int nclear = (int)(kHdrClearBytes / sizeof(uint32_t));
-    const int r = launch_pdl(router_split_kernel, dim3((unsigned)grid), dim3(256), 0, st, w_router, w3,
-                             router_rows(d), npw, d.d, a.hdr, nclear);
+    uint16_t* w3c = (w3 == nullptr) ? ws_ptr<uint16_t>(ws, L.wprep) : nullptr;
+    const int r = launch_router_split(d, w_router, w3c, st, ws);
     if (r != MOE_OK) return r;
+    if (w3 == nullptr) w3 = w3c;
   }
   // the weight's box: all 3 npw rows, or half of them for each CTA of a pair
   const uint32_t wbox = (uint32_t)(route_pairs(L.nblk) ? 3 * npw / 2 : 3 * npw);

@@ -50,8 +50,12 @@ def dp_forward(layer, x, tok_null_bias, out, sums, group=None):
     from . import binding as B
     dm = layer.dims(x.shape[0])
     ws = out["workspace"]
-    B.route(dm, x, layer.w_router, layer.router_bias, tok_null_bias, out.get("logits"), out["topk_idx"],
-            out["topk_gate"], out["n_real"], ws)
+    if getattr(layer, "router_split", None) is not None:
+        B.route_prepared(dm, x, layer.router_split, layer.router_bias, tok_null_bias, out.get("logits"),
+                         out["topk_idx"], out["topk_gate"], out["n_real"], ws)
+    else:
+        B.route(dm, x, layer.w_router, layer.router_bias, tok_null_bias, out.get("logits"), out["topk_idx"],
+                out["topk_gate"], out["n_real"], ws)
     B.aux_sums(dm, ws, sums)
     allreduce_aux_sums(sums, group)
     B.aux_finalize(dm, sums, out["counts_ext"], out["P"], out["losses"])

@@ -252,8 +252,12 @@ def ep_forward(shard: ExpertShard, x: torch.Tensor, tok_null_bias: Optional[torc
     ws = out["workspace"]
     if out.get("shared_out") is None or out.get("xs") is None:
         raise ValueError("expert parallelism needs xs and a shared-expert output buffer (or y)")
-    B.route(dm, x, layer.w_router, layer.router_bias, tok_null_bias, out.get("logits"), out["topk_idx"],
-            out["topk_gate"], out["n_real"], ws)
+    if layer.router_split is not None:
+        B.route_prepared(dm, x, layer.router_split, layer.router_bias, tok_null_bias, out.get("logits"),
+                         out["topk_idx"], out["topk_gate"], out["n_real"], ws)
+    else:
+        B.route(dm, x, layer.w_router, layer.router_bias, tok_null_bias, out.get("logits"), out["topk_idx"],
+                out["topk_gate"], out["n_real"], ws)
     B.aux_sums(dm, ws, sums)
     transport.all_reduce_sum(sums)
     B.aux_finalize(dm, sums, out["counts_ext"], out["P"], out["losses"])

@@ -60,11 +60,17 @@ class MoENullLayer:
         self.shared_gate_up = torch.empty(B.packed_gate_up_elems(dm, True), dtype=torch.bfloat16, device=dev)
         B.pack_gate_up(dm, w_gate.contiguous(), w_up.contiguous(), ws_gate.contiguous(), ws_up.contiguous(),
                        self.gate_up, self.shared_gate_up)
+        # the tensor-core router's three-term split of W_r, prepared once (moe_prepare_router)
+        self.router_split = None
+        if router == "tensor":
+            self.router_split = torch.empty(B.router_split_elems(dm), dtype=torch.bfloat16, device=dev)
+            B.prepare_router(dm, self.w_router, self.router_split)
         self._weights = B.Weights(self.w_router.data_ptr(),
                                   None if self.router_bias is None else self.router_bias.data_ptr(),
                                   self.gate_up.data_ptr(), self.w_down.data_ptr(),
                                   self.shared_gate_up.data_ptr(), self.shared_down.data_ptr(),
-                                  None if self.const_vectors is None else self.const_vectors.data_ptr())
+                                  None if self.const_vectors is None else self.const_vectors.data_ptr(),
+                                  None if self.router_split is None else self.router_split.data_ptr())
 
     @classmethod
     def from_inputs(cls, inp, device="cuda", router: str = "tensor", ffn: str = "auto") -> "MoENullLayer":
