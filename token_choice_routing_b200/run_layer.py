@@ -32,7 +32,7 @@ def main(argv=None) -> int:
     ap.add_argument("--combine", default="inplace", choices=["inplace", "separate", "fused"])
     ap.add_argument("--forwards", type=int, default=3)
     ap.add_argument("--router", default="tensor", choices=["tensor", "fp32_cores"])
-    ap.add_argument("--ffn", default="single", choices=["single", "pair"])
+    ap.add_argument("--ffn", default="auto", choices=["auto", "single", "pair"])
     ap.add_argument("--backwards", type=int, default=0)
     ap.add_argument("--save-preact", action="store_true")
     a = ap.parse_args(argv)
