@@ -649,7 +649,7 @@ def main():
 
     from token_choice_routing_b200 import binding as B
     from token_choice_routing_b200 import inputs as I
-    from token_choice_routing_b200.dist import dp_forward
+    from token_choice_routing_b200.dist import allreduce_aux_sums, dp_forward
     from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
 
     rank = int(os.environ.get("RANK", "0"))
@@ -693,6 +693,8 @@ def main():
 
     with ClockSampler(local) as clk:
         step_ms = timed_events(step, args.steps, 0, flush, sync_before=dist.barrier if world > 1 else None)
+    if world > 1:
+        dist.barrier()
     total_ms = sum(step_ms)
     med_ms = statistics.median(step_ms)
     if world > 1:
@@ -748,11 +750,13 @@ def main():
     pipe = layer.alloc_host_pipeline(chunk)
 
     def e2e_step():
-        st = layer.forward_host(x_pin, y_pin, pipe, tnb_pin)
+        st = layer.forward_host(x_pin, y_pin, pipe, tnb_pin, reduce_sums=allreduce_aux_sums if world > 1 else None)
         loss_pin.copy_(st["losses"], non_blocking=True)
         cext_pin.copy_(st["counts_ext"], non_blocking=True)
 
-    e2e_ms = timed_events(e2e_step, args.steps, args.warmup, flush)
+    e2e_ms = timed_events(e2e_step, args.steps, args.warmup, flush, sync_before=dist.barrier if world > 1 else None)
+    if world > 1:
+        dist.barrier()
     e2e_total = sum(e2e_ms)
     if world > 1:
         t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)

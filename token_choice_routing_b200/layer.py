@@ -211,7 +211,8 @@ class MoENullLayer:
                     copy_in=torch.cuda.Stream(device=dev), copy_out=torch.cuda.Stream(device=dev))
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, pipe: Dict[str, object],
-                     tok_null_bias_host: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+                     tok_null_bias_host: Optional[torch.Tensor] = None,
+                     reduce_sums=None) -> Dict[str, torch.Tensor]:
         """The forward from and to host memory (pinned, for asynchronous copies), in token
         chunks: while chunk i runs on the current stream, chunk i+1's tokens are copied in on
         one stream and chunk i-1's y copied out on another. Every step of the layer is per
@@ -219,7 +220,9 @@ class MoENullLayer:
         L_bal and L_z, which are means over the whole batch, are summed over the chunks on the
         device (moe_aux_sums / moe_aux_sums_accumulate) and finalised once. Returns the device
         counts_ext, P and losses of the batch. The current stream is ordered after the last
-        copy, so synchronising it makes y_host complete."""
+        copy, so synchronising it makes y_host complete. reduce_sums (data parallel: e.g.
+        dist.allreduce_aux_sums) is applied to the summed statistics before they are
+        finalised, so the losses are the whole job's."""
         T = x_host.shape[0]
         chunk = pipe["chunk"]
         comp = torch.cuda.current_stream(self.device)
@@ -259,6 +262,8 @@ class MoENullLayer:
                 cout.wait_event(ev_done[k])
                 y_host[a:b].copy_(o["y"][:Tc], non_blocking=True)
                 ev_out[k].record(cout)
+        if reduce_sums is not None:
+            reduce_sums(pipe["sums"])
         B.aux_finalize(self.dims(T), pipe["sums"], pipe["counts_ext"], pipe["P"], pipe["losses"], comp)
         comp.wait_stream(cout)
         return dict(counts_ext=pipe["counts_ext"], P=pipe["P"], losses=pipe["losses"])
