@@ -650,7 +650,7 @@ def main():
     from token_choice_routing_b200 import binding as B
     from token_choice_routing_b200 import inputs as I
     from token_choice_routing_b200.dist import allreduce_aux_sums, dp_forward
-    from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor
+    from token_choice_routing_b200.layer import MoENullLayer, bf16_tensor, chunk_bounds
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -747,7 +747,7 @@ def main():
     loss_pin = torch.empty(2, dtype=torch.float32).pin_memory()
     cext_pin = torch.empty(out["counts_ext"].numel(), dtype=torch.int32).pin_memory()
     chunk = min(T, args.e2e_chunk)
-    pipe = layer.alloc_host_pipeline(chunk)
+    pipe = layer.alloc_host_pipeline(chunk, nsets=3)
 
     def e2e_step():
         st = layer.forward_host(x_pin, y_pin, pipe, tnb_pin, reduce_sums=allreduce_aux_sums if world > 1 else None)
@@ -770,8 +770,8 @@ def main():
            "h2d_bytes_per_step": int(h2d),
            "d2h_bytes_per_step": int(y_pin.numel() * 2 + 4 * loss_pin.numel() + 4 * cext_pin.numel()),
            "ms_per_step": e2e_total / args.steps, "ms_per_step_median": statistics.median(e2e_ms),
-           "chunk_tokens": chunk,
-           "launches_per_step": (FWD_LAUNCHES + 1) * ((T + chunk - 1) // chunk) + 1}
+           "chunk_tokens": chunk, "chunks_per_step": len(chunk_bounds(T, chunk)),
+           "launches_per_step": (FWD_LAUNCHES + 1) * len(chunk_bounds(T, chunk)) + 1}
     del x_pin, y_pin, pipe
 
     backward = None

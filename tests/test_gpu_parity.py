@@ -428,13 +428,13 @@ def test_down_combine_entry_point_called_alone_twice():
         assert torch.equal(out["y"], y0)
 
 
-@pytest.mark.parametrize("name,chunk", [("qwen3_0p6b", 4096), ("qwen3_0p6b", 5000), ("skew_small", 200),
-                                        ("tiny", 256), ("pp_a", 128)])
-def test_forward_from_host_memory_in_chunks(name, chunk):
-    """MoENullLayer.forward_host: the batch in token chunks from and to pinned host memory,
-    copies overlapping the chunks' compute. y is bit-identical to one forward over the whole
-    batch; the batch's statistics (summed over the chunks) give its counts exactly and P and
-    the losses to fp64 summation order."""
+@pytest.mark.parametrize("name,chunk,nsets", [("qwen3_0p6b", 4096, 2), ("qwen3_0p6b", 5000, 3),
+                                              ("skew_small", 200, 2), ("tiny", 256, 2), ("pp_a", 128, 3)])
+def test_forward_from_host_memory_in_chunks(name, chunk, nsets):
+    """MoENullLayer.forward_host: the batch in token chunks (short ones at both ends) from and
+    to pinned host memory, copies overlapping the chunks' compute, two or three buffer sets.
+    y is bit-identical to one forward over the whole batch; the batch's statistics (summed
+    over the chunks) give its counts exactly and P and the losses to fp64 summation order."""
     cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP[name]
     inp = I.make_inputs(cfg)
     layer, x, tnb = H.make_layer(inp)
@@ -443,7 +443,7 @@ def test_forward_from_host_memory_in_chunks(name, chunk):
     x_pin = x.cpu().pin_memory()
     y_pin = torch.empty_like(x_pin).pin_memory()
     tnb_pin = None if tnb is None else tnb.cpu().pin_memory()
-    pipe = layer.alloc_host_pipeline(chunk)
+    pipe = layer.alloc_host_pipeline(chunk, nsets)
     for _ in range(2):  # twice: the pipeline's buffers are reused
         y_pin.zero_()
         st = layer.forward_host(x_pin, y_pin, pipe, tnb_pin)

@@ -8,6 +8,8 @@
 // deterministic: fp32 accumulation in rank order, one bf16 rounding.
 #include "moe_internal.cuh"
 
+#include <algorithm>
+
 namespace moe {
 
 constexpr int kCombineThreads = 256;
@@ -23,15 +25,17 @@ constexpr int kCombineThreads = 256;
 // having been applied upstream; copy slots still take g times their row of x.
 // INPLACE (sh == y, the shared expert's output written into y by the down GEMM): a token
 // without a source already holds its result, bf16(shared), and is skipped.
-template <bool UNIT_ROWS, bool INPLACE>
-__global__ void __launch_bounds__(kCombineThreads, 3)
+// THREADS: 256 for the persistent grid (one wave, each warp looping over tokens with the
+// next token's slots prefetched), 64 for a grid of one token per warp (small batches).
+template <bool UNIT_ROWS, bool INPLACE, int THREADS>
+__global__ void __launch_bounds__(THREADS, 768 / THREADS)
 combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* sh, const float* __restrict__ gate,
                const int32_t* __restrict__ slot_row, const int32_t* __restrict__ topk_idx,
                const uint16_t* __restrict__ x, const uint16_t* __restrict__ cv, uint16_t* y, int T, int d, int K,
                long long rcap, int NM, int C, int V, uint32_t* status) {
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
-  const int wpb = kCombineThreads / 32;
+  const int wpb = THREADS / 32;
   const int nch = d >> 3;
   const int stride = gridDim.x * wpb;
   int t = blockIdx.x * wpb + (threadIdx.x >> 5);
@@ -135,33 +139,54 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* sh, const float*
   }
 }
 
-// one wave of resident CTAs; each warp then loops over tokens
-static int combine_grid(const moe_dims_t& d) {
+// Grid choice. A persistent grid (one wave of 256-thread CTAs, each warp looping over
+// tokens and prefetching the next token's slots) hides the slot lookups, but its warps take
+// fixed shares of the tokens: with few tokens per warp the share with the most sources sets
+// the time. Below kCombineTokensPerWarp tokens per resident warp the grid is one token per
+// warp in 64-thread CTAs instead, and the block scheduler balances the load.
+// (B200, in place, L2 flushed: T = 16384 at the 1.7B shape with K = 8, 73 -> 53 us; at
+// T = 131072 the persistent grid stays ahead, 162 against 169-179 us.)
+constexpr int kCombineTokensPerWarp = 16;
+constexpr int kCombineSmallThreads = 64;
+
+struct CombineGrid {
+  int blocks;
+  bool persistent;
+};
+
+static CombineGrid combine_grid(const moe_dims_t& d) {
   static int per_sm[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   int occ = (dev >= 0 && dev < 64) ? per_sm[dev] : 0;
   if (occ == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_kernel<false, false>, kCombineThreads, 0) !=
-            cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_kernel<false, false, kCombineThreads>,
+                                                      kCombineThreads, 0) != cudaSuccess ||
         occ < 1)
       occ = 1;
     if (dev >= 0 && dev < 64) per_sm[dev] = occ;
   }
   const int wpb = kCombineThreads / 32;
-  int grid = (d.T + wpb - 1) / wpb;
-  const int cap = sm_count() * occ;
-  if (grid > cap) grid = cap;
-  return grid < 1 ? 1 : grid;
+  const long long resident_warps = (long long)sm_count() * occ * wpb;
+  if ((long long)d.T < kCombineTokensPerWarp * resident_warps) {
+    const int swpb = kCombineSmallThreads / 32;
+    return {(int)std::max<long long>(1, ((long long)d.T + swpb - 1) / swpb), false};
+  }
+  return {(int)std::max<long long>(1, resident_warps / wpb), true};
 }
 
 int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
                    const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
                    const uint16_t* const_vectors, uint16_t* y, cudaStream_t st) {
-  const int grid = combine_grid(d);
+  const CombineGrid g = combine_grid(d);
   // shared_out == y: the shared expert's output is already in y; tokens without a source keep it
-  auto kern = (shared_out == y) ? combine_kernel<false, true> : combine_kernel<false, false>;
-  return launch_pdl(kern, dim3(grid), dim3(kCombineThreads), 0, st, ys, shared_out, topk_gate, slot_row, topk_idx, x,
+  const bool inplace = shared_out == y;
+  auto kern = g.persistent ? (inplace ? combine_kernel<false, true, kCombineThreads>
+                                      : combine_kernel<false, false, kCombineThreads>)
+                           : (inplace ? combine_kernel<false, true, kCombineSmallThreads>
+                                      : combine_kernel<false, false, kCombineSmallThreads>);
+  const int threads = g.persistent ? kCombineThreads : kCombineSmallThreads;
+  return launch_pdl(kern, dim3(g.blocks), dim3(threads), 0, st, ys, shared_out, topk_gate, slot_row, topk_idx, x,
                     const_vectors, y, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, d.V, nullptr);
 }
 
@@ -171,10 +196,12 @@ int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shar
 int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint16_t* dxs, const int32_t* slot_row,
                       const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, uint16_t* dx,
                       uint32_t* status, cudaStream_t st) {
-  const int grid = combine_grid(d);
-  return launch_pdl(combine_kernel<true, false>, dim3(grid), dim3(kCombineThreads), 0, st, dxs, dx_shared, topk_gate,
-                    slot_row, topk_idx, dy, (const uint16_t*)nullptr, dx, d.T, d.d, d.K, (long long)d.T * d.K,
-                    d.N + d.M, d.C, 0, status);
+  const CombineGrid g = combine_grid(d);
+  auto kern = g.persistent ? combine_kernel<true, false, kCombineThreads>
+                           : combine_kernel<true, false, kCombineSmallThreads>;
+  const int threads = g.persistent ? kCombineThreads : kCombineSmallThreads;
+  return launch_pdl(kern, dim3(g.blocks), dim3(threads), 0, st, dxs, dx_shared, topk_gate, slot_row, topk_idx, dy,
+                    (const uint16_t*)nullptr, dx, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, 0, status);
 }
 
 }  // namespace moe

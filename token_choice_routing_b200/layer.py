@@ -6,7 +6,7 @@ caller-owned buffers and workspace with torch, and runs the forward through
 """
 from __future__ import annotations
 
-from typing import Dict, Optional
+from typing import Dict, List, Optional, Tuple
 
 import numpy as np
 import torch
@@ -18,6 +18,37 @@ def bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
     """uint16 bf16 bit array (host) -> torch.bfloat16 tensor on ``device``."""
     t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
     return t.to(device)
+
+
+def chunk_bounds(T: int, chunk: int) -> List[Tuple[int, int]]:
+    """Token ranges [a, b) of the host-buffer forward's chunks, none longer than ``chunk``.
+
+    Nothing overlaps the first chunk's copy in or the last chunk's copy out, so the batch
+    starts and ends with short chunks (chunk/8, chunk/4, chunk/2, ... and the same in reverse),
+    and the tokens between them are split into equal chunks of at most ``chunk``. A batch too
+    short for both ramps is split into equal chunks of at most chunk/8 (or one chunk)."""
+    if T <= 0:
+        return []
+    chunk = max(1, int(chunk))
+    ramp = []
+    s = max(1, chunk // 8)
+    while s < chunk:
+        ramp.append(s)
+        s *= 2
+    middle = T - 2 * sum(ramp)
+    if ramp and middle >= 1:
+        m = -(-middle // chunk)
+        sizes = ramp + [middle // m + (1 if i < middle % m else 0) for i in range(m)] + ramp[::-1]
+    else:
+        piece = max(1, chunk // 8) if ramp else chunk
+        n = -(-T // piece)
+        sizes = [T // n + (1 if i < T % n else 0) for i in range(n)]
+    bounds, a = [], 0
+    for sz in sizes:
+        bounds.append((a, a + sz))
+        a += sz
+    assert a == T
+    return bounds
 
 
 class MoENullLayer:
@@ -191,13 +222,13 @@ class MoENullLayer:
         B.backward(self.dims(T), self._weights, sv, dy, alpha, beta, g, grads["workspace"], stream)
         return grads
 
-    def alloc_host_pipeline(self, chunk: int) -> Dict[str, object]:
-        """Device buffers for forward_host with token chunks of ``chunk``: two chunk-sized
-        output sets and input stagings (one chunk computes while the next is copied in and the
-        previous one copied out), the summed statistics and the batch's counts, P and losses,
-        and the two copy streams."""
+    def alloc_host_pipeline(self, chunk: int, nsets: int = 2) -> Dict[str, object]:
+        """Device buffers for forward_host with token chunks of at most ``chunk``: ``nsets``
+        chunk-sized output sets and input stagings (one chunk computes while the next is copied
+        in and the previous one copied out), the summed statistics and the batch's counts, P
+        and losses, and the two copy streams."""
         dev = self.device
-        sets = [self.alloc(chunk, logits=False) for _ in range(2)]
+        sets = [self.alloc(chunk, logits=False) for _ in range(max(2, int(nsets)))]
         for o in sets:
             o["x_stage"] = torch.empty((chunk, self.d), dtype=torch.bfloat16, device=dev)
             o["tnb_stage"] = torch.empty((chunk,), dtype=torch.float32, device=dev)
@@ -214,8 +245,8 @@ class MoENullLayer:
                      tok_null_bias_host: Optional[torch.Tensor] = None,
                      reduce_sums=None) -> Dict[str, torch.Tensor]:
         """The forward from and to host memory (pinned, for asynchronous copies), in token
-        chunks: while chunk i runs on the current stream, chunk i+1's tokens are copied in on
-        one stream and chunk i-1's y copied out on another. Every step of the layer is per
+        chunks (``chunk_bounds``): while chunk i runs on the current stream, chunk i+1's tokens
+        are copied in on one stream and chunk i-1's y copied out on another. Every step of the layer is per
         token, so y is bit-identical to one forward over the whole batch; the statistics of
         L_bal and L_z, which are means over the whole batch, are summed over the chunks on the
         device (moe_aux_sums / moe_aux_sums_accumulate) and finalised once. Returns the device
@@ -229,25 +260,24 @@ class MoENullLayer:
         cin, cout = pipe["copy_in"], pipe["copy_out"]
         sets = pipe["sets"]
         cin.wait_stream(comp)  # nothing is copied in before earlier work on this stream
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        ev_out = [torch.cuda.Event() for _ in range(2)]
-        n = (T + chunk - 1) // chunk
-        for c in range(n):
-            k = c % 2
+        ev_in = [torch.cuda.Event() for _ in sets]
+        ev_done = [torch.cuda.Event() for _ in sets]
+        ev_out = [torch.cuda.Event() for _ in sets]
+        ns = len(sets)
+        for c, (a, b) in enumerate(chunk_bounds(T, chunk)):
+            k = c % ns
             o = sets[k]
-            a, b = c * chunk, min(T, (c + 1) * chunk)
             Tc = b - a
             with torch.cuda.stream(cin):
-                if c >= 2:
-                    cin.wait_event(ev_done[k])  # chunk c-2 no longer reads this staging
+                if c >= ns:
+                    cin.wait_event(ev_done[k])  # the set's previous chunk no longer reads this staging
                 o["x_stage"][:Tc].copy_(x_host[a:b], non_blocking=True)
                 if tok_null_bias_host is not None:
                     o["tnb_stage"][:Tc].copy_(tok_null_bias_host[a:b], non_blocking=True)
                 ev_in[k].record(cin)
             comp.wait_event(ev_in[k])
-            if c >= 2:
-                comp.wait_event(ev_out[k])  # chunk c-2's y has been copied out of this set
+            if c >= ns:
+                comp.wait_event(ev_out[k])  # the set's previous chunk's y has been copied out
             dm = self.dims(Tc)
             x = o["x_stage"][:Tc]
             tnb = None if tok_null_bias_host is None else o["tnb_stage"][:Tc]
