@@ -412,7 +412,9 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         "preactivations": "saved by the forward (training mode); the SwiGLU derivative is an elementwise pass",
         "forward_training_ms": fwd_train_ms, "backward_recompute_ms": recompute_ms,
         "ffn_tflops_real_rows": gemm_flops / (gemm_ms * 1e9),
-        "roofline": {"kernel": f"{top} grouped GEMM (tcgen05)", "bound": "tensor",
+        "roofline": {"kernel": f"{top} grouped GEMM (tcgen05"
+                               + (", CTA pairs)" if top.startswith("wgrad") and layer.wgrad == "pair" else ")"),
+                     "bound": "tensor",
                      "achieved": fl[top] / (kms[top] * 1e9), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": fl[top] / (kms[top] * 1e9) / bf16_peak, "peak_kind": f"{peak_kind} bf16 burst",
                      "traffic": recorded_traffic(cfg.name, top, BWD_GEMM_PROFILE, BWD_GEMM_SOURCES),

@@ -98,6 +98,15 @@ typedef enum {
  * up to fp32 accumulation order. */
 #define MOE_FLAG_FFN_CTA_PAIR 2u
 
+/* Weight gradients of the backward's expert GEMMs (moe_expert_wgrad_down,
+ * moe_expert_wgrad_gate_up, moe_backward) on CTA pairs: 256 output rows x 256
+ * columns per tile, one tcgen05 MMA shared by the two CTAs of a cluster, where
+ * the output rows per expert are a multiple of 256 (d for W_down, 2 F and
+ * 2 F_shared for gate/up) and the columns a multiple of 256 (F and F_shared,
+ * d); otherwise single-CTA tiles. The same fp32 sums in the same order as the
+ * single-CTA tiles, so the same results bit for bit. */
+#define MOE_FLAG_WGRAD_CTA_PAIR 4u
+
 typedef struct moe_dims {
   int32_t T, d, N, M, K, F, F_shared;
   uint32_t flags;

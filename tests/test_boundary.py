@@ -74,10 +74,11 @@ def test_check_dims(lib):
     assert B.check_dims(B.dims(**dict(ok, M=0, K=9), C=0, V=0)) == B.ERR_INVALID_ARG  # K > N+M
     assert B.check_dims(B.dims(**dict(ok, M=0, K=9), C=1, V=0)) == B.OK  # K <= N+M+C+V
     dm = good()
-    for f in (B.FLAG_ROUTER_FP32_CORES, B.FLAG_FFN_CTA_PAIR, B.FLAG_ROUTER_FP32_CORES | B.FLAG_FFN_CTA_PAIR):
+    for f in (B.FLAG_ROUTER_FP32_CORES, B.FLAG_FFN_CTA_PAIR, B.FLAG_ROUTER_FP32_CORES | B.FLAG_FFN_CTA_PAIR,
+              B.FLAG_WGRAD_CTA_PAIR, B.FLAG_FFN_CTA_PAIR | B.FLAG_WGRAD_CTA_PAIR):
         dm.flags = f
         assert B.check_dims(dm) == B.OK, f
-    for f in (4, 8, 0x80000000, B.FLAG_ROUTER_FP32_CORES | 4):
+    for f in (8, 16, 0x80000000, B.FLAG_ROUTER_FP32_CORES | 8):
         dm.flags = f
         assert B.check_dims(dm) == B.ERR_INVALID_ARG, f
 

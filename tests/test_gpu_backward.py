@@ -196,6 +196,62 @@ def test_backward_step_entry_points_match_the_whole_call():
         assert torch.equal(g[k], g3[k]), k
 
 
+# shapes where the weight gradients can run on CTA pairs: output rows per expert (d for
+# W_down, 2 F and 2 F_shared for gate/up) and columns (F, F_shared, d) multiples of 256
+PAIR_CASES = {
+    "plain": I.small_config("wgp_plain", T=700, d=512, N=6, F=256, F_shared=256, K=2, M=2, config_id=941),
+    # T > 2048: the shared expert's K chunks (fp32 partials, then the reduce)
+    "split": I.small_config("wgp_split", T=4500, d=256, N=8, F=256, F_shared=512, K=4, M=8, config_id=942),
+    # experts without rows, ragged tails of every length
+    "skew": I.small_config("wgp_skew", T=1500, d=512, N=64, F=256, F_shared=256, K=8, M=64, config_id=943,
+                           skew=True, seqs=2),
+}
+
+
+@pytest.mark.parametrize("name", list(PAIR_CASES))
+def test_wgrad_on_cta_pairs_is_bitwise_the_single_cta_wgrad(name):
+    """moe_expert_wgrad_down / moe_expert_wgrad_gate_up with MOE_FLAG_WGRAD_CTA_PAIR (256 x 256
+    tiles, one MMA shared by two CTAs) give exactly the single-CTA weight gradients: the same
+    fp32 sums over the same 16-row steps, in the same order. The layer's backward (pairs by
+    default) is checked against the oracle here too."""
+    from token_choice_routing_b200 import binding as B
+    cfg = PAIR_CASES[name]
+    inp, layer, x, out, dy, dy_bits, g = run(cfg)
+    T, c = cfg.T, cfg
+    flags = layer.dims(T).flags & ~B.FLAG_WGRAD_CTA_PAIR
+    dm = B.dims(T, c.d, c.N, c.M, c.K, c.F, c.F_shared, flags, c.C, c.V)
+    dmp = B.dims(T, c.d, c.N, c.M, c.K, c.F, c.F_shared, flags | B.FLAG_WGRAD_CTA_PAIR, c.C, c.V)
+    g2 = layer.alloc_grads(T)
+    bws = g2["workspace"]
+    R = T * c.K
+    dys = torch.empty((R, c.d), dtype=torch.bfloat16, device="cuda")
+    dg = torch.empty((T, c.K), dtype=torch.float32, device="cuda")
+    ds = torch.empty((T, c.N + 1), dtype=torch.float32, device="cuda")
+    B.clear_device_status(bws)
+    B.combine_backward(dm, dy, out["ys"], out["topk_gate"], out["slot_row"], dys, dg, bws)
+    B.router_backward(dm, out["logits"], out["topk_idx"], out["topk_gate"], dg, out["counts_ext"], T, ALPHA, BETA,
+                      ds, bws, g2["dtok_null_bias"])
+    B.expert_dgrad_down(dm, out["offsets"], dys, dy, layer.w_down, layer.shared_down, bws)
+    B.expert_swiglu_backward(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, bws)
+    res = {}
+    for tag, d_ in (("single", dm), ("pair", dmp)):
+        o = {k: torch.full_like(g[k], float("nan")) for k in ("dw_down", "dws_down", "dw_gate", "dw_up", "dws_gate",
+                                                             "dws_up")}
+        B.expert_wgrad_down(d_, out["offsets"], dys, dy, out["h"], out["h_shared"], o["dw_down"], o["dws_down"], bws)
+        B.expert_wgrad_gate_up(d_, out["offsets"], out["xs"], x, o["dw_gate"], o["dw_up"], o["dws_gate"],
+                               o["dws_up"], bws)
+        torch.cuda.synchronize()
+        assert B.get_device_status(bws) == B.OK
+        res[tag] = o
+    for k in res["single"]:
+        assert torch.equal(res["single"][k].view(torch.int16), res["pair"][k].view(torch.int16)), k
+        assert torch.equal(res["single"][k], g[k]), k
+    # the layer's backward (weight gradients on pairs by default) against the oracle
+    assert layer.dims(T).flags & B.FLAG_WGRAD_CTA_PAIR
+    ref = oracle_backward(inp, out, dy_bits, ALPHA, BETA)
+    check_all(inp, out, g, ref, out["counts"].cpu().numpy())
+
+
 def test_backward_is_deterministic():
     cfg = CASES["split"]
     inp, layer, x, out, dy, dy_bits, g = run(cfg)

@@ -154,9 +154,11 @@ def _check(fn: str, code: int):
 
 
 # moe_dims_t.flags: router product on the fp32 CUDA cores instead of the tensor cores;
-# expert GEMMs on CTA pairs instead of single-CTA tiles
+# expert GEMMs on CTA pairs instead of single-CTA tiles; the backward's weight gradients on
+# CTA pairs
 FLAG_ROUTER_FP32_CORES = 1
 FLAG_FFN_CTA_PAIR = 2
+FLAG_WGRAD_CTA_PAIR = 4
 
 
 def dims(T, d, N, M, K, F, F_shared, flags=0, C=0, V=0) -> Dims:

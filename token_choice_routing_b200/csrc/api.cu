@@ -24,7 +24,8 @@ int sm_count() {
 
 int check_dims(const moe_dims_t* d) {
   if (d == nullptr) return MOE_ERR_INVALID_ARG;
-  if ((d->flags & ~(MOE_FLAG_ROUTER_FP32_CORES | MOE_FLAG_FFN_CTA_PAIR)) != 0u) return MOE_ERR_INVALID_ARG;
+  if ((d->flags & ~(MOE_FLAG_ROUTER_FP32_CORES | MOE_FLAG_FFN_CTA_PAIR | MOE_FLAG_WGRAD_CTA_PAIR)) != 0u)
+    return MOE_ERR_INVALID_ARG;
   if (d->T < 0 || d->d <= 0 || d->N < 1 || d->M < 0 || d->K < 1 || d->F <= 0 || d->F_shared <= 0)
     return MOE_ERR_INVALID_ARG;
   if (d->C < 0 || d->V < 0) return MOE_ERR_INVALID_ARG;

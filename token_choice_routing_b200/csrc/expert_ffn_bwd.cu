@@ -649,6 +649,480 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const float* __restri
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Weight gradients on CTA pairs. C[m, n] = sum_r A[r, m] B[r, n] over one expert's rows (or
+// one K chunk of the shared expert's T rows), as kWgrad above, with a pair tile of 256
+// output rows x 256 columns: one tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16, both
+// operands MN-major) per 16 rows. Each CTA loads its own 128 output rows of A and its half
+// (128) of the 256 columns of B per 64-row k-block: 32 KB, against 48 KB for the same work
+// on one CTA (a 128 x 256 tile), so a third less operand data crosses into shared memory per
+// flop. Each CTA's TMEM holds its 128 output rows x 256 columns, drained by the kWgrad
+// epilogue as the 128-row tile 2 p + rank of pair tile p.
+// A full k-block's copies (both CTAs') complete on the leader's full barrier, as in the
+// forward's pair kernel. The rows of an expert's last k-block past its end (another
+// expert's rows, or rows never written) are zeroed before the MMA reads them, in both CTAs:
+// that k-block's copies complete on a barrier of the CTA's own, and a ready warp in each CTA
+// waits for it and zeroes those rows: the leader's then gives the full barrier its one
+// arrival, the other CTA's arrives on the leader's zeroed barrier, and the MMA thread waits
+// for both. (Remote arrivals on every k-block, from the producer or a ready warp, measured
+// 1.5-2 times slower.)
+// Roles (224 threads per CTA): warp 0 lane 0 TMA producer; warp 1 TMEM allocation and, in
+// the leader, the single MMA thread; warps 2-5 epilogue; warp 6 ready warp. Every wait is
+// bounded.
+// Bounded wait with cluster-scope acquire, for a barrier that the other CTA of the pair
+// arrives on after writing shared memory the waiter's MMAs read. Returns false (and records
+// a timeout in *status) if limit_ns passed or *abort became non-zero meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
+                                                          volatile int* abort, uint32_t* status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((++spins & 63u) == 0u) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (status) atomicOr(status, kStatusTimeout);
+        if (abort) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+constexpr int kPStages = 6;
+constexpr int kPThreads = 224;
+constexpr int kPBN = 256;
+
+struct PairWSmem {
+  static constexpr int A_BYTES = kBM * kBK * 2;             // 16 KB: this CTA's 128 output rows
+  static constexpr int B_BYTES = (kPBN / 2) * kBK * 2;      // 16 KB: this CTA's 128 columns
+  static constexpr size_t off_a = 0;
+  static constexpr size_t off_b = off_a + (size_t)kPStages * A_BYTES;
+  static constexpr size_t off_stg = off_b + (size_t)kPStages * B_BYTES;
+  static constexpr size_t off_bar = off_stg + (size_t)kBM * kStgRow;
+  static constexpr int n_bar = 4 * kPStages + 5;  // lfull, full, empty, zdone, tfull[2], tempty[2], drain
+  static constexpr size_t off_misc = off_bar + 8 * n_bar;
+  static constexpr size_t off_tab = off_misc + 16;
+  static constexpr size_t end = off_tab + sizeof(int) * 3 * (kMaxN + 2);
+  static constexpr size_t bytes = end + 1024;
+  static_assert(bytes <= 232448, "shared memory per CTA");
+};
+
+// a.mt_r / a.mt_s count pair tiles here (output rows / 256).
+__global__ void __launch_bounds__(kPThreads, 1)
+wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
+                  const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmB_s, const Args a) {
+  pdl_wait_then_release();
+  using SM = PairWSmem;
+  constexpr int BN = kPBN;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr uint32_t IDESC = idesc_t(2 * kBM, BN, true, true);
+  constexpr uint32_t TX_BYTES = SM::A_BYTES + SM::B_BYTES;  // this CTA's copies of one stage
+
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base + SM::off_a;
+  unsigned char* sB = base + SM::off_b;
+  unsigned char* stg = base + SM::off_stg;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + SM::off_bar);
+  volatile int* misc = reinterpret_cast<volatile int*>(base + SM::off_misc);  // [0] tmem, [1] abort
+  int* s_tstart = reinterpret_cast<int*>(base + SM::off_tab);
+  int* s_row0 = s_tstart + (kMaxN + 2);
+  int* s_m = s_row0 + (kMaxN + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  auto lfull_bar = [&](int s) { return smem_u32(bars + s); };
+  auto full_bar = [&](int s) { return smem_u32(bars + kPStages + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + 2 * kPStages + s); };
+  auto zdone_bar = [&](int s) { return smem_u32(bars + 3 * kPStages + s); };
+  auto tfull_bar = [&](int s) { return smem_u32(bars + 4 * kPStages + s); };
+  auto tempty_bar = [&](int s) { return smem_u32(bars + 4 * kPStages + 2 + s); };
+  const uint32_t drain_bar = smem_u32(bars + 4 * kPStages + 4);
+  volatile int* abort_flag = misc + 1;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA_r);
+    prefetch_tmap(&tmB_r);
+    if (a.has_shared) {
+      prefetch_tmap(&tmA_s);
+      prefetch_tmap(&tmB_s);
+    }
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(lfull_bar(s), 1);  // a last k-block: this CTA's expect_tx arrival and its bytes
+      mbar_init(full_bar(s), 1);   // leader: its expect_tx arrival (with both CTAs' bytes), or,
+                                   // for a last k-block, its ready warp's arrival
+      mbar_init(empty_bar(s), 1);  // one commit from the leader's MMA thread
+      mbar_init(zdone_bar(s), 1);  // leader: the other CTA's tail rows are zeroed
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(tfull_bar(s), 1);
+      mbar_init(tempty_bar(s), 2 * 128);  // leader: every epilogue thread of both CTAs
+    }
+    mbar_init(drain_bar, 1);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(const_cast<int*>(misc)), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 2 && lane == 0) {
+    // Per-group tile table from the device-resident offsets (both CTAs build the same one);
+    // the shared expert's K chunks come first: they are the longest tiles.
+    int acc = 0, prev = 0;
+    bool bad = false;
+    if (a.has_shared) {
+      s_tstart[N] = 0;
+      acc = a.nsplit * a.mt_s * a.nt_s;
+    }
+    for (int g = 0; g <= N; ++g) {
+      int m, row0;
+      if (g < N) {
+        const int o0 = a.offsets[g], o1 = a.offsets[g + 1];
+        if (o0 != prev || o1 < o0 || (long long)o1 > a.rows_cap) bad = true;
+        prev = o1;
+        m = bad ? 0 : o1 - o0;
+        row0 = o0;
+        s_tstart[g] = acc;
+        acc += a.mt_r * a.nt_r;
+      } else {
+        m = a.has_shared ? a.T : 0;
+        row0 = 0;
+      }
+      s_row0[g] = row0;
+      s_m[g] = m;
+    }
+    s_tstart[N + 1] = acc;
+    if (bad && leader) atomicOr(a.status, kStatusBounds);
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated, tables built
+  tc_fence_after();
+  const uint32_t tmem_base = (uint32_t)misc[0];
+  const int total = s_tstart[N + 1];
+  const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
+
+  // t.mt: pair tile (256 output rows); this CTA's 128-row tile is 2 t.mt + rank
+  auto decode = [&](int tile) {
+    Tile ti;
+    const int nsh = a.has_shared ? a.nsplit * a.mt_s * a.nt_s : 0;
+    if (tile < nsh) {
+      const int per = a.mt_s * a.nt_s;
+      ti.g = N;
+      ti.chunk = tile / per;
+      const int local = tile - ti.chunk * per;
+      ti.mt = local / a.nt_s;
+      ti.nt = local - ti.mt * a.nt_s;
+      ti.row0 = ti.chunk * a.chunk_kb * kBK;
+      ti.krows = max(0, min(a.chunk_kb * kBK, s_m[N] - ti.row0));
+    } else {
+      const int per = a.mt_r * a.nt_r;
+      const int e = (tile - nsh) / per;
+      const int local = tile - nsh - e * per;
+      ti.g = e;
+      ti.chunk = 0;
+      ti.mt = local / a.nt_r;
+      ti.nt = local - ti.mt * a.nt_r;
+      ti.row0 = s_row0[e];
+      ti.krows = s_m[e];
+    }
+    ti.nkb = (ti.krows + kBK - 1) / kBK;
+    ti.mvalid = kBM;
+    ti.brow = 0;
+    return ti;
+  };
+  auto tile_at = [&](int r) { return r * npairs + pair; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------ TMA producer (both CTAs): this CTA's A rows and B half
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;     // stages whose copies count on the leader's barrier
+      uint32_t larmed = 0, lpar = 0;         // stages whose copies count on this CTA's barrier
+      for (int r = 0;; ++r) {
+        const int tile = tile_at(r);
+        if (tile >= total) break;
+        const Tile ti = decode(tile);
+        const void* ta = (ti.g < N) ? (const void*)&tmA_r : (const void*)&tmA_s;
+        const void* tb = (ti.g < N) ? (const void*)&tmB_r : (const void*)&tmB_s;
+        const int ax = (2 * ti.mt + (int)rank) * kBM;
+        const int bx = ti.nt * BN + (int)rank * (BN / 2);
+        bool ok = true;
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, a.limit_ns, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dA = smem_u32(sA + stage * SM::A_BYTES);
+          const uint32_t dB = smem_u32(sB + stage * SM::B_BYTES);
+          const int kr = ti.row0 + kb * kBK;
+          if (ti.krows - kb * kBK >= kBK) {
+            const uint32_t fb = map_to_rank(full_bar(stage), 0);
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * TX_BYTES);
+            tma_load_2d_pair(dA, ta, fb, ax, kr);
+            tma_load_2d_pair(dA + kBox, ta, fb, ax + 64, kr);
+            tma_load_2d_pair(dB, tb, fb, bx, kr);
+            tma_load_2d_pair(dB + kBox, tb, fb, bx + 64, kr);
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          } else {
+            // the expert's last k-block: the ready warp zeroes its tail rows first
+            mbar_arrive_expect_tx(lfull_bar(stage), TX_BYTES);
+            tma_load_2d(dA, ta, lfull_bar(stage), ax, kr);
+            tma_load_2d(dA + kBox, ta, lfull_bar(stage), ax + 64, kr);
+            tma_load_2d(dB, tb, lfull_bar(stage), bx, kr);
+            tma_load_2d(dB + kBox, tb, lfull_bar(stage), bx + 64, kr);
+            larmed |= 1u << stage;
+            lpar ^= 1u << stage;  // parity of the phase this use completes, plus one
+          }
+          if (++stage == kPStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // copies still in flight land before the CTA leaves: a full k-block's on the leader's
+        // barrier (both CTAs' bytes), a last one's on this CTA's
+        for (int s = 0; s < kPStages; ++s) {
+          if (leader && (armed & (1u << s)))
+            (void)mbar_wait_bounded(full_bar(s), (armed_par >> s) & 1u, a.limit_ns, nullptr, a.status);
+          if (larmed & (1u << s))
+            (void)mbar_wait_bounded(lfull_bar(s), ((lpar >> s) & 1u) ^ 1u, a.limit_ns, nullptr, a.status);
+        }
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------ ready warp (both CTAs): an expert's last k-block has its
+    // tail rows zeroed in both CTAs before the leader's full barrier counts it
+    int stage = 0;
+    uint32_t lpar = 0;  // per stage: parity of the next phase of this CTA's barrier
+    for (int r = 0;; ++r) {
+      const int tile = tile_at(r);
+      if (tile >= total) break;
+      const Tile ti = decode(tile);
+      bool ok = true;
+      for (int kb = 0; kb < ti.nkb; ++kb) {
+        const int rem = ti.krows - kb * kBK;
+        if (rem >= kBK) {
+          if (++stage == kPStages) stage = 0;
+          continue;
+        }
+        int f = 1;
+        if (lane == 0)
+          f = mbar_wait_bounded(lfull_bar(stage), (lpar >> stage) & 1u, a.limit_ns, abort_flag, a.status);
+        if (!__shfl_sync(0xffffffffu, f, 0)) {
+          ok = false;
+          break;
+        }
+        {
+          // rows [rem, 16 * ceil(rem / 16)) of every box belong to another expert (or were
+          // never written): zeroed in both operands; later 16-row steps are skipped
+          const int z0 = rem, z1 = ((rem + 15) >> 4) * 16;
+          const int nrows = z1 - z0;
+          for (int i = lane; i < 4 * nrows * 8; i += 32) {
+            const int box = i / (nrows * 8);
+            const int rr = (i / 8) % nrows + z0;
+            const int ch = i & 7;
+            unsigned char* p = (box < 2) ? sA + stage * SM::A_BYTES + box * kBox
+                                         : sB + stage * SM::B_BYTES + (box - 2) * kBox;
+            *reinterpret_cast<uint4*>(p + rr * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_shared();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          if (leader) mbar_arrive(full_bar(stage));
+          else mbar_arrive_cluster(map_to_rank(zdone_bar(stage), 0));
+        }
+        lpar ^= 1u << stage;
+        if (++stage == kPStages) stage = 0;
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------ MMA issuer (leader CTA, one thread)
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t zpar = 0;  // per stage: parity of the next phase of the zeroed barrier
+      for (int li = 0;; ++li) {
+        const int tile = tile_at(li);
+        if (tile >= total) break;
+        const Tile ti = decode(tile);
+        const int acc = li & 1;
+        const uint32_t ap = (uint32_t)(li >> 1) & 1u;
+        if (!mbar_wait_bounded_cluster(tempty_bar(acc), ap ^ 1u, a.limit_ns, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, a.limit_ns, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          const int rem = ti.krows - kb * kBK;
+          if (rem < kBK) {
+            // an expert's last k-block: the other CTA's tail rows are zeroed too
+            if (!mbar_wait_bounded_cluster(zdone_bar(stage), (zpar >> stage) & 1u, a.limit_ns, abort_flag,
+                                           a.status)) {
+              ok = false;
+              break;
+            }
+            zpar ^= 1u << stage;
+          }
+          tc_fence_after();
+          const int nk16 = (rem < kBK) ? (rem + 15) >> 4 : kBK / 16;
+          const uint32_t aS = smem_u32(sA + stage * SM::A_BYTES);
+          const uint32_t bS = smem_u32(sB + stage * SM::B_BYTES);
+          for (int k = 0; k < nk16; ++k)
+            tc_mma_pair(d_tmem, desc_mn_sw128(aS + (uint32_t)(k * 2048), kBox),
+                        desc_mn_sw128(bS + (uint32_t)(k * 2048), kBox), IDESC, (kb | k) != 0 ? 1u : 0u);
+          // free this stage in both CTAs
+          tc_commit_pair(empty_bar(stage));
+          tc_commit_pair(map_to_rank(empty_bar(stage), 1));
+          if (++stage == kPStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(tfull_bar(acc));
+        tc_commit_pair(map_to_rank(tfull_bar(acc), 1));
+      }
+      // all MMAs issued by this thread have completed once the drain barrier fires
+      tc_commit_pair(drain_bar);
+      (void)mbar_wait_bounded(drain_bar, 0, a.limit_ns, nullptr, a.status);
+    }
+  } else {
+    // ------------------------------ epilogue warpgroup (warps 2..5 of each CTA)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int etid = (warp - 2) * 32 + lane;
+    const uint32_t tempty_leader = map_to_rank(tempty_bar(0), 0);
+    for (int li = 0;; ++li) {
+      const int tile = tile_at(li);
+      if (tile >= total) break;
+      const Tile ti = decode(tile);
+      const int acc = li & 1;
+      const uint32_t ap = (uint32_t)(li >> 1) & 1u;
+      if (!mbar_wait_bounded(tfull_bar(acc), ap, a.limit_ns, abort_flag, a.status)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int mt = 2 * ti.mt + (int)rank;  // this CTA's 128-row output tile
+      const bool sh = ti.g == N;
+      const bool partial = sh && (a.nsplit > 1 || a.part_only);
+      const bool empty = ti.nkb == 0;
+      const int ld = sh ? a.ld_s : a.ld_r;
+      if (partial) {
+        // fp32 partial of one K chunk, straight from registers
+        const size_t mrows_s = (size_t)a.mt_s * 2 * kBM;
+        float* P = a.part_s + ((size_t)ti.chunk * mrows_s + (size_t)mt * kBM + row) * a.ld_s + ti.nt * BN;
+#pragma unroll 1
+        for (int g16 = 0; g16 < BN / 16; ++g16) {
+          uint32_t r[16];
+          if (!empty) {
+            tmem_ld16(tb + (uint32_t)(g16 * 16), r);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[j] = 0u;
+          }
+          float4* dst = reinterpret_cast<float4*>(P + g16 * 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+      } else {
+        uint16_t* o1 = sh ? a.out_s : a.out_r;
+        uint16_t* o2 = sh ? a.out_s2 : a.out_r2;
+        const int e = sh ? 0 : ti.g;
+        const int mrows = (sh ? a.mt_s : a.mt_r) * 2 * kBM;  // packed output rows per group
+        uint16_t *out, *out_hi;
+        size_t rowoff_lo, rowoff_hi;
+        if (o2) {  // packed gate/up: tile rows 0..63 are gate rows, 64..127 the up rows
+          const size_t half = (size_t)(mrows / 2) * ld;
+          out = o1 + e * half;
+          out_hi = o2 + e * half;
+          rowoff_lo = (size_t)(mt * 64) * ld;
+          rowoff_hi = rowoff_lo;
+        } else {
+          out = o1 + (size_t)e * mrows * ld;
+          out_hi = out;
+          rowoff_lo = (size_t)(mt * kBM) * ld;
+          rowoff_hi = rowoff_lo + (size_t)64 * ld;
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN / 64; ++c) {
+#pragma unroll
+          for (int g16 = 0; g16 < 4; ++g16) {
+            uint32_t r[16];
+            if (!empty) {
+              tmem_ld16(tb + (uint32_t)(c * 64 + g16 * 16), r);
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) r[j] = 0u;
+            }
+            uint32_t packed[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              packed[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(stg + row * kStgRow + g16 * 32);
+            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          }
+          if (c == BN / 64 - 1) {
+            // this CTA's half of the accumulator is drained: let the leader reuse it
+            tc_fence_before();
+            mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+          }
+          named_bar_sync(1, 128);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int idx = it * 128 + etid;
+            const int rr = idx >> 3, ch = idx & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * kStgRow + ch * 16);
+            const int col = ti.nt * BN + c * 64 + ch * 8;
+            uint16_t* dst = (rr < 64) ? out + rowoff_lo + (size_t)rr * ld : out_hi + rowoff_hi + (size_t)(rr - 64) * ld;
+            *reinterpret_cast<uint4*>(dst + col) = v;
+          }
+          named_bar_sync(1, 128);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // the leader's MMAs read both CTAs' shared memory: nobody leaves early
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 template <int BN, int MODE>
 static int launch(const CUtensorMap& ar, const CUtensorMap& br, const CUtensorMap& as_, const CUtensorMap& bs,
                   const CUtensorMap& zr, const CUtensorMap& zs, const Args& a, long long max_tiles, cudaStream_t st) {
@@ -811,17 +1285,63 @@ int launch_dgrad_gate_up(const moe_dims_t& d, const int32_t* offsets, const uint
                    : launch<128, kDgradPlain>(ar, br, as_, bs, xr, xw, a, mt, st);
 }
 
+// One wave of CTA pairs (clusters of two), at most one per pair tile.
+static int launch_wgrad_pair(const CUtensorMap& ar, const CUtensorMap& br, const CUtensorMap& as_,
+                             const CUtensorMap& bs, const Args& a, long long max_tiles, cudaStream_t st) {
+  static int clusters[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kern = wgrad_pair_kernel;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.dynamicSmemBytes = PairWSmem::bytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
+  if (dev >= 0 && dev < 64 && clusters[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PairWSmem::bytes);
+    if (e != cudaSuccess) return cuda_status(e);
+    int n = 0;
+    cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess || n < 1) n = sm_count() / 2;
+    clusters[dev] = n;
+  }
+  long long np = (dev >= 0 && dev < 64) ? clusters[dev] : sm_count() / 2;
+  if (max_tiles < np) np = max_tiles;
+  if (np < 1) np = 1;
+  cfg.gridDim = dim3((unsigned)(2 * np), 1, 1);
+  cfg.numAttrs = 2;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, ar, br, as_, bs, a));
+}
+
+// With MOE_FLAG_WGRAD_CTA_PAIR, 256-column tiles and an even number of 128-row output tiles
+// per group, the weight gradients run on CTA pairs (wgrad_pair_kernel); else on one CTA.
 static int launch_wgrad(const moe_dims_t& d, const Args& a0, int BN, const CUtensorMap& ar, const CUtensorMap& br,
                         const CUtensorMap& as_, const CUtensorMap& bs, int mrows_s, uint16_t* out_s,
                         uint16_t* out_s2, cudaStream_t st) {
   Args a = a0;
   if (a.nsplit > 1 && !a.part_s) return MOE_ERR_INVALID_ARG;
-  const long long tiles = (long long)a.nsplit * a.mt_s * a.nt_s + (long long)d.N * a.mt_r * a.nt_r;
   int r;
-  switch (BN) {
-    case 256: r = launch<256, kWgrad>(ar, br, as_, bs, ar, ar, a, tiles, st); break;
-    case 128: r = launch<128, kWgrad>(ar, br, as_, bs, ar, ar, a, tiles, st); break;
-    default: r = launch<64, kWgrad>(ar, br, as_, bs, ar, ar, a, tiles, st); break;
+  if ((d.flags & MOE_FLAG_WGRAD_CTA_PAIR) && BN == kPBN && a.mt_r % 2 == 0 && a.mt_s % 2 == 0) {
+    a.mt_r /= 2;
+    a.mt_s /= 2;
+    const long long tiles = (long long)a.nsplit * a.mt_s * a.nt_s + (long long)d.N * a.mt_r * a.nt_r;
+    r = launch_wgrad_pair(ar, br, as_, bs, a, tiles, st);
+  } else {
+    const long long tiles = (long long)a.nsplit * a.mt_s * a.nt_s + (long long)d.N * a.mt_r * a.nt_r;
+    switch (BN) {
+      case 256: r = launch<256, kWgrad>(ar, br, as_, bs, ar, ar, a, tiles, st); break;
+      case 128: r = launch<128, kWgrad>(ar, br, as_, bs, ar, ar, a, tiles, st); break;
+      default: r = launch<64, kWgrad>(ar, br, as_, bs, ar, ar, a, tiles, st); break;
+    }
   }
   if (r != MOE_OK || a.nsplit <= 1) return r;
   const long long n8 = (long long)mrows_s * a.ld_s / 8;

@@ -57,26 +57,31 @@ class MoENullLayer:
                  w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
                  ws_gate: torch.Tensor, ws_up: torch.Tensor, ws_down: torch.Tensor,
                  router: str = "tensor", ffn: str = "auto", C: int = 0, V: int = 0,
-                 const_vectors: Optional[torch.Tensor] = None):
+                 const_vectors: Optional[torch.Tensor] = None, wgrad: str = "pair"):
         """router: "tensor" (router product on the tensor cores, fp32 weights split
         exactly into three bf16 terms) or "fp32_cores" (fp32 FMA on the CUDA cores).
         ffn: "single" (single-CTA tiles), "pair" (expert GEMMs on CTA pairs where the
         shape allows) or "auto" (pairs for calls of at least PAIR_MIN_TOKENS tokens,
-        where they measured faster; single-CTA tiles below). C, V: MoE++ copy and
-        constant experts (router rows N+1 .. N+C+V after the null logit;
-        const_vectors [V, d] bf16)."""
+        where they measured faster; single-CTA tiles below). wgrad: the backward's weight
+        gradients on CTA pairs where the shape allows ("pair", the default: faster on every
+        measured workload) or on single CTAs ("single"); the results are the same bit for
+        bit. C, V: MoE++ copy and constant experts (router rows N+1 .. N+C+V after the null
+        logit; const_vectors [V, d] bf16)."""
         if router not in ("tensor", "fp32_cores"):
             raise ValueError(f"router must be 'tensor' or 'fp32_cores', not {router!r}")
         if ffn not in ("pair", "single", "auto"):
             raise ValueError(f"ffn must be 'pair', 'single' or 'auto', not {ffn!r}")
+        if wgrad not in ("pair", "single"):
+            raise ValueError(f"wgrad must be 'pair' or 'single', not {wgrad!r}")
         self.d, self.N, self.M, self.K, self.F, self.F_shared = d, N, M, K, F, F_shared
         self.C, self.V = C, V
-        self.router, self.ffn = router, ffn
+        self.router, self.ffn, self.wgrad = router, ffn, wgrad
         if V > 0 and (const_vectors is None or tuple(const_vectors.shape) != (V, d)):
             raise ValueError("const_vectors [V, d] bf16 is required when V > 0")
         self.const_vectors = None if V == 0 else const_vectors.contiguous()
         self.flags = ((B.FLAG_ROUTER_FP32_CORES if router == "fp32_cores" else 0) |
-                      (B.FLAG_FFN_CTA_PAIR if ffn == "pair" else 0))
+                      (B.FLAG_FFN_CTA_PAIR if ffn == "pair" else 0) |
+                      (B.FLAG_WGRAD_CTA_PAIR if wgrad == "pair" else 0))
         dev = w_router.device
         self.device = dev
         self.w_router = w_router.contiguous()
@@ -104,7 +109,8 @@ class MoENullLayer:
                                   None if self.router_split is None else self.router_split.data_ptr())
 
     @classmethod
-    def from_inputs(cls, inp, device="cuda", router: str = "tensor", ffn: str = "auto") -> "MoENullLayer":
+    def from_inputs(cls, inp, device="cuda", router: str = "tensor", ffn: str = "auto",
+                    wgrad: str = "pair") -> "MoENullLayer":
         c = inp.cfg
         f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         cv = None if c.V == 0 else bf16_tensor(inp.const_vectors, device)
@@ -113,7 +119,7 @@ class MoENullLayer:
                    w_gate=bf16_tensor(inp.w_gate, device), w_up=bf16_tensor(inp.w_up, device),
                    w_down=bf16_tensor(inp.w_down, device), ws_gate=bf16_tensor(inp.ws_gate, device),
                    ws_up=bf16_tensor(inp.ws_up, device), ws_down=bf16_tensor(inp.ws_down, device),
-                   router=router, ffn=ffn, C=c.C, V=c.V, const_vectors=cv)
+                   router=router, ffn=ffn, C=c.C, V=c.V, const_vectors=cv, wgrad=wgrad)
 
     # With ffn="auto", calls of at least this many tokens run the expert GEMMs on CTA pairs:
     # on the 131072-token skewed workload they measured ~4.5% faster per forward, on 16384-token
