@@ -360,8 +360,8 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         ("input_grad", lambda: B.input_grad(dm, dxsh, dxs, o["slot_row"], o["topk_idx"], o["topk_gate"], dy,
                                             grads["dx"], bws)),
     ]
-    acc = {n: 0.0 for n, _ in stages}
-    nb = max(3, min(args.steps, 10))
+    acc = {n: [] for n, _ in stages}
+    nb = max(5, min(args.steps, 11))
     for _ in range(nb):
         flush.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
@@ -371,11 +371,11 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
             ev[i + 1].record()
         torch.cuda.synchronize()
         for i, (n, _) in enumerate(stages):
-            acc[n] += ev[i].elapsed_time(ev[i + 1])
+            acc[n].append(ev[i].elapsed_time(ev[i + 1]))
     st = B.get_device_status(bws)
     if st != B.OK:
         raise SystemExit(f"backward device status: {B.status_string(st)}")
-    kms = {n: acc[n] / nb for n in acc}
+    kms = {n: statistics.median(acc[n]) for n in acc}  # median over the passes
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     # the router's input gradient ds W_r rides in dgrad_gate_up (extra k-blocks of the shared tiles)
@@ -475,15 +475,16 @@ def timed_events(fn, steps, warmup, flush, sync_before=None):
 
 
 def forward_stage_ms(layer, dm, x, tnb, out, flush, nb):
-    """Mean device ms of the forward's stages, each launched through its own entry point in
-    the forward's order with CUDA events between them (L2 flushed before each pass). With no
+    """Median device ms of the forward's stages over nb passes, each stage launched through its
+    own entry point in the forward's order with CUDA events between them (L2 flushed before
+    each pass; the median, so that a pass disturbed by a clock dip does not set it). With no
     shared_out buffer the combine runs inside the down GEMM ("down_combine"), as in the
     forward; otherwise "down" and "combine" are separate launches."""
     import torch
     from token_choice_routing_b200 import binding as B
     fused = out.get("shared_out") is None
     names = ["route", "dispatch", "gate_up"] + (["down_combine"] if fused else ["down", "combine"])
-    acc = {n: 0.0 for n in names}
+    acc = {n: [] for n in names}
     for _ in range(nb):
         flush.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
@@ -521,8 +522,8 @@ def forward_stage_ms(layer, dm, x, tnb, out, flush, nb):
             ev[5].record()
         torch.cuda.synchronize()
         for i, n in enumerate(names):
-            acc[n] += ev[i].elapsed_time(ev[i + 1])
-    return {n: acc[n] / nb for n in names}
+            acc[n].append(ev[i].elapsed_time(ev[i + 1]))
+    return {n: statistics.median(acc[n]) for n in names}
 
 
 def forward_figures(cfg, R, kms, peaks, args, out):
@@ -596,7 +597,7 @@ def measure_per_config(args, names, dev, flush, peaks):
         out = layer.alloc(cfg.T, logits=False, xs=not args.gather, combine=args.combine)
         ms = timed_events(lambda: layer.forward(x, tnb, out), steps, warmup, flush)
         R = int(out["offsets"][-1].item())
-        kms = forward_stage_ms(layer, layer.dims(cfg.T), x, tnb, out, flush, 3)
+        kms = forward_stage_ms(layer, layer.dims(cfg.T), x, tnb, out, flush, 5)
         b, ffn_tflops, _ = forward_figures(cfg, R, kms, peaks, args, out)
         med = statistics.median(ms)
         res[name] = {"T": cfg.T, "K": cfg.K, "M": cfg.M, "rho": cfg.rho, "real_slots_per_step": R,
@@ -710,7 +711,7 @@ def main():
         raise SystemExit(f"device status after timing: {B.status_string(st)}")
 
     # ---- per-kernel breakdown (separately timed passes, same launches, CUDA events between them)
-    kms = forward_stage_ms(layer, dm, x, tnb, out, flush, max(3, min(args.steps, 10)))
+    kms = forward_stage_ms(layer, dm, x, tnb, out, flush, max(5, min(args.steps, 11)))
     peaks, peak_kind = load_peaks()
     breakdown, ffn_tflops, flops_gu = forward_figures(cfg, R, kms, peaks, args, out)
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
