@@ -67,6 +67,7 @@ GEMM_PROFILE = "profiles/grouped_gemm_qwen3_0p6b.md"
 GEMM_PROFILES = (GEMM_PROFILE, "profiles/grouped_gemm_skew.md")
 BWD_GEMM_SOURCES = ("token_choice_routing_b200/csrc/expert_ffn_bwd.cu", "token_choice_routing_b200/csrc/moe_internal.cuh")
 BWD_GEMM_PROFILE = "profiles/bwd_gemm_kernel_qwen3_0p6b.md"
+BWD_GEMM_PROFILES = (BWD_GEMM_PROFILE, "profiles/wgrad_pair_kernel_qwen3_0p6b.md", "profiles/wgrad_pair_kernel_skew.md")
 
 
 def gemm_source_digest(sources=GEMM_SOURCES) -> str:
@@ -400,6 +401,10 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         kernels[n] = k
     gemm = ["dgrad_down", "wgrad_down", "dgrad_gate_up", "wgrad_gate_up"]
     top = max(gemm, key=lambda n: kms[n])
+    # the weight gradients ran on CTA pairs (the layer's default) where the shape allows
+    pair_ok = {"wgrad_down": d % 256 == 0 and F % 256 == 0 and Fs % 256 == 0,
+               "wgrad_gate_up": d % 256 == 0 and (2 * F) % 256 == 0 and (2 * Fs) % 256 == 0}
+    top_pair = layer.wgrad == "pair" and pair_ok.get(top, False)
     gemm_ms = sum(kms[n] for n in gemm)
     gemm_flops = sum(fl[n] for n in gemm)
     # combine_bwd, router_bwd, router wgrad (+ its reduce), W_r split, dgrad down, SwiGLU backward,
@@ -412,12 +417,12 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
         "preactivations": "saved by the forward (training mode); the SwiGLU derivative is an elementwise pass",
         "forward_training_ms": fwd_train_ms, "backward_recompute_ms": recompute_ms,
         "ffn_tflops_real_rows": gemm_flops / (gemm_ms * 1e9),
-        "roofline": {"kernel": f"{top} grouped GEMM (tcgen05"
-                               + (", CTA pairs)" if top.startswith("wgrad") and layer.wgrad == "pair" else ")"),
+        "roofline": {"kernel": f"{top} grouped GEMM (tcgen05" + (", CTA pairs)" if top_pair else ")"),
                      "bound": "tensor",
                      "achieved": fl[top] / (kms[top] * 1e9), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": fl[top] / (kms[top] * 1e9) / bf16_peak, "peak_kind": f"{peak_kind} bf16 burst",
-                     "traffic": recorded_traffic(cfg.name, top, BWD_GEMM_PROFILE, BWD_GEMM_SOURCES),
+                     "traffic": recorded_traffic(cfg.name, top + ("_pair" if top_pair else ""), BWD_GEMM_PROFILES,
+                                                 BWD_GEMM_SOURCES),
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "flops_per_launch": fl[top], "ms_per_launch": kms[top]},
         "kernels": kernels,
