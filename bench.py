@@ -564,7 +564,10 @@ def forward_figures(cfg, R, kms, peaks, args, out):
         "dispatch": {"ms": kms["dispatch"], "bound": "hbm", "GB/s": bytes_dispatch / (kms["dispatch"] * 1e6)},
         "gate_up": {"ms": kms["gate_up"], "bound": "tensor", "TFLOP/s": flops_gu / (kms["gate_up"] * 1e9)},
     }
-    b["route"]["frac_fp32_alu"] = b["route"]["TFLOP/s"] / fp32_peak
+    if args.router == "fp32_cores":  # the CUDA-core product: its bound is the fp32 FMA rate
+        b["route"]["frac_fp32_alu"] = b["route"]["TFLOP/s"] / fp32_peak
+    else:  # on the tensor cores the route is bound by reading x from HBM
+        b["route"]["frac"] = b["route"]["GB/s"] / hbm_peak
     b["route"]["frac_hbm"] = b["route"]["GB/s"] / hbm_peak
     b["dispatch"]["frac"] = b["dispatch"]["GB/s"] / hbm_peak
     b["gate_up"]["frac"] = b["gate_up"]["TFLOP/s"] / bf16_peak
