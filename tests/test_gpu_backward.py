@@ -205,6 +205,8 @@ PAIR_CASES = {
     # experts without rows, ragged tails of every length
     "skew": I.small_config("wgp_skew", T=1500, d=512, N=64, F=256, F_shared=256, K=8, M=64, config_id=943,
                            skew=True, seqs=2),
+    # F = 384: gate/up on pairs (2F = 768 output rows), down on single CTAs (384 columns)
+    "mixed": I.small_config("wgp_mixed", T=900, d=256, N=8, F=384, F_shared=384, K=2, M=2, config_id=944),
 }
 
 
