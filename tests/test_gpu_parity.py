@@ -109,6 +109,30 @@ def test_large_configs_routing_and_sampled_output(name, ffn):
     H.check_layer_output(inp, out, r, tokens=tokens)
 
 
+def test_route_on_cta_pairs_with_an_odd_tile_count():
+    """Above 148 route tiles the route runs on CTA pairs; with an odd tile count the last
+    pair's second CTA has no tokens (loaded as zeros, never written). T = 19250: 151 tiles,
+    the last one holding 50 tokens. Routing, dispatch and statistics against the oracle, and
+    the prepared-weight route bit-identical to the one that splits the weight per call."""
+    from token_choice_routing_b200 import binding as B
+    cfg = I.small_config("odd_pairs", T=19250, d=256, N=16, F=128, F_shared=128, K=4, M=8, config_id=914)
+    assert (cfg.T + 127) // 128 == 151
+    inp = I.make_inputs(cfg)
+    inp.bias[cfg.N] = np.float32(0.3)
+    layer, x, tnb, out = H.run_forward(inp)
+    r = H.check_routing(inp, out)
+    H.check_dispatch(inp, out, r)
+    H.check_aux(inp, out, r)
+    dm = layer.dims(cfg.T)
+    o = [torch.empty_like(out[k]) for k in ("topk_idx", "topk_gate", "n_real")]
+    ws = torch.empty(B.workspace_bytes(dm), dtype=torch.uint8, device="cuda")
+    B.route(dm, x, layer.w_router, layer.router_bias, tnb, None, o[0], o[1], o[2], ws)
+    torch.cuda.synchronize()
+    assert B.get_device_status(ws) == B.OK
+    for a, k in zip(o, ("topk_idx", "topk_gate", "n_real")):
+        assert torch.equal(a, out[k]), k
+
+
 @pytest.mark.parametrize("name", ["qwen3_0p6b", "ragged_b", "skew_small", "t1"])
 def test_row_gather_matches_row_copy_bitwise(name):
     """Gate/up reading the routed rows of x through TMA row gathers feeds the
