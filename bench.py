@@ -523,8 +523,13 @@ def forward_stage_ms(layer, dm, x, tnb, out, flush, nb):
             B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down,
                           out["ys"], out["shared_out"], out["workspace"])
             ev[4].record()
-            B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
-                      topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
+            if out["shared_out"].data_ptr() == out["y"].data_ptr():
+                # in place, as moe_forward runs it: only the tokens the route listed
+                B.combine_inplace(dm, out["ys"], out["topk_gate"], out["slot_row"], out["y"], out["workspace"],
+                                  topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
+            else:
+                B.combine(dm, out["ys"], out["shared_out"], out["topk_gate"], out["slot_row"], out["y"],
+                          topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
             ev[5].record()
         torch.cuda.synchronize()
         for i, n in enumerate(names):

@@ -48,7 +48,9 @@
  *
  * Workspace: moe_workspace_bytes(dims) bytes, 256-byte aligned. moe_route
  * writes it (it clears what must start at zero itself); moe_dispatch,
- * moe_aux* and moe_expert_ffn read it. One workspace serves one layer call at
+ * moe_aux*, moe_expert_ffn and moe_combine_inplace read it. Among what moe_route
+ * leaves there is the list of tokens with a source (a real, copy or constant
+ * expert among their K slots), which the in-place combine visits. One workspace serves one layer call at
  * a time: two calls in flight on different streams must use two workspaces.
  */
 #ifndef MOE_NULL_H
@@ -67,7 +69,7 @@
 extern "C" {
 #endif
 
-#define MOE_NULL_ABI_VERSION 5
+#define MOE_NULL_ABI_VERSION 6
 
 typedef void* moe_stream_t; /* a cudaStream_t */
 
@@ -362,6 +364,21 @@ MOE_API int moe_expert_down_combine(const moe_dims_t* dims, const int32_t* offse
 MOE_API int moe_combine(const moe_dims_t* dims, const uint16_t* ys, const uint16_t* shared_out,
                 const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx,
                 const uint16_t* x, const uint16_t* const_vectors, uint16_t* y, moe_stream_t stream);
+
+/* moe_combine in place (shared_out == y) over the route's list of tokens with a
+ * source (section 三 / 核心公式 and Null Expert 机制: a token whose K slots are
+ * all null copies takes only the shared expert, so y[t] = bf16(shared[t]) is
+ * already its result). y [T, d] holds the shared expert's output on entry, as
+ * moe_expert_down writes it with shared_out == y. workspace is the one moe_route
+ * filled for this batch (same dims); the token list there decides which rows are
+ * touched, and y is bit-identical to moe_combine(..., shared_out = y, ...). The
+ * list's order depends on the route's timing; the result does not. A list entry
+ * outside [0, T) is skipped and sets MOE_ERR_DEVICE_BOUNDS in the status word.
+ * topk_idx, x and const_vectors are read only when C + V > 0. */
+MOE_API int moe_combine_inplace(const moe_dims_t* dims, const uint16_t* ys, const float* topk_gate,
+                                const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                                const uint16_t* const_vectors, uint16_t* y, void* workspace,
+                                moe_stream_t stream);
 
 /* Number of doubles in the additive aux statistics of a token shard:
  * [counts_real (N) | null histogram (K+1), then the C+V copy/constant expert

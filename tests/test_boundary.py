@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.LIB.moe_abi_version() == 5
+    assert lib.LIB.moe_abi_version() == 6
     for code in (0, -1, -2, -3, -4, -5, 7):
         assert isinstance(lib.status_string(code), str) and lib.status_string(code)
 

@@ -452,6 +452,53 @@ def test_down_combine_entry_point_called_alone_twice():
         assert torch.equal(out["y"], y0)
 
 
+@pytest.mark.parametrize("name,router", [("skew_small", "tensor"), ("pp_a", "tensor"), ("pp_b", "tensor"),
+                                         ("m0", "fp32_cores"), ("t1", "tensor"), ("ragged_b", "tensor"),
+                                         ("qwen3_1p7b", "tensor"), ("sweep_k8_m192", "tensor")])
+def test_inplace_combine_over_the_route_token_list(name, router):
+    """moe_combine_inplace visits only the tokens the route listed as having a source (a real,
+    copy or constant expert): called alone after a forward, with y reset to the shared expert's
+    output, it gives the forward's y and moe_combine's in-place y bit for bit. The small grid
+    (one token per warp) and the persistent one (sweep_k8_m192, 65536 tokens) both run; every
+    token with no source keeps bf16(shared) untouched."""
+    from token_choice_routing_b200 import binding as B
+    cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP[name]
+    inp = I.make_inputs(cfg)
+    if cfg.C + cfg.V:
+        inp.bias[cfg.N] = np.float32(0.4)
+        inp.bias[cfg.N + 1:] = np.float32(0.6)
+    layer, x, tnb = H.make_layer(inp, router=router)
+    out = layer.forward(x, tnb, layer.alloc(cfg.T, combine="inplace"))
+    torch.cuda.synchronize()
+    assert B.get_device_status(out["workspace"]) == B.OK
+    y_fwd = out["y"].clone()
+    dm = layer.dims(cfg.T)
+
+    def reset_to_shared():
+        B.expert_down(dm, out["offsets"], out["h"], out["h_shared"], layer.w_down, layer.shared_down, out["ys"],
+                      out["y"], out["workspace"])
+
+    reset_to_shared()
+    torch.cuda.synchronize()
+    shared = out["y"].clone()
+    extra = dict(topk_idx=out["topk_idx"], x=x, const_vectors=layer.const_vectors)
+    B.combine(dm, out["ys"], out["y"], out["topk_gate"], out["slot_row"], out["y"], **extra)
+    torch.cuda.synchronize()
+    y_scan = out["y"].clone()
+    for _ in range(2):
+        reset_to_shared()
+        B.combine_inplace(dm, out["ys"], out["topk_gate"], out["slot_row"], out["y"], out["workspace"], **extra)
+        torch.cuda.synchronize()
+        assert B.get_device_status(out["workspace"]) == B.OK
+        assert torch.equal(out["y"], y_fwd) and torch.equal(out["y"], y_scan)
+    # a token has a source iff one of its slots is a real, copy or constant expert
+    idx = out["topk_idx"].cpu().numpy()
+    has = ((idx < cfg.N) | (idx >= cfg.N + cfg.M)).any(axis=1)
+    assert 0 < has.sum() <= cfg.T
+    none = torch.from_numpy(~has).to(out["y"].device)
+    assert torch.equal(y_fwd[none], shared[none])
+
+
 @pytest.mark.parametrize("name,chunk,nsets", [("qwen3_0p6b", 4096, 2), ("qwen3_0p6b", 5000, 3),
                                               ("skew_small", 200, 2), ("tiny", 256, 2), ("pp_a", 128, 3)])
 def test_forward_from_host_memory_in_chunks(name, chunk, nsets):

@@ -86,6 +86,7 @@ def _load() -> C.CDLL:
         "moe_expert_gate_up_gather": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_down": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_combine": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_combine_inplace": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_down_combine": (i32, [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_gate_up_rows": (i32, [pd, C.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_expert_down_rows": (i32, [pd, C.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -121,7 +122,7 @@ def _load() -> C.CDLL:
         f = getattr(lib, name)
         f.restype = res
         f.argtypes = args
-    if lib.moe_abi_version() != 5:
+    if lib.moe_abi_version() != 6:
         raise ImportError("libmoe_null ABI version mismatch")
     return lib
 
@@ -269,6 +270,13 @@ def combine(dm, ys, shared_out, topk_gate, slot_row, y, stream=None, topk_idx=No
     """topk_idx, x and const_vectors are needed only with MoE++ copy/constant experts."""
     _check("moe_combine", LIB.moe_combine(C.byref(dm), _p(ys), _p(shared_out), _p(topk_gate), _p(slot_row),
                                           _p(topk_idx), _p(x), _p(const_vectors), _p(y), _stream(stream)))
+
+
+def combine_inplace(dm, ys, topk_gate, slot_row, y, ws, stream=None, topk_idx=None, x=None, const_vectors=None):
+    """y holds the shared expert's output; adds the routed rows of the tokens the route listed in ws."""
+    _check("moe_combine_inplace",
+           LIB.moe_combine_inplace(C.byref(dm), _p(ys), _p(topk_gate), _p(slot_row), _p(topk_idx), _p(x),
+                                   _p(const_vectors), _p(y), _p(ws), _stream(stream)))
 
 
 def aux(dm, ws, counts_ext, P, losses, stream=None):

@@ -232,6 +232,17 @@ int moe_combine(const moe_dims_t* dims, const uint16_t* ys, const uint16_t* shar
   return launch_combine(*dims, ys, shared_out, topk_gate, slot_row, topk_idx, x, const_vectors, y, S(stream));
 }
 
+int moe_combine_inplace(const moe_dims_t* dims, const uint16_t* ys, const float* topk_gate,
+                        const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
+                        const uint16_t* const_vectors, uint16_t* y, void* workspace, moe_stream_t stream) {
+  MOE_CHECK(check_dims(dims));
+  if (dims->T == 0) return MOE_OK;
+  if (!ys || !topk_gate || !slot_row || !y || !workspace) return MOE_ERR_INVALID_ARG;
+  if (dims->C + dims->V > 0 && (!topk_idx || (dims->C > 0 && !x) || (dims->V > 0 && !const_vectors)))
+    return MOE_ERR_INVALID_ARG;
+  return launch_combine(*dims, ys, y, topk_gate, slot_row, topk_idx, x, const_vectors, y, S(stream), workspace);
+}
+
 int moe_aux_sums(const moe_dims_t* dims, const void* workspace, double* sums, moe_stream_t stream) {
   MOE_CHECK(check_dims(dims));
   if (!workspace || !sums) return MOE_ERR_INVALID_ARG;
@@ -295,8 +306,9 @@ int moe_forward(const moe_dims_t* dims, const moe_weights_t* w, const uint16_t* 
                                workspace, st);
   MOE_CHECK(launch_down(*dims, out->offsets, out->h, out->h_shared, w->w_down, w->shared_down, out->ys,
                         out->shared_out, workspace, st));
+  // in place (shared_out == y): only the tokens the route listed as having a source
   return launch_combine(*dims, out->ys, out->shared_out, out->topk_gate, out->slot_row, out->topk_idx, x,
-                        w->const_vectors, out->y, st);
+                        w->const_vectors, out->y, st, out->shared_out == out->y ? workspace : nullptr);
 }
 
 int moe_get_device_status(const void* workspace, moe_stream_t stream) {

@@ -27,18 +27,37 @@ constexpr int kCombineThreads = 256;
 // without a source already holds its result, bf16(shared), and is skipped.
 // THREADS: 256 for the persistent grid (one wave, each warp looping over tokens with the
 // next token's slots prefetched), 64 for a grid of one token per warp (small batches).
-template <bool UNIT_ROWS, bool INPLACE, int THREADS>
+// LISTED (in place only): the warps visit the route's list of tokens with a source
+// (srctok[0 .. *nsrc)) instead of every token, so tokens without one cost no slot lookup
+// and every warp gets an equal share of the tokens that have work. Each token's sum is the
+// same either way, so y is the same bit for bit.
+template <bool UNIT_ROWS, bool INPLACE, int THREADS, bool LISTED = false>
 __global__ void __launch_bounds__(THREADS, 768 / THREADS)
 combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* sh, const float* __restrict__ gate,
                const int32_t* __restrict__ slot_row, const int32_t* __restrict__ topk_idx,
                const uint16_t* __restrict__ x, const uint16_t* __restrict__ cv, uint16_t* y, int T, int d, int K,
-               long long rcap, int NM, int C, int V, uint32_t* status) {
+               long long rcap, int NM, int C, int V, uint32_t* status, const int32_t* __restrict__ srctok,
+               const int32_t* __restrict__ nsrc) {
+  static_assert(!LISTED || INPLACE, "a token list leaves the tokens it omits untouched: in place only");
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const int wpb = THREADS / 32;
   const int nch = d >> 3;
   const int stride = gridDim.x * wpb;
-  int t = blockIdx.x * wpb + (threadIdx.x >> 5);
+  // visit i = 0 .. nvis-1: token i, or the i-th listed token
+  const int nvis = LISTED ? min(max(__ldg(nsrc), 0), T) : T;
+  auto token_at = [&](int i) {
+    if (i >= nvis) return T;  // past the end: no slots, skipped
+    if (!LISTED) return i;
+    const int tt = __ldg(srctok + i);
+    if (tt < 0 || tt >= T) {
+      if (status) atomicOr(status, kStatusBounds);
+      return T;
+    }
+    return tt;
+  };
+  int i = blockIdx.x * wpb + (threadIdx.x >> 5);
+  int t = token_at(i);
   auto load_slot = [&](int tt, int& row, float& g) {
     row = -1;
     g = 0.f;
@@ -65,12 +84,14 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* sh, const float*
   int row, rown;
   float g, gn;
   load_slot(t, row, g);
-  for (; t < T; t += stride) {
-    load_slot(t + stride, rown, gn);  // next token's slots, in flight during this one
+  for (; i < nvis; i += stride) {
+    const int tn = token_at(i + stride);
+    load_slot(tn, rown, gn);  // next token's slots, in flight during this one
     const unsigned srcs = __ballot_sync(0xffffffffu, row != -1);  // lanes >= K hold -1
     if (INPLACE && srcs == 0u) {
       row = rown;
       g = gn;
+      t = tn;
       continue;
     }
     // the shared row's pieces of the next pass are loaded before this pass's stores (in place
@@ -136,6 +157,7 @@ combine_kernel(const uint16_t* __restrict__ ys, const uint16_t* sh, const float*
     }
     row = rown;
     g = gn;
+    t = tn;
   }
 }
 
@@ -177,17 +199,28 @@ static CombineGrid combine_grid(const moe_dims_t& d) {
 
 int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
                    const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
-                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st) {
+                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st, void* ws) {
   const CombineGrid g = combine_grid(d);
   // shared_out == y: the shared expert's output is already in y; tokens without a source keep it
   const bool inplace = shared_out == y;
+  const int threads = g.persistent ? kCombineThreads : kCombineSmallThreads;
+  const long long rcap = (long long)d.T * d.K;
+  if (inplace && ws != nullptr) {  // only the tokens the route listed
+    const WsLayout L = ws_layout(d);
+    auto kern = g.persistent ? combine_kernel<false, true, kCombineThreads, true>
+                             : combine_kernel<false, true, kCombineSmallThreads, true>;
+    return launch_pdl(kern, dim3(g.blocks), dim3(threads), 0, st, ys, shared_out, topk_gate, slot_row, topk_idx, x,
+                      const_vectors, y, d.T, d.d, d.K, rcap, d.N + d.M, d.C, d.V,
+                      ws_ptr<uint32_t>(ws, L.hdr), (const int32_t*)ws_ptr<int32_t>(ws, L.srctok),
+                      (const int32_t*)ws_ptr<int32_t>(ws, L.hdr + kHdrSrcOffset));
+  }
   auto kern = g.persistent ? (inplace ? combine_kernel<false, true, kCombineThreads>
                                       : combine_kernel<false, false, kCombineThreads>)
                            : (inplace ? combine_kernel<false, true, kCombineSmallThreads>
                                       : combine_kernel<false, false, kCombineSmallThreads>);
-  const int threads = g.persistent ? kCombineThreads : kCombineSmallThreads;
   return launch_pdl(kern, dim3(g.blocks), dim3(threads), 0, st, ys, shared_out, topk_gate, slot_row, topk_idx, x,
-                    const_vectors, y, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, d.V, nullptr);
+                    const_vectors, y, d.T, d.d, d.K, rcap, d.N + d.M, d.C, d.V, (uint32_t*)nullptr,
+                    (const int32_t*)nullptr, (const int32_t*)nullptr);
 }
 
 // Input gradient of the backward pass: dx[t] = dx_shared[t] (the shared expert's and the
@@ -201,7 +234,8 @@ int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint
                            : combine_kernel<true, false, kCombineSmallThreads>;
   const int threads = g.persistent ? kCombineThreads : kCombineSmallThreads;
   return launch_pdl(kern, dim3(g.blocks), dim3(threads), 0, st, dxs, dx_shared, topk_gate, slot_row, topk_idx, dy,
-                    (const uint16_t*)nullptr, dx, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, 0, status);
+                    (const uint16_t*)nullptr, dx, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, 0, status,
+                    (const int32_t*)nullptr, (const int32_t*)nullptr);
 }
 
 }  // namespace moe

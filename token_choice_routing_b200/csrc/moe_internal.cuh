@@ -31,12 +31,18 @@ constexpr uint32_t kStatusBounds = 2u;
 
 // Byte offset of the per-expert row totals inside the workspace header.
 constexpr size_t kHdrTotOffset = 16;
+// Byte offset of the count of tokens with a source (int32): the route appends each token
+// that takes a real expert or a copy or constant expert to the workspace's token list.
+constexpr size_t kHdrSrcOffset = 384;
 // Byte offset of the two counters of the down GEMM with the combine folded in: routed
 // tiles whose ys rows are stored, and CTAs that have exited (the last one resets both).
 constexpr size_t kHdrCombineOffset = 448;
-// Bytes of the header that every route call clears: status word, per-expert totals and
-// the down GEMM's counters.
+// Bytes of the header that every route call clears: status word, per-expert totals, the
+// count of tokens with a source and the down GEMM's counters.
 constexpr size_t kHdrClearBytes = kHdrCombineOffset + 8;
+static_assert(kHdrTotOffset + sizeof(int32_t) * kMaxN <= kHdrSrcOffset &&
+                  kHdrSrcOffset + sizeof(int32_t) <= kHdrCombineOffset,
+              "workspace header fields overlap");
 
 // Default limit of every device-side wait, in ns of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -45,14 +51,17 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 struct WsLayout {
   int blk_tokens;    // tokens per route block (route_block_tokens)
   int nblk;          // route CTAs = ceil(T / blk_tokens)
-  size_t hdr;        // uint32 status at 0; int32 per-expert totals at kHdrTotOffset; the down
-                     // GEMM's counters at kHdrCombineOffset (512 B)
+  size_t hdr;        // uint32 status at 0; int32 per-expert totals at kHdrTotOffset; the count
+                     // of tokens with a source at kHdrSrcOffset; the down GEMM's counters at
+                     // kHdrCombineOffset (512 B)
   size_t counts_blk; // int32 [N][nblk]
   size_t bases;      // int32 [N][nblk]
   size_t ppart;      // float [nblk][N+1+C+V]
   size_t lsq;        // float [nblk]
   size_t hist;       // int32 [nblk][K+1+C+V]: null histogram, then copy/constant expert counts
   size_t lrank;      // int32 [T][K]
+  size_t srctok;     // int32 [T]: the tokens with a source, in the order the route blocks
+                     // appended them (the first header count entries are valid)
   size_t counts;     // int32 [N]
   size_t offsets;    // int32 [N+1]
   size_t sums;       // double [aux sums count]
@@ -107,6 +116,7 @@ inline WsLayout ws_layout(const moe_dims_t& d) {
   L.lsq = o; o = align_up(o + sizeof(float) * (size_t)L.nblk, 256);
   L.hist = o; o = align_up(o + sizeof(int32_t) * (size_t)hist_cols(d) * L.nblk, 256);
   L.lrank = o; o = align_up(o + sizeof(int32_t) * (size_t)d.T * d.K, 256);
+  L.srctok = o; o = align_up(o + sizeof(int32_t) * (size_t)d.T, 256);
   L.counts = o; o = align_up(o + sizeof(int32_t) * (size_t)d.N, 256);
   L.offsets = o; o = align_up(o + sizeof(int32_t) * (size_t)(d.N + 1), 256);
   L.sums = o; o = align_up(o + sizeof(double) * aux_sums_count(d), 256);
@@ -247,9 +257,11 @@ int launch_dispatch(const moe_dims_t& d, const uint16_t* x, const int32_t* topk_
 int launch_aux(const moe_dims_t& d, const void* ws, double* sums_out, const double* sums_in,
                int32_t* counts_ext, float* P, float* losses, cudaStream_t st,
                bool accumulate = false);
+// ws (optional, in place only: shared_out == y): the workspace the route of this forward
+// filled; the combine then visits only the tokens it listed as having a source.
 int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shared_out,
                    const float* topk_gate, const int32_t* slot_row, const int32_t* topk_idx, const uint16_t* x,
-                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st);
+                   const uint16_t* const_vectors, uint16_t* y, cudaStream_t st, void* ws = nullptr);
 // perm (optional): token of each routed row; when given, gate/up gathers the
 // routed rows of x by TMA instead of reading a gathered copy xs (xs unused).
 int launch_gate_up_perm(const moe_dims_t& d, const uint16_t* xs, const uint16_t* x, const int32_t* offsets,

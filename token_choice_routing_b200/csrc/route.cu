@@ -57,6 +57,8 @@ struct RouteArgs {
   int32_t* lrank;
   int32_t* counts;
   int32_t* offsets;
+  int32_t* srctok;  // [T] tokens with a source, appended per tile
+  int32_t* nsrc;    // their count (zero at the start of every call)
   unsigned long long limit_ns;
   int T, d, N, M, K, nblk;
   int ncols;  // router rows N + 1 + C + V (MoE++ copy and constant experts after the null logit)
@@ -139,7 +141,8 @@ struct RouteSmem {
   static constexpr size_t off_tokbits = off_tkv + sizeof(float) * kRouteTokens * kMaxK;  // u32 [4][kMaxN]
   static constexpr int HIST = kMaxK + 1 + kMaxPP;  // null histogram + copy/constant counts
   static constexpr size_t off_hist = off_tokbits + sizeof(unsigned) * 4 * kMaxN;         // int [HIST]
-  static constexpr size_t scratch_end = off_hist + sizeof(int) * HIST;
+  static constexpr size_t off_srcw = off_hist + sizeof(int) * HIST;  // u32 [4]: tokens with a source
+  static constexpr size_t scratch_end = off_srcw + sizeof(unsigned) * 4;
   // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   static constexpr size_t off_bar = align_up(scratch_end, 8);
   static constexpr size_t off_misc = off_bar + 8 * (2 * STAGES + 5);  // [0] TMEM base, [1] abort
@@ -343,6 +346,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     float* tkv = reinterpret_cast<float*>(base + SM::off_tkv);
     unsigned* tokbits = reinterpret_cast<unsigned*>(base + SM::off_tokbits);  // [4][kMaxN]
     int* s_hist = reinterpret_cast<int*>(base + SM::off_hist);                // [kMaxK+1]
+    unsigned* srcw = reinterpret_cast<unsigned*>(base + SM::off_srcw);        // [4]: bit per token
     int li = 0;
     for (int u = unit0; u < nunit; u += ustep, ++li) {
     const int b = tile_of(u);
@@ -362,6 +366,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACOLS;
       const float tn = (a.tnb != nullptr && t < nvalid) ? __ldg(a.tnb + tok0 + t) : 0.f;
       if (etid < SM::HIST) s_hist[etid] = 0;
+      if (etid < 4) srcw[etid] = 0u;
 #pragma unroll 1
       for (int c0 = part * 8; c0 < NPW; c0 += 32) {
         uint32_t rh[8], rm[8], rl[8];
@@ -525,6 +530,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         if (q == 0) {
           a.n_real[tok] = r;
           atomicAdd(s_hist + (K - r - rpp), 1);  // null slots; integer: order does not matter
+          if (r + rpp > 0) atomicOr(srcw + (t >> 5), 1u << (t & 31));  // a source to combine
         }
         mask[t] = msk;  // identical on the token's four lanes
         if (a.logits) {
@@ -602,6 +608,27 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
             for (int w2 = 0; w2 < w; ++w2) rank += __popc(tokbits[w2 * kMaxN + id]);
           }
           a.lrank[(size_t)(tok0 + t) * K + k] = rank;
+        }
+      }
+      // the tile's tokens with a source, appended to the token list with one atomic (the
+      // list's order depends on the tiles' timing; the combine's sums do not)
+      if (live && ew == 15) {
+        const unsigned w0 = srcw[0], w1 = srcw[1], w2 = srcw[2], w3 = srcw[3];
+        const int c0 = __popc(w0), c1 = __popc(w1), c2 = __popc(w2);
+        const int n = c0 + c1 + c2 + __popc(w3);
+        if (n > 0) {
+          int at = 0;
+          if (lane == 0) at = atomicAdd(a.nsrc, n);
+          at = __shfl_sync(0xffffffffu, at, 0);
+          const unsigned below = (1u << lane) - 1u;
+          if (at >= 0 && at + n <= T) {
+            if ((w0 >> lane) & 1u) a.srctok[at + __popc(w0 & below)] = tok0 + lane;
+            if ((w1 >> lane) & 1u) a.srctok[at + c0 + __popc(w1 & below)] = tok0 + 32 + lane;
+            if ((w2 >> lane) & 1u) a.srctok[at + c0 + c1 + __popc(w2 & below)] = tok0 + 64 + lane;
+            if ((w3 >> lane) & 1u) a.srctok[at + c0 + c1 + c2 + __popc(w3 & below)] = tok0 + 96 + lane;
+          } else if (lane == 0) {
+            atomicOr(a.hdr, kStatusBounds);  // more tokens than T: the count was not cleared
+          }
         }
       }
     }
@@ -841,6 +868,8 @@ int launch_route(const moe_dims_t& d, const uint16_t* x, const float* w_router, 
   a.lrank = ws_ptr<int32_t>(ws, L.lrank);
   a.counts = ws_ptr<int32_t>(ws, L.counts);
   a.offsets = ws_ptr<int32_t>(ws, L.offsets);
+  a.srctok = ws_ptr<int32_t>(ws, L.srctok);
+  a.nsrc = ws_ptr<int32_t>(ws, L.hdr + kHdrSrcOffset);
   a.limit_ns = kWaitLimitNs;
   a.T = d.T;
   a.d = d.d;

@@ -55,6 +55,8 @@ struct RouteArgs {
   int32_t* lrank;
   int32_t* counts;
   int32_t* offsets;
+  int32_t* srctok;  // [T] tokens with a source, appended per block
+  int32_t* nsrc;    // their count (zero at the start of every call)
   int T, d, N, M, K, nblk;
 };
 
@@ -447,6 +449,27 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteArgs a) {
       a.lrank[(size_t)tok * K + k] = rank;
     }
   }
+  // the block's tokens with a source (a real expert: this route has no copy or constant
+  // experts), appended to the token list with one atomic
+  if (tid >= 224) {
+    const int lane = tid & 31;
+    const bool s0 = lane < nvalid && mask[lane] != 0ull;
+    const bool s1 = 32 + lane < nvalid && mask[32 + lane] != 0ull;
+    const unsigned w0 = __ballot_sync(0xffffffffu, s0), w1 = __ballot_sync(0xffffffffu, s1);
+    const int c0 = __popc(w0), n = c0 + __popc(w1);
+    if (n > 0) {
+      int at = 0;
+      if (lane == 0) at = atomicAdd(a.nsrc, n);
+      at = __shfl_sync(0xffffffffu, at, 0);
+      const unsigned below = (1u << lane) - 1u;
+      if (at >= 0 && at + n <= T) {
+        if (s0) a.srctok[at + __popc(w0 & below)] = tok0 + lane;
+        if (s1) a.srctok[at + c0 + __popc(w1 & below)] = tok0 + 32 + lane;
+      } else if (lane == 0) {
+        atomicOr(a.hdr, kStatusBounds);  // more tokens than T: the count was not cleared
+      }
+    }
+  }
 }
 
 template <int LG>
@@ -494,6 +517,8 @@ int launch_route_fp32(const moe_dims_t& d, const uint16_t* x, const float* w_rou
   a.lrank = ws_ptr<int32_t>(ws, L.lrank);
   a.counts = ws_ptr<int32_t>(ws, L.counts);
   a.offsets = ws_ptr<int32_t>(ws, L.offsets);
+  a.srctok = ws_ptr<int32_t>(ws, L.srctok);
+  a.nsrc = ws_ptr<int32_t>(ws, L.hdr + kHdrSrcOffset);
   a.T = d.T;
   a.d = d.d;
   a.N = d.N;
