@@ -611,7 +611,7 @@ def measure_per_config(args, names, dev, flush, peaks):
         out = layer.alloc(cfg.T, logits=False, xs=not args.gather, combine=args.combine)
         ms = timed_events(lambda: layer.forward(x, tnb, out), steps, warmup, flush)
         R = int(out["offsets"][-1].item())
-        kms = forward_stage_ms(layer, layer.dims(cfg.T), x, tnb, out, flush, 5)
+        kms = forward_stage_ms(layer, layer.dims(cfg.T), x, tnb, out, flush, 9)  # median of 9 passes
         b, ffn_tflops, _ = forward_figures(cfg, R, kms, peaks, args, out)
         med = statistics.median(ms)
         res[name] = {"T": cfg.T, "K": cfg.K, "M": cfg.M, "rho": cfg.rho, "real_slots_per_step": R,
