@@ -76,7 +76,7 @@ typedef void* moe_stream_t; /* a cudaStream_t */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = -1,   /* null pointer, negative size, K < 1, ... */
-  MOE_ERR_UNSUPPORTED = -2,   /* valid but outside this build's limits */
+  MOE_ERR_UNSUPPORTED = -2,   /* valid but outside this library's limits */
   MOE_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed */
   MOE_ERR_TIMEOUT = -4,       /* a device-side bounded wait ran out */
   MOE_ERR_DEVICE_BOUNDS = -5  /* a device-side guard saw an out-of-range index */
