@@ -525,6 +525,26 @@ def test_forward_from_host_memory_in_chunks(name, chunk, nsets):
         np.testing.assert_allclose(st["losses"].cpu().numpy(), ref["losses"].cpu().numpy(), rtol=1e-6)
 
 
+def test_forward_host_batches_of_growing_size_reuse_the_pipeline():
+    """One pipeline, host-buffer forwards of 1000 tokens, then 2600, then 1000 again, with
+    per-token null offsets (copied in once per call into a device buffer the pipeline keeps
+    and grows): each y is bit-identical to the device forward of the same tokens."""
+    cfg = I.small_config("skew_3k", T=3072, d=256, N=64, F=128, F_shared=128, K=8, M=64, config_id=930,
+                         skew=True, seqs=3)
+    inp = I.make_inputs(cfg)
+    layer, x, tnb = H.make_layer(inp)
+    assert tnb is not None
+    pipe = layer.alloc_host_pipeline(512, 3)
+    for n in (1000, 2600, 1000):
+        ref = layer.forward(x[:n], tnb[:n], layer.alloc(n))
+        torch.cuda.synchronize()
+        x_pin = x[:n].cpu().pin_memory()
+        y_pin = torch.zeros_like(x_pin).pin_memory()
+        layer.forward_host(x_pin, y_pin, pipe, tnb[:n].cpu().pin_memory())
+        torch.cuda.synchronize()
+        assert torch.equal(y_pin, ref["y"][:n].cpu())
+
+
 @pytest.mark.parametrize("name", ["tiny", "ragged_b", "pp_80rows", "skew"])
 def test_route_from_the_prepared_router_weight_is_bitwise_moe_route(name):
     """moe_route_prepared (the weight split once by moe_prepare_router, as the layer's forward

@@ -237,7 +237,6 @@ class MoENullLayer:
         sets = [self.alloc(chunk, logits=False) for _ in range(max(2, int(nsets)))]
         for o in sets:
             o["x_stage"] = torch.empty((chunk, self.d), dtype=torch.bfloat16, device=dev)
-            o["tnb_stage"] = torch.empty((chunk,), dtype=torch.float32, device=dev)
         n = B.aux_sums_count(self.dims(1))
         pool = self.N + self.M + self.C + self.V
         return dict(chunk=chunk, sets=sets,
@@ -257,7 +256,10 @@ class MoENullLayer:
         L_bal and L_z, which are means over the whole batch, are summed over the chunks on the
         device (moe_aux_sums / moe_aux_sums_accumulate) and finalised once. Returns the device
         counts_ext, P and losses of the batch. The current stream is ordered after the last
-        copy, so synchronising it makes y_host complete. reduce_sums (data parallel: e.g.
+        copy, so synchronising it makes y_host complete. The per-token null offsets (4 B a
+        token) are copied in once for the whole batch, ahead of the first chunk, into a device
+        buffer the pipeline keeps (allocated by the first call that needs it, grown with T):
+        one small copy per chunk would leave a gap in the copy-in stream each time. reduce_sums (data parallel: e.g.
         dist.allreduce_aux_sums) is applied to the summed statistics before they are
         finalised, so the losses are the whole job's."""
         T = x_host.shape[0]
@@ -270,6 +272,14 @@ class MoENullLayer:
         ev_done = [torch.cuda.Event() for _ in sets]
         ev_out = [torch.cuda.Event() for _ in sets]
         ns = len(sets)
+        tnb_dev = None
+        if tok_null_bias_host is not None:
+            tnb_dev = pipe.get("tnb_batch")
+            if tnb_dev is None or tnb_dev.numel() < T:
+                tnb_dev = torch.empty((T,), dtype=torch.float32, device=self.device)
+                pipe["tnb_batch"] = tnb_dev
+            with torch.cuda.stream(cin):
+                tnb_dev[:T].copy_(tok_null_bias_host, non_blocking=True)
         for c, (a, b) in enumerate(chunk_bounds(T, chunk)):
             k = c % ns
             o = sets[k]
@@ -278,15 +288,13 @@ class MoENullLayer:
                 if c >= ns:
                     cin.wait_event(ev_done[k])  # the set's previous chunk no longer reads this staging
                 o["x_stage"][:Tc].copy_(x_host[a:b], non_blocking=True)
-                if tok_null_bias_host is not None:
-                    o["tnb_stage"][:Tc].copy_(tok_null_bias_host[a:b], non_blocking=True)
-                ev_in[k].record(cin)
+                ev_in[k].record(cin)  # also covers the offsets' copy, issued before chunk 0's
             comp.wait_event(ev_in[k])
             if c >= ns:
                 comp.wait_event(ev_out[k])  # the set's previous chunk's y has been copied out
             dm = self.dims(Tc)
             x = o["x_stage"][:Tc]
-            tnb = None if tok_null_bias_host is None else o["tnb_stage"][:Tc]
+            tnb = None if tnb_dev is None else tnb_dev[a:b]
             ob = B.Outputs(*[None if o.get(f) is None else o[f].data_ptr() for f in B.OUTPUT_FIELDS])
             B.forward(dm, self._weights, x, tnb, ob, o["workspace"], comp)
             if c == 0:
