@@ -724,6 +724,21 @@ def main():
     if st != B.OK:
         raise SystemExit(f"device status after timing: {B.status_string(st)}")
 
+    # ---- the same forward replayed from a CUDA graph (one GPU): no host launch work per step,
+    # which is what bounds decode-sized steps; same buffers, same L2 flush between steps
+    graph = None
+    if world == 1:
+        y_eager = out["y"].clone()
+        g = layer.capture_forward(x, tnb, out)
+        g_ms = timed_events(g.replay, args.steps, args.warmup, flush)
+        torch.cuda.synchronize()
+        if not torch.equal(out["y"], y_eager) or B.get_device_status(out["workspace"]) != B.OK:
+            raise SystemExit("graph replay: y differs from the eager forward's, or the device status is set")
+        graph = {"value": R * args.steps / (sum(g_ms) * 1e-3), "unit": UNIT, "ms_per_step": sum(g_ms) / args.steps,
+                 "ms_per_step_median": statistics.median(g_ms),
+                 "what": "the forward captured once in a CUDA graph (torch.cuda.graph) and replayed"}
+        del g, y_eager
+
     # ---- per-kernel breakdown (separately timed passes, same launches, CUDA events between them);
     # the SM clock is sampled here too: under the 1000 W cap it can settle lower than in the step loop
     with ClockSampler(local) as stage_clk:
@@ -832,7 +847,7 @@ def main():
             # the FLOPs behind it: routed real slots and the shared expert's T rows (one launch each GEMM)
             "ffn_gflop_per_step": {"routed": 6.0 * cfg.d * cfg.F * R / 1e9,
                                    "shared": 6.0 * cfg.d * cfg.F_shared * cfg.T / 1e9},
-            "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk.summary(),
             "backward": backward,

@@ -525,6 +525,38 @@ def test_forward_from_host_memory_in_chunks(name, chunk, nsets):
         np.testing.assert_allclose(st["losses"].cpu().numpy(), ref["losses"].cpu().numpy(), rtol=1e-6)
 
 
+@pytest.mark.parametrize("name", ["decode_0p6b", "skew_small", "pp_a", "t1"])
+def test_captured_forward_graph_replays_the_eager_forward(name):
+    """MoENullLayer.capture_forward: replaying the CUDA graph of one forward gives the eager
+    forward's outputs bit for bit, and after new tokens are copied into x in place it gives
+    the eager forward of those tokens; replays are deterministic and leave the status OK."""
+    from token_choice_routing_b200 import binding as B
+    cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP[name]
+    inp = I.make_inputs(cfg)
+    if cfg.C + cfg.V:
+        inp.bias[cfg.N] = np.float32(0.4)
+        inp.bias[cfg.N + 1:] = np.float32(0.6)
+    layer, x, tnb = H.make_layer(inp)
+    x_static = x.clone()
+    out = layer.alloc(cfg.T)
+    g = layer.capture_forward(x_static, tnb, out)
+    ref1 = layer.forward(x, tnb, layer.alloc(cfg.T))
+    x2 = torch.flip(x, dims=[0]).contiguous()  # other tokens: the batch reversed
+    ref2 = layer.forward(x2, tnb, layer.alloc(cfg.T))
+    torch.cuda.synchronize()
+    keys = ("y", "topk_idx", "topk_gate", "n_real", "counts", "offsets", "slot_row", "counts_ext", "P", "losses")
+    for xin, ref in ((x, ref1), (x2, ref2), (x, ref1)):
+        x_static.copy_(xin)
+        for k in ("y", "topk_idx", "counts"):
+            out[k].zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert B.get_device_status(out["workspace"]) == B.OK
+        for k in keys:
+            assert torch.equal(out[k], ref[k]), k
+    del g
+
+
 def test_forward_host_batches_of_growing_size_reuse_the_pipeline():
     """One pipeline, host-buffer forwards of 1000 tokens, then 2600, then 1000 again, with
     per-token null offsets (copied in once per call into a device buffer the pipeline keeps

@@ -312,6 +312,25 @@ class MoENullLayer:
         comp.wait_stream(cout)
         return dict(counts_ext=pipe["counts_ext"], P=pipe["P"], losses=pipe["losses"])
 
+    def capture_forward(self, x: torch.Tensor, tok_null_bias: Optional[torch.Tensor],
+                        out: Dict[str, torch.Tensor]) -> "torch.cuda.CUDAGraph":
+        """A CUDA graph of one forward over fixed buffers. replay() recomputes ``out`` from the
+        current contents of x (and tok_null_bias) with no host-side launch work, which is what
+        bounds a decode-sized step: seven launches of a few microseconds of GPU work each. The
+        graph holds the addresses of x, tok_null_bias, the weights and every buffer of ``out``,
+        so new tokens are copied into x in place between replays, and the buffers must outlive
+        the graph. One eager forward runs first, so that one-time work (kernel attributes,
+        cached device properties) happens outside the capture."""
+        self.forward(x, tok_null_bias, out)
+        cur = torch.cuda.current_stream(self.device)
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(cur)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self.forward(x, tok_null_bias, out)
+        cur.wait_stream(side)
+        return g
+
     def forward(self, x: torch.Tensor, tok_null_bias: Optional[torch.Tensor] = None,
                 out: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
         T = x.shape[0]
