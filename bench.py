@@ -341,7 +341,6 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     dg = torch.empty((T, K), dtype=torch.float32, device=dev)
     ds = torch.empty((T, rows), dtype=torch.float32, device=dev)
     dxs = torch.empty((Rc, d), dtype=torch.bfloat16, device=dev)
-    dxsh = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     o = bout
     stages = [
         ("combine_bwd", lambda: B.combine_backward(dm, dy, o["ys"], o["topk_gate"], o["slot_row"], dys, dg, bws,
@@ -355,11 +354,13 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
                                                                   layer.shared_gate_up, bws)),
         ("wgrad_down", lambda: B.expert_wgrad_down(dm, o["offsets"], dys, dy, o["h"], o["h_shared"],
                                                    grads["dw_down"], grads["dws_down"], bws)),
+        # as moe_backward runs them: the shared expert's input gradient written straight into dx,
+        # then the input gradient gather in place over the tokens with a real or copy-expert slot
         ("dgrad_gate_up", lambda: B.expert_dgrad_gate_up(dm, o["offsets"], layer.gate_up, layer.shared_gate_up,
-                                                         layer.w_router, dxs, dxsh, bws)),
+                                                         layer.w_router, dxs, grads["dx"], bws)),
         ("wgrad_gate_up", lambda: B.expert_wgrad_gate_up(dm, o["offsets"], o["xs"], x, grads["dw_gate"],
                                                          grads["dw_up"], grads["dws_gate"], grads["dws_up"], bws)),
-        ("input_grad", lambda: B.input_grad(dm, dxsh, dxs, o["slot_row"], o["topk_idx"], o["topk_gate"], dy,
+        ("input_grad", lambda: B.input_grad(dm, grads["dx"], dxs, o["slot_row"], o["topk_idx"], o["topk_gate"], dy,
                                             grads["dx"], bws)),
     ]
     acc = {n: [] for n, _ in stages}
@@ -380,6 +381,9 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     kms = {n: statistics.median(acc[n]) for n in acc}  # median over the passes
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    # the in-place input gradient reads and writes dx only for the tokens with a real or copy slot
+    idx = o["topk_idx"][:T]
+    t_src = int(((idx < cfg.N) | ((idx >= cfg.N + cfg.M) & (idx < cfg.N + cfg.M + cfg.C))).any(dim=1).sum().item())
     # the router's input gradient ds W_r rides in dgrad_gate_up (extra k-blocks of the shared tiles)
     fl = {"swiglu_bwd_recompute": 4.0 * d * (F * R + Fs * T), "dgrad_down": 2.0 * d * (F * R + Fs * T),
           "wgrad_down": 2.0 * d * (F * R + Fs * T), "dgrad_gate_up": 4.0 * d * (F * R + Fs * T) + 2.0 * rows * d * T,
@@ -387,7 +391,7 @@ def measure_backward(args, cfg, layer, x, tnb, flush, peaks, peak_kind):
     # the saved-pre-activation SwiGLU backward reads z (4F B) and dh (2F B) and writes dz (4F B) per row
     by = {"swiglu_bwd": 10.0 * (F * R + Fs * T), "combine_bwd": 2.0 * d * T + 4.0 * d * R + 12.0 * K * T,
           "router_bwd": 8.0 * rows * T + 12.0 * K * T,
-          "input_grad": 4.0 * d * T + 2.0 * d * R + 8.0 * K * T}
+          "input_grad": 4.0 * d * t_src + 2.0 * d * R + 8.0 * K * T}
     kernels = {}
     for n, ms in kms.items():
         k = {"ms": ms}

@@ -571,7 +571,9 @@ MOE_API int moe_expert_wgrad_gate_up(const moe_dims_t* dims, const int32_t* offs
 
 /* Input gradient: dx[t] = dx_shared[t] (the shared expert's and the router's input
  * gradient) + sum over the token's real slots of dxs[slot_row] + sum over its copy-expert
- * slots of g dy[t], accumulated in fp32 in rank order and rounded once to bf16. */
+ * slots of g dy[t], accumulated in fp32 in rank order and rounded once to bf16. dx_shared
+ * may be dx itself (in place, as moe_backward runs it): a token with no real or copy-expert
+ * slot is then left as it is, which is the same value bit for bit. */
 MOE_API int moe_input_grad(const moe_dims_t* dims, const uint16_t* dx_shared, const uint16_t* dxs,
                            const int32_t* slot_row, const int32_t* topk_idx, const float* topk_gate,
                            const uint16_t* dy, uint16_t* dx, void* bwd_workspace, moe_stream_t stream);

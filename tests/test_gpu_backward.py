@@ -147,7 +147,9 @@ def test_backward_loss_terms_only(name):
 
 def test_backward_step_entry_points_match_the_whole_call():
     """combine, router, router weight, expert FFN and input-gradient entry points called one
-    by one give bit-identical gradients to moe_backward."""
+    by one give bit-identical gradients to moe_backward: with the shared expert's input
+    gradient in a buffer of its own, and in place (written into dx, then the gather over the
+    tokens with a real or copy slot, as moe_backward runs it)."""
     from token_choice_routing_b200 import binding as B
     cfg = CASES["ragged"]
     inp, layer, x, out, dy, dy_bits, g = run(cfg)
@@ -176,7 +178,7 @@ def test_backward_step_entry_points_match_the_whole_call():
     for k in ("dx", "dw_router", "dbias", "dtok_null_bias", "dw_gate", "dw_up", "dw_down", "dws_gate", "dws_up",
               "dws_down"):
         assert torch.equal(g[k], g2[k]), k
-    # and the five GEMM stages one by one give the same expert gradients and dx
+    # and the five GEMM stages one by one give the same expert gradients and dx, in place
     g3 = layer.alloc_grads(T)
     bws3 = g3["workspace"]
     B.clear_device_status(bws3)
@@ -186,10 +188,12 @@ def test_backward_step_entry_points_match_the_whole_call():
     B.expert_dgrad_down(dm, out["offsets"], dys, dy, layer.w_down, layer.shared_down, bws3)
     B.expert_swiglu_backward(dm, out["xs"], x, out["offsets"], layer.gate_up, layer.shared_gate_up, bws3)
     B.expert_wgrad_down(dm, out["offsets"], dys, dy, out["h"], out["h_shared"], g3["dw_down"], g3["dws_down"], bws3)
-    B.expert_dgrad_gate_up(dm, out["offsets"], layer.gate_up, layer.shared_gate_up, layer.w_router, dxs, dxsh, bws3)
+    g3["dx"].fill_(7.0)  # every row is overwritten by the shared expert's input gradient
+    B.expert_dgrad_gate_up(dm, out["offsets"], layer.gate_up, layer.shared_gate_up, layer.w_router, dxs, g3["dx"],
+                           bws3)
     B.expert_wgrad_gate_up(dm, out["offsets"], out["xs"], x, g3["dw_gate"], g3["dw_up"], g3["dws_gate"],
                            g3["dws_up"], bws3)
-    B.input_grad(dm, dxsh, dxs, out["slot_row"], out["topk_idx"], out["topk_gate"], dy, g3["dx"], bws3)
+    B.input_grad(dm, g3["dx"], dxs, out["slot_row"], out["topk_idx"], out["topk_gate"], dy, g3["dx"], bws3)
     torch.cuda.synchronize()
     assert B.get_device_status(bws3) == B.OK
     for k in ("dx", "dw_gate", "dw_up", "dw_down", "dws_gate", "dws_up", "dws_down"):

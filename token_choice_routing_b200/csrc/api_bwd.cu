@@ -242,7 +242,6 @@ int moe_backward(const moe_dims_t* dims, const moe_weights_t* w, const moe_saved
   uint32_t* status = ws_ptr<uint32_t>(ws, L.hdr);
   uint16_t* dys = ws_ptr<uint16_t>(ws, L.dys);
   uint16_t* dxs = ws_ptr<uint16_t>(ws, L.dxs);
-  uint16_t* dxsh = ws_ptr<uint16_t>(ws, L.dxsh);
   float* dg = ws_ptr<float>(ws, L.dg);
   float* ds = ws_ptr<float>(ws, L.ds);
   MOE_CHECK(cuda_status(cudaMemsetAsync(status, 0, sizeof(uint32_t), st)));
@@ -252,8 +251,11 @@ int moe_backward(const moe_dims_t* dims, const moe_weights_t* w, const moe_saved
                               (long long)saved->t_total, alpha, beta, ds, g->dtok_null_bias,
                               ws_ptr<uint16_t>(ws, L.dsplit), ws_ptr<float>(ws, L.bpart), st));
   MOE_CHECK(router_wgrad(d, saved->x, g->dw_router, g->dbias, ws, st));
-  MOE_CHECK(expert_ffn_bwd(d, w, saved, dys, dy, dxs, dxsh, g, ws, st));
-  MOE_CHECK(launch_input_grad(d, dxsh, dxs, saved->slot_row, saved->topk_idx, saved->topk_gate, dy, g->dx, status,
+  // the shared expert's (and the router's) input gradient goes straight into dx; the input
+  // gradient gather then adds the routed and copy-expert terms in place, skipping the tokens
+  // that have none
+  MOE_CHECK(expert_ffn_bwd(d, w, saved, dys, dy, dxs, g->dx, g, ws, st));
+  MOE_CHECK(launch_input_grad(d, g->dx, dxs, saved->slot_row, saved->topk_idx, saved->topk_gate, dy, g->dx, status,
                               st));
   return launch_const_grad(d, saved->topk_idx, saved->topk_gate, dy, g->dconst, st);
 }

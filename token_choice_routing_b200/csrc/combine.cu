@@ -225,13 +225,18 @@ int launch_combine(const moe_dims_t& d, const uint16_t* ys, const uint16_t* shar
 
 // Input gradient of the backward pass: dx[t] = dx_shared[t] (the shared expert's and the
 // router's input gradient) + sum over the token's real slots of dxs[slot_row] + sum over
-// its copy-expert slots of g dy[t]; the same gather as the forward combine.
+// its copy-expert slots of g dy[t]; the same gather as the forward combine. In place
+// (dx_shared == dx, as moe_backward runs it) tokens without such slots are skipped.
 int launch_input_grad(const moe_dims_t& d, const uint16_t* dx_shared, const uint16_t* dxs, const int32_t* slot_row,
                       const int32_t* topk_idx, const float* topk_gate, const uint16_t* dy, uint16_t* dx,
                       uint32_t* status, cudaStream_t st) {
   const CombineGrid g = combine_grid(d);
-  auto kern = g.persistent ? combine_kernel<true, false, kCombineThreads>
-                           : combine_kernel<true, false, kCombineSmallThreads>;
+  // dx_shared == dx (in place): a token with no routed or copy slot already holds its result
+  const bool inplace = dx_shared == dx;
+  auto kern = g.persistent ? (inplace ? combine_kernel<true, true, kCombineThreads>
+                                      : combine_kernel<true, false, kCombineThreads>)
+                           : (inplace ? combine_kernel<true, true, kCombineSmallThreads>
+                                      : combine_kernel<true, false, kCombineSmallThreads>);
   const int threads = g.persistent ? kCombineThreads : kCombineSmallThreads;
   return launch_pdl(kern, dim3(g.blocks), dim3(threads), 0, st, dxs, dx_shared, topk_gate, slot_row, topk_idx, dy,
                     (const uint16_t*)nullptr, dx, d.T, d.d, d.K, (long long)d.T * d.K, d.N + d.M, d.C, 0, status,

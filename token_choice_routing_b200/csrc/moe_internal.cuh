@@ -146,8 +146,8 @@ struct BwdLayout {
   size_t dz;     // bf16 [R_cap, 2F] gradients of the gate/up pre-activations (packed order)
   size_t dzs;    // bf16 [T, 2F_shared]
   size_t dys;    // bf16 [R_cap, d] upstream gradient of each routed row: g * dy
-  size_t dxs;    // bf16 [R_cap, d] input gradient of each routed row
-  size_t dxsh;   // bf16 [T, d] input gradient through the shared expert
+  size_t dxs;    // bf16 [R_cap, d] input gradient of each routed row (the shared expert's
+                 // input gradient goes straight into the caller's dx)
   size_t dg;     // fp32 [T, K] gate gradients
   size_t ds;     // fp32 [T, N+1+C+V] logit gradients
   size_t dsplit; // bf16 [T, 2 RP] logit gradients as two terms (hi | lo), RP = router_split_rows
@@ -172,7 +172,6 @@ inline BwdLayout bwd_layout(const moe_dims_t& d) {
   L.dzs = o; o = align_up(o + 2 * T * 2 * d.F_shared, 256);
   L.dys = o; o = align_up(o + 2 * rcap * d.d, 256);
   L.dxs = o; o = align_up(o + 2 * rcap * d.d, 256);
-  L.dxsh = o; o = align_up(o + 2 * T * d.d, 256);
   L.dg = o; o = align_up(o + 4 * T * d.K, 256);
   L.ds = o; o = align_up(o + 4 * T * rows, 256);
   L.dsplit = o; o = align_up(o + 2 * T * 2 * rp, 256);
