@@ -452,9 +452,16 @@ def test_down_combine_entry_point_called_alone_twice():
         assert torch.equal(out["y"], y0)
 
 
+# a ragged batch above the persistent grid's threshold (16 tokens per resident warp), routed on
+# CTA pairs (more tiles than SMs), with a ragged last tile
+LIST_CASES = {"ragged_60k": I.small_config("ragged_60k", T=60001, d=128, N=16, F=64, F_shared=64, K=4, M=16,
+                                           config_id=931)}
+
+
 @pytest.mark.parametrize("name,router", [("skew_small", "tensor"), ("pp_a", "tensor"), ("pp_b", "tensor"),
                                          ("m0", "fp32_cores"), ("t1", "tensor"), ("ragged_b", "tensor"),
-                                         ("qwen3_1p7b", "tensor"), ("sweep_k8_m192", "tensor")])
+                                         ("qwen3_1p7b", "tensor"), ("sweep_k8_m192", "tensor"),
+                                         ("ragged_60k", "tensor"), ("ragged_60k", "fp32_cores")])
 def test_inplace_combine_over_the_route_token_list(name, router):
     """moe_combine_inplace visits only the tokens the route listed as having a source (a real,
     copy or constant expert): called alone after a forward, with y reset to the shared expert's
@@ -462,7 +469,7 @@ def test_inplace_combine_over_the_route_token_list(name, router):
     (one token per warp) and the persistent one (sweep_k8_m192, 65536 tokens) both run; every
     token with no source keeps bf16(shared) untouched."""
     from token_choice_routing_b200 import binding as B
-    cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP[name]
+    cfg = I.CONFIGS.get(name) or SMALL.get(name) or PP.get(name) or LIST_CASES[name]
     inp = I.make_inputs(cfg)
     if cfg.C + cfg.V:
         inp.bias[cfg.N] = np.float32(0.4)
