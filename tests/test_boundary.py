@@ -122,6 +122,10 @@ def test_host_side_rejections_touch_no_device(lib):
     assert L.moe_route(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_dispatch(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_combine(C.byref(dm), nul, nul, nul, nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
+    assert L.moe_combine_inplace(C.byref(dm), *([nul] * 9)) == B.ERR_INVALID_ARG
+    # the in-place combine needs the route's workspace (its token list): a missing one is refused
+    fake = C.c_void_p(16)
+    assert L.moe_combine_inplace(C.byref(dm), fake, fake, fake, nul, nul, nul, fake, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_aux(C.byref(dm), nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_forward(C.byref(dm), nul, nul, nul, nul, nul, nul) == B.ERR_INVALID_ARG
     assert L.moe_get_device_status(nul, nul) == B.ERR_INVALID_ARG
